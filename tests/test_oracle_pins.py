@@ -1,0 +1,400 @@
+"""Pins for the fp64 oracle against what the pages and mathematics fix.
+
+Nothing here compares the oracle with itself: every expected value comes from
+a closed form, a hand-derived case (tests/golden), a brute-force enumeration
+written independently of the oracle's sort-and-prefix code, a numpy library
+routine, an invariance of the definitions, or central finite differences.
+"""
+
+import itertools
+import json
+import math
+from pathlib import Path
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+
+GOLDEN = Path(__file__).parent / "golden" / "support_cases.json"
+
+
+def _eval(expr):
+    if expr == "-inf":
+        return -math.inf
+    return eval(expr, {"log": math.log, "exp": math.exp, "e": math.e, "__builtins__": {}})
+
+
+def _logits(vals):
+    out = []
+    for v in vals:
+        if isinstance(v, str) and v.startswith("log:"):
+            out.append(math.log(float(v[4:])))
+        else:
+            out.append(float(v))
+    return np.array(out, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# hand-derived golden cases
+
+
+def test_golden_computed_support_cases():
+    cases = json.loads(GOLDEN.read_text())["cases"]
+    for c in cases:
+        l = _logits(c["logits"])
+        n = len(l)
+        for t_i, y in enumerate(c["targets"]):
+            r = oracle.score(l[None, :], [y], temperature=c["temperature"], top_k=c["top_k"],
+                             top_p=c["top_p"], min_p=c["min_p"], want_mask=True)
+            got = sorted(np.nonzero(r["mask"][0])[0].tolist())
+            assert got == c["support"], c["name"]
+            assert r["support_size"][0] == len(c["support"])
+            exp_lp = _eval(c["lp_support"][t_i])
+            if exp_lp == -math.inf:
+                assert r["lp_support"][0] == -math.inf, c["name"]
+                assert r["status"][0] & oracle.TARGET_NOT_IN_SUPPORT
+            else:
+                assert abs(r["lp_support"][0] - exp_lp) < 1e-12, c["name"]
+            if c["h_support"] is None:
+                assert abs(r["h_support"][0] - r["h_full"][0]) < 1e-12
+            else:
+                assert abs(r["h_support"][0] - _eval(c["h_support"])) < 1e-12, c["name"]
+            if c.get("exact_zero"):
+                assert r["h_support"][0] == 0.0
+                if exp_lp == 0:
+                    assert r["lp_support"][0] == 0.0
+            assert r["valid"][0] == 1
+
+
+def test_golden_recorded_support_cases():
+    names = {"DUP_SUPPORT_ID": oracle.DUP_SUPPORT_ID,
+             "TARGET_NOT_IN_SUPPORT": oracle.TARGET_NOT_IN_SUPPORT}
+    for c in json.loads(GOLDEN.read_text())["recorded"]:
+        l = _logits(c["logits"])
+        sup = np.array([c["support_ids"]], dtype=np.int32)
+        for t_i, y in enumerate(c["targets"]):
+            r = oracle.score(l[None, :], [y], support=sup, want_mask=True)
+            assert sorted(np.nonzero(r["mask"][0])[0].tolist()) == c["support"]
+            exp_lp = _eval(c["lp_support"][t_i])
+            if exp_lp == -math.inf:
+                assert r["lp_support"][0] == -math.inf
+            else:
+                assert abs(r["lp_support"][0] - exp_lp) < 1e-12
+            if "status" in c:
+                want = 0
+                for part in c["status"][t_i].split("|"):
+                    want |= names[part]
+                assert r["status"][0] == want
+            if "valid" in c:
+                assert r["valid"][0] == c["valid"]
+                assert r["h_support"][0] == 0.0
+
+
+# ---------------------------------------------------------------------------
+# closed forms
+
+
+@pytest.mark.parametrize("vocab", [1024, workloads.VOCAB])
+def test_uniform_logits_closed_form(vocab):
+    l = np.full((2, vocab), 0.75, dtype=np.float32)
+    r = oracle.score(l, [0, vocab - 1], temperature=0.9)
+    assert np.allclose(r["lp_full"], -math.log(vocab), rtol=0, atol=1e-11)
+    assert np.allclose(r["h_full"], math.log(vocab), rtol=1e-12)
+    # no filter: the support is the full vocabulary
+    assert np.array_equal(r["support_size"], [vocab, vocab])
+    assert np.allclose(r["h_support"], math.log(vocab), rtol=1e-12)
+    assert np.allclose(r["lp_support"], -math.log(vocab), atol=1e-11)
+
+
+def test_uniform_over_recorded_support_is_log_size():
+    rng = np.random.default_rng(5)
+    l = rng.normal(size=(1, 200))
+    ids = np.array([[3, 17, 40, 41, 99, -1, -1]], dtype=np.int32)
+    l[0, ids[0, :5]] = 2.5  # equal logits on the support
+    r = oracle.score(l, [17], support=ids)
+    assert abs(r["h_support"][0] - math.log(5)) < 1e-12
+    assert abs(r["lp_support"][0] + math.log(5)) < 1e-12
+
+
+def test_singleton_support_exact_zeros():
+    rng = np.random.default_rng(7)
+    l = rng.normal(size=(3, 50)) * 3
+    ids = np.array([[4, -1, -1], [-1, 9, -1], [-1, -1, 31]], dtype=np.int32)
+    y = [4, 9, 31]
+    r = oracle.score(l, y, support=ids)
+    assert np.all(r["h_support"] == 0.0)
+    assert np.all(r["lp_support"] == 0.0)
+    assert np.all(r["valid"] == 1)
+    g = oracle.score_grad(l, y, g_h_support=np.ones(3), support=ids)
+    assert np.all(g == 0.0)  # zero entropy gradient for a singleton
+    g = oracle.score_grad(l, y, g_lp_support=np.ones(3), support=ids)
+    assert np.all(g == 0.0)  # lp_S is identically 0
+
+
+def test_bf16_and_fp32_widening():
+    # bf16 patterns and their exact values, widened independently of the oracle
+    bits = np.array([[0x3F80, 0xC000, 0x4049, 0x0000, 0xBF00, 0x4180]], dtype=np.uint16)
+    vals = np.array([[1.0, -2.0, 3.140625, 0.0, -0.5, 16.0]])
+    a = oracle.score(bits, [2])
+    b = oracle.score(vals, [2])
+    for k in ("lp_full", "h_full"):
+        assert a[k][0] == b[k][0]
+    f = workloads.bf16_bits_to_f32(bits).astype(np.float32)
+    c = oracle.score(f, [2])
+    assert c["lp_full"][0] == a["lp_full"][0]
+
+
+def test_lmhead_logits_match_numpy_matmul():
+    rng = np.random.default_rng(11)
+    h = workloads.to_bf16_bits(rng.normal(size=(6, 96)).astype(np.float32))
+    w = workloads.to_bf16_bits((rng.normal(size=(40, 96)) * 0.02).astype(np.float32))
+    sel = np.array([5, 0, 3], dtype=np.int32)
+    got = oracle.lmhead_logits(h, w, sel, 0.8)
+    hf = workloads.bf16_bits_to_f32(h).astype(np.float64)
+    wf = workloads.bf16_bits_to_f32(w).astype(np.float64)
+    want = hf[sel] @ wf.T / 0.8
+    assert np.allclose(got, want, rtol=1e-13, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# brute force on tiny rows, written without sorting or prefix scans
+
+
+def _stable_rank(z):
+    """rank_j = #{i : z_i > z_j or (z_i == z_j and i < j)} (descending value,
+    ascending id)."""
+    n = len(z)
+    return np.array([sum(1 for i in range(n) if z[i] > z[j] or (z[i] == z[j] and i < j))
+                     for j in range(n)])
+
+
+def _brute_support(z, k, p, min_p):
+    n = len(z)
+    rank = _stable_rank(z)
+    s1 = [j for j in range(n) if (k <= 0 or k >= n) or rank[j] < k]
+    w = np.exp(z - z.max())
+    mass1 = w[s1].sum()
+    if p < 1.0:
+        # smallest cardinality of any subset of S1 whose mass reaches p * mass1
+        best = None
+        for size in range(1, len(s1) + 1):
+            for sub in itertools.combinations(s1, size):
+                if w[list(sub)].sum() >= p * mass1:
+                    best = size
+                    break
+            if best is not None:
+                break
+        s2 = [j for j in s1 if rank[j] < best]
+    else:
+        s2 = s1
+    if min_p > 0:
+        s2 = [j for j in s2 if w[j] >= min_p * w.max()]
+    return sorted(s2)
+
+
+def test_brute_force_support_with_ties():
+    rng = np.random.default_rng(3)
+    checked = 0
+    for trial in range(300):
+        n = int(rng.integers(2, 11))
+        # small integer grid so that ties are frequent
+        z = rng.integers(-3, 4, size=n).astype(np.float64) * 0.5
+        k = int(rng.integers(0, n + 2))
+        p = float(rng.choice([1.0, rng.uniform(0.05, 0.999)]))
+        min_p = float(rng.choice([0.0, rng.uniform(0.01, 0.9)]))
+        r = oracle.score(z[None, :], [0], top_k=k, top_p=p, min_p=min_p, want_mask=True)
+        # skip decisions within rounding distance of the boundary
+        if r["topp_margin"][0] < 1e-9 or r["minp_margin"][0] < 1e-9:
+            continue
+        want = _brute_support(z, k, p, min_p)
+        got = sorted(np.nonzero(r["mask"][0])[0].tolist())
+        assert got == want, (z, k, p, min_p)
+        checked += 1
+    assert checked > 250
+
+
+def test_support_size_monotone_in_p_and_k():
+    rng = np.random.default_rng(9)
+    l = (rng.normal(size=(4, 300)) * 2).astype(np.float32)
+    y = [0, 1, 2, 3]
+    prev = np.zeros(4, dtype=np.int64)
+    for p in [0.1, 0.3, 0.5, 0.7, 0.9, 0.99, 1.0]:
+        s = oracle.score(l, y, top_p=p)["support_size"]
+        assert np.all(s >= prev)
+        prev = s
+    prev = np.zeros(4, dtype=np.int64)
+    for k in [1, 2, 5, 20, 100, 299, 0]:
+        s = oracle.score(l, y, top_k=k, top_p=0.8)["support_size"]
+        assert np.all(s >= prev)
+        prev = s
+
+
+def test_topk_keeps_exactly_k_lowest_ids_on_all_equal_row():
+    l = np.zeros((1, 64), dtype=np.float32)
+    r = oracle.score(l, [0], top_k=7, want_mask=True)
+    assert np.nonzero(r["mask"][0])[0].tolist() == list(range(7))
+
+
+def test_min_p_to_zero_gives_topp_support():
+    rng = np.random.default_rng(1)
+    l = rng.normal(size=(3, 500)) * 3
+    a = oracle.score(l, [0, 0, 0], top_p=0.9, want_mask=True)
+    b = oracle.score(l, [0, 0, 0], top_p=0.9, min_p=1e-300, want_mask=True)
+    assert np.array_equal(a["mask"], b["mask"])
+
+
+# ---------------------------------------------------------------------------
+# invariances of the definitions
+
+
+def test_shift_and_temperature_invariance():
+    rng = np.random.default_rng(21)
+    l = rng.normal(size=(5, 400)) * 2
+    y = rng.integers(0, 400, size=5)
+    kw = dict(top_k=100, top_p=0.9, min_p=0.01, want_mask=True)
+    a = oracle.score(l, y, temperature=0.7, **kw)
+    b = oracle.score(l + 3.25, y, temperature=0.7, **kw)   # constant shift
+    c = oracle.score(l * 2.0, y, temperature=1.4, **kw)    # (a l) / (a T)
+    for o in (b, c):
+        assert np.array_equal(a["mask"], o["mask"])
+        for k in ("lp_full", "lp_support", "h_full", "h_support"):
+            assert np.allclose(a[k], o[k], rtol=1e-12, atol=1e-11)
+
+
+# ---------------------------------------------------------------------------
+# gradients: central finite differences in fp64
+
+
+def _fd_check(l, y, T, kind, **filt):
+    rows, n = l.shape
+    h = 1e-6
+    g = np.zeros(rows)
+    g[:] = 1.0
+    kw = {kind: g}
+    grad = oracle.score_grad(l, y, temperature=T, **kw, **filt)
+    key = {"g_lp_full": "lp_full", "g_lp_support": "lp_support", "g_h_full": "h_full",
+           "g_h_support": "h_support"}[kind]
+    fd = np.zeros_like(l)
+    for j in range(n):
+        lp, lm = l.copy(), l.copy()
+        lp[:, j] += h
+        lm[:, j] -= h
+        fp = oracle.score(lp, y, temperature=T, **filt)[key]
+        fm = oracle.score(lm, y, temperature=T, **filt)[key]
+        fd[:, j] = (fp - fm) / (2 * h)
+    scale = np.abs(fd).max()
+    assert np.abs(grad - fd).max() <= 1e-6 * max(scale, 1e-3), kind
+    return grad
+
+
+@pytest.mark.parametrize("kind", ["g_lp_full", "g_lp_support", "g_h_full", "g_h_support"])
+def test_finite_difference_computed_support(kind):
+    rng = np.random.default_rng(31)
+    rows, n = 3, 40
+    filt = dict(top_k=25, top_p=0.8, min_p=0.02)
+    # continuous logits; keep rows whose support decisions are far from a boundary
+    while True:
+        l = rng.normal(size=(rows, n)) * 1.5
+        r = oracle.score(l, np.zeros(rows, np.int32), temperature=0.8, **filt)
+        if (r["topp_margin"].min() > 1e-3 and r["minp_margin"].min() > 1e-3
+                and r["topk_gap"].min() > 1e-3):
+            break
+    # targets inside the support
+    mask = oracle.score(l, np.zeros(rows, np.int32), temperature=0.8, want_mask=True,
+                        **filt)["mask"]
+    y = np.array([np.nonzero(mask[i])[0][-1] for i in range(rows)], dtype=np.int32)
+    g = _fd_check(l, y, 0.8, kind, **filt)
+    # softmax shift invariance: gradients sum to zero over the row
+    assert np.allclose(g.sum(axis=1), 0.0, atol=1e-12)
+
+
+@pytest.mark.parametrize("kind", ["g_lp_support", "g_h_support"])
+def test_finite_difference_recorded_support(kind):
+    rng = np.random.default_rng(41)
+    l = rng.normal(size=(3, 30)) * 2
+    ids = np.array([[1, 5, 7, -1], [-1, 2, 2, 29], [-1, -1, -1, -1]], dtype=np.int32)
+    y = np.array([5, 29, 11], dtype=np.int32)  # last row: empty support
+    _fd_check(l, y, 1.3, kind, support=ids)
+
+
+def test_empty_support_gradient_is_full_vocab_logprob_gradient():
+    rng = np.random.default_rng(43)
+    l = rng.normal(size=(2, 25))
+    ids = np.full((2, 3), -1, dtype=np.int32)
+    y = np.array([3, 7], dtype=np.int32)
+    a = oracle.score_grad(l, y, g_lp_support=np.ones(2), support=ids)
+    b = oracle.score_grad(l, y, g_lp_full=np.ones(2))
+    assert np.array_equal(a, b)
+    r = oracle.score(l, y, support=ids)
+    assert np.all(r["valid"] == 0) and np.all(r["lp_support"] == r["lp_full"])
+
+
+# ---------------------------------------------------------------------------
+# L1 distance
+
+
+def test_l1_identical_rows():
+    rng = np.random.default_rng(2)
+    d = workloads.to_bf16_bits(rng.normal(size=(3, 1000)).astype(np.float32) * 3)
+    r = oracle.l1(d, d.copy(), want_grad=True)
+    assert np.all(r["l1"] == 0.0) and np.all(r["accept"] == 1.0)
+    assert np.all(r["grad"] == 0.0)
+
+
+def test_l1_two_point_closed_form():
+    a = np.array([0.3, -1.2, 2.0, 5.0])
+    d = np.stack([a, np.zeros(4)], axis=1)
+    t = np.zeros((4, 2))
+    r = oracle.l1(d, t, weight=np.array([1.0, 2.0, 0.5, 0.0]))
+    sig = 1.0 / (1.0 + np.exp(-a))
+    want = 2.0 * np.abs(sig - 0.5)
+    assert np.allclose(r["l1"], want, rtol=1e-13)
+    assert np.allclose(r["accept"], 1.0 - np.abs(sig - 0.5), rtol=1e-13)
+
+
+def test_l1_identities_and_bounds():
+    rng = np.random.default_rng(4)
+    d = rng.normal(size=(6, 300)) * 3
+    t = d + rng.normal(size=(6, 300)) * 0.5
+    r = oracle.l1(d, t)
+    p = np.exp(d - d.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    q = np.exp(t - t.max(1, keepdims=True))
+    q /= q.sum(1, keepdims=True)
+    # total-variation identity: 1 - L1 / 2 = sum_j min(p_j, q_j)
+    assert np.allclose(1.0 - r["l1"] / 2.0, np.minimum(p, q).sum(1), rtol=1e-12)
+    assert np.all((r["l1"] >= 0) & (r["l1"] <= 2))
+
+
+def test_l1_weighted_loss_special_cases():
+    rng = np.random.default_rng(6)
+    d = rng.normal(size=(5, 200)) * 2
+    t = rng.normal(size=(5, 200)) * 2
+    base = oracle.l1(d, t)
+    one_hot = oracle.l1(d, t, weight=np.array([0, 0, 1.0, 0, 0]))
+    assert abs(one_hot["loss"] - base["l1"][2]) < 1e-15
+    equal = oracle.l1(d, t, weight=np.full(5, 0.37))
+    assert abs(equal["loss"] - base["l1"].mean()) < 1e-14
+    unweighted = oracle.l1(d, t)
+    assert abs(unweighted["loss"] - base["l1"].mean()) < 1e-14
+    zero = oracle.l1(d, t, weight=np.zeros(5), want_grad=True)
+    assert zero["loss"] == 0.0 and np.all(zero["grad"] == 0.0)
+
+
+def test_l1_finite_difference_gradient():
+    rng = np.random.default_rng(8)
+    d = rng.normal(size=(2, 20)) * 2
+    t = d + rng.normal(size=(2, 20))
+    w = np.array([0.3, 0.9])
+    r = oracle.l1(d, t, weight=w, want_grad=True)
+    h = 1e-6
+    fd = np.zeros_like(d)
+    for i in range(2):
+        for j in range(20):
+            dp, dm = d.copy(), d.copy()
+            dp[i, j] += h
+            dm[i, j] -= h
+            fd[i, j] = (oracle.l1(dp, t, weight=w)["loss"] - oracle.l1(dm, t, weight=w)["loss"]) / (2 * h)
+    assert np.abs(r["grad"] - fd).max() < 1e-7
