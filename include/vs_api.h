@@ -1,0 +1,253 @@
+/*
+ * vs_api.h -- C ABI of the B200 (sm_100a) vocabulary-scoring library libvs.so.
+ *
+ * Per-row scoring of language-model logits over the full vocabulary and over
+ * a sampling support, following these pages:
+ *
+ *  [SkyRL]  SkyRL PR #2004 "perf(sample-support): reuse replay scores for
+ *           entropy", section "Implementation": logprobs, optional entropy and
+ *           valid-row metadata returned together; entropy conditioned on the
+ *           recorded support; a singleton support has exactly zero entropy
+ *           and zero entropy gradient; rows without recorded support fall
+ *           back to the full-vocabulary logprob and leave the entropy
+ *           reduction; entropy computation and gradient tracking are separate
+ *           controls; dense support representation.
+ *  [xorl]   xorl issue #71 "Consolidate the exact and generic scoring paths;
+ *           implement top-k/top-p/min-p", section 3: the transform program
+ *           (temperature, then stable token-id top-k, then inclusive top-p,
+ *           then min-p relative to the original row max; top_p == 1 is the
+ *           identity) and section 1: chunked projection, fixed-order LSE,
+ *           support, selected logprob and VJP.
+ *  [DSpark] DeepSpec PR #87 "[Perf] Reuse DSpark probability distance across
+ *           loss and metrics", section "Purpose": per-token L1 distance
+ *           between softmax(draft) and softmax(target), accept_rate =
+ *           clamp(1 - 0.5 L1, 0, 1), weighted L1 loss.
+ *
+ * Notation: row i has logits l[i, 0..V-1] and temperature T_i; z = l / T_i;
+ * p = softmax(z) over the vocabulary; S = support; q = softmax(z on S).
+ *
+ * Conventions for every entry point
+ *  - All array pointers are DEVICE pointers owned by the caller.  The library
+ *    allocates no device memory; where scratch is needed the caller passes a
+ *    workspace sized by the matching *_workspace_size query.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls are asynchronous: they enqueue kernels and return.
+ *  - Every call returns a vs_status.  Argument errors are detected on the
+ *    host before anything is enqueued (VS_ERR_INVALID_ARG /
+ *    VS_ERR_UNSUPPORTED / VS_ERR_WORKSPACE); a failed launch returns
+ *    VS_ERR_CUDA.  vs_last_error() then describes the failure (thread-local
+ *    string, valid until the next call on the same thread).  Nothing is
+ *    thrown across the ABI and nothing traps on the device.
+ *  - Problems in the data of one row (bad target, bad support id, non-finite
+ *    logits) never fail the call: they are reported in that row's status word
+ *    (VS_ROW_* bits) and the row's outputs follow the rules stated below.
+ *  - Logits are row-major [rows, ld] with ld >= vocab.  The logits pointer
+ *    must be 16-byte aligned and ld * sizeof(element) a multiple of 16
+ *    (elements beyond `vocab` in each row are never used).
+ */
+#ifndef VS_API_H
+#define VS_API_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t vs_status;
+#define VS_OK 0
+#define VS_ERR_INVALID_ARG 1
+#define VS_ERR_UNSUPPORTED 2
+#define VS_ERR_WORKSPACE 3
+#define VS_ERR_CUDA 4
+
+typedef int32_t vs_dtype;
+#define VS_F32 0
+#define VS_BF16 1
+
+/* vs_score_args.flags */
+#define VS_WANT_ENTROPY (1u << 0)      /* write entropy_full / entropy_support */
+#define VS_WANT_SUPPORT_MASK (1u << 1) /* write the support_mask bitset */
+#define VS_WANT_GRAD (1u << 2)         /* write ctx for vs_score_bwd */
+
+/* per-row status bits (vs_score_out.status) */
+#define VS_ROW_TARGET_OUT_OF_RANGE (1u << 0)   /* target outside [0, vocab): logprobs NaN */
+#define VS_ROW_TARGET_NOT_IN_SUPPORT (1u << 1) /* non-empty S without y: lp_S = -inf */
+#define VS_ROW_BAD_SUPPORT_ID (1u << 2)        /* a recorded id < -1 or >= vocab: ignored */
+#define VS_ROW_DUP_SUPPORT_ID (1u << 3)        /* a recorded id repeated: counted once */
+#define VS_ROW_NONFINITE_INPUT (1u << 4)       /* NaN/inf logit: outputs NaN, valid 0 */
+
+/* bytes of saved state per row written when VS_WANT_GRAD is set */
+#define VS_CTX_BYTES_PER_ROW 64
+
+/* maximum recorded-support width and fused-head top-k */
+#define VS_MAX_SUPPORT_WIDTH 1024
+#define VS_MAX_FUSED_TOPK 64
+
+/* Arguments shared by vs_score_fwd and vs_score_bwd. */
+typedef struct vs_score_args {
+  int32_t rows;        /* R >= 0 */
+  int32_t vocab;       /* V >= 1 */
+  int64_t ld;          /* row stride of logits, in elements, >= V */
+  vs_dtype dtype;      /* VS_BF16 or VS_F32 */
+  const void* logits;  /* [R, ld] */
+  /* per-row temperature [R] (> 0, finite), or NULL to use temperature_scalar */
+  const float* temperature;
+  float temperature_scalar;
+  const int32_t* targets; /* [R] selected token ids y_i */
+  /* computed support ([xorl] section 3); per-row arrays or NULL + scalar.
+   * A filter is disabled by top_k <= 0 or >= V, top_p >= 1, min_p <= 0.
+   * top_p must lie in (0, 1], min_p in [0, 1). */
+  const int32_t* top_k;
+  int32_t top_k_scalar;
+  const float* top_p;
+  float top_p_scalar;
+  const float* min_p;
+  float min_p_scalar;
+  /* recorded support ([SkyRL]): [R, support_ld] int32 ids, the first
+   * support_width of each row used, -1 = padding anywhere in the row.
+   * NULL selects the computed support.  Giving a recorded support together
+   * with an active filter is VS_ERR_INVALID_ARG. */
+  const int32_t* support_ids;
+  int32_t support_width; /* 0 .. VS_MAX_SUPPORT_WIDTH */
+  int64_t support_ld;    /* >= support_width */
+  uint32_t flags;        /* VS_WANT_* */
+} vs_score_args;
+
+/* Outputs of vs_score_fwd.  Every pointer may be NULL (that output is not
+ * written) unless a flag requires it. */
+typedef struct vs_score_out {
+  float* logprob_full;    /* [R] lp_V = z_y - logsumexp(z) */
+  float* logprob_support; /* [R] lp_S = z_y - logsumexp(z on S); lp_V if S is empty;
+                             -inf if y is not in a non-empty S */
+  float* entropy_full;    /* [R] H_V (needs VS_WANT_ENTROPY) */
+  float* entropy_support; /* [R] H_S, 0 for an empty S (needs VS_WANT_ENTROPY) */
+  uint8_t* valid;         /* [R] 1 iff S is non-empty and the row is finite */
+  uint32_t* status;       /* [R] VS_ROW_* bits */
+  int32_t* support_size;  /* [R] |S| */
+  uint32_t* support_mask; /* [R, ceil(V/32)] bit j%32 of word j/32 set iff j in S
+                             (needs VS_WANT_SUPPORT_MASK) */
+  void* ctx;              /* [R, VS_CTX_BYTES_PER_ROW] saved state (needs VS_WANT_GRAD),
+                             16-byte aligned; opaque, pass unchanged to vs_score_bwd */
+  double* entropy_sum;    /* [1] sum over valid rows of H_S (needs VS_WANT_ENTROPY) */
+  int32_t* valid_count;   /* [1] number of valid rows */
+} vs_score_out;
+
+/* Forward scoring ([SkyRL] Implementation; [xorl] sections 1 and 3).
+ *
+ * Computed support (support_ids == NULL): S = min-p(top-p(top-k(row))) in
+ * the total order (z descending, token id ascending): top-k keeps the first
+ * k; top-p keeps the shortest prefix of that set whose probability, renormalised
+ * over the top-k set, is >= top_p (the crossing token is kept); min-p keeps
+ * tokens with p_j >= min_p * max_j p_j.  With no active filter S is the whole
+ * vocabulary.  Full-vocabulary statistics are always computed.
+ *
+ * Recorded support: S = the distinct ids >= 0 among the first support_width
+ * entries of the row.  Full-vocabulary statistics (and hence a full read of
+ * the row) are computed for every row when logprob_full or entropy_full is
+ * requested, else only for rows whose S is empty (the lp_V fallback).
+ *
+ * Returns VS_ERR_INVALID_ARG for NULL required pointers, R < 0, V < 1,
+ * ld < V, bad alignment, a non-positive or non-finite temperature_scalar,
+ * top_p_scalar outside (0, 1], min_p_scalar outside [0, 1), a flag whose
+ * output pointer is NULL; VS_ERR_UNSUPPORTED for V beyond the resident-row
+ * limit (vs_score_max_vocab) or support_width > VS_MAX_SUPPORT_WIDTH.
+ * Per-row arrays (temperature, top_k, top_p, min_p) are not range-checked on
+ * the host; out-of-range entries behave as documented for the scalars' edges
+ * (top_p >= 1 disables, min_p <= 0 disables, a temperature <= 0 gives NaN). */
+vs_status vs_score_fwd(const vs_score_args* args, const vs_score_out* out, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* Workspace bytes vs_score_fwd needs for these arguments (0 today). */
+size_t vs_score_fwd_workspace_size(const vs_score_args* args);
+
+/* Largest vocabulary vs_score_fwd accepts for a dtype. */
+int32_t vs_score_max_vocab(vs_dtype dtype);
+
+/* dlogits modes for vs_score_bwd */
+#define VS_GRAD_DENSE 0      /* dlogits [R, V] (row stride grad_ld) overwritten */
+#define VS_GRAD_ACCUMULATE 1 /* dlogits [R, V] += gradient */
+#define VS_GRAD_SPARSE 2     /* recorded support only: dlogits [R, support_width] fp32,
+                                the gradient at each listed id (0 at pads, bad ids and
+                                repeats); valid only when no full-vocabulary term
+                                (g_lp_full, g_h_full, or an empty-support row's g_lp_support)
+                                is non-zero */
+
+/* Backward of the forward outputs ([xorl] section 1 "selected logprob + VJP";
+ * [SkyRL] Implementation).  With g_* the upstream gradients of lp_V, lp_S,
+ * H_V, H_S (each [R] fp32 or NULL = 0), and 1_S the support indicator:
+ *
+ *   dl_j = (1/T) * ( g_lpV ([j==y] - p_j) + g_lpS 1_S(j) ([j==y] - q_j)
+ *                   - g_HV p_j (log p_j + H_V) - g_HS 1_S(j) q_j (log q_j + H_S) )
+ *
+ * Empty S: lp_S is lp_V, so g_lpS joins the full-vocabulary term; H_S has no
+ * gradient.  y outside a non-empty S, an out-of-range y, or a non-finite row:
+ * no logprob gradient (and no gradient at all for a non-finite row).
+ * `args` must be the arguments of the forward call and `ctx` its saved state.
+ * dlogits has dtype dl_dtype (VS_F32 or VS_BF16, rounded to nearest even),
+ * row stride grad_ld elements (>= V in the dense modes, >= support_width in
+ * the sparse mode), 16-byte aligned with grad_ld * sizeof a multiple of 16. */
+vs_status vs_score_bwd(const vs_score_args* args, const void* ctx, const float* g_lp_full,
+                       const float* g_lp_support, const float* g_h_full,
+                       const float* g_h_support, void* dlogits, vs_dtype dl_dtype,
+                       int64_t grad_ld, int32_t mode, void* stream);
+
+/* Draft/target probability distance ([DSpark] Purpose).  Per row i:
+ *   p = softmax(draft_i), q = softmax(target_i)          (no temperature)
+ *   l1[i] = sum_j |p_j - q_j|
+ *   accept_rate[i] = clamp(1 - 0.5 * l1[i], 0, 1)
+ *   loss_num_den_loss[0..2] = { sum_i w_i l1_i, sum_i w_i, num / den (0 if den == 0) }
+ * with w = row_weight (NULL = all ones).  When grad_draft is non-NULL it
+ * receives d loss / d draft (target detached):
+ *   (w_i / sum w) p_j (s_j - sum_k p_k s_k),  s = sign(p - q), sign(0) = 0.
+ * Any of l1, accept_rate, loss_num_den_loss, grad_draft may be NULL.
+ * draft and target are [rows, ld] of `dtype`; grad_draft is [rows, grad_ld]
+ * of grad_dtype.  Needs a workspace of vs_l1_distance_workspace_size(rows)
+ * bytes (16-byte aligned) when loss_num_den_loss or grad_draft is requested. */
+vs_status vs_l1_distance(int32_t rows, int32_t vocab, int64_t ld, vs_dtype dtype,
+                         const void* draft, const void* target, const float* row_weight,
+                         float* l1, float* accept_rate, float* loss_num_den_loss,
+                         void* grad_draft, vs_dtype grad_dtype, int64_t grad_ld,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+size_t vs_l1_distance_workspace_size(int32_t rows);
+
+/* Fused LM-head scoring ([xorl] section 1: chunked projection -> fixed-order
+ * LSE -> support -> selected logprob; [SkyRL] Performance: the full logits
+ * are never materialised).
+ *   z[i, v] = (sum_k hidden[i, k] * weight[v, k]) / T_i
+ * computed on tcgen05 tensor cores (bf16 inputs, fp32 accumulation) tile by
+ * tile; each tile updates per-row online (max, sum exp, sum z exp) and a
+ * per-row top-k candidate list; a merge step then forms S = min-p(top-p(
+ * top-k)) over the k candidates and writes lp_V, lp_S, H_V, H_S (entropy
+ * outputs need VS_WANT_ENTROPY), valid, status, support_size, and, when
+ * non-NULL, topk_ids [rows, top_k] (the top-k token ids in the total order)
+ * and topk_logprob [rows, top_k] (their full-vocabulary logprobs).
+ * hidden [rows, hidden_dim] and weight [vocab, hidden_dim] are bf16, K-major,
+ * row strides ldh/ldw elements (multiples of 8), 16-byte aligned; hidden_dim
+ * a multiple of 64.  top_k in [1, VS_MAX_FUSED_TOPK] (top-p without top-k is
+ * not offered here).  Needs vs_fused_lmhead_workspace_size(...) bytes. */
+vs_status vs_fused_lmhead_score(int32_t rows, int32_t vocab, int32_t hidden_dim,
+                                const void* hidden, int64_t ldh, const void* weight,
+                                int64_t ldw, const float* temperature,
+                                float temperature_scalar, const int32_t* targets,
+                                int32_t top_k, float top_p, float min_p, uint32_t flags,
+                                const vs_score_out* out, int32_t* topk_ids,
+                                float* topk_logprob, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+size_t vs_fused_lmhead_workspace_size(int32_t rows, int32_t vocab, int32_t hidden_dim,
+                                      int32_t top_k);
+
+/* Message describing the last failed call on this thread ("" after success). */
+const char* vs_last_error(void);
+
+/* Library version, e.g. "0.1.0". */
+const char* vs_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VS_API_H */

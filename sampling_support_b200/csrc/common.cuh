@@ -1,0 +1,238 @@
+// Device helpers shared by the scoring kernels (sm_100a).
+#pragma once
+
+#include <cooperative_groups.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace cg = cooperative_groups;
+
+namespace vs {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kInf = __builtin_huge_valf();
+
+// Iteration cap for every mbarrier wait: try_wait suspends the thread for a
+// hardware-defined interval per attempt, so this bounds a wait to seconds.
+constexpr uint32_t kWaitLimit = 1u << 24;
+
+// Per-row status bit set when a bounded device wait gave up (never expected).
+constexpr uint32_t kRowDeviceTimeout = 1u << 5;
+
+// 2^x on the MUFU unit (ex2.approx.ftz.f32: PTX ISA instruction, relative
+// error about 2^-22; -inf -> +0).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ---------------------------------------------------------------------------
+// monotone integer keys: key(a) < key(b)  <=>  a < b  for finite values, with
+// -0 mapped onto +0 so that equal values have equal keys.
+
+__device__ __forceinline__ uint32_t key_of(uint16_t raw) {
+  uint32_t x = raw;
+  if (x == 0x8000u) x = 0;
+  return (x & 0x8000u) ? (~x & 0xFFFFu) : (x | 0x8000u);
+}
+__device__ __forceinline__ uint32_t key_of(uint32_t raw) {
+  uint32_t x = raw;
+  if (x == 0x80000000u) x = 0;
+  return (x & 0x80000000u) ? ~x : (x | 0x80000000u);
+}
+__device__ __forceinline__ float value_of(uint16_t raw) {
+  return __uint_as_float(static_cast<uint32_t>(raw) << 16);
+}
+__device__ __forceinline__ float value_of(uint32_t raw) { return __uint_as_float(raw); }
+
+template <typename Raw>
+struct KeyTraits;
+template <>
+struct KeyTraits<uint16_t> {
+  static constexpr int kBits = 16;
+  static constexpr uint32_t kInfKey = 0xFF80u;  // key of +inf
+  __device__ static float decode(uint32_t k) {
+    uint32_t bits = (k & 0x8000u) ? (k & 0x7FFFu) : (~k & 0xFFFFu);
+    return __uint_as_float(bits << 16);
+  }
+};
+template <>
+struct KeyTraits<uint32_t> {
+  static constexpr int kBits = 32;
+  static constexpr uint32_t kInfKey = 0xFF800000u;
+  __device__ static float decode(uint32_t k) {
+    uint32_t bits = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+    return __uint_as_float(bits);
+  }
+};
+
+// Unpack one 16-byte vector of raw elements.
+__device__ __forceinline__ void unpack(const uint4& q, uint16_t (&r)[8]) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    r[2 * i] = static_cast<uint16_t>(w[i] & 0xFFFFu);
+    r[2 * i + 1] = static_cast<uint16_t>(w[i] >> 16);
+  }
+}
+__device__ __forceinline__ void unpack(const uint4& q, uint32_t (&r)[4]) {
+  r[0] = q.x;
+  r[1] = q.y;
+  r[2] = q.z;
+  r[3] = q.w;
+}
+
+// ---------------------------------------------------------------------------
+// online (max, sum 2^(u - max), sum (u - max) 2^(u - max)) in base-2 units.
+// A row's natural-log statistics follow as
+//   LSE = ln2 (m + log2 Z),   H = ln2 (log2 Z - A / Z)   (A <= 0).
+
+struct Stats {
+  float m, z, a;
+};
+
+__device__ __forceinline__ Stats stats_empty() { return {-kInf, 0.f, 0.f}; }
+
+// Merge b into s.  An empty side (z == 0) is skipped; NaN/inf propagate.
+__device__ __forceinline__ void stats_merge(Stats& s, const Stats& b) {
+  if (b.z == 0.f) return;
+  if (s.z == 0.f) {
+    s = b;
+    return;
+  }
+  const float mn = fmaxf(s.m, b.m);
+  const float f1 = ex2(s.m - mn), f2 = ex2(b.m - mn);
+  s.a = f1 * fmaf(s.m - mn, s.z, s.a) + f2 * fmaf(b.m - mn, b.z, b.a);
+  s.z = f1 * s.z + f2 * b.z;
+  s.m = mn;
+}
+
+// Add a batch of N values u[] (already scaled to base-2 units).
+template <int N>
+__device__ __forceinline__ void stats_add(Stats& s, const float (&u)[N]) {
+  float bm = u[0];
+#pragma unroll
+  for (int i = 1; i < N; ++i) bm = fmaxf(bm, u[i]);
+  if (bm > s.m) {
+    if (s.z != 0.f) {
+      const float f = ex2(s.m - bm);
+      s.a = f * fmaf(s.m - bm, s.z, s.a);
+      s.z *= f;
+    }
+    s.m = bm;
+  }
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    const float d = u[i] - s.m;
+    const float e = ex2(d);
+    s.z += e;
+    s.a = fmaf(d, e, s.a);
+  }
+}
+
+__device__ __forceinline__ Stats shfl_xor(const Stats& s, int lane_mask) {
+  return {__shfl_xor_sync(0xffffffffu, s.m, lane_mask), __shfl_xor_sync(0xffffffffu, s.z, lane_mask),
+          __shfl_xor_sync(0xffffffffu, s.a, lane_mask)};
+}
+
+// Deterministic block reduction; result valid in every thread.  `scratch`
+// holds at least blockDim.x / 32 entries.
+__device__ __forceinline__ Stats block_reduce(Stats s, Stats* scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) stats_merge(s, shfl_xor(s, o));
+  if (lane == 0) scratch[warp] = s;
+  __syncthreads();
+  Stats t = stats_empty();
+  const int nw = blockDim.x >> 5;
+  for (int w = 0; w < nw; ++w) stats_merge(t, scratch[w]);
+  __syncthreads();
+  return t;
+}
+
+template <typename T>
+__device__ __forceinline__ T block_sum(T v, T* scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  T t = 0;
+  const int nw = blockDim.x >> 5;
+  for (int w = 0; w < nw; ++w) t += scratch[w];
+  __syncthreads();
+  return t;
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier + bulk async copy (global -> shared), PTX ISA.
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete; false after the
+// iteration cap.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// Bulk copy `bytes` (multiple of 16, both addresses 16-byte aligned) from
+// global memory into this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Largest bulk piece issued at once (keeps each instruction modest).
+constexpr uint32_t kBulkPiece = 32768;
+
+// Load `bytes` from src into dst via bulk copies on `bar` (thread 0 only).
+// The caller arms the barrier with the full byte count first.
+__device__ __forceinline__ void bulk_load_all(void* dst, const void* src, uint32_t bytes,
+                                              uint64_t* bar) {
+  for (uint32_t off = 0; off < bytes; off += kBulkPiece) {
+    const uint32_t n = min(kBulkPiece, bytes - off);
+    bulk_load(static_cast<char*>(dst) + off, static_cast<const char*>(src) + off, n, bar);
+  }
+}
+
+}  // namespace vs

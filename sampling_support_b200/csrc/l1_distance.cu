@@ -1,0 +1,345 @@
+// Draft/target probability distance (DeepSpec PR #87, DSpark, section
+// "Purpose"): one softmax of the draft row and one of the target row, one
+// |p - q| reduction, reused for accept_rate = clamp(1 - 0.5 L1, 0, 1) and for
+// the weighted L1 loss; gradient with respect to the draft logits only.
+//
+// One thread-block cluster per row.  Each CTA bulk-copies its slice of BOTH
+// rows into shared memory once; the three passes (online max / sum for p and
+// q, the |p - q| and sum p s reduction, the gradient) read that copy, so the
+// whole job reads each logit from HBM exactly once and writes the gradient
+// once.  Cross-CTA sums go through distributed shared memory in rank order;
+// cross-row sums (the loss) are reduced by a single block in row order.
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace vs {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+struct L1Shared {
+  uint64_t bar;
+  Stats part[2];
+  Stats gathered[8][2];
+  Stats red[kWarps];
+  float fred[kWarps];
+  float agg_l1, agg_ps;
+  uint32_t timeout;
+};
+
+struct L1Params {
+  int32_t rows, vocab;
+  int64_t ld;
+  const void* draft;
+  const void* target;
+  const float* row_weight;
+  float* l1;
+  float* accept;
+  void* grad;
+  int64_t grad_ld;
+  double* ws_wsum;  // [1] sum of weights (written by l1_wsum_kernel)
+  double* ws_wl1;   // [rows] w_i * L1_i
+  int32_t chunk;
+};
+
+__device__ __forceinline__ float sgn(float d) { return d > 0.f ? 1.f : (d < 0.f ? -1.f : 0.f); }
+
+template <typename Raw, typename G>
+__global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
+  constexpr int VEC = 16 / sizeof(Raw);
+  cg::cluster_group cluster = cg::this_cluster();
+  const uint32_t rank = cluster.block_rank();
+  const uint32_t CL = cluster.num_blocks();
+  const int row = blockIdx.x / CL;
+  const int tid = threadIdx.x;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  Raw* bd = reinterpret_cast<Raw*>(smem_raw);
+  Raw* bt = bd + P.chunk;
+  L1Shared& sh = *reinterpret_cast<L1Shared*>(smem_raw + 2 * static_cast<size_t>(P.chunk) * sizeof(Raw));
+
+  const int V = P.vocab;
+  const int c0 = static_cast<int>(rank) * P.chunk;
+  const int c1 = min(V, c0 + P.chunk);
+  const int n = max(0, c1 - c0);
+  const Raw* gd = static_cast<const Raw*>(P.draft) + static_cast<int64_t>(row) * P.ld;
+  const Raw* gt = static_cast<const Raw*>(P.target) + static_cast<int64_t>(row) * P.ld;
+
+  if (tid == 0) {
+    mbar_init(&sh.bar, 1);
+    fence_barrier_init();
+    sh.timeout = 0;
+  }
+  __syncthreads();
+  const uint32_t bytes = static_cast<uint32_t>((static_cast<size_t>(n) * sizeof(Raw) + 15) & ~size_t(15));
+  if (tid == 0 && bytes > 0) {
+    mbar_arrive_expect_tx(&sh.bar, 2 * bytes);
+    bulk_load_all(bd, gd + c0, bytes, &sh.bar);
+    bulk_load_all(bt, gt + c0, bytes, &sh.bar);
+  }
+  if (bytes > 0 && !mbar_wait(&sh.bar, 0)) {
+    atomicOr(&sh.timeout, 1u);
+    mbar_wait(&sh.bar, 0);
+  }
+  __syncthreads();
+
+  // pass 1: online statistics of both rows (base-2 units, no temperature)
+  Stats sd = stats_empty(), st = stats_empty();
+  const int nfull = n / VEC;
+  const uint4* d4 = reinterpret_cast<const uint4*>(bd);
+  const uint4* t4 = reinterpret_cast<const uint4*>(bt);
+  for (int v = tid; v < nfull; v += blockDim.x) {
+    Raw rd[VEC], rt[VEC];
+    unpack(d4[v], rd);
+    unpack(t4[v], rt);
+    float ud[VEC], ut[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) {
+      ud[i] = __fmul_rn(value_of(rd[i]), kLog2e);
+      ut[i] = __fmul_rn(value_of(rt[i]), kLog2e);
+    }
+    stats_add(sd, ud);
+    stats_add(st, ut);
+  }
+  for (int j = nfull * VEC + tid; j < n; j += blockDim.x) {
+    float ud[1] = {__fmul_rn(value_of(bd[j]), kLog2e)};
+    float ut[1] = {__fmul_rn(value_of(bt[j]), kLog2e)};
+    stats_add(sd, ud);
+    stats_add(st, ut);
+  }
+  sd = block_reduce(sd, sh.red);
+  st = block_reduce(st, sh.red);
+  if (tid == 0) {
+    sh.part[0] = sd;
+    sh.part[1] = st;
+  }
+  cluster.sync();
+  if (tid < static_cast<int>(CL)) {
+    const L1Shared* rsh = cluster.map_shared_rank(&sh, tid);
+    sh.gathered[tid][0] = rsh->part[0];
+    sh.gathered[tid][1] = rsh->part[1];
+  }
+  __syncthreads();
+  Stats Sd = stats_empty(), St = stats_empty();
+  for (uint32_t r = 0; r < CL; ++r) {
+    stats_merge(Sd, sh.gathered[r][0]);
+    stats_merge(St, sh.gathered[r][1]);
+  }
+  const float md = Sd.m, ld2 = log2f(Sd.z);
+  const float mt = St.m, lt2 = log2f(St.z);
+
+  // pass 2: L1 = sum |p - q| and sum_k p_k sign(p_k - q_k)
+  float l1 = 0.f, ps = 0.f;
+  for (int v = tid; v < nfull; v += blockDim.x) {
+    Raw rd[VEC], rt[VEC];
+    unpack(d4[v], rd);
+    unpack(t4[v], rt);
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) {
+      const float p = ex2((__fmul_rn(value_of(rd[i]), kLog2e) - md) - ld2);
+      const float q = ex2((__fmul_rn(value_of(rt[i]), kLog2e) - mt) - lt2);
+      const float d = p - q;
+      l1 += fabsf(d);
+      ps = fmaf(p, sgn(d), ps);
+    }
+  }
+  for (int j = nfull * VEC + tid; j < n; j += blockDim.x) {
+    const float p = ex2((__fmul_rn(value_of(bd[j]), kLog2e) - md) - ld2);
+    const float q = ex2((__fmul_rn(value_of(bt[j]), kLog2e) - mt) - lt2);
+    const float d = p - q;
+    l1 += fabsf(d);
+    ps = fmaf(p, sgn(d), ps);
+  }
+  l1 = block_sum(l1, sh.fred);
+  ps = block_sum(ps, sh.fred);
+  if (tid == 0) {
+    sh.agg_l1 = l1;
+    sh.agg_ps = ps;
+  }
+  cluster.sync();
+  float L1 = 0.f, PS = 0.f;
+  for (uint32_t r = 0; r < CL; ++r) {
+    const L1Shared* rsh = cluster.map_shared_rank(&sh, r);
+    L1 += rsh->agg_l1;
+    PS += rsh->agg_ps;
+  }
+  const float w = P.row_weight ? P.row_weight[row] : 1.f;
+  if (rank == 0 && tid == 0) {
+    if (P.l1) P.l1[row] = L1;
+    if (P.accept) P.accept[row] = fminf(1.f, fmaxf(0.f, 1.f - 0.5f * L1));
+    if (P.ws_wl1) P.ws_wl1[row] = static_cast<double>(w) * static_cast<double>(L1);
+  }
+
+  // pass 3: d loss / d draft_j = (w / sum w) p_j (s_j - sum_k p_k s_k)
+  if (P.grad) {
+    const double wsum = *P.ws_wsum;
+    const float coef = wsum > 0.0 ? static_cast<float>(static_cast<double>(w) / wsum) : 0.f;
+    G* go = static_cast<G*>(P.grad) + static_cast<int64_t>(row) * P.grad_ld + c0;
+    for (int v = tid; v < nfull; v += blockDim.x) {
+      Raw rd[VEC], rt[VEC];
+      unpack(d4[v], rd);
+      unpack(t4[v], rt);
+      float out[VEC];
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) {
+        const float p = ex2((__fmul_rn(value_of(rd[i]), kLog2e) - md) - ld2);
+        const float q = ex2((__fmul_rn(value_of(rt[i]), kLog2e) - mt) - lt2);
+        out[i] = coef * p * (sgn(p - q) - PS);
+      }
+      G* dst = go + v * VEC;
+      if constexpr (sizeof(G) == 2) {
+        uint32_t wv[VEC / 2];
+#pragma unroll
+        for (int i = 0; i < VEC / 2; ++i)
+          wv[i] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(out[2 * i]))) |
+                  (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(out[2 * i + 1]))) << 16);
+        if constexpr (VEC == 8)
+          __stcs(reinterpret_cast<uint4*>(dst), make_uint4(wv[0], wv[1], wv[2], wv[3]));
+        else
+          __stcs(reinterpret_cast<uint2*>(dst), make_uint2(wv[0], wv[1]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < VEC; i += 4)
+          __stcs(reinterpret_cast<float4*>(dst + i), make_float4(out[i], out[i + 1], out[i + 2], out[i + 3]));
+      }
+    }
+    for (int j = nfull * VEC + tid; j < n; j += blockDim.x) {
+      const float p = ex2((__fmul_rn(value_of(bd[j]), kLog2e) - md) - ld2);
+      const float q = ex2((__fmul_rn(value_of(bt[j]), kLog2e) - mt) - lt2);
+      const float g = coef * p * (sgn(p - q) - PS);
+      if constexpr (sizeof(G) == 2)
+        go[j] = static_cast<G>(__bfloat16_as_ushort(__float2bfloat16_rn(g)));
+      else
+        go[j] = g;
+    }
+  }
+  if (sh.timeout && tid == 0 && P.l1) P.l1[row] = __int_as_float(0x7fc00000);
+  cluster.sync();
+}
+
+// sum of row weights, in row order (one block)
+__global__ void l1_wsum_kernel(const float* w, int rows, double* out) {
+  __shared__ double red[32];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < rows; i += blockDim.x) s += w ? static_cast<double>(w[i]) : 1.0;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) red[warp] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) t += red[i];
+    *out = t;
+  }
+}
+
+// loss numerator / denominator / value (one block)
+__global__ void l1_loss_kernel(const double* wl1, const double* wsum, int rows, float* out3) {
+  __shared__ double red[32];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < rows; i += blockDim.x) s += wl1[i];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) red[warp] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) t += red[i];
+    const double den = *wsum;
+    out3[0] = static_cast<float>(t);
+    out3[1] = static_cast<float>(den);
+    out3[2] = den > 0.0 ? static_cast<float>(t / den) : 0.f;
+  }
+}
+
+}  // namespace
+
+size_t l1_workspace_bytes(int rows) { return 16 + 8 * static_cast<size_t>(rows > 0 ? rows : 0); }
+
+// Cluster size and per-CTA slice for a pair of rows of `vocab` elements.
+int l1_cluster_size(int vocab, vs_dtype dtype, int* chunk) {
+  const int esize = dtype == VS_BF16 ? 2 : 4;
+  const int target = 40 * 1024 / (2 * esize);
+  int cl = 1;
+  while (cl < 8 && (vocab + cl - 1) / cl > target) ++cl;
+  int e = (vocab + cl - 1) / cl;
+  e = (e + 31) & ~31;
+  *chunk = e;
+  return cl;
+}
+
+int l1_max_vocab(vs_dtype dtype) {
+  const int esize = dtype == VS_BF16 ? 2 : 4;
+  return 8 * (96 * 1024 / (2 * esize));
+}
+
+cudaError_t launch_l1(int rows, int vocab, int64_t ld, vs_dtype dtype, const void* draft,
+                      const void* target, const float* row_weight, float* l1, float* accept,
+                      float* loss3, void* grad, vs_dtype gdtype, int64_t grad_ld, void* ws,
+                      cudaStream_t s) {
+  int chunk = 0;
+  const int cl = l1_cluster_size(vocab, dtype, &chunk);
+  L1Params P{};
+  P.rows = rows;
+  P.vocab = vocab;
+  P.ld = ld;
+  P.draft = draft;
+  P.target = target;
+  P.row_weight = row_weight;
+  P.l1 = l1;
+  P.accept = accept;
+  P.grad = grad;
+  P.grad_ld = grad_ld;
+  P.chunk = chunk;
+  const bool need_ws = loss3 != nullptr || grad != nullptr;
+  P.ws_wsum = need_ws ? static_cast<double*>(ws) : nullptr;
+  P.ws_wl1 = need_ws ? static_cast<double*>(ws) + 2 : nullptr;
+  if (need_ws) {
+    l1_wsum_kernel<<<1, 1024, 0, s>>>(row_weight, rows, P.ws_wsum);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const size_t esize = dtype == VS_BF16 ? 2 : 4;
+  const size_t smem = 2 * static_cast<size_t>(chunk) * esize + sizeof(L1Shared);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(rows) * cl, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cl;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaSuccess;
+#define VS_L1_LAUNCH(RAW, G)                                                                  \
+  do {                                                                                        \
+    e = cudaFuncSetAttribute(l1_kernel<RAW, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             static_cast<int>(smem));                                         \
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, l1_kernel<RAW, G>, P);                 \
+  } while (0)
+  if (rows > 0) {
+    if (dtype == VS_BF16) {
+      if (gdtype == VS_BF16) VS_L1_LAUNCH(uint16_t, uint16_t);
+      else VS_L1_LAUNCH(uint16_t, float);
+    } else {
+      if (gdtype == VS_BF16) VS_L1_LAUNCH(uint32_t, uint16_t);
+      else VS_L1_LAUNCH(uint32_t, float);
+    }
+  }
+#undef VS_L1_LAUNCH
+  if (e != cudaSuccess) return e;
+  if (loss3) {
+    l1_loss_kernel<<<1, 1024, 0, s>>>(P.ws_wl1, P.ws_wsum, rows, loss3);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+}  // namespace vs

@@ -1,0 +1,878 @@
+// Forward scoring kernels.
+//
+//  * score_computed_kernel: computed support (temperature -> stable token-id
+//    top-k -> inclusive top-p -> min-p against the original row max; xorl
+//    issue #71, section 3).  One thread-block cluster per row; each CTA pulls
+//    its slice of the row from HBM once, with bulk asynchronous copies, into
+//    shared memory, and every later pass (radix select, support sums, tie
+//    resolution, mask) reads that copy.  Row statistics and histograms are
+//    combined across the cluster through distributed shared memory in a
+//    fixed rank order, so results are deterministic.
+//  * score_recorded_kernel: recorded support (SkyRL PR #2004,
+//    "Implementation": dense -1-padded id list).  One CTA per row gathers the
+//    support logits; rows with an empty support (full-vocabulary fallback),
+//    or every row when full statistics are requested, also stream the whole
+//    row once with 16-byte loads.
+
+#include <climits>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace vs {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kBins = 256;
+
+// Shared state of one CTA, placed after the row slice in dynamic smem.
+struct SelShared {
+  unsigned long long mass[2][kBins];  // fixed-point mass histogram (double-buffered)
+  unsigned long long gmass[kBins];    // cluster-reduced
+  uint32_t cnt[2][kBins];
+  uint32_t gcnt[kBins];
+  uint64_t bar;
+  Stats part;  // this CTA's row statistics
+  Stats gathered[8];
+  Stats red[kWarps];
+  float fred[kWarps];
+  uint32_t ured[kWarps];
+  // aggregate pass partials (this CTA)
+  float agg_mass, agg_a;
+  uint32_t agg_ngt, agg_eq;
+  // broadcast slots
+  unsigned long long b_target, b_above_cnt, b_above_mass, b_at_cnt, b_at_mass;
+  uint32_t b_digit;
+  int32_t tie_cut;
+  uint32_t timeout;
+  uint32_t scan_tot[kWarps];
+};
+
+struct Desc {
+  uint32_t key;
+  unsigned long long above_cnt, above_mass, at_cnt, at_mass;
+};
+
+__device__ __forceinline__ float fx_scale(int shift) {
+  return __int_as_float((127 + shift) << 23);
+}
+
+// Visit every element of the CTA's slice: f(local_index, raw).
+template <typename Raw, typename F>
+__device__ __forceinline__ void for_each(const Raw* buf, int n, F&& f) {
+  constexpr int VEC = 16 / sizeof(Raw);
+  const int nfull = n / VEC;
+  const uint4* v4 = reinterpret_cast<const uint4*>(buf);
+  for (int v = threadIdx.x; v < nfull; v += blockDim.x) {
+    Raw r[VEC];
+    unpack(v4[v], r);
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) f(v * VEC + i, r[i]);
+  }
+  for (int j = nfull * VEC + threadIdx.x; j < n; j += blockDim.x) f(j, buf[j]);
+}
+
+// Warp 0: find, scanning bins from the top (largest key first), the bin where
+// the cumulative `by` quantity first reaches `need` (>= 1).  Returns the
+// digit and the sums (count and mass) of the bins strictly above it, in lane 0.
+__device__ void scan_bins(const uint32_t* gcnt, const unsigned long long* gmass, bool by_mass,
+                          unsigned long long need, uint32_t& digit,
+                          unsigned long long& above_cnt, unsigned long long& above_mass) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long v[8];
+  unsigned long long lsum = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int b = 255 - 8 * lane - i;
+    v[i] = by_mass ? gmass[b] : static_cast<unsigned long long>(gcnt[b]);
+    lsum += v[i];
+  }
+  unsigned long long incl = lsum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  const unsigned long long excl = incl - lsum;
+  const bool hit = excl < need && need <= incl;
+  const uint32_t ballot = __ballot_sync(0xffffffffu, hit);
+  int d = -1;
+  if (ballot != 0) {
+    const int hl = __ffs(ballot) - 1;
+    int local = -1;
+    if (lane == hl) {
+      unsigned long long s = excl;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (local < 0 && s + v[i] >= need) local = 255 - 8 * lane - i;
+        if (local < 0) s += v[i];
+      }
+    }
+    d = __shfl_sync(0xffffffffu, local, hl);
+  } else {
+    // target beyond the total (cannot happen for consistent targets): take
+    // the lowest non-empty bin so that the result stays well defined.
+    unsigned long long any = 0;
+    int lowest = -1;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int b = 255 - 8 * lane - i;
+      if (gcnt[b] != 0) lowest = b;
+      any |= gcnt[b];
+    }
+    (void)any;
+    int best = lowest < 0 ? 256 : lowest;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) best = min(best, __shfl_xor_sync(0xffffffffu, best, o));
+    d = best == 256 ? 0 : best;
+  }
+  unsigned long long ac = 0, am = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int b = 255 - 8 * lane - i;
+    if (b > d) {
+      ac += gcnt[b];
+      am += gmass[b];
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ac += __shfl_xor_sync(0xffffffffu, ac, o);
+    am += __shfl_xor_sync(0xffffffffu, am, o);
+  }
+  digit = static_cast<uint32_t>(d);
+  above_cnt = ac;
+  above_mass = am;
+}
+
+// Radix descent over 8-bit digits of the key (most significant first) for
+// the position where the cumulative count (by_mass = false) or fixed-point
+// mass (by_mass = true) of the total order first reaches `target`.
+// target == 0 with by_mass means "ceil(p * total mass)", with the total taken
+// from the first level's histogram.  `hb` selects the histogram buffer and
+// alternates per level, so one cluster barrier per level suffices.
+template <typename Raw>
+__device__ Desc descend(const Raw* buf, int n, float c, float m2, int fx_shift, bool by_mass,
+                        bool need_mass, unsigned long long target, float p, SelShared& sh,
+                        cg::cluster_group& cluster, int& hb) {
+  constexpr int KB = KeyTraits<Raw>::kBits;
+  const uint32_t CL = cluster.num_blocks();
+  const float fxs = fx_scale(fx_shift);
+  uint32_t prefix = 0;
+  unsigned long long above_cnt = 0, above_mass = 0;
+  Desc out{};
+  for (int shift = KB - 8; shift >= 0; shift -= 8) {
+    uint32_t* cnt = sh.cnt[hb];
+    unsigned long long* mass = sh.mass[hb];
+    for (int b = threadIdx.x; b < kBins; b += blockDim.x) {
+      cnt[b] = 0;
+      mass[b] = 0;
+    }
+    __syncthreads();
+    const int pshift = shift + 8;
+    const uint32_t pre = prefix;
+    for_each(buf, n, [&](int, Raw raw) {
+      const uint32_t key = key_of(raw);
+      const bool match = pshift >= KB ? true : ((key >> pshift) == pre);
+      if (match) {
+        const uint32_t digit = (key >> shift) & 255u;
+        atomicAdd(&cnt[digit], 1u);
+        if (need_mass) {
+          const float e = ex2(__fmul_rn(value_of(raw), c) - m2);
+          const unsigned long long fx = __float2ull_rn(e * fxs);
+          if (fx) atomicAdd(&mass[digit], fx);
+        }
+      }
+    });
+    __syncthreads();
+    cluster.sync();
+    for (int b = threadIdx.x; b < kBins; b += blockDim.x) {
+      uint32_t sc = 0;
+      unsigned long long sm = 0;
+      for (uint32_t r = 0; r < CL; ++r) {
+        sc += *cluster.map_shared_rank(&cnt[b], r);
+        sm += *cluster.map_shared_rank(&mass[b], r);
+      }
+      sh.gcnt[b] = sc;
+      sh.gmass[b] = sm;
+    }
+    __syncthreads();
+    hb ^= 1;
+    if (threadIdx.x < 32) {
+      unsigned long long tgt = target;
+      if (tgt == 0) {
+        // implicit target: ceil(p * total mass), clamped to [1, total]
+        unsigned long long tot = 0;
+        for (int i = threadIdx.x; i < kBins; i += 32) tot += sh.gmass[i];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+        double want = ceil(static_cast<double>(p) * static_cast<double>(tot));
+        unsigned long long t = want <= 1.0 ? 1ull
+                               : want >= static_cast<double>(tot)
+                                   ? tot
+                                   : static_cast<unsigned long long>(want);
+        tgt = t < 1 ? 1 : t;
+      }
+      const unsigned long long have = by_mass ? above_mass : above_cnt;
+      const unsigned long long need = tgt > have ? tgt - have : 1;
+      uint32_t digit;
+      unsigned long long ac, am;
+      scan_bins(sh.gcnt, sh.gmass, by_mass, need, digit, ac, am);
+      if (threadIdx.x == 0) {
+        sh.b_target = tgt;
+        sh.b_digit = digit;
+        sh.b_above_cnt = ac;
+        sh.b_above_mass = am;
+        sh.b_at_cnt = sh.gcnt[digit];
+        sh.b_at_mass = sh.gmass[digit];
+      }
+    }
+    __syncthreads();
+    target = sh.b_target;
+    above_cnt += sh.b_above_cnt;
+    above_mass += sh.b_above_mass;
+    prefix = (prefix << 8) | sh.b_digit;
+    out.at_cnt = sh.b_at_cnt;
+    out.at_mass = sh.b_at_mass;
+    __syncthreads();
+  }
+  out.key = prefix;
+  out.above_cnt = above_cnt;
+  out.above_mass = above_mass;
+  return out;
+}
+
+template <typename Raw>
+__global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P) {
+  constexpr int VEC = 16 / sizeof(Raw);
+  using KT = KeyTraits<Raw>;
+  cg::cluster_group cluster = cg::this_cluster();
+  const uint32_t rank = cluster.block_rank();
+  const uint32_t CL = cluster.num_blocks();
+  const int row = blockIdx.x / CL;
+  const int tid = threadIdx.x;
+
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  Raw* buf = reinterpret_cast<Raw*>(smem_raw);
+  SelShared& sh = *reinterpret_cast<SelShared*>(smem_raw + static_cast<size_t>(P.chunk) * sizeof(Raw));
+
+  const int V = P.vocab;
+  const int c0 = static_cast<int>(rank) * P.chunk;
+  const int c1 = min(V, c0 + P.chunk);
+  const int n = max(0, c1 - c0);
+  const Raw* grow = static_cast<const Raw*>(P.logits) + static_cast<int64_t>(row) * P.ld;
+
+  if (tid == 0) {
+    mbar_init(&sh.bar, 1);
+    fence_barrier_init();
+    sh.timeout = 0;
+    sh.tie_cut = INT_MAX;
+  }
+  __syncthreads();
+  const uint32_t bytes = static_cast<uint32_t>((static_cast<size_t>(n) * sizeof(Raw) + 15) & ~size_t(15));
+  if (tid == 0 && bytes > 0) {
+    mbar_arrive_expect_tx(&sh.bar, bytes);
+    bulk_load_all(buf, grow + c0, bytes, &sh.bar);
+  }
+  if (bytes > 0 && !mbar_wait(&sh.bar, 0)) {
+    atomicOr(&sh.timeout, 1u);
+    mbar_wait(&sh.bar, 0);  // give the copy a second bounded chance to land
+  }
+  __syncthreads();
+
+  // ---- pass 1: online max / sum / entropy sum over the slice
+  const float T = P.temperature ? P.temperature[row] : P.temperature_scalar;
+  const float c = kLog2e / T;
+  Stats s = stats_empty();
+  {
+    const int nfull = n / VEC;
+    const uint4* v4 = reinterpret_cast<const uint4*>(buf);
+    for (int v = tid; v < nfull; v += blockDim.x) {
+      Raw r[VEC];
+      unpack(v4[v], r);
+      float u[VEC];
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) u[i] = __fmul_rn(value_of(r[i]), c);
+      stats_add(s, u);
+    }
+    for (int j = nfull * VEC + tid; j < n; j += blockDim.x) {
+      float u[1] = {__fmul_rn(value_of(buf[j]), c)};
+      stats_add(s, u);
+    }
+  }
+  s = block_reduce(s, sh.red);
+  if (tid == 0) sh.part = s;
+  cluster.sync();
+  if (tid < static_cast<int>(CL)) sh.gathered[tid] = *cluster.map_shared_rank(&sh.part, tid);
+  __syncthreads();
+  Stats rs = stats_empty();
+  for (uint32_t r = 0; r < CL; ++r) stats_merge(rs, sh.gathered[r]);
+
+  const bool nonfinite = !(isfinite(rs.m) && isfinite(rs.z) && isfinite(rs.a));
+  const float m2 = rs.m;
+  const float log2z = log2f(rs.z);
+  const float h_full = kLn2 * (log2z - rs.a / rs.z);
+
+  const int kk = P.top_k ? P.top_k[row] : P.top_k_scalar;
+  const float pp = P.top_p ? P.top_p[row] : P.top_p_scalar;
+  const float mp = P.min_p ? P.min_p[row] : P.min_p_scalar;
+  const bool use_k = kk > 0 && kk < V;
+  const bool use_p = pp < 1.f;
+  const bool use_minp = mp > 0.f;
+  const bool filtered = !nonfinite && (use_k || use_p || use_minp);
+
+  uint32_t tkey = 0;
+  int32_t tie_cut = INT_MAX;
+  float log2zs = log2z;
+  float h_support = h_full;
+  int32_t n_support = nonfinite ? 0 : V;
+
+  if (filtered) {
+    int hb = 0;
+    bool all_ties = true;
+    unsigned long long cnum = 0;  // ties kept at tkey when !all_ties
+    bool have_t = false;
+    if (use_k) {
+      Desc d = descend(buf, n, c, m2, P.fx_shift, false, use_p,
+                       static_cast<unsigned long long>(kk), 1.f, sh, cluster, hb);
+      const unsigned long long ck = static_cast<unsigned long long>(kk) - d.above_cnt;
+      tkey = d.key;
+      cnum = ck;
+      all_ties = ck >= d.at_cnt;
+      have_t = true;
+      if (use_p) {
+        const unsigned long long fx_t = d.at_cnt ? d.at_mass / d.at_cnt : 0;
+        const unsigned long long mass1 = d.above_mass + ck * fx_t;
+        double want = ceil(static_cast<double>(pp) * static_cast<double>(mass1));
+        unsigned long long tp = want <= 1.0 ? 1ull
+                                : want >= static_cast<double>(mass1)
+                                    ? mass1
+                                    : static_cast<unsigned long long>(want);
+        if (tp < 1) tp = 1;
+        Desc e = descend(buf, n, c, m2, P.fx_shift, true, true, tp, pp, sh, cluster, hb);
+        const unsigned long long fxe = e.at_cnt ? e.at_mass / e.at_cnt : 0;
+        const unsigned long long need = tp > e.above_mass ? tp - e.above_mass : 0;
+        unsigned long long cp = fxe ? (need + fxe - 1) / fxe : e.at_cnt;
+        if (cp < 1) cp = 1;
+        if (cp > e.at_cnt) cp = e.at_cnt;
+        if (e.key == tkey && cp > ck) cp = ck;
+        tkey = e.key;
+        cnum = cp;
+        all_ties = cp >= e.at_cnt;
+      }
+    } else if (use_p) {
+      Desc e = descend(buf, n, c, m2, P.fx_shift, true, true, 0ull, pp, sh, cluster, hb);
+      const unsigned long long tp = sh.b_target;
+      const unsigned long long fxe = e.at_cnt ? e.at_mass / e.at_cnt : 0;
+      const unsigned long long need = tp > e.above_mass ? tp - e.above_mass : 0;
+      unsigned long long cp = fxe ? (need + fxe - 1) / fxe : e.at_cnt;
+      if (cp < 1) cp = 1;
+      if (cp > e.at_cnt) cp = e.at_cnt;
+      tkey = e.key;
+      cnum = cp;
+      all_ties = cp >= e.at_cnt;
+      have_t = true;
+    }
+    if (use_minp) {
+      // smallest key whose probability ratio to the row max reaches min_p
+      uint32_t lo = 0, hi = KT::kInfKey;
+      while (lo < hi) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        const float r = ex2(__fmul_rn(KT::decode(mid), c) - m2);
+        if (r >= mp)
+          hi = mid;
+        else
+          lo = mid + 1;
+      }
+      if (!have_t || lo > tkey) {
+        tkey = lo;
+        all_ties = true;
+        have_t = true;
+      }
+    }
+
+    // ---- support sums: keys above tkey, and the tie group at tkey
+    uint32_t ngt = 0, neq = 0;
+    float smass = 0.f, sa = 0.f;
+    {
+      const uint32_t t = tkey;
+      for_each(buf, n, [&](int, Raw raw) {
+        const uint32_t key = key_of(raw);
+        if (key > t) {
+          const float d = __fmul_rn(value_of(raw), c) - m2;
+          const float e = ex2(d);
+          ++ngt;
+          smass += e;
+          sa = fmaf(d, e, sa);
+        } else if (key == t) {
+          ++neq;
+        }
+      });
+    }
+    ngt = block_sum(ngt, sh.ured);
+    neq = block_sum(neq, sh.ured);
+    smass = block_sum(smass, sh.fred);
+    sa = block_sum(sa, sh.fred);
+    if (tid == 0) {
+      sh.agg_ngt = ngt;
+      sh.agg_eq = neq;
+      sh.agg_mass = smass;
+      sh.agg_a = sa;
+    }
+    cluster.sync();
+    uint32_t tot_gt = 0, tot_eq = 0;
+    float tot_mass = 0.f, tot_a = 0.f;
+    uint32_t eq_rank[8];
+    for (uint32_t r = 0; r < CL; ++r) {
+      const SelShared* rsh = cluster.map_shared_rank(&sh, r);
+      tot_gt += rsh->agg_ngt;
+      eq_rank[r] = rsh->agg_eq;
+      tot_eq += eq_rank[r];
+      tot_mass += rsh->agg_mass;
+      tot_a += rsh->agg_a;
+    }
+    const unsigned long long ckeep = all_ties ? tot_eq : (cnum < tot_eq ? cnum : tot_eq);
+    const float dt = __fmul_rn(KT::decode(tkey), c) - m2;
+    const float et = ex2(dt);
+    const float mass_s = tot_mass + static_cast<float>(ckeep) * et;
+    const float a_s = tot_a + static_cast<float>(ckeep) * dt * et;
+    log2zs = log2f(mass_s);
+    h_support = kLn2 * (log2zs - a_s / mass_s);
+    n_support = static_cast<int32_t>(tot_gt + ckeep);
+
+    // ---- tie resolution: id of the last tie kept (ascending id order)
+    if (ckeep < tot_eq) {
+      unsigned long long off = 0;
+      uint32_t owner = 0;
+      for (uint32_t r = 0; r < CL; ++r) {
+        if (off + eq_rank[r] >= ckeep) {
+          owner = r;
+          break;
+        }
+        off += eq_rank[r];
+      }
+      if (rank == owner) {
+        const int need = static_cast<int>(ckeep - off);
+        int base_count = 0;
+        const uint32_t t = tkey;
+        const int lane = tid & 31, warp = tid >> 5;
+        for (int base = 0; base < n; base += kThreads * VEC) {
+          const int j0 = base + tid * VEC;
+          int mine = 0;
+#pragma unroll
+          for (int i = 0; i < VEC; ++i) {
+            const int j = j0 + i;
+            if (j < n && key_of(buf[j]) == t) ++mine;
+          }
+          int incl = mine;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int x = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += x;
+          }
+          if (lane == 31) sh.scan_tot[warp] = incl;
+          __syncthreads();
+          int wpre = 0, total = 0;
+          for (int w = 0; w < kWarps; ++w) {
+            if (w < warp) wpre += sh.scan_tot[w];
+            total += sh.scan_tot[w];
+          }
+          const int excl = base_count + wpre + incl - mine;
+          if (excl < need && need <= excl + mine) {
+            int cn = excl;
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) {
+              const int j = j0 + i;
+              if (j < n && key_of(buf[j]) == t) {
+                ++cn;
+                if (cn == need) sh.tie_cut = c0 + j;
+              }
+            }
+          }
+          base_count += total;
+          __syncthreads();
+          if (base_count >= need) break;
+        }
+      }
+      cluster.sync();
+      tie_cut = *cluster.map_shared_rank(&sh.tie_cut, owner);
+    } else {
+      tie_cut = INT_MAX;
+    }
+  }
+
+  // ---- per-row outputs (rank 0, thread 0)
+  if (rank == 0 && tid == 0) {
+    const int y = P.targets[row];
+    const bool target_ok = y >= 0 && y < V;
+    uint32_t status = 0;
+    float lp_v = __int_as_float(0x7fc00000), lp_s = __int_as_float(0x7fc00000);
+    bool in_s = false;
+    if (!target_ok) status |= VS_ROW_TARGET_OUT_OF_RANGE;
+    if (nonfinite) {
+      status |= VS_ROW_NONFINITE_INPUT;
+    } else if (target_ok) {
+      const Raw ry = grow[y];
+      const float uy = __fmul_rn(value_of(ry), c);
+      lp_v = kLn2 * (uy - m2 - log2z);
+      if (!filtered) {
+        in_s = true;
+      } else {
+        const uint32_t ky = key_of(ry);
+        in_s = ky > tkey || (ky == tkey && y <= tie_cut);
+      }
+      if (in_s) {
+        lp_s = filtered ? kLn2 * (uy - m2 - log2zs) : lp_v;
+      } else {
+        lp_s = -kInf;
+        status |= VS_ROW_TARGET_NOT_IN_SUPPORT;
+      }
+    }
+    if (sh.timeout) status |= kRowDeviceTimeout;
+    const float nan = __int_as_float(0x7fc00000);
+    if (P.lp_full) P.lp_full[row] = lp_v;
+    if (P.lp_support) P.lp_support[row] = lp_s;
+    if (P.want_entropy) {
+      if (P.h_full) P.h_full[row] = nonfinite ? nan : h_full;
+      if (P.h_support) P.h_support[row] = nonfinite ? nan : h_support;
+    }
+    if (P.valid) P.valid[row] = nonfinite ? 0 : 1;
+    if (P.status) P.status[row] = status;
+    if (P.support_size) P.support_size[row] = n_support;
+    if (P.ctx) {
+      RowCtx cx{};
+      cx.m2 = m2;
+      cx.log2z = log2z;
+      cx.msup = m2;
+      cx.log2zs = log2zs;
+      cx.h_full = h_full;
+      cx.h_support = h_support;
+      cx.c = c;
+      cx.tkey = tkey;
+      cx.tie_cut = tie_cut;
+      uint32_t f = kCtxFullStats;
+      if (nonfinite) f |= kCtxNonFinite | kCtxEmpty;
+      else if (!filtered) f |= kCtxAllVocab;
+      else f |= kCtxThreshold;
+      if (target_ok) f |= kCtxTargetOk;
+      if (in_s) f |= kCtxTargetInS;
+      cx.flags = f;
+      cx.n_support = n_support;
+      cx.status = status;
+      P.ctx[row] = cx;
+    }
+  }
+
+  // ---- support bitmask for this CTA's slice (words never straddle CTAs)
+  if (P.support_mask) {
+    const int words = (n + 31) / 32;
+    const int64_t wstride = (V + 31) / 32;
+    uint32_t* mrow = P.support_mask + static_cast<int64_t>(row) * wstride + c0 / 32;
+    const int lane = tid & 31, warp = tid >> 5;
+    for (int w = warp; w < words; w += kWarps) {
+      const int j = w * 32 + lane;
+      bool in = false;
+      if (j < n && !nonfinite) {
+        if (!filtered) {
+          in = true;
+        } else {
+          const uint32_t key = key_of(buf[j]);
+          in = key > tkey || (key == tkey && (c0 + j) <= tie_cut);
+        }
+      }
+      const uint32_t bits = __ballot_sync(0xffffffffu, in);
+      if (lane == 0) mrow[w] = bits;
+    }
+  }
+  cluster.sync();  // no CTA leaves while a peer may still read its shared memory
+}
+
+// ---------------------------------------------------------------------------
+// recorded support
+
+constexpr int kRecThreads = 256;
+
+template <typename Raw>
+__global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams P) {
+  constexpr int VEC = 16 / sizeof(Raw);
+  const int row = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int V = P.vocab;
+  const int W = P.support_width;
+  __shared__ int32_t ids[VS_MAX_SUPPORT_WIDTH];
+  __shared__ Stats red[kRecThreads / 32];
+  __shared__ uint32_t ured[kRecThreads / 32];
+  __shared__ uint32_t flags_sh;
+  __shared__ int32_t target_hit;
+
+  const Raw* grow = static_cast<const Raw*>(P.logits) + static_cast<int64_t>(row) * P.ld;
+  const int32_t* srow = P.support_ids + static_cast<int64_t>(row) * P.support_ld;
+  const float T = P.temperature ? P.temperature[row] : P.temperature_scalar;
+  const float c = kLog2e / T;
+  const int y = P.targets[row];
+  const bool target_ok = y >= 0 && y < V;
+
+  if (tid == 0) {
+    flags_sh = 0;
+    target_hit = 0;
+  }
+  for (int w = tid; w < W; w += blockDim.x) ids[w] = srow[w];
+  __syncthreads();
+
+  // keep[w]: id valid and first occurrence
+  uint32_t local_flags = 0;
+  Stats s = stats_empty();
+  uint32_t nkeep = 0;
+  bool nonfinite_sup = false;
+  for (int w = tid; w < W; w += blockDim.x) {
+    const int32_t id = ids[w];
+    if (id == -1) continue;
+    if (id < -1 || id >= V) {
+      local_flags |= VS_ROW_BAD_SUPPORT_ID;
+      continue;
+    }
+    bool dup = false;
+    for (int w2 = 0; w2 < w; ++w2)
+      if (ids[w2] == id) {
+        dup = true;
+        break;
+      }
+    if (dup) {
+      local_flags |= VS_ROW_DUP_SUPPORT_ID;
+      continue;
+    }
+    ++nkeep;
+    const float u = __fmul_rn(value_of(grow[id]), c);
+    if (!isfinite(u)) nonfinite_sup = true;
+    float uu[1] = {u};
+    stats_add(s, uu);
+    if (id == y) target_hit = 1;
+  }
+  if (local_flags) atomicOr(&flags_sh, local_flags);
+  s = block_reduce(s, red);
+  nkeep = block_sum(nkeep, ured);
+  const uint32_t any_nf = block_sum(static_cast<uint32_t>(nonfinite_sup), ured);
+  const bool empty = nkeep == 0;
+
+  // full-vocabulary statistics: for empty rows (fallback) or on request
+  const bool need_full = empty || P.full_stats;
+  Stats f = stats_empty();
+  if (need_full) {
+    const int nfull = V / VEC;
+    const uint4* g4 = reinterpret_cast<const uint4*>(grow);
+    int v = tid;
+    for (; v + 3 * kRecThreads < nfull; v += 4 * kRecThreads) {
+      uint4 q[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) q[k] = __ldcs(g4 + v + k * kRecThreads);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        Raw r[VEC];
+        unpack(q[k], r);
+        float u[VEC];
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) u[i] = __fmul_rn(value_of(r[i]), c);
+        stats_add(f, u);
+      }
+    }
+    for (; v < nfull; v += kRecThreads) {
+      Raw r[VEC];
+      unpack(__ldcs(g4 + v), r);
+      float u[VEC];
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) u[i] = __fmul_rn(value_of(r[i]), c);
+      stats_add(f, u);
+    }
+    for (int j = nfull * VEC + tid; j < V; j += kRecThreads) {
+      float u[1] = {__fmul_rn(value_of(grow[j]), c)};
+      stats_add(f, u);
+    }
+    f = block_reduce(f, red);
+  }
+
+  if (tid == 0) {
+    const float nan = __int_as_float(0x7fc00000);
+    uint32_t status = flags_sh;
+    bool nonfinite = any_nf != 0;
+    float m2 = nan, log2z = nan, h_full = nan;
+    if (need_full) {
+      if (!(isfinite(f.m) && isfinite(f.z) && isfinite(f.a))) nonfinite = true;
+      m2 = f.m;
+      log2z = log2f(f.z);
+      h_full = kLn2 * (log2z - f.a / f.z);
+    }
+    const float msup = s.m;
+    const float log2zs = empty ? nan : log2f(s.z);
+    const float h_sup = empty ? 0.f : kLn2 * (log2zs - s.a / s.z);
+    float lp_v = nan, lp_s = nan;
+    bool in_s = false;
+    if (!target_ok) status |= VS_ROW_TARGET_OUT_OF_RANGE;
+    if (nonfinite) {
+      status |= VS_ROW_NONFINITE_INPUT;
+    } else if (target_ok) {
+      const float uy = __fmul_rn(value_of(grow[y]), c);
+      if (need_full) lp_v = kLn2 * (uy - m2 - log2z);
+      in_s = target_hit != 0;
+      if (empty) {
+        lp_s = lp_v;
+      } else if (in_s) {
+        lp_s = kLn2 * (uy - msup - log2zs);
+      } else {
+        lp_s = -kInf;
+        status |= VS_ROW_TARGET_NOT_IN_SUPPORT;
+      }
+    }
+    const bool valid = !nonfinite && !empty;
+    if (P.lp_full) P.lp_full[row] = lp_v;
+    if (P.lp_support) P.lp_support[row] = lp_s;
+    if (P.want_entropy) {
+      if (P.h_full) P.h_full[row] = nonfinite ? nan : h_full;
+      if (P.h_support) P.h_support[row] = nonfinite ? nan : h_sup;
+    }
+    if (P.valid) P.valid[row] = valid ? 1 : 0;
+    if (P.status) P.status[row] = status;
+    if (P.support_size) P.support_size[row] = nonfinite ? 0 : static_cast<int32_t>(nkeep);
+    if (P.ctx) {
+      RowCtx cx{};
+      cx.m2 = m2;
+      cx.log2z = log2z;
+      cx.msup = msup;
+      cx.log2zs = log2zs;
+      cx.h_full = h_full;
+      cx.h_support = h_sup;
+      cx.c = c;
+      cx.tkey = 0;
+      cx.tie_cut = 0;
+      uint32_t fl = kCtxRecorded;
+      if (need_full) fl |= kCtxFullStats;
+      if (nonfinite) fl |= kCtxNonFinite;
+      if (empty || nonfinite) fl |= kCtxEmpty;
+      if (target_ok) fl |= kCtxTargetOk;
+      if (in_s) fl |= kCtxTargetInS;
+      cx.flags = fl;
+      cx.n_support = nonfinite ? 0 : static_cast<int32_t>(nkeep);
+      cx.status = status;
+      P.ctx[row] = cx;
+    }
+  }
+  // support bitmask: clear the row, then set the kept ids
+  if (P.support_mask) {
+    const int64_t wstride = (V + 31) / 32;
+    uint32_t* mrow = P.support_mask + static_cast<int64_t>(row) * wstride;
+    for (int64_t w = tid; w < wstride; w += blockDim.x) mrow[w] = 0u;
+    __syncthreads();
+    if (any_nf == 0) {
+      for (int w = tid; w < W; w += blockDim.x) {
+        const int32_t id = ids[w];
+        if (id < 0 || id >= V) continue;
+        atomicOr(&mrow[id >> 5], 1u << (id & 31));
+      }
+    }
+  }
+}
+
+// Deterministic reduction of the entropy sum and valid count over rows.
+__global__ void score_reduce_kernel(const float* h_support, const uint8_t* valid, int rows,
+                                    double* entropy_sum, int32_t* valid_count) {
+  __shared__ double dred[32];
+  __shared__ int ired[32];
+  double s = 0.0;
+  int cnt = 0;
+  for (int i = threadIdx.x; i < rows; i += blockDim.x) {
+    if (valid[i]) {
+      ++cnt;
+      if (h_support) s += static_cast<double>(h_support[i]);
+    }
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s += __shfl_xor_sync(0xffffffffu, s, o);
+    cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  }
+  if (lane == 0) {
+    dred[warp] = s;
+    ired[warp] = cnt;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    int tc = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) {
+      t += dred[w];
+      tc += ired[w];
+    }
+    if (entropy_sum) *entropy_sum = t;
+    if (valid_count) *valid_count = tc;
+  }
+}
+
+constexpr int kMaxChunkBytes = 96 * 1024;
+
+}  // namespace
+
+int score_max_vocab(vs_dtype dtype) {
+  const int esize = dtype == VS_BF16 ? 2 : 4;
+  return 8 * (kMaxChunkBytes / esize);
+}
+
+// Cluster size and per-CTA slice (elements, multiple of 32) for a row of
+// `vocab` elements: the smallest cluster whose slices fit a 40 KB budget, so
+// several CTAs share an SM; larger rows grow the slice up to 96 KB.
+int score_cluster_size(int vocab, vs_dtype dtype, int* chunk) {
+  const int esize = dtype == VS_BF16 ? 2 : 4;
+  const int target = 40 * 1024 / esize;
+  int cl = 1;
+  while (cl < 8 && (vocab + cl - 1) / cl > target) ++cl;
+  int e = (vocab + cl - 1) / cl;
+  e = (e + 31) & ~31;
+  *chunk = e;
+  return cl;
+}
+
+cudaError_t launch_score_computed(const ScoreParams& p, vs_dtype dtype, int cluster,
+                                  cudaStream_t s) {
+  const size_t esize = dtype == VS_BF16 ? 2 : 4;
+  const size_t smem = static_cast<size_t>(p.chunk) * esize + sizeof(SelShared);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(p.rows) * cluster, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
+  if (dtype == VS_BF16) {
+    e = cudaFuncSetAttribute(score_computed_kernel<uint16_t>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    return cudaLaunchKernelEx(&cfg, score_computed_kernel<uint16_t>, p);
+  }
+  e = cudaFuncSetAttribute(score_computed_kernel<uint32_t>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernelEx(&cfg, score_computed_kernel<uint32_t>, p);
+}
+
+cudaError_t launch_score_recorded(const ScoreParams& p, vs_dtype dtype, cudaStream_t s) {
+  if (dtype == VS_BF16)
+    score_recorded_kernel<uint16_t><<<p.rows, kRecThreads, 0, s>>>(p);
+  else
+    score_recorded_kernel<uint32_t><<<p.rows, kRecThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_score_reduce(const float* h_support, const uint8_t* valid, int rows,
+                                double* entropy_sum, int32_t* valid_count, cudaStream_t s) {
+  score_reduce_kernel<<<1, 1024, 0, s>>>(h_support, valid, rows, entropy_sum, valid_count);
+  return cudaGetLastError();
+}
+
+}  // namespace vs

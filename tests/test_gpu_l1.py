@@ -1,0 +1,101 @@
+"""GPU parity of vs_l1_distance against the fp64 oracle (DSpark distance,
+accept rate, weighted loss and draft gradient), through the C ABI."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sampling_support_b200 as vsb
+import workloads
+from _util import assert_close_rel, compare_grad, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def _check(draft, target, weight, grad_dtype=torch.float32, sample=None):
+    rows, vocab = draft.shape
+    d, t = to_device(draft), to_device(target)
+    w = None if weight is None else torch.from_numpy(weight).cuda()
+    out = vsb.l1_distance(d, t, w, want_loss=True, want_grad=True, grad_dtype=grad_dtype)
+    torch.cuda.synchronize()
+    w64 = None if weight is None else weight.astype(np.float64)
+    ref = oracle.l1(draft, target, weight=w64)
+    assert_close_rel(out["l1"].cpu().numpy(), ref["l1"], 1e-4, "l1")
+    acc = out["accept"].cpu().numpy().astype(np.float64)
+    assert np.abs(acc - ref["accept"]).max() <= 1e-4
+    loss = out["loss"].cpu().numpy().astype(np.float64)
+    assert_close_rel(loss[:1], [ref["loss_num"]], 1e-4, "loss numerator")
+    assert_close_rel(loss[1:2], [ref["loss_den"]], 1e-6, "loss denominator")
+    assert_close_rel(loss[2:], [ref["loss"]], 1e-4, "loss")
+    sel = np.arange(rows) if sample is None else sample
+    # gradient rows: oracle on the selected rows, rescaled to the full weight sum
+    ws = np.ones(rows) if weight is None else weight.astype(np.float64)
+    gref = oracle.l1(draft[sel], target[sel], weight=ws[sel], want_grad=True)
+    gref_g = gref["grad"] * (ws[sel].sum() / ws.sum())
+    near = np.abs(_probs(draft[sel]) - _probs(target[sel])) < 1e-6
+    g = out["grad"][torch.from_numpy(sel).cuda()].float().cpu().numpy()
+    compare_grad(g, gref_g, exclude=near,
+                 rtol=2e-3 if grad_dtype == torch.float32 else 6e-3)
+    return out
+
+
+def _probs(bits):
+    x = bits.astype(np.float64) if bits.dtype != np.uint16 else workloads.bf16_bits_to_f32(bits).astype(np.float64)
+    x = np.exp(x - x.max(1, keepdims=True))
+    return x / x.sum(1, keepdims=True)
+
+
+@pytest.mark.parametrize("vocab", [20_011, 1000, 33, 1])
+def test_l1_ragged_bf16(vocab):
+    w = workloads.distance(rows=16, vocab=vocab, seed=5)
+    _check(w["draft"], w["target"], w["weight"])
+
+
+def test_l1_row_stride_beyond_vocab():
+    vocab, ld = 10_001, 10_008
+    w = workloads.distance(rows=4, vocab=vocab, seed=6)
+    pad = lambda a: np.pad(a, ((0, 0), (0, ld - vocab)), constant_values=0x7FC0)  # NaN pads
+    d, t = to_device(pad(w["draft"])), to_device(pad(w["target"]))
+    out = vsb.l1_distance(d, t, torch.from_numpy(w["weight"]).cuda(), want_grad=True, vocab=vocab)
+    torch.cuda.synchronize()
+    ref = oracle.l1(w["draft"], w["target"], weight=w["weight"].astype(np.float64), want_grad=True)
+    assert_close_rel(out["l1"].cpu().numpy(), ref["l1"], 1e-4, "l1")
+    compare_grad(out["grad"].cpu().numpy()[:, :vocab], ref["grad"])
+
+
+def test_l1_f32_and_bf16_grad():
+    rng = np.random.default_rng(3)
+    d = (rng.normal(size=(8, 4096)) * 2).astype(np.float32)
+    t = (d + rng.normal(size=d.shape) * 0.7).astype(np.float32)
+    wt = rng.uniform(size=8).astype(np.float32)
+    _check(d, t, wt)
+    _check(workloads.to_bf16_bits(d), workloads.to_bf16_bits(t), wt, grad_dtype=torch.bfloat16)
+
+
+def test_l1_identical_rows_exact():
+    w = workloads.distance(rows=6, vocab=30_000, seed=9)
+    d = to_device(w["draft"])
+    out = vsb.l1_distance(d, d.clone(), torch.from_numpy(w["weight"]).cuda(), want_grad=True)
+    torch.cuda.synchronize()
+    assert torch.all(out["l1"] == 0) and torch.all(out["accept"] == 1)
+    assert torch.all(out["grad"] == 0)
+    assert out["loss"][0].item() == 0.0 and out["loss"][2].item() == 0.0
+
+
+def test_l1_unweighted_and_zero_weights():
+    w = workloads.distance(rows=5, vocab=8000, seed=1)
+    _check(w["draft"], w["target"], None)
+    d, t = to_device(w["draft"]), to_device(w["target"])
+    out = vsb.l1_distance(d, t, torch.zeros(5, device="cuda"), want_grad=True)
+    torch.cuda.synchronize()
+    assert out["loss"][2].item() == 0.0 and torch.all(out["grad"] == 0)
+
+
+@pytest.mark.slow
+def test_distance_workload_full_size():
+    w = workloads.distance()
+    rng = np.random.default_rng(0)
+    sel = np.sort(rng.choice(w["rows"], 48, replace=False))
+    out = _check(w["draft"], w["target"], w["weight"], grad_dtype=torch.bfloat16, sample=sel)
+    assert out["grad"].dtype == torch.bfloat16
