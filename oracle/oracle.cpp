@@ -76,6 +76,23 @@ double load_value(const void* base, int dtype, int64_t index) {
   return static_cast<double>(f);
 }
 
+// log sum_j exp(z_j - m) over the selected entries, with m their maximum,
+// evaluated as log(#{z_j == m}) + log1p(sum_{z_j < m} exp(z_j - m) / #{z_j == m}):
+// the same sum, split so that a row dominated by one token (sum = 1 + tiny)
+// keeps its relative precision.
+double log_sum_exp_shifted(const std::vector<double>& z, const std::vector<uint8_t>* sel,
+                           double m) {
+  double top = 0.0, rest = 0.0;
+  for (size_t j = 0; j < z.size(); ++j) {
+    if (sel && !(*sel)[j]) continue;
+    if (z[j] == m)
+      top += 1.0;
+    else
+      rest += std::exp(z[j] - m);
+  }
+  return std::log(top) + std::log1p(rest / top);
+}
+
 // Everything the oracle knows about one scored row.
 struct RowResult {
   double lse_full = kNaN;      // log sum_j exp(z_j)
@@ -84,6 +101,8 @@ struct RowResult {
   double h_full = kNaN;        // -sum_j p_j log p_j
   double h_support = 0.0;      // -sum_{j in S} q_j log q_j
   double lse_support = kNaN;
+  double m_full = kNaN, lz_full = kNaN;        // lse_full = m_full + lz_full
+  double m_support = kNaN, lz_support = kNaN;  // lse_support = m_support + lz_support
   uint8_t valid = 0;
   uint32_t status = 0;
   int32_t support_size = 0;
@@ -117,18 +136,19 @@ RowResult score_row(const void* logits, int dtype, int64_t row_offset, int vocab
     return r;
   }
 
-  // Full-vocabulary log-sum-exp, logprob and entropy.
+  // Full-vocabulary log-sum-exp, logprob and entropy; log p_j = (z_j - m) - log sum exp(z - m).
   const double m = *std::max_element(r.z.begin(), r.z.end());
-  double zsum = 0.0;
-  for (int j = 0; j < vocab; ++j) zsum += std::exp(r.z[j] - m);
-  r.lse_full = m + std::log(zsum);
+  const double lz = log_sum_exp_shifted(r.z, nullptr, m);
+  r.m_full = m;
+  r.lz_full = lz;
+  r.lse_full = m + lz;
   double h = 0.0;
   for (int j = 0; j < vocab; ++j) {
-    double logp = r.z[j] - r.lse_full;
+    double logp = (r.z[j] - m) - lz;
     h -= std::exp(logp) * logp;
   }
   r.h_full = h;
-  r.lp_full = target_ok ? r.z[target] - r.lse_full : kNaN;
+  r.lp_full = target_ok ? (r.z[target] - m) - lz : kNaN;
 
   // Support S.
   r.in_support.assign(vocab, 0);
@@ -218,21 +238,21 @@ RowResult score_row(const void* logits, int dtype, int64_t row_offset, int vocab
   double ms = -kInf;
   for (int j = 0; j < vocab; ++j)
     if (r.in_support[j]) ms = std::max(ms, r.z[j]);
-  double ssum = 0.0;
-  for (int j = 0; j < vocab; ++j)
-    if (r.in_support[j]) ssum += std::exp(r.z[j] - ms);
-  r.lse_support = ms + std::log(ssum);
+  const double lzs = log_sum_exp_shifted(r.z, &r.in_support, ms);
+  r.m_support = ms;
+  r.lz_support = lzs;
+  r.lse_support = ms + lzs;
   double hs = 0.0;
   for (int j = 0; j < vocab; ++j) {
     if (!r.in_support[j]) continue;
-    double logq = r.z[j] - r.lse_support;
+    double logq = (r.z[j] - ms) - lzs;
     hs -= std::exp(logq) * logq;
   }
   r.h_support = hs;
   if (!target_ok) {
     r.lp_support = kNaN;
   } else if (r.in_support[target]) {
-    r.lp_support = r.z[target] - r.lse_support;
+    r.lp_support = (r.z[target] - ms) - lzs;
   } else {
     r.status |= ORC_TARGET_NOT_IN_SUPPORT;
     r.lp_support = -kInf;
@@ -331,11 +351,11 @@ int vso_score_grad(int rows, int vocab, int64_t ld, int dtype, const void* logit
         g_supp_lp = gls;
     }
     for (int j = 0; j < vocab; ++j) {
-      const double logp = r.z[j] - r.lse_full;
+      const double logp = (r.z[j] - r.m_full) - r.lz_full;
       const double p = std::exp(logp);
       double dz = g_full_lp * ((j == y ? 1.0 : 0.0) - p) + ghv * (-p * (logp + r.h_full));
       if (r.support_size > 0 && r.in_support[j]) {
-        const double logq = r.z[j] - r.lse_support;
+        const double logq = (r.z[j] - r.m_support) - r.lz_support;
         const double q = std::exp(logq);
         dz += g_supp_lp * ((j == y ? 1.0 : 0.0) - q) + ghs * (-q * (logq + r.h_support));
       }

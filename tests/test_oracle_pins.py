@@ -398,3 +398,16 @@ def test_l1_finite_difference_gradient():
             dm[i, j] -= h
             fd[i, j] = (oracle.l1(dp, t, weight=w)["loss"] - oracle.l1(dm, t, weight=w)["loss"]) / (2 * h)
     assert np.abs(r["grad"] - fd).max() < 1e-7
+
+
+def test_dominant_token_entropy_closed_form():
+    # one logit L above V-1 equal logits at 0: with d = (V-1) e^-L,
+    # H = log1p(d) + L d / (1 + d),  lp(max) = -log1p(d)
+    V, L = 4096, 40.0
+    l = np.zeros((1, V))
+    l[0, 7] = L
+    r = oracle.score(l, [7])
+    d = (V - 1) * math.exp(-L)
+    h = math.log1p(d) + L * d / (1.0 + d)
+    assert abs(r["h_full"][0] - h) <= 1e-12 * h
+    assert abs(r["lp_full"][0] + math.log1p(d)) <= 1e-12 * math.log1p(d)
