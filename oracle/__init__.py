@@ -150,18 +150,19 @@ def score_grad(logits, targets, g_lp_full=None, g_lp_support=None, g_h_full=None
     return d
 
 
-def l1(draft, target, weight=None, want_grad=False, tie_eps=1e-6):
+def l1(draft, target, weight=None, want_grad=False, tie_eps=1e-6, vocab=None):
     draft = np.ascontiguousarray(draft)
     target = np.ascontiguousarray(target)
     assert draft.dtype == target.dtype and draft.shape == target.shape
-    rows, vocab = draft.shape
+    rows, ld = draft.shape
+    vocab = ld if vocab is None else vocab
     w = None if weight is None else np.ascontiguousarray(weight, np.float64)
     out = {k: np.empty(rows, np.float64) for k in ("l1", "accept")}
     nd = np.empty(3, np.float64)
     ties = np.empty(rows, np.int32)
     g = np.empty((rows, vocab), np.float64) if want_grad else None
     L = lib()
-    rc = L.vso_l1(ctypes.c_int(rows), ctypes.c_int(vocab), ctypes.c_int64(vocab),
+    rc = L.vso_l1(ctypes.c_int(rows), ctypes.c_int(vocab), ctypes.c_int64(ld),
                   ctypes.c_int(_dtype_code(draft)), _ptr(draft), _ptr(target), _ptr(w),
                   _ptr(out["l1"]), _ptr(out["accept"]), _ptr(nd), _ptr(g),
                   ctypes.c_double(tie_eps), _ptr(ties))

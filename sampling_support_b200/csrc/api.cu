@@ -112,6 +112,7 @@ vs_status vs_score_fwd(const vs_score_args* a, const vs_score_out* o, void* work
   vs_status st = check_args(a);
   if (st != VS_OK) return st;
   if (!o) return fail(VS_ERR_INVALID_ARG, "out is NULL");
+  if (a->rows == 0) return ok();
   const bool want_entropy = a->flags & VS_WANT_ENTROPY;
   if ((a->flags & VS_WANT_SUPPORT_MASK) && !o->support_mask)
     return fail(VS_ERR_INVALID_ARG, "VS_WANT_SUPPORT_MASK needs support_mask");

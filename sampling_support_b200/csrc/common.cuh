@@ -85,28 +85,58 @@ __device__ __forceinline__ void unpack(const uint4& q, uint32_t (&r)[4]) {
 }
 
 // ---------------------------------------------------------------------------
-// online (max, sum 2^(u - max), sum (u - max) 2^(u - max)) in base-2 units.
-// A row's natural-log statistics follow as
-//   LSE = ln2 (m + log2 Z),   H = ln2 (log2 Z - A / Z)   (A <= 0).
+// online log-sum-exp and entropy statistics in base-2 units (u = z log2 e):
+//   m  = max u
+//   c0 = number of elements with u == m      (each contributes 2^0 = 1)
+//   zr = sum over the other elements of 2^(u - m)
+//   a  = sum over all elements of (u - m) 2^(u - m)      (<= 0)
+// Keeping the max elements' count apart from the rest lets
+//   log2 Z = log2 c0 + log1p(zr / c0) / ln 2,   Z = c0 + zr
+// keep full relative precision when one token dominates (Z close to 1),
+// and then  LSE = ln2 (m + log2 Z),  H = ln2 (log2 Z - a / Z).
 
 struct Stats {
-  float m, z, a;
+  float m, c0, zr, a;
 };
 
-__device__ __forceinline__ Stats stats_empty() { return {-kInf, 0.f, 0.f}; }
+__device__ __forceinline__ Stats stats_empty() { return {-kInf, 0.f, 0.f, 0.f}; }
 
-// Merge b into s.  An empty side (z == 0) is skipped; NaN/inf propagate.
-__device__ __forceinline__ void stats_merge(Stats& s, const Stats& b) {
-  if (b.z == 0.f) return;
-  if (s.z == 0.f) {
+__device__ __forceinline__ float stats_z(const Stats& s) { return s.c0 + s.zr; }
+
+__device__ __forceinline__ float stats_log2z(const Stats& s) {
+  return log2f(s.c0) + log1pf(s.zr / s.c0) * kLog2e;
+}
+
+// True when the statistics describe only finite values.
+__device__ __forceinline__ bool stats_finite(const Stats& s) {
+  return isfinite(s.m) && isfinite(s.zr) && isfinite(s.a) && s.c0 >= 1.f;
+}
+
+// Re-express `s` relative to a new maximum mn >= s.m (s non-empty).
+__device__ __forceinline__ void stats_rebase(Stats& s, float mn) {
+  if (s.m == mn) return;
+  const float f = ex2(s.m - mn);
+  const float z = s.c0 + s.zr;
+  s.a = f * fmaf(s.m - mn, z, s.a);
+  s.zr = f * z;
+  s.c0 = 0.f;
+  s.m = mn;
+}
+
+// Merge b into s.  An empty side (c0 == 0 and zr == 0) is skipped; NaN/inf
+// propagate through zr / a.
+__device__ __forceinline__ void stats_merge(Stats& s, Stats b) {
+  if (b.c0 == 0.f && b.zr == 0.f) return;
+  if (s.c0 == 0.f && s.zr == 0.f) {
     s = b;
     return;
   }
   const float mn = fmaxf(s.m, b.m);
-  const float f1 = ex2(s.m - mn), f2 = ex2(b.m - mn);
-  s.a = f1 * fmaf(s.m - mn, s.z, s.a) + f2 * fmaf(b.m - mn, b.z, b.a);
-  s.z = f1 * s.z + f2 * b.z;
-  s.m = mn;
+  stats_rebase(s, mn);
+  stats_rebase(b, mn);
+  s.c0 += b.c0;
+  s.zr += b.zr;
+  s.a += b.a;
 }
 
 // Add a batch of N values u[] (already scaled to base-2 units).
@@ -116,25 +146,23 @@ __device__ __forceinline__ void stats_add(Stats& s, const float (&u)[N]) {
 #pragma unroll
   for (int i = 1; i < N; ++i) bm = fmaxf(bm, u[i]);
   if (bm > s.m) {
-    if (s.z != 0.f) {
-      const float f = ex2(s.m - bm);
-      s.a = f * fmaf(s.m - bm, s.z, s.a);
-      s.z *= f;
-    }
+    if (s.c0 != 0.f || s.zr != 0.f) stats_rebase(s, bm);
     s.m = bm;
   }
 #pragma unroll
   for (int i = 0; i < N; ++i) {
     const float d = u[i] - s.m;
     const float e = ex2(d);
-    s.z += e;
+    const bool top = d == 0.f;
+    s.c0 += top ? 1.f : 0.f;
+    s.zr += top ? 0.f : e;
     s.a = fmaf(d, e, s.a);
   }
 }
 
 __device__ __forceinline__ Stats shfl_xor(const Stats& s, int lane_mask) {
-  return {__shfl_xor_sync(0xffffffffu, s.m, lane_mask), __shfl_xor_sync(0xffffffffu, s.z, lane_mask),
-          __shfl_xor_sync(0xffffffffu, s.a, lane_mask)};
+  return {__shfl_xor_sync(0xffffffffu, s.m, lane_mask), __shfl_xor_sync(0xffffffffu, s.c0, lane_mask),
+          __shfl_xor_sync(0xffffffffu, s.zr, lane_mask), __shfl_xor_sync(0xffffffffu, s.a, lane_mask)};
 }
 
 // Deterministic block reduction; result valid in every thread.  `scratch`

@@ -23,7 +23,9 @@ struct alignas(16) RowCtx {
   uint32_t flags;   // kCtx*
   int32_t n_support;
   uint32_t status;
-  uint32_t pad[4];
+  // split normalisers (see Stats): Z = c0 + zr, for 1 - p_y when y is a max
+  float c0_full, zr_full;
+  float c0_sup, zr_sup;
 };
 static_assert(sizeof(RowCtx) == VS_CTX_BYTES_PER_ROW, "ctx layout");
 

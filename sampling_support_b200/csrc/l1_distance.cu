@@ -127,8 +127,8 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
     stats_merge(Sd, sh.gathered[r][0]);
     stats_merge(St, sh.gathered[r][1]);
   }
-  const float md = Sd.m, ld2 = log2f(Sd.z);
-  const float mt = St.m, lt2 = log2f(St.z);
+  const float md = Sd.m, ld2 = stats_log2z(Sd);
+  const float mt = St.m, lt2 = stats_log2z(St);
 
   // pass 2: L1 = sum |p - q| and sum_k p_k sign(p_k - q_k)
   float l1 = 0.f, ps = 0.f;

@@ -43,6 +43,7 @@ struct GradStore<uint16_t> {
 struct RowCoef {
   float gv, gs, ghv, ghs;  // effective upstream gradients
   float m2, log2z, msup, log2zs, h_full, h_sup, c, scale;
+  float omp_full, omp_sup;  // 1 - p_y and 1 - q_y when y holds the maximum
   uint32_t tkey;
   int32_t tie_cut;
   uint32_t flags;
@@ -74,23 +75,34 @@ __device__ __forceinline__ RowCoef row_coef(const BwdParams& P, int row) {
   k.flags = cx.flags;
   k.y = P.targets[row];
   k.zero = (cx.flags & kCtxNonFinite) != 0;
+  k.omp_full = (cx.c0_full - 1.f + cx.zr_full) / (cx.c0_full + cx.zr_full);
+  k.omp_sup = (cx.c0_sup - 1.f + cx.zr_sup) / (cx.c0_sup + cx.zr_sup);
   k.need_full = !k.zero && (k.gv != 0.f || k.ghv != 0.f);
   k.need_sup = !k.zero && !empty && (k.gs != 0.f || k.ghs != 0.f);
   return k;
 }
 
+// [j == y] - p_j, with 1 - p_y taken from the split normaliser when y holds
+// the maximum (there 1 - p_y = (c0 - 1 + zr) / (c0 + zr) without cancellation).
+__device__ __forceinline__ float ind_minus(float p, bool is_y, bool is_max, float omp) {
+  if (!is_y) return -p;
+  return is_max ? omp : 1.f - p;
+}
+
 __device__ __forceinline__ float grad_elem(const RowCoef& k, float u, int j, bool in_s) {
   float dz = 0.f;
-  const float ind = j == k.y ? 1.f : 0.f;
+  const bool is_y = j == k.y;
   if (k.need_full) {
-    const float lp2 = (u - k.m2) - k.log2z;
+    const float d = u - k.m2;
+    const float lp2 = d - k.log2z;
     const float p = ex2(lp2);
-    dz += k.gv * (ind - p) - k.ghv * p * fmaf(lp2, kLn2, k.h_full);
+    dz += k.gv * ind_minus(p, is_y, d == 0.f, k.omp_full) - k.ghv * p * fmaf(lp2, kLn2, k.h_full);
   }
   if (in_s && k.need_sup) {
-    const float lq2 = (u - k.msup) - k.log2zs;
+    const float d = u - k.msup;
+    const float lq2 = d - k.log2zs;
     const float q = ex2(lq2);
-    dz += k.gs * (ind - q) - k.ghs * q * fmaf(lq2, kLn2, k.h_sup);
+    dz += k.gs * ind_minus(q, is_y, d == 0.f, k.omp_sup) - k.ghs * q * fmaf(lq2, kLn2, k.h_sup);
   }
   return dz * k.scale;
 }
@@ -132,8 +144,9 @@ __global__ void __launch_bounds__(kThreads) score_bwd_kernel(BwdParams P, int nc
     }
     s = block_reduce(s, red);
     k.m2 = s.m;
-    k.log2z = log2f(s.z);
-    k.h_full = kLn2 * (k.log2z - s.a / s.z);
+    k.log2z = stats_log2z(s);
+    k.h_full = kLn2 * (k.log2z - s.a / stats_z(s));
+    k.omp_full = (s.c0 - 1.f + s.zr) / (s.c0 + s.zr);
   }
 
   if (recorded && k.need_sup) {

@@ -41,7 +41,7 @@ struct SelShared {
   uint32_t ured[kWarps];
   // aggregate pass partials (this CTA)
   float agg_mass, agg_a;
-  uint32_t agg_ngt, agg_eq;
+  uint32_t agg_ngt, agg_eq, agg_top;
   // broadcast slots
   unsigned long long b_target, b_above_cnt, b_above_mass, b_at_cnt, b_at_mass;
   uint32_t b_digit;
@@ -310,10 +310,10 @@ __global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P)
   Stats rs = stats_empty();
   for (uint32_t r = 0; r < CL; ++r) stats_merge(rs, sh.gathered[r]);
 
-  const bool nonfinite = !(isfinite(rs.m) && isfinite(rs.z) && isfinite(rs.a));
+  const bool nonfinite = !stats_finite(rs);
   const float m2 = rs.m;
-  const float log2z = log2f(rs.z);
-  const float h_full = kLn2 * (log2z - rs.a / rs.z);
+  const float log2z = stats_log2z(rs);
+  const float h_full = kLn2 * (log2z - rs.a / stats_z(rs));
 
   const int kk = P.top_k ? P.top_k[row] : P.top_k_scalar;
   const float pp = P.top_p ? P.top_p[row] : P.top_p_scalar;
@@ -326,6 +326,7 @@ __global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P)
   uint32_t tkey = 0;
   int32_t tie_cut = INT_MAX;
   float log2zs = log2z;
+  float c0s = rs.c0, zrs = rs.zr;
   float h_support = h_full;
   int32_t n_support = nonfinite ? 0 : V;
 
@@ -394,7 +395,8 @@ __global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P)
     }
 
     // ---- support sums: keys above tkey, and the tie group at tkey
-    uint32_t ngt = 0, neq = 0;
+    // (elements equal to the row max are counted apart, as in Stats)
+    uint32_t ngt = 0, neq = 0, ntop = 0;
     float smass = 0.f, sa = 0.f;
     {
       const uint32_t t = tkey;
@@ -404,7 +406,10 @@ __global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P)
           const float d = __fmul_rn(value_of(raw), c) - m2;
           const float e = ex2(d);
           ++ngt;
-          smass += e;
+          if (d == 0.f)
+            ++ntop;
+          else
+            smass += e;
           sa = fmaf(d, e, sa);
         } else if (key == t) {
           ++neq;
@@ -413,16 +418,18 @@ __global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P)
     }
     ngt = block_sum(ngt, sh.ured);
     neq = block_sum(neq, sh.ured);
+    ntop = block_sum(ntop, sh.ured);
     smass = block_sum(smass, sh.fred);
     sa = block_sum(sa, sh.fred);
     if (tid == 0) {
       sh.agg_ngt = ngt;
       sh.agg_eq = neq;
+      sh.agg_top = ntop;
       sh.agg_mass = smass;
       sh.agg_a = sa;
     }
     cluster.sync();
-    uint32_t tot_gt = 0, tot_eq = 0;
+    uint32_t tot_gt = 0, tot_eq = 0, tot_top = 0;
     float tot_mass = 0.f, tot_a = 0.f;
     uint32_t eq_rank[8];
     for (uint32_t r = 0; r < CL; ++r) {
@@ -430,16 +437,22 @@ __global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P)
       tot_gt += rsh->agg_ngt;
       eq_rank[r] = rsh->agg_eq;
       tot_eq += eq_rank[r];
+      tot_top += rsh->agg_top;
       tot_mass += rsh->agg_mass;
       tot_a += rsh->agg_a;
     }
     const unsigned long long ckeep = all_ties ? tot_eq : (cnum < tot_eq ? cnum : tot_eq);
     const float dt = __fmul_rn(KT::decode(tkey), c) - m2;
     const float et = ex2(dt);
-    const float mass_s = tot_mass + static_cast<float>(ckeep) * et;
-    const float a_s = tot_a + static_cast<float>(ckeep) * dt * et;
-    log2zs = log2f(mass_s);
-    h_support = kLn2 * (log2zs - a_s / mass_s);
+    Stats ss;
+    ss.m = m2;
+    ss.c0 = static_cast<float>(tot_top) + (dt == 0.f ? static_cast<float>(ckeep) : 0.f);
+    ss.zr = tot_mass + (dt == 0.f ? 0.f : static_cast<float>(ckeep) * et);
+    ss.a = tot_a + static_cast<float>(ckeep) * dt * et;
+    log2zs = stats_log2z(ss);
+    h_support = kLn2 * (log2zs - ss.a / stats_z(ss));
+    c0s = ss.c0;
+    zrs = ss.zr;
     n_support = static_cast<int32_t>(tot_gt + ckeep);
 
     // ---- tie resolution: id of the last tie kept (ascending id order)
@@ -561,6 +574,10 @@ __global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P)
       cx.flags = f;
       cx.n_support = n_support;
       cx.status = status;
+      cx.c0_full = rs.c0;
+      cx.zr_full = rs.zr;
+      cx.c0_sup = c0s;
+      cx.zr_sup = zrs;
       P.ctx[row] = cx;
     }
   }
@@ -698,14 +715,14 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
     bool nonfinite = any_nf != 0;
     float m2 = nan, log2z = nan, h_full = nan;
     if (need_full) {
-      if (!(isfinite(f.m) && isfinite(f.z) && isfinite(f.a))) nonfinite = true;
+      if (!stats_finite(f)) nonfinite = true;
       m2 = f.m;
-      log2z = log2f(f.z);
-      h_full = kLn2 * (log2z - f.a / f.z);
+      log2z = stats_log2z(f);
+      h_full = kLn2 * (log2z - f.a / stats_z(f));
     }
     const float msup = s.m;
-    const float log2zs = empty ? nan : log2f(s.z);
-    const float h_sup = empty ? 0.f : kLn2 * (log2zs - s.a / s.z);
+    const float log2zs = empty ? nan : stats_log2z(s);
+    const float h_sup = empty ? 0.f : kLn2 * (log2zs - s.a / stats_z(s));
     float lp_v = nan, lp_s = nan;
     bool in_s = false;
     if (!target_ok) status |= VS_ROW_TARGET_OUT_OF_RANGE;
@@ -754,6 +771,10 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
       cx.flags = fl;
       cx.n_support = nonfinite ? 0 : static_cast<int32_t>(nkeep);
       cx.status = status;
+      cx.c0_full = f.c0;
+      cx.zr_full = f.zr;
+      cx.c0_sup = s.c0;
+      cx.zr_sup = s.zr;
       P.ctx[row] = cx;
     }
   }

@@ -312,7 +312,8 @@ def test_backward_recorded_support(mode):
     g_lps = rng.normal(size=rows).astype(F32)
     g_hs = rng.normal(size=rows).astype(F32)
     if mode == "sparse":
-        g_lps[(sup >= 0).sum(1) == 0] = 0.0  # empty rows' lp_S gradient is dense
+        empty = ((sup >= 0) & (sup < vocab)).sum(1) == 0
+        g_lps[empty] = 0.0  # empty rows' lp_S gradient is dense (full vocabulary)
     gref = oracle.score_grad(logits, targets, None, g_lps.astype(np.float64), None,
                              g_hs.astype(np.float64), temperature=float(temp[0]), support=sup)
     if mode == "dense":
