@@ -26,24 +26,52 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 256;
+// Exact-key window of the bf16 select: the kWin keys at and below the row's
+// maximum key (32 binades of bf16 below the maximum value, same sign).
+constexpr int kWin = 4096;
 
-// Shared state of one CTA, placed after the row slice in dynamic smem.
-struct SelShared {
-  unsigned long long mass[2][kBins];  // fixed-point mass histogram (double-buffered)
-  unsigned long long gmass[kBins];    // cluster-reduced
+typedef unsigned long long u64;
+
+// Arrays of the general radix descent (fp32 keys, or a bf16 row whose
+// crossing lies below the window).  They alias the window area.
+struct RadixArrays {
+  u64 mass[2][kBins];  // fixed-point mass histogram (double-buffered)
+  u64 gmass[kBins];    // cluster-reduced
   uint32_t cnt[2][kBins];
   uint32_t gcnt[kBins];
+};
+
+// Bytes of the window / radix area of a CTA in a cluster of `cl`.
+__host__ __device__ constexpr size_t big_area_bytes(int cl) {
+  return (static_cast<size_t>(kWin) + (kWin + cl - 1) / cl) * 4 > sizeof(RadixArrays)
+             ? (static_cast<size_t>(kWin) + (kWin + cl - 1) / cl) * 4
+             : sizeof(RadixArrays);
+}
+
+// Small shared state of one CTA.
+struct SelShared {
   uint64_t bar;
   Stats part;  // this CTA's row statistics
+  float vmax_part;
   Stats gathered[8];
+  float vmax_g[8];
   Stats red[kWarps];
   float fred[kWarps];
   uint32_t ured[kWarps];
-  // aggregate pass partials (this CTA)
+  u64 ulred[kWarps];
+  u64 scan_a[kWarps], scan_b[kWarps];
+  // window slice totals (this CTA) and their cluster gather
+  u64 slice_cnt, slice_mass;
+  u64 g_slice_cnt[8], g_slice_mass[8];
+  // window search results (written by the owning CTA; one slot per search so
+  // that a second search never overwrites a result a peer may still read)
+  uint32_t res_key[2];
+  u64 res_above_cnt[2], res_above_mass[2], res_at_cnt[2], res_at_mass[2];
+  // support-sum partials (this CTA)
   float agg_mass, agg_a;
   uint32_t agg_ngt, agg_eq, agg_top;
-  // broadcast slots
-  unsigned long long b_target, b_above_cnt, b_above_mass, b_at_cnt, b_at_mass;
+  // radix broadcast slots
+  u64 b_target, b_above_cnt, b_above_mass, b_at_cnt, b_at_mass;
   uint32_t b_digit;
   int32_t tie_cut;
   uint32_t timeout;
@@ -52,7 +80,7 @@ struct SelShared {
 
 struct Desc {
   uint32_t key;
-  unsigned long long above_cnt, above_mass, at_cnt, at_mass;
+  u64 above_cnt, above_mass, at_cnt, at_mass;
 };
 
 __device__ __forceinline__ float fx_scale(int shift) {
@@ -74,36 +102,65 @@ __device__ __forceinline__ void for_each(const Raw* buf, int n, F&& f) {
   for (int j = nfull * VEC + threadIdx.x; j < n; j += blockDim.x) f(j, buf[j]);
 }
 
+// Exclusive suffix sums over the threads of the block (thread t gets the sum
+// of a and b over threads t' > t).  Uniform call.
+__device__ __forceinline__ void block_suffix_excl(u64 a, u64 b, u64& ea, u64& eb, SelShared& sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  u64 ia = a, ib = b;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const u64 ta = __shfl_down_sync(0xffffffffu, ia, o);
+    const u64 tb = __shfl_down_sync(0xffffffffu, ib, o);
+    if (lane + o < 32) {
+      ia += ta;
+      ib += tb;
+    }
+  }
+  if (lane == 0) {
+    sh.scan_a[warp] = ia;
+    sh.scan_b[warp] = ib;
+  }
+  __syncthreads();
+  u64 wa = 0, wb = 0;
+  const int nw = blockDim.x >> 5;
+  for (int w = warp + 1; w < nw; ++w) {
+    wa += sh.scan_a[w];
+    wb += sh.scan_b[w];
+  }
+  ea = wa + ia - a;
+  eb = wb + ib - b;
+  __syncthreads();
+}
+
 // Warp 0: find, scanning bins from the top (largest key first), the bin where
 // the cumulative `by` quantity first reaches `need` (>= 1).  Returns the
 // digit and the sums (count and mass) of the bins strictly above it, in lane 0.
-__device__ void scan_bins(const uint32_t* gcnt, const unsigned long long* gmass, bool by_mass,
-                          unsigned long long need, uint32_t& digit,
-                          unsigned long long& above_cnt, unsigned long long& above_mass) {
+__device__ void scan_bins(const uint32_t* gcnt, const u64* gmass, bool by_mass, u64 need,
+                          uint32_t& digit, u64& above_cnt, u64& above_mass) {
   const int lane = threadIdx.x & 31;
-  unsigned long long v[8];
-  unsigned long long lsum = 0;
+  u64 v[8];
+  u64 lsum = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int b = 255 - 8 * lane - i;
-    v[i] = by_mass ? gmass[b] : static_cast<unsigned long long>(gcnt[b]);
+    v[i] = by_mass ? gmass[b] : static_cast<u64>(gcnt[b]);
     lsum += v[i];
   }
-  unsigned long long incl = lsum;
+  u64 incl = lsum;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const unsigned long long t = __shfl_up_sync(0xffffffffu, incl, o);
+    const u64 t = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += t;
   }
-  const unsigned long long excl = incl - lsum;
+  const u64 excl = incl - lsum;
   const bool hit = excl < need && need <= incl;
   const uint32_t ballot = __ballot_sync(0xffffffffu, hit);
-  int d = -1;
+  int d;
   if (ballot != 0) {
     const int hl = __ffs(ballot) - 1;
     int local = -1;
     if (lane == hl) {
-      unsigned long long s = excl;
+      u64 s = excl;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         if (local < 0 && s + v[i] >= need) local = 255 - 8 * lane - i;
@@ -114,21 +171,17 @@ __device__ void scan_bins(const uint32_t* gcnt, const unsigned long long* gmass,
   } else {
     // target beyond the total (cannot happen for consistent targets): take
     // the lowest non-empty bin so that the result stays well defined.
-    unsigned long long any = 0;
-    int lowest = -1;
+    int lowest = 256;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int b = 255 - 8 * lane - i;
       if (gcnt[b] != 0) lowest = b;
-      any |= gcnt[b];
     }
-    (void)any;
-    int best = lowest < 0 ? 256 : lowest;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) best = min(best, __shfl_xor_sync(0xffffffffu, best, o));
-    d = best == 256 ? 0 : best;
+    for (int o = 16; o > 0; o >>= 1) lowest = min(lowest, __shfl_xor_sync(0xffffffffu, lowest, o));
+    d = lowest == 256 ? 0 : lowest;
   }
-  unsigned long long ac = 0, am = 0;
+  u64 ac = 0, am = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int b = 255 - 8 * lane - i;
@@ -155,17 +208,17 @@ __device__ void scan_bins(const uint32_t* gcnt, const unsigned long long* gmass,
 // alternates per level, so one cluster barrier per level suffices.
 template <typename Raw>
 __device__ Desc descend(const Raw* buf, int n, float c, float m2, int fx_shift, bool by_mass,
-                        bool need_mass, unsigned long long target, float p, SelShared& sh,
+                        bool need_mass, u64 target, float p, SelShared& sh, RadixArrays& ra,
                         cg::cluster_group& cluster, int& hb) {
   constexpr int KB = KeyTraits<Raw>::kBits;
   const uint32_t CL = cluster.num_blocks();
   const float fxs = fx_scale(fx_shift);
   uint32_t prefix = 0;
-  unsigned long long above_cnt = 0, above_mass = 0;
+  u64 above_cnt = 0, above_mass = 0;
   Desc out{};
   for (int shift = KB - 8; shift >= 0; shift -= 8) {
-    uint32_t* cnt = sh.cnt[hb];
-    unsigned long long* mass = sh.mass[hb];
+    uint32_t* cnt = ra.cnt[hb];
+    u64* mass = ra.mass[hb];
     for (int b = threadIdx.x; b < kBins; b += blockDim.x) {
       cnt[b] = 0;
       mass[b] = 0;
@@ -181,7 +234,7 @@ __device__ Desc descend(const Raw* buf, int n, float c, float m2, int fx_shift, 
         atomicAdd(&cnt[digit], 1u);
         if (need_mass) {
           const float e = ex2(__fmul_rn(value_of(raw), c) - m2);
-          const unsigned long long fx = __float2ull_rn(e * fxs);
+          const u64 fx = __float2ull_rn(e * fxs);
           if (fx) atomicAdd(&mass[digit], fx);
         }
       }
@@ -189,44 +242,43 @@ __device__ Desc descend(const Raw* buf, int n, float c, float m2, int fx_shift, 
     __syncthreads();
     cluster.sync();
     for (int b = threadIdx.x; b < kBins; b += blockDim.x) {
-      uint32_t sc = 0;
-      unsigned long long sm = 0;
+      uint32_t scnt = 0;
+      u64 smass = 0;
       for (uint32_t r = 0; r < CL; ++r) {
-        sc += *cluster.map_shared_rank(&cnt[b], r);
-        sm += *cluster.map_shared_rank(&mass[b], r);
+        scnt += *cluster.map_shared_rank(&cnt[b], r);
+        smass += *cluster.map_shared_rank(&mass[b], r);
       }
-      sh.gcnt[b] = sc;
-      sh.gmass[b] = sm;
+      ra.gcnt[b] = scnt;
+      ra.gmass[b] = smass;
     }
     __syncthreads();
     hb ^= 1;
     if (threadIdx.x < 32) {
-      unsigned long long tgt = target;
+      u64 tgt = target;
       if (tgt == 0) {
         // implicit target: ceil(p * total mass), clamped to [1, total]
-        unsigned long long tot = 0;
-        for (int i = threadIdx.x; i < kBins; i += 32) tot += sh.gmass[i];
+        u64 tot = 0;
+        for (int i = threadIdx.x; i < kBins; i += 32) tot += ra.gmass[i];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
-        double want = ceil(static_cast<double>(p) * static_cast<double>(tot));
-        unsigned long long t = want <= 1.0 ? 1ull
-                               : want >= static_cast<double>(tot)
-                                   ? tot
-                                   : static_cast<unsigned long long>(want);
+        const double want = ceil(static_cast<double>(p) * static_cast<double>(tot));
+        const u64 t = want <= 1.0 ? 1ull
+                      : want >= static_cast<double>(tot) ? tot
+                                                         : static_cast<u64>(want);
         tgt = t < 1 ? 1 : t;
       }
-      const unsigned long long have = by_mass ? above_mass : above_cnt;
-      const unsigned long long need = tgt > have ? tgt - have : 1;
+      const u64 have = by_mass ? above_mass : above_cnt;
+      const u64 need = tgt > have ? tgt - have : 1;
       uint32_t digit;
-      unsigned long long ac, am;
-      scan_bins(sh.gcnt, sh.gmass, by_mass, need, digit, ac, am);
+      u64 ac, am;
+      scan_bins(ra.gcnt, ra.gmass, by_mass, need, digit, ac, am);
       if (threadIdx.x == 0) {
         sh.b_target = tgt;
         sh.b_digit = digit;
         sh.b_above_cnt = ac;
         sh.b_above_mass = am;
-        sh.b_at_cnt = sh.gcnt[digit];
-        sh.b_at_mass = sh.gmass[digit];
+        sh.b_at_cnt = ra.gcnt[digit];
+        sh.b_at_mass = ra.gmass[digit];
       }
     }
     __syncthreads();
@@ -244,9 +296,144 @@ __device__ Desc descend(const Raw* buf, int n, float c, float m2, int fx_shift, 
   return out;
 }
 
+// ---------------------------------------------------------------------------
+// exact-key window (bf16): the histogram of keys klo .. klo + kWin - 1,
+// cluster-reduced so that CTA r holds bins [r S, r S + S).
+
+struct Window {
+  uint32_t klo, kmax;
+  int S;          // bins per CTA slice
+  uint32_t* hist;  // this CTA's unreduced histogram [kWin]
+  uint32_t* red;   // this CTA's reduced slice [S]
+  float c, m2, fxs;
+};
+
+__device__ __forceinline__ u64 bin_fx(const Window& w, uint32_t key) {
+  const float e = ex2(__fmul_rn(KeyTraits<uint16_t>::decode(key), w.c) - w.m2);
+  return __float2ull_rn(e * w.fxs);
+}
+
+// Build the window histogram, reduce it across the cluster and gather the
+// per-slice totals (count and fixed-point mass) into every CTA.
+__device__ void window_build(const uint16_t* buf, int n, Window& w, SelShared& sh,
+                             cg::cluster_group& cluster) {
+  const uint32_t CL = cluster.num_blocks();
+  const uint32_t rank = cluster.block_rank();
+  for (int b = threadIdx.x; b < kWin; b += blockDim.x) w.hist[b] = 0u;
+  __syncthreads();
+  const uint32_t klo = w.klo;
+  uint32_t* hist = w.hist;
+  for_each(buf, n, [&](int, uint16_t raw) {
+    const uint32_t key = key_of(raw);
+    if (key >= klo) atomicAdd(&hist[key - klo], 1u);
+  });
+  __syncthreads();
+  cluster.sync();
+  const int b0 = static_cast<int>(rank) * w.S;
+  const int b1 = min(kWin, b0 + w.S);
+  u64 tc = 0, tm = 0;
+  for (int b = b0 + threadIdx.x; b < b1; b += blockDim.x) {
+    uint32_t sum = 0;
+    for (uint32_t r = 0; r < CL; ++r) sum += *cluster.map_shared_rank(&hist[b], r);
+    w.red[b - b0] = sum;
+    if (sum) {
+      tc += sum;
+      tm += static_cast<u64>(sum) * bin_fx(w, klo + b);
+    }
+  }
+  tc = block_sum(tc, sh.ulred);
+  tm = block_sum(tm, sh.ulred);
+  if (threadIdx.x == 0) {
+    sh.slice_cnt = tc;
+    sh.slice_mass = tm;
+  }
+  cluster.sync();
+  if (threadIdx.x < static_cast<int>(CL)) {
+    const SelShared* rsh = cluster.map_shared_rank(&sh, threadIdx.x);
+    sh.g_slice_cnt[threadIdx.x] = rsh->slice_cnt;
+    sh.g_slice_mass[threadIdx.x] = rsh->slice_mass;
+  }
+  __syncthreads();
+}
+
+// Find, from the largest key down, the window bin where the cumulative count
+// (by_mass false) or fixed-point mass first reaches `need` (>= 1).  Returns
+// false (uniformly across the cluster) when the window holds less.
+__device__ bool window_search(const Window& w, bool by_mass, u64 need, int slot, Desc& out,
+                              SelShared& sh, cg::cluster_group& cluster) {
+  const int CL = static_cast<int>(cluster.num_blocks());
+  const int rank = static_cast<int>(cluster.block_rank());
+  u64 cum = 0, cum_c = 0, cum_m = 0;
+  int rs = -1;
+  for (int r = CL - 1; r >= 0; --r) {
+    const u64 t = by_mass ? sh.g_slice_mass[r] : sh.g_slice_cnt[r];
+    if (cum + t >= need) {
+      rs = r;
+      break;
+    }
+    cum += t;
+    cum_c += sh.g_slice_cnt[r];
+    cum_m += sh.g_slice_mass[r];
+  }
+  if (rs < 0) return false;
+  if (rank == rs) {
+    const int b0 = rs * w.S;
+    const int nb = min(kWin, b0 + w.S) - b0;
+    const int per = (nb + blockDim.x - 1) / blockDim.x;
+    const int i0 = threadIdx.x * per, i1 = min(nb, i0 + per);
+    u64 lc = 0, lm = 0;
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t cnt = w.red[i];
+      if (cnt) {
+        lc += cnt;
+        lm += static_cast<u64>(cnt) * bin_fx(w, w.klo + b0 + i);
+      }
+    }
+    u64 ec, em;
+    block_suffix_excl(lc, lm, ec, em, sh);
+    const u64 base = cum + (by_mass ? em : ec);
+    const u64 mine = by_mass ? lm : lc;
+    if (base < need && need <= base + mine) {
+      u64 ac = cum_c + ec, am = cum_m + em;
+      for (int i = i1 - 1; i >= i0; --i) {
+        const uint32_t cnt = w.red[i];
+        const u64 fx = cnt ? static_cast<u64>(cnt) * bin_fx(w, w.klo + b0 + i) : 0ull;
+        const u64 v = by_mass ? fx : cnt;
+        if (cnt && (by_mass ? am : ac) + v >= need) {
+          sh.res_key[slot] = w.klo + b0 + i;
+          sh.res_above_cnt[slot] = ac;
+          sh.res_above_mass[slot] = am;
+          sh.res_at_cnt[slot] = cnt;
+          sh.res_at_mass[slot] = fx;
+          break;
+        }
+        ac += cnt;
+        am += fx;
+      }
+    }
+  }
+  cluster.sync();
+  const SelShared* rsh = cluster.map_shared_rank(&sh, rs);
+  out.key = rsh->res_key[slot];
+  out.above_cnt = rsh->res_above_cnt[slot];
+  out.above_mass = rsh->res_above_mass[slot];
+  out.at_cnt = rsh->res_at_cnt[slot];
+  out.at_mass = rsh->res_at_mass[slot];
+  return true;
+}
+
+// Target mass of inclusive top-p: ceil(p * mass), clamped to [1, mass].
+__device__ __forceinline__ u64 topp_target(float p, double mass) {
+  const double want = ceil(static_cast<double>(p) * mass);
+  if (want <= 1.0) return 1ull;
+  if (want >= mass) return static_cast<u64>(mass);
+  return static_cast<u64>(want);
+}
+
 template <typename Raw>
-__global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P) {
+__global__ void __launch_bounds__(kThreads, 3) score_computed_kernel(ScoreParams P) {
   constexpr int VEC = 16 / sizeof(Raw);
+  constexpr bool kBf16 = sizeof(Raw) == 2;
   using KT = KeyTraits<Raw>;
   cg::cluster_group cluster = cg::this_cluster();
   const uint32_t rank = cluster.block_rank();
@@ -256,7 +443,10 @@ __global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P)
 
   extern __shared__ __align__(128) uint8_t smem_raw[];
   Raw* buf = reinterpret_cast<Raw*>(smem_raw);
-  SelShared& sh = *reinterpret_cast<SelShared*>(smem_raw + static_cast<size_t>(P.chunk) * sizeof(Raw));
+  const size_t chunk_bytes = static_cast<size_t>(P.chunk) * sizeof(Raw);
+  SelShared& sh = *reinterpret_cast<SelShared*>(smem_raw + chunk_bytes);
+  uint8_t* big = smem_raw + chunk_bytes + ((sizeof(SelShared) + 127) & ~size_t(127));
+  RadixArrays& ra = *reinterpret_cast<RadixArrays*>(big);
 
   const int V = P.vocab;
   const int c0 = static_cast<int>(rank) * P.chunk;
@@ -282,10 +472,11 @@ __global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P)
   }
   __syncthreads();
 
-  // ---- pass 1: online max / sum / entropy sum over the slice
+  // ---- pass 1: online max / sum / entropy sum over the slice (and the max value)
   const float T = P.temperature ? P.temperature[row] : P.temperature_scalar;
   const float c = kLog2e / T;
   Stats s = stats_empty();
+  float vmax = -kInf;
   {
     const int nfull = n / VEC;
     const uint4* v4 = reinterpret_cast<const uint4*>(buf);
@@ -294,21 +485,44 @@ __global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P)
       unpack(v4[v], r);
       float u[VEC];
 #pragma unroll
-      for (int i = 0; i < VEC; ++i) u[i] = __fmul_rn(value_of(r[i]), c);
+      for (int i = 0; i < VEC; ++i) {
+        const float x = value_of(r[i]);
+        vmax = fmaxf(vmax, x);
+        u[i] = __fmul_rn(x, c);
+      }
       stats_add(s, u);
     }
     for (int j = nfull * VEC + tid; j < n; j += blockDim.x) {
-      float u[1] = {__fmul_rn(value_of(buf[j]), c)};
+      const float x = value_of(buf[j]);
+      vmax = fmaxf(vmax, x);
+      float u[1] = {__fmul_rn(x, c)};
       stats_add(s, u);
     }
   }
   s = block_reduce(s, sh.red);
-  if (tid == 0) sh.part = s;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+  if ((tid & 31) == 0) sh.fred[tid >> 5] = vmax;
+  __syncthreads();
+  if (tid == 0) {
+    float vm = -kInf;
+    for (int w = 0; w < kWarps; ++w) vm = fmaxf(vm, sh.fred[w]);
+    sh.part = s;
+    sh.vmax_part = vm;
+  }
   cluster.sync();
-  if (tid < static_cast<int>(CL)) sh.gathered[tid] = *cluster.map_shared_rank(&sh.part, tid);
+  if (tid < static_cast<int>(CL)) {
+    const SelShared* rsh = cluster.map_shared_rank(&sh, tid);
+    sh.gathered[tid] = rsh->part;
+    sh.vmax_g[tid] = rsh->vmax_part;
+  }
   __syncthreads();
   Stats rs = stats_empty();
-  for (uint32_t r = 0; r < CL; ++r) stats_merge(rs, sh.gathered[r]);
+  float vmax_row = -kInf;
+  for (uint32_t r = 0; r < CL; ++r) {
+    stats_merge(rs, sh.gathered[r]);
+    vmax_row = fmaxf(vmax_row, sh.vmax_g[r]);
+  }
 
   const bool nonfinite = !stats_finite(rs);
   const float m2 = rs.m;
@@ -326,56 +540,115 @@ __global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P)
   uint32_t tkey = 0;
   int32_t tie_cut = INT_MAX;
   float log2zs = log2z;
-  float c0s = rs.c0, zrs = rs.zr;
   float h_support = h_full;
+  float c0s = rs.c0, zrs = rs.zr;
   int32_t n_support = nonfinite ? 0 : V;
 
   if (filtered) {
-    int hb = 0;
-    bool all_ties = true;
-    unsigned long long cnum = 0;  // ties kept at tkey when !all_ties
+    bool all_ties = true;  // every element with key == tkey is kept
+    u64 cnum = 0;          // ties kept at tkey when !all_ties
     bool have_t = false;
-    if (use_k) {
-      Desc d = descend(buf, n, c, m2, P.fx_shift, false, use_p,
-                       static_cast<unsigned long long>(kk), 1.f, sh, cluster, hb);
-      const unsigned long long ck = static_cast<unsigned long long>(kk) - d.above_cnt;
-      tkey = d.key;
-      cnum = ck;
-      all_ties = ck >= d.at_cnt;
-      have_t = true;
-      if (use_p) {
-        const unsigned long long fx_t = d.at_cnt ? d.at_mass / d.at_cnt : 0;
-        const unsigned long long mass1 = d.above_mass + ck * fx_t;
-        double want = ceil(static_cast<double>(pp) * static_cast<double>(mass1));
-        unsigned long long tp = want <= 1.0 ? 1ull
-                                : want >= static_cast<double>(mass1)
-                                    ? mass1
-                                    : static_cast<unsigned long long>(want);
-        if (tp < 1) tp = 1;
-        Desc e = descend(buf, n, c, m2, P.fx_shift, true, true, tp, pp, sh, cluster, hb);
-        const unsigned long long fxe = e.at_cnt ? e.at_mass / e.at_cnt : 0;
-        const unsigned long long need = tp > e.above_mass ? tp - e.above_mass : 0;
-        unsigned long long cp = fxe ? (need + fxe - 1) / fxe : e.at_cnt;
+    bool sums_done = false;
+    uint32_t tot_gt = 0, tot_eq = 0, tot_top = 0;
+    float tot_mass = 0.f, tot_a = 0.f;
+    uint32_t eq_rank[8];
+    const float fxs = fx_scale(P.fx_shift);
+
+    // ---- exact-key window select (bf16 keys with top-k and/or top-p)
+    bool win_ok = false;
+    Window w{};
+    if constexpr (kBf16) {
+      if (use_k || use_p) {
+        w.kmax = key_of(static_cast<uint16_t>(__float_as_uint(vmax_row) >> 16));
+        w.klo = w.kmax >= static_cast<uint32_t>(kWin - 1) ? w.kmax - (kWin - 1) : 0u;
+        w.S = (kWin + CL - 1) / CL;
+        w.hist = reinterpret_cast<uint32_t*>(big);
+        w.red = w.hist + kWin;
+        w.c = c;
+        w.m2 = m2;
+        w.fxs = fxs;
+        window_build(buf, n, w, sh, cluster);
+        win_ok = true;
+        Desc dk{}, dp{};
+        u64 ck = 0;
+        if (use_k) {
+          win_ok = window_search(w, false, static_cast<u64>(kk), 0, dk, sh, cluster);
+          if (win_ok) {
+            ck = static_cast<u64>(kk) - dk.above_cnt;
+            tkey = dk.key;
+            cnum = ck;
+            all_ties = ck >= dk.at_cnt;
+            have_t = true;
+          }
+        }
+        if (win_ok && use_p) {
+          double mass1;
+          if (use_k) {
+            const u64 fx_t = dk.at_cnt ? dk.at_mass / dk.at_cnt : 0;
+            mass1 = static_cast<double>(dk.above_mass + ck * fx_t);
+          } else {
+            mass1 = (static_cast<double>(rs.c0) + static_cast<double>(rs.zr)) * static_cast<double>(fxs);
+          }
+          const u64 tp = topp_target(pp, mass1);
+          win_ok = window_search(w, true, tp, 1, dp, sh, cluster);
+          if (win_ok) {
+            const u64 fxe = dp.at_cnt ? dp.at_mass / dp.at_cnt : 0;
+            const u64 need = tp > dp.above_mass ? tp - dp.above_mass : 0;
+            u64 cp = fxe ? (need + fxe - 1) / fxe : dp.at_cnt;
+            if (cp < 1) cp = 1;
+            if (cp > dp.at_cnt) cp = dp.at_cnt;
+            if (use_k && dp.key == tkey && cp > ck) cp = ck;
+            tkey = dp.key;
+            cnum = cp;
+            all_ties = cp >= dp.at_cnt;
+            have_t = true;
+          }
+        }
+      }
+    }
+
+    if (!win_ok && (use_k || use_p)) {
+      // ---- general radix descent (fp32 keys, or the crossing lies below the window)
+      int hb = 0;
+      have_t = false;
+      all_ties = true;
+      if (use_k) {
+        Desc d = descend(buf, n, c, m2, P.fx_shift, false, use_p, static_cast<u64>(kk), 1.f, sh,
+                         ra, cluster, hb);
+        const u64 ck = static_cast<u64>(kk) - d.above_cnt;
+        tkey = d.key;
+        cnum = ck;
+        all_ties = ck >= d.at_cnt;
+        have_t = true;
+        if (use_p) {
+          const u64 fx_t = d.at_cnt ? d.at_mass / d.at_cnt : 0;
+          const u64 tp = topp_target(pp, static_cast<double>(d.above_mass + ck * fx_t));
+          Desc e = descend(buf, n, c, m2, P.fx_shift, true, true, tp, pp, sh, ra, cluster, hb);
+          const u64 fxe = e.at_cnt ? e.at_mass / e.at_cnt : 0;
+          const u64 need = tp > e.above_mass ? tp - e.above_mass : 0;
+          u64 cp = fxe ? (need + fxe - 1) / fxe : e.at_cnt;
+          if (cp < 1) cp = 1;
+          if (cp > e.at_cnt) cp = e.at_cnt;
+          if (e.key == tkey && cp > ck) cp = ck;
+          tkey = e.key;
+          cnum = cp;
+          all_ties = cp >= e.at_cnt;
+        }
+      } else {
+        Desc e = descend(buf, n, c, m2, P.fx_shift, true, true, 0ull, pp, sh, ra, cluster, hb);
+        const u64 tp = sh.b_target;
+        const u64 fxe = e.at_cnt ? e.at_mass / e.at_cnt : 0;
+        const u64 need = tp > e.above_mass ? tp - e.above_mass : 0;
+        u64 cp = fxe ? (need + fxe - 1) / fxe : e.at_cnt;
         if (cp < 1) cp = 1;
         if (cp > e.at_cnt) cp = e.at_cnt;
-        if (e.key == tkey && cp > ck) cp = ck;
         tkey = e.key;
         cnum = cp;
         all_ties = cp >= e.at_cnt;
+        have_t = true;
       }
-    } else if (use_p) {
-      Desc e = descend(buf, n, c, m2, P.fx_shift, true, true, 0ull, pp, sh, cluster, hb);
-      const unsigned long long tp = sh.b_target;
-      const unsigned long long fxe = e.at_cnt ? e.at_mass / e.at_cnt : 0;
-      const unsigned long long need = tp > e.above_mass ? tp - e.above_mass : 0;
-      unsigned long long cp = fxe ? (need + fxe - 1) / fxe : e.at_cnt;
-      if (cp < 1) cp = 1;
-      if (cp > e.at_cnt) cp = e.at_cnt;
-      tkey = e.key;
-      cnum = cp;
-      all_ties = cp >= e.at_cnt;
-      have_t = true;
     }
+
     if (use_minp) {
       // smallest key whose probability ratio to the row max reaches min_p
       uint32_t lo = 0, hi = KT::kInfKey;
@@ -398,7 +671,31 @@ __global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P)
     // (elements equal to the row max are counted apart, as in Stats)
     uint32_t ngt = 0, neq = 0, ntop = 0;
     float smass = 0.f, sa = 0.f;
-    {
+    if constexpr (kBf16) {
+      if (win_ok && tkey >= w.klo) {
+        // from the reduced window bins of this CTA's slice
+        const int b0 = static_cast<int>(rank) * w.S;
+        const int b1 = min(kWin, b0 + w.S);
+        for (int b = b0 + tid; b < b1; b += blockDim.x) {
+          const uint32_t cnt = w.red[b - b0];
+          const uint32_t key = w.klo + b;
+          if (cnt && key > tkey) {
+            const float d = __fmul_rn(KT::decode(key), c) - m2;
+            const float e = ex2(d);
+            const float fc = static_cast<float>(cnt);
+            ngt += cnt;
+            if (d == 0.f)
+              ntop += cnt;
+            else
+              smass = fmaf(fc, e, smass);
+            sa = fmaf(fc * d, e, sa);
+          }
+        }
+        neq = w.hist[tkey - w.klo];  // this CTA's own elements at tkey
+        sums_done = true;
+      }
+    }
+    if (!sums_done) {
       const uint32_t t = tkey;
       for_each(buf, n, [&](int, Raw raw) {
         const uint32_t key = key_of(raw);
@@ -429,9 +726,6 @@ __global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P)
       sh.agg_a = sa;
     }
     cluster.sync();
-    uint32_t tot_gt = 0, tot_eq = 0, tot_top = 0;
-    float tot_mass = 0.f, tot_a = 0.f;
-    uint32_t eq_rank[8];
     for (uint32_t r = 0; r < CL; ++r) {
       const SelShared* rsh = cluster.map_shared_rank(&sh, r);
       tot_gt += rsh->agg_ngt;
@@ -441,7 +735,7 @@ __global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P)
       tot_mass += rsh->agg_mass;
       tot_a += rsh->agg_a;
     }
-    const unsigned long long ckeep = all_ties ? tot_eq : (cnum < tot_eq ? cnum : tot_eq);
+    const u64 ckeep = all_ties ? tot_eq : (cnum < tot_eq ? cnum : tot_eq);
     const float dt = __fmul_rn(KT::decode(tkey), c) - m2;
     const float et = ex2(dt);
     Stats ss;
@@ -457,7 +751,7 @@ __global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P)
 
     // ---- tie resolution: id of the last tie kept (ascending id order)
     if (ckeep < tot_eq) {
-      unsigned long long off = 0;
+      u64 off = 0;
       uint32_t owner = 0;
       for (uint32_t r = 0; r < CL; ++r) {
         if (off + eq_rank[r] >= ckeep) {
@@ -488,9 +782,9 @@ __global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P)
           if (lane == 31) sh.scan_tot[warp] = incl;
           __syncthreads();
           int wpre = 0, total = 0;
-          for (int w = 0; w < kWarps; ++w) {
-            if (w < warp) wpre += sh.scan_tot[w];
-            total += sh.scan_tot[w];
+          for (int ww = 0; ww < kWarps; ++ww) {
+            if (ww < warp) wpre += sh.scan_tot[ww];
+            total += sh.scan_tot[ww];
           }
           const int excl = base_count + wpre + incl - mine;
           if (excl < need && need <= excl + mine) {
@@ -588,8 +882,8 @@ __global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P)
     const int64_t wstride = (V + 31) / 32;
     uint32_t* mrow = P.support_mask + static_cast<int64_t>(row) * wstride + c0 / 32;
     const int lane = tid & 31, warp = tid >> 5;
-    for (int w = warp; w < words; w += kWarps) {
-      const int j = w * 32 + lane;
+    for (int wd = warp; wd < words; wd += kWarps) {
+      const int j = wd * 32 + lane;
       bool in = false;
       if (j < n && !nonfinite) {
         if (!filtered) {
@@ -600,7 +894,7 @@ __global__ void __launch_bounds__(kThreads) score_computed_kernel(ScoreParams P)
         }
       }
       const uint32_t bits = __ballot_sync(0xffffffffu, in);
-      if (lane == 0) mrow[w] = bits;
+      if (lane == 0) mrow[wd] = bits;
     }
   }
   cluster.sync();  // no CTA leaves while a peer may still read its shared memory
@@ -856,7 +1150,8 @@ int score_cluster_size(int vocab, vs_dtype dtype, int* chunk) {
 cudaError_t launch_score_computed(const ScoreParams& p, vs_dtype dtype, int cluster,
                                   cudaStream_t s) {
   const size_t esize = dtype == VS_BF16 ? 2 : 4;
-  const size_t smem = static_cast<size_t>(p.chunk) * esize + sizeof(SelShared);
+  const size_t smem = static_cast<size_t>(p.chunk) * esize +
+                      ((sizeof(SelShared) + 127) & ~size_t(127)) + big_area_bytes(cluster);
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(p.rows) * cluster, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);

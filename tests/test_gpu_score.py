@@ -108,6 +108,26 @@ def test_edge_rows_nonfinite_targets_ties_singletons():
     assert out["h_support"][4].item() == 0.0 and out["lp_support"][4].item() == 0.0
 
 
+@pytest.mark.parametrize("filt", [(100, 1.0, 0.0), (0, 0.5, 0.0), (50, 0.9, 0.01)])
+def test_crossing_below_the_key_window(filt):
+    # one logit tens of binades above the rest: with a huge temperature the
+    # selection crossing lies deep below the maximum's key, outside the
+    # exact-key window, so the general radix descent decides
+    rows, vocab = 4, 20_000
+    x = workloads.normal((rows, vocab), 1.0, seed=8, stream=1)
+    x[:, 3] = 3e9
+    logits = workloads.to_bf16_bits(x)
+    _run(logits, np.arange(rows, dtype=np.int32), np.full(rows, 1e9, F32), *filt)
+
+
+def test_all_negative_rows():
+    rows, vocab = 5, 30_000
+    x = workloads.normal((rows, vocab), 3.0, seed=12, stream=1) - 60.0
+    logits = workloads.to_bf16_bits(x)
+    for filt in [(0, 0.95, 0.0), (64, 0.8, 0.0), (0, 1.0, 0.1)]:
+        _run(logits, np.arange(rows, dtype=np.int32), np.full(rows, 0.9, F32), *filt)
+
+
 def test_singletons_are_exact_zeros():
     rows, vocab = 16, 20_000
     logits = workloads.random_logits(rows, vocab, 3.0, seed=21)
