@@ -691,7 +691,7 @@ __global__ void __launch_bounds__(kThreads, 3) score_computed_kernel(ScoreParams
             sa = fmaf(fc * d, e, sa);
           }
         }
-        neq = w.hist[tkey - w.klo];  // this CTA's own elements at tkey
+        if (tid == 0) neq = w.hist[tkey - w.klo];  // this CTA's own elements at tkey
         sums_done = true;
       }
     }
