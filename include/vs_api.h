@@ -213,6 +213,29 @@ vs_status vs_l1_distance(int32_t rows, int32_t vocab, int64_t ld, vs_dtype dtype
 
 size_t vs_l1_distance_workspace_size(int32_t rows);
 
+/* vs_l1_distance without a caller workspace.  The pages have no counterpart:
+ * this entry point exists for callers that cannot call cudaMalloc -- for
+ * example a plugin inside a host application whose device memory pool it
+ * cannot reach, or a serving loop that must not allocate after start-up
+ * because cudaMalloc may synchronise the device.  Arguments and results are
+ * those of vs_l1_distance; the scratch comes from a file-scope device array
+ * of VS_L1_STATIC_SCRATCH_BYTES inside libvs.so, which every GPU that loads
+ * the library holds until the process exits.  Nothing is allocated.
+ *  - rows above VS_L1_STATIC_MAX_ROWS: VS_ERR_UNSUPPORTED, nothing enqueued.
+ *  - The first call on a device, with that device current, looks up the
+ *    array's device address (cudaGetSymbolAddress) and caches it; make that
+ *    first call before any stream capture.
+ *  - Every call on a device shares the one array, which keeps the last call's
+ *    contents (each call overwrites what it reads), so calls that overlap on
+ *    the GPU (concurrent streams, or threads without ordering) race. */
+#define VS_L1_STATIC_MAX_ROWS 65536
+#define VS_L1_STATIC_SCRATCH_BYTES (16 + 8 * VS_L1_STATIC_MAX_ROWS)
+vs_status vs_l1_distance_static(int32_t rows, int32_t vocab, int64_t ld, vs_dtype dtype,
+                                const void* draft, const void* target, const float* row_weight,
+                                float* l1, float* accept_rate, float* loss_num_den_loss,
+                                void* grad_draft, vs_dtype grad_dtype, int64_t grad_ld,
+                                void* stream);
+
 /* Fused LM-head scoring ([xorl] section 1: chunked projection -> fixed-order
  * LSE -> support -> selected logprob; [SkyRL] Performance: the full logits
  * are never materialised).

@@ -89,6 +89,17 @@ vs_status check_args(const vs_score_args* a) {
 
 }  // namespace
 
+namespace vs {
+// Record the outcome of a C-ABI call made from another translation unit.
+vs_status set_last_error(vs_status code, const char* msg) {
+  if (code == VS_OK)
+    g_err.clear();
+  else
+    g_err = msg;
+  return code;
+}
+}  // namespace vs
+
 extern "C" {
 
 const char* vs_last_error(void) { return g_err.c_str(); }

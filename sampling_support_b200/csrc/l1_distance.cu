@@ -10,6 +10,8 @@
 // once.  Cross-CTA sums go through distributed shared memory in rank order;
 // cross-row sums (the loss) are reduced by a single block in row order.
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -343,3 +345,63 @@ cudaError_t launch_l1(int rows, int vocab, int64_t ld, vs_dtype dtype, const voi
 }
 
 }  // namespace vs
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of vs_l1_distance: the scratch (weight sum and the
+// per-row weighted distances) lives in a file-scope device array instead of a
+// caller workspace.
+
+namespace vs {
+vs_status set_last_error(vs_status code, const char* msg);
+}  // namespace vs
+
+namespace {
+
+static_assert(VS_L1_STATIC_SCRATCH_BYTES >= 16 + 8 * VS_L1_STATIC_MAX_ROWS, "scratch size");
+
+// One copy per GPU that loads the library, alive until the process exits.
+static __device__ __align__(256) unsigned char g_l1_scratch[VS_L1_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_l1_scratch on the current device, looked up once per
+// device (host code sees only a stand-in for the symbol, never its address).
+vs_status scratch_for_current_device(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return vs::set_last_error(VS_ERR_CUDA, cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices)
+    return vs::set_last_error(VS_ERR_UNSUPPORTED, "device ordinal beyond the scratch table");
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_l1_scratch);
+    if (e != cudaSuccess || !p)
+      return vs::set_last_error(VS_ERR_CUDA, e != cudaSuccess ? cudaGetErrorString(e)
+                                                              : "scratch address is NULL");
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return VS_OK;
+}
+
+}  // namespace
+
+extern "C" vs_status vs_l1_distance_static(int32_t rows, int32_t vocab, int64_t ld,
+                                           vs_dtype dtype, const void* draft, const void* target,
+                                           const float* row_weight, float* l1,
+                                           float* accept_rate, float* loss_num_den_loss,
+                                           void* grad_draft, vs_dtype grad_dtype, int64_t grad_ld,
+                                           void* stream) {
+  if (rows > VS_L1_STATIC_MAX_ROWS)
+    return vs::set_last_error(VS_ERR_UNSUPPORTED,
+                              "rows exceed VS_L1_STATIC_MAX_ROWS: use vs_l1_distance with a workspace");
+  void* scratch = nullptr;
+  const vs_status st = scratch_for_current_device(&scratch);
+  if (st != VS_OK) return st;
+  return vs_l1_distance(rows, vocab, ld, dtype, draft, target, row_weight, l1, accept_rate,
+                        loss_num_den_loss, grad_draft, grad_dtype, grad_ld, scratch,
+                        VS_L1_STATIC_SCRATCH_BYTES, stream);
+}
