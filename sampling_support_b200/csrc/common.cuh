@@ -29,18 +29,17 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // ---------------------------------------------------------------------------
-// monotone integer keys: key(a) < key(b)  <=>  a < b  for finite values, with
-// -0 mapped onto +0 so that equal values have equal keys.
+// monotone integer keys:  key(a) < key(b)  <=>  a < b  for finite values, and
+// key(-0) == key(+0).  For raw IEEE bits x of width W with sign bit S:
+//   negative x:      key = (2^W - 1) - x      (0 .. S - 1;  -0 -> S - 1)
+//   non-negative x:  key = x + (S - 1)        (S - 1 .. 2^W - 2; +0 -> S - 1)
 
 __device__ __forceinline__ uint32_t key_of(uint16_t raw) {
-  uint32_t x = raw;
-  if (x == 0x8000u) x = 0;
-  return (x & 0x8000u) ? (~x & 0xFFFFu) : (x | 0x8000u);
+  const uint32_t x = raw;
+  return (x & 0x8000u) ? (0xFFFFu - x) : (x + 0x7FFFu);
 }
 __device__ __forceinline__ uint32_t key_of(uint32_t raw) {
-  uint32_t x = raw;
-  if (x == 0x80000000u) x = 0;
-  return (x & 0x80000000u) ? ~x : (x | 0x80000000u);
+  return (raw & 0x80000000u) ? (0xFFFFFFFFu - raw) : (raw + 0x7FFFFFFFu);
 }
 __device__ __forceinline__ float value_of(uint16_t raw) {
   return __uint_as_float(static_cast<uint32_t>(raw) << 16);
@@ -52,18 +51,18 @@ struct KeyTraits;
 template <>
 struct KeyTraits<uint16_t> {
   static constexpr int kBits = 16;
-  static constexpr uint32_t kInfKey = 0xFF80u;  // key of +inf
+  static constexpr uint32_t kInfKey = 0x7F80u + 0x7FFFu;  // key of +inf
   __device__ static float decode(uint32_t k) {
-    uint32_t bits = (k & 0x8000u) ? (k & 0x7FFFu) : (~k & 0xFFFFu);
+    const uint32_t bits = k >= 0x7FFFu ? k - 0x7FFFu : 0xFFFFu - k;
     return __uint_as_float(bits << 16);
   }
 };
 template <>
 struct KeyTraits<uint32_t> {
   static constexpr int kBits = 32;
-  static constexpr uint32_t kInfKey = 0xFF800000u;
+  static constexpr uint32_t kInfKey = 0x7F800000u + 0x7FFFFFFFu;
   __device__ static float decode(uint32_t k) {
-    uint32_t bits = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+    const uint32_t bits = k >= 0x7FFFFFFFu ? k - 0x7FFFFFFFu : 0xFFFFFFFFu - k;
     return __uint_as_float(bits);
   }
 };
@@ -192,6 +191,41 @@ __device__ __forceinline__ T block_sum(T v, T* scratch) {
   for (int w = 0; w < nw; ++w) t += scratch[w];
   __syncthreads();
   return t;
+}
+
+// ---------------------------------------------------------------------------
+// packed fp32x2 arithmetic (sm_100a: add/sub/mul/fma.rn.f32x2), two lanes per
+// 64-bit register; each lane rounds exactly as the scalar instruction.
+
+typedef unsigned long long f32x2;
+
+__device__ __forceinline__ f32x2 pack2(float lo, float hi) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack2(f32x2 v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b) {
+  f32x2 r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+  f32x2 r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
+  f32x2 r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
 }
 
 // ---------------------------------------------------------------------------

@@ -89,17 +89,18 @@ __device__ __forceinline__ float ind_minus(float p, bool is_y, bool is_max, floa
   return is_max ? omp : 1.f - p;
 }
 
+// u is the raw logit value; row maxima in the saved state are raw values too.
 __device__ __forceinline__ float grad_elem(const RowCoef& k, float u, int j, bool in_s) {
   float dz = 0.f;
   const bool is_y = j == k.y;
   if (k.need_full) {
-    const float d = u - k.m2;
+    const float d = (u - k.m2) * k.c;
     const float lp2 = d - k.log2z;
     const float p = ex2(lp2);
     dz += k.gv * ind_minus(p, is_y, d == 0.f, k.omp_full) - k.ghv * p * fmaf(lp2, kLn2, k.h_full);
   }
   if (in_s && k.need_sup) {
-    const float d = u - k.msup;
+    const float d = (u - k.msup) * k.c;
     const float lq2 = d - k.log2zs;
     const float q = ex2(lq2);
     dz += k.gs * ind_minus(q, is_y, d == 0.f, k.omp_sup) - k.ghs * q * fmaf(lq2, kLn2, k.h_sup);
@@ -111,7 +112,7 @@ template <typename Raw, typename G, bool ACC>
 __global__ void __launch_bounds__(kThreads) score_bwd_kernel(BwdParams P, int nchunks) {
   constexpr int VEC = 16 / sizeof(Raw);
   extern __shared__ __align__(16) uint32_t bitmap[];  // recorded support bits of this slice
-  __shared__ Stats red[kThreads / 32];
+  __shared__ float fred[kThreads / 32];
   const int row = blockIdx.x / nchunks;
   const int part = blockIdx.x % nchunks;
   const int V = P.vocab;
@@ -127,23 +128,39 @@ __global__ void __launch_bounds__(kThreads) score_bwd_kernel(BwdParams P, int nc
   // full-vocabulary statistics missing from the forward (recorded support
   // without full statistics): this launch covers whole rows, compute them.
   if (k.need_full && !(k.flags & kCtxFullStats)) {
-    Stats s = stats_empty();
+    // maximum, then sums relative to it (value domain, as the forward)
     const int nfull = V / VEC;
     const uint4* g4 = reinterpret_cast<const uint4*>(grow);
+    float vm = -kInf;
     for (int v = threadIdx.x; v < nfull; v += blockDim.x) {
       Raw r[VEC];
       unpack(g4[v], r);
-      float u[VEC];
 #pragma unroll
-      for (int i = 0; i < VEC; ++i) u[i] = __fmul_rn(value_of(r[i]), k.c);
-      stats_add(s, u);
+      for (int i = 0; i < VEC; ++i) vm = fmaxf(vm, value_of(r[i]));
     }
-    for (int j = nfull * VEC + threadIdx.x; j < V; j += blockDim.x) {
-      float u[1] = {__fmul_rn(value_of(grow[j]), k.c)};
-      stats_add(s, u);
+    for (int j = nfull * VEC + threadIdx.x; j < V; j += blockDim.x) vm = fmaxf(vm, value_of(grow[j]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, o));
+    if ((threadIdx.x & 31) == 0) fred[threadIdx.x >> 5] = vm;
+    __syncthreads();
+    vm = -kInf;
+    for (int i = 0; i < kThreads / 32; ++i) vm = fmaxf(vm, fred[i]);
+    __syncthreads();
+    float c0 = 0.f, zr = 0.f, a = 0.f;
+    for (int j = threadIdx.x; j < V; j += blockDim.x) {
+      const float d = (value_of(grow[j]) - vm) * k.c;
+      const float e = ex2(d);
+      if (d == 0.f)
+        c0 += 1.f;
+      else
+        zr += e;
+      a = fmaf(d, e, a);
     }
-    s = block_reduce(s, red);
-    k.m2 = s.m;
+    c0 = block_sum(c0, fred);
+    zr = block_sum(zr, fred);
+    a = block_sum(a, fred);
+    const Stats s{vm, c0, zr, a};
+    k.m2 = vm;
     k.log2z = stats_log2z(s);
     k.h_full = kLn2 * (k.log2z - s.a / stats_z(s));
     k.omp_full = (s.c0 - 1.f + s.zr) / (s.c0 + s.zr);
@@ -179,8 +196,7 @@ __global__ void __launch_bounds__(kThreads) score_bwd_kernel(BwdParams P, int nc
 #pragma unroll
       for (int i = 0; i < VEC; ++i) {
         const int jl = v * VEC + i;
-        const float u = __fmul_rn(value_of(r[i]), k.c);
-        out[i] = grad_elem(k, u, c0 + jl, in_support(jl, r[i]));
+        out[i] = grad_elem(k, value_of(r[i]), c0 + jl, in_support(jl, r[i]));
       }
     } else {
 #pragma unroll
@@ -214,7 +230,7 @@ __global__ void __launch_bounds__(kThreads) score_bwd_kernel(BwdParams P, int nc
     const Raw raw = grow[c0 + jl];
     float g = 0.f;
     if (k.need_full || k.need_sup)
-      g = grad_elem(k, __fmul_rn(value_of(raw), k.c), c0 + jl, in_support(jl, raw));
+      g = grad_elem(k, value_of(raw), c0 + jl, in_support(jl, raw));
     G* dst = gout + c0 + jl;
     if (ACC) g += GradStore<G>::load(dst);
     GradStore<G>::store(dst, g);
@@ -242,7 +258,7 @@ __global__ void __launch_bounds__(kThreads) score_bwd_sparse_kernel(BwdParams P)
       if (!dup) {
         RowCoef ks = k;
         ks.need_full = false;  // full-vocabulary terms are not representable here
-        g = grad_elem(ks, __fmul_rn(value_of(grow[id]), k.c), id, true);
+        g = grad_elem(ks, value_of(grow[id]), id, true);
       }
     }
     gout[w] = g;

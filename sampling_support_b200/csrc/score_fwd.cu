@@ -16,6 +16,8 @@
 
 #include <climits>
 
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -207,7 +209,7 @@ __device__ void scan_bins(const uint32_t* gcnt, const u64* gmass, bool by_mass, 
 // from the first level's histogram.  `hb` selects the histogram buffer and
 // alternates per level, so one cluster barrier per level suffices.
 template <typename Raw>
-__device__ Desc descend(const Raw* buf, int n, float c, float m2, int fx_shift, bool by_mass,
+__device__ Desc descend(const Raw* buf, int n, float c, float vmax, int fx_shift, bool by_mass,
                         bool need_mass, u64 target, float p, SelShared& sh, RadixArrays& ra,
                         cg::cluster_group& cluster, int& hb) {
   constexpr int KB = KeyTraits<Raw>::kBits;
@@ -233,7 +235,7 @@ __device__ Desc descend(const Raw* buf, int n, float c, float m2, int fx_shift, 
         const uint32_t digit = (key >> shift) & 255u;
         atomicAdd(&cnt[digit], 1u);
         if (need_mass) {
-          const float e = ex2(__fmul_rn(value_of(raw), c) - m2);
+          const float e = ex2((value_of(raw) - vmax) * c);
           const u64 fx = __float2ull_rn(e * fxs);
           if (fx) atomicAdd(&mass[digit], fx);
         }
@@ -305,30 +307,24 @@ struct Window {
   int S;          // bins per CTA slice
   uint32_t* hist;  // this CTA's unreduced histogram [kWin]
   uint32_t* red;   // this CTA's reduced slice [S]
-  float c, m2, fxs;
+  float c, vmax, fxs;
 };
 
+// Fixed-point mass 2^((v - vmax) c) * 2^fx_shift of one element of a bin.
 __device__ __forceinline__ u64 bin_fx(const Window& w, uint32_t key) {
-  const float e = ex2(__fmul_rn(KeyTraits<uint16_t>::decode(key), w.c) - w.m2);
+  const float e = ex2((KeyTraits<uint16_t>::decode(key) - w.vmax) * w.c);
   return __float2ull_rn(e * w.fxs);
 }
 
-// Build the window histogram, reduce it across the cluster and gather the
-// per-slice totals (count and fixed-point mass) into every CTA.
-__device__ void window_build(const uint16_t* buf, int n, Window& w, SelShared& sh,
-                             cg::cluster_group& cluster) {
+// Reduce the (already filled) window histograms across the cluster, CTA r
+// keeping bins [r S, r S + S), and gather the per-slice totals (count and
+// fixed-point mass) into every CTA.  The caller has passed a cluster barrier
+// since the histograms were filled.
+__device__ void window_reduce(Window& w, SelShared& sh, cg::cluster_group& cluster) {
   const uint32_t CL = cluster.num_blocks();
   const uint32_t rank = cluster.block_rank();
-  for (int b = threadIdx.x; b < kWin; b += blockDim.x) w.hist[b] = 0u;
-  __syncthreads();
   const uint32_t klo = w.klo;
   uint32_t* hist = w.hist;
-  for_each(buf, n, [&](int, uint16_t raw) {
-    const uint32_t key = key_of(raw);
-    if (key >= klo) atomicAdd(&hist[key - klo], 1u);
-  });
-  __syncthreads();
-  cluster.sync();
   const int b0 = static_cast<int>(rank) * w.S;
   const int b1 = min(kWin, b0 + w.S);
   u64 tc = 0, tm = 0;
@@ -430,9 +426,152 @@ __device__ __forceinline__ u64 topp_target(float p, double mass) {
   return static_cast<u64>(want);
 }
 
+// Window mode of the fused pass (bf16): how an element's bin is derived.
+enum WinMode : int {
+  kWinNone = 0,  // no histogram
+  kWinPos = 1,   // window within positive values: bin = (F - Fconst) >> 16 on raw float bits
+  kWinNeg = 2,   // window within negative values: bin = (Fconst - F) >> 16
+  kWinKey = 3,   // general: bin = key - klo
+};
+
+// Sums of a slice relative to the known row maximum vmax (base 2, d =
+// (v - vmax) c <= 0): count of elements equal to vmax, the sum of 2^d over the
+// others, and the sum of d 2^d.
+struct FSums {
+  float c0, zr, a;
+};
+
+// One element of the fused pass.  kTop: the element's vector holds the row
+// maximum, so elements with d == 0 are counted apart (exactly 1 each).
+template <bool kTop>
+__device__ __forceinline__ void fused_elem(float x, float vmax, float c, FSums& s) {
+  const float d = (x - vmax) * c;
+  const float e = ex2(d);
+  if (kTop && d == 0.f)
+    s.c0 += 1.f;
+  else
+    s.zr += e;
+  s.a = fmaf(d, e, s.a);
+}
+
+template <int kMode>
+__device__ __forceinline__ void win_count(uint32_t F, uint32_t fconst, uint32_t klo,
+                                          uint32_t* hist) {
+  if constexpr (kMode == kWinPos) {
+    const uint32_t b = F - fconst;
+    if (b < (static_cast<uint32_t>(kWin) << 16)) atomicAdd(&hist[b >> 16], 1u);
+  } else if constexpr (kMode == kWinNeg) {
+    const uint32_t b = fconst - F;
+    if (b < (static_cast<uint32_t>(kWin) << 16)) atomicAdd(&hist[b >> 16], 1u);
+  } else if constexpr (kMode == kWinKey) {
+    const uint32_t b = key_of(static_cast<uint16_t>(F >> 16)) - klo;
+    if (b < static_cast<uint32_t>(kWin)) atomicAdd(&hist[b], 1u);
+  }
+}
+
+// Fused pass over a bf16 slice: statistics relative to vmax and, when
+// kMode != kWinNone, the exact-key window histogram.
+template <int kMode>
+__device__ void fused_pass_bf16(const uint16_t* buf, int n, float vmax, float c, uint32_t fconst,
+                                uint32_t klo, uint32_t* hist, FSums& s) {
+  const int nfull = n / 8;
+  const uint4* v4 = reinterpret_cast<const uint4*>(buf);
+  const f32x2 vm2 = pack2(vmax, vmax), c2 = pack2(c, c);
+  f32x2 zr2 = pack2(0.f, 0.f), a2 = pack2(0.f, 0.f);
+  for (int v = threadIdx.x; v < nfull; v += blockDim.x) {
+    const uint4 q = v4[v];
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    // does this vector hold the row maximum?  (packed max, rare)
+    __nv_bfloat162 m01 = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&w[0]),
+                                 *reinterpret_cast<const __nv_bfloat162*>(&w[1]));
+    __nv_bfloat162 m23 = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&w[2]),
+                                 *reinterpret_cast<const __nv_bfloat162*>(&w[3]));
+    const __nv_bfloat162 mm = __hmax2(m01, m23);
+    const bool top = fmaxf(__low2float(mm), __high2float(mm)) == vmax;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t F0 = w[i] << 16, F1 = w[i] & 0xFFFF0000u;
+      if (top) {
+        fused_elem<true>(__uint_as_float(F0), vmax, c, s);
+        fused_elem<true>(__uint_as_float(F1), vmax, c, s);
+      } else {
+        // both elements at once: d = (x - vmax) c, e = 2^d, zr += e, a += d e
+        const f32x2 d2 = mul2(sub2(pack2(__uint_as_float(F0), __uint_as_float(F1)), vm2), c2);
+        float d0, d1;
+        unpack2(d2, d0, d1);
+        const f32x2 e2 = pack2(ex2(d0), ex2(d1));
+        zr2 = add2(zr2, e2);
+        a2 = fma2(d2, e2, a2);
+      }
+      win_count<kMode>(F0, fconst, klo, hist);
+      win_count<kMode>(F1, fconst, klo, hist);
+    }
+  }
+  {
+    float z0, z1, a0, a1;
+    unpack2(zr2, z0, z1);
+    unpack2(a2, a0, a1);
+    s.zr += z0 + z1;
+    s.a += a0 + a1;
+  }
+  for (int j = nfull * 8 + threadIdx.x; j < n; j += blockDim.x) {
+    const uint32_t F = static_cast<uint32_t>(buf[j]) << 16;
+    fused_elem<true>(__uint_as_float(F), vmax, c, s);
+    win_count<kMode>(F, fconst, klo, hist);
+  }
+}
+
+// Statistics pass over an fp32 slice relative to vmax.
+__device__ void fused_pass_f32(const uint32_t* buf, int n, float vmax, float c, FSums& s) {
+  const int nfull = n / 4;
+  const uint4* v4 = reinterpret_cast<const uint4*>(buf);
+  for (int v = threadIdx.x; v < nfull; v += blockDim.x) {
+    const uint4 q = v4[v];
+    const float x[4] = {__uint_as_float(q.x), __uint_as_float(q.y), __uint_as_float(q.z),
+                        __uint_as_float(q.w)};
+    const float bm = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+    if (bm == vmax) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) fused_elem<true>(x[i], vmax, c, s);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) fused_elem<false>(x[i], vmax, c, s);
+    }
+  }
+  for (int j = nfull * 4 + threadIdx.x; j < n; j += blockDim.x)
+    fused_elem<true>(__uint_as_float(buf[j]), vmax, c, s);
+}
+
+// Largest value of a slice (NaN ignored).
 template <typename Raw>
-__global__ void __launch_bounds__(kThreads, 3) score_computed_kernel(ScoreParams P) {
-  constexpr int VEC = 16 / sizeof(Raw);
+__device__ float slice_max(const Raw* buf, int n) {
+  float m = -kInf;
+  if constexpr (sizeof(Raw) == 2) {
+    const int nfull = n / 8;
+    const uint4* v4 = reinterpret_cast<const uint4*>(buf);
+    __nv_bfloat162 acc = __float2bfloat162_rn(-kInf);
+    for (int v = threadIdx.x; v < nfull; v += blockDim.x) {
+      const uint4 q = v4[v];
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
+      acc = __hmax2(acc, __hmax2(__hmax2(h[0], h[1]), __hmax2(h[2], h[3])));
+    }
+    m = fmaxf(__low2float(acc), __high2float(acc));
+    for (int j = nfull * 8 + threadIdx.x; j < n; j += blockDim.x) m = fmaxf(m, value_of(buf[j]));
+  } else {
+    const int nfull = n / 4;
+    const uint4* v4 = reinterpret_cast<const uint4*>(buf);
+    for (int v = threadIdx.x; v < nfull; v += blockDim.x) {
+      const uint4 q = v4[v];
+      m = fmaxf(m, fmaxf(fmaxf(__uint_as_float(q.x), __uint_as_float(q.y)),
+                         fmaxf(__uint_as_float(q.z), __uint_as_float(q.w))));
+    }
+    for (int j = nfull * 4 + threadIdx.x; j < n; j += blockDim.x) m = fmaxf(m, value_of(buf[j]));
+  }
+  return m;
+}
+
+template <typename Raw>
+__global__ void __launch_bounds__(kThreads, 2) score_computed_kernel(ScoreParams P) {
   constexpr bool kBf16 = sizeof(Raw) == 2;
   using KT = KeyTraits<Raw>;
   cg::cluster_group cluster = cg::this_cluster();
@@ -472,70 +611,99 @@ __global__ void __launch_bounds__(kThreads, 3) score_computed_kernel(ScoreParams
   }
   __syncthreads();
 
-  // ---- pass 1: online max / sum / entropy sum over the slice (and the max value)
   const float T = P.temperature ? P.temperature[row] : P.temperature_scalar;
   const float c = kLog2e / T;
-  Stats s = stats_empty();
-  float vmax = -kInf;
-  {
-    const int nfull = n / VEC;
-    const uint4* v4 = reinterpret_cast<const uint4*>(buf);
-    for (int v = tid; v < nfull; v += blockDim.x) {
-      Raw r[VEC];
-      unpack(v4[v], r);
-      float u[VEC];
-#pragma unroll
-      for (int i = 0; i < VEC; ++i) {
-        const float x = value_of(r[i]);
-        vmax = fmaxf(vmax, x);
-        u[i] = __fmul_rn(x, c);
-      }
-      stats_add(s, u);
-    }
-    for (int j = nfull * VEC + tid; j < n; j += blockDim.x) {
-      const float x = value_of(buf[j]);
-      vmax = fmaxf(vmax, x);
-      float u[1] = {__fmul_rn(x, c)};
-      stats_add(s, u);
-    }
-  }
-  s = block_reduce(s, sh.red);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-  if ((tid & 31) == 0) sh.fred[tid >> 5] = vmax;
-  __syncthreads();
-  if (tid == 0) {
-    float vm = -kInf;
-    for (int w = 0; w < kWarps; ++w) vm = fmaxf(vm, sh.fred[w]);
-    sh.part = s;
-    sh.vmax_part = vm;
-  }
-  cluster.sync();
-  if (tid < static_cast<int>(CL)) {
-    const SelShared* rsh = cluster.map_shared_rank(&sh, tid);
-    sh.gathered[tid] = rsh->part;
-    sh.vmax_g[tid] = rsh->vmax_part;
-  }
-  __syncthreads();
-  Stats rs = stats_empty();
-  float vmax_row = -kInf;
-  for (uint32_t r = 0; r < CL; ++r) {
-    stats_merge(rs, sh.gathered[r]);
-    vmax_row = fmaxf(vmax_row, sh.vmax_g[r]);
-  }
-
-  const bool nonfinite = !stats_finite(rs);
-  const float m2 = rs.m;
-  const float log2z = stats_log2z(rs);
-  const float h_full = kLn2 * (log2z - rs.a / stats_z(rs));
-
   const int kk = P.top_k ? P.top_k[row] : P.top_k_scalar;
   const float pp = P.top_p ? P.top_p[row] : P.top_p_scalar;
   const float mp = P.min_p ? P.min_p[row] : P.min_p_scalar;
   const bool use_k = kk > 0 && kk < V;
   const bool use_p = pp < 1.f;
   const bool use_minp = mp > 0.f;
-  const bool filtered = !nonfinite && (use_k || use_p || use_minp);
+  const bool any_filter = use_k || use_p || use_minp;
+
+  // ---- pass 0: row maximum (cluster-wide, rank order)
+  {
+    float vm = slice_max(buf, n);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, o));
+    if ((tid & 31) == 0) sh.fred[tid >> 5] = vm;
+    __syncthreads();
+    if (tid == 0) {
+      float m = -kInf;
+      for (int w = 0; w < kWarps; ++w) m = fmaxf(m, sh.fred[w]);
+      sh.vmax_part = m;
+    }
+  }
+  cluster.sync();
+  if (tid < static_cast<int>(CL)) sh.vmax_g[tid] = cluster.map_shared_rank(&sh, tid)->vmax_part;
+  __syncthreads();
+  float vmax = -kInf;
+  for (uint32_t r = 0; r < CL; ++r) vmax = fmaxf(vmax, sh.vmax_g[r]);
+
+  // ---- window geometry (bf16 with a filter): exact keys kmax - kWin + 1 .. kmax
+  Window w{};
+  int wmode = kWinNone;
+  if constexpr (kBf16) {
+    if (any_filter && isfinite(vmax)) {
+      const uint32_t hmax = __float_as_uint(vmax) >> 16;
+      w.kmax = key_of(static_cast<uint16_t>(hmax));
+      w.klo = w.kmax >= static_cast<uint32_t>(kWin - 1) ? w.kmax - (kWin - 1) : 0u;
+      w.S = (kWin + CL - 1) / CL;
+      w.hist = reinterpret_cast<uint32_t*>(big);
+      w.red = w.hist + kWin;
+      w.c = c;
+      w.vmax = vmax;
+      w.fxs = fx_scale(P.fx_shift);
+      if (!(hmax & 0x8000u) && hmax >= static_cast<uint32_t>(kWin))
+        wmode = kWinPos;  // lowest window value > +0
+      else if ((hmax & 0x8000u) && hmax != 0x8000u && hmax <= 0xFFFFu - (kWin - 1))
+        wmode = kWinNeg;  // vmax < 0: every value is negative
+      else
+        wmode = kWinKey;
+      for (int b = tid; b < kWin; b += blockDim.x) w.hist[b] = 0u;
+      __syncthreads();
+    }
+  }
+
+  // ---- pass 1 (fused): sums relative to vmax (+ window histogram)
+  FSums fs{0.f, 0.f, 0.f};
+  if constexpr (kBf16) {
+    const uint32_t hmax = __float_as_uint(vmax) >> 16;
+    switch (wmode) {
+      case kWinPos:
+        fused_pass_bf16<kWinPos>(buf, n, vmax, c, (hmax - (kWin - 1)) << 16, 0u, w.hist, fs);
+        break;
+      case kWinNeg:
+        fused_pass_bf16<kWinNeg>(buf, n, vmax, c, (hmax + (kWin - 1)) << 16, 0u, w.hist, fs);
+        break;
+      case kWinKey:
+        fused_pass_bf16<kWinKey>(buf, n, vmax, c, 0u, w.klo, w.hist, fs);
+        break;
+      default:
+        fused_pass_bf16<kWinNone>(buf, n, vmax, c, 0u, 0u, nullptr, fs);
+        break;
+    }
+  } else {
+    fused_pass_f32(reinterpret_cast<const uint32_t*>(buf), n, vmax, c, fs);
+  }
+  fs.c0 = block_sum(fs.c0, sh.fred);
+  fs.zr = block_sum(fs.zr, sh.fred);
+  fs.a = block_sum(fs.a, sh.fred);
+  if (tid == 0) sh.part = Stats{vmax, fs.c0, fs.zr, fs.a};
+  cluster.sync();  // sums and window histograms complete everywhere
+  if (tid < static_cast<int>(CL)) sh.gathered[tid] = cluster.map_shared_rank(&sh, tid)->part;
+  __syncthreads();
+  Stats rs{vmax, 0.f, 0.f, 0.f};
+  for (uint32_t r = 0; r < CL; ++r) {
+    rs.c0 += sh.gathered[r].c0;
+    rs.zr += sh.gathered[r].zr;
+    rs.a += sh.gathered[r].a;
+  }
+
+  const bool nonfinite = !(isfinite(vmax) && isfinite(rs.zr) && isfinite(rs.a) && rs.c0 >= 1.f);
+  const float log2z = stats_log2z(rs);
+  const float h_full = kLn2 * (log2z - rs.a / stats_z(rs));
+  const bool filtered = !nonfinite && any_filter;
 
   uint32_t tkey = 0;
   int32_t tie_cut = INT_MAX;
@@ -554,21 +722,12 @@ __global__ void __launch_bounds__(kThreads, 3) score_computed_kernel(ScoreParams
     uint32_t eq_rank[8];
     const float fxs = fx_scale(P.fx_shift);
 
-    // ---- exact-key window select (bf16 keys with top-k and/or top-p)
+    // ---- exact-key window select (bf16)
     bool win_ok = false;
-    Window w{};
     if constexpr (kBf16) {
+      window_reduce(w, sh, cluster);
+      win_ok = true;
       if (use_k || use_p) {
-        w.kmax = key_of(static_cast<uint16_t>(__float_as_uint(vmax_row) >> 16));
-        w.klo = w.kmax >= static_cast<uint32_t>(kWin - 1) ? w.kmax - (kWin - 1) : 0u;
-        w.S = (kWin + CL - 1) / CL;
-        w.hist = reinterpret_cast<uint32_t*>(big);
-        w.red = w.hist + kWin;
-        w.c = c;
-        w.m2 = m2;
-        w.fxs = fxs;
-        window_build(buf, n, w, sh, cluster);
-        win_ok = true;
         Desc dk{}, dp{};
         u64 ck = 0;
         if (use_k) {
@@ -613,8 +772,8 @@ __global__ void __launch_bounds__(kThreads, 3) score_computed_kernel(ScoreParams
       have_t = false;
       all_ties = true;
       if (use_k) {
-        Desc d = descend(buf, n, c, m2, P.fx_shift, false, use_p, static_cast<u64>(kk), 1.f, sh,
-                         ra, cluster, hb);
+        Desc d = descend(buf, n, c, vmax, P.fx_shift, false, use_p, static_cast<u64>(kk), 1.f,
+                         sh, ra, cluster, hb);
         const u64 ck = static_cast<u64>(kk) - d.above_cnt;
         tkey = d.key;
         cnum = ck;
@@ -623,7 +782,7 @@ __global__ void __launch_bounds__(kThreads, 3) score_computed_kernel(ScoreParams
         if (use_p) {
           const u64 fx_t = d.at_cnt ? d.at_mass / d.at_cnt : 0;
           const u64 tp = topp_target(pp, static_cast<double>(d.above_mass + ck * fx_t));
-          Desc e = descend(buf, n, c, m2, P.fx_shift, true, true, tp, pp, sh, ra, cluster, hb);
+          Desc e = descend(buf, n, c, vmax, P.fx_shift, true, true, tp, pp, sh, ra, cluster, hb);
           const u64 fxe = e.at_cnt ? e.at_mass / e.at_cnt : 0;
           const u64 need = tp > e.above_mass ? tp - e.above_mass : 0;
           u64 cp = fxe ? (need + fxe - 1) / fxe : e.at_cnt;
@@ -635,7 +794,7 @@ __global__ void __launch_bounds__(kThreads, 3) score_computed_kernel(ScoreParams
           all_ties = cp >= e.at_cnt;
         }
       } else {
-        Desc e = descend(buf, n, c, m2, P.fx_shift, true, true, 0ull, pp, sh, ra, cluster, hb);
+        Desc e = descend(buf, n, c, vmax, P.fx_shift, true, true, 0ull, pp, sh, ra, cluster, hb);
         const u64 tp = sh.b_target;
         const u64 fxe = e.at_cnt ? e.at_mass / e.at_cnt : 0;
         const u64 need = tp > e.above_mass ? tp - e.above_mass : 0;
@@ -654,7 +813,7 @@ __global__ void __launch_bounds__(kThreads, 3) score_computed_kernel(ScoreParams
       uint32_t lo = 0, hi = KT::kInfKey;
       while (lo < hi) {
         const uint32_t mid = lo + ((hi - lo) >> 1);
-        const float r = ex2(__fmul_rn(KT::decode(mid), c) - m2);
+        const float r = ex2((KT::decode(mid) - vmax) * c);
         if (r >= mp)
           hi = mid;
         else
@@ -680,7 +839,7 @@ __global__ void __launch_bounds__(kThreads, 3) score_computed_kernel(ScoreParams
           const uint32_t cnt = w.red[b - b0];
           const uint32_t key = w.klo + b;
           if (cnt && key > tkey) {
-            const float d = __fmul_rn(KT::decode(key), c) - m2;
+            const float d = (KT::decode(key) - vmax) * c;
             const float e = ex2(d);
             const float fc = static_cast<float>(cnt);
             ngt += cnt;
@@ -700,7 +859,7 @@ __global__ void __launch_bounds__(kThreads, 3) score_computed_kernel(ScoreParams
       for_each(buf, n, [&](int, Raw raw) {
         const uint32_t key = key_of(raw);
         if (key > t) {
-          const float d = __fmul_rn(value_of(raw), c) - m2;
+          const float d = (value_of(raw) - vmax) * c;
           const float e = ex2(d);
           ++ngt;
           if (d == 0.f)
@@ -736,10 +895,10 @@ __global__ void __launch_bounds__(kThreads, 3) score_computed_kernel(ScoreParams
       tot_a += rsh->agg_a;
     }
     const u64 ckeep = all_ties ? tot_eq : (cnum < tot_eq ? cnum : tot_eq);
-    const float dt = __fmul_rn(KT::decode(tkey), c) - m2;
+    const float dt = (KT::decode(tkey) - vmax) * c;
     const float et = ex2(dt);
     Stats ss;
-    ss.m = m2;
+    ss.m = vmax;
     ss.c0 = static_cast<float>(tot_top) + (dt == 0.f ? static_cast<float>(ckeep) : 0.f);
     ss.zr = tot_mass + (dt == 0.f ? 0.f : static_cast<float>(ckeep) * et);
     ss.a = tot_a + static_cast<float>(ckeep) * dt * et;
@@ -761,46 +920,35 @@ __global__ void __launch_bounds__(kThreads, 3) score_computed_kernel(ScoreParams
         off += eq_rank[r];
       }
       if (rank == owner) {
+        // each thread owns a contiguous id range of the slice: count its ties,
+        // one exclusive scan over threads, then the thread holding the
+        // need-th tie walks its range again to find it
         const int need = static_cast<int>(ckeep - off);
-        int base_count = 0;
         const uint32_t t = tkey;
+        const int per = (n + kThreads - 1) / kThreads;
+        const int j0 = tid * per, j1 = min(n, j0 + per);
+        int mine = 0;
+        for (int j = j0; j < j1; ++j) mine += key_of(buf[j]) == t;
         const int lane = tid & 31, warp = tid >> 5;
-        for (int base = 0; base < n; base += kThreads * VEC) {
-          const int j0 = base + tid * VEC;
-          int mine = 0;
+        int incl = mine;
 #pragma unroll
-          for (int i = 0; i < VEC; ++i) {
-            const int j = j0 + i;
-            if (j < n && key_of(buf[j]) == t) ++mine;
-          }
-          int incl = mine;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int x = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += x;
-          }
-          if (lane == 31) sh.scan_tot[warp] = incl;
-          __syncthreads();
-          int wpre = 0, total = 0;
-          for (int ww = 0; ww < kWarps; ++ww) {
-            if (ww < warp) wpre += sh.scan_tot[ww];
-            total += sh.scan_tot[ww];
-          }
-          const int excl = base_count + wpre + incl - mine;
-          if (excl < need && need <= excl + mine) {
-            int cn = excl;
-#pragma unroll
-            for (int i = 0; i < VEC; ++i) {
-              const int j = j0 + i;
-              if (j < n && key_of(buf[j]) == t) {
-                ++cn;
-                if (cn == need) sh.tie_cut = c0 + j;
-              }
+        for (int o = 1; o < 32; o <<= 1) {
+          const int x = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += x;
+        }
+        if (lane == 31) sh.scan_tot[warp] = incl;
+        __syncthreads();
+        int wpre = 0;
+        for (int ww = 0; ww < warp; ++ww) wpre += sh.scan_tot[ww];
+        const int excl = wpre + incl - mine;
+        if (excl < need && need <= excl + mine) {
+          int cn = excl;
+          for (int j = j0; j < j1; ++j) {
+            if (key_of(buf[j]) == t && ++cn == need) {
+              sh.tie_cut = c0 + j;
+              break;
             }
           }
-          base_count += total;
-          __syncthreads();
-          if (base_count >= need) break;
         }
       }
       cluster.sync();
@@ -822,8 +970,8 @@ __global__ void __launch_bounds__(kThreads, 3) score_computed_kernel(ScoreParams
       status |= VS_ROW_NONFINITE_INPUT;
     } else if (target_ok) {
       const Raw ry = grow[y];
-      const float uy = __fmul_rn(value_of(ry), c);
-      lp_v = kLn2 * (uy - m2 - log2z);
+      const float dy = (value_of(ry) - vmax) * c;
+      lp_v = kLn2 * (dy - log2z);
       if (!filtered) {
         in_s = true;
       } else {
@@ -831,7 +979,7 @@ __global__ void __launch_bounds__(kThreads, 3) score_computed_kernel(ScoreParams
         in_s = ky > tkey || (ky == tkey && y <= tie_cut);
       }
       if (in_s) {
-        lp_s = filtered ? kLn2 * (uy - m2 - log2zs) : lp_v;
+        lp_s = filtered ? kLn2 * (dy - log2zs) : lp_v;
       } else {
         lp_s = -kInf;
         status |= VS_ROW_TARGET_NOT_IN_SUPPORT;
@@ -850,9 +998,9 @@ __global__ void __launch_bounds__(kThreads, 3) score_computed_kernel(ScoreParams
     if (P.support_size) P.support_size[row] = n_support;
     if (P.ctx) {
       RowCtx cx{};
-      cx.m2 = m2;
+      cx.m2 = vmax;
       cx.log2z = log2z;
-      cx.msup = m2;
+      cx.msup = vmax;
       cx.log2zs = log2zs;
       cx.h_full = h_full;
       cx.h_support = h_support;
@@ -913,8 +1061,10 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
   const int V = P.vocab;
   const int W = P.support_width;
   __shared__ int32_t ids[VS_MAX_SUPPORT_WIDTH];
+  __shared__ float vals[VS_MAX_SUPPORT_WIDTH];  // kept support values, NaN elsewhere
   __shared__ Stats red[kRecThreads / 32];
   __shared__ uint32_t ured[kRecThreads / 32];
+  __shared__ float fred[kRecThreads / 32];
   __shared__ uint32_t flags_sh;
   __shared__ int32_t target_hit;
 
@@ -932,13 +1082,14 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
   for (int w = tid; w < W; w += blockDim.x) ids[w] = srow[w];
   __syncthreads();
 
-  // keep[w]: id valid and first occurrence
+  // kept: id valid and first occurrence; gather the kept values
   uint32_t local_flags = 0;
-  Stats s = stats_empty();
   uint32_t nkeep = 0;
   bool nonfinite_sup = false;
+  float lmax = -kInf;
   for (int w = tid; w < W; w += blockDim.x) {
     const int32_t id = ids[w];
+    vals[w] = __int_as_float(0x7fc00000);
     if (id == -1) continue;
     if (id < -1 || id >= V) {
       local_flags |= VS_ROW_BAD_SUPPORT_ID;
@@ -955,21 +1106,44 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
       continue;
     }
     ++nkeep;
-    const float u = __fmul_rn(value_of(grow[id]), c);
-    if (!isfinite(u)) nonfinite_sup = true;
-    float uu[1] = {u};
-    stats_add(s, uu);
+    const float x = value_of(grow[id]);
+    if (!isfinite(x)) nonfinite_sup = true;
+    vals[w] = x;
+    lmax = fmaxf(lmax, x);
     if (id == y) target_hit = 1;
   }
   if (local_flags) atomicOr(&flags_sh, local_flags);
-  s = block_reduce(s, red);
   nkeep = block_sum(nkeep, ured);
   const uint32_t any_nf = block_sum(static_cast<uint32_t>(nonfinite_sup), ured);
   const bool empty = nkeep == 0;
+  // support statistics relative to the support maximum (value domain)
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+  if ((tid & 31) == 0) fred[tid >> 5] = lmax;
+  __syncthreads();
+  float vsmax = -kInf;
+  for (int i = 0; i < kRecThreads / 32; ++i) vsmax = fmaxf(vsmax, fred[i]);
+  __syncthreads();
+  Stats s{vsmax, 0.f, 0.f, 0.f};
+  for (int w = tid; w < W; w += blockDim.x) {
+    const float x = vals[w];
+    if (x != x) continue;  // not kept
+    const float d = (x - vsmax) * c;
+    const float e = ex2(d);
+    if (d == 0.f)
+      s.c0 += 1.f;
+    else
+      s.zr += e;
+    s.a = fmaf(d, e, s.a);
+  }
+  s.c0 = block_sum(s.c0, fred);
+  s.zr = block_sum(s.zr, fred);
+  s.a = block_sum(s.a, fred);
 
   // full-vocabulary statistics: for empty rows (fallback) or on request
   const bool need_full = empty || P.full_stats;
   Stats f = stats_empty();
+  float fvmax = -kInf;  // value-domain maximum of the row
   if (need_full) {
     const int nfull = V / VEC;
     const uint4* g4 = reinterpret_cast<const uint4*>(grow);
@@ -984,7 +1158,11 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
         unpack(q[k], r);
         float u[VEC];
 #pragma unroll
-        for (int i = 0; i < VEC; ++i) u[i] = __fmul_rn(value_of(r[i]), c);
+        for (int i = 0; i < VEC; ++i) {
+          const float x = value_of(r[i]);
+          fvmax = fmaxf(fvmax, x);
+          u[i] = __fmul_rn(x, c);
+        }
         stats_add(f, u);
       }
     }
@@ -993,14 +1171,26 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
       unpack(__ldcs(g4 + v), r);
       float u[VEC];
 #pragma unroll
-      for (int i = 0; i < VEC; ++i) u[i] = __fmul_rn(value_of(r[i]), c);
+      for (int i = 0; i < VEC; ++i) {
+        const float x = value_of(r[i]);
+        fvmax = fmaxf(fvmax, x);
+        u[i] = __fmul_rn(x, c);
+      }
       stats_add(f, u);
     }
     for (int j = nfull * VEC + tid; j < V; j += kRecThreads) {
-      float u[1] = {__fmul_rn(value_of(grow[j]), c)};
+      const float x = value_of(grow[j]);
+      fvmax = fmaxf(fvmax, x);
+      float u[1] = {__fmul_rn(x, c)};
       stats_add(f, u);
     }
     f = block_reduce(f, red);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) fvmax = fmaxf(fvmax, __shfl_xor_sync(0xffffffffu, fvmax, o));
+    if ((tid & 31) == 0) fred[tid >> 5] = fvmax;
+    __syncthreads();
+    fvmax = -kInf;
+    for (int i = 0; i < kRecThreads / 32; ++i) fvmax = fmaxf(fvmax, fred[i]);
   }
 
   if (tid == 0) {
@@ -1014,7 +1204,7 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
       log2z = stats_log2z(f);
       h_full = kLn2 * (log2z - f.a / stats_z(f));
     }
-    const float msup = s.m;
+    const float msup = vsmax;
     const float log2zs = empty ? nan : stats_log2z(s);
     const float h_sup = empty ? 0.f : kLn2 * (log2zs - s.a / stats_z(s));
     float lp_v = nan, lp_s = nan;
@@ -1029,7 +1219,7 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
       if (empty) {
         lp_s = lp_v;
       } else if (in_s) {
-        lp_s = kLn2 * (uy - msup - log2zs);
+        lp_s = kLn2 * ((value_of(grow[y]) - msup) * c - log2zs);
       } else {
         lp_s = -kInf;
         status |= VS_ROW_TARGET_NOT_IN_SUPPORT;
@@ -1047,7 +1237,7 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
     if (P.support_size) P.support_size[row] = nonfinite ? 0 : static_cast<int32_t>(nkeep);
     if (P.ctx) {
       RowCtx cx{};
-      cx.m2 = m2;
+      cx.m2 = fvmax;  // value domain (the stream's sums are relative to fl(fvmax c))
       cx.log2z = log2z;
       cx.msup = msup;
       cx.log2zs = log2zs;
@@ -1134,11 +1324,12 @@ int score_max_vocab(vs_dtype dtype) {
 }
 
 // Cluster size and per-CTA slice (elements, multiple of 32) for a row of
-// `vocab` elements: the smallest cluster whose slices fit a 40 KB budget, so
-// several CTAs share an SM; larger rows grow the slice up to 96 KB.
+// `vocab` elements: the smallest cluster whose slices fit an 80 KB budget
+// (two CTAs per SM; small clusters pack the GPCs densely); larger rows grow
+// the slice up to 96 KB.
 int score_cluster_size(int vocab, vs_dtype dtype, int* chunk) {
   const int esize = dtype == VS_BF16 ? 2 : 4;
-  const int target = 40 * 1024 / esize;
+  const int target = 80 * 1024 / esize;
   int cl = 1;
   while (cl < 8 && (vocab + cl - 1) / cl > target) ++cl;
   int e = (vocab + cl - 1) / cl;
