@@ -379,6 +379,29 @@ def secondary(args, pk):
                      "fwd_bytes_est": fbytes, "bwd_bytes": wbytes}
     del lg, dlog, holder
     torch.cuda.empty_cache()
+
+    # fused LM head: 8192 x 4096 hidden, 151,936 x 4096 weight, top-20 -> top-p -> min-p
+    w = workloads.lmhead()
+    hs, wt = to_dev(w["hidden_states"]), to_dev(w["weight"])
+    tg = to_dev(w["targets"])
+    lm = vsb.load()
+    nbytes = lm.vs_fused_lmhead_workspace_size(w["rows"], w["vocab"], w["hidden"], w["top_k"])
+    wsp = torch.empty(nbytes + 16, dtype=torch.uint8, device="cuda")
+
+    def lm_step():
+        vsb.fused_lmhead_score(hs, wt, tg, w["temperature"], w["top_k"],
+                               float(np.float32(w["top_p"])), float(np.float32(w["min_p"])),
+                               workspace=wsp)
+
+    ms = time_steps(lm_step, 2, max(3, min(steps, 10)))
+    flops = 2.0 * w["rows"] * w["vocab"] * w["hidden"]
+    tf = flops / (ms / 1e3) / 1e12
+    out["lmhead"] = {"rows": w["rows"], "vocab": w["vocab"], "hidden": w["hidden"],
+                     "ms_per_step": ms, "rows_per_s": w["rows"] / (ms / 1e3), "tflops": tf,
+                     "frac_bf16_burst": tf / pk["bf16"], "frac_bf16_sustained": tf / pk["bf16_sustained"],
+                     "flops": flops}
+    del hs, wt, wsp
+    torch.cuda.empty_cache()
     return out
 
 

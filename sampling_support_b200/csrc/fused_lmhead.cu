@@ -1,13 +1,635 @@
-// Fused LM-head scoring (placeholder until the tensor-core kernel lands).
+// Fused LM-head scoring (xorl issue #71, section 1: chunked projection ->
+// fixed-order LSE -> support -> selected logprob; SkyRL PR #2004,
+// "Performance": the full-vocabulary logits are never materialised).
+//
+//   z[i, v] = (sum_k H[i, k] W[v, k]) / T_i
+//
+// Kernel 1 (lmhead_gemm_kernel), persistent and warp-specialised, one CTA per
+// SM.  Work units are (128-row block, vocabulary split) pairs; a unit walks
+// its split in 256-column tiles:
+//   warp 0   TMA producer: 128x64 tiles of H and 256x64 tiles of W into a
+//            ring of shared-memory stages (128-byte swizzle, mbarriers);
+//   warp 1   MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32),
+//            M = 128, N = 256, K = 16 per instruction, accumulating each tile
+//            in one of two TMEM buffers (256 columns each);
+//   warps 2-5 epilogue: one thread per row reads its 256 accumulators with
+//            tcgen05.ld, releases the buffer, and folds the values into the
+//            row's online (max, count of max, sum 2^(u - max), sum (u - max)
+//            2^(u - max)) and into a top-k list (value desc, id asc) kept in
+//            shared memory.  At the end of a unit the row's partials go to
+//            the workspace.
+// Kernel 2 (lmhead_merge_kernel), one thread per row: merges the split
+// partials in a fixed order, takes the top-k, applies inclusive top-p on the
+// top-k mass and min-p against the row max, and writes the outputs.
+
+#include <cuda.h>
+
+#include <climits>
+#include <cmath>
 #include <string>
 
+#include "common.cuh"
 #include "internal.h"
 
 namespace vs {
 
+namespace {
+
+constexpr int kBM = 128;  // rows per tile (TMEM lanes)
+constexpr int kBN = 256;  // vocabulary columns per tile
+constexpr int kBK = 64;   // hidden elements per stage (128 bytes of bf16)
+constexpr int kUK = 16;   // K per tcgen05.mma (kind::f16)
+constexpr int kThreads = 192;
+constexpr int kStageABytes = kBM * kBK * 2;  // 16 KB
+constexpr int kStageBBytes = kBN * kBK * 2;  // 32 KB
+constexpr int kStageBytes = kStageABytes + kStageBBytes;
+constexpr uint32_t kTmemCols = 2 * kBN;  // two accumulators
+
+// UMMA instruction descriptor, kind::f16: D fp32, A and B bf16, both
+// K-major, N = 256, M = 128.
+constexpr uint32_t kIDesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) |
+                            (uint32_t(kBM >> 4) << 24);
+
+struct LmParams {
+  int32_t rows, vocab, hidden;
+  int32_t top_k;
+  int32_t splits;       // vocabulary splits
+  int32_t tiles_per_split;
+  int32_t n_tiles;      // ceil(vocab / kBN)
+  int32_t m_blocks;     // ceil(rows / kBM)
+  int32_t stages;
+  const float* temperature;
+  float temperature_scalar;
+  const int32_t* targets;
+  float4* ws_stats;  // [rows, splits] (m, c0, zr, a) in base-2 units of z log2(e)
+  float* ws_val;     // [rows, splits, top_k] accumulator values (desc)
+  int32_t* ws_id;    // [rows, splits, top_k]
+  float* ws_zy;      // [rows] accumulator at the target id
+  uint32_t* ws_err;  // [1] bounded-wait timeouts
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers (tcgen05, TMA tensor loads)
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t smem_desc_sw128(const void* p) {
+  // start address >> 4 | LBO 1 (16 B) | SBO 64 (1024 B = 8 rows of 128 B) |
+  // version 1 | layout SWIZZLE_128B
+  const uint64_t a = (smem_addr(p) >> 4) & 0x3FFFu;
+  return a | (uint64_t(1) << 16) | (uint64_t(64) << 32) | (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(kIDesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ---------------------------------------------------------------------------
+// shared-memory layout of the GEMM kernel (after 1024-byte alignment):
+//   [stages x (A 16 KB | B 32 KB)] [top-k values 128 x k] [top-k ids 128 x k]
+//   [barriers] [tmem slot]
+
+struct Barriers {
+  uint64_t full[4];
+  uint64_t empty[4];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint32_t tmem_base;
+  uint32_t abort;
+};
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Barriers* bs,
+                                              uint32_t* err) {
+  if (mbar_wait(bar, parity)) return true;
+  atomicOr(&bs->abort, 1u);
+  atomicOr(err, 1u);
+  return false;
+}
+
+// Insert (x, id) into a descending list of length k (count entries used);
+// equal values keep the earlier (lower) id first.
+__device__ __forceinline__ void topk_insert(float* vals, int32_t* ids, int k, int& count, float x,
+                                            int32_t id) {
+  int pos = count < k ? count : k - 1;
+  while (pos > 0 && vals[pos - 1] < x) {
+    vals[pos] = vals[pos - 1];
+    ids[pos] = ids[pos - 1];
+    --pos;
+  }
+  vals[pos] = x;
+  ids[pos] = id;
+  if (count < k) ++count;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    lmhead_gemm_kernel(const __grid_constant__ CUtensorMap map_h,
+                       const __grid_constant__ CUtensorMap map_w, LmParams P) {
+  extern __shared__ uint8_t smem_dyn[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
+                                             ~uintptr_t(1023));
+  const int S = P.stages;
+  uint8_t* stage0 = base;
+  float* tk_val = reinterpret_cast<float*>(base + S * kStageBytes);
+  int32_t* tk_id = reinterpret_cast<int32_t*>(tk_val + kBM * P.top_k);
+  Barriers* bs = reinterpret_cast<Barriers*>(
+      (reinterpret_cast<uintptr_t>(tk_id + kBM * P.top_k) + 15) & ~uintptr_t(15));
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int units = P.m_blocks * P.splits;
+  const int nkb = P.hidden / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&bs->full[s], 1);
+      mbar_init(&bs->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bs->tfull[b], 1);
+      mbar_init(&bs->tempty[b], kBM);
+    }
+    bs->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    // allocate the two accumulators (512 TMEM columns) for this CTA
+    asm volatile(
+        "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+            smem_addr(&bs->tmem_base)),
+        "r"(kTmemCols)
+        : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bs->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_h)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
+      uint32_t it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const int mb = u % P.m_blocks, sp = u / P.m_blocks;
+        const int t0 = sp * P.tiles_per_split, t1 = min(P.n_tiles, t0 + P.tiles_per_split);
+        for (int t = t0; t < t1 && ok; ++t) {
+          for (int kb = 0; kb < nkb; ++kb, ++it) {
+            const int s = it % S;
+            const uint32_t wrap = it / S;
+            if (!wait_or_abort(&bs->empty[s], (wrap & 1u) ^ 1u, bs, P.ws_err)) {
+              ok = false;
+              break;
+            }
+            uint8_t* sa = stage0 + s * kStageBytes;
+            mbar_arrive_expect_tx(&bs->full[s], kStageBytes);
+            tma_load_2d(sa, &map_h, kb * kBK, mb * kBM, &bs->full[s]);
+            tma_load_2d(sa + kStageABytes, &map_w, kb * kBK, t * kBN, &bs->full[s]);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, tile = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const int sp = u / P.m_blocks;
+        const int t0 = sp * P.tiles_per_split, t1 = min(P.n_tiles, t0 + P.tiles_per_split);
+        for (int t = t0; t < t1 && ok; ++t, ++tile) {
+          const int b = tile & 1;
+          const uint32_t use = tile >> 1;
+          if (!wait_or_abort(&bs->tempty[b], (use & 1u) ^ 1u, bs, P.ws_err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t dacc = tmem + b * kBN;
+          for (int kb = 0; kb < nkb; ++kb, ++it) {
+            const int s = it % S;
+            const uint32_t wrap = it / S;
+            if (!wait_or_abort(&bs->full[s], wrap & 1u, bs, P.ws_err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            uint8_t* sa = stage0 + s * kStageBytes;
+            const uint64_t ad = smem_desc_sw128(sa);
+            const uint64_t bd = smem_desc_sw128(sa + kStageABytes);
+#pragma unroll
+            for (int kk = 0; kk < kBK / kUK; ++kk) {
+              // advance 16 elements (32 bytes) along K inside the swizzle atom
+              umma_f16(dacc, ad + 2 * kk, bd + 2 * kk, (kb | kk) ? 1u : 0u);
+            }
+            umma_commit(&bs->empty[s]);  // frees the stage once these MMAs finish
+          }
+          if (ok) umma_commit(&bs->tfull[b]);  // accumulator b complete
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int r = q * 32 + lane;
+    const int k = P.top_k;
+    float* my_val = tk_val + r * k;
+    int32_t* my_id = tk_id + r * k;
+    uint32_t tile = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      const int mb = u % P.m_blocks, sp = u / P.m_blocks;
+      const int t0 = sp * P.tiles_per_split, t1 = min(P.n_tiles, t0 + P.tiles_per_split);
+      const int row = mb * kBM + r;
+      const bool row_ok = row < P.rows;
+      const float T = row_ok ? (P.temperature ? P.temperature[row] : P.temperature_scalar) : 1.f;
+      const float c = kLog2e / T;
+      const int y = row_ok ? P.targets[row] : -1;
+      Stats st = stats_empty();
+      int count = 0;
+      float thr = -kInf;  // current k-th value (lists are full)
+      for (int t = t0; t < t1 && ok; ++t, ++tile) {
+        const int b = tile & 1;
+        const uint32_t use = tile >> 1;
+        if (!wait_or_abort(&bs->tfull[b], use & 1u, bs, P.ws_err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tmem + (uint32_t(q * 32) << 16) + b * kBN;
+        for (int ch = 0; ch < kBN / 32; ++ch) {
+          float v[32];
+          tmem_ld32(taddr + ch * 32, v);
+          if (ch == kBN / 32 - 1) {
+            // every column of this buffer has been read: hand it back
+            tc_fence_before();
+            mbar_arrive(&bs->tempty[b]);
+          }
+          const int col0 = t * kBN + ch * 32;
+          if (!row_ok) continue;
+          if (col0 + 32 <= P.vocab) {
+            float uu[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) uu[i] = __fmul_rn(v[i], c);
+            stats_add(st, uu);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (v[i] > thr) {
+                topk_insert(my_val, my_id, k, count, v[i], col0 + i);
+                if (count == k) thr = my_val[k - 1];
+              }
+            if (y >= col0 && y < col0 + 32) {
+              float zy = 0.f;
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (y == col0 + i) zy = v[i];
+              P.ws_zy[row] = zy;
+            }
+          } else {
+            for (int i = 0; i < 32 && col0 + i < P.vocab; ++i) {
+              float uu[1] = {__fmul_rn(v[i], c)};
+              stats_add(st, uu);
+              if (v[i] > thr) {
+                topk_insert(my_val, my_id, k, count, v[i], col0 + i);
+                if (count == k) thr = my_val[k - 1];
+              }
+              if (y == col0 + i) P.ws_zy[row] = v[i];
+            }
+          }
+        }
+      }
+      if (row_ok) {
+        const int64_t slot = static_cast<int64_t>(row) * P.splits + sp;
+        P.ws_stats[slot] = make_float4(st.m, st.c0, st.zr, st.a);
+        float* dv = P.ws_val + slot * k;
+        int32_t* di = P.ws_id + slot * k;
+        for (int i = 0; i < k; ++i) {
+          dv[i] = i < count ? my_val[i] : -kInf;
+          di[i] = i < count ? my_id[i] : -1;
+        }
+      }
+    }
+  }
+
+  // teardown: every role has left its loop (bounded waits); make sure the
+  // MMAs of this CTA have completed before the accumulators are freed
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// merge: one thread per row
+
+struct MergeParams {
+  int32_t rows, vocab, splits, top_k;
+  float top_p, min_p;
+  const float* temperature;
+  float temperature_scalar;
+  const int32_t* targets;
+  const float4* ws_stats;
+  const float* ws_val;
+  const int32_t* ws_id;
+  const float* ws_zy;
+  const uint32_t* ws_err;
+  float* lp_full;
+  float* lp_support;
+  float* h_full;
+  float* h_support;
+  uint8_t* valid;
+  uint32_t* status;
+  int32_t* support_size;
+  int32_t* topk_ids;
+  float* topk_logprob;
+  int32_t want_entropy;
+};
+
+constexpr int kMaxSplits = 64;
+
+__global__ void __launch_bounds__(128) lmhead_merge_kernel(MergeParams P) {
+  const int row = blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= P.rows) return;
+  const int k = P.top_k;
+  const float T = P.temperature ? P.temperature[row] : P.temperature_scalar;
+  const float c = kLog2e / T;
+  const float nan = __int_as_float(0x7fc00000);
+  // statistics over the full vocabulary, splits merged in order
+  Stats st = stats_empty();
+  for (int s = 0; s < P.splits; ++s) {
+    const float4 v = P.ws_stats[static_cast<int64_t>(row) * P.splits + s];
+    stats_merge(st, Stats{v.x, v.y, v.z, v.w});
+  }
+  const bool timeout = *P.ws_err != 0;
+  const bool nonfinite = !stats_finite(st);
+  const float log2z = stats_log2z(st);
+  const float h_full = kLn2 * (log2z - st.a / stats_z(st));
+  // top-k by (value desc, id asc): k-way merge of the sorted split lists
+  int cur[kMaxSplits];
+  for (int s = 0; s < P.splits; ++s) cur[s] = 0;
+  float tv[VS_MAX_FUSED_TOPK];
+  int32_t ti[VS_MAX_FUSED_TOPK];
+  const int64_t base = static_cast<int64_t>(row) * P.splits * k;
+  for (int i = 0; i < k; ++i) {
+    int best = -1;
+    float bv = -kInf;
+    int32_t bi = INT_MAX;
+    for (int s = 0; s < P.splits; ++s) {
+      if (cur[s] >= k) continue;
+      const float v = P.ws_val[base + s * k + cur[s]];
+      const int32_t id = P.ws_id[base + s * k + cur[s]];
+      if (id < 0) continue;
+      if (best < 0 || v > bv || (v == bv && id < bi)) {
+        best = s;
+        bv = v;
+        bi = id;
+      }
+    }
+    if (best < 0) {
+      tv[i] = -kInf;
+      ti[i] = -1;
+    } else {
+      tv[i] = bv;
+      ti[i] = bi;
+      ++cur[best];
+    }
+  }
+  // support: inclusive top-p on the top-k mass, then min-p against the max
+  int n = 0;
+  double mass1 = 0.0;
+  for (int i = 0; i < k; ++i)
+    if (ti[i] >= 0) mass1 += static_cast<double>(ex2(__fmul_rn(tv[i], c) - st.m));
+  {
+    double cum = 0.0;
+    n = k;
+    if (P.top_p < 1.f) {
+      for (int i = 0; i < k; ++i) {
+        if (ti[i] < 0) {
+          n = i;
+          break;
+        }
+        cum += static_cast<double>(ex2(__fmul_rn(tv[i], c) - st.m));
+        if (cum >= static_cast<double>(P.top_p) * mass1) {
+          n = i + 1;
+          break;
+        }
+      }
+    } else {
+      for (int i = 0; i < k; ++i)
+        if (ti[i] < 0) {
+          n = i;
+          break;
+        }
+    }
+    if (P.min_p > 0.f) {
+      int nm = 0;
+      for (int i = 0; i < n; ++i)
+        if (ex2(__fmul_rn(tv[i], c) - st.m) >= P.min_p) nm = i + 1;
+      n = nm;
+    }
+  }
+  // support statistics (relative to its maximum, the top-1 value)
+  Stats ss = stats_empty();
+  if (n > 0) {
+    const float ms = __fmul_rn(tv[0], c);
+    ss = Stats{ms, 0.f, 0.f, 0.f};
+    for (int i = 0; i < n; ++i) {
+      const float d = __fmul_rn(tv[i], c) - ms;
+      const float e = ex2(d);
+      if (d == 0.f)
+        ss.c0 += 1.f;
+      else
+        ss.zr += e;
+      ss.a = fmaf(d, e, ss.a);
+    }
+  }
+  const float log2zs = n > 0 ? stats_log2z(ss) : nan;
+  const float h_sup = n > 0 ? kLn2 * (log2zs - ss.a / stats_z(ss)) : 0.f;
+  const int y = P.targets[row];
+  uint32_t status = 0;
+  float lp_v = nan, lp_s = nan;
+  if (y < 0 || y >= P.vocab) status |= VS_ROW_TARGET_OUT_OF_RANGE;
+  if (nonfinite) {
+    status |= VS_ROW_NONFINITE_INPUT;
+  } else if (!(status & VS_ROW_TARGET_OUT_OF_RANGE)) {
+    const float uy = __fmul_rn(P.ws_zy[row], c);
+    lp_v = kLn2 * (uy - st.m - log2z);
+    bool in_s = false;
+    for (int i = 0; i < n; ++i) in_s |= ti[i] == y;
+    if (in_s) {
+      lp_s = kLn2 * (uy - ss.m - log2zs);
+    } else {
+      lp_s = -kInf;
+      status |= VS_ROW_TARGET_NOT_IN_SUPPORT;
+    }
+  }
+  if (timeout) status |= kRowDeviceTimeout;
+  if (P.lp_full) P.lp_full[row] = lp_v;
+  if (P.lp_support) P.lp_support[row] = lp_s;
+  if (P.want_entropy) {
+    if (P.h_full) P.h_full[row] = nonfinite ? nan : h_full;
+    if (P.h_support) P.h_support[row] = nonfinite ? nan : h_sup;
+  }
+  if (P.valid) P.valid[row] = (!nonfinite && n > 0) ? 1 : 0;
+  if (P.status) P.status[row] = status;
+  if (P.support_size) P.support_size[row] = nonfinite ? 0 : n;
+  for (int i = 0; i < k; ++i) {
+    if (P.topk_ids) P.topk_ids[static_cast<int64_t>(row) * k + i] = ti[i];
+    if (P.topk_logprob)
+      P.topk_logprob[static_cast<int64_t>(row) * k + i] =
+          (ti[i] >= 0 && !nonfinite) ? kLn2 * (__fmul_rn(tv[i], c) - st.m - log2z) : nan;
+  }
+}
+
+__global__ void lmhead_clear_kernel(uint32_t* err) { *err = 0u; }
+
+// ---------------------------------------------------------------------------
+// host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int64_t ld,
+              uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+// Vocabulary splits: the fewest (up to kMaxSplits) that keep the units
+// (row blocks x splits) at >= 97% of a whole number of waves over the SMs.
+int choose_splits(int m_blocks, int n_tiles, int sms) {
+  int best = 1;
+  double best_eff = 0.0;
+  for (int s = 1; s <= kMaxSplits && s <= n_tiles; ++s) {
+    const long units = static_cast<long>(m_blocks) * s;
+    const long waves = (units + sms - 1) / sms;
+    const double eff = static_cast<double>(units) / static_cast<double>(waves * sms);
+    if (eff >= 0.97) return s;
+    if (eff > best_eff) {
+      best_eff = eff;
+      best = s;
+    }
+  }
+  return best;
+}
+
+struct LmLayout {
+  int m_blocks, n_tiles, splits, tiles_per_split;
+  size_t off_stats, off_val, off_id, off_zy, off_err, total;
+};
+
+LmLayout lm_layout(int rows, int vocab, int top_k) {
+  LmLayout L{};
+  L.m_blocks = (rows + kBM - 1) / kBM;
+  L.n_tiles = (vocab + kBN - 1) / kBN;
+  L.splits = choose_splits(L.m_blocks, L.n_tiles, num_sms());
+  L.tiles_per_split = (L.n_tiles + L.splits - 1) / L.splits;
+  L.splits = (L.n_tiles + L.tiles_per_split - 1) / L.tiles_per_split;
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t rs = static_cast<size_t>(rows) * L.splits;
+  L.off_stats = 0;
+  L.off_val = up(L.off_stats + rs * sizeof(float4));
+  L.off_id = up(L.off_val + rs * top_k * sizeof(float));
+  L.off_zy = up(L.off_id + rs * top_k * sizeof(int32_t));
+  L.off_err = up(L.off_zy + static_cast<size_t>(rows) * sizeof(float));
+  L.total = up(L.off_err + 16);
+  return L;
+}
+
+}  // namespace
+
 size_t lmhead_workspace_bytes(int rows, int vocab, int hidden, int top_k) {
-  (void)rows; (void)vocab; (void)hidden; (void)top_k;
-  return 0;
+  (void)hidden;
+  if (rows <= 0 || vocab <= 0 || top_k <= 0) return 0;
+  return lm_layout(rows, vocab, top_k).total;
 }
 
 vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh, const void* W,
@@ -16,8 +638,97 @@ vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh
                      uint32_t flags, const vs_score_out* out, int32_t* topk_ids,
                      float* topk_logprob, void* ws, size_t ws_bytes, cudaStream_t s,
                      std::string* err) {
-  *err = "vs_fused_lmhead_score is not available in this build";
-  return VS_ERR_UNSUPPORTED;
+  auto bad = [&](vs_status code, const char* msg) {
+    *err = msg;
+    return code;
+  };
+  auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (rows < 0) return bad(VS_ERR_INVALID_ARG, "rows must be >= 0");
+  if (vocab < 1) return bad(VS_ERR_INVALID_ARG, "vocab must be >= 1");
+  if (hidden < kBK || hidden % kBK != 0) return bad(VS_ERR_UNSUPPORTED, "hidden_dim must be a positive multiple of 64");
+  if (top_k < 1 || top_k > VS_MAX_FUSED_TOPK || top_k > vocab)
+    return bad(VS_ERR_UNSUPPORTED, "top_k must lie in [1, min(VS_MAX_FUSED_TOPK, vocab)]");
+  if (!(top_p > 0.f && top_p <= 1.f)) return bad(VS_ERR_INVALID_ARG, "top_p must lie in (0, 1]");
+  if (!(min_p >= 0.f && min_p < 1.f)) return bad(VS_ERR_INVALID_ARG, "min_p must lie in [0, 1)");
+  if (!temperature && !(std::isfinite(temperature_scalar) && temperature_scalar > 0.f))
+    return bad(VS_ERR_INVALID_ARG, "temperature_scalar must be finite and > 0");
+  if (!out) return bad(VS_ERR_INVALID_ARG, "out is NULL");
+  const bool want_entropy = flags & VS_WANT_ENTROPY;
+  if (!want_entropy && (out->entropy_full || out->entropy_support))
+    return bad(VS_ERR_INVALID_ARG, "entropy outputs need VS_WANT_ENTROPY");
+  if (rows == 0) return VS_OK;
+  if (!H || !W || !targets) return bad(VS_ERR_INVALID_ARG, "hidden, weight and targets must be non-NULL");
+  if (!a16(H) || !a16(W) || ldh % 8 != 0 || ldw % 8 != 0 || ldh < hidden || ldw < hidden)
+    return bad(VS_ERR_INVALID_ARG, "hidden/weight must be 16-byte aligned with ld >= hidden_dim, ld % 8 == 0");
+  const LmLayout L = lm_layout(rows, vocab, top_k);
+  if (!ws || !a16(ws) || ws_bytes < L.total)
+    return bad(VS_ERR_WORKSPACE, "workspace missing, misaligned or smaller than vs_fused_lmhead_workspace_size");
+
+  CUtensorMap map_h, map_w;
+  if (!make_map(&map_h, H, rows, hidden, ldh, kBM) || !make_map(&map_w, W, vocab, hidden, ldw, kBN))
+    return bad(VS_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  LmParams P{};
+  P.rows = rows;
+  P.vocab = vocab;
+  P.hidden = hidden;
+  P.top_k = top_k;
+  P.splits = L.splits;
+  P.tiles_per_split = L.tiles_per_split;
+  P.n_tiles = L.n_tiles;
+  P.m_blocks = L.m_blocks;
+  P.stages = top_k <= 24 ? 4 : 3;
+  P.temperature = temperature;
+  P.temperature_scalar = temperature_scalar;
+  P.targets = targets;
+  P.ws_stats = reinterpret_cast<float4*>(w8 + L.off_stats);
+  P.ws_val = reinterpret_cast<float*>(w8 + L.off_val);
+  P.ws_id = reinterpret_cast<int32_t*>(w8 + L.off_id);
+  P.ws_zy = reinterpret_cast<float*>(w8 + L.off_zy);
+  P.ws_err = reinterpret_cast<uint32_t*>(w8 + L.off_err);
+
+  const size_t smem = 1024 + static_cast<size_t>(P.stages) * kStageBytes +
+                      static_cast<size_t>(kBM) * top_k * 8 + 16 + sizeof(Barriers);
+  cudaError_t e = cudaFuncSetAttribute(lmhead_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return bad(VS_ERR_CUDA, cudaGetErrorString(e));
+  lmhead_clear_kernel<<<1, 1, 0, s>>>(P.ws_err);
+  const int units = L.m_blocks * L.splits;
+  const int grid = units < num_sms() ? units : num_sms();
+  lmhead_gemm_kernel<<<grid, kThreads, smem, s>>>(map_h, map_w, P);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return bad(VS_ERR_CUDA, cudaGetErrorString(e));
+
+  MergeParams M{};
+  M.rows = rows;
+  M.vocab = vocab;
+  M.splits = L.splits;
+  M.top_k = top_k;
+  M.top_p = top_p;
+  M.min_p = min_p;
+  M.temperature = temperature;
+  M.temperature_scalar = temperature_scalar;
+  M.targets = targets;
+  M.ws_stats = P.ws_stats;
+  M.ws_val = P.ws_val;
+  M.ws_id = P.ws_id;
+  M.ws_zy = P.ws_zy;
+  M.ws_err = P.ws_err;
+  M.lp_full = out->logprob_full;
+  M.lp_support = out->logprob_support;
+  M.h_full = want_entropy ? out->entropy_full : nullptr;
+  M.h_support = want_entropy ? out->entropy_support : nullptr;
+  M.valid = out->valid;
+  M.status = out->status;
+  M.support_size = out->support_size;
+  M.topk_ids = topk_ids;
+  M.topk_logprob = topk_logprob;
+  M.want_entropy = want_entropy ? 1 : 0;
+  lmhead_merge_kernel<<<(rows + 127) / 128, 128, 0, s>>>(M);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return bad(VS_ERR_CUDA, cudaGetErrorString(e));
+  return VS_OK;
 }
 
 }  // namespace vs

@@ -454,9 +454,14 @@ __device__ __forceinline__ void fused_elem(float x, float vmax, float c, FSums& 
   s.a = fmaf(d, e, s.a);
 }
 
+// Count one element in the window.  Elements with d < dcut are skipped: for
+// top-p alone dcut = log2((1 - p) / V) - 1, and every such element lies
+// outside the support (together they hold less than (1 - p) of the mass,
+// since the row total is at least 1); otherwise dcut = -inf.
 template <int kMode>
-__device__ __forceinline__ void win_count(uint32_t F, uint32_t fconst, uint32_t klo,
-                                          uint32_t* hist) {
+__device__ __forceinline__ void win_count(uint32_t F, float d, float dcut, uint32_t fconst,
+                                          uint32_t klo, uint32_t* hist) {
+  if (!(d >= dcut)) return;
   if constexpr (kMode == kWinPos) {
     const uint32_t b = F - fconst;
     if (b < (static_cast<uint32_t>(kWin) << 16)) atomicAdd(&hist[b >> 16], 1u);
@@ -472,8 +477,8 @@ __device__ __forceinline__ void win_count(uint32_t F, uint32_t fconst, uint32_t 
 // Fused pass over a bf16 slice: statistics relative to vmax and, when
 // kMode != kWinNone, the exact-key window histogram.
 template <int kMode>
-__device__ void fused_pass_bf16(const uint16_t* buf, int n, float vmax, float c, uint32_t fconst,
-                                uint32_t klo, uint32_t* hist, FSums& s) {
+__device__ void fused_pass_bf16(const uint16_t* buf, int n, float vmax, float c, float dcut,
+                                uint32_t fconst, uint32_t klo, uint32_t* hist, FSums& s) {
   const int nfull = n / 8;
   const uint4* v4 = reinterpret_cast<const uint4*>(buf);
   const f32x2 vm2 = pack2(vmax, vmax), c2 = pack2(c, c);
@@ -491,20 +496,21 @@ __device__ void fused_pass_bf16(const uint16_t* buf, int n, float vmax, float c,
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint32_t F0 = w[i] << 16, F1 = w[i] & 0xFFFF0000u;
+      // both elements at once: d = (x - vmax) c
+      const f32x2 d2 = mul2(sub2(pack2(__uint_as_float(F0), __uint_as_float(F1)), vm2), c2);
+      float d0, d1;
+      unpack2(d2, d0, d1);
       if (top) {
         fused_elem<true>(__uint_as_float(F0), vmax, c, s);
         fused_elem<true>(__uint_as_float(F1), vmax, c, s);
       } else {
-        // both elements at once: d = (x - vmax) c, e = 2^d, zr += e, a += d e
-        const f32x2 d2 = mul2(sub2(pack2(__uint_as_float(F0), __uint_as_float(F1)), vm2), c2);
-        float d0, d1;
-        unpack2(d2, d0, d1);
+        // e = 2^d, zr += e, a += d e
         const f32x2 e2 = pack2(ex2(d0), ex2(d1));
         zr2 = add2(zr2, e2);
         a2 = fma2(d2, e2, a2);
       }
-      win_count<kMode>(F0, fconst, klo, hist);
-      win_count<kMode>(F1, fconst, klo, hist);
+      win_count<kMode>(F0, d0, dcut, fconst, klo, hist);
+      win_count<kMode>(F1, d1, dcut, fconst, klo, hist);
     }
   }
   {
@@ -517,7 +523,7 @@ __device__ void fused_pass_bf16(const uint16_t* buf, int n, float vmax, float c,
   for (int j = nfull * 8 + threadIdx.x; j < n; j += blockDim.x) {
     const uint32_t F = static_cast<uint32_t>(buf[j]) << 16;
     fused_elem<true>(__uint_as_float(F), vmax, c, s);
-    win_count<kMode>(F, fconst, klo, hist);
+    win_count<kMode>(F, (__uint_as_float(F) - vmax) * c, dcut, fconst, klo, hist);
   }
 }
 
@@ -669,18 +675,22 @@ __global__ void __launch_bounds__(kThreads, 2) score_computed_kernel(ScoreParams
   FSums fs{0.f, 0.f, 0.f};
   if constexpr (kBf16) {
     const uint32_t hmax = __float_as_uint(vmax) >> 16;
+    // top-p alone: elements below 2^dcut = (1 - p) / V can never be kept
+    const float dcut = (use_p && !use_k && !use_minp && pp > 0.f)
+                           ? log2f((1.f - pp) / static_cast<float>(V)) - 1.f
+                           : -kInf;
     switch (wmode) {
       case kWinPos:
-        fused_pass_bf16<kWinPos>(buf, n, vmax, c, (hmax - (kWin - 1)) << 16, 0u, w.hist, fs);
+        fused_pass_bf16<kWinPos>(buf, n, vmax, c, dcut, (hmax - (kWin - 1)) << 16, 0u, w.hist, fs);
         break;
       case kWinNeg:
-        fused_pass_bf16<kWinNeg>(buf, n, vmax, c, (hmax + (kWin - 1)) << 16, 0u, w.hist, fs);
+        fused_pass_bf16<kWinNeg>(buf, n, vmax, c, dcut, (hmax + (kWin - 1)) << 16, 0u, w.hist, fs);
         break;
       case kWinKey:
-        fused_pass_bf16<kWinKey>(buf, n, vmax, c, 0u, w.klo, w.hist, fs);
+        fused_pass_bf16<kWinKey>(buf, n, vmax, c, dcut, 0u, w.klo, w.hist, fs);
         break;
       default:
-        fused_pass_bf16<kWinNone>(buf, n, vmax, c, 0u, 0u, nullptr, fs);
+        fused_pass_bf16<kWinNone>(buf, n, vmax, c, -kInf, 0u, 0u, nullptr, fs);
         break;
     }
   } else {
