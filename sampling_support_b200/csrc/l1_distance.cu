@@ -49,6 +49,24 @@ struct L1Params {
 
 __device__ __forceinline__ float sgn(float d) { return d > 0.f ? 1.f : (d < 0.f ? -1.f : 0.f); }
 
+// p_j (in [0, 1], so bits 30 and 31 of its fp32 pattern are zero) and
+// s_j = sign(p_j - q_j) in one 32-bit word: bit 31 set for s = -1, bit 30 set
+// for s = 0.  Pass 2 writes it over the element's two shared-memory slots so
+// the gradient pass needs no second exponentiation.
+__device__ __forceinline__ uint32_t enc_ps(float p, float d) {
+  uint32_t w = __float_as_uint(p);
+  if (d < 0.f)
+    w |= 0x80000000u;
+  else if (!(d > 0.f))
+    w |= 0x40000000u;
+  return w;
+}
+__device__ __forceinline__ float dec_grad(uint32_t w, float coef, float ps) {
+  const float p = __uint_as_float(w & 0x3FFFFFFFu);
+  const float s = (w & 0x40000000u) ? 0.f : ((w & 0x80000000u) ? -1.f : 1.f);
+  return coef * p * (s - ps);
+}
+
 template <typename Raw, typename G>
 __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
   constexpr int VEC = 16 / sizeof(Raw);
@@ -132,12 +150,17 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
   const float md = Sd.m, ld2 = stats_log2z(Sd);
   const float mt = St.m, lt2 = stats_log2z(St);
 
-  // pass 2: L1 = sum |p - q| and sum_k p_k sign(p_k - q_k)
+  // pass 2: L1 = sum |p - q| and sum_k p_k sign(p_k - q_k); (p, s) kept in
+  // place for the gradient pass
   float l1 = 0.f, ps = 0.f;
+  const bool keep = P.grad != nullptr;
+  uint4* d4w = reinterpret_cast<uint4*>(bd);
+  uint4* t4w = reinterpret_cast<uint4*>(bt);
   for (int v = tid; v < nfull; v += blockDim.x) {
     Raw rd[VEC], rt[VEC];
     unpack(d4[v], rd);
     unpack(t4[v], rt);
+    uint32_t enc[VEC];
 #pragma unroll
     for (int i = 0; i < VEC; ++i) {
       const float p = ex2((__fmul_rn(value_of(rd[i]), kLog2e) - md) - ld2);
@@ -145,6 +168,21 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
       const float d = p - q;
       l1 += fabsf(d);
       ps = fmaf(p, sgn(d), ps);
+      enc[i] = enc_ps(p, d);
+    }
+    if (keep) {
+      if constexpr (sizeof(Raw) == 2) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          hi[i] = (enc[2 * i] >> 16) | (enc[2 * i + 1] & 0xFFFF0000u);
+          lo[i] = (enc[2 * i] & 0xFFFFu) | (enc[2 * i + 1] << 16);
+        }
+        d4w[v] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        t4w[v] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      } else {
+        d4w[v] = make_uint4(enc[0], enc[1], enc[2], enc[3]);
+      }
     }
   }
   for (int j = nfull * VEC + tid; j < n; j += blockDim.x) {
@@ -153,6 +191,15 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
     const float d = p - q;
     l1 += fabsf(d);
     ps = fmaf(p, sgn(d), ps);
+    if (keep) {
+      const uint32_t e = enc_ps(p, d);
+      if constexpr (sizeof(Raw) == 2) {
+        bd[j] = static_cast<Raw>(e >> 16);
+        bt[j] = static_cast<Raw>(e & 0xFFFFu);
+      } else {
+        bd[j] = e;
+      }
+    }
   }
   l1 = block_sum(l1, sh.fred);
   ps = block_sum(ps, sh.fred);
@@ -180,15 +227,20 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
     const float coef = wsum > 0.0 ? static_cast<float>(static_cast<double>(w) / wsum) : 0.f;
     G* go = static_cast<G*>(P.grad) + static_cast<int64_t>(row) * P.grad_ld + c0;
     for (int v = tid; v < nfull; v += blockDim.x) {
-      Raw rd[VEC], rt[VEC];
-      unpack(d4[v], rd);
-      unpack(t4[v], rt);
       float out[VEC];
+      if constexpr (sizeof(Raw) == 2) {
+        const uint4 hv = d4[v], lv = t4[v];
+        const uint32_t hi[4] = {hv.x, hv.y, hv.z, hv.w}, lo[4] = {lv.x, lv.y, lv.z, lv.w};
 #pragma unroll
-      for (int i = 0; i < VEC; ++i) {
-        const float p = ex2((__fmul_rn(value_of(rd[i]), kLog2e) - md) - ld2);
-        const float q = ex2((__fmul_rn(value_of(rt[i]), kLog2e) - mt) - lt2);
-        out[i] = coef * p * (sgn(p - q) - PS);
+        for (int i = 0; i < 4; ++i) {
+          out[2 * i] = dec_grad((hi[i] << 16) | (lo[i] & 0xFFFFu), coef, PS);
+          out[2 * i + 1] = dec_grad((hi[i] & 0xFFFF0000u) | (lo[i] >> 16), coef, PS);
+        }
+      } else {
+        const uint4 e = d4[v];
+        const uint32_t ee[4] = {e.x, e.y, e.z, e.w};
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) out[i] = dec_grad(ee[i], coef, PS);
       }
       G* dst = go + v * VEC;
       if constexpr (sizeof(G) == 2) {
@@ -208,9 +260,12 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
       }
     }
     for (int j = nfull * VEC + tid; j < n; j += blockDim.x) {
-      const float p = ex2((__fmul_rn(value_of(bd[j]), kLog2e) - md) - ld2);
-      const float q = ex2((__fmul_rn(value_of(bt[j]), kLog2e) - mt) - lt2);
-      const float g = coef * p * (sgn(p - q) - PS);
+      uint32_t e;
+      if constexpr (sizeof(Raw) == 2)
+        e = (static_cast<uint32_t>(bd[j]) << 16) | static_cast<uint32_t>(bt[j]);
+      else
+        e = bd[j];
+      const float g = dec_grad(e, coef, PS);
       if constexpr (sizeof(G) == 2)
         go[j] = static_cast<G>(__bfloat16_as_ushort(__float2bfloat16_rn(g)));
       else

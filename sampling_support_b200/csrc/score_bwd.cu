@@ -190,7 +190,16 @@ __global__ void __launch_bounds__(kThreads) score_bwd_kernel(BwdParams P, int nc
   const uint4* g4 = reinterpret_cast<const uint4*>(grow + c0);
   for (int v = threadIdx.x; v < nfull; v += blockDim.x) {
     float out[VEC];
-    if (k.need_full || k.need_sup) {
+    // off-support elements of a recorded support carry no gradient unless a
+    // full-vocabulary term is active: such groups are written as zeros (or
+    // left alone when accumulating) without reading their logits
+    bool load = k.need_full || k.need_sup;
+    if (load && recorded && !k.need_full) {
+      const int j0 = v * VEC;
+      load = ((bitmap[j0 >> 5] >> (j0 & 31)) & ((1u << VEC) - 1u)) != 0u;
+    }
+    if (ACC && !load) continue;
+    if (load) {
       Raw r[VEC];
       unpack(__ldcs(g4 + v), r);
 #pragma unroll

@@ -304,6 +304,7 @@ __device__ Desc descend(const Raw* buf, int n, float c, float vmax, int fx_shift
 
 struct Window {
   uint32_t klo, kmax;
+  int nbins;      // kmax - klo + 1 (<= kWin)
   int S;          // bins per CTA slice
   uint32_t* hist;  // this CTA's unreduced histogram [kWin]
   uint32_t* red;   // this CTA's reduced slice [S]
@@ -326,7 +327,7 @@ __device__ void window_reduce(Window& w, SelShared& sh, cg::cluster_group& clust
   const uint32_t klo = w.klo;
   uint32_t* hist = w.hist;
   const int b0 = static_cast<int>(rank) * w.S;
-  const int b1 = min(kWin, b0 + w.S);
+  const int b1 = min(w.nbins, b0 + w.S);
   u64 tc = 0, tm = 0;
   for (int b = b0 + threadIdx.x; b < b1; b += blockDim.x) {
     uint32_t sum = 0;
@@ -374,7 +375,7 @@ __device__ bool window_search(const Window& w, bool by_mass, u64 need, int slot,
   if (rs < 0) return false;
   if (rank == rs) {
     const int b0 = rs * w.S;
-    const int nb = min(kWin, b0 + w.S) - b0;
+    const int nb = max(0, min(w.nbins, b0 + w.S) - b0);
     const int per = (nb + blockDim.x - 1) / blockDim.x;
     const int i0 = threadIdx.x * per, i1 = min(nb, i0 + per);
     u64 lc = 0, lm = 0;
@@ -454,30 +455,26 @@ __device__ __forceinline__ void fused_elem(float x, float vmax, float c, FSums& 
   s.a = fmaf(d, e, s.a);
 }
 
-// Count one element in the window.  Elements with d < dcut are skipped: for
-// top-p alone dcut = log2((1 - p) / V) - 1, and every such element lies
-// outside the support (together they hold less than (1 - p) of the mass,
-// since the row total is at least 1); otherwise dcut = -inf.
+// Count one element (raw float bits F) in the window of `nbins` exact keys.
 template <int kMode>
-__device__ __forceinline__ void win_count(uint32_t F, float d, float dcut, uint32_t fconst,
+__device__ __forceinline__ void win_count(uint32_t F, uint32_t nbins, uint32_t fconst,
                                           uint32_t klo, uint32_t* hist) {
-  if (!(d >= dcut)) return;
   if constexpr (kMode == kWinPos) {
     const uint32_t b = F - fconst;
-    if (b < (static_cast<uint32_t>(kWin) << 16)) atomicAdd(&hist[b >> 16], 1u);
+    if (b < (nbins << 16)) atomicAdd(&hist[b >> 16], 1u);
   } else if constexpr (kMode == kWinNeg) {
     const uint32_t b = fconst - F;
-    if (b < (static_cast<uint32_t>(kWin) << 16)) atomicAdd(&hist[b >> 16], 1u);
+    if (b < (nbins << 16)) atomicAdd(&hist[b >> 16], 1u);
   } else if constexpr (kMode == kWinKey) {
     const uint32_t b = key_of(static_cast<uint16_t>(F >> 16)) - klo;
-    if (b < static_cast<uint32_t>(kWin)) atomicAdd(&hist[b], 1u);
+    if (b < nbins) atomicAdd(&hist[b], 1u);
   }
 }
 
 // Fused pass over a bf16 slice: statistics relative to vmax and, when
 // kMode != kWinNone, the exact-key window histogram.
 template <int kMode>
-__device__ void fused_pass_bf16(const uint16_t* buf, int n, float vmax, float c, float dcut,
+__device__ void fused_pass_bf16(const uint16_t* buf, int n, float vmax, float c, uint32_t nbins,
                                 uint32_t fconst, uint32_t klo, uint32_t* hist, FSums& s) {
   const int nfull = n / 8;
   const uint4* v4 = reinterpret_cast<const uint4*>(buf);
@@ -509,8 +506,8 @@ __device__ void fused_pass_bf16(const uint16_t* buf, int n, float vmax, float c,
         zr2 = add2(zr2, e2);
         a2 = fma2(d2, e2, a2);
       }
-      win_count<kMode>(F0, d0, dcut, fconst, klo, hist);
-      win_count<kMode>(F1, d1, dcut, fconst, klo, hist);
+      win_count<kMode>(F0, nbins, fconst, klo, hist);
+      win_count<kMode>(F1, nbins, fconst, klo, hist);
     }
   }
   {
@@ -523,7 +520,7 @@ __device__ void fused_pass_bf16(const uint16_t* buf, int n, float vmax, float c,
   for (int j = nfull * 8 + threadIdx.x; j < n; j += blockDim.x) {
     const uint32_t F = static_cast<uint32_t>(buf[j]) << 16;
     fused_elem<true>(__uint_as_float(F), vmax, c, s);
-    win_count<kMode>(F, (__uint_as_float(F) - vmax) * c, dcut, fconst, klo, hist);
+    win_count<kMode>(F, nbins, fconst, klo, hist);
   }
 }
 
@@ -646,27 +643,46 @@ __global__ void __launch_bounds__(kThreads, 2) score_computed_kernel(ScoreParams
   float vmax = -kInf;
   for (uint32_t r = 0; r < CL; ++r) vmax = fmaxf(vmax, sh.vmax_g[r]);
 
-  // ---- window geometry (bf16 with a filter): exact keys kmax - kWin + 1 .. kmax
+  // ---- window geometry (bf16 with a filter): exact keys klo .. kmax, at most
+  // kWin of them.  With top-p alone the window starts at the first key whose
+  // d = (v - vmax) c reaches dcut = log2((1 - p) / V) - 1: every element
+  // below it lies outside the support (together they hold less than (1 - p)
+  // of the mass, the row total being at least 1).
   Window w{};
   int wmode = kWinNone;
   if constexpr (kBf16) {
     if (any_filter && isfinite(vmax)) {
       const uint32_t hmax = __float_as_uint(vmax) >> 16;
       w.kmax = key_of(static_cast<uint16_t>(hmax));
-      w.klo = w.kmax >= static_cast<uint32_t>(kWin - 1) ? w.kmax - (kWin - 1) : 0u;
-      w.S = (kWin + CL - 1) / CL;
+      uint32_t klo = w.kmax >= static_cast<uint32_t>(kWin - 1) ? w.kmax - (kWin - 1) : 0u;
+      if (use_p && !use_k && !use_minp && pp > 0.f) {
+        const float dcut = log2f((1.f - pp) / static_cast<float>(V)) - 1.f;
+        uint32_t lo = klo, hi = w.kmax;  // smallest key with d >= dcut (kmax has d = 0)
+        while (lo < hi) {
+          const uint32_t mid = lo + ((hi - lo) >> 1);
+          if ((KT::decode(mid) - vmax) * c >= dcut)
+            hi = mid;
+          else
+            lo = mid + 1;
+        }
+        klo = lo;
+      }
+      w.klo = klo;
+      w.nbins = static_cast<int>(w.kmax - klo) + 1;
+      w.S = (w.nbins + CL - 1) / CL;
       w.hist = reinterpret_cast<uint32_t*>(big);
       w.red = w.hist + kWin;
       w.c = c;
       w.vmax = vmax;
       w.fxs = fx_scale(P.fx_shift);
-      if (!(hmax & 0x8000u) && hmax >= static_cast<uint32_t>(kWin))
-        wmode = kWinPos;  // lowest window value > +0
-      else if ((hmax & 0x8000u) && hmax != 0x8000u && hmax <= 0xFFFFu - (kWin - 1))
-        wmode = kWinNeg;  // vmax < 0: every value is negative
+      if (klo > 0x7FFFu && (w.kmax - 0x7FFFu) < 0x7000u)
+        wmode = kWinPos;  // every window key is a positive nonzero value (below 2^97, so
+                          // no negative raw pattern lands within kWin bins of raw(klo))
+      else if (w.kmax < 0x7FFFu)
+        wmode = kWinNeg;  // every window key is a negative nonzero value
       else
         wmode = kWinKey;
-      for (int b = tid; b < kWin; b += blockDim.x) w.hist[b] = 0u;
+      for (int b = tid; b < w.nbins; b += blockDim.x) w.hist[b] = 0u;
       __syncthreads();
     }
   }
@@ -674,23 +690,19 @@ __global__ void __launch_bounds__(kThreads, 2) score_computed_kernel(ScoreParams
   // ---- pass 1 (fused): sums relative to vmax (+ window histogram)
   FSums fs{0.f, 0.f, 0.f};
   if constexpr (kBf16) {
-    const uint32_t hmax = __float_as_uint(vmax) >> 16;
-    // top-p alone: elements below 2^dcut = (1 - p) / V can never be kept
-    const float dcut = (use_p && !use_k && !use_minp && pp > 0.f)
-                           ? log2f((1.f - pp) / static_cast<float>(V)) - 1.f
-                           : -kInf;
+    const uint32_t nb = static_cast<uint32_t>(w.nbins);
     switch (wmode) {
-      case kWinPos:
-        fused_pass_bf16<kWinPos>(buf, n, vmax, c, dcut, (hmax - (kWin - 1)) << 16, 0u, w.hist, fs);
+      case kWinPos:  // bin = raw - raw(klo), on the fp32 bit pattern
+        fused_pass_bf16<kWinPos>(buf, n, vmax, c, nb, (w.klo - 0x7FFFu) << 16, 0u, w.hist, fs);
         break;
-      case kWinNeg:
-        fused_pass_bf16<kWinNeg>(buf, n, vmax, c, dcut, (hmax + (kWin - 1)) << 16, 0u, w.hist, fs);
+      case kWinNeg:  // bin = raw(klo) - raw
+        fused_pass_bf16<kWinNeg>(buf, n, vmax, c, nb, (0xFFFFu - w.klo) << 16, 0u, w.hist, fs);
         break;
       case kWinKey:
-        fused_pass_bf16<kWinKey>(buf, n, vmax, c, dcut, 0u, w.klo, w.hist, fs);
+        fused_pass_bf16<kWinKey>(buf, n, vmax, c, nb, 0u, w.klo, w.hist, fs);
         break;
       default:
-        fused_pass_bf16<kWinNone>(buf, n, vmax, c, -kInf, 0u, 0u, nullptr, fs);
+        fused_pass_bf16<kWinNone>(buf, n, vmax, c, 0u, 0u, 0u, nullptr, fs);
         break;
     }
   } else {
@@ -844,7 +856,7 @@ __global__ void __launch_bounds__(kThreads, 2) score_computed_kernel(ScoreParams
       if (win_ok && tkey >= w.klo) {
         // from the reduced window bins of this CTA's slice
         const int b0 = static_cast<int>(rank) * w.S;
-        const int b1 = min(kWin, b0 + w.S);
+        const int b1 = min(w.nbins, b0 + w.S);
         for (int b = b0 + tid; b < b1; b += blockDim.x) {
           const uint32_t cnt = w.red[b - b0];
           const uint32_t key = w.klo + b;
@@ -935,10 +947,21 @@ __global__ void __launch_bounds__(kThreads, 2) score_computed_kernel(ScoreParams
         // need-th tie walks its range again to find it
         const int need = static_cast<int>(ckeep - off);
         const uint32_t t = tkey;
-        const int per = (n + kThreads - 1) / kThreads;
+        constexpr int kV = 16 / sizeof(Raw);
+        const int per = ((n + kThreads - 1) / kThreads + kV - 1) / kV * kV;
         const int j0 = tid * per, j1 = min(n, j0 + per);
         int mine = 0;
-        for (int j = j0; j < j1; ++j) mine += key_of(buf[j]) == t;
+        {
+          int j = j0;
+          const uint4* v4 = reinterpret_cast<const uint4*>(buf);
+          for (; j + kV <= j1; j += kV) {
+            Raw r[kV];
+            unpack(v4[j / kV], r);
+#pragma unroll
+            for (int i = 0; i < kV; ++i) mine += key_of(r[i]) == t;
+          }
+          for (; j < j1; ++j) mine += key_of(buf[j]) == t;
+        }
         const int lane = tid & 31, warp = tid >> 5;
         int incl = mine;
 #pragma unroll

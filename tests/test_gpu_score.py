@@ -120,6 +120,18 @@ def test_crossing_below_the_key_window(filt):
     _run(logits, np.arange(rows, dtype=np.int32), np.full(rows, 1e9, F32), *filt)
 
 
+@pytest.mark.parametrize("scale,shift", [(0.01, 0.0), (1.0, 2e30), (3.0, 0.004)])
+def test_window_crossing_zero_and_huge_values(scale, shift):
+    # tiny logits: the top-p window reaches across zero into negative keys;
+    # huge logits: positive-only raw-bit binning is not used
+    rows, vocab = 4, 9000
+    x = workloads.normal((rows, vocab), scale, seed=17, stream=1) + np.float32(shift)
+    logits = workloads.to_bf16_bits(x)
+    temp = np.full(rows, 1.0 if shift < 1e3 else 2e29, F32)
+    for filt in [(0, 0.5, 0.0), (0, 0.999, 0.0), (300, 1.0, 0.0), (0, 1.0, 0.3)]:
+        _run(logits, np.arange(rows, dtype=np.int32), temp, *filt)
+
+
 def test_all_negative_rows():
     rows, vocab = 5, 30_000
     x = workloads.normal((rows, vocab), 3.0, seed=12, stream=1) - 60.0
