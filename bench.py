@@ -220,9 +220,12 @@ def headline(args, world, rank, pk):
     sp = ctypes.c_void_p(stream.cuda_stream)
     fwd = lib.vs_score_fwd
     oref = ctypes.byref(o)
+    ws = B.score_workspace(lib.vs_score_fwd_workspace_size(ctypes.byref(argsets[0])), dev)
+    ws_ptr = 0 if ws is None else ws.data_ptr()
+    ws_n = 0 if ws is None else ws.numel()
 
     def step(i):
-        rc = fwd(ctypes.byref(argsets[i % nbuf]), oref, None, 0, sp)
+        rc = fwd(ctypes.byref(argsets[i % nbuf]), oref, ws_ptr, ws_n, sp)
         if rc:
             raise RuntimeError(lib.vs_last_error().decode())
 

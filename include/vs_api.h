@@ -148,7 +148,14 @@ typedef struct vs_score_out {
  * the row) are computed for every row when logprob_full or entropy_full is
  * requested, else only for rows whose S is empty (the lp_V fallback).
  *
- * Returns VS_ERR_INVALID_ARG for NULL required pointers, R < 0, V < 1,
+ * Workspace: bf16 rows with a computed support (no support_ids) need
+ * vs_score_fwd_workspace_size(args) bytes of device scratch, 16-byte
+ * aligned, no initial contents required.  One call at a time per workspace
+ * (calls on different streams need different workspaces).  Other argument
+ * sets need none (NULL, 0).
+ *
+ * Returns VS_ERR_WORKSPACE when a needed workspace is missing, misaligned or
+ * too small; VS_ERR_INVALID_ARG for NULL required pointers, R < 0, V < 1,
  * ld < V, bad alignment, a non-positive or non-finite temperature_scalar,
  * top_p_scalar outside (0, 1], min_p_scalar outside [0, 1), a flag whose
  * output pointer is NULL; VS_ERR_UNSUPPORTED for V beyond the resident-row
@@ -159,7 +166,10 @@ typedef struct vs_score_out {
 vs_status vs_score_fwd(const vs_score_args* args, const vs_score_out* out, void* workspace,
                        size_t workspace_bytes, void* stream);
 
-/* Workspace bytes vs_score_fwd needs for these arguments (0 today). */
+/* Workspace bytes vs_score_fwd needs for these arguments: 0 for fp32 rows
+ * and for a recorded support; for bf16 rows with a computed support it grows
+ * with R (per-chunk statistics and 8 KB key histograms) and is capped near
+ * 64 MB by processing large batches in several launches. */
 size_t vs_score_fwd_workspace_size(const vs_score_args* args);
 
 /* Largest vocabulary vs_score_fwd accepts for a dtype. */

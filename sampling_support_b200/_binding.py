@@ -164,10 +164,29 @@ def make_args(logits, targets, temperature=1.0, top_k=0, top_p=1.0, min_p=0.0,
     return a, keep
 
 
+_SCORE_WS = {}
+
+
+def score_workspace(nbytes, device):
+    """A device workspace of at least nbytes, kept per device (vs_score_fwd
+    needs no initial contents; calls on one stream may share it)."""
+    if nbytes <= 0:
+        return None
+    key = (device.type, device.index)
+    ws = _SCORE_WS.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty((nbytes + 15) // 16 * 16, dtype=torch.uint8, device=device)
+        _SCORE_WS[key] = ws
+    return ws
+
+
 def score_fwd(logits, targets, temperature=1.0, top_k=0, top_p=1.0, min_p=0.0,
               support_ids=None, want_entropy=True, want_mask=False, want_grad=False,
-              want_full=True, want_reduce=False, vocab=None, stream=None):
-    """Run vs_score_fwd; returns a dict of device tensors."""
+              want_full=True, want_reduce=False, vocab=None, workspace=None, stream=None):
+    """Run vs_score_fwd; returns a dict of device tensors.
+
+    workspace: a uint8 device tensor of at least vs_score_fwd_workspace_size
+    bytes (one call at a time); by default a buffer cached per device."""
     lib = load()
     rows, ld = logits.shape
     vocab = ld if vocab is None else vocab
@@ -207,7 +226,10 @@ def score_fwd(logits, targets, temperature=1.0, top_k=0, top_p=1.0, min_p=0.0,
     o.ctx = _p(out.get("ctx"))
     o.entropy_sum = _p(out.get("entropy_sum") if want_entropy else None)
     o.valid_count = _p(out.get("valid_count"))
-    _check(lib.vs_score_fwd(ctypes.byref(a), ctypes.byref(o), None, 0, _stream(stream)))
+    if workspace is None:
+        workspace = score_workspace(lib.vs_score_fwd_workspace_size(ctypes.byref(a)), dev)
+    _check(lib.vs_score_fwd(ctypes.byref(a), ctypes.byref(o), _p(workspace),
+                            0 if workspace is None else workspace.numel(), _stream(stream)))
     del keep
     return out
 

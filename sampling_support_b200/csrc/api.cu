@@ -112,14 +112,13 @@ int32_t vs_score_max_vocab(vs_dtype dtype) {
 }
 
 size_t vs_score_fwd_workspace_size(const vs_score_args* args) {
-  (void)args;
-  return 0;
+  if (!args || args->rows <= 0 || args->vocab < 1 || args->support_ids || args->dtype != VS_BF16)
+    return 0;
+  return vs::score_split_workspace_bytes(args->rows, args->vocab);
 }
 
 vs_status vs_score_fwd(const vs_score_args* a, const vs_score_out* o, void* workspace,
                        size_t workspace_bytes, void* stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   vs_status st = check_args(a);
   if (st != VS_OK) return st;
   if (!o) return fail(VS_ERR_INVALID_ARG, "out is NULL");
@@ -141,7 +140,13 @@ vs_status vs_score_fwd(const vs_score_args* a, const vs_score_out* o, void* work
   const bool recorded = a->support_ids != nullptr;
   if (!recorded && a->vocab > vs::score_max_vocab(a->dtype))
     return fail(VS_ERR_UNSUPPORTED, "vocab exceeds vs_score_max_vocab for this dtype");
-  if (a->rows == 0) return ok();
+  const bool split = !recorded && a->dtype == VS_BF16;
+  if (split) {
+    const size_t need = vs::score_split_workspace_bytes(a->rows, a->vocab);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < need)
+      return fail(VS_ERR_WORKSPACE,
+                  "workspace missing, misaligned or smaller than vs_score_fwd_workspace_size(args)");
+  }
 
   vs::ScoreParams p{};
   p.rows = a->rows;
@@ -178,15 +183,12 @@ vs_status vs_score_fwd(const vs_score_args* a, const vs_score_out* o, void* work
   if (p.fx_shift > 60) p.fx_shift = 60;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (recorded) {
-    p.chunk = 0;
+  if (recorded)
     e = vs::launch_score_recorded(p, a->dtype, s);
-  } else {
-    int chunk = 0;
-    const int cl = vs::score_cluster_size(a->vocab, a->dtype, &chunk);
-    p.chunk = chunk;
-    e = vs::launch_score_computed(p, a->dtype, cl, s);
-  }
+  else if (split)
+    e = vs::launch_score_split(p, workspace, s);
+  else
+    e = vs::launch_score_computed(p, a->dtype, s);
   if (e != cudaSuccess) return cuda_fail(e, "vs_score_fwd launch");
   if (o->entropy_sum || o->valid_count) {
     e = vs::launch_score_reduce(p.h_support, o->valid, a->rows, o->entropy_sum, o->valid_count, s);

@@ -165,16 +165,36 @@ __device__ __forceinline__ Stats shfl_xor(const Stats& s, int lane_mask) {
 }
 
 // Deterministic block reduction; result valid in every thread.  `scratch`
-// holds at least blockDim.x / 32 entries.
+// holds at least blockDim.x / 32 entries.  The block max comes first, then
+// every thread rebases its own statistics onto it once and plain sums
+// follow (no chain of rebases).
 __device__ __forceinline__ Stats block_reduce(Stats s, Stats* scratch) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) stats_merge(s, shfl_xor(s, o));
-  if (lane == 0) scratch[warp] = s;
-  __syncthreads();
-  Stats t = stats_empty();
   const int nw = blockDim.x >> 5;
-  for (int w = 0; w < nw; ++w) stats_merge(t, scratch[w]);
+  float m = s.m;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) scratch[warp].m = m;
+  __syncthreads();
+  m = -kInf;
+  for (int w = 0; w < nw; ++w) m = fmaxf(m, scratch[w].m);
+  __syncthreads();
+  if (s.c0 != 0.f || s.zr != 0.f) stats_rebase(s, m);
+  float c0 = s.c0, zr = s.zr, a = s.a;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    c0 += __shfl_xor_sync(0xffffffffu, c0, o);
+    zr += __shfl_xor_sync(0xffffffffu, zr, o);
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+  }
+  if (lane == 0) scratch[warp] = Stats{m, c0, zr, a};
+  __syncthreads();
+  Stats t{m, 0.f, 0.f, 0.f};
+  for (int w = 0; w < nw; ++w) {
+    t.c0 += scratch[w].c0;
+    t.zr += scratch[w].zr;
+    t.a += scratch[w].a;
+  }
   __syncthreads();
   return t;
 }

@@ -68,7 +68,6 @@ struct ScoreParams {
   RowCtx* ctx;
   int32_t want_entropy;
   int32_t full_stats;  // recorded support: compute full-vocabulary stats for every row
-  int32_t chunk;       // elements per CTA of a row (multiple of 32)
   int32_t fx_shift;    // fixed-point scale of mass histograms: 2^fx_shift
 };
 
@@ -91,15 +90,16 @@ struct BwdParams {
 };
 
 // launchers (return a cudaError_t from the launch)
-cudaError_t launch_score_computed(const ScoreParams& p, vs_dtype dtype, int cluster,
-                                  cudaStream_t s);
+cudaError_t launch_score_computed(const ScoreParams& p, vs_dtype dtype, cudaStream_t s);
 cudaError_t launch_score_recorded(const ScoreParams& p, vs_dtype dtype, cudaStream_t s);
 cudaError_t launch_score_reduce(const float* h_support, const uint8_t* valid, int rows,
                                 double* entropy_sum, int32_t* valid_count, cudaStream_t s);
 cudaError_t launch_score_bwd(const BwdParams& p, vs_dtype dtype, vs_dtype gdtype, int mode,
                              bool whole_rows, int nchunks, cudaStream_t s);
 
-int score_cluster_size(int vocab, vs_dtype dtype, int* chunk);
+cudaError_t launch_score_split(const ScoreParams& p, void* ws, cudaStream_t s);
+size_t score_split_workspace_bytes(int rows, int vocab);
+int32_t score_split_max_vocab();
 int score_max_vocab(vs_dtype dtype);
 
 }  // namespace vs

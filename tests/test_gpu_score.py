@@ -151,10 +151,15 @@ def test_singletons_are_exact_zeros():
     assert np.all(out["support_size"].cpu().numpy() == 1)
 
 
-def test_max_vocab():
-    vmax = vsb.load().vs_score_max_vocab(1)
-    logits = workloads.random_logits(2, vmax, 3.0, seed=9)
-    _run(logits, np.array([0, vmax - 1], np.int32), np.array([0.7, 1.1], F32), 0, 0.9, 0.0)
+def test_large_vocab():
+    # well beyond a shared-memory-resident row; rows are streamed
+    vocab = 1_000_003
+    ld = (vocab + 7) // 8 * 8
+    logits = workloads.random_logits(2, vocab, 3.0, seed=9, ld=ld)
+    _run(logits, np.array([0, vocab - 1], np.int32), np.array([0.7, 1.1], F32), 0, 0.9, 0.0,
+         vocab=vocab)
+    _run(logits, np.array([5, 17], np.int32), np.array([1.0, 1.0], F32), 1000, 0.99, 0.0,
+         vocab=vocab)
 
 
 def test_zero_rows():
