@@ -508,15 +508,14 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
         if (win_ok && use_p) {
           double mass1;
           if (use_k) {
-            const u64 fx_t = dk.at_cnt ? dk.at_mass / dk.at_cnt : 0;
-            mass1 = static_cast<double>(dk.above_mass + ck * fx_t);
+            mass1 = static_cast<double>(dk.above_mass + ck * bin_fx(w, dk.key));
           } else {
             mass1 = (static_cast<double>(s.c0) + static_cast<double>(s.zr)) * static_cast<double>(fxs);
           }
           const u64 tp = topp_target(pp, mass1);
           win_ok = win_search<kRT>(w, true, tp, dp, sh.sel);
           if (win_ok) {
-            u64 cp = topp_ties(dp, tp);
+            u64 cp = topp_ties(dp, tp, bin_fx(w, dp.key));
             if (use_k && dp.key == tkey && cp > ck) cp = ck;
             tkey = dp.key;
             cnum = cp;
@@ -538,10 +537,10 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
         all_ties = ck >= d.at_cnt;
         have_t = true;
         if (use_p) {
-          const u64 fx_t = d.at_cnt ? d.at_mass / d.at_cnt : 0;
+          const u64 fx_t = key_fx<Raw>(d.key, c, m, fx_scale(P.fx_shift));
           const u64 tp = topp_target(pp, static_cast<double>(d.above_mass + ck * fx_t));
           Desc e = descend(ring, c, m, P.fx_shift, true, true, tp, pp, sh, ra);
-          u64 cp = topp_ties(e, tp);
+          u64 cp = topp_ties(e, tp, key_fx<Raw>(e.key, c, m, fx_scale(P.fx_shift)));
           if (e.key == tkey && cp > ck) cp = ck;
           tkey = e.key;
           cnum = cp;
@@ -550,7 +549,7 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
       } else {
         Desc e = descend(ring, c, m, P.fx_shift, true, true, 0ull, pp, sh, ra);
         const u64 tp = sh.ulred[1];
-        const u64 cp = topp_ties(e, tp);
+        const u64 cp = topp_ties(e, tp, key_fx<Raw>(e.key, c, m, fx_scale(P.fx_shift)));
         tkey = e.key;
         cnum = cp;
         all_ties = cp >= e.at_cnt;

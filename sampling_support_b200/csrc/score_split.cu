@@ -43,20 +43,24 @@ namespace {
 constexpr int kCT = 128;          // threads per chunk CTA
 constexpr int kMT = 512;          // threads per merge CTA
 constexpr int kMW = kMT / 32;     // warps per merge CTA
-constexpr int kUnroll = 8;        // 16-byte loads in flight per thread
+constexpr int kRound = 4;         // vectors per thread and round of the chunk pass
 constexpr int kMaxChunks = 256;   // chunks per row
 constexpr int kChunkAlign = 256;  // chunk length granularity (elements)
 constexpr int kMaxChunk = 65280;  // 16-bit histogram counts
-constexpr int kHistWords = kSelWin / 2;  // one chunk histogram, u16 pairs
+constexpr int kHead = 256;        // histogram headroom above the first-round max (keys)
+constexpr int kCW = kSelWin + kHead;     // bins of a chunk histogram
+constexpr int kHistWords = kCW / 2;      // one chunk histogram, u16 pairs
 constexpr size_t kSplitWsCap = size_t(64) << 20;
 
-// Per (row, chunk) record.
+// Per (row, chunk) record.  The statistics' reference is the chunk max; the
+// histogram's top key ktop is at or above the chunk max key.
 struct alignas(16) ChunkRec {
   float vmax;       // chunk maximum (value)
   float c0, zr, a;  // statistics relative to fl(vmax c)
   uint32_t nb;      // histogram bins written (bins >= nb hold nothing)
   uint32_t ylt;     // chunk holding the target: its earlier ties (else 0)
-  uint32_t pad0, pad1;
+  uint32_t ktop;    // key of histogram bin 0 (bin b counts key ktop - b)
+  uint32_t pad;
 };
 static_assert(sizeof(ChunkRec) == 32, "record layout");
 
@@ -145,6 +149,73 @@ __device__ __forceinline__ uint32_t block_max_u(uint32_t v, uint32_t* scratch) {
 
 __device__ __forceinline__ SupSums block_sum_sup(SupSums v, MergeShared& sh);
 
+// block_reduce of the statistics that also takes the block max of v (one
+// exchange for both maxima, one for the rebased sums).
+__device__ __forceinline__ Stats block_reduce_vmax(Stats s, float& v, Stats* scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nw = blockDim.x >> 5;
+  float m = s.m, vv = v;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    vv = fmaxf(vv, __shfl_xor_sync(0xffffffffu, vv, o));
+  }
+  if (lane == 0) {
+    scratch[warp].m = m;
+    scratch[warp].c0 = vv;
+  }
+  __syncthreads();
+  m = -kInf;
+  vv = -kInf;
+  for (int w = 0; w < nw; ++w) {
+    m = fmaxf(m, scratch[w].m);
+    vv = fmaxf(vv, scratch[w].c0);
+  }
+  __syncthreads();
+  if (s.c0 != 0.f || s.zr != 0.f) stats_rebase(s, m);
+  float c0 = s.c0, zr = s.zr, a = s.a;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    c0 += __shfl_xor_sync(0xffffffffu, c0, o);
+    zr += __shfl_xor_sync(0xffffffffu, zr, o);
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+  }
+  if (lane == 0) scratch[warp] = Stats{m, c0, zr, a};
+  __syncthreads();
+  Stats t{m, 0.f, 0.f, 0.f};
+  for (int w = 0; w < nw; ++w) {
+    t.c0 += scratch[w].c0;
+    t.zr += scratch[w].zr;
+    t.a += scratch[w].a;
+  }
+  __syncthreads();
+  v = vv;
+  return t;
+}
+
+// Words holding the 16-bit counts [sh, sh + 8) of the 16 counts in lo, hi
+// (sh in 0..7; uniform across the warp, so the selection does not diverge).
+__device__ __forceinline__ void take8(const uint4& lo, const uint4& hi, int sh, uint32_t (&out)[4]) {
+  uint32_t a0, a1, a2, a3, a4;
+  switch (sh >> 1) {
+    case 0: a0 = lo.x; a1 = lo.y; a2 = lo.z; a3 = lo.w; a4 = hi.x; break;
+    case 1: a0 = lo.y; a1 = lo.z; a2 = lo.w; a3 = hi.x; a4 = hi.y; break;
+    case 2: a0 = lo.z; a1 = lo.w; a2 = hi.x; a3 = hi.y; a4 = hi.z; break;
+    default: a0 = lo.w; a1 = hi.x; a2 = hi.y; a3 = hi.z; a4 = hi.w; break;
+  }
+  if (sh & 1) {
+    out[0] = __funnelshift_r(a0, a1, 16);
+    out[1] = __funnelshift_r(a1, a2, 16);
+    out[2] = __funnelshift_r(a2, a3, 16);
+    out[3] = __funnelshift_r(a3, a4, 16);
+  } else {
+    out[0] = a0;
+    out[1] = a1;
+    out[2] = a2;
+    out[3] = a3;
+  }
+}
+
 // f(raw, id) for every element of g[j0, j1) (j0 a multiple of 8), the
 // block's NT threads striding 16-byte vectors read through L2.
 template <int NT, typename F>
@@ -168,7 +239,7 @@ __device__ __forceinline__ void for_each_elem(const uint16_t* g, int j0, int j1,
 // cumulative count (by_mass false) or mass reaches target.  target 0 with
 // by_mass asks for the top-p target of the full mass (p).
 template <int NT>
-__device__ Desc descend_row(const uint16_t* g, int V, float c, float m, float fxs, bool by_mass,
+__device__ __noinline__ Desc descend_row(const uint16_t* g, int V, float c, float m, float fxs, bool by_mass,
                             bool need_mass, u64 target, float p, MergeShared& sh,
                             RadixArrays& ra) {
   uint32_t prefix = 0;
@@ -238,7 +309,7 @@ __device__ Desc descend_row(const uint16_t* g, int V, float c, float m, float fx
 // order; INT_MAX when there are fewer.  Thread t owns a contiguous run of
 // every segment, so a block scan of the runs' counts orders them.
 template <int NT>
-__device__ int32_t tie_scan(const uint16_t* g, int j0, int j1, uint32_t t, int need,
+__device__ __noinline__ int32_t tie_scan(const uint16_t* g, int j0, int j1, uint32_t t, int need,
                             MergeShared& sh) {
   constexpr int kRun = 256;  // elements per thread and segment (multiple of 8)
   if (threadIdx.x == 0) sh.tie_cut = INT_MAX;
@@ -296,50 +367,151 @@ __device__ __forceinline__ SupSums block_sum_sup(SupSums v, MergeShared& sh) {
   return t;
 }
 
-// Pass b of a chunk: count each element whose bin b = kmax - key lies below
-// nbw.  MODE 1 (every kept key is a positive non-zero value): b = rmax - r;
-// MODE 2 (the chunk max is negative): b = r - rmax; MODE 0: the key map.
-// Out-of-window raw values wrap to huge bins in modes 1 and 2.  CNTY also
-// counts the elements tied with key ky whose id is below y.
-template <int MODE, bool CNTY>
-__device__ __forceinline__ uint32_t hist_pass(const uint4* v4, int nv, int j0, uint32_t kmax,
-                                              uint32_t rmax, uint32_t nbw, uint32_t ky, int y,
-                                              uint32_t* hist) {
-  uint32_t ylt = 0;
-  auto one = [&](uint32_t r, int id) {
-    uint32_t b;
+// Per-thread state of the chunk pass: running max (value vr, u units mr),
+// the count of max-valued elements, packed sums of 2^(u - mr) and
+// (u - mr) 2^(u - mr) over the others, the target's earlier ties, and
+// whether an element lay above the histogram's top key.
+struct ChunkAcc {
+  float vr, mr;
+  uint32_t c0, ylt, ovf;
+  f32x2 z2, a2;
+};
+
+// The chunk pass over 16-byte vectors: online statistics (a vector that
+// raises the running max rebases the sums) and, with HIST, the window
+// histogram: each element whose bin b = ktop - key lies below nbw is
+// counted.  MODE 1 (every kept key is a positive non-zero value):
+// b = rtop - r; MODE 2 (every kept key is a negative value): b = r - rtop;
+// MODE 0: the key map.  Raw values outside the window wrap to huge bins in
+// modes 1 and 2.  With CNTY the elements tied with key ky whose id is below
+// y are counted.  The thread's first-round vectors q1 are already loaded.
+template <int MODE, bool HIST, bool CNTY>
+__device__ __forceinline__ void chunk_pass(const uint4 (&q1)[kRound], const uint4* v4, int nv,
+                                           int j0, float c, uint32_t ktop, uint32_t rtop,
+                                           uint32_t nbw, uint32_t ky, int y, uint32_t* hist,
+                                           ChunkAcc& acc) {
+  const f32x2 c2 = pack2(c, c);
+  auto bin = [&](uint32_t r) -> uint32_t {
     if constexpr (MODE == 1)
-      b = rmax - r;
+      return rtop - r;
     else if constexpr (MODE == 2)
-      b = r - rmax;
+      return r - rtop;
     else
-      b = kmax - bf16_key(r);
-    if (b < nbw) atomicAdd(&hist[b], 1u);
-    if constexpr (CNTY) ylt += static_cast<uint32_t>(bf16_key(r) == ky) & static_cast<uint32_t>(id < y);
+      return ktop - bf16_key(r);
   };
   auto vec = [&](const uint4& q, int vi) {
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    const int id = j0 + vi * 8;
+    const uint32_t mv = bmax2(bmax2(q.x, q.y), bmax2(q.z, q.w));
+    const float vm = fmaxf(__uint_as_float(mv << 16), __uint_as_float(mv & 0xFFFF0000u));
+    if (vm >= acc.vr) {
+      // rare: the vector holds the running max, or raises it
+      if (vm > acc.vr) {
+        const float mn = __fmul_rn(vm, c);
+        if (acc.vr != -kInf) {
+          // rebase onto the new max: the old max-valued elements join the rest
+          float z0, z1, a0, a1;
+          unpack2(acc.z2, z0, z1);
+          unpack2(acc.a2, a0, a1);
+          const float f = ex2(acc.mr - mn);
+          const float z = static_cast<float>(acc.c0) + z0 + z1;
+          acc.z2 = pack2(f * z, 0.f);
+          acc.a2 = pack2(f * fmaf(acc.mr - mn, z, a0 + a1), 0.f);
+        }
+        acc.c0 = 0;
+        acc.vr = vm;
+        acc.mr = mn;
+        if constexpr (HIST) {
+          if (bf16_key(__float_as_uint(vm) >> 16) > ktop) acc.ovf = 1;
+        }
+      }
+      // max-valued elements are counted apart (by value)
+      float zs = 0.f, as = 0.f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      one(w[i] & 0xFFFFu, id + 2 * i);
-      one(w[i] >> 16, id + 2 * i + 1);
+      for (int i = 0; i < 8; ++i) {
+        const float x = __uint_as_float(i & 1 ? w[i >> 1] & 0xFFFF0000u : w[i >> 1] << 16);
+        if (x == acc.vr) {
+          ++acc.c0;
+        } else {
+          const float d = fmaf(x, c, -acc.mr);
+          const float e = ex2(d);
+          zs += e;
+          as = fmaf(d, e, as);
+        }
+      }
+      acc.z2 = add2(acc.z2, pack2(zs, 0.f));
+      acc.a2 = add2(acc.a2, pack2(as, 0.f));
+    } else {
+      // every element lies below the running max
+      const f32x2 nm2 = pack2(-acc.mr, -acc.mr);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const f32x2 d2 = fma2(pack2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u)), c2, nm2);
+        float d0, d1;
+        unpack2(d2, d0, d1);
+        const f32x2 e2 = pack2(ex2(d0), ex2(d1));
+        acc.z2 = add2(acc.z2, e2);
+        acc.a2 = fma2(d2, e2, acc.a2);
+      }
+    }
+    if constexpr (HIST) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t r0 = w[i] & 0xFFFFu, r1 = w[i] >> 16;
+        const uint32_t b0 = bin(r0), b1 = bin(r1);
+        if (b0 < nbw) atomicAdd(&hist[b0], 1u);
+        if (b1 < nbw) atomicAdd(&hist[b1], 1u);
+        if constexpr (CNTY) {
+          const int id = j0 + vi * 8 + 2 * i;
+          acc.ylt += static_cast<uint32_t>(bf16_key(r0) == ky) & static_cast<uint32_t>(id < y);
+          acc.ylt += static_cast<uint32_t>(bf16_key(r1) == ky) & static_cast<uint32_t>(id + 1 < y);
+        }
+      }
     }
   };
-  int v = threadIdx.x;
-  for (; v + (kUnroll - 1) * kCT < nv; v += kUnroll * kCT) {
-    uint4 q[kUnroll];
+  // rounds of kRound vectors per thread, one copy of the loop body; the
+  // first round's vectors arrive preloaded
+  uint4 q[kRound];
 #pragma unroll
-    for (int k = 0; k < kUnroll; ++k) q[k] = __ldcg(v4 + v + k * kCT);
+  for (int k = 0; k < kRound; ++k) q[k] = q1[k];
+  for (int v0 = threadIdx.x;;) {
 #pragma unroll
-    for (int k = 0; k < kUnroll; ++k) vec(q[k], v + k * kCT);
+    for (int k = 0; k < kRound; ++k)
+      if (v0 + k * kCT < nv) vec(q[k], v0 + k * kCT);
+    v0 += kRound * kCT;
+    if (v0 >= nv) break;
+#pragma unroll
+    for (int k = 0; k < kRound; ++k) q[k] = v0 + k * kCT < nv ? __ldg(v4 + v0 + k * kCT) : make_uint4(0, 0, 0, 0);
   }
-  for (; v < nv; v += kCT) vec(__ldcg(v4 + v), v);
-  return ylt;
+}
+
+// Re-count the chunk's window histogram below its exact max key (after an
+// element rose above the first estimate of the top), from L2.
+__device__ __noinline__ void chunk_rehist(const uint16_t* g, int j0, int j1, uint32_t ktop,
+                                          uint32_t nbw, uint32_t* hist) {
+  for (int b = threadIdx.x; b < kCW; b += kCT) hist[b] = 0u;
+  __syncthreads();
+  for_each_elem<kCT>(g, j0, j1, [&](uint32_t r, int) {
+    const uint32_t b = ktop - bf16_key(r);
+    if (b < nbw) atomicAdd(&hist[b], 1u);
+  });
+  __syncthreads();
+}
+
+// Smallest key in [lo, hi] whose u-offset from m reaches dlo (hi if none).
+__device__ __forceinline__ uint32_t key_at_level(uint32_t lo, uint32_t hi, float c, float m,
+                                                 float dlo) {
+  while (lo < hi) {
+    const uint32_t mid = lo + ((hi - lo) >> 1);
+    if (key_u(mid, c) - m >= dlo)
+      hi = mid;
+    else
+      lo = mid + 1;
+  }
+  return lo;
 }
 
 __global__ void __launch_bounds__(kCT, 8) score_chunk_kernel(ScoreParams P, SplitArgs Q) {
-  __shared__ __align__(16) uint32_t hist[kSelWin];
+  __shared__ __align__(16) uint32_t hist[kCW];
   __shared__ ChunkShared sh;
   pdl_launch_dependents();
 
@@ -363,126 +535,95 @@ __global__ void __launch_bounds__(kCT, 8) score_chunk_kernel(ScoreParams P, Spli
   const bool any_filter = use_k || use_p || use_minp;
 
   if (any_filter)
-    for (int b = tid; b < kSelWin; b += kCT) hist[b] = 0u;
+    for (int b = tid; b < kCW; b += kCT) hist[b] = 0u;
 
-  // ---- pass a (HBM): online statistics.  Each thread keeps the running max
-  // (value vr, u-units mr), the count of max-valued elements c0 and packed
-  // sums of 2^(u - mr) and (u - mr) 2^(u - mr) over the others.
-  float vr = -kInf, mr = -kInf;
-  uint32_t c0 = 0;
-  f32x2 z2 = pack2(0.f, 0.f), a2 = pack2(0.f, 0.f);
-  const f32x2 c2 = pack2(c, c);
-  auto stats_vec = [&](const uint4& q) {
-    const uint32_t mv = bmax2(bmax2(q.x, q.y), bmax2(q.z, q.w));
-    const float vm = fmaxf(__uint_as_float(mv << 16), __uint_as_float(mv & 0xFFFF0000u));
-    if (vm > vr) {  // rare after the first few vectors
-      const float mn = __fmul_rn(vm, c);
-      if (vr != -kInf) {
-        // rebase onto the new max: the old max-valued elements join the rest
-        float z0, z1, a0, a1;
-        unpack2(z2, z0, z1);
-        unpack2(a2, a0, a1);
-        const float f = ex2(mr - mn);
-        const float z = static_cast<float>(c0) + z0 + z1;
-        z2 = pack2(f * z, 0.f);
-        a2 = pack2(f * fmaf(mr - mn, z, a0 + a1), 0.f);
-      }
-      c0 = 0;
-      vr = vm;
-      mr = mn;
-    }
-    const f32x2 m2 = pack2(mr, mr);
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+  // ---- first round: each thread's first kRound vectors, and their block
+  // max m1 (a lower bound of the chunk max that fixes the histogram window)
+  uint4 q1[kRound];
+  uint32_t mx = 0xFF80FF80u;  // (-inf, -inf)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float x0 = __uint_as_float(w[i] << 16), x1 = __uint_as_float(w[i] & 0xFFFF0000u);
-      const f32x2 d2 = sub2(mul2(pack2(x0, x1), c2), m2);
-      float d0, d1;
-      unpack2(d2, d0, d1);
-      // max-valued elements are counted apart (compared by value: the packed
-      // product need not round like the scalar one that made mr)
-      const bool t0 = x0 == vr, t1 = x1 == vr;
-      c0 += static_cast<uint32_t>(t0) + static_cast<uint32_t>(t1);
-      const f32x2 e2 = pack2(t0 ? 0.f : ex2(d0), t1 ? 0.f : ex2(d1));
-      z2 = add2(z2, e2);
-      a2 = fma2(d2, e2, a2);
-    }
-  };
-  int v = tid;
-  for (; v + (kUnroll - 1) * kCT < nv; v += kUnroll * kCT) {
-    uint4 q[kUnroll];
-#pragma unroll
-    for (int k = 0; k < kUnroll; ++k) q[k] = __ldg(v4 + v + k * kCT);
-#pragma unroll
-    for (int k = 0; k < kUnroll; ++k) stats_vec(q[k]);
+  for (int k = 0; k < kRound; ++k) {
+    const int v = tid + k * kCT;
+    q1[k] = v < nv ? __ldg(v4 + v) : make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u);
+    mx = bmax2(mx, bmax2(bmax2(q1[k].x, q1[k].y), bmax2(q1[k].z, q1[k].w)));
   }
-  for (; v < nv; v += kCT) stats_vec(__ldg(v4 + v));
-  Stats st;
-  {
-    float z0, z1, a0, a1;
-    unpack2(z2, z0, z1);
-    unpack2(a2, a0, a1);
-    st = Stats{mr, static_cast<float>(c0), z0 + z1, a0 + a1};
-  }
-  // ragged tail (the last chunk of a row whose length is not a multiple of 8)
-  for (int j = j0 + nv * 8 + tid; j < j1; j += kCT) {
-    float u[1] = {__fmul_rn(value_of(grow[j]), c)};
-    vr = fmaxf(vr, value_of(grow[j]));
-    stats_add(st, u);
-  }
-  st = block_reduce(st, sh.wst);
-  const float vmax = block_max(vr, sh.fred);
+  const float m1 = block_max(fmaxf(__uint_as_float(mx << 16), __uint_as_float(mx & 0xFFFF0000u)), sh.fred);
 
-  // ---- pass b (L2): window histogram of the filtered rows
-  uint32_t nb = 0, ylt = 0;
-  if (any_filter) {
-    const uint32_t kmax = bf16_key(__float_as_uint(vmax) >> 16);
-    // Elements below these levels (relative to the chunk max, hence also to
-    // the row max) never enter the support: min-p keeps 2^(u - m) >= min_p;
-    // top-p alone keeps a prefix whose complement holds at most (1 - p) of
-    // the mass, while all elements with 2^(u - m) < (1 - p) / (2 V) hold less
-    // than half of that (the row total is at least 1).  One more octave of
-    // margin each.
+  ChunkAcc acc{m1, __fmul_rn(m1, c), 0u, 0u, 0u, pack2(0.f, 0.f), pack2(0.f, 0.f)};
+  uint32_t ktop = 0, nbw = 0, ky = 0xFFFFFFFFu;
+  const int y = P.targets[row];
+  const bool cnty = any_filter && y > j0 && y < j1;
+  if (!any_filter) {
+    chunk_pass<0, false, false>(q1, v4, nv, j0, c, 0u, 0u, 0u, 0u, 0, hist, acc);
+  } else {
+    // window: keys ktop - nbw + 1 .. ktop, ktop kHead keys above m1's key
+    const uint32_t k1 = bf16_key(__float_as_uint(m1) >> 16);
+    ktop = min(k1 + static_cast<uint32_t>(kHead), KeyTraits<uint16_t>::kInfKey);
+    uint32_t kbot = ktop >= static_cast<uint32_t>(kCW - 1) ? ktop - (kCW - 1) : 0u;
+    // Elements below these levels (relative to m1, hence also to the row
+    // max) never enter the support: min-p keeps 2^(u - m) >= min_p; top-p
+    // alone keeps a prefix whose complement holds at most (1 - p) of the
+    // mass, while all elements with 2^(u - m) < (1 - p) / (2 V) hold less than
+    // half of that (the row total is at least 1).  One more octave of margin.
     float dlo = -kInf;
     if (use_minp) dlo = log2f(mp) - 1.f;
     if (use_p && !use_k && pp > 0.f) dlo = fmaxf(dlo, log2f((1.f - pp) / static_cast<float>(V)) - 2.f);
-    uint32_t nbw = kSelWin;
-    if (dlo > -kInf && isfinite(st.m)) {
-      // smallest key at or above the level: bins b < kmax - kskip + 1
-      uint32_t lo = kmax >= static_cast<uint32_t>(kSelWin - 1) ? kmax - (kSelWin - 1) : 0u, hi = kmax;
-      while (lo < hi) {
-        const uint32_t mid = lo + ((hi - lo) >> 1);
-        if (key_u(mid, c) - st.m >= dlo)
-          hi = mid;
-        else
-          lo = mid + 1;
-      }
-      nbw = kmax - lo + 1;
-    }
-    // the chunk holding the target also counts the target's earlier ties
-    const int y = P.targets[row];
-    const bool cnty = y > j0 && y < j1;
-    const uint32_t ky = cnty ? bf16_key(grow[y]) : 0xFFFFFFFFu;
-    const uint32_t rmax = __float_as_uint(vmax) >> 16;
-    const int mode = kmax - (nbw - 1) > 0x7FFFu ? 1 : (kmax < 0x7FFFu ? 2 : 0);
+    if (dlo > -kInf && isfinite(acc.mr)) kbot = key_at_level(kbot, k1, c, acc.mr, dlo);
+    nbw = ktop - kbot + 1;
+    if (cnty) ky = bf16_key(grow[y]);
+    const int mode = kbot > 0x7FFFu ? 1 : (ktop < 0x7FFFu ? 2 : 0);
+    const uint32_t rtop = mode == 1 ? ktop - 0x7FFFu : 0xFFFFu - ktop;
     if (cnty) {
-      if (mode == 1) ylt = hist_pass<1, true>(v4, nv, j0, kmax, rmax, nbw, ky, y, hist);
-      else if (mode == 2) ylt = hist_pass<2, true>(v4, nv, j0, kmax, rmax, nbw, ky, y, hist);
-      else ylt = hist_pass<0, true>(v4, nv, j0, kmax, rmax, nbw, ky, y, hist);
+      if (mode == 1) chunk_pass<1, true, true>(q1, v4, nv, j0, c, ktop, rtop, nbw, ky, y, hist, acc);
+      else if (mode == 2) chunk_pass<2, true, true>(q1, v4, nv, j0, c, ktop, rtop, nbw, ky, y, hist, acc);
+      else chunk_pass<0, true, true>(q1, v4, nv, j0, c, ktop, rtop, nbw, ky, y, hist, acc);
     } else {
-      if (mode == 1) hist_pass<1, false>(v4, nv, j0, kmax, rmax, nbw, ky, y, hist);
-      else if (mode == 2) hist_pass<2, false>(v4, nv, j0, kmax, rmax, nbw, ky, y, hist);
-      else hist_pass<0, false>(v4, nv, j0, kmax, rmax, nbw, ky, y, hist);
+      if (mode == 1) chunk_pass<1, true, false>(q1, v4, nv, j0, c, ktop, rtop, nbw, ky, y, hist, acc);
+      else if (mode == 2) chunk_pass<2, true, false>(q1, v4, nv, j0, c, ktop, rtop, nbw, ky, y, hist, acc);
+      else chunk_pass<0, true, false>(q1, v4, nv, j0, c, ktop, rtop, nbw, ky, y, hist, acc);
     }
-    for (int j = j0 + nv * 8 + tid; j < j1; j += kCT) {
-      const uint32_t key = bf16_key(grow[j]);
-      if (kmax - key < nbw) atomicAdd(&hist[kmax - key], 1u);
+  }
+  Stats st;
+  {
+    float z0, z1, a0, a1;
+    unpack2(acc.z2, z0, z1);
+    unpack2(acc.a2, a0, a1);
+    st = Stats{acc.mr, static_cast<float>(acc.c0), z0 + z1, a0 + a1};
+    if (acc.vr == -kInf && acc.c0 == 0 && z0 + z1 == 0.f) st = stats_empty();
+  }
+  // ragged tail (the last chunk of a row whose length is not a multiple of 8)
+  float vr = acc.vr;
+  uint32_t ylt = acc.ylt, ovf = acc.ovf;
+  for (int j = j0 + nv * 8 + tid; j < j1; j += kCT) {
+    const uint32_t r = grow[j];
+    const float x = value_of(static_cast<uint16_t>(r));
+    float u[1] = {__fmul_rn(x, c)};
+    vr = fmaxf(vr, x);
+    stats_add(st, u);
+    if (any_filter) {
+      const uint32_t key = bf16_key(r);
+      if (key > ktop) ovf = 1u;
+      if (ktop - key < nbw) atomicAdd(&hist[ktop - key], 1u);
       if (cnty) ylt += static_cast<uint32_t>(key == ky) & static_cast<uint32_t>(j < y);
     }
+  }
+  st = block_reduce_vmax(st, vr, sh.wst);
+  const float vmax = vr;
+
+  uint32_t nb = 0;
+  if (any_filter) {
     if (cnty) ylt = block_sum(ylt, sh.ured);
+    if (__syncthreads_or(ovf != 0u)) {
+      // an element rose above the window: count again below the exact max
+      const uint32_t kx = bf16_key(__float_as_uint(vmax) >> 16);
+      const uint32_t kb = ktop - (nbw - 1);  // keep the same lowest key (clamped)
+      ktop = kx;
+      nbw = kx >= kb ? min(kx - kb + 1, static_cast<uint32_t>(kCW)) : 1u;
+      chunk_rehist(grow, j0, j1, ktop, nbw, hist);
+    }
     __syncthreads();
     uint32_t hi = 0;
-    for (int b = tid; b < kSelWin; b += kCT)
+    for (int b = tid; b < kCW; b += kCT)
       if (hist[b]) hi = b + 1;
     nb = block_max_u(hi, sh.ured);
     const int64_t slot = static_cast<int64_t>(row) * Q.S + cs;
@@ -501,7 +642,8 @@ __global__ void __launch_bounds__(kCT, 8) score_chunk_kernel(ScoreParams P, Spli
     r.a = st.a;
     r.nb = nb;
     r.ylt = ylt;
-    r.pad0 = r.pad1 = 0;
+    r.ktop = ktop;
+    r.pad = 0;
     Q.recs[static_cast<int64_t>(row) * Q.S + cs] = r;
   }
 }
@@ -540,10 +682,9 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
     stats_merge(st, t);
     vr = fmaxf(vr, h0.x);
     sh.cnb[k] = h1.x;
-    sh.coff[k] = static_cast<int32_t>(bf16_key(__float_as_uint(h0.x) >> 16));  // chunk kmax for now
+    sh.coff[k] = static_cast<int32_t>(h1.z);  // histogram top key for now
   }
-  st = block_reduce(st, sh.wst);
-  vr = block_max(vr, sh.fred);
+  st = block_reduce_vmax(st, vr, sh.wst);
 
   const bool nonfinite = !stats_finite(st) || !isfinite(vr);
   const float mr = st.m;  // = fl(vr c)
@@ -571,42 +712,55 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
     w.c = c;
     w.m = mr;
     w.fxs = fxs;
-    // merged window: hist[key - klo]; chunk bin b holds key kmax_k - b
+    // merged window: hist[key - klo]; chunk bin b holds key ktop_k - b
     for (int k = tid; k < S; k += kMT) {
-      const int off = static_cast<int>(kmr) - sh.coff[k];  // >= 0
-      sh.coff[k] = w.nbins - 1 - off;  // row bin of chunk bin 0 (negative: none)
+      // a chunk's histogram top is at most kHead keys above the row max
+      const int off = static_cast<int>(kmr) - sh.coff[k];
+      sh.coff[k] = w.nbins - 1 - off;  // row bin of chunk bin 0
     }
-    for (int b = tid; b < kSelWin; b += kMT) hist[b] = 0u;
-    __syncthreads();
+    __syncthreads();  // coff / cnb
     {
-      // thread t adds vector t (bins 8t .. 8t+7) of every chunk histogram
-      static_assert(kSelWin / 8 == kMT, "one histogram vector per merge thread");
+      // Thread t builds row bins [8t, 8t + 8).  Row bin i holds chunk bin
+      // coff_k - i, so from chunk k it needs the descending run of chunk bins
+      // s .. s + 7 with s = coff_k - 8t - 7: two aligned 16-byte vectors,
+      // and the run's offset inside them, s mod 8, is the same for every
+      // thread.  Counts are summed in registers: no atomics.
+      static_assert(kSelWin / 8 == kMT, "eight row bins per merge thread");
+      constexpr int kB = 4;  // chunks per batch of loads
       const uint4* hrow = reinterpret_cast<const uint4*>(Q.hists + static_cast<int64_t>(row) * S * kHistWords);
-      for (int k0 = 0; k0 < S; k0 += 8) {
-        uint4 q[8];
-        int base[8];
+      uint32_t acc[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      for (int k0 = 0; k0 < S; k0 += kB) {
+        uint4 lo[kB], hi[kB];
+        int sh8[kB];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < kB; ++u) {
           const int k = k0 + u;
-          base[u] = -1;
-          q[u] = make_uint4(0, 0, 0, 0);
-          if (k < S && static_cast<uint32_t>(tid * 8) < sh.cnb[k] && sh.coff[k] - tid * 8 >= 0) {
-            base[u] = sh.coff[k] - tid * 8;  // row bin of this vector's first count
-            q[u] = __ldcg(hrow + static_cast<int64_t>(k) * (kHistWords / 4) + tid);
+          lo[u] = hi[u] = make_uint4(0, 0, 0, 0);
+          sh8[u] = 0;
+          if (k < S) {
+            const int sb = sh.coff[k] - 8 * tid - 7;
+            const int va = sb >> 3;  // floor
+            const int nvk = static_cast<int>((sh.cnb[k] + 7) >> 3);
+            const uint4* hk = hrow + static_cast<int64_t>(k) * (kHistWords / 4);
+            if (va >= 0 && va < nvk) lo[u] = __ldcg(hk + va);
+            if (va + 1 >= 0 && va + 1 < nvk) hi[u] = __ldcg(hk + va + 1);
+            sh8[u] = sb & 7;
           }
         }
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          if (base[u] < 0) continue;
-          const uint32_t wd[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+        for (int u = 0; u < kB; ++u) {
+          uint32_t run[4];
+          take8(lo[u], hi[u], sh8[u], run);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint32_t cnt = (wd[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu;
-            const int rb = base[u] - i;
-            if (cnt && rb >= 0) atomicAdd(&hist[rb], cnt);
+          for (int jj = 0; jj < 8; ++jj) {
+            const int j2 = 7 - jj;  // row bin 8t + jj holds chunk bin s + 7 - jj
+            acc[jj] += (run[j2 >> 1] >> ((j2 & 1) * 16)) & 0xFFFFu;
           }
         }
       }
+      uint4* h4 = reinterpret_cast<uint4*>(hist);
+      h4[2 * tid] = make_uint4(acc[0], acc[1], acc[2], acc[3]);
+      h4[2 * tid + 1] = make_uint4(acc[4], acc[5], acc[6], acc[7]);
     }
     __syncthreads();
 
@@ -630,15 +784,14 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
       if (win_ok && use_p) {
         double mass1;
         if (use_k) {
-          const u64 fx_t = dk.at_cnt ? dk.at_mass / dk.at_cnt : 0;
-          mass1 = static_cast<double>(dk.above_mass + ck * fx_t);
+          mass1 = static_cast<double>(dk.above_mass + ck * bin_fx(w, dk.key));
         } else {
           mass1 = (static_cast<double>(st.c0) + static_cast<double>(st.zr)) * static_cast<double>(fxs);
         }
         const u64 tp = topp_target(pp, mass1);
         win_ok = win_search<kMT>(w, true, tp, dp, sh.sel);
         if (win_ok) {
-          u64 cp = topp_ties(dp, tp);
+          u64 cp = topp_ties(dp, tp, bin_fx(w, dp.key));
           if (use_k && dp.key == tkey && cp > ck) cp = ck;
           tkey = dp.key;
           cnum = cp;
@@ -658,10 +811,10 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
           all_ties = ck2 >= d.at_cnt;
           have_t = true;
           if (use_p) {
-            const u64 fx_t = d.at_cnt ? d.at_mass / d.at_cnt : 0;
+            const u64 fx_t = key_fx<uint16_t>(d.key, c, mr, fxs);
             const u64 tp = topp_target(pp, static_cast<double>(d.above_mass + ck2 * fx_t));
             const Desc e = descend_row<kMT>(grow, V, c, mr, fxs, true, true, tp, pp, sh, ra);
-            u64 cp = topp_ties(e, tp);
+            u64 cp = topp_ties(e, tp, key_fx<uint16_t>(e.key, c, mr, fxs));
             if (e.key == tkey && cp > ck2) cp = ck2;
             tkey = e.key;
             cnum = cp;
@@ -669,7 +822,7 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
           }
         } else {
           const Desc e = descend_row<kMT>(grow, V, c, mr, fxs, true, true, 0ull, pp, sh, ra);
-          const u64 cp = topp_ties(e, sh.ulred[1]);
+          const u64 cp = topp_ties(e, sh.ulred[1], key_fx<uint16_t>(e.key, c, mr, fxs));
           tkey = e.key;
           cnum = cp;
           all_ties = cp >= e.at_cnt;
@@ -691,10 +844,13 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
     from_bins = win_ok && tkey >= w.klo;
     SupSums sums{0u, 0u, 0u, 0.f, 0.f};
     if (from_bins) {
-      const int per = (w.nbins + kMT - 1) / kMT;
-      const int i0 = tid * per, i1 = min(w.nbins, i0 + per);
-      for (int i = i0; i < i1; ++i) {
-        const uint32_t cnt = hist[i];
+      const uint4 ha = reinterpret_cast<const uint4*>(hist)[2 * tid];
+      const uint4 hb = reinterpret_cast<const uint4*>(hist)[2 * tid + 1];
+      const uint32_t hv[8] = {ha.x, ha.y, ha.z, ha.w, hb.x, hb.y, hb.z, hb.w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = 8 * tid + j;
+        const uint32_t cnt = i < w.nbins ? hv[j] : 0u;
         const uint32_t key = w.klo + i;
         if (cnt && key > tkey) {
           const float d = key_u(key, c) - mr;
@@ -757,8 +913,7 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
             sh.found_chunk = -1;
             int before = 0;
             for (int k = 0; k < S && sh.found_chunk < 0; ++k) {
-              const float vk = __ldcg(&rr[k].vmax);
-              const uint32_t kk2 = bf16_key(__float_as_uint(vk) >> 16);
+              const uint32_t kk2 = __ldcg(&rr[k].ktop);
               const uint32_t nbk = __ldcg(&rr[k].nb);
               uint32_t cnt = 0;
               if (kk2 >= tkey && kk2 - tkey < nbk) {
@@ -798,7 +953,7 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
         if (k == cy) {
           part += __ldcg(&rr[k].ylt);
         } else {
-          const uint32_t kk2 = bf16_key(__float_as_uint(__ldcg(&rr[k].vmax)) >> 16);
+          const uint32_t kk2 = __ldcg(&rr[k].ktop);
           const uint32_t nbk = __ldcg(&rr[k].nb);
           if (kk2 >= tkey && kk2 - tkey < nbk) {
             const uint32_t b = kk2 - tkey;

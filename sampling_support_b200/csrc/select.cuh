@@ -133,20 +133,28 @@ __device__ __forceinline__ u64 bin_fx(const Window& w, uint32_t key) {
 // Search the window from the largest key for the bin where the cumulative
 // count (by_mass false) or fixed-point mass first reaches need (>= 1).
 // False when the whole window holds less than need.  Each thread owns a run
-// of at most 8 consecutive bins, whose masses it keeps in registers.
+// of 8 consecutive bins (hist 16-byte aligned, kSelWin entries readable),
+// whose masses it keeps in registers.
 template <int NT>
-__device__ bool win_search(const Window& w, bool by_mass, u64 need, Desc& out,
+__device__ __noinline__ bool win_search(const Window& w, bool by_mass, u64 need, Desc& out,
                            SelShared<NT / 32>& sh) {
   constexpr int kPer = (kSelWin + NT - 1) / NT;
   static_assert(kPer <= 8, "window search keeps a thread's bins in registers");
+  static_assert(kPer == 8, "two 16-byte reads per thread");
   const int i0 = threadIdx.x * kPer;
   uint32_t cnt[kPer];
   u64 fx[kPer];
   u64 lc = 0, lm = 0;
+  {
+    const uint4 ha = reinterpret_cast<const uint4*>(w.hist)[2 * threadIdx.x];
+    const uint4 hb = reinterpret_cast<const uint4*>(w.hist)[2 * threadIdx.x + 1];
+    cnt[0] = ha.x; cnt[1] = ha.y; cnt[2] = ha.z; cnt[3] = ha.w;
+    cnt[4] = hb.x; cnt[5] = hb.y; cnt[6] = hb.z; cnt[7] = hb.w;
+  }
 #pragma unroll
   for (int j = 0; j < kPer; ++j) {
     const int i = i0 + j;
-    cnt[j] = i < w.nbins ? w.hist[i] : 0u;
+    if (i >= w.nbins) cnt[j] = 0u;
     fx[j] = cnt[j] ? static_cast<u64>(cnt[j]) * bin_fx(w, w.klo + i) : 0ull;
     lc += cnt[j];
     lm += fx[j];
@@ -249,12 +257,27 @@ __device__ inline void scan_bins(const uint32_t* gcnt, const u64* gmass, bool by
   above_mass = am;
 }
 
-// Number of the top-p tie group's elements to keep: enough that the mass
-// reaches the target (at least one, at most the group).
-__device__ __forceinline__ u64 topp_ties(const Desc& d, u64 target) {
-  const u64 fxe = d.at_cnt ? d.at_mass / d.at_cnt : 0;
+// Fixed-point mass of one element with this key: 2^(u - m) 2^fx_shift.
+template <typename Raw>
+__device__ __forceinline__ u64 key_fx(uint32_t key, float c, float m, float fxs) {
+  return __float2ull_rn(ex2(__fmul_rn(KeyTraits<Raw>::decode(key), c) - m) * fxs);
+}
+
+// Number of the top-p tie group's elements to keep (each of fixed-point
+// mass fxe): enough that the mass reaches the target, at least one, at most
+// the group.  The quotient comes from one double division, made exact by
+// an integer correction (products stay below 2^64).
+__device__ __forceinline__ u64 topp_ties(const Desc& d, u64 target, u64 fxe) {
   const u64 need = target > d.above_mass ? target - d.above_mass : 0;
-  u64 cp = fxe ? (need + fxe - 1) / fxe : d.at_cnt;
+  u64 cp = d.at_cnt;
+  if (fxe != 0) {
+    const double q = ceil(static_cast<double>(need) / static_cast<double>(fxe));
+    cp = q >= static_cast<double>(d.at_cnt) + 1.0 ? d.at_cnt + 1 : static_cast<u64>(q);
+    if (cp > 0 && (cp - 1) * fxe >= need)
+      --cp;
+    else if (cp * fxe < need)
+      ++cp;
+  }
   if (cp < 1) cp = 1;
   if (cp > d.at_cnt) cp = d.at_cnt;
   return cp;
