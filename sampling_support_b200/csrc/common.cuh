@@ -102,8 +102,16 @@ __device__ __forceinline__ Stats stats_empty() { return {-kInf, 0.f, 0.f, 0.f}; 
 
 __device__ __forceinline__ float stats_z(const Stats& s) { return s.c0 + s.zr; }
 
+// log2 Z = log2 c0 + log2(1 + t), t = zr / c0: for t < 2^-6 the series
+// t - t^2/2 + t^3/3 - t^4/4 + t^5/5 (remainder below t^6/6 < 2^-38) keeps
+// full precision of a small t; above, log2 of the rounded sum c0 + zr is
+// within 2^-24 / ln 2 absolute, under 4e-6 relative to log2 Z.
 __device__ __forceinline__ float stats_log2z(const Stats& s) {
-  return log2f(s.c0) + log1pf(s.zr / s.c0) * kLog2e;
+  const float t = s.zr / s.c0;
+  const bool small = t < 0.015625f;
+  const float l = log2f(small ? s.c0 : s.c0 + s.zr);
+  const float p = fmaf(fmaf(fmaf(fmaf(t, 0.2f, -0.25f), t, 1.f / 3.f), t, -0.5f), t, 1.f);
+  return small ? fmaf(t * p, kLog2e, l) : l;
 }
 
 // True when the statistics describe only finite values.
