@@ -367,6 +367,15 @@ __device__ __forceinline__ SupSums block_sum_sup(SupSums v, MergeShared& sh) {
   return t;
 }
 
+// One shared-memory count increment at the 32-bit shared address a, only
+// when c holds (a predicated reduction, no branch around it).
+__device__ __forceinline__ void red_inc_if(uint32_t a, bool c) {
+  asm volatile(
+      "{\n .reg .pred q;\n setp.ne.u32 q, %1, 0;\n @q red.shared.add.u32 [%0], 1;\n}\n" ::"r"(a),
+      "r"(static_cast<uint32_t>(c))
+      : "memory");
+}
+
 // Per-thread state of the chunk pass: running max (value vr, u units mr),
 // the count of max-valued elements, packed sums of 2^(u - mr) and
 // (u - mr) 2^(u - mr) over the others, the target's earlier ties, and
@@ -391,6 +400,7 @@ __device__ __forceinline__ void chunk_pass(const uint4 (&q1)[kRound], const uint
                                            uint32_t nbw, uint32_t ky, int y, uint32_t* hist,
                                            ChunkAcc& acc) {
   const f32x2 c2 = pack2(c, c);
+  const uint32_t hist_s = smem_addr(hist);
   auto bin = [&](uint32_t r) -> uint32_t {
     if constexpr (MODE == 1)
       return rtop - r;
@@ -458,8 +468,8 @@ __device__ __forceinline__ void chunk_pass(const uint4 (&q1)[kRound], const uint
       for (int i = 0; i < 4; ++i) {
         const uint32_t r0 = w[i] & 0xFFFFu, r1 = w[i] >> 16;
         const uint32_t b0 = bin(r0), b1 = bin(r1);
-        if (b0 < nbw) atomicAdd(&hist[b0], 1u);
-        if (b1 < nbw) atomicAdd(&hist[b1], 1u);
+        red_inc_if(hist_s + (b0 << 2), b0 < nbw);
+        red_inc_if(hist_s + (b1 << 2), b1 < nbw);
         if constexpr (CNTY) {
           const int id = j0 + vi * 8 + 2 * i;
           acc.ylt += static_cast<uint32_t>(bf16_key(r0) == ky) & static_cast<uint32_t>(id < y);
@@ -844,13 +854,9 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
     from_bins = win_ok && tkey >= w.klo;
     SupSums sums{0u, 0u, 0u, 0.f, 0.f};
     if (from_bins) {
-      const uint4 ha = reinterpret_cast<const uint4*>(hist)[2 * tid];
-      const uint4 hb = reinterpret_cast<const uint4*>(hist)[2 * tid + 1];
-      const uint32_t hv[8] = {ha.x, ha.y, ha.z, ha.w, hb.x, hb.y, hb.z, hb.w};
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = 8 * tid + j;
-        const uint32_t cnt = i < w.nbins ? hv[j] : 0u;
+#pragma unroll 1
+      for (int i = 8 * tid; i < min(w.nbins, 8 * tid + 8); ++i) {
+        const uint32_t cnt = hist[i];
         const uint32_t key = w.klo + i;
         if (cnt && key > tkey) {
           const float d = key_u(key, c) - mr;

@@ -133,31 +133,22 @@ __device__ __forceinline__ u64 bin_fx(const Window& w, uint32_t key) {
 // Search the window from the largest key for the bin where the cumulative
 // count (by_mass false) or fixed-point mass first reaches need (>= 1).
 // False when the whole window holds less than need.  Each thread owns a run
-// of 8 consecutive bins (hist 16-byte aligned, kSelWin entries readable),
-// whose masses it keeps in registers.
+// of NB = ceil(4096 / NT) consecutive bins; loops stay rolled (the search
+// runs once per row, so short code matters more than unrolling), and the one
+// thread whose run holds the crossing walks it again.
 template <int NT>
 __device__ __noinline__ bool win_search(const Window& w, bool by_mass, u64 need, Desc& out,
-                           SelShared<NT / 32>& sh) {
-  constexpr int kPer = (kSelWin + NT - 1) / NT;
-  static_assert(kPer <= 8, "window search keeps a thread's bins in registers");
-  static_assert(kPer == 8, "two 16-byte reads per thread");
-  const int i0 = threadIdx.x * kPer;
-  uint32_t cnt[kPer];
-  u64 fx[kPer];
+                                        SelShared<NT / 32>& sh) {
+  constexpr int NB = (kSelWin + NT - 1) / NT;
+  const int i0 = threadIdx.x * NB, i1 = min(w.nbins, i0 + NB);
   u64 lc = 0, lm = 0;
-  {
-    const uint4 ha = reinterpret_cast<const uint4*>(w.hist)[2 * threadIdx.x];
-    const uint4 hb = reinterpret_cast<const uint4*>(w.hist)[2 * threadIdx.x + 1];
-    cnt[0] = ha.x; cnt[1] = ha.y; cnt[2] = ha.z; cnt[3] = ha.w;
-    cnt[4] = hb.x; cnt[5] = hb.y; cnt[6] = hb.z; cnt[7] = hb.w;
-  }
-#pragma unroll
-  for (int j = 0; j < kPer; ++j) {
-    const int i = i0 + j;
-    if (i >= w.nbins) cnt[j] = 0u;
-    fx[j] = cnt[j] ? static_cast<u64>(cnt[j]) * bin_fx(w, w.klo + i) : 0ull;
-    lc += cnt[j];
-    lm += fx[j];
+#pragma unroll 1
+  for (int i = i0; i < i1; ++i) {
+    const uint32_t cnt = w.hist[i];
+    if (cnt) {
+      lc += cnt;
+      lm += static_cast<u64>(cnt) * bin_fx(w, w.klo + i);
+    }
   }
   u64 ec, em;
   block_suffix_excl<NT>(lc, lm, ec, em, sh);
@@ -167,20 +158,21 @@ __device__ __noinline__ bool win_search(const Window& w, bool by_mass, u64 need,
   const u64 mine = by_mass ? lm : lc;
   if (base < need && need <= base + mine) {
     u64 ac = ec, am = em;
-    bool done = false;
-#pragma unroll
-    for (int j = kPer - 1; j >= 0; --j) {
-      if (!done && cnt[j] && (by_mass ? am + fx[j] : ac + cnt[j]) >= need) {
-        sh.b_key = w.klo + i0 + j;
+#pragma unroll 1
+    for (int i = i1 - 1; i >= i0; --i) {
+      const uint32_t cnt = w.hist[i];
+      const u64 fx = cnt ? static_cast<u64>(cnt) * bin_fx(w, w.klo + i) : 0ull;
+      if (cnt && (by_mass ? am + fx : ac + cnt) >= need) {
+        sh.b_key = w.klo + i;
         sh.b_above_cnt = ac;
         sh.b_above_mass = am;
-        sh.b_at_cnt = cnt[j];
-        sh.b_at_mass = fx[j];
+        sh.b_at_cnt = cnt;
+        sh.b_at_mass = fx;
         sh.b_found = 1;
-        done = true;
+        break;
       }
-      ac += cnt[j];
-      am += fx[j];
+      ac += cnt;
+      am += fx;
     }
   }
   __syncthreads();
