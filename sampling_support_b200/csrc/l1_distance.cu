@@ -12,6 +12,8 @@
 
 #include <mutex>
 
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -67,6 +69,254 @@ __device__ __forceinline__ float dec_grad(uint32_t w, float coef, float ps) {
   return coef * p * (s - ps);
 }
 
+__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
+  const __nv_bfloat162 r = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&a),
+                                   *reinterpret_cast<const __nv_bfloat162*>(&b));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+__device__ __forceinline__ float l1_block_max(float v, float* scratch) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float t = -kInf;
+  for (int w = 0; w < kWarps; ++w) t = fmaxf(t, scratch[w]);
+  __syncthreads();
+  return t;
+}
+
+// Largest of the eight bf16 values of a vector.
+__device__ __forceinline__ float vec_max(const uint4& a) {
+  const uint32_t m = bmax2(bmax2(a.x, a.y), bmax2(a.z, a.w));
+  return fmaxf(__uint_as_float(m << 16), __uint_as_float(m & 0xFFFF0000u));
+}
+
+// Element i of the eight bf16 values in w[4].
+__device__ __forceinline__ float bf16_at(const uint32_t (&w)[4], int i) {
+  return __uint_as_float(i & 1 ? w[i >> 1] & 0xFFFF0000u : w[i >> 1] << 16);
+}
+
+// One element of pass 2: accumulates |p - q| and p sign(p - q) and returns
+// the in-place (p, sign) word (branch-free form of enc_ps).
+__device__ __forceinline__ uint32_t l1_step(float p, float q, float& l1, float& ps) {
+  const float d = p - q;
+  l1 += fabsf(d);
+  const bool pos = d > 0.f, neg = d < 0.f;
+  ps = fmaf(p, pos ? 1.f : (neg ? -1.f : 0.f), ps);
+  return __float_as_uint(p) | (neg ? 0x80000000u : 0u) | (!(pos || neg) ? 0x40000000u : 0u);
+}
+
+// Gradient of one element from its (p, sign) word: k_pos, k_neg, k_zero are
+// coef (s - sum p s) for s = +1, -1, 0.
+__device__ __forceinline__ float l1_grad(uint32_t w, float k_pos, float k_neg, float k_zero) {
+  const float p = __uint_as_float(w & 0x3FFFFFFFu);
+  return p * ((w & 0x40000000u) ? k_zero : ((w & 0x80000000u) ? k_neg : k_pos));
+}
+
+// bf16 rows: the row pair's slice sits in shared memory; four passes over it
+// with packed fp32x2 arithmetic.  Pass 0: slice maxima.  Pass 1: sum of
+// 2^(u - m) over the slice for both rows (u = z log2 e; the log-sum-exp
+// needs no count of max-valued elements here), merged across the cluster.
+// Pass 2: |p - q|, p sign(p - q), (p, sign) written in place.  Pass 3: the
+// gradient.
+template <typename G>
+__device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, int c0, int row,
+                                             uint32_t rank, uint32_t CL, cg::cluster_group& cluster,
+                                             L1Shared& sh, const L1Params& P) {
+  const int tid = threadIdx.x;
+  const int nfull = n / 8;
+  const uint4* d4 = reinterpret_cast<const uint4*>(bd);
+  const uint4* t4 = reinterpret_cast<const uint4*>(bt);
+  const f32x2 l2e = pack2(kLog2e, kLog2e);
+
+  // pass 0
+  uint32_t mxd = 0xFF80FF80u, mxt = 0xFF80FF80u;
+  for (int v = tid; v < nfull; v += kThreads) {
+    const uint4 a = d4[v], b = t4[v];
+    mxd = bmax2(mxd, bmax2(bmax2(a.x, a.y), bmax2(a.z, a.w)));
+    mxt = bmax2(mxt, bmax2(bmax2(b.x, b.y), bmax2(b.z, b.w)));
+  }
+  float vd = fmaxf(__uint_as_float(mxd << 16), __uint_as_float(mxd & 0xFFFF0000u));
+  float vt = fmaxf(__uint_as_float(mxt << 16), __uint_as_float(mxt & 0xFFFF0000u));
+  for (int j = nfull * 8 + tid; j < n; j += kThreads) {
+    vd = fmaxf(vd, value_of(bd[j]));
+    vt = fmaxf(vt, value_of(bt[j]));
+  }
+  vd = l1_block_max(vd, sh.fred);
+  vt = l1_block_max(vt, sh.fred);
+
+  // pass 1
+  const float md = __fmul_rn(vd, kLog2e), mt = __fmul_rn(vt, kLog2e);
+  {
+    const f32x2 nmd = pack2(-md, -md), nmt = pack2(-mt, -mt);
+    f32x2 zd = pack2(0.f, 0.f), zt = pack2(0.f, 0.f);
+    // A vector holding the slice max takes the exact scalar form, so that a
+    // max-valued element contributes exactly 1 (u - m computed without
+    // fusion); the others take the packed fused form.
+    auto zsum = [&](const uint4& a, float vmax, float m, f32x2 nm, f32x2& z) {
+      const uint32_t wa[4] = {a.x, a.y, a.z, a.w};
+      if (vec_max(a) == vmax) {
+        float zs = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          zs += ex2(__fsub_rn(__fmul_rn(bf16_at(wa, i), kLog2e), m));
+        z = add2(z, pack2(zs, 0.f));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float e0, e1;
+          unpack2(fma2(pack2(__uint_as_float(wa[i] << 16), __uint_as_float(wa[i] & 0xFFFF0000u)), l2e, nm), e0, e1);
+          z = add2(z, pack2(ex2(e0), ex2(e1)));
+        }
+      }
+    };
+    for (int v = tid; v < nfull; v += kThreads) {
+      zsum(d4[v], vd, md, nmd, zd);
+      zsum(t4[v], vt, mt, nmt, zt);
+    }
+    float z0, z1, y0, y1;
+    unpack2(zd, z0, z1);
+    unpack2(zt, y0, y1);
+    float sz = z0 + z1, sy = y0 + y1;
+    for (int j = nfull * 8 + tid; j < n; j += kThreads) {
+      sz += ex2(__fsub_rn(__fmul_rn(value_of(bd[j]), kLog2e), md));
+      sy += ex2(__fsub_rn(__fmul_rn(value_of(bt[j]), kLog2e), mt));
+    }
+    Stats sd{md, 0.f, sz, 0.f}, st{mt, 0.f, sy, 0.f};
+    if (vd == -kInf && sz == 0.f) sd = stats_empty();
+    if (vt == -kInf && sy == 0.f) st = stats_empty();
+    sd = block_reduce(sd, sh.red);
+    st = block_reduce(st, sh.red);
+    if (tid == 0) {
+      sh.part[0] = sd;
+      sh.part[1] = st;
+    }
+  }
+  cluster.sync();
+  if (tid < static_cast<int>(CL)) {
+    const L1Shared* rsh = cluster.map_shared_rank(&sh, tid);
+    sh.gathered[tid][0] = rsh->part[0];
+    sh.gathered[tid][1] = rsh->part[1];
+  }
+  __syncthreads();
+  Stats Sd = stats_empty(), St = stats_empty();
+  for (uint32_t r = 0; r < CL; ++r) {
+    stats_merge(Sd, sh.gathered[r][0]);
+    stats_merge(St, sh.gathered[r][1]);
+  }
+  const float ld2 = stats_log2z(Sd), lt2 = stats_log2z(St);
+  const float cd = Sd.m + ld2, ct = St.m + lt2;
+
+  // pass 2
+  float l1 = 0.f, ps = 0.f;
+  const bool keep = P.grad != nullptr;
+  uint4* d4w = reinterpret_cast<uint4*>(bd);
+  uint4* t4w = reinterpret_cast<uint4*>(bt);
+  {
+    const f32x2 ncd = pack2(-cd, -cd), nct = pack2(-ct, -ct);
+    for (int v = tid; v < nfull; v += kThreads) {
+      const uint4 a = d4[v], b = t4[v];
+      const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+      uint32_t enc[8];
+      if (__fmul_rn(vec_max(a), kLog2e) == Sd.m || __fmul_rn(vec_max(b), kLog2e) == St.m) {
+        // a row max: the exact scalar form (p = 1 exactly for a single token)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          enc[i] = l1_step(ex2(__fsub_rn(__fsub_rn(__fmul_rn(bf16_at(wa, i), kLog2e), Sd.m), ld2)),
+                           ex2(__fsub_rn(__fsub_rn(__fmul_rn(bf16_at(wb, i), kLog2e), St.m), lt2)),
+                           l1, ps);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float p0, p1, q0, q1;
+          unpack2(fma2(pack2(__uint_as_float(wa[i] << 16), __uint_as_float(wa[i] & 0xFFFF0000u)), l2e, ncd), p0, p1);
+          unpack2(fma2(pack2(__uint_as_float(wb[i] << 16), __uint_as_float(wb[i] & 0xFFFF0000u)), l2e, nct), q0, q1);
+          enc[2 * i] = l1_step(ex2(p0), ex2(q0), l1, ps);
+          enc[2 * i + 1] = l1_step(ex2(p1), ex2(q1), l1, ps);
+        }
+      }
+      if (keep) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          hi[i] = (enc[2 * i] >> 16) | (enc[2 * i + 1] & 0xFFFF0000u);
+          lo[i] = (enc[2 * i] & 0xFFFFu) | (enc[2 * i + 1] << 16);
+        }
+        d4w[v] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        t4w[v] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+    }
+    for (int j = nfull * 8 + tid; j < n; j += kThreads) {
+      const uint32_t e = l1_step(ex2(__fsub_rn(__fsub_rn(__fmul_rn(value_of(bd[j]), kLog2e), Sd.m), ld2)),
+                                 ex2(__fsub_rn(__fsub_rn(__fmul_rn(value_of(bt[j]), kLog2e), St.m), lt2)),
+                                 l1, ps);
+      if (keep) {
+        bd[j] = static_cast<uint16_t>(e >> 16);
+        bt[j] = static_cast<uint16_t>(e & 0xFFFFu);
+      }
+    }
+  }
+  l1 = block_sum(l1, sh.fred);
+  ps = block_sum(ps, sh.fred);
+  if (tid == 0) {
+    sh.agg_l1 = l1;
+    sh.agg_ps = ps;
+  }
+  cluster.sync();
+  float L1 = 0.f, PS = 0.f;
+  for (uint32_t r = 0; r < CL; ++r) {
+    const L1Shared* rsh = cluster.map_shared_rank(&sh, r);
+    L1 += rsh->agg_l1;
+    PS += rsh->agg_ps;
+  }
+  const float w = P.row_weight ? P.row_weight[row] : 1.f;
+  if (rank == 0 && tid == 0) {
+    if (P.l1) P.l1[row] = L1;
+    if (P.accept) P.accept[row] = fminf(1.f, fmaxf(0.f, 1.f - 0.5f * L1));
+    if (P.ws_wl1) P.ws_wl1[row] = static_cast<double>(w) * static_cast<double>(L1);
+  }
+
+  // pass 3: d loss / d draft_j = (w / sum w) p_j (s_j - sum_k p_k s_k)
+  if (P.grad) {
+    const double wsum = *P.ws_wsum;
+    const float coef = wsum > 0.0 ? static_cast<float>(static_cast<double>(w) / wsum) : 0.f;
+    const float k_pos = coef * (1.f - PS), k_neg = coef * (-1.f - PS), k_zero = coef * (-PS);
+    G* go = static_cast<G*>(P.grad) + static_cast<int64_t>(row) * P.grad_ld + c0;
+    for (int v = tid; v < nfull; v += kThreads) {
+      const uint4 hv = d4[v], lv = t4[v];
+      const uint32_t hi[4] = {hv.x, hv.y, hv.z, hv.w}, lo[4] = {lv.x, lv.y, lv.z, lv.w};
+      float out[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        out[2 * i] = l1_grad((hi[i] << 16) | (lo[i] & 0xFFFFu), k_pos, k_neg, k_zero);
+        out[2 * i + 1] = l1_grad((hi[i] & 0xFFFF0000u) | (lo[i] >> 16), k_pos, k_neg, k_zero);
+      }
+      G* dst = go + v * 8;
+      if constexpr (sizeof(G) == 2) {
+        uint32_t wv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(out[2 * i], out[2 * i + 1]);
+          wv[i] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+        __stcs(reinterpret_cast<uint4*>(dst), make_uint4(wv[0], wv[1], wv[2], wv[3]));
+      } else {
+        __stcs(reinterpret_cast<float4*>(dst), make_float4(out[0], out[1], out[2], out[3]));
+        __stcs(reinterpret_cast<float4*>(dst + 4), make_float4(out[4], out[5], out[6], out[7]));
+      }
+    }
+    for (int j = nfull * 8 + tid; j < n; j += kThreads) {
+      const float g = l1_grad((static_cast<uint32_t>(bd[j]) << 16) | static_cast<uint32_t>(bt[j]),
+                              k_pos, k_neg, k_zero);
+      if constexpr (sizeof(G) == 2)
+        go[j] = static_cast<G>(__bfloat16_as_ushort(__float2bfloat16_rn(g)));
+      else
+        go[j] = g;
+    }
+  }
+}
+
 template <typename Raw, typename G>
 __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
   constexpr int VEC = 16 / sizeof(Raw);
@@ -105,7 +355,10 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
   }
   __syncthreads();
 
-  // pass 1: online statistics of both rows (base-2 units, no temperature)
+  if constexpr (sizeof(Raw) == 2) {
+    l1_rows_bf16<G>(bd, bt, n, c0, row, rank, CL, cluster, sh, P);
+  } else {
+  // fp32 rows: pass 1, online statistics of both rows (base-2 units)
   Stats sd = stats_empty(), st = stats_empty();
   const int nfull = n / VEC;
   const uint4* d4 = reinterpret_cast<const uint4*>(bd);
@@ -271,6 +524,7 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
       else
         go[j] = g;
     }
+  }
   }
   if (sh.timeout && tid == 0 && P.l1) P.l1[row] = __int_as_float(0x7fc00000);
   cluster.sync();
