@@ -167,9 +167,10 @@ vs_status vs_score_fwd(const vs_score_args* args, const vs_score_out* out, void*
                        size_t workspace_bytes, void* stream);
 
 /* Workspace bytes vs_score_fwd needs for these arguments: 0 for fp32 rows
- * and for a recorded support; for bf16 rows with a computed support it grows
- * with R (per-chunk statistics and 8 KB key histograms) and is capped near
- * 64 MB by processing large batches in several launches. */
+ * and for a recorded support; for bf16 rows with a computed support a few
+ * hundred bytes per row (16-byte statistics per row chunk and a per-row
+ * support decision), for at most the rows of one launch (large batches run
+ * as several launches of rows whose logits fit in L2). */
 size_t vs_score_fwd_workspace_size(const vs_score_args* args);
 
 /* Largest vocabulary vs_score_fwd accepts for a dtype. */

@@ -1,32 +1,27 @@
-// Computed-support forward scoring of bf16 rows, each row split into S
-// contiguous chunks (temperature -> stable token-id top-k -> inclusive top-p
-// -> min-p against the original row max; xorl issue #71, section 3).
+// Computed-support forward scoring of bf16 rows (temperature -> stable
+// token-id top-k -> inclusive top-p -> min-p against the original row max;
+// xorl issue #71, section 3).
 //
-// Kernel 1, one CTA per (row, chunk):
-//   pass a (HBM)  online statistics of the chunk: running max, count of
-//                 max-valued elements, sum 2^(u - m), sum (u - m) 2^(u - m)
-//                 (u = z log2 e), rebased whenever a vector raises the max;
-//   pass b (L2)   only for filtered rows: a histogram of the EXACT 16-bit keys
-//                 in the 4,096 keys at and below the chunk max, skipping
-//                 elements that provably cannot enter the support, and the
-//                 number of elements tied with the target's value that
-//                 precede it;
-//   then a 32-byte record and the histogram (16-bit counts) are written.
-// Kernel 2, one 512-thread CTA per row (programmatic dependent launch, so its
-// launch overlaps kernel 1): the row max is the largest chunk max, the
-// statistics are rebased onto it, and the chunk histograms are added at their
-// offsets into the row's window of 4,096 keys below the row max (every chunk
-// window reaches at least as low as the row window, so the merged window is
-// exact).  Each bin holds one value, so its mass is count x 2^(u - m); block
-// scans over the bins give the k-th element and the top-p crossing, and the
-// support sums.  A crossing below the window falls back to an 8-bit radix
-// descent over the row (rows whose support reaches far below the max).
-// Kernel 3 (only when the bitmask is requested) writes the support bitmask.
-//
-// The tie cut (which of the elements equal to the threshold value are kept:
+// Kernel 1 (score_chunk_kernel), one 128-thread CTA per (row, chunk): each
+// row is cut into S chunks so that one wave covers the GPU.  The chunk is
+// streamed once from HBM with online statistics (max, count of max-valued
+// elements, sum 2^(u - m), sum (u - m) 2^(u - m); u = z log2 e) and a 16-byte
+// record is written.
+// Kernel 2 (score_merge_kernel), one 512-thread CTA per row, launched with
+// programmatic dependent launch so that its launch overlaps kernel 1: the
+// statistics are rebased onto the row max; for a filtered row the row is
+// streamed again from L2 (kernel 1 read it moments before) into a histogram
+// of the EXACT 16-bit keys in the window of up to 4,096 keys below the row
+// max, skipping elements that provably cannot enter the support.  Each bin
+// holds one value, so its mass is count x 2^(u - m); block scans over the
+// bins find the k-th element and the top-p crossing, and the support sums.
+// A crossing below the window falls back to an 8-bit radix descent over the
+// row.  The tie cut (which elements equal to the threshold value are kept:
 // the lowest ids) is resolved to an id only for the saved state or the
-// bitmask; the target's own membership comes from the count of its earlier
+// bitmask; the target's membership otherwise uses the count of its earlier
 // ties.
+// Kernel 3 (score_split_mask_kernel, only when the bitmask is requested)
+// writes the support bitmask from the row's decision.
 
 #include <climits>
 
@@ -44,25 +39,18 @@ constexpr int kCT = 128;          // threads per chunk CTA
 constexpr int kMT = 512;          // threads per merge CTA
 constexpr int kMW = kMT / 32;     // warps per merge CTA
 constexpr int kRound = 4;         // vectors per thread and round of the chunk pass
+constexpr int kHistUnroll = 8;    // 16-byte loads in flight per merge thread
 constexpr int kMaxChunks = 256;   // chunks per row
 constexpr int kChunkAlign = 256;  // chunk length granularity (elements)
-constexpr int kMaxChunk = 65280;  // 16-bit histogram counts
-constexpr int kHead = 256;        // histogram headroom above the first-round max (keys)
-constexpr int kCW = kSelWin + kHead;     // bins of a chunk histogram
-constexpr int kHistWords = kCW / 2;      // one chunk histogram, u16 pairs
+constexpr size_t kRowsL2Bytes = size_t(48) << 20;  // logits per launch kept for the L2 re-read
 constexpr size_t kSplitWsCap = size_t(64) << 20;
 
-// Per (row, chunk) record.  The statistics' reference is the chunk max; the
-// histogram's top key ktop is at or above the chunk max key.
+// Per (row, chunk) statistics relative to fl(vmax c).
 struct alignas(16) ChunkRec {
-  float vmax;       // chunk maximum (value)
-  float c0, zr, a;  // statistics relative to fl(vmax c)
-  uint32_t nb;      // histogram bins written (bins >= nb hold nothing)
-  uint32_t ylt;     // chunk holding the target: its earlier ties (else 0)
-  uint32_t ktop;    // key of histogram bin 0 (bin b counts key ktop - b)
-  uint32_t pad;
+  float vmax;  // chunk maximum (value)
+  float c0, zr, a;
 };
-static_assert(sizeof(ChunkRec) == 32, "record layout");
+static_assert(sizeof(ChunkRec) == 16, "record layout");
 
 // Per-row support decision, for the bitmask kernel.
 struct alignas(16) RowDecision {
@@ -75,7 +63,6 @@ struct alignas(16) RowDecision {
 struct ChunkShared {
   Stats wst[kCT / 32];
   float fred[kCT / 32];
-  uint32_t ured[kCT / 32];
 };
 
 // Support sums: counts above the threshold, of its tie group and of the
@@ -92,18 +79,13 @@ struct MergeShared {
   float fred[kMW];
   uint32_t ured[kMW];
   u64 ulred[kMW];
-  int32_t coff[kMaxChunks];  // row bin of each chunk's bin 0 (negative: none)
-  uint32_t cnb[kMaxChunks];  // bins each chunk wrote
   int32_t tie_cut;
-  int32_t found_chunk;
-  int32_t found_need;
 };
 
 struct SplitArgs {
   int S;              // chunks per row
   int chunk;          // elements per chunk (multiple of kChunkAlign)
   ChunkRec* recs;     // [rows * S]
-  uint32_t* hists;    // [rows * S * kHistWords]
   RowDecision* dec;   // [rows]
 };
 
@@ -134,20 +116,6 @@ __device__ __forceinline__ float block_max(float v, float* scratch) {
   __syncthreads();
   return t;
 }
-
-__device__ __forceinline__ uint32_t block_max_u(uint32_t v, uint32_t* scratch) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
-  if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = v;
-  __syncthreads();
-  uint32_t t = 0;
-  const int nw = blockDim.x >> 5;
-  for (int w = 0; w < nw; ++w) t = max(t, scratch[w]);
-  __syncthreads();
-  return t;
-}
-
-__device__ __forceinline__ SupSums block_sum_sup(SupSums v, MergeShared& sh);
 
 // block_reduce of the statistics that also takes the block max of v (one
 // exchange for both maxima, one for the rebased sums).
@@ -191,29 +159,6 @@ __device__ __forceinline__ Stats block_reduce_vmax(Stats s, float& v, Stats* scr
   __syncthreads();
   v = vv;
   return t;
-}
-
-// Words holding the 16-bit counts [sh, sh + 8) of the 16 counts in lo, hi
-// (sh in 0..7; uniform across the warp, so the selection does not diverge).
-__device__ __forceinline__ void take8(const uint4& lo, const uint4& hi, int sh, uint32_t (&out)[4]) {
-  uint32_t a0, a1, a2, a3, a4;
-  switch (sh >> 1) {
-    case 0: a0 = lo.x; a1 = lo.y; a2 = lo.z; a3 = lo.w; a4 = hi.x; break;
-    case 1: a0 = lo.y; a1 = lo.z; a2 = lo.w; a3 = hi.x; a4 = hi.y; break;
-    case 2: a0 = lo.z; a1 = lo.w; a2 = hi.x; a3 = hi.y; a4 = hi.z; break;
-    default: a0 = lo.w; a1 = hi.x; a2 = hi.y; a3 = hi.z; a4 = hi.w; break;
-  }
-  if (sh & 1) {
-    out[0] = __funnelshift_r(a0, a1, 16);
-    out[1] = __funnelshift_r(a1, a2, 16);
-    out[2] = __funnelshift_r(a2, a3, 16);
-    out[3] = __funnelshift_r(a3, a4, 16);
-  } else {
-    out[0] = a0;
-    out[1] = a1;
-    out[2] = a2;
-    out[3] = a3;
-  }
 }
 
 // f(raw, id) for every element of g[j0, j1) (j0 a multiple of 8), the
@@ -367,54 +312,33 @@ __device__ __forceinline__ SupSums block_sum_sup(SupSums v, MergeShared& sh) {
   return t;
 }
 
-// One shared-memory count increment at the 32-bit shared address a, only
-// when c holds (a predicated reduction, no branch around it).
-__device__ __forceinline__ void red_inc_if(uint32_t a, bool c) {
-  asm volatile(
-      "{\n .reg .pred q;\n setp.ne.u32 q, %1, 0;\n @q red.shared.add.u32 [%0], 1;\n}\n" ::"r"(a),
-      "r"(static_cast<uint32_t>(c))
-      : "memory");
+// One shared-memory count increment at the 32-bit shared address a.
+__device__ __forceinline__ void red_inc(uint32_t a) {
+  asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(a) : "memory");
 }
 
 // Per-thread state of the chunk pass: running max (value vr, u units mr),
-// the count of max-valued elements, packed sums of 2^(u - mr) and
-// (u - mr) 2^(u - mr) over the others, the target's earlier ties, and
-// whether an element lay above the histogram's top key.
+// the count of max-valued elements, and packed sums of 2^(u - mr) and
+// (u - mr) 2^(u - mr) over the others.
 struct ChunkAcc {
   float vr, mr;
-  uint32_t c0, ylt, ovf;
+  uint32_t c0;
   f32x2 z2, a2;
 };
 
-// The chunk pass over 16-byte vectors: online statistics (a vector that
-// raises the running max rebases the sums) and, with HIST, the window
-// histogram: each element whose bin b = ktop - key lies below nbw is
-// counted.  MODE 1 (every kept key is a positive non-zero value):
-// b = rtop - r; MODE 2 (every kept key is a negative value): b = r - rtop;
-// MODE 0: the key map.  Raw values outside the window wrap to huge bins in
-// modes 1 and 2.  With CNTY the elements tied with key ky whose id is below
-// y are counted.  The thread's first-round vectors q1 are already loaded.
-template <int MODE, bool HIST, bool CNTY>
+// The chunk pass over 16-byte vectors: online statistics.  A vector below
+// the running max takes a packed path with no per-element compares; a
+// vector that reaches or raises it (rare once the first round has fixed a
+// high running max) rebases the sums and counts its max-valued elements.
+// The thread's first-round vectors q1 are already loaded.
 __device__ __forceinline__ void chunk_pass(const uint4 (&q1)[kRound], const uint4* v4, int nv,
-                                           int j0, float c, uint32_t ktop, uint32_t rtop,
-                                           uint32_t nbw, uint32_t ky, int y, uint32_t* hist,
-                                           ChunkAcc& acc) {
+                                           float c, ChunkAcc& acc) {
   const f32x2 c2 = pack2(c, c);
-  const uint32_t hist_s = smem_addr(hist);
-  auto bin = [&](uint32_t r) -> uint32_t {
-    if constexpr (MODE == 1)
-      return rtop - r;
-    else if constexpr (MODE == 2)
-      return r - rtop;
-    else
-      return ktop - bf16_key(r);
-  };
-  auto vec = [&](const uint4& q, int vi) {
+  auto vec = [&](const uint4& q) {
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
     const uint32_t mv = bmax2(bmax2(q.x, q.y), bmax2(q.z, q.w));
     const float vm = fmaxf(__uint_as_float(mv << 16), __uint_as_float(mv & 0xFFFF0000u));
     if (vm >= acc.vr) {
-      // rare: the vector holds the running max, or raises it
       if (vm > acc.vr) {
         const float mn = __fmul_rn(vm, c);
         if (acc.vr != -kInf) {
@@ -430,9 +354,6 @@ __device__ __forceinline__ void chunk_pass(const uint4 (&q1)[kRound], const uint
         acc.c0 = 0;
         acc.vr = vm;
         acc.mr = mn;
-        if constexpr (HIST) {
-          if (bf16_key(__float_as_uint(vm) >> 16) > ktop) acc.ovf = 1;
-        }
       }
       // max-valued elements are counted apart (by value)
       float zs = 0.f, as = 0.f;
@@ -463,48 +384,20 @@ __device__ __forceinline__ void chunk_pass(const uint4 (&q1)[kRound], const uint
         acc.a2 = fma2(d2, e2, acc.a2);
       }
     }
-    if constexpr (HIST) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t r0 = w[i] & 0xFFFFu, r1 = w[i] >> 16;
-        const uint32_t b0 = bin(r0), b1 = bin(r1);
-        red_inc_if(hist_s + (b0 << 2), b0 < nbw);
-        red_inc_if(hist_s + (b1 << 2), b1 < nbw);
-        if constexpr (CNTY) {
-          const int id = j0 + vi * 8 + 2 * i;
-          acc.ylt += static_cast<uint32_t>(bf16_key(r0) == ky) & static_cast<uint32_t>(id < y);
-          acc.ylt += static_cast<uint32_t>(bf16_key(r1) == ky) & static_cast<uint32_t>(id + 1 < y);
-        }
-      }
-    }
   };
-  // rounds of kRound vectors per thread, one copy of the loop body; the
-  // first round's vectors arrive preloaded
+  // rounds of kRound vectors per thread, one copy of the loop body
   uint4 q[kRound];
 #pragma unroll
   for (int k = 0; k < kRound; ++k) q[k] = q1[k];
   for (int v0 = threadIdx.x;;) {
 #pragma unroll
     for (int k = 0; k < kRound; ++k)
-      if (v0 + k * kCT < nv) vec(q[k], v0 + k * kCT);
+      if (v0 + k * kCT < nv) vec(q[k]);
     v0 += kRound * kCT;
     if (v0 >= nv) break;
 #pragma unroll
     for (int k = 0; k < kRound; ++k) q[k] = v0 + k * kCT < nv ? __ldg(v4 + v0 + k * kCT) : make_uint4(0, 0, 0, 0);
   }
-}
-
-// Re-count the chunk's window histogram below its exact max key (after an
-// element rose above the first estimate of the top), from L2.
-__device__ __noinline__ void chunk_rehist(const uint16_t* g, int j0, int j1, uint32_t ktop,
-                                          uint32_t nbw, uint32_t* hist) {
-  for (int b = threadIdx.x; b < kCW; b += kCT) hist[b] = 0u;
-  __syncthreads();
-  for_each_elem<kCT>(g, j0, j1, [&](uint32_t r, int) {
-    const uint32_t b = ktop - bf16_key(r);
-    if (b < nbw) atomicAdd(&hist[b], 1u);
-  });
-  __syncthreads();
 }
 
 // Smallest key in [lo, hi] whose u-offset from m reaches dlo (hi if none).
@@ -521,7 +414,6 @@ __device__ __forceinline__ uint32_t key_at_level(uint32_t lo, uint32_t hi, float
 }
 
 __global__ void __launch_bounds__(kCT, 8) score_chunk_kernel(ScoreParams P, SplitArgs Q) {
-  __shared__ __align__(16) uint32_t hist[kCW];
   __shared__ ChunkShared sh;
   pdl_launch_dependents();
 
@@ -533,22 +425,11 @@ __global__ void __launch_bounds__(kCT, 8) score_chunk_kernel(ScoreParams P, Spli
   const int j0 = cs * Q.chunk, j1 = min(V, j0 + Q.chunk);
   const int nv = (j1 - j0) / 8;
   const uint4* v4 = reinterpret_cast<const uint4*>(grow + j0);
-
   const float T = P.temperature ? P.temperature[row] : P.temperature_scalar;
   const float c = kLog2e / T;
-  const int kk = P.top_k ? P.top_k[row] : P.top_k_scalar;
-  const float pp = P.top_p ? P.top_p[row] : P.top_p_scalar;
-  const float mp = P.min_p ? P.min_p[row] : P.min_p_scalar;
-  const bool use_k = kk > 0 && kk < V;
-  const bool use_p = pp < 1.f;
-  const bool use_minp = mp > 0.f;
-  const bool any_filter = use_k || use_p || use_minp;
 
-  if (any_filter)
-    for (int b = tid; b < kCW; b += kCT) hist[b] = 0u;
-
-  // ---- first round: each thread's first kRound vectors, and their block
-  // max m1 (a lower bound of the chunk max that fixes the histogram window)
+  // first round: each thread's first kRound vectors; their block max m1
+  // starts every thread's running max, so later rebases are rare
   uint4 q1[kRound];
   uint32_t mx = 0xFF80FF80u;  // (-inf, -inf)
 #pragma unroll
@@ -559,107 +440,76 @@ __global__ void __launch_bounds__(kCT, 8) score_chunk_kernel(ScoreParams P, Spli
   }
   const float m1 = block_max(fmaxf(__uint_as_float(mx << 16), __uint_as_float(mx & 0xFFFF0000u)), sh.fred);
 
-  ChunkAcc acc{m1, __fmul_rn(m1, c), 0u, 0u, 0u, pack2(0.f, 0.f), pack2(0.f, 0.f)};
-  uint32_t ktop = 0, nbw = 0, ky = 0xFFFFFFFFu;
-  const int y = P.targets[row];
-  const bool cnty = any_filter && y > j0 && y < j1;
-  if (!any_filter) {
-    chunk_pass<0, false, false>(q1, v4, nv, j0, c, 0u, 0u, 0u, 0u, 0, hist, acc);
-  } else {
-    // window: keys ktop - nbw + 1 .. ktop, ktop kHead keys above m1's key
-    const uint32_t k1 = bf16_key(__float_as_uint(m1) >> 16);
-    ktop = min(k1 + static_cast<uint32_t>(kHead), KeyTraits<uint16_t>::kInfKey);
-    uint32_t kbot = ktop >= static_cast<uint32_t>(kCW - 1) ? ktop - (kCW - 1) : 0u;
-    // Elements below these levels (relative to m1, hence also to the row
-    // max) never enter the support: min-p keeps 2^(u - m) >= min_p; top-p
-    // alone keeps a prefix whose complement holds at most (1 - p) of the
-    // mass, while all elements with 2^(u - m) < (1 - p) / (2 V) hold less than
-    // half of that (the row total is at least 1).  One more octave of margin.
-    float dlo = -kInf;
-    if (use_minp) dlo = log2f(mp) - 1.f;
-    if (use_p && !use_k && pp > 0.f) dlo = fmaxf(dlo, log2f((1.f - pp) / static_cast<float>(V)) - 2.f);
-    if (dlo > -kInf && isfinite(acc.mr)) kbot = key_at_level(kbot, k1, c, acc.mr, dlo);
-    nbw = ktop - kbot + 1;
-    if (cnty) ky = bf16_key(grow[y]);
-    const int mode = kbot > 0x7FFFu ? 1 : (ktop < 0x7FFFu ? 2 : 0);
-    const uint32_t rtop = mode == 1 ? ktop - 0x7FFFu : 0xFFFFu - ktop;
-    if (cnty) {
-      if (mode == 1) chunk_pass<1, true, true>(q1, v4, nv, j0, c, ktop, rtop, nbw, ky, y, hist, acc);
-      else if (mode == 2) chunk_pass<2, true, true>(q1, v4, nv, j0, c, ktop, rtop, nbw, ky, y, hist, acc);
-      else chunk_pass<0, true, true>(q1, v4, nv, j0, c, ktop, rtop, nbw, ky, y, hist, acc);
-    } else {
-      if (mode == 1) chunk_pass<1, true, false>(q1, v4, nv, j0, c, ktop, rtop, nbw, ky, y, hist, acc);
-      else if (mode == 2) chunk_pass<2, true, false>(q1, v4, nv, j0, c, ktop, rtop, nbw, ky, y, hist, acc);
-      else chunk_pass<0, true, false>(q1, v4, nv, j0, c, ktop, rtop, nbw, ky, y, hist, acc);
-    }
-  }
+  ChunkAcc acc{m1, __fmul_rn(m1, c), 0u, pack2(0.f, 0.f), pack2(0.f, 0.f)};
+  chunk_pass(q1, v4, nv, c, acc);
   Stats st;
   {
     float z0, z1, a0, a1;
     unpack2(acc.z2, z0, z1);
     unpack2(acc.a2, a0, a1);
     st = Stats{acc.mr, static_cast<float>(acc.c0), z0 + z1, a0 + a1};
-    if (acc.vr == -kInf && acc.c0 == 0 && z0 + z1 == 0.f) st = stats_empty();
   }
   // ragged tail (the last chunk of a row whose length is not a multiple of 8)
   float vr = acc.vr;
-  uint32_t ylt = acc.ylt, ovf = acc.ovf;
   for (int j = j0 + nv * 8 + tid; j < j1; j += kCT) {
-    const uint32_t r = grow[j];
-    const float x = value_of(static_cast<uint16_t>(r));
+    const float x = value_of(grow[j]);
     float u[1] = {__fmul_rn(x, c)};
     vr = fmaxf(vr, x);
     stats_add(st, u);
-    if (any_filter) {
-      const uint32_t key = bf16_key(r);
-      if (key > ktop) ovf = 1u;
-      if (ktop - key < nbw) atomicAdd(&hist[ktop - key], 1u);
-      if (cnty) ylt += static_cast<uint32_t>(key == ky) & static_cast<uint32_t>(j < y);
-    }
   }
   st = block_reduce_vmax(st, vr, sh.wst);
-  const float vmax = vr;
+  if (tid == 0) Q.recs[static_cast<int64_t>(row) * Q.S + cs] = ChunkRec{vr, st.c0, st.zr, st.a};
+}
 
-  uint32_t nb = 0;
-  if (any_filter) {
-    if (cnty) ylt = block_sum(ylt, sh.ured);
-    if (__syncthreads_or(ovf != 0u)) {
-      // an element rose above the window: count again below the exact max
-      const uint32_t kx = bf16_key(__float_as_uint(vmax) >> 16);
-      const uint32_t kb = ktop - (nbw - 1);  // keep the same lowest key (clamped)
-      ktop = kx;
-      nbw = kx >= kb ? min(kx - kb + 1, static_cast<uint32_t>(kCW)) : 1u;
-      chunk_rehist(grow, j0, j1, ktop, nbw, hist);
+// Histogram pass of the merge kernel: counts the row's elements whose key
+// lies in [klo, klo + nbins), hist[key - klo], streaming the row from L2
+// (hist holds kSelWin + 32 words).
+// MODE 1 (every kept key is a positive non-zero value): i = r - rlo; MODE 2
+// (every kept key is negative): i = rlo - r; MODE 0: the key map.  Raw
+// values outside the window wrap to huge indices in modes 1 and 2.
+template <int MODE>
+__device__ __forceinline__ void row_hist(const uint16_t* g, int V, uint32_t klo, uint32_t rlo,
+                                         uint32_t nbins, uint32_t hist_s) {
+  auto idx = [&](uint32_t r) -> uint32_t {
+    if constexpr (MODE == 1)
+      return r - rlo;
+    else if constexpr (MODE == 2)
+      return rlo - r;
+    else
+      return bf16_key(r) - klo;
+  };
+  const int nv = V / 8;
+  const uint4* v4 = reinterpret_cast<const uint4*>(g);
+  // out-of-window elements count into this lane's spill bin (never read):
+  // no predicate or branch, and the spill bins of a warp sit in 32 banks
+  const uint32_t spill = kSelWin + (threadIdx.x & 31);
+  auto vec = [&](const uint4& q) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t i0 = idx(w[i] & 0xFFFFu), i1 = idx(w[i] >> 16);
+      red_inc(hist_s + ((i0 < nbins ? i0 : spill) << 2));
+      red_inc(hist_s + ((i1 < nbins ? i1 : spill) << 2));
     }
-    __syncthreads();
-    uint32_t hi = 0;
-    for (int b = tid; b < kCW; b += kCT)
-      if (hist[b]) hi = b + 1;
-    nb = block_max_u(hi, sh.ured);
-    const int64_t slot = static_cast<int64_t>(row) * Q.S + cs;
-    uint4* hout = reinterpret_cast<uint4*>(Q.hists + slot * kHistWords);
-    for (int vv = tid; vv < static_cast<int>((nb + 7) / 8); vv += kCT) {
-      const uint32_t* h = hist + vv * 8;
-      hout[vv] = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16),
-                            h[6] | (h[7] << 16));
-    }
+  };
+  int v = threadIdx.x;
+  for (; v + (kHistUnroll - 1) * kMT < nv; v += kHistUnroll * kMT) {
+    uint4 q[kHistUnroll];
+#pragma unroll
+    for (int k = 0; k < kHistUnroll; ++k) q[k] = __ldcg(v4 + v + k * kMT);
+#pragma unroll
+    for (int k = 0; k < kHistUnroll; ++k) vec(q[k]);
   }
-  if (tid == 0) {
-    ChunkRec r;
-    r.vmax = vmax;
-    r.c0 = st.c0;
-    r.zr = st.zr;
-    r.a = st.a;
-    r.nb = nb;
-    r.ylt = ylt;
-    r.ktop = ktop;
-    r.pad = 0;
-    Q.recs[static_cast<int64_t>(row) * Q.S + cs] = r;
+  for (; v < nv; v += kMT) vec(__ldcg(v4 + v));
+  for (int j = nv * 8 + threadIdx.x; j < V; j += kMT) {
+    const uint32_t i0 = idx(g[j]);
+    red_inc(hist_s + ((i0 < nbins ? i0 : spill) << 2));
   }
 }
 
 __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, SplitArgs Q) {
-  __shared__ __align__(16) uint32_t hist[kSelWin];
+  // kSelWin window bins, then one spill bin per lane for out-of-window elements
+  __shared__ __align__(16) uint32_t hist[kSelWin + 32];
   __shared__ MergeShared sh;
   RadixArrays& ra = *reinterpret_cast<RadixArrays*>(hist);
 
@@ -680,19 +530,16 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
   const bool target_ok = y >= 0 && y < V;
   const int S = Q.S;
   const uint32_t ry = target_ok ? static_cast<uint32_t>(grow[y]) : 0u;
-  pdl_wait();  // the chunk kernel's records and histograms
+  pdl_wait();  // the chunk kernel's records
 
   const ChunkRec* rr = Q.recs + static_cast<int64_t>(row) * S;
   Stats st = stats_empty();
   float vr = -kInf;
   for (int k = tid; k < S; k += kMT) {
-    const float4 h0 = __ldcg(reinterpret_cast<const float4*>(rr + k));
-    const uint4 h1 = __ldcg(reinterpret_cast<const uint4*>(rr + k) + 1);
-    Stats t{__fmul_rn(h0.x, c), h0.y, h0.z, h0.w};
+    const float4 h = __ldcg(reinterpret_cast<const float4*>(rr + k));
+    Stats t{__fmul_rn(h.x, c), h.y, h.z, h.w};
     stats_merge(st, t);
-    vr = fmaxf(vr, h0.x);
-    sh.cnb[k] = h1.x;
-    sh.coff[k] = static_cast<int32_t>(h1.z);  // histogram top key for now
+    vr = fmaxf(vr, h.x);
   }
   st = block_reduce_vmax(st, vr, sh.wst);
 
@@ -709,68 +556,43 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
   u64 ckeep = 0;
   float log2zs = log2z, h_support = h_full, c0s = st.c0, zrs = st.zr;
   int32_t n_support = nonfinite ? 0 : V;
-  bool from_bins = false;  // the threshold lies inside the merged window
+  bool from_bins = false;  // the threshold lies inside the window
 
   if (filtered) {
     const float fxs = fx_scale(P.fx_shift);
     const uint32_t kmr = bf16_key(__float_as_uint(vr) >> 16);
+    // Elements below these levels never enter the support: min-p keeps
+    // 2^(u - m) >= min_p; top-p alone keeps a prefix whose complement holds
+    // at most (1 - p) of the mass Z, while all elements with 2^(u - m) <
+    // (1 - p) Z / (2 V) together hold less than half of that.  One more
+    // octave of margin each.
+    // (No skipping with top-k: its count and the top-k mass need every key.)
+    float dlo = -kInf;
+    if (!use_k) {
+      if (use_minp) dlo = log2f(mp) - 1.f;
+      if (use_p && pp > 0.f)
+        dlo = fmaxf(dlo, log2f((1.f - pp) * stats_z(st) / static_cast<float>(V)) - 2.f);
+    }
+    uint32_t klo = kmr >= static_cast<uint32_t>(kSelWin - 1) ? kmr - (kSelWin - 1) : 0u;
+    if (dlo > -kInf) klo = key_at_level(klo, kmr, c, mr, dlo);
     Window w{};
     w.kmax = kmr;
-    w.klo = kmr >= static_cast<uint32_t>(kSelWin - 1) ? kmr - (kSelWin - 1) : 0u;
-    w.nbins = static_cast<int>(kmr - w.klo) + 1;
+    w.klo = klo;
+    w.nbins = static_cast<int>(kmr - klo) + 1;
     w.hist = hist;
     w.c = c;
     w.m = mr;
     w.fxs = fxs;
-    // merged window: hist[key - klo]; chunk bin b holds key ktop_k - b
-    for (int k = tid; k < S; k += kMT) {
-      // a chunk's histogram top is at most kHead keys above the row max
-      const int off = static_cast<int>(kmr) - sh.coff[k];
-      sh.coff[k] = w.nbins - 1 - off;  // row bin of chunk bin 0
-    }
-    __syncthreads();  // coff / cnb
+    for (int b = tid; b < kSelWin; b += kMT) hist[b] = 0u;
+    __syncthreads();
     {
-      // Thread t builds row bins [8t, 8t + 8).  Row bin i holds chunk bin
-      // coff_k - i, so from chunk k it needs the descending run of chunk bins
-      // s .. s + 7 with s = coff_k - 8t - 7: two aligned 16-byte vectors,
-      // and the run's offset inside them, s mod 8, is the same for every
-      // thread.  Counts are summed in registers: no atomics.
-      static_assert(kSelWin / 8 == kMT, "eight row bins per merge thread");
-      constexpr int kB = 4;  // chunks per batch of loads
-      const uint4* hrow = reinterpret_cast<const uint4*>(Q.hists + static_cast<int64_t>(row) * S * kHistWords);
-      uint32_t acc[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-      for (int k0 = 0; k0 < S; k0 += kB) {
-        uint4 lo[kB], hi[kB];
-        int sh8[kB];
-#pragma unroll
-        for (int u = 0; u < kB; ++u) {
-          const int k = k0 + u;
-          lo[u] = hi[u] = make_uint4(0, 0, 0, 0);
-          sh8[u] = 0;
-          if (k < S) {
-            const int sb = sh.coff[k] - 8 * tid - 7;
-            const int va = sb >> 3;  // floor
-            const int nvk = static_cast<int>((sh.cnb[k] + 7) >> 3);
-            const uint4* hk = hrow + static_cast<int64_t>(k) * (kHistWords / 4);
-            if (va >= 0 && va < nvk) lo[u] = __ldcg(hk + va);
-            if (va + 1 >= 0 && va + 1 < nvk) hi[u] = __ldcg(hk + va + 1);
-            sh8[u] = sb & 7;
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < kB; ++u) {
-          uint32_t run[4];
-          take8(lo[u], hi[u], sh8[u], run);
-#pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            const int j2 = 7 - jj;  // row bin 8t + jj holds chunk bin s + 7 - jj
-            acc[jj] += (run[j2 >> 1] >> ((j2 & 1) * 16)) & 0xFFFFu;
-          }
-        }
-      }
-      uint4* h4 = reinterpret_cast<uint4*>(hist);
-      h4[2 * tid] = make_uint4(acc[0], acc[1], acc[2], acc[3]);
-      h4[2 * tid + 1] = make_uint4(acc[4], acc[5], acc[6], acc[7]);
+      const uint32_t hist_s = smem_addr(hist), nb = static_cast<uint32_t>(w.nbins);
+      if (klo > 0x7FFFu)
+        row_hist<1>(grow, V, klo, klo - 0x7FFFu, nb, hist_s);
+      else if (kmr < 0x7FFFu)
+        row_hist<2>(grow, V, klo, 0xFFFFu - klo, nb, hist_s);
+      else
+        row_hist<0>(grow, V, klo, 0u, nb, hist_s);
     }
     __syncthreads();
 
@@ -808,6 +630,13 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
           all_ties = cp >= dp.at_cnt;
           have_t = true;
         }
+      }
+      if (!win_ok && use_p && !use_k && use_minp && minp_key<uint16_t>(mp, c, mr) >= w.klo) {
+        // the top-p crossing lies below the window, hence below the min-p
+        // level: min-p decides the support (applied below)
+        win_ok = true;
+        have_t = false;
+        all_ties = true;
       }
       if (!win_ok) {
         // the k-th element or the crossing lies below the window
@@ -912,36 +741,7 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
       cut_known = false;
       if (want_cut) {
         const int need = static_cast<int>(ckeep);
-        if (from_bins) {
-          // the chunk holding the need-th tie, from the chunk histograms
-          // (every chunk window reaches down to the row window)
-          if (tid == 0) {
-            sh.found_chunk = -1;
-            int before = 0;
-            for (int k = 0; k < S && sh.found_chunk < 0; ++k) {
-              const uint32_t kk2 = __ldcg(&rr[k].ktop);
-              const uint32_t nbk = __ldcg(&rr[k].nb);
-              uint32_t cnt = 0;
-              if (kk2 >= tkey && kk2 - tkey < nbk) {
-                const uint32_t b = kk2 - tkey;
-                const uint32_t wd = __ldcg(Q.hists + (static_cast<int64_t>(row) * S + k) * kHistWords + (b >> 1));
-                cnt = (wd >> ((b & 1) * 16)) & 0xFFFFu;
-              }
-              if (before + static_cast<int>(cnt) >= need) {
-                sh.found_chunk = k;
-                sh.found_need = need - before;
-              }
-              before += static_cast<int>(cnt);
-            }
-          }
-          __syncthreads();
-          const int k = sh.found_chunk, nd = sh.found_need;
-          __syncthreads();
-          tie_cut = k >= 0 ? tie_scan<kMT>(grow, k * Q.chunk, min(V, (k + 1) * Q.chunk), tkey, nd, sh)
-                           : INT_MAX;
-        } else {
-          tie_cut = tie_scan<kMT>(grow, 0, V, tkey, need, sh);
-        }
+        tie_cut = tie_scan<kMT>(grow, 0, V, tkey, need, sh);
         cut_known = true;
       }
     }
@@ -951,27 +751,8 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
   uint32_t ylt_row = 0;
   if (filtered && !cut_known && target_ok && bf16_key(ry) == tkey) {
     uint32_t part = 0;
-    if (from_bins) {
-      // chunks before the target's: their histogram count at tkey; the
-      // target's chunk counted its own earlier ties
-      const int cy = y / Q.chunk;
-      for (int k = tid; k <= cy; k += kMT) {
-        if (k == cy) {
-          part += __ldcg(&rr[k].ylt);
-        } else {
-          const uint32_t kk2 = __ldcg(&rr[k].ktop);
-          const uint32_t nbk = __ldcg(&rr[k].nb);
-          if (kk2 >= tkey && kk2 - tkey < nbk) {
-            const uint32_t b = kk2 - tkey;
-            const uint32_t wd = __ldcg(Q.hists + (static_cast<int64_t>(row) * S + k) * kHistWords + (b >> 1));
-            part += (wd >> ((b & 1) * 16)) & 0xFFFFu;
-          }
-        }
-      }
-    } else {
-      const uint32_t t = tkey;
-      for_each_elem<kMT>(grow, 0, y, [&](uint32_t raw, int) { part += bf16_key(raw) == t; });
-    }
+    const uint32_t t = tkey;
+    for_each_elem<kMT>(grow, 0, y, [&](uint32_t raw, int) { part += bf16_key(raw) == t; });
     ylt_row = block_sum(part, sh.ured);
   }
 
@@ -1090,7 +871,7 @@ __global__ void __launch_bounds__(kCT) score_split_mask_kernel(ScoreParams P, Sp
 
 struct SplitPlan {
   int S, chunk, rows_per_launch;
-  size_t off_hists, off_dec, bytes;
+  size_t off_dec, bytes;
 };
 
 // Chunk CTAs resident on the whole device (one wave).
@@ -1113,28 +894,25 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 SplitPlan split_plan(int rows, int vocab) {
   SplitPlan p{};
+  // rows per launch: their logits stay in L2 between the two kernels
+  size_t rpl = kRowsL2Bytes / (2 * static_cast<size_t>(vocab));
+  if (rpl < 1) rpl = 1;
+  if (rpl > static_cast<size_t>(rows)) rpl = rows;
   const int cap = resident_ctas();
-  // chunks of about 48 KB keep a wave's working set inside L2; small
-  // batches split further so that one wave fills the GPU; at most
-  // kMaxChunks chunks (vocab <= kMaxChunks * kMaxChunk is checked upstream)
+  // chunks of about 48 KB; small batches split further so that one wave
+  // fills the GPU
   int S = (vocab + 24575) / 24576;
-  const int fill = rows > 0 ? cap / rows : 1;
+  const int fill = cap / static_cast<int>(rpl);
   if (fill > S) S = fill;
   if (S > kMaxChunks) S = kMaxChunks;
   int chunk = (vocab + S - 1) / S;
   chunk = (chunk + kChunkAlign - 1) / kChunkAlign * kChunkAlign;
   if (chunk < kChunkAlign * 8) chunk = kChunkAlign * 8;
-  if (chunk > kMaxChunk) chunk = kMaxChunk;
   S = (vocab + chunk - 1) / chunk;
   p.S = S;
   p.chunk = chunk;
-  const size_t per_row = static_cast<size_t>(S) * (sizeof(ChunkRec) + kHistWords * 4) + sizeof(RowDecision);
-  size_t rpl = kSplitWsCap / per_row;
-  if (rpl < 1) rpl = 1;
-  if (rpl > static_cast<size_t>(rows)) rpl = rows;
   p.rows_per_launch = static_cast<int>(rpl);
-  p.off_hists = align256(rpl * S * sizeof(ChunkRec));
-  p.off_dec = p.off_hists + align256(rpl * S * static_cast<size_t>(kHistWords) * 4);
+  p.off_dec = align256(rpl * S * sizeof(ChunkRec));
   p.bytes = p.off_dec + align256(rpl * sizeof(RowDecision));
   return p;
 }
@@ -1163,7 +941,7 @@ ScoreParams offset_rows(const ScoreParams& P, int r0, int n) {
 
 }  // namespace
 
-int32_t score_split_max_vocab() { return kMaxChunks * kMaxChunk; }
+int32_t score_split_max_vocab() { return 1 << 26; }
 
 size_t score_split_workspace_bytes(int rows, int vocab) {
   if (rows <= 0) return 0;
@@ -1177,7 +955,6 @@ cudaError_t launch_score_split(const ScoreParams& p, void* ws, cudaStream_t s) {
   q.S = plan.S;
   q.chunk = plan.chunk;
   q.recs = reinterpret_cast<ChunkRec*>(base);
-  q.hists = reinterpret_cast<uint32_t*>(base + plan.off_hists);
   q.dec = reinterpret_cast<RowDecision*>(base + plan.off_dec);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
