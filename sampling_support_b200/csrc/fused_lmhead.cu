@@ -5,8 +5,12 @@
 //   z[i, v] = (sum_k H[i, k] W[v, k]) / T_i
 //
 // Kernel 1 (lmhead_gemm_kernel), persistent and warp-specialised, one CTA per
-// SM.  Work units are (128-row block, vocabulary split) pairs; a unit walks
-// its split in 256-column tiles:
+// SM.  Work units are (row unit, vocabulary split) pairs; a unit walks its
+// split in 256-column tiles.  In pair mode two CTAs of a cluster share each
+// tile as one 256 x 256 tcgen05 MMA (cta_group::2): each loads its 128 rows
+// of H and its 128 of the tile's 256 W rows, the first CTA issues the MMAs
+// for both, and each receives its 128 rows of the accumulator, so a CTA
+// moves two thirds of the operand bytes of a single-CTA 128 x 256 tile:
 //   warp 0   TMA producer: 128x64 tiles of H and 256x64 tiles of W into a
 //            ring of shared-memory stages (128-byte swizzle, mbarriers);
 //   warp 1   MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32),
@@ -44,6 +48,16 @@ constexpr int kStageABytes = kBM * kBK * 2;  // 16 KB
 constexpr int kStageBBytes = kBN * kBK * 2;  // 32 KB
 constexpr int kStageBytes = kStageABytes + kStageBBytes;
 constexpr uint32_t kTmemCols = 2 * kBN;  // two accumulators
+constexpr int kMaxStages = 6;
+
+// Pair mode (tcgen05 cta_group::2): a cluster of two CTAs computes a
+// 256 x 256 tile; each CTA holds its 128 rows of the H tile and 128 of the
+// 256 W rows, and receives its 128 rows x 256 columns of the accumulator.
+constexpr int kBNh = kBN / 2;                     // W rows per CTA of a pair
+constexpr int kStageBytes2 = kStageABytes + kBNh * kBK * 2;  // 32 KB
+// kind::f16 descriptor for M = 256 (the pair), N = 256
+constexpr uint32_t kIDesc2 = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) |
+                             (uint32_t(256 >> 4) << 24);
 
 // UMMA instruction descriptor, kind::f16: D fp32, A and B bf16, both
 // K-major, N = 256, M = 128.
@@ -52,6 +66,7 @@ constexpr uint32_t kIDesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kBN >
 
 struct LmParams {
   int32_t rows, vocab, hidden;
+  int32_t m_units;      // row units: 128-row blocks, or 256-row block pairs in pair mode
   int32_t top_k;
   int32_t splits;       // vocabulary splits
   int32_t tiles_per_split;
@@ -103,6 +118,71 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
       : "memory");
 }
 
+// Pair-mode tensor load: lands in this CTA's shared memory and completes its
+// bytes on the leader CTA's barrier at the same offset (cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, int c0, int c1,
+                                                 uint64_t* bar) {
+  asm volatile(
+      "{\n .reg .b32 lb;\n mapa.shared::cluster.u32 lb, %4, 0;\n"
+      " cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [lb];\n}\n" ::
+          "r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_f16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(kIDesc2), "r"(accumulate)
+      : "memory");
+}
+
+// Completion of the pair's MMAs arrives on the barrier at this offset in
+// both CTAs of the pair.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_addr(bar)),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
+}
+
+// Arrive on the leader CTA's barrier at this offset.
+__device__ __forceinline__ void mbar_arrive_leader(uint64_t* bar) {
+  asm volatile(
+      "{\n .reg .b32 ra;\n mapa.shared::cluster.u32 ra, %0, 0;\n"
+      " mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n}\n" ::"r"(smem_addr(bar))
+      : "memory");
+}
+
+// Bounded wait for a barrier phase whose arrivals come from the peer CTA
+// (acquire at cluster scope); false after the iteration cap.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -139,8 +219,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 //   [barriers] [tmem slot]
 
 struct Barriers {
-  uint64_t full[4];
-  uint64_t empty[4];
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint32_t tmem_base;
@@ -170,23 +250,31 @@ __device__ __forceinline__ void topk_insert(float* vals, int32_t* ids, int k, in
   if (count < k) ++count;
 }
 
+template <bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     lmhead_gemm_kernel(const __grid_constant__ CUtensorMap map_h,
                        const __grid_constant__ CUtensorMap map_w, LmParams P) {
+  constexpr int SB = PAIR ? kStageBytes2 : kStageBytes;  // bytes per stage in this CTA
+  constexpr int SA = kStageABytes;
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
                                              ~uintptr_t(1023));
   const int S = P.stages;
   uint8_t* stage0 = base;
-  float* tk_val = reinterpret_cast<float*>(base + S * kStageBytes);
+  float* tk_val = reinterpret_cast<float*>(base + S * SB);
   int32_t* tk_id = reinterpret_cast<int32_t*>(tk_val + kBM * P.top_k);
   Barriers* bs = reinterpret_cast<Barriers*>(
       (reinterpret_cast<uintptr_t>(tk_id + kBM * P.top_k) + 15) & ~uintptr_t(15));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int units = P.m_blocks * P.splits;
+  const int units = P.m_units * P.splits;
   const int nkb = P.hidden / kBK;
+  // work-unit walk: CTAs (or CTA pairs) stride over (row unit, split)
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const bool leader = rank == 0;
+  const int u_first = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int u_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -195,22 +283,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bs->tfull[b], 1);
-      mbar_init(&bs->tempty[b], kBM);
+      mbar_init(&bs->tempty[b], PAIR ? 2 * kBM : kBM);  // both CTAs' epilogues in pair mode
     }
     bs->abort = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    // allocate the two accumulators (512 TMEM columns) for this CTA
-    asm volatile(
-        "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-            smem_addr(&bs->tmem_base)),
-        "r"(kTmemCols)
-        : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    // allocate the two accumulators (512 TMEM columns) for this CTA (both
+    // CTAs of a pair, same warp, same slot)
+    if constexpr (PAIR) {
+      asm volatile(
+          "tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+              smem_addr(&bs->tmem_base)),
+          "r"(kTmemCols)
+          : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      asm volatile(
+          "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+              smem_addr(&bs->tmem_base)),
+          "r"(kTmemCols)
+          : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_barrier();  // the peer's barriers are initialised
   tc_fence_after();
   const uint32_t tmem = bs->tmem_base;
 
@@ -221,8 +320,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
       uint32_t it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-        const int mb = u % P.m_blocks, sp = u / P.m_blocks;
+      for (int u = u_first; u < units && ok; u += u_step) {
+        const int mu = u % P.m_units, sp = u / P.m_units;
+        const int mb = PAIR ? 2 * mu + static_cast<int>(rank) : mu;
         const int t0 = sp * P.tiles_per_split, t1 = min(P.n_tiles, t0 + P.tiles_per_split);
         for (int t = t0; t < t1 && ok; ++t) {
           for (int kb = 0; kb < nkb; ++kb, ++it) {
@@ -232,26 +332,39 @@ __global__ void __launch_bounds__(kThreads, 1)
               ok = false;
               break;
             }
-            uint8_t* sa = stage0 + s * kStageBytes;
-            mbar_arrive_expect_tx(&bs->full[s], kStageBytes);
-            tma_load_2d(sa, &map_h, kb * kBK, mb * kBM, &bs->full[s]);
-            tma_load_2d(sa + kStageABytes, &map_w, kb * kBK, t * kBN, &bs->full[s]);
+            uint8_t* sa = stage0 + s * SB;
+            if constexpr (PAIR) {
+              // the leader's barrier counts both CTAs' bytes
+              if (leader) mbar_arrive_expect_tx(&bs->full[s], 2 * SB);
+              tma_load_2d_pair(sa, &map_h, kb * kBK, mb * kBM, &bs->full[s]);
+              tma_load_2d_pair(sa + SA, &map_w, kb * kBK, t * kBN + static_cast<int>(rank) * kBNh,
+                               &bs->full[s]);
+            } else {
+              mbar_arrive_expect_tx(&bs->full[s], SB);
+              tma_load_2d(sa, &map_h, kb * kBK, mb * kBM, &bs->full[s]);
+              tma_load_2d(sa + SA, &map_w, kb * kBK, t * kBN, &bs->full[s]);
+            }
           }
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // (pair mode: the leader CTA issues for both)
+    if (lane == 0 && leader) {
       uint32_t it = 0, tile = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-        const int sp = u / P.m_blocks;
+      for (int u = u_first; u < units && ok; u += u_step) {
+        const int sp = u / P.m_units;
         const int t0 = sp * P.tiles_per_split, t1 = min(P.n_tiles, t0 + P.tiles_per_split);
         for (int t = t0; t < t1 && ok; ++t, ++tile) {
           const int b = tile & 1;
           const uint32_t use = tile >> 1;
-          if (!wait_or_abort(&bs->tempty[b], (use & 1u) ^ 1u, bs, P.ws_err)) {
+          const bool freed = PAIR ? mbar_wait_cluster(&bs->tempty[b], (use & 1u) ^ 1u)
+                                  : wait_or_abort(&bs->tempty[b], (use & 1u) ^ 1u, bs, P.ws_err);
+          if (!freed) {
+            atomicOr(&bs->abort, 1u);
+            atomicOr(P.ws_err, 1u);
             ok = false;
             break;
           }
@@ -265,17 +378,29 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc_fence_after();
-            uint8_t* sa = stage0 + s * kStageBytes;
+            uint8_t* sa = stage0 + s * SB;
             const uint64_t ad = smem_desc_sw128(sa);
-            const uint64_t bd = smem_desc_sw128(sa + kStageABytes);
+            const uint64_t bd = smem_desc_sw128(sa + SA);
 #pragma unroll
             for (int kk = 0; kk < kBK / kUK; ++kk) {
               // advance 16 elements (32 bytes) along K inside the swizzle atom
-              umma_f16(dacc, ad + 2 * kk, bd + 2 * kk, (kb | kk) ? 1u : 0u);
+              if constexpr (PAIR)
+                umma_f16_pair(dacc, ad + 2 * kk, bd + 2 * kk, (kb | kk) ? 1u : 0u);
+              else
+                umma_f16(dacc, ad + 2 * kk, bd + 2 * kk, (kb | kk) ? 1u : 0u);
             }
-            umma_commit(&bs->empty[s]);  // frees the stage once these MMAs finish
+            // frees the stage (in both CTAs of a pair) once these MMAs finish
+            if constexpr (PAIR)
+              umma_commit_pair(&bs->empty[s]);
+            else
+              umma_commit(&bs->empty[s]);
           }
-          if (ok) umma_commit(&bs->tfull[b]);  // accumulator b complete
+          if (ok) {  // accumulator b complete
+            if constexpr (PAIR)
+              umma_commit_pair(&bs->tfull[b]);
+            else
+              umma_commit(&bs->tfull[b]);
+          }
         }
       }
     }
@@ -288,8 +413,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int32_t* my_id = tk_id + r * k;
     uint32_t tile = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-      const int mb = u % P.m_blocks, sp = u / P.m_blocks;
+    for (int u = u_first; u < units && ok; u += u_step) {
+      const int mu = u % P.m_units, sp = u / P.m_units;
+      const int mb = PAIR ? 2 * mu + static_cast<int>(rank) : mu;
       const int t0 = sp * P.tiles_per_split, t1 = min(P.n_tiles, t0 + P.tiles_per_split);
       const int row = mb * kBM + r;
       const bool row_ok = row < P.rows;
@@ -312,9 +438,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           float v[32];
           tmem_ld32(taddr + ch * 32, v);
           if (ch == kBN / 32 - 1) {
-            // every column of this buffer has been read: hand it back
+            // every column of this buffer has been read: hand it back (to
+            // the leader, which issues the pair's MMAs)
             tc_fence_before();
-            mbar_arrive(&bs->tempty[b]);
+            if constexpr (PAIR)
+              mbar_arrive_leader(&bs->tempty[b]);
+            else
+              mbar_arrive(&bs->tempty[b]);
           }
           const int col0 = t * kBN + ch * 32;
           if (!row_ok) continue;
@@ -366,11 +496,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   // MMAs of this CTA have completed before the accumulators are freed
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_barrier();  // the pair's MMAs and arrivals are done
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(kTmemCols)
-                 : "memory");
+    if constexpr (PAIR)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                   "r"(kTmemCols)
+                   : "memory");
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                   "r"(kTmemCols)
+                   : "memory");
   }
 }
 
@@ -602,15 +738,18 @@ int choose_splits(int m_blocks, int n_tiles, int sms) {
 }
 
 struct LmLayout {
-  int m_blocks, n_tiles, splits, tiles_per_split;
+  int m_blocks, m_units, n_tiles, splits, tiles_per_split;
   size_t off_stats, off_val, off_id, off_zy, off_err, total;
 };
 
-LmLayout lm_layout(int rows, int vocab, int top_k) {
+// Work layout and workspace.  Pair mode: row units of 256 rows over half as
+// many workers (CTA pairs).
+LmLayout lm_layout(int rows, int vocab, int top_k, bool pair) {
   LmLayout L{};
   L.m_blocks = (rows + kBM - 1) / kBM;
+  L.m_units = pair ? (L.m_blocks + 1) / 2 : L.m_blocks;
   L.n_tiles = (vocab + kBN - 1) / kBN;
-  L.splits = choose_splits(L.m_blocks, L.n_tiles, num_sms());
+  L.splits = choose_splits(L.m_units, L.n_tiles, pair ? num_sms() / 2 : num_sms());
   L.tiles_per_split = (L.n_tiles + L.splits - 1) / L.splits;
   L.splits = (L.n_tiles + L.tiles_per_split - 1) / L.tiles_per_split;
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
@@ -629,7 +768,10 @@ LmLayout lm_layout(int rows, int vocab, int top_k) {
 size_t lmhead_workspace_bytes(int rows, int vocab, int hidden, int top_k) {
   (void)hidden;
   if (rows <= 0 || vocab <= 0 || top_k <= 0) return 0;
-  return lm_layout(rows, vocab, top_k).total;
+  // enough for either launch mode
+  const size_t a = lm_layout(rows, vocab, top_k, true).total;
+  const size_t b = lm_layout(rows, vocab, top_k, false).total;
+  return a > b ? a : b;
 }
 
 vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh, const void* W,
@@ -660,12 +802,47 @@ vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh
   if (!H || !W || !targets) return bad(VS_ERR_INVALID_ARG, "hidden, weight and targets must be non-NULL");
   if (!a16(H) || !a16(W) || ldh % 8 != 0 || ldw % 8 != 0 || ldh < hidden || ldw < hidden)
     return bad(VS_ERR_INVALID_ARG, "hidden/weight must be 16-byte aligned with ld >= hidden_dim, ld % 8 == 0");
-  const LmLayout L = lm_layout(rows, vocab, top_k);
-  if (!ws || !a16(ws) || ws_bytes < L.total)
+  if (!ws || !a16(ws) || ws_bytes < lmhead_workspace_bytes(rows, vocab, hidden, top_k))
     return bad(VS_ERR_WORKSPACE, "workspace missing, misaligned or smaller than vs_fused_lmhead_workspace_size");
 
+  // Pair mode (two SMs per 256 x 256 tile, half the operand traffic per SM)
+  // when the device schedules clusters of two with this shared memory;
+  // otherwise one CTA per 128 x 256 tile.
+  const size_t lists = static_cast<size_t>(kBM) * top_k * 8;
+  const size_t fixed = 1024 + lists + 16 + sizeof(Barriers);
+  int stages2 = static_cast<int>((227 * 1024 - fixed) / kStageBytes2);
+  if (stages2 > kMaxStages) stages2 = kMaxStages;
+  const size_t smem2 = fixed + static_cast<size_t>(stages2) * kStageBytes2;
+  bool pair = stages2 >= 3;
+  cudaLaunchConfig_t cfg2{};
+  cudaLaunchAttribute attr2[1];
+  if (pair) {
+    cudaError_t e = cudaFuncSetAttribute(lmhead_gemm_kernel<true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem2));
+    attr2[0].id = cudaLaunchAttributeClusterDimension;
+    attr2[0].val.clusterDim.x = 2;
+    attr2[0].val.clusterDim.y = 1;
+    attr2[0].val.clusterDim.z = 1;
+    cfg2.gridDim = dim3(2, 1, 1);
+    cfg2.blockDim = dim3(kThreads, 1, 1);
+    cfg2.dynamicSmemBytes = smem2;
+    cfg2.stream = s;
+    cfg2.attrs = attr2;
+    cfg2.numAttrs = 1;
+    int nc = 0;
+    if (e != cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&nc, lmhead_gemm_kernel<true>, &cfg2) != cudaSuccess ||
+        nc < 1) {
+      cudaGetLastError();
+      pair = false;
+    }
+  }
+  const LmLayout L = lm_layout(rows, vocab, top_k, pair);
+
   CUtensorMap map_h, map_w;
-  if (!make_map(&map_h, H, rows, hidden, ldh, kBM) || !make_map(&map_w, W, vocab, hidden, ldw, kBN))
+  if (!make_map(&map_h, H, rows, hidden, ldh, kBM) ||
+      !make_map(&map_w, W, vocab, hidden, ldw, pair ? kBNh : kBN))
     return bad(VS_ERR_CUDA, "cuTensorMapEncodeTiled failed");
 
   uint8_t* w8 = static_cast<uint8_t*>(ws);
@@ -678,7 +855,8 @@ vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh
   P.tiles_per_split = L.tiles_per_split;
   P.n_tiles = L.n_tiles;
   P.m_blocks = L.m_blocks;
-  P.stages = top_k <= 24 ? 4 : 3;
+  P.m_units = L.m_units;
+  P.stages = pair ? stages2 : (top_k <= 24 ? 4 : 3);
   P.temperature = temperature;
   P.temperature_scalar = temperature_scalar;
   P.targets = targets;
@@ -688,16 +866,22 @@ vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh
   P.ws_zy = reinterpret_cast<float*>(w8 + L.off_zy);
   P.ws_err = reinterpret_cast<uint32_t*>(w8 + L.off_err);
 
-  const size_t smem = 1024 + static_cast<size_t>(P.stages) * kStageBytes +
-                      static_cast<size_t>(kBM) * top_k * 8 + 16 + sizeof(Barriers);
-  cudaError_t e = cudaFuncSetAttribute(lmhead_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return bad(VS_ERR_CUDA, cudaGetErrorString(e));
   lmhead_clear_kernel<<<1, 1, 0, s>>>(P.ws_err);
-  const int units = L.m_blocks * L.splits;
-  const int grid = units < num_sms() ? units : num_sms();
-  lmhead_gemm_kernel<<<grid, kThreads, smem, s>>>(map_h, map_w, P);
-  e = cudaGetLastError();
+  const int units = L.m_units * L.splits;
+  cudaError_t e;
+  if (pair) {
+    const int workers = num_sms() / 2;
+    cfg2.gridDim = dim3(2 * (units < workers ? units : workers), 1, 1);
+    e = cudaLaunchKernelEx(&cfg2, lmhead_gemm_kernel<true>, map_h, map_w, P);
+  } else {
+    const size_t smem = fixed + static_cast<size_t>(P.stages) * kStageBytes;
+    e = cudaFuncSetAttribute(lmhead_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return bad(VS_ERR_CUDA, cudaGetErrorString(e));
+    const int grid = units < num_sms() ? units : num_sms();
+    lmhead_gemm_kernel<false><<<grid, kThreads, smem, s>>>(map_h, map_w, P);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return bad(VS_ERR_CUDA, cudaGetErrorString(e));
 
   MergeParams M{};
