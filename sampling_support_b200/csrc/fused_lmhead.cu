@@ -19,9 +19,11 @@
 //   warps 2-5 epilogue: one thread per row reads its 256 accumulators with
 //            tcgen05.ld, releases the buffer, and folds the values into the
 //            row's online (max, count of max, sum 2^(u - max), sum (u - max)
-//            2^(u - max)) and into a top-k list (value desc, id asc) kept in
-//            shared memory.  At the end of a unit the row's partials go to
-//            the workspace.
+//            2^(u - max)) and into an unsorted top-k list in shared memory
+//            (per 32-column chunk each lane marks its candidates against the
+//            list's threshold and inserts them itself, so the lanes of a warp
+//            insert side by side).  At the end of a unit the row's partials
+//            go to the workspace, the list sorted by rank.
 // Kernel 2 (lmhead_merge_kernel), one thread per row: merges the split
 // partials in a fixed order, takes the top-k, applies inclusive top-p on the
 // top-k mass and min-p against the row max, and writes the outputs.
@@ -235,19 +237,47 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Ba
   return false;
 }
 
-// Insert (x, id) into a descending list of length k (count entries used);
-// equal values keep the earlier (lower) id first.
-__device__ __forceinline__ void topk_insert(float* vals, int32_t* ids, int k, int& count, float x,
-                                            int32_t id) {
-  int pos = count < k ? count : k - 1;
-  while (pos > 0 && vals[pos - 1] < x) {
-    vals[pos] = vals[pos - 1];
-    ids[pos] = ids[pos - 1];
-    --pos;
+// A row's running top-k is an unsorted list of up to k (value, id) entries.
+// Within a work unit ids arrive in ascending order, so a new element ranks
+// below every listed entry of equal value: once the list is full it is taken
+// only when it exceeds `thr`, the smallest listed value, and it replaces the
+// lowest-ranked entry (smallest value, then largest id) at `low`.
+__device__ __forceinline__ void topk_push(float* vals, int32_t* ids, int k, int& count, int& low,
+                                          float& thr, float x, int32_t id) {
+  const int slot = count < k ? count++ : low;
+  vals[slot] = x;
+  ids[slot] = id;
+  if (count == k) {
+    float mv = vals[0];
+    int32_t mi = ids[0];
+    int mp = 0;
+    for (int j = 1; j < k; ++j) {
+      const float vj = vals[j];
+      const int32_t ij = ids[j];
+      if (vj < mv || (vj == mv && ij > mi)) {
+        mv = vj;
+        mi = ij;
+        mp = j;
+      }
+    }
+    low = mp;
+    thr = mv;
   }
-  vals[pos] = x;
-  ids[pos] = id;
-  if (count < k) ++count;
+}
+
+// v[i] for a per-lane index i, by a five-level select tree on the bits of i
+// (static register indices only, so v stays in registers).
+__device__ __forceinline__ float pick32(const float (&v)[32], int i) {
+  float a[16], b[8], c[4];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) a[j] = (i & 1) ? v[2 * j + 1] : v[2 * j];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) b[j] = (i & 2) ? a[2 * j + 1] : a[2 * j];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) c[j] = (i & 4) ? b[2 * j + 1] : b[2 * j];
+  const float d0 = (i & 8) ? c[1] : c[0];
+  const float d1 = (i & 8) ? c[3] : c[2];
+  return (i & 16) ? d1 : d0;
 }
 
 template <bool PAIR>
@@ -423,8 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float c = kLog2e / T;
       const int y = row_ok ? P.targets[row] : -1;
       Stats st = stats_empty();
-      int count = 0;
-      float thr = -kInf;  // current k-th value (lists are full)
+      int count = 0, low = 0;
+      float thr = -kInf;  // smallest listed value once the list is full
       for (int t = t0; t < t1 && ok; ++t, ++tile) {
         const int b = tile & 1;
         const uint32_t use = tile >> 1;
@@ -448,34 +478,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const int col0 = t * kBN + ch * 32;
           if (!row_ok) continue;
+          // top-k candidates of this chunk against the threshold at its
+          // start (a stale threshold only admits extra candidates, which the
+          // exact test below drops); each lane walks its own candidates in
+          // ascending column order, so the warp's lanes insert side by side
+          uint32_t cand = 0;
           if (col0 + 32 <= P.vocab) {
             float uu[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) uu[i] = __fmul_rn(v[i], c);
             stats_add(st, uu);
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (v[i] > thr) {
-                topk_insert(my_val, my_id, k, count, v[i], col0 + i);
-                if (count == k) thr = my_val[k - 1];
-              }
-            if (y >= col0 && y < col0 + 32) {
-              float zy = 0.f;
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (y == col0 + i) zy = v[i];
-              P.ws_zy[row] = zy;
-            }
+            for (int i = 0; i < 32; ++i) cand |= (v[i] > thr ? 1u : 0u) << i;
           } else {
             for (int i = 0; i < 32 && col0 + i < P.vocab; ++i) {
-              float uu[1] = {__fmul_rn(v[i], c)};
+              float uu[1] = {__fmul_rn(pick32(v, i), c)};
               stats_add(st, uu);
-              if (v[i] > thr) {
-                topk_insert(my_val, my_id, k, count, v[i], col0 + i);
-                if (count == k) thr = my_val[k - 1];
-              }
-              if (y == col0 + i) P.ws_zy[row] = v[i];
             }
+            const int nv = P.vocab - col0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) cand |= (i < nv && v[i] > thr ? 1u : 0u) << i;
+          }
+          if (y >= col0 && y < col0 + 32) P.ws_zy[row] = pick32(v, y - col0);
+          while (cand != 0u) {
+            const int i = __ffs(cand) - 1;
+            cand &= cand - 1u;
+            const float x = pick32(v, i);
+            if (x > thr) topk_push(my_val, my_id, k, count, low, thr, x, col0 + i);
           }
         }
       }
@@ -484,9 +513,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         P.ws_stats[slot] = make_float4(st.m, st.c0, st.zr, st.a);
         float* dv = P.ws_val + slot * k;
         int32_t* di = P.ws_id + slot * k;
-        for (int i = 0; i < k; ++i) {
-          dv[i] = i < count ? my_val[i] : -kInf;
-          di[i] = i < count ? my_id[i] : -1;
+        // the split's list in the total order (value desc, id asc): each
+        // entry goes to its rank (ids are distinct, so ranks are too)
+        for (int j = 0; j < count; ++j) {
+          const float vj = my_val[j];
+          const int32_t ij = my_id[j];
+          int rk = 0;
+          for (int l = 0; l < count; ++l) {
+            const float vl = my_val[l];
+            rk += (vl > vj || (vl == vj && my_id[l] < ij)) ? 1 : 0;
+          }
+          dv[rk] = vj;
+          di[rk] = ij;
+        }
+        for (int j = count; j < k; ++j) {
+          dv[j] = -kInf;
+          di[j] = -1;
         }
       }
     }

@@ -107,3 +107,41 @@ def test_lmhead_workload_full_size_sampled_rows():
     nb, n = _check(wl["hidden_states"], wl["weight"], wl["targets"], wl["temperature"],
                    wl["top_k"], wl["top_p"], wl["min_p"], rows_checked=sel)
     print(f"lmhead full size: {nb} boundary rows of {n} checked")
+
+
+# ids of two groups of duplicated weight rows.  Group A holds a block of 24
+# consecutive ids inside one tile, so a top-k list fills with A entries tied
+# at its minimum; group B (the larger logit) follows in the same tile and
+# must evict the A entry with the largest id.  Both groups also straddle tile
+# and split boundaries.
+_TIE_A = list(range(1030, 1054)) + [2000, 2990]
+_TIE_B = [1250, 2500, 2999]
+
+
+@pytest.mark.parametrize("rows,vocab,k", [(130, 3000, 8), (130, 3000, 2), (2048, 4096, 20)])
+def test_fused_head_exact_ties(rows, vocab, k):
+    """Exactly tied logits (duplicated weight rows) come out in the total
+    order, value descending then id ascending, across in-list evictions and
+    the merge of vocabulary splits."""
+    hidden = 64
+    h, w, y = _case(rows, vocab, hidden, seed=31)
+    h[:, 0] = 0x4080  # 4.0: the duplicated rows' logits stand far above the rest
+    rest = w[7].copy()
+    for ids, lead in ((_TIE_A, 0x3F80), (_TIE_B, 0x3FA0)):  # 1.0, 1.25
+        w[ids] = rest
+        w[ids, 0] = lead
+    want = np.array(_TIE_B + _TIE_A, dtype=np.int32)
+    n = min(k, len(want))
+    out = vsb.fused_lmhead_score(to_device(h), to_device(w), torch.from_numpy(y).cuda(), 1.0, k,
+                                 1.0, 0.0)
+    torch.cuda.synchronize()
+    ids = out["topk_ids"].cpu().numpy()
+    lp = out["topk_logprob"].cpu().numpy()
+    assert np.array_equal(ids[:, :n], np.broadcast_to(want[:n], (rows, n)))
+    # a tie group shares one logprob bit for bit
+    nb = min(n, len(_TIE_B))
+    assert np.all(lp[:, :nb] == lp[:, :1])
+    if n > nb:
+        assert np.all(lp[:, nb:n] == lp[:, nb:nb + 1])
+    sel = np.linspace(0, rows - 1, 16).astype(np.int64)
+    _check(h, w, y, 1.0, k, 1.0, 0.0, rows_checked=sel)
