@@ -180,6 +180,40 @@ __device__ __forceinline__ void for_each_elem(const uint16_t* g, int j0, int j1,
   for (int j = j0 + nv * 8 + threadIdx.x; j < j1; j += NT) f(static_cast<uint32_t>(g[j]), j);
 }
 
+// Number of elements in [j0, j1) whose raw bits are r0 or r1 (the two
+// encodings of one key): the block's NT threads read 16-byte vectors
+// through L2 with kHistUnroll loads in flight each; j0 need not be a
+// multiple of 8.
+template <int NT>
+__device__ __forceinline__ uint32_t count_raw(const uint16_t* g, int j0, int j1, uint32_t r0,
+                                              uint32_t r1) {
+  uint32_t n = 0;
+  auto one = [&](uint32_t r) { n += (r == r0) | (r == r1) ? 1u : 0u; };
+  auto vec = [&](const uint4& q) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      one(w[i] & 0xFFFFu);
+      one(w[i] >> 16);
+    }
+  };
+  const int ja = min(j1, (j0 + 7) & ~7);
+  for (int j = j0 + static_cast<int>(threadIdx.x); j < ja; j += NT) one(g[j]);
+  const int nv = (j1 - ja) >> 3;
+  const uint4* v4 = reinterpret_cast<const uint4*>(g + ja);
+  int v = threadIdx.x;
+  for (; v + (kHistUnroll - 1) * NT < nv; v += kHistUnroll * NT) {
+    uint4 q[kHistUnroll];
+#pragma unroll
+    for (int k = 0; k < kHistUnroll; ++k) q[k] = __ldcg(v4 + v + k * NT);
+#pragma unroll
+    for (int k = 0; k < kHistUnroll; ++k) vec(q[k]);
+  }
+  for (; v < nv; v += NT) vec(__ldcg(v4 + v));
+  for (int j = ja + nv * 8 + static_cast<int>(threadIdx.x); j < j1; j += NT) one(g[j]);
+  return n;
+}
+
 // 8-bit radix descent over the keys of the whole row: the key where the
 // cumulative count (by_mass false) or mass reaches target.  target 0 with
 // by_mass asks for the top-p target of the full mass (p).
@@ -554,6 +588,7 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
   int32_t tie_cut = INT_MAX;
   bool cut_known = true;  // tie_cut resolved (or not needed: every tie kept)
   u64 ckeep = 0;
+  u64 tie_group = 0;  // elements holding the threshold key
   float log2zs = log2z, h_support = h_full, c0s = st.c0, zrs = st.zr;
   int32_t n_support = nonfinite ? 0 : V;
   bool from_bins = false;  // the threshold lies inside the window
@@ -722,6 +757,7 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
     const uint32_t ngt = sums.ngt, neq = sums.neq, ntp = sums.ntp;
     const float smass = sums.smass, sa = sums.sa;
     const u64 tot_eq = neq;
+    tie_group = tot_eq;
     ckeep = all_ties ? tot_eq : (cnum < tot_eq ? cnum : tot_eq);
     const float dt = key_u(tkey, c) - mr;
     const float et = ex2(dt);
@@ -750,10 +786,15 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
   // ---- the target's earlier ties, when its membership hinges on them
   uint32_t ylt_row = 0;
   if (filtered && !cut_known && target_ok && bf16_key(ry) == tkey) {
-    uint32_t part = 0;
-    const uint32_t t = tkey;
-    for_each_elem<kMT>(grow, 0, y, [&](uint32_t raw, int) { part += bf16_key(raw) == t; });
-    ylt_row = block_sum(part, sh.ured);
+    // counted on the shorter side of y: after y, the group less the target
+    // and the ties that follow it
+    const uint32_t r0 = tkey >= 0x7FFFu ? tkey - 0x7FFFu : 0xFFFFu - tkey;
+    const uint32_t r1 = tkey == 0x7FFFu ? 0x8000u : r0;  // -0 shares the key of +0
+    const bool before = y <= V - 1 - y;
+    const uint32_t part = before ? count_raw<kMT>(grow, 0, y, r0, r1)
+                                 : count_raw<kMT>(grow, y + 1, V, r0, r1);
+    const uint32_t n = block_sum(part, sh.ured);
+    ylt_row = before ? n : static_cast<uint32_t>(tie_group) - 1u - n;
   }
 
   // ---- per-row outputs

@@ -396,3 +396,66 @@ def test_replay_backward_full_size_sampled_rows():
     gref = oracle.score_grad(w["logits"][sel], w["targets"][sel], None, np.ones(len(sel)), None,
                              np.full(len(sel), 0.01), support=w["support"][sel])
     compare_grad(dl[torch.from_numpy(sel).cuda()].cpu().numpy()[:, :vocab], gref)
+
+
+def _run_nomask(logits, targets, temperature, top_k, top_p, min_p):
+    """GPU forward as a caller with no support mask and no saved state asks
+    for it (the tie cut at the threshold is then resolved for the target
+    alone), against the oracle; rows off the top-p / min-p boundary band."""
+    rows, vocab = logits.shape
+    t_np = np.asarray(temperature, F32)
+    k_arg = torch.from_numpy(np.asarray(top_k, np.int32)).cuda() if np.ndim(top_k) else top_k
+    out = vsb.score_fwd(to_device(logits), torch.from_numpy(np.asarray(targets, np.int32)).cuda(),
+                        temperature=torch.from_numpy(t_np).cuda() if t_np.ndim else float(t_np),
+                        top_k=k_arg, top_p=float(F32(top_p)), min_p=float(F32(min_p)))
+    torch.cuda.synchronize()
+    t64 = t_np.astype(np.float64)
+    ref = oracle.score(logits, targets, temperature=t64 if t64.ndim else float(t64),
+                       top_k=np.asarray(top_k, np.int32) if np.ndim(top_k) else top_k,
+                       top_p=float(F32(top_p)), min_p=float(F32(min_p)))
+    sure = ~((ref["topp_margin"] < 1e-6) | (ref["minp_margin"] < 1e-6))
+    get = {k: v.cpu().numpy() for k, v in out.items()}
+    assert np.array_equal(get["valid"], ref["valid"])
+    assert np.array_equal(get["support_size"][sure], ref["support_size"][sure])
+    assert np.array_equal(get["status"][sure].astype(np.int64), map_status(ref["status"][sure]))
+    lps = get["lp_support"].astype(np.float64)[sure]
+    want = ref["lp_support"][sure]
+    assert np.array_equal(lps == -np.inf, want == -np.inf)
+    fin = np.isfinite(want)
+    assert np.abs(lps[fin] - want[fin]).max(initial=0) <= 1e-4
+    return ref, sure
+
+
+def test_target_in_threshold_tie_group_without_mask():
+    """The target inside the threshold's tie group with part of the group
+    kept (the lowest ids first): membership is decided by the ties before
+    it, counted on either side of the target."""
+    rows, vocab, G, H = 8, 40_000, 400, 50
+    x = np.minimum(workloads.normal((rows, vocab), 1.0, 23, stream=1), 3.5)
+    rng = np.random.default_rng(23)
+    top_k = np.zeros(rows, np.int32)
+    targets = np.zeros(rows, np.int32)
+    for i in range(rows):
+        lo = 0 if i < 4 else vocab // 2 + 1  # rows 4-7: the whole group after the middle
+        ids = rng.choice(np.arange(lo, vocab), G + H, replace=False)
+        grp, hi = np.sort(ids[:G]), ids[G:]
+        x[i, grp] = 5.0
+        x[i, hi] = 6.0
+        c = G // 2 if i < 4 else G - 2
+        top_k[i] = H + c
+        targets[i] = [grp[c - 1], grp[c], grp[-1], grp[0], grp[c - 1], grp[c], grp[-1], hi[0]][i]
+    logits = workloads.to_bf16_bits(x)
+    ref, sure = _run_nomask(logits, targets, 1.0, top_k, 1.0, 0.0)
+    assert sure.all()
+    kept = np.isfinite(ref["lp_support"])
+    assert kept.tolist() == [True, False, False, True, True, False, False, True]
+
+
+@pytest.mark.slow
+def test_fullvocab_workload_full_size_without_mask():
+    """The fullvocab workload (128 x 151,936 bf16, top-p 0.95) exactly as the
+    benchmark calls it: no support mask, no saved state."""
+    w = workloads.fullvocab()
+    ref, sure = _run_nomask(w["logits"], w["targets"], w["temperature"], w["top_k"], w["top_p"],
+                            w["min_p"])
+    print(f"fullvocab without mask: {int((~sure).sum())} boundary rows skipped")
