@@ -333,8 +333,9 @@ def secondary(args, pk, only=None):
         distance_workload(args, pk, steps, out)
     if only in (None, "replay"):
         replay_workload(args, pk, steps, out)
-    if only in (None, "lmhead"):
-        lmhead_workload(args, pk, steps, out)
+    if only in (None, "lmhead", "support_head"):
+        lmhead_workload(args, pk, steps, out, fused=only in (None, "lmhead"),
+                        support=only in (None, "support_head"))
     return out
 
 
@@ -405,8 +406,10 @@ def replay_workload(args, pk, steps, out):
     torch.cuda.empty_cache()
 
 
-def lmhead_workload(args, pk, steps, out):
-    """Fused LM head: 8192 x 4096 hidden, 151,936 x 4096 weight, top-20 -> top-p -> min-p."""
+def lmhead_workload(args, pk, steps, out, fused=True, support=True):
+    """Fused LM head: 8192 x 4096 hidden, 151,936 x 4096 weight, top-20 -> top-p -> min-p;
+    and the support-only projection of the same hidden states and weight over
+    replay-recipe supports (Zipf ids, up to 64 per row)."""
     import torch
 
     import sampling_support_b200 as vsb
@@ -415,23 +418,63 @@ def lmhead_workload(args, pk, steps, out):
     w = workloads.lmhead()
     hs, wt = to_dev(w["hidden_states"]), to_dev(w["weight"])
     tg = to_dev(w["targets"])
-    lm = vsb.load()
-    nbytes = lm.vs_fused_lmhead_workspace_size(w["rows"], w["vocab"], w["hidden"], w["top_k"])
-    wsp = torch.empty(nbytes + 16, dtype=torch.uint8, device="cuda")
+    if fused:
+        lm = vsb.load()
+        nbytes = lm.vs_fused_lmhead_workspace_size(w["rows"], w["vocab"], w["hidden"], w["top_k"])
+        wsp = torch.empty(nbytes + 16, dtype=torch.uint8, device="cuda")
 
-    def lm_step():
-        vsb.fused_lmhead_score(hs, wt, tg, w["temperature"], w["top_k"],
-                               float(np.float32(w["top_p"])), float(np.float32(w["min_p"])),
-                               workspace=wsp)
+        def lm_step():
+            vsb.fused_lmhead_score(hs, wt, tg, w["temperature"], w["top_k"],
+                                   float(np.float32(w["top_p"])), float(np.float32(w["min_p"])),
+                                   workspace=wsp)
 
-    ms = time_steps(lm_step, 2, max(3, min(steps, 10)))
-    flops = 2.0 * w["rows"] * w["vocab"] * w["hidden"]
-    tf = flops / (ms / 1e3) / 1e12
-    out["lmhead"] = {"rows": w["rows"], "vocab": w["vocab"], "hidden": w["hidden"],
-                     "ms_per_step": ms, "rows_per_s": w["rows"] / (ms / 1e3), "tflops": tf,
-                     "frac_bf16_burst": tf / pk["bf16"], "frac_bf16_sustained": tf / pk["bf16_sustained"],
-                     "flops": flops}
-    del hs, wt, wsp
+        ms = time_steps(lm_step, 2, max(3, min(steps, 10)))
+        flops = 2.0 * w["rows"] * w["vocab"] * w["hidden"]
+        tf = flops / (ms / 1e3) / 1e12
+        out["lmhead"] = {"rows": w["rows"], "vocab": w["vocab"], "hidden": w["hidden"],
+                         "ms_per_step": ms, "rows_per_s": w["rows"] / (ms / 1e3), "tflops": tf,
+                         "frac_bf16_burst": tf / pk["bf16"],
+                         "frac_bf16_sustained": tf / pk["bf16_sustained"], "flops": flops}
+        del wsp
+    if support:
+        sup = workloads.support_lists(rows=w["rows"], vocab=w["vocab"])
+        ids, ty = to_dev(sup["support"]), to_dev(sup["targets"])
+        # L2 flushed before every timed call: only the reuse of weight rows
+        # within one call (rows sharing support ids) is served from L2
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        s = torch.cuda.current_stream()
+
+        def sh_step():
+            vsb.support_lmhead_score(hs, wt, ty, w["temperature"], ids)
+
+        for _ in range(3):
+            sh_step()
+        torch.cuda.synchronize()
+        n = max(5, min(steps, 20))
+        tot = 0.0
+        for _ in range(n):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(s)
+            sh_step()
+            b.record(s)
+            torch.cuda.synchronize()
+            tot += a.elapsed_time(b)
+        ms = tot / n
+        kept = int(sum(len(set(int(x) for x in r if x >= 0)) for r in sup["support"]))
+        uniq = len(set(int(x) for x in sup["support"].reshape(-1) if x >= 0))
+        gathered = 2 * w["hidden"] * (w["rows"] + kept) + 4 * sup["support"].size + 17 * w["rows"]
+        unique_bytes = 2 * w["hidden"] * (w["rows"] + uniq) + 4 * sup["support"].size
+        out["support_head"] = {
+            "rows": w["rows"], "hidden": w["hidden"], "vocab": w["vocab"],
+            "width": int(sup["support"].shape[1]), "kept_ids": kept, "unique_ids": uniq,
+            "ms_per_step": ms, "rows_per_s": w["rows"] / (ms / 1e3),
+            "gather_gbs": gathered / (ms / 1e3) / 1e9,
+            "frac_hbm_unique": unique_bytes / (ms / 1e3) / 1e9 / pk["hbm"],
+            "note": "gather_gbs counts every kept id's weight row; frac_hbm_unique counts each "
+                    "distinct weight row once (the rest can come from L2); L2 flushed per call"}
+        del flush, ids, ty
+    del hs, wt
     torch.cuda.empty_cache()
 
 
@@ -514,7 +557,7 @@ def main():
     ap.add_argument("--sub-steps", type=int, default=50)
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["distance", "replay", "lmhead"], default=None,
+    ap.add_argument("--only", choices=["distance", "replay", "lmhead", "support_head"], default=None,
                     help="time one secondary workload alone (one GPU) and print its line")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -77,6 +77,8 @@ typedef int32_t vs_dtype;
 #define VS_ROW_BAD_SUPPORT_ID (1u << 2)        /* a recorded id < -1 or >= vocab: ignored */
 #define VS_ROW_DUP_SUPPORT_ID (1u << 3)        /* a recorded id repeated: counted once */
 #define VS_ROW_NONFINITE_INPUT (1u << 4)       /* NaN/inf logit: outputs NaN, valid 0 */
+#define VS_ROW_DEVICE_TIMEOUT (1u << 5)        /* a bounded device wait gave up: outputs unreliable */
+#define VS_ROW_EMPTY_SUPPORT (1u << 6)         /* vs_support_lmhead_score: no kept id, lp_S NaN */
 
 /* bytes of saved state per row written when VS_WANT_GRAD is set */
 #define VS_CTX_BYTES_PER_ROW 64
@@ -273,6 +275,38 @@ vs_status vs_fused_lmhead_score(int32_t rows, int32_t vocab, int32_t hidden_dim,
 
 size_t vs_fused_lmhead_workspace_size(int32_t rows, int32_t vocab, int32_t hidden_dim,
                                       int32_t top_k);
+
+/* Support-only fused projection ([SkyRL] Performance: with a fused LM head
+ * the replay path projects only the selected hidden-state / weight pairs and
+ * never materialises vocabulary logits; Implementation: dense -1-padded
+ * support lists).  For row i and each kept id s of support_ids[i, :width]
+ * (0 <= s < vocab, first occurrence; -1 pads anywhere are skipped, other
+ * out-of-range ids set VS_ROW_BAD_SUPPORT_ID, repeats VS_ROW_DUP_SUPPORT_ID):
+ *   z[i, s] = (sum_k hidden[i, k] * weight[s, k]) / T_i
+ * (bf16 inputs, fp32 accumulation), then over the kept set S_i:
+ * logprob_support = z_y - log sum_S exp z (-inf and
+ * VS_ROW_TARGET_NOT_IN_SUPPORT when y is not kept), entropy_support =
+ * -sum_S q log q (exactly 0 for a singleton; needs VS_WANT_ENTROPY), valid,
+ * status and support_size, as vs_score_fwd gives them for a recorded
+ * support.  The work scales with the support width, not with vocab.
+ * A row with no kept id has no full-vocabulary fallback here (it needs the
+ * full projection, vs_fused_lmhead_score): logprob_support NaN, entropy 0,
+ * valid 0, status VS_ROW_EMPTY_SUPPORT.  Non-finite projections: outputs NaN,
+ * valid 0, VS_ROW_NONFINITE_INPUT.
+ * hidden [rows, hidden_dim] (row stride ldh) and weight [vocab, hidden_dim]
+ * (row stride ldw) are bf16, 16-byte aligned, strides multiples of 8;
+ * hidden_dim a multiple of 8, at most 16384.  support_ids [rows, support_ld]
+ * int32, width in [0, VS_MAX_SUPPORT_WIDTH].  out->logprob_full,
+ * entropy_full, support_mask and ctx must be NULL (VS_ERR_INVALID_ARG).  When
+ * support_logits is non-NULL it receives [rows, logits_ld] fp32: z[i, s] at
+ * each kept slot, -inf at pads, bad and repeated ids.  No workspace. */
+vs_status vs_support_lmhead_score(int32_t rows, int32_t vocab, int32_t hidden_dim,
+                                  const void* hidden, int64_t ldh, const void* weight,
+                                  int64_t ldw, const float* temperature, float temperature_scalar,
+                                  const int32_t* targets, const int32_t* support_ids,
+                                  int32_t support_width, int64_t support_ld, uint32_t flags,
+                                  const vs_score_out* out, float* support_logits,
+                                  int64_t logits_ld, void* stream);
 
 /* Message describing the last failed call on this thread ("" after success). */
 const char* vs_last_error(void);

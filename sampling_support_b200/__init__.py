@@ -10,11 +10,13 @@ from ._binding import (  # noqa: F401
     load,
     score_bwd,
     score_fwd,
+    support_lmhead_score,
 )
 from ._binding import (  # noqa: F401
     ROW_BAD_SUPPORT_ID,
     ROW_DEVICE_TIMEOUT,
     ROW_DUP_SUPPORT_ID,
+    ROW_EMPTY_SUPPORT,
     ROW_NONFINITE_INPUT,
     ROW_TARGET_NOT_IN_SUPPORT,
     ROW_TARGET_OUT_OF_RANGE,

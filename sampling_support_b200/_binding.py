@@ -30,6 +30,7 @@ ROW_BAD_SUPPORT_ID = 1 << 2
 ROW_DUP_SUPPORT_ID = 1 << 3
 ROW_NONFINITE_INPUT = 1 << 4
 ROW_DEVICE_TIMEOUT = 1 << 5
+ROW_EMPTY_SUPPORT = 1 << 6
 
 _vp = ctypes.c_void_p
 
@@ -94,6 +95,11 @@ def load() -> ctypes.CDLL:
         lib.vs_fused_lmhead_score.restype = i32
         lib.vs_fused_lmhead_workspace_size.argtypes = [i32, i32, i32, i32]
         lib.vs_fused_lmhead_workspace_size.restype = sz
+        lib.vs_support_lmhead_score.argtypes = [i32, i32, i32, _vp, ctypes.c_int64, _vp,
+                                                ctypes.c_int64, _vp, ctypes.c_float, _vp, _vp, i32,
+                                                ctypes.c_int64, ctypes.c_uint32,
+                                                ctypes.POINTER(ScoreOut), _vp, ctypes.c_int64, _vp]
+        lib.vs_support_lmhead_score.restype = i32
         lib.vs_last_error.restype = ctypes.c_char_p
         lib.vs_version.restype = ctypes.c_char_p
         _lib = lib
@@ -317,4 +323,43 @@ def fused_lmhead_score(hidden, weight, targets, temperature, top_k, top_p, min_p
                                      VS_WANT_ENTROPY if want_entropy else 0, ctypes.byref(o),
                                      _p(out["topk_ids"]), _p(out["topk_logprob"]), _p(workspace),
                                      workspace.numel(), _stream(stream)))
+    return out
+
+
+def support_lmhead_score(hidden, weight, targets, temperature, support_ids, want_entropy=True,
+                         want_logits=False, stream=None):
+    """Support-only fused projection: z = hidden[i] . weight[s] / T_i for the
+    kept ids s of each row's recorded support, then lp_S, H_S, valid, status
+    and support size (no full-vocabulary quantity)."""
+    lib = load()
+    rows, hdim = hidden.shape
+    vocab = weight.shape[0]
+    width = support_ids.shape[1]
+    dev = hidden.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {
+        "lp_support": torch.empty(rows, **f32),
+        "valid": torch.empty(rows, dtype=torch.uint8, device=dev),
+        "status": torch.empty(rows, dtype=torch.int32, device=dev),
+        "support_size": torch.empty(rows, dtype=torch.int32, device=dev),
+    }
+    if want_entropy:
+        out["h_support"] = torch.empty(rows, **f32)
+    if want_logits:
+        out["support_logits"] = torch.empty((rows, width), **f32)
+    o = ScoreOut()
+    o.logprob_support = _p(out["lp_support"])
+    o.entropy_support = _p(out.get("h_support"))
+    o.valid = _p(out["valid"])
+    o.status = _p(out["status"])
+    o.support_size = _p(out["support_size"])
+    t_arr = temperature if isinstance(temperature, torch.Tensor) else None
+    t_s = 1.0 if t_arr is not None else float(temperature)
+    lg = out.get("support_logits")
+    _check(lib.vs_support_lmhead_score(rows, vocab, hdim, _p(hidden), hidden.stride(0), _p(weight),
+                                       weight.stride(0), _p(t_arr), t_s, _p(targets),
+                                       _p(support_ids), width, support_ids.stride(0),
+                                       VS_WANT_ENTROPY if want_entropy else 0, ctypes.byref(o),
+                                       _p(lg), lg.stride(0) if lg is not None else 0,
+                                       _stream(stream)))
     return out

@@ -22,6 +22,12 @@ vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh
                      uint32_t flags, const vs_score_out* out, int32_t* topk_ids,
                      float* topk_logprob, void* ws, size_t ws_bytes, cudaStream_t s,
                      std::string* err);
+vs_status support_head_run(int rows, int vocab, int hidden, const void* H, int64_t ldh,
+                           const void* W, int64_t ldw, const float* temperature,
+                           float temperature_scalar, const int32_t* targets,
+                           const int32_t* support_ids, int width, int64_t support_ld,
+                           uint32_t flags, const vs_score_out* out, float* support_logits,
+                           int64_t logits_ld, cudaStream_t s, std::string* err);
 }  // namespace vs
 
 namespace {
@@ -316,6 +322,22 @@ vs_status vs_fused_lmhead_score(int32_t rows, int32_t vocab, int32_t hidden_dim,
                                 temperature_scalar, targets, top_k, top_p, min_p, flags, out,
                                 topk_ids, topk_logprob, workspace, workspace_bytes,
                                 static_cast<cudaStream_t>(stream), &err);
+  if (st != VS_OK) return fail(st, err);
+  return ok();
+}
+
+vs_status vs_support_lmhead_score(int32_t rows, int32_t vocab, int32_t hidden_dim,
+                                  const void* hidden, int64_t ldh, const void* weight,
+                                  int64_t ldw, const float* temperature, float temperature_scalar,
+                                  const int32_t* targets, const int32_t* support_ids,
+                                  int32_t support_width, int64_t support_ld, uint32_t flags,
+                                  const vs_score_out* out, float* support_logits,
+                                  int64_t logits_ld, void* stream) {
+  std::string err;
+  vs_status st = vs::support_head_run(rows, vocab, hidden_dim, hidden, ldh, weight, ldw,
+                                      temperature, temperature_scalar, targets, support_ids,
+                                      support_width, support_ld, flags, out, support_logits,
+                                      logits_ld, static_cast<cudaStream_t>(stream), &err);
   if (st != VS_OK) return fail(st, err);
   return ok();
 }

@@ -18,7 +18,7 @@ constexpr float kInf = __builtin_huge_valf();
 constexpr uint32_t kWaitLimit = 1u << 24;
 
 // Per-row status bit set when a bounded device wait gave up (never expected).
-constexpr uint32_t kRowDeviceTimeout = 1u << 5;
+constexpr uint32_t kRowDeviceTimeout = 1u << 5;  // VS_ROW_DEVICE_TIMEOUT
 
 // 2^x on the MUFU unit (ex2.approx.ftz.f32: PTX ISA instruction, relative
 // error about 2^-22; -inf -> +0).

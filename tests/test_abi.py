@@ -138,3 +138,55 @@ def test_score_fwd_workspace_only_for_bf16_computed_support():
         B.VS_ERR_WORKSPACE
     assert lib.vs_score_fwd(ctypes.byref(a), ctypes.byref(o), FAKE, size(a) - 16, None) == \
         B.VS_ERR_WORKSPACE
+
+
+def _support_head(rows=4, vocab=1000, hidden=64, H=FAKE, ldh=64, W=FAKE, ldw=64, temp=1.0,
+                  targets=FAKE, ids=FAKE, width=8, sld=8, flags=None, out=None, logits=None,
+                  lld=0):
+    lib = vsb.load()
+    o = out if out is not None else B.ScoreOut()
+    flags = B.VS_WANT_ENTROPY if flags is None else flags
+    return lib.vs_support_lmhead_score(rows, vocab, hidden, H, ldh, W, ldw, None, temp, targets,
+                                       ids, width, sld, flags, ctypes.byref(o), logits, lld, None)
+
+
+def test_support_head_rejects_bad_arguments():
+    inv, uns = B.VS_ERR_INVALID_ARG, B.VS_ERR_UNSUPPORTED
+    assert _support_head(rows=-1) == inv
+    assert _support_head(vocab=0) == inv
+    assert _support_head(hidden=60, ldh=64, ldw=64) == uns      # not a multiple of 8
+    assert _support_head(hidden=16392, ldh=16392, ldw=16392) == uns  # beyond 16384
+    assert _support_head(width=B.VS_MAX_SUPPORT_WIDTH + 1, sld=2048) == uns
+    assert _support_head(width=8, sld=7) == inv
+    assert _support_head(temp=0.0) == inv
+    assert _support_head(temp=float("nan")) == inv
+    assert _support_head(H=FAKE + 8) == inv
+    assert _support_head(ldh=60, hidden=56) == inv
+    assert _support_head(ldh=56, hidden=64) == inv
+    assert _support_head(targets=0) == inv
+    assert _support_head(ids=0) == inv
+    assert _support_head(flags=1 << 1) == inv                  # no mask on this path
+    assert _support_head(logits=FAKE, lld=7) == inv
+    for field in ("logprob_full", "entropy_full", "support_mask", "ctx"):
+        o = B.ScoreOut()
+        setattr(o, field, FAKE)
+        assert _support_head(out=o) == inv, field
+    o = B.ScoreOut()
+    o.entropy_support = FAKE
+    assert _support_head(out=o, flags=0) == inv               # entropy needs VS_WANT_ENTROPY
+    assert "full projection" in _last_error_after(lambda: _support_head(
+        out=_with(B.ScoreOut(), "logprob_full", FAKE)))
+
+
+def _with(o, field, value):
+    setattr(o, field, value)
+    return o
+
+
+def _last_error_after(call):
+    call()
+    return vsb.load().vs_last_error().decode()
+
+
+def test_support_head_zero_rows_is_a_no_op():
+    assert _support_head(rows=0, H=0, W=0, targets=0, ids=0) == B.VS_OK

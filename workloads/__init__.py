@@ -183,9 +183,11 @@ def _zipf_cdf(vocab: int, s: float) -> np.ndarray:
     return c / c[-1]
 
 
-def replay(rows: int = 8192, vocab: int = VOCAB, seed: int = 3, width: int = 64,
-           boost: float = 6.0, zipf_s: float = 1.1) -> dict:
-    x = normal((rows, vocab), 3.0, seed, stream=1)
+def _zipf_support_lists(rows: int, vocab: int, seed: int, width: int, zipf_s: float):
+    """Per row `width` distinct ids drawn from Zipf(zipf_s) over ranks 1..V
+    (id = rank - 1), and a recorded width per row: 0 with probability 0.02, 1
+    with 0.10, else U{1..width}; returns (ids [rows, width], widths,
+    support [rows, width] -1 padded)."""
     cdf = _zipf_cdf(vocab, zipf_s)
     g = _gen(np.random.SeedSequence([seed, 2, 0x21]))
     boosted = np.empty((rows, width), dtype=np.int32)
@@ -202,15 +204,22 @@ def replay(rows: int = 8192, vocab: int = VOCAB, seed: int = 3, width: int = 64,
                     if len(chosen) == width:
                         break
         boosted[i] = chosen
-    rows_idx = np.repeat(np.arange(rows), width)
-    x[rows_idx, boosted.reshape(-1)] += np.float32(boost)
-    logits = to_bf16_bits(x)
     u = uniform(rows, 0.0, 1.0, seed, 3)
     widths = integers(rows, 1, width + 1, seed, 4)
     widths = np.where(u < 0.02, 0, np.where(u < 0.12, 1, widths)).astype(np.int32)
     support = np.full((rows, width), -1, dtype=np.int32)
     for i in range(rows):
         support[i, : widths[i]] = boosted[i, : widths[i]]
+    return boosted, widths, support
+
+
+def replay(rows: int = 8192, vocab: int = VOCAB, seed: int = 3, width: int = 64,
+           boost: float = 6.0, zipf_s: float = 1.1) -> dict:
+    x = normal((rows, vocab), 3.0, seed, stream=1)
+    boosted, widths, support = _zipf_support_lists(rows, vocab, seed, width, zipf_s)
+    rows_idx = np.repeat(np.arange(rows), width)
+    x[rows_idx, boosted.reshape(-1)] += np.float32(boost)
+    logits = to_bf16_bits(x)
     # targets: Gumbel-max over the recorded support at T = 1; uniform when empty
     gt = _gen(np.random.SeedSequence([seed, 5, 0x6B]))
     lf = bf16_bits_to_f32(logits)
@@ -226,6 +235,22 @@ def replay(rows: int = 8192, vocab: int = VOCAB, seed: int = 3, width: int = 64,
     return dict(name="replay", rows=rows, vocab=vocab, dtype="bf16", logits=logits,
                 support=support, widths=widths, targets=targets,
                 temperature=np.ones(rows, dtype=np.float32))
+
+
+def support_lists(rows: int = 8192, vocab: int = VOCAB, seed: int = 3, width: int = 64,
+                  zipf_s: float = 1.1) -> dict:
+    """Recorded supports of the replay recipe (Zipf ids, width mix) for the
+    support-only projection, with targets drawn uniformly from each row's
+    support (uniform over the vocabulary for an empty support)."""
+    _, widths, support = _zipf_support_lists(rows, vocab, seed, width, zipf_s)
+    pick = uniform(rows, 0.0, 1.0, seed, 7)
+    uni = integers(rows, 0, vocab, seed, 6)
+    targets = np.empty(rows, dtype=np.int32)
+    for i in range(rows):
+        w = int(widths[i])
+        targets[i] = uni[i] if w == 0 else support[i, min(w - 1, int(pick[i] * w))]
+    return dict(name="support_lists", rows=rows, vocab=vocab, support=support, widths=widths,
+                targets=targets)
 
 
 def lmhead(rows: int = 8192, vocab: int = VOCAB, hidden: int = 4096, seed: int = 4) -> dict:
