@@ -9,10 +9,11 @@
 //
 // then the support-conditioned log-probability of the target and the
 // support entropy, as for a recorded support.  The work scales with the
-// support width, not the vocabulary: one CTA per row stages the hidden state
-// in shared memory, and its warps each stream whole weight rows (coalesced
-// 16-byte loads, several in flight per lane) into one dot product per kept
-// id.  Weight rows that several rows' supports share are read from L2.
+// support width, not the vocabulary: one 128-thread CTA per row stages the
+// hidden state in shared memory, and its warps each stream whole weight rows
+// (coalesced 16-byte loads, eight in flight per lane; one mixed-precision
+// bf16 x bf16 + fp32 FMA per element) into one dot product per kept id.
+// Weight rows that several rows' supports share are read from L2.
 
 #include <cmath>
 #include <string>
@@ -26,9 +27,9 @@ static_assert(kRowDeviceTimeout == VS_ROW_DEVICE_TIMEOUT, "status bit of a devic
 
 namespace {
 
-constexpr int kSHThreads = 256;
+constexpr int kSHThreads = 128;
 constexpr int kSHWarps = kSHThreads / 32;
-constexpr int kSHUnroll = 4;         // 16-byte weight loads in flight per lane
+constexpr int kSHUnroll = 8;         // 16-byte weight loads in flight per lane
 constexpr int kSHMaxHidden = 16384;  // hidden state staged in shared memory (32 KB)
 
 struct SupportHeadParams {
@@ -52,23 +53,28 @@ struct SupportHeadParams {
   int64_t logits_ld;
 };
 
+// lo += h.lo * w.lo, hi += h.hi * w.hi for the bf16 pairs of two words: one
+// mixed-precision FMA per element (bf16 operands widen exactly, one fp32
+// rounding), so no separate conversion instructions.
+__device__ __forceinline__ void fma_bf16x2(uint32_t h, uint32_t w, float& lo, float& hi) {
+  asm("{\n .reg .b16 hl, hh, wl, wh;\n mov.b32 {hl, hh}, %2;\n mov.b32 {wl, wh}, %3;\n"
+      " fma.rn.f32.bf16 %0, hl, wl, %0;\n fma.rn.f32.bf16 %1, hh, wh, %1;\n}\n"
+      : "+f"(lo), "+f"(hi)
+      : "r"(h), "r"(w));
+}
+
 // Dot product of the staged hidden state with weight row w (the warp's
 // lanes take 8 consecutive elements per 256-element step); every lane
 // returns the warp's sum, reduced in a fixed order.
 __device__ __forceinline__ float warp_dot(const uint4* hs4, const uint4* w4, int nvec) {
   const int lane = threadIdx.x & 31;
-  f32x2 acc0 = pack2(0.f, 0.f), acc1 = pack2(0.f, 0.f);
+  // four accumulators: elements 0,4 / 1,5 / 2,6 / 3,7 of each 8-element vector
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
   auto fma8 = [&](const uint4& h, const uint4& w) {
-    const uint32_t hw[4] = {h.x, h.y, h.z, h.w}, ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const f32x2 hv = pack2(__uint_as_float(hw[i] << 16), __uint_as_float(hw[i] & 0xFFFF0000u));
-      const f32x2 wv = pack2(__uint_as_float(ww[i] << 16), __uint_as_float(ww[i] & 0xFFFF0000u));
-      if (i & 1)
-        acc1 = fma2(hv, wv, acc1);
-      else
-        acc0 = fma2(hv, wv, acc0);
-    }
+    fma_bf16x2(h.x, w.x, s0, s1);
+    fma_bf16x2(h.y, w.y, s2, s3);
+    fma_bf16x2(h.z, w.z, s0, s1);
+    fma_bf16x2(h.w, w.w, s2, s3);
   };
   int v = lane;
   for (; v + (kSHUnroll - 1) * 32 < nvec; v += kSHUnroll * 32) {
@@ -79,10 +85,7 @@ __device__ __forceinline__ float warp_dot(const uint4* hs4, const uint4* w4, int
     for (int u = 0; u < kSHUnroll; ++u) fma8(hs4[v + u * 32], w[u]);
   }
   for (; v < nvec; v += 32) fma8(hs4[v], __ldg(w4 + v));
-  float a0, a1, b0, b1;
-  unpack2(acc0, a0, a1);
-  unpack2(acc1, b0, b1);
-  float s = (a0 + a1) + (b0 + b1);
+  float s = (s0 + s1) + (s2 + s3);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   return s;
