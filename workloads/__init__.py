@@ -6,7 +6,7 @@ distance): both the CUDA path and the oracle consume the arrays it returns,
 and the same bit patterns reach both (bf16 values are produced here, on the
 host, and copied to the device unchanged).
 
-Random numbers come from numpy's Philox4x32-10 counter-based generator
+Random numbers come from numpy's Philox (4x64, 10 rounds) counter-based generator
 (Salmon et al., "Parallel random numbers: as easy as 1, 2, 3", SC 2011),
 one stream per (seed, block) via SeedSequence, so results do not depend on
 the number of worker threads.
