@@ -36,7 +36,7 @@ def build(force: bool = False) -> Path:
     """Compile oracle.cpp into liboracle.so (g++, OpenMP)."""
     if force or not _LIB.exists() or _LIB.stat().st_mtime < _SRC.stat().st_mtime:
         tmp = _LIB.with_suffix(f".so.tmp{os.getpid()}")
-        subprocess.run(["g++", "-O2", "-std=c++17", "-fopenmp", "-shared", "-fPIC", "-o",
+        subprocess.run(["g++", "-O2", "-std=c++17", "-ffp-contract=off", "-fopenmp", "-shared", "-fPIC", "-o",
                         str(tmp), str(_SRC)], check=True)
         os.replace(tmp, _LIB)
     return _LIB
@@ -207,3 +207,54 @@ def max_threads() -> int:
         return int(gomp.omp_get_max_threads())
     except OSError:
         return 1
+
+
+def philox4x64_10(counter, key):
+    """One Philox4x64-10 block: four 64-bit words for a 4-word counter and a
+    2-word key."""
+    c = np.ascontiguousarray(counter, np.uint64)
+    k = np.ascontiguousarray(key, np.uint64)
+    out = np.empty(4, np.uint64)
+    lib().vso_philox4x64_10(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def log_f32(x):
+    """The oracle's fp32 natural logarithm (fixed operation sequence)."""
+    L = lib()
+    L.vso_log_f32.restype = ctypes.c_float
+    L.vso_log_f32.argtypes = [ctypes.c_float]
+    return np.float32(L.vso_log_f32(float(np.float32(x))))
+
+
+def gumbel_f32(seed, row, j):
+    """G_j of the sampling recipe for (seed, row, token j), fp32."""
+    L = lib()
+    L.vso_gumbel_f32.restype = ctypes.c_float
+    L.vso_gumbel_f32.argtypes = [ctypes.c_uint64, ctypes.c_int, ctypes.c_int64]
+    return np.float32(L.vso_gumbel_f32(int(seed), int(row), int(j)))
+
+
+def gumbel_sample(logits, temperature, mask, seed, vocab=None):
+    """Seeded Gumbel-max token per row over the support `mask` ([rows, vocab]
+    bytes): argmax_j fl32(l_j / T) + G_j in fp32, smallest j on ties, -1 for
+    an empty support.  temperature: scalar or fp32 per row."""
+    logits = np.ascontiguousarray(logits)
+    rows, ld = logits.shape
+    vocab = ld if vocab is None else vocab
+    mask = np.ascontiguousarray(mask, np.uint8)
+    t_arr = None
+    t_s = 1.0
+    if np.ndim(temperature):
+        t_arr = np.ascontiguousarray(temperature, np.float32)
+    else:
+        t_s = float(np.float32(temperature))
+    out = np.empty(rows, np.int32)
+    L = lib()
+    rc = L.vso_gumbel_sample(ctypes.c_int(rows), ctypes.c_int(vocab), ctypes.c_int64(ld),
+                             ctypes.c_int(_dtype_code(logits)), _ptr(logits), _ptr(t_arr),
+                             ctypes.c_float(t_s), _ptr(mask), ctypes.c_uint64(int(seed)),
+                             _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return out

@@ -464,3 +464,143 @@ int vso_lmhead_logits(int nsel, const int32_t* rows_sel, int vocab, int hidden,
 }
 
 }  // extern "C"
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Seeded Gumbel-max sampling over the support ([xorl] section 3: the
+// program ends in a "seeded gumbel" step; the pages fix neither the
+// generator nor the noise recipe, so this is the project's reading):
+//
+//   score_j = fl32(l_j / T) + G_j,   G_j = -log(-log U_j)      (fp32)
+//   y       = argmax over j in S of score_j, the smallest j among equal scores
+//   U_j     = (bits 63..40 of r_j + 1/2) * 2^-24,  r_j = word (j mod 4) of
+//             Philox4x64-10(counter = (floor(j / 4), 0, 0, 0), key = (seed, row))
+//
+// The decision is taken in fp32 with one fixed sequence of IEEE operations
+// (each rounded separately, no fused multiply-add), so any implementation
+// that follows the same sequence reaches the same token.
+
+uint64_t mulhilo64(uint64_t a, uint64_t b, uint64_t* hi) {
+  const unsigned __int128 p = static_cast<unsigned __int128>(a) * b;
+  *hi = static_cast<uint64_t>(p >> 64);
+  return static_cast<uint64_t>(p);
+}
+
+// Philox4x64 with 10 rounds (Salmon, Moraes, Dror, Shaw, "Parallel random
+// numbers: as easy as 1, 2, 3", SC 2011): each round multiplies words 0 and
+// 2 by the two Philox-4x64 multipliers, swaps and xors the halves with the
+// round key; the key advances by the two Weyl constants between rounds.
+void philox4x64_10(const uint64_t ctr[4], const uint64_t key[2], uint64_t out[4]) {
+  const uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+  const uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+  uint64_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3];
+  uint64_t k0 = key[0], k1 = key[1];
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += W0;
+      k1 += W1;
+    }
+    uint64_t hi0, hi1;
+    const uint64_t lo0 = mulhilo64(M0, x0, &hi0);
+    const uint64_t lo1 = mulhilo64(M1, x2, &hi1);
+    const uint64_t y0 = hi1 ^ x1 ^ k0, y2 = hi0 ^ x3 ^ k1;
+    x0 = y0;
+    x1 = lo1;
+    x2 = y2;
+    x3 = lo0;
+  }
+  out[0] = x0;
+  out[1] = x1;
+  out[2] = x2;
+  out[3] = x3;
+}
+
+// Natural logarithm of a positive normal fp32 value: x = m 2^e with m in
+// [sqrt(1/2), sqrt(2)), log m = 2 atanh(s), s = (m - 1) / (m + 1), by the
+// series 2 (s + s^3/3 + s^5/5 + s^7/7 + s^9/9) (|s| < 0.172, so the next
+// term is below 2^-29 of the sum), and e ln 2 with ln 2 split into a head
+// exact in fp32 products and a tail (Cody and Waite's reduction).
+float log_f32(float x) {
+  uint32_t b;
+  std::memcpy(&b, &x, 4);
+  int e = static_cast<int>(b >> 23) - 127;
+  uint32_t mb = (b & 0x007FFFFFu) | 0x3F800000u;
+  float m;
+  std::memcpy(&m, &mb, 4);
+  if (m > 1.41421356f) {
+    m = m * 0.5f;
+    e += 1;
+  }
+  const float f = m - 1.0f;
+  const float s = f / (f + 2.0f);
+  const float z = s * s;
+  float t = 1.0f / 9.0f;
+  t = t * z;
+  t = t + 1.0f / 7.0f;
+  t = t * z;
+  t = t + 1.0f / 5.0f;
+  t = t * z;
+  t = t + 1.0f / 3.0f;
+  const float s2 = s * 2.0f;
+  const float zt = z * t;
+  const float lm = s2 + s2 * zt;
+  const float ef = static_cast<float>(e);
+  const float ln2_hi = 0.693145751953125f;       // 0x3F317200
+  const float ln2_lo = 1.42860677e-06f;          // fl32(ln 2 - ln2_hi)
+  const float tail = ef * ln2_lo + lm;
+  return ef * ln2_hi + tail;
+}
+
+// U_j and G_j of the recipe above.
+float gumbel_f32(uint64_t seed, int row, int64_t j) {
+  const uint64_t ctr[4] = {static_cast<uint64_t>(j) >> 2, 0, 0, 0};
+  const uint64_t key[2] = {seed, static_cast<uint64_t>(row)};
+  uint64_t w[4];
+  philox4x64_10(ctr, key, w);
+  const uint64_t r = w[j & 3];
+  const float u = (static_cast<float>(r >> 40) + 0.5f) * 5.9604644775390625e-08f;  // 2^-24
+  return -log_f32(-log_f32(u));
+}
+
+}  // namespace
+
+extern "C" {
+
+// One Philox4x64-10 block (for the tests that pin the generator).
+void vso_philox4x64_10(const uint64_t* ctr, const uint64_t* key, uint64_t* out) {
+  philox4x64_10(ctr, key, out);
+}
+
+float vso_log_f32(float x) { return log_f32(x); }
+
+float vso_gumbel_f32(uint64_t seed, int row, int64_t j) { return gumbel_f32(seed, row, j); }
+
+// Sample one token per row from the support given as a byte mask
+// ([rows, vocab], 1 = in S): y = argmax_{j in S} fl32(l_j / T) + G_j, the
+// smallest j on equal scores; -1 when the row's support is empty.
+// temperature (fp32 per row) may be null, then temperature_scalar.
+int vso_gumbel_sample(int rows, int vocab, int64_t ld, int dtype, const void* logits,
+                      const float* temperature, float temperature_scalar, const uint8_t* mask,
+                      uint64_t seed, int32_t* out) {
+  if (rows < 0 || vocab <= 0 || ld < vocab || !logits || !mask || !out) return 1;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int i = 0; i < rows; ++i) {
+    const float T = temperature ? temperature[i] : temperature_scalar;
+    int32_t best = -1;
+    float best_score = 0.f;
+    for (int j = 0; j < vocab; ++j) {
+      if (!mask[static_cast<int64_t>(i) * vocab + j]) continue;
+      const float l = static_cast<float>(load_value(logits, dtype, static_cast<int64_t>(i) * ld + j));
+      const float score = l / T + gumbel_f32(seed, i, j);
+      if (best < 0 || score > best_score) {
+        best = j;
+        best_score = score;
+      }
+    }
+    out[i] = best;
+  }
+  return 0;
+}
+
+}  // extern "C"

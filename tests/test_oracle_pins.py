@@ -411,3 +411,91 @@ def test_dominant_token_entropy_closed_form():
     h = math.log1p(d) + L * d / (1.0 + d)
     assert abs(r["h_full"][0] - h) <= 1e-12 * h
     assert abs(r["lp_full"][0] + math.log1p(d)) <= 1e-12 * math.log1p(d)
+
+
+# ---------------------------------------------------------------------------
+# seeded Gumbel-max sampling: the generator, the logarithm and the sampler,
+# each pinned to something other than itself
+
+
+def test_philox4x64_matches_numpy():
+    """The oracle's Philox4x64-10 equals numpy's (a library implementation of
+    the same published generator); numpy advances its counter before each
+    block, so its first block is the oracle's block at counter + 1,
+    including the carry into the next counter word."""
+    for key in ([0, 0], [0x123456789ABCDEF0, 0x0FEDCBA987654321], [2**64 - 1, 7]):
+        for start in ([0, 0, 0, 0], [5, 0, 0, 0], [2**64 - 1, 0, 0, 0], [2**64 - 2, 3, 1, 9]):
+            raw = np.random.Philox(key=np.array(key, np.uint64),
+                                   counter=np.array(start, np.uint64)).random_raw(8)
+            c = list(start)
+            for blk in range(2):
+                # counter + 1 as a 256-bit little-endian integer
+                v = sum(int(w) << (64 * i) for i, w in enumerate(c)) + 1
+                c = [(v >> (64 * i)) & (2**64 - 1) for i in range(4)]
+                got = oracle.philox4x64_10(c, key)
+                assert np.array_equal(got, raw[4 * blk: 4 * blk + 4]), (key, start, blk)
+
+
+def test_log_f32_within_two_ulp_of_the_exact_log():
+    """The fixed-sequence fp32 logarithm stays within 2 ulp of log(x) over
+    the range the sampler feeds it (2^-25 .. 20), including values around 1
+    and around the sqrt(2) split, where a dropped series term or a wrong
+    reduction would show."""
+    xs = np.concatenate([
+        np.geomspace(2.0**-25, 20.0, 4001),
+        1.0 + np.linspace(-0.05, 0.05, 2001),
+        math.sqrt(2.0) * (1.0 + np.linspace(-1e-3, 1e-3, 201)),
+        np.array([1.0, 2.0, 0.5, 0.75, 3.0, 1e-7, 17.3]),
+    ]).astype(np.float32)
+    for x in xs:
+        got = float(oracle.log_f32(x))
+        want = math.log(float(x))
+        ulp = float(np.spacing(np.float32(abs(want)))) if want != 0.0 else 2.0**-149
+        assert abs(got - want) <= 2 * ulp + 1e-45, (float(x), got, want)
+    assert float(oracle.log_f32(np.float32(1.0))) == 0.0
+
+
+def test_gumbel_noise_moments():
+    """G = -log(-log U) has mean the Euler-Mascheroni constant and variance
+    pi^2/6; 40,000 draws along one row must agree within 5 standard errors."""
+    g = np.array([oracle.gumbel_f32(11, 3, j) for j in range(40_000)], np.float64)
+    n = len(g)
+    assert abs(g.mean() - 0.5772156649) < 5 * math.sqrt(math.pi**2 / 6 / n)
+    # the sample variance of a Gumbel has standard error ~ sqrt((mu4 - s^4) / n), mu4 = 2.4 pi^4 / 15
+    s2 = math.pi**2 / 6
+    se = math.sqrt((2.4 * math.pi**4 / 15 - s2**2) / n)
+    assert abs(g.var() - s2) < 5 * se
+    assert len(set(g.tolist())) > 0.99 * n  # distinct draws per token
+
+
+def test_gumbel_max_frequencies_follow_the_support_softmax():
+    """Over many seeds the sampled token of one row has the distribution
+    softmax(l / T) restricted to the support (each probability within 5
+    binomial standard errors); tokens outside the support never appear."""
+    vocab = 12
+    l = np.array([0.5, 2.0, -1.0, 1.0, 3.0, 0.0, 2.5, -0.5, 1.5, 0.25, 2.25, -2.0], np.float32)
+    mask = np.array([1, 1, 0, 1, 1, 0, 0, 1, 1, 0, 1, 1], np.uint8)
+    T = np.float32(0.8)
+    n = 6000
+    logits = np.tile(l, (n, 1))
+    masks = np.tile(mask, (n, 1))
+    # one row, many seeds: draw seed s for row 0 by sampling a 1-row batch
+    picks = np.array([oracle.gumbel_sample(logits[:1], T, masks[:1], seed=s)[0] for s in range(n)])
+    assert np.all(mask[picks] == 1)
+    z = l.astype(np.float64) / float(T)
+    q = np.where(mask == 1, np.exp(z - z.max()), 0.0)
+    q /= q.sum()
+    freq = np.bincount(picks, minlength=vocab) / n
+    se = np.sqrt(q * (1 - q) / n)
+    assert np.all(np.abs(freq - q) <= 5 * se + 1e-12), (freq, q)
+
+
+def test_gumbel_sample_edge_cases():
+    logits = np.array([[1.0, 2.0, 3.0, 4.0]] * 3, np.float32)
+    mask = np.array([[0, 0, 0, 0], [0, 0, 1, 0], [1, 1, 1, 1]], np.uint8)
+    got = oracle.gumbel_sample(logits, 1.0, mask, seed=5)
+    assert got[0] == -1 and got[1] == 2
+    # rows are independent streams: the same logits in another row may differ,
+    # and re-running is deterministic
+    again = oracle.gumbel_sample(logits, 1.0, mask, seed=5)
+    assert np.array_equal(got, again)
