@@ -70,6 +70,7 @@ typedef int32_t vs_dtype;
 #define VS_WANT_ENTROPY (1u << 0)      /* write entropy_full / entropy_support */
 #define VS_WANT_SUPPORT_MASK (1u << 1) /* write the support_mask bitset */
 #define VS_WANT_GRAD (1u << 2)         /* write ctx for vs_score_bwd */
+#define VS_WANT_SAMPLE (1u << 3)       /* write sampled: a seeded Gumbel-max token from S */
 
 /* per-row status bits (vs_score_out.status) */
 #define VS_ROW_TARGET_OUT_OF_RANGE (1u << 0)   /* target outside [0, vocab): logprobs NaN */
@@ -115,6 +116,9 @@ typedef struct vs_score_args {
   int32_t support_width; /* 0 .. VS_MAX_SUPPORT_WIDTH */
   int64_t support_ld;    /* >= support_width */
   uint32_t flags;        /* VS_WANT_* */
+  /* seed of the Gumbel noise (VS_WANT_SAMPLE): row i of a call draws from
+   * the Philox4x64-10 stream keyed by (sample_seed, i) */
+  uint64_t sample_seed;
 } vs_score_args;
 
 /* Outputs of vs_score_fwd.  Every pointer may be NULL (that output is not
@@ -134,6 +138,15 @@ typedef struct vs_score_out {
                              16-byte aligned; opaque, pass unchanged to vs_score_bwd */
   double* entropy_sum;    /* [1] sum over valid rows of H_S (needs VS_WANT_ENTROPY) */
   int32_t* valid_count;   /* [1] number of valid rows */
+  /* [R] (needs VS_WANT_SAMPLE; [xorl] section 3, the program's final
+   * "seeded gumbel" step, here): argmax over j in S of fl32(l_j / T) + G_j,
+   * the smallest j on equal scores, -1 for an empty S or a non-finite row.
+   * G_j = -log(-log U_j), U_j = (bits 63..40 of r + 1/2) 2^-24, r = word
+   * (j mod 4) of Philox4x64-10(counter = (floor(j / 4), 0, 0, 0),
+   * key = (sample_seed, i)); every step one IEEE fp32 round-to-nearest
+   * operation (the logarithm by a fixed reduction and series), so the
+   * token is reproducible bit for bit. */
+  int32_t* sampled;
 } vs_score_out;
 
 /* Forward scoring ([SkyRL] Implementation; [xorl] sections 1 and 3).

@@ -18,7 +18,7 @@ LIB_PATH = _PKG / "libvs.so"
 
 VS_OK, VS_ERR_INVALID_ARG, VS_ERR_UNSUPPORTED, VS_ERR_WORKSPACE, VS_ERR_CUDA = 0, 1, 2, 3, 4
 VS_F32, VS_BF16 = 0, 1
-VS_WANT_ENTROPY, VS_WANT_SUPPORT_MASK, VS_WANT_GRAD = 1, 2, 4
+VS_WANT_ENTROPY, VS_WANT_SUPPORT_MASK, VS_WANT_GRAD, VS_WANT_SAMPLE = 1, 2, 4, 8
 VS_GRAD_DENSE, VS_GRAD_ACCUMULATE, VS_GRAD_SPARSE = 0, 1, 2
 VS_CTX_BYTES_PER_ROW = 64
 VS_MAX_SUPPORT_WIDTH = 1024
@@ -45,7 +45,7 @@ class ScoreArgs(ctypes.Structure):
         ("top_p", _vp), ("top_p_scalar", ctypes.c_float),
         ("min_p", _vp), ("min_p_scalar", ctypes.c_float),
         ("support_ids", _vp), ("support_width", ctypes.c_int32), ("support_ld", ctypes.c_int64),
-        ("flags", ctypes.c_uint32),
+        ("flags", ctypes.c_uint32), ("sample_seed", ctypes.c_uint64),
     ]
 
 
@@ -54,6 +54,7 @@ class ScoreOut(ctypes.Structure):
         ("logprob_full", _vp), ("logprob_support", _vp), ("entropy_full", _vp),
         ("entropy_support", _vp), ("valid", _vp), ("status", _vp), ("support_size", _vp),
         ("support_mask", _vp), ("ctx", _vp), ("entropy_sum", _vp), ("valid_count", _vp),
+        ("sampled", _vp),
     ]
 
 
@@ -188,18 +189,23 @@ def score_workspace(nbytes, device):
 
 def score_fwd(logits, targets, temperature=1.0, top_k=0, top_p=1.0, min_p=0.0,
               support_ids=None, want_entropy=True, want_mask=False, want_grad=False,
-              want_full=True, want_reduce=False, vocab=None, workspace=None, stream=None):
+              want_full=True, want_reduce=False, vocab=None, workspace=None, stream=None,
+              sample_seed=None):
     """Run vs_score_fwd; returns a dict of device tensors.
 
     workspace: a uint8 device tensor of at least vs_score_fwd_workspace_size
-    bytes (one call at a time); by default a buffer cached per device."""
+    bytes (one call at a time); by default a buffer cached per device.
+    sample_seed: when given, out["sampled"] holds one seeded Gumbel-max token
+    per row drawn from its support."""
     lib = load()
     rows, ld = logits.shape
     vocab = ld if vocab is None else vocab
     dev = logits.device
     flags = (VS_WANT_ENTROPY if want_entropy else 0) | (VS_WANT_SUPPORT_MASK if want_mask else 0) \
-        | (VS_WANT_GRAD if want_grad else 0)
+        | (VS_WANT_GRAD if want_grad else 0) | (VS_WANT_SAMPLE if sample_seed is not None else 0)
     a, keep = make_args(logits, targets, temperature, top_k, top_p, min_p, support_ids, vocab, flags)
+    if sample_seed is not None:
+        a.sample_seed = int(sample_seed)
     f32 = dict(dtype=torch.float32, device=dev)
     out = {
         "lp_support": torch.empty(rows, **f32),
@@ -217,6 +223,8 @@ def score_fwd(logits, targets, temperature=1.0, top_k=0, top_p=1.0, min_p=0.0,
         out["mask"] = torch.empty((rows, (vocab + 31) // 32), dtype=torch.int32, device=dev)
     if want_grad:
         out["ctx"] = torch.empty((rows, VS_CTX_BYTES_PER_ROW), dtype=torch.uint8, device=dev)
+    if sample_seed is not None:
+        out["sampled"] = torch.empty(rows, dtype=torch.int32, device=dev)
     if want_reduce:
         out["entropy_sum"] = torch.empty(1, dtype=torch.float64, device=dev)
         out["valid_count"] = torch.empty(1, dtype=torch.int32, device=dev)
@@ -232,6 +240,7 @@ def score_fwd(logits, targets, temperature=1.0, top_k=0, top_p=1.0, min_p=0.0,
     o.ctx = _p(out.get("ctx"))
     o.entropy_sum = _p(out.get("entropy_sum") if want_entropy else None)
     o.valid_count = _p(out.get("valid_count"))
+    o.sampled = _p(out.get("sampled"))
     if workspace is None:
         workspace = score_workspace(lib.vs_score_fwd_workspace_size(ctypes.byref(a)), dev)
     _check(lib.vs_score_fwd(ctypes.byref(a), ctypes.byref(o), _p(workspace),

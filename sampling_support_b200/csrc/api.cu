@@ -134,6 +134,8 @@ vs_status vs_score_fwd(const vs_score_args* a, const vs_score_out* o, void* work
     return fail(VS_ERR_INVALID_ARG, "VS_WANT_SUPPORT_MASK needs support_mask");
   if ((a->flags & VS_WANT_GRAD) && !o->ctx)
     return fail(VS_ERR_INVALID_ARG, "VS_WANT_GRAD needs ctx");
+  if (((a->flags & VS_WANT_SAMPLE) != 0) != (o->sampled != nullptr))
+    return fail(VS_ERR_INVALID_ARG, "VS_WANT_SAMPLE and sampled go together");
   if (o->ctx && !aligned16(o->ctx)) return fail(VS_ERR_INVALID_ARG, "ctx must be 16-byte aligned");
   if (want_entropy && !o->entropy_full && !o->entropy_support)
     return fail(VS_ERR_INVALID_ARG, "VS_WANT_ENTROPY needs entropy_full or entropy_support");
@@ -182,6 +184,9 @@ vs_status vs_score_fwd(const vs_score_args* a, const vs_score_out* o, void* work
   p.ctx = static_cast<vs::RowCtx*>((a->flags & VS_WANT_GRAD) ? o->ctx : nullptr);
   p.want_entropy = want_entropy ? 1 : 0;
   p.full_stats = (o->logprob_full || (want_entropy && o->entropy_full)) ? 1 : 0;
+  p.sampled = (a->flags & VS_WANT_SAMPLE) ? o->sampled : nullptr;
+  p.sample_seed = a->sample_seed;
+  p.row_base = 0;
   // fixed-point scale: vocab * 2^shift <= 2^63
   int bits = 0;
   while ((1ll << bits) <= static_cast<long long>(a->vocab)) ++bits;

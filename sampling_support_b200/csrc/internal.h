@@ -69,6 +69,9 @@ struct ScoreParams {
   int32_t want_entropy;
   int32_t full_stats;  // recorded support: compute full-vocabulary stats for every row
   int32_t fx_shift;    // fixed-point scale of mass histograms: 2^fx_shift
+  int32_t* sampled;    // [R] seeded Gumbel-max token, or nullptr
+  uint64_t sample_seed;
+  int32_t row_base;    // index of row 0 of this launch within the call (noise key)
 };
 
 struct BwdParams {

@@ -12,6 +12,7 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "gumbel.cuh"
 #include "internal.h"
 
 namespace vs {
@@ -37,6 +38,7 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
   __shared__ float fred[kRecThreads / 32];
   __shared__ uint32_t flags_sh;
   __shared__ int32_t target_hit;
+  __shared__ unsigned long long kred[kRecThreads / 32];
 
   const Raw* grow = static_cast<const Raw*>(P.logits) + static_cast<int64_t>(row) * P.ld;
   const int32_t* srow = P.support_ids + static_cast<int64_t>(row) * P.support_ld;
@@ -232,6 +234,26 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
       P.ctx[row] = cx;
     }
   }
+  // seeded Gumbel-max token over the kept ids
+  if (P.sampled) {
+    unsigned long long best = 0ull;
+    // a non-finite row (its support, or the whole row when its statistics
+    // were taken) samples nothing
+    if (!empty && any_nf == 0 && !(need_full && !stats_finite(f))) {
+      for (int w = tid; w < W; w += blockDim.x) {
+        const float x = vals[w];
+        if (x != x) continue;  // not kept
+        const int32_t id = ids[w];
+        float g[4];
+        gumbel4(P.sample_seed, static_cast<uint32_t>(P.row_base + row), static_cast<uint64_t>(id) >> 2, g);
+        const unsigned long long k = gumbel_key(gumbel_score(x, T, g[id & 3]), id);
+        best = k > best ? k : best;
+      }
+    }
+    best = block_max_key(best, kred);
+    if (tid == 0) P.sampled[row] = gumbel_key_id(best);
+  }
+
   // support bitmask: clear the row, then set the kept ids
   if (P.support_mask) {
     const int64_t wstride = (V + 31) / 32;

@@ -27,6 +27,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "gumbel.cuh"
 #include "select.cuh"
 
 namespace vs {
@@ -51,6 +52,7 @@ struct RowSh {
   uint32_t outstanding;  // loads issued and not yet consumed (broadcast by thread 0)
   int32_t tie_cut;
   uint32_t timeout;
+  unsigned long long kred[kRW];
 };
 
 // ---------------------------------------------------------------------------
@@ -778,6 +780,45 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
       }
       return false;
     });
+  }
+
+  // ---- pass 5 (L2): seeded Gumbel-max token over the support, one Philox
+  // block per group of four tokens that holds a member (stages start on
+  // multiples of four)
+  if (P.sampled) {
+    unsigned long long best = 0ull;
+    if (!nonfinite) {
+      const uint32_t nrow = static_cast<uint32_t>(P.row_base + row);
+      ring.pass(0, ring.nst(), [&](const Raw* st, int n, int base) {
+        for (int q = tid; 4 * q < n; q += kRT) {
+          bool mem[4];
+          bool any = false;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int j = 4 * q + i;
+            mem[i] = j < n;
+            if (mem[i] && filtered) {
+              const uint32_t key = key_of(st[j]);
+              mem[i] = key > tkey || (key == tkey && base + j <= tie_cut);
+            }
+            any |= mem[i];
+          }
+          if (!any) continue;
+          float g[4];
+          gumbel4(P.sample_seed, nrow, static_cast<uint64_t>(base + 4 * q) >> 2, g);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (!mem[i]) continue;
+            const unsigned long long k =
+                gumbel_key(gumbel_score(value_of(st[4 * q + i]), T, g[i]), base + 4 * q + i);
+            best = k > best ? k : best;
+          }
+        }
+        return false;
+      });
+    }
+    best = block_max_key(best, sh.kred);
+    if (tid == 0) P.sampled[row] = gumbel_key_id(best);
   }
 }
 

@@ -28,6 +28,7 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "gumbel.cuh"
 #include "internal.h"
 #include "select.cuh"
 
@@ -43,7 +44,6 @@ constexpr int kHistUnroll = 8;    // 16-byte loads in flight per merge thread
 constexpr int kMaxChunks = 256;   // chunks per row
 constexpr int kChunkAlign = 256;  // chunk length granularity (elements)
 constexpr size_t kRowsL2Bytes = size_t(48) << 20;  // logits per launch kept for the L2 re-read
-constexpr size_t kSplitWsCap = size_t(64) << 20;
 
 // Per (row, chunk) statistics relative to fl(vmax c).
 struct alignas(16) ChunkRec {
@@ -87,6 +87,7 @@ struct SplitArgs {
   int chunk;          // elements per chunk (multiple of kChunkAlign)
   ChunkRec* recs;     // [rows * S]
   RowDecision* dec;   // [rows]
+  unsigned long long* best;  // [rows] best Gumbel-max key of the row (sampling)
 };
 
 __device__ __forceinline__ uint32_t bf16_key(uint32_t r) { return key_of(static_cast<uint16_t>(r)); }
@@ -582,7 +583,7 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
   const float log2z = stats_log2z(st);
   const float h_full = kLn2 * (log2z - st.a / stats_z(st));
   const bool filtered = !nonfinite && any_filter;
-  const bool want_cut = P.ctx != nullptr || P.support_mask != nullptr;
+  const bool want_cut = P.ctx != nullptr || P.support_mask != nullptr || P.sampled != nullptr;
 
   uint32_t tkey = 0;
   int32_t tie_cut = INT_MAX;
@@ -831,7 +832,7 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
     if (P.valid) P.valid[row] = nonfinite ? 0 : 1;
     if (P.status) P.status[row] = status;
     if (P.support_size) P.support_size[row] = n_support;
-    if (P.support_mask) {
+    if (P.support_mask || P.sampled) {
       RowDecision d;
       d.tkey = tkey;
       d.tie_cut = tie_cut;
@@ -839,6 +840,7 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
       d.pad = 0;
       Q.dec[row] = d;
     }
+    if (P.sampled) Q.best[row] = 0ull;
     if (P.ctx) {
       RowCtx cx{};
       cx.m2 = vr;
@@ -910,9 +912,71 @@ __global__ void __launch_bounds__(kCT) score_split_mask_kernel(ScoreParams P, Sp
   }
 }
 
+// Seeded Gumbel-max candidates of each chunk from the row's decision: one
+// Philox block per group of four tokens holding a member (chunks start on
+// multiples of 256), the chunk's best key folded into the row's by an
+// unsigned max (order-independent).
+__global__ void __launch_bounds__(kCT) score_split_sample_kernel(ScoreParams P, SplitArgs Q) {
+  __shared__ unsigned long long kred[kCT / 32];
+  const int row = blockIdx.x / Q.S;
+  const int cs = blockIdx.x - row * Q.S;
+  const int V = P.vocab;
+  const uint16_t* grow = static_cast<const uint16_t*>(P.logits) + static_cast<int64_t>(row) * P.ld;
+  const int j0 = cs * Q.chunk, j1 = min(V, j0 + Q.chunk);
+  const RowDecision d = Q.dec[row];
+  const float T = P.temperature ? P.temperature[row] : P.temperature_scalar;
+  const uint32_t nrow = static_cast<uint32_t>(P.row_base + row);
+  unsigned long long best = 0ull;
+  if (d.mode != 0u) {
+    for (int q = j0 / 4 + static_cast<int>(threadIdx.x); 4 * q < j1; q += kCT) {
+      const int jb = 4 * q;
+      uint32_t r[4];
+      if (jb + 4 <= j1) {
+        const uint2 v = __ldcg(reinterpret_cast<const uint2*>(grow + jb));
+        r[0] = v.x & 0xFFFFu;
+        r[1] = v.x >> 16;
+        r[2] = v.y & 0xFFFFu;
+        r[3] = v.y >> 16;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) r[i] = jb + i < j1 ? grow[jb + i] : 0u;
+      }
+      bool mem[4];
+      bool any = false;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        mem[i] = jb + i < j1;
+        if (mem[i] && d.mode == 2u) {
+          const uint32_t key = bf16_key(r[i]);
+          mem[i] = key > d.tkey || (key == d.tkey && jb + i <= d.tie_cut);
+        }
+        any |= mem[i];
+      }
+      if (!any) continue;
+      float g[4];
+      gumbel4(P.sample_seed, nrow, static_cast<uint64_t>(q), g);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (!mem[i]) continue;
+        const unsigned long long k =
+            gumbel_key(gumbel_score(value_of(static_cast<uint16_t>(r[i])), T, g[i]), jb + i);
+        best = k > best ? k : best;
+      }
+    }
+  }
+  best = block_max_key(best, kred);
+  if (threadIdx.x == 0 && best != 0ull) atomicMax(Q.best + row, best);
+}
+
+// The sampled token of each row from its best key (-1: no member).
+__global__ void score_split_sample_final_kernel(ScoreParams P, SplitArgs Q) {
+  const int row = blockIdx.x * blockDim.x + threadIdx.x;
+  if (row < P.rows) P.sampled[row] = gumbel_key_id(Q.best[row]);
+}
+
 struct SplitPlan {
   int S, chunk, rows_per_launch;
-  size_t off_dec, bytes;
+  size_t off_dec, off_best, bytes;
 };
 
 // Chunk CTAs resident on the whole device (one wave).
@@ -954,7 +1018,8 @@ SplitPlan split_plan(int rows, int vocab) {
   p.chunk = chunk;
   p.rows_per_launch = static_cast<int>(rpl);
   p.off_dec = align256(rpl * S * sizeof(ChunkRec));
-  p.bytes = p.off_dec + align256(rpl * sizeof(RowDecision));
+  p.off_best = p.off_dec + align256(rpl * sizeof(RowDecision));
+  p.bytes = p.off_best + align256(rpl * sizeof(unsigned long long));
   return p;
 }
 
@@ -976,6 +1041,8 @@ ScoreParams offset_rows(const ScoreParams& P, int r0, int n) {
   if (P.status) q.status = P.status + r0;
   if (P.support_size) q.support_size = P.support_size + r0;
   if (P.support_mask) q.support_mask = P.support_mask + static_cast<int64_t>(r0) * ((P.vocab + 31) / 32);
+  if (P.sampled) q.sampled = P.sampled + r0;
+  q.row_base = P.row_base + r0;
   if (P.ctx) q.ctx = P.ctx + r0;
   return q;
 }
@@ -997,6 +1064,7 @@ cudaError_t launch_score_split(const ScoreParams& p, void* ws, cudaStream_t s) {
   q.chunk = plan.chunk;
   q.recs = reinterpret_cast<ChunkRec*>(base);
   q.dec = reinterpret_cast<RowDecision*>(base + plan.off_dec);
+  q.best = reinterpret_cast<unsigned long long*>(base + plan.off_best);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -1014,6 +1082,10 @@ cudaError_t launch_score_split(const ScoreParams& p, void* ws, cudaStream_t s) {
     cudaError_t e = cudaLaunchKernelEx(&cfg, score_merge_kernel, pr, q);
     if (e != cudaSuccess) return e;
     if (pr.support_mask) score_split_mask_kernel<<<n * plan.S, kCT, 0, s>>>(pr, q);
+    if (pr.sampled) {
+      score_split_sample_kernel<<<n * plan.S, kCT, 0, s>>>(pr, q);
+      score_split_sample_final_kernel<<<(n + 127) / 128, 128, 0, s>>>(pr, q);
+    }
   }
   return cudaGetLastError();
 }

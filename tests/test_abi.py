@@ -190,3 +190,14 @@ def _last_error_after(call):
 
 def test_support_head_zero_rows_is_a_no_op():
     assert _support_head(rows=0, H=0, W=0, targets=0, ids=0) == B.VS_OK
+
+
+def test_sample_flag_and_output_go_together():
+    lib = vsb.load()
+    a = _args(flags=8)  # VS_WANT_SAMPLE without an output
+    o = B.ScoreOut()
+    assert lib.vs_score_fwd(ctypes.byref(a), ctypes.byref(o), FAKE, 1 << 20, None) == B.VS_ERR_INVALID_ARG
+    a = _args()
+    o = B.ScoreOut()
+    o.sampled = FAKE  # an output without the flag
+    assert lib.vs_score_fwd(ctypes.byref(a), ctypes.byref(o), FAKE, 1 << 20, None) == B.VS_ERR_INVALID_ARG
