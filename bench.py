@@ -333,6 +333,8 @@ def secondary(args, pk, only=None):
         distance_workload(args, pk, steps, out)
     if only in (None, "replay"):
         replay_workload(args, pk, steps, out)
+    if only in (None, "sample"):
+        sample_workload(args, pk, steps, out)
     if only in (None, "lmhead", "support_head"):
         lmhead_workload(args, pk, steps, out, fused=only in (None, "lmhead"),
                         support=only in (None, "support_head"))
@@ -403,6 +405,64 @@ def replay_workload(args, pk, steps, out):
                      "bwd_frac_hbm": wbytes / (ms_b / 1e3) / 1e9 / pk["hbm"],
                      "fwd_bytes_est": fbytes, "bwd_bytes": wbytes}
     del lg, dlog, holder
+    torch.cuda.empty_cache()
+
+
+def sample_workload(args, pk, steps, out):
+    """The fullvocab scoring call with the seeded Gumbel-max sample added
+    (inputs rotating over buffers larger than L2, as in the headline; the
+    same C-ABI call with preallocated outputs)."""
+    import ctypes
+
+    import torch
+
+    import sampling_support_b200 as vsb
+    import workloads
+    from sampling_support_b200 import _binding as B
+
+    lib = vsb.load()
+    w = workloads.fullvocab()
+    rows = w["rows"]
+    nbuf = max(2, int(np.ceil(4 * L2_BYTES / w["logits"].nbytes)))
+    base = to_dev(w["logits"])
+    bufs = [base] + [base.clone() for _ in range(nbuf - 1)]
+    temp, tgt = to_dev(w["temperature"]), to_dev(w["targets"])
+    dev = base.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    keep = [torch.empty(rows, **f32) for _ in range(4)]
+    valid = torch.empty(rows, dtype=torch.uint8, device=dev)
+    status = torch.empty(rows, dtype=torch.int32, device=dev)
+    size = torch.empty(rows, dtype=torch.int32, device=dev)
+    sampled = torch.empty(rows, dtype=torch.int32, device=dev)
+    o = B.ScoreOut()
+    o.logprob_full, o.logprob_support, o.entropy_full, o.entropy_support = [t.data_ptr() for t in keep]
+    o.valid, o.status, o.support_size, o.sampled = (valid.data_ptr(), status.data_ptr(),
+                                                    size.data_ptr(), sampled.data_ptr())
+    argsets = []
+    for b in bufs:
+        a, _ = B.make_args(b, tgt, temp, 0, float(np.float32(w["top_p"])), 0.0,
+                           flags=B.VS_WANT_ENTROPY | B.VS_WANT_SAMPLE)
+        a.sample_seed = 1234
+        argsets.append(a)
+    ws = B.score_workspace(lib.vs_score_fwd_workspace_size(ctypes.byref(argsets[0])), dev)
+    sp = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    oref = ctypes.byref(o)
+    it = [0]
+
+    def step():
+        a = argsets[it[0] % nbuf]
+        a.sample_seed = 1234 + it[0]
+        it[0] += 1
+        rc = lib.vs_score_fwd(ctypes.byref(a), oref, ws.data_ptr(), ws.numel(), sp)
+        if rc:
+            raise RuntimeError(lib.vs_last_error().decode())
+
+    ms = time_steps(step, 3, max(20, min(steps, 500)))
+    out["sample"] = {"rows": rows, "vocab": w["vocab"], "ms_per_step": ms,
+                     "rows_per_s": rows / (ms / 1e3),
+                     "note": "fullvocab scoring (top-p 0.95, entropy) plus one seeded Gumbel-max "
+                             "token per row over its support; kernels: chunk, merge, sample, finalize"}
+    del bufs, base
     torch.cuda.empty_cache()
 
 
@@ -557,7 +617,7 @@ def main():
     ap.add_argument("--sub-steps", type=int, default=50)
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["distance", "replay", "lmhead", "support_head"], default=None,
+    ap.add_argument("--only", choices=["distance", "replay", "sample", "lmhead", "support_head"], default=None,
                     help="time one secondary workload alone (one GPU) and print its line")
     args = ap.parse_args()
     if args.warmup < 3:
