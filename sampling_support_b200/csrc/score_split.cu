@@ -912,57 +912,82 @@ __global__ void __launch_bounds__(kCT) score_split_mask_kernel(ScoreParams P, Sp
   }
 }
 
-// Seeded Gumbel-max candidates of each chunk from the row's decision: one
-// Philox block per group of four tokens holding a member (chunks start on
-// multiples of 256), the chunk's best key folded into the row's by an
-// unsigned max (order-independent).
+// Seeded Gumbel-max candidates of each chunk from the row's decision.  The
+// chunk is read from L2 in groups of four tokens (chunks start on multiples
+// of 256); each warp queues its groups that hold a member (group index,
+// member bits and the four raw values) in shared memory and drains the
+// queue 32 groups at a time, so the Philox block and the logarithms run
+// on full warps and only for members.  The chunk's best key goes into the
+// row's slot by an unsigned max (order-independent).
 __global__ void __launch_bounds__(kCT) score_split_sample_kernel(ScoreParams P, SplitArgs Q) {
   __shared__ unsigned long long kred[kCT / 32];
+  __shared__ uint4 queue[kCT / 32][64];
   const int row = blockIdx.x / Q.S;
   const int cs = blockIdx.x - row * Q.S;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int V = P.vocab;
   const uint16_t* grow = static_cast<const uint16_t*>(P.logits) + static_cast<int64_t>(row) * P.ld;
   const int j0 = cs * Q.chunk, j1 = min(V, j0 + Q.chunk);
   const RowDecision d = Q.dec[row];
   const float T = P.temperature ? P.temperature[row] : P.temperature_scalar;
   const uint32_t nrow = static_cast<uint32_t>(P.row_base + row);
+  uint4* wq = queue[warp];
   unsigned long long best = 0ull;
+  // one queued group: .x = group index, .y = member bits, .z / .w = raw pairs
+  auto take = [&](const uint4& e) {
+    uint64_t w[4];
+    philox4x64_10(e.x, 0, 0, 0, P.sample_seed, nrow, w);
+    const uint32_t r[4] = {e.z & 0xFFFFu, e.z >> 16, e.w & 0xFFFFu, e.w >> 16};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (!((e.y >> i) & 1u)) continue;
+      const int j = static_cast<int>(4 * e.x) + i;
+      const unsigned long long k =
+          gumbel_key(gumbel_score(value_of(static_cast<uint16_t>(r[i])), T, gumbel_of(w[i])), j);
+      best = k > best ? k : best;
+    }
+  };
   if (d.mode != 0u) {
-    for (int q = j0 / 4 + static_cast<int>(threadIdx.x); 4 * q < j1; q += kCT) {
+    int count = 0;  // queued groups of this warp (warp-uniform)
+    const int q_end = (j1 + 3) / 4;
+    for (int qb = j0 / 4 + warp * 32; qb < q_end; qb += kCT) {
+      const int q = qb + lane;
       const int jb = 4 * q;
-      uint32_t r[4];
-      if (jb + 4 <= j1) {
-        const uint2 v = __ldcg(reinterpret_cast<const uint2*>(grow + jb));
-        r[0] = v.x & 0xFFFFu;
-        r[1] = v.x >> 16;
-        r[2] = v.y & 0xFFFFu;
-        r[3] = v.y >> 16;
-      } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) r[i] = jb + i < j1 ? grow[jb + i] : 0u;
-      }
-      bool mem[4];
-      bool any = false;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        mem[i] = jb + i < j1;
-        if (mem[i] && d.mode == 2u) {
-          const uint32_t key = bf16_key(r[i]);
-          mem[i] = key > d.tkey || (key == d.tkey && jb + i <= d.tie_cut);
+      uint32_t lo = 0u, hi = 0u, mbits = 0u;
+      if (q < q_end) {
+        if (jb + 4 <= j1) {
+          const uint2 v = __ldcg(reinterpret_cast<const uint2*>(grow + jb));
+          lo = v.x;
+          hi = v.y;
+        } else {
+          for (int i = 0; i < 4 && jb + i < j1; ++i) {
+            const uint32_t r = grow[jb + i];
+            if (i < 2) lo |= r << (16 * i);
+            else hi |= r << (16 * (i - 2));
+          }
         }
-        any |= mem[i];
-      }
-      if (!any) continue;
-      float g[4];
-      gumbel4(P.sample_seed, nrow, static_cast<uint64_t>(q), g);
+        const uint32_t r[4] = {lo & 0xFFFFu, lo >> 16, hi & 0xFFFFu, hi >> 16};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (!mem[i]) continue;
-        const unsigned long long k =
-            gumbel_key(gumbel_score(value_of(static_cast<uint16_t>(r[i])), T, g[i]), jb + i);
-        best = k > best ? k : best;
+        for (int i = 0; i < 4; ++i) {
+          bool in = jb + i < j1;
+          if (in && d.mode == 2u) {
+            const uint32_t key = bf16_key(r[i]);
+            in = key > d.tkey || (key == d.tkey && jb + i <= d.tie_cut);
+          }
+          mbits |= in ? (1u << i) : 0u;
+        }
+      }
+      const uint32_t ball = __ballot_sync(0xffffffffu, mbits != 0u);
+      if (mbits) wq[count + __popc(ball & ((1u << lane) - 1u))] = make_uint4(q, mbits, lo, hi);
+      count += __popc(ball);
+      __syncwarp();
+      if (count >= 32) {
+        count -= 32;
+        take(wq[count + lane]);
+        __syncwarp();
       }
     }
+    if (lane < count) take(wq[lane]);
   }
   best = block_max_key(best, kred);
   if (threadIdx.x == 0 && best != 0ull) atomicMax(Q.best + row, best);
