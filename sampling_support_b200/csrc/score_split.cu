@@ -719,9 +719,10 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
     from_bins = win_ok && tkey >= w.klo;
     SupSums sums{0u, 0u, 0u, 0.f, 0.f};
     if (from_bins) {
-#pragma unroll 1
-      for (int i = 8 * tid; i < min(w.nbins, 8 * tid + 8); ++i) {
-        const uint32_t cnt = hist[i];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int i = 8 * tid + k;
+        const uint32_t cnt = i < w.nbins ? hist[i] : 0u;
         const uint32_t key = w.klo + i;
         if (cnt && key > tkey) {
           const float d = key_u(key, c) - mr;

@@ -133,22 +133,28 @@ __device__ __forceinline__ u64 bin_fx(const Window& w, uint32_t key) {
 // Search the window from the largest key for the bin where the cumulative
 // count (by_mass false) or fixed-point mass first reaches need (>= 1).
 // False when the whole window holds less than need.  Each thread owns a run
-// of NB = ceil(4096 / NT) consecutive bins; loops stay rolled (the search
-// runs once per row, so short code matters more than unrolling), and the one
-// thread whose run holds the crossing walks it again.
+// of NB = ceil(4096 / NT) consecutive bins, loads them and their fixed-point
+// masses into registers at once (independent loads and exponentials, no
+// chain through the loop), and the one thread whose run holds the crossing
+// walks its registers back down.
 template <int NT>
-__device__ __noinline__ bool win_search(const Window& w, bool by_mass, u64 need, Desc& out,
+__device__ __forceinline__ bool win_search(const Window& w, bool by_mass, u64 need, Desc& out,
                                         SelShared<NT / 32>& sh) {
   constexpr int NB = (kSelWin + NT - 1) / NT;
-  const int i0 = threadIdx.x * NB, i1 = min(w.nbins, i0 + NB);
+  const int i0 = threadIdx.x * NB;
+  const int nb = w.nbins;
+  const uint32_t* hist = w.hist;
+  const uint32_t klo = w.klo;
+  uint32_t cnt[NB];
+  u64 fx[NB];
+#pragma unroll
+  for (int k = 0; k < NB; ++k) cnt[k] = i0 + k < nb ? hist[i0 + k] : 0u;
   u64 lc = 0, lm = 0;
-#pragma unroll 1
-  for (int i = i0; i < i1; ++i) {
-    const uint32_t cnt = w.hist[i];
-    if (cnt) {
-      lc += cnt;
-      lm += static_cast<u64>(cnt) * bin_fx(w, w.klo + i);
-    }
+#pragma unroll
+  for (int k = 0; k < NB; ++k) {
+    fx[k] = cnt[k] ? static_cast<u64>(cnt[k]) * bin_fx(w, klo + i0 + k) : 0ull;
+    lc += cnt[k];
+    lm += fx[k];
   }
   u64 ec, em;
   block_suffix_excl<NT>(lc, lm, ec, em, sh);
@@ -158,21 +164,22 @@ __device__ __noinline__ bool win_search(const Window& w, bool by_mass, u64 need,
   const u64 mine = by_mass ? lm : lc;
   if (base < need && need <= base + mine) {
     u64 ac = ec, am = em;
-#pragma unroll 1
-    for (int i = i1 - 1; i >= i0; --i) {
-      const uint32_t cnt = w.hist[i];
-      const u64 fx = cnt ? static_cast<u64>(cnt) * bin_fx(w, w.klo + i) : 0ull;
-      if (cnt && (by_mass ? am + fx : ac + cnt) >= need) {
-        sh.b_key = w.klo + i;
+    bool done = false;
+#pragma unroll
+    for (int k = NB - 1; k >= 0; --k) {
+      if (!done && cnt[k] && (by_mass ? am + fx[k] : ac + cnt[k]) >= need) {
+        sh.b_key = klo + i0 + k;
         sh.b_above_cnt = ac;
         sh.b_above_mass = am;
-        sh.b_at_cnt = cnt;
-        sh.b_at_mass = fx;
+        sh.b_at_cnt = cnt[k];
+        sh.b_at_mass = fx[k];
         sh.b_found = 1;
-        break;
+        done = true;
       }
-      ac += cnt;
-      am += fx;
+      if (!done) {
+        ac += cnt[k];
+        am += fx[k];
+      }
     }
   }
   __syncthreads();
