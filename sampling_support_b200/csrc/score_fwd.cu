@@ -22,7 +22,7 @@ namespace {
 // ---------------------------------------------------------------------------
 // recorded support
 
-constexpr int kRecThreads = 256;
+constexpr int kRecThreads = 128;
 
 template <typename Raw>
 __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams P) {
