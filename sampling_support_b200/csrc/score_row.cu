@@ -53,6 +53,7 @@ struct RowSh {
   int32_t tie_cut;
   uint32_t timeout;
   unsigned long long kred[kRW];
+  uint32_t squeue[kRW][64];  // sampling: per-warp queue of member groups (index | bits << 28)
 };
 
 // ---------------------------------------------------------------------------
@@ -782,38 +783,60 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
     });
   }
 
-  // ---- pass 5 (L2): seeded Gumbel-max token over the support, one Philox
-  // block per group of four tokens that holds a member (stages start on
-  // multiples of four)
+  // ---- pass 5 (L2): seeded Gumbel-max token over the support.  Tokens go
+  // in groups of four (stages start on multiples of four); each warp queues
+  // its groups that hold a member and drains the queue 32 groups at a time
+  // (and at the end of each stage), so the Philox block and the logarithms
+  // run on full warps and only for members.
   if (P.sampled) {
     unsigned long long best = 0ull;
     if (!nonfinite) {
       const uint32_t nrow = static_cast<uint32_t>(P.row_base + row);
+      const int lane = tid & 31, warp = tid >> 5;
+      uint32_t* wq = sh.squeue[warp];
       ring.pass(0, ring.nst(), [&](const Raw* st, int n, int base) {
-        for (int q = tid; 4 * q < n; q += kRT) {
-          bool mem[4];
-          bool any = false;
+        auto take = [&](uint32_t e) {
+          const int q = static_cast<int>(e & 0x0FFFFFFFu);
+          uint64_t w[4];
+          philox4x64_10(static_cast<uint64_t>(base >> 2) + q, 0, 0, 0, P.sample_seed, nrow, w);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
+            if (!((e >> (28 + i)) & 1u)) continue;
             const int j = 4 * q + i;
-            mem[i] = j < n;
-            if (mem[i] && filtered) {
-              const uint32_t key = key_of(st[j]);
-              mem[i] = key > tkey || (key == tkey && base + j <= tie_cut);
-            }
-            any |= mem[i];
-          }
-          if (!any) continue;
-          float g[4];
-          gumbel4(P.sample_seed, nrow, static_cast<uint64_t>(base + 4 * q) >> 2, g);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            if (!mem[i]) continue;
             const unsigned long long k =
-                gumbel_key(gumbel_score(value_of(st[4 * q + i]), T, g[i]), base + 4 * q + i);
+                gumbel_key(gumbel_score(value_of(st[j]), T, gumbel_of(w[i])), base + j);
             best = k > best ? k : best;
           }
+        };
+        const int ng = (n + 3) / 4;
+        int count = 0;  // queued groups of this warp (warp-uniform)
+        for (int qb = warp * 32; qb < ng; qb += kRT) {
+          const int q = qb + lane;
+          uint32_t mbits = 0u;
+          if (q < ng) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int j = 4 * q + i;
+              bool in = j < n;
+              if (in && filtered) {
+                const uint32_t key = key_of(st[j]);
+                in = key > tkey || (key == tkey && base + j <= tie_cut);
+              }
+              mbits |= in ? (1u << i) : 0u;
+            }
+          }
+          const uint32_t ball = __ballot_sync(0xffffffffu, mbits != 0u);
+          if (mbits) wq[count + __popc(ball & ((1u << lane) - 1u))] = static_cast<uint32_t>(q) | (mbits << 28);
+          count += __popc(ball);
+          __syncwarp();
+          if (count >= 32) {
+            count -= 32;
+            take(wq[count + lane]);
+            __syncwarp();
+          }
         }
+        if (lane < count) take(wq[lane]);
+        __syncwarp();
         return false;
       });
     }
