@@ -5,7 +5,8 @@
 //    "Implementation": dense -1-padded id list).  One CTA per row gathers the
 //    support logits; rows with an empty support (full-vocabulary fallback),
 //    or every row when full statistics are requested, also stream the whole
-//    row once with 16-byte loads.
+//    row once with 16-byte loads.  A requested sample is the seeded
+//    Gumbel-max token over the kept ids (noise recipe in gumbel.cuh).
 
 #include <climits>
 

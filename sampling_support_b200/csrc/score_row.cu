@@ -15,7 +15,9 @@
 //   pass 3 (L2)   only when the support ends inside a tie group: an ordered
 //                 count of that group's elements finds the id of the last one
 //                 kept (ties go to the lower token id);
-//   pass 4 (L2)   only when the support bitmask is requested.
+//   pass 4 (L2)   only when the support bitmask is requested;
+//   pass 5 (L2)   only when a sample is requested: a seeded Gumbel-max token
+//                 over the support (noise recipe in gumbel.cuh).
 // fp32 rows, and bf16 rows whose crossing lies below the window, fall back to
 // an 8-bit radix descent over all keys (one streamed pass per digit).
 // Everything is block-local (no cluster barriers), deterministic, and each

@@ -17,11 +17,14 @@
 // bins find the k-th element and the top-p crossing, and the support sums.
 // A crossing below the window falls back to an 8-bit radix descent over the
 // row.  The tie cut (which elements equal to the threshold value are kept:
-// the lowest ids) is resolved to an id only for the saved state or the
-// bitmask; the target's membership otherwise uses the count of its earlier
-// ties.
+// the lowest ids) is resolved to an id only for the saved state, the
+// bitmask or a sample; the target's membership otherwise uses the count of
+// its earlier ties.
 // Kernel 3 (score_split_mask_kernel, only when the bitmask is requested)
 // writes the support bitmask from the row's decision.
+// Kernels 4 and 5 (score_split_sample_kernel and its finalize kernel, only
+// when a sample is requested): a seeded Gumbel-max token over the support
+// (the noise recipe is in gumbel.cuh).
 
 #include <climits>
 
