@@ -453,6 +453,10 @@ __device__ __forceinline__ uint32_t key_at_level(uint32_t lo, uint32_t hi, float
 
 __global__ void __launch_bounds__(kCT, 8) score_chunk_kernel(ScoreParams P, SplitArgs Q) {
   __shared__ ChunkShared sh;
+  // launched programmatically after whatever kernel precedes it on the
+  // stream: wait for that grid (and its memory) before touching anything,
+  // then let this call's merge kernel launch
+  pdl_wait();
   pdl_launch_dependents();
 
   const int row = blockIdx.x / Q.S;
@@ -551,6 +555,8 @@ __global__ void __launch_bounds__(kMT, 1) score_merge_kernel(ScoreParams P, Spli
   __shared__ MergeShared sh;
   RadixArrays& ra = *reinterpret_cast<RadixArrays*>(hist);
 
+  // the next call's chunk kernel may launch now; it waits for this grid
+  pdl_launch_dependents();
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
   const int V = P.vocab;
@@ -1100,7 +1106,15 @@ cudaError_t launch_score_split(const ScoreParams& p, void* ws, cudaStream_t s) {
   for (int r0 = 0; r0 < p.rows; r0 += plan.rows_per_launch) {
     const int n = min(plan.rows_per_launch, p.rows - r0);
     const ScoreParams pr = offset_rows(p, r0, n);
-    score_chunk_kernel<<<n * plan.S, kCT, 0, s>>>(pr, q);
+    cudaLaunchConfig_t ccfg{};
+    ccfg.gridDim = dim3(n * plan.S);
+    ccfg.blockDim = dim3(kCT);
+    ccfg.dynamicSmemBytes = 0;
+    ccfg.stream = s;
+    ccfg.attrs = attr;
+    ccfg.numAttrs = 1;
+    cudaError_t ec = cudaLaunchKernelEx(&ccfg, score_chunk_kernel, pr, q);
+    if (ec != cudaSuccess) return ec;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(n);
     cfg.blockDim = dim3(kMT);
