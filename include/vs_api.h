@@ -276,7 +276,8 @@ vs_status vs_l1_distance_static(int32_t rows, int32_t vocab, int64_t ld, vs_dtyp
  * hidden [rows, hidden_dim] and weight [vocab, hidden_dim] are bf16, K-major,
  * row strides ldh/ldw elements (multiples of 8), 16-byte aligned; hidden_dim
  * a multiple of 64.  top_k in [1, VS_MAX_FUSED_TOPK] (top-p without top-k is
- * not offered here).  Needs vs_fused_lmhead_workspace_size(...) bytes. */
+ * not offered here).  out->support_mask, ctx and sampled must be NULL (and
+ * VS_WANT_SAMPLE unset).  Needs vs_fused_lmhead_workspace_size(...) bytes. */
 vs_status vs_fused_lmhead_score(int32_t rows, int32_t vocab, int32_t hidden_dim,
                                 const void* hidden, int64_t ldh, const void* weight,
                                 int64_t ldw, const float* temperature,
@@ -310,7 +311,8 @@ size_t vs_fused_lmhead_workspace_size(int32_t rows, int32_t vocab, int32_t hidde
  * (row stride ldw) are bf16, 16-byte aligned, strides multiples of 8;
  * hidden_dim a multiple of 8, at most 16384.  support_ids [rows, support_ld]
  * int32, width in [0, VS_MAX_SUPPORT_WIDTH].  out->logprob_full,
- * entropy_full, support_mask and ctx must be NULL (VS_ERR_INVALID_ARG).  When
+ * entropy_full, support_mask, ctx and sampled must be NULL
+ * (VS_ERR_INVALID_ARG).  When
  * support_logits is non-NULL it receives [rows, logits_ld] fp32: z[i, s] at
  * each kept slot, -inf at pads, bad and repeated ids.  No workspace. */
 vs_status vs_support_lmhead_score(int32_t rows, int32_t vocab, int32_t hidden_dim,

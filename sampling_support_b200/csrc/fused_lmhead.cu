@@ -837,6 +837,8 @@ vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh
   if (!temperature && !(std::isfinite(temperature_scalar) && temperature_scalar > 0.f))
     return bad(VS_ERR_INVALID_ARG, "temperature_scalar must be finite and > 0");
   if (!out) return bad(VS_ERR_INVALID_ARG, "out is NULL");
+  if (out->sampled || out->support_mask || out->ctx || (flags & VS_WANT_SAMPLE))
+    return bad(VS_ERR_INVALID_ARG, "sampled, support_mask and ctx are not offered by the fused head: pass NULL");
   const bool want_entropy = flags & VS_WANT_ENTROPY;
   if (!want_entropy && (out->entropy_full || out->entropy_support))
     return bad(VS_ERR_INVALID_ARG, "entropy outputs need VS_WANT_ENTROPY");

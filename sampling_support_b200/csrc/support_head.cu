@@ -249,10 +249,10 @@ vs_status support_head_run(int rows, int vocab, int hidden, const void* H, int64
   if (!temperature && !(std::isfinite(temperature_scalar) && temperature_scalar > 0.f))
     return bad(VS_ERR_INVALID_ARG, "temperature_scalar must be finite and > 0");
   if (!out) return bad(VS_ERR_INVALID_ARG, "out is NULL");
-  if (out->logprob_full || out->entropy_full || out->support_mask || out->ctx)
+  if (out->logprob_full || out->entropy_full || out->support_mask || out->ctx || out->sampled)
     return bad(VS_ERR_INVALID_ARG,
-               "logprob_full, entropy_full, support_mask and ctx need the full projection "
-               "(vs_fused_lmhead_score): pass NULL");
+               "logprob_full, entropy_full, support_mask, ctx and sampled are not offered by "
+               "the support-only projection: pass NULL");
   const bool want_entropy = flags & VS_WANT_ENTROPY;
   if (flags & ~static_cast<uint32_t>(VS_WANT_ENTROPY))
     return bad(VS_ERR_INVALID_ARG, "flags other than VS_WANT_ENTROPY are not offered here");

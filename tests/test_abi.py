@@ -167,14 +167,14 @@ def test_support_head_rejects_bad_arguments():
     assert _support_head(ids=0) == inv
     assert _support_head(flags=1 << 1) == inv                  # no mask on this path
     assert _support_head(logits=FAKE, lld=7) == inv
-    for field in ("logprob_full", "entropy_full", "support_mask", "ctx"):
+    for field in ("logprob_full", "entropy_full", "support_mask", "ctx", "sampled"):
         o = B.ScoreOut()
         setattr(o, field, FAKE)
         assert _support_head(out=o) == inv, field
     o = B.ScoreOut()
     o.entropy_support = FAKE
     assert _support_head(out=o, flags=0) == inv               # entropy needs VS_WANT_ENTROPY
-    assert "full projection" in _last_error_after(lambda: _support_head(
+    assert "not offered" in _last_error_after(lambda: _support_head(
         out=_with(B.ScoreOut(), "logprob_full", FAKE)))
 
 
@@ -201,3 +201,17 @@ def test_sample_flag_and_output_go_together():
     o = B.ScoreOut()
     o.sampled = FAKE  # an output without the flag
     assert lib.vs_score_fwd(ctypes.byref(a), ctypes.byref(o), FAKE, 1 << 20, None) == B.VS_ERR_INVALID_ARG
+
+
+def test_fused_head_rejects_outputs_it_does_not_offer():
+    lib = vsb.load()
+    for field in ("sampled", "support_mask", "ctx"):
+        o = B.ScoreOut()
+        setattr(o, field, FAKE)
+        rc = lib.vs_fused_lmhead_score(4, 1000, 64, FAKE, 64, FAKE, 64, None, 1.0, FAKE, 8, 1.0, 0.0,
+                                       0, ctypes.byref(o), None, None, FAKE, 1 << 30, None)
+        assert rc == B.VS_ERR_INVALID_ARG, field
+    o = B.ScoreOut()
+    rc = lib.vs_fused_lmhead_score(4, 1000, 64, FAKE, 64, FAKE, 64, None, 1.0, FAKE, 8, 1.0, 0.0,
+                                   8, ctypes.byref(o), None, None, FAKE, 1 << 30, None)
+    assert rc == B.VS_ERR_INVALID_ARG  # VS_WANT_SAMPLE
