@@ -39,6 +39,8 @@ METRIC = "rows/s and HBM GB/s vs peak at V=151,936 bf16; fused LM-head TFLOP/s"
 VOCAB = 151_936
 ROWS = 128
 L2_BYTES = 126 * 1024 * 1024
+GRAPH_CALLS = 56  # scoring calls per captured graph of the K-step region
+DIST_REPLAYS = 200  # samples of the per-call time distribution
 
 
 def peaks():
@@ -224,37 +226,81 @@ def headline(args, world, rank, pk):
     ws_ptr = 0 if ws is None else ws.data_ptr()
     ws_n = 0 if ws is None else ws.numel()
 
-    def step(i):
-        rc = fwd(ctypes.byref(argsets[i % nbuf]), oref, ws_ptr, ws_n, sp)
+    def call(i, sptr):
+        rc = fwd(ctypes.byref(argsets[i % nbuf]), oref, ws_ptr, ws_n, sptr)
         if rc:
             raise RuntimeError(lib.vs_last_error().decode())
 
     for i in range(args.warmup):
-        step(i)
-    barrier(world)
+        call(i, sp)
+    torch.cuda.synchronize()
+    # The timed steps replay CUDA graphs of back-to-back calls (each call one
+    # kernel launch reading the next rotating buffer): a Python loop issuing
+    # one ctypes call per ~10 us kernel would time the host, not the GPU.
     K = args.steps
+    G = max(1, min(K, GRAPH_CALLS))
+    cap = torch.cuda.Stream()
+
+    def capture(n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(cap):
+            with torch.cuda.graph(g, stream=cap):
+                cptr = ctypes.c_void_p(cap.cuda_stream)
+                for i in range(n):
+                    call(i, cptr)
+        return g
+
+    g_full = capture(G)
+    g_rest = capture(K % G) if K % G else None
+    g_dist = capture(nbuf)
+    reps = K // G
+    for _ in range(2):
+        g_full.replay()
+        g_dist.replay()
+    torch.cuda.synchronize()
+    nd = DIST_REPLAYS
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
+          for _ in range(nd)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(torch.cuda.current_device()) as clk:
         barrier(world)
         t0.record(stream)
-        for i in range(K):
-            ev[i][0].record(stream)
-            step(i)
-            ev[i][1].record(stream)
+        for _ in range(reps):
+            g_full.replay()
+        if g_rest is not None:
+            g_rest.replay()
         t1.record(stream)
         barrier(world)
+        # the distribution of the call time: DIST_REPLAYS replays of a graph
+        # of nbuf calls (one pass over the rotating buffers), outside the
+        # K-step region
+        for r in range(nd):
+            ev[r][0].record(stream)
+            g_dist.replay()
+            ev[r][1].record(stream)
+        torch.cuda.synchronize()
     total_ms = t0.elapsed_time(t1)
-    kernel_ms = [a.elapsed_time(b) for a, b in ev]
+    per_call = np.array([a.elapsed_time(b) / nbuf for a, b in ev])
     total_ms = max_over_ranks(total_ms, world)
-    k_avg = max_over_ranks(float(np.mean(kernel_ms)), world)
     ms_step = total_ms / K
+    # every step is one kernel launch, back to back: its average duration is
+    # the timed region over the launches
+    k_avg = ms_step
     value = weak_value(ROWS, world, ms_step)
     achieved = in_bytes / (k_avg / 1e3) / 1e9
-    res = dict(value=value, ms_per_step=ms_step, kernel_ms=k_avg,
-               kernel_ms_median=float(np.median(kernel_ms)), achieved=achieved,
-               clocks=clk.summary(), nbuf=nbuf, in_bytes=in_bytes)
+    q1, med, q3 = (float(x) for x in np.percentile(per_call, [25, 50, 75]))
+    res = dict(value=value, ms_per_step=ms_step, kernel_ms=k_avg, achieved=achieved,
+               clocks=clk.summary(), nbuf=nbuf, in_bytes=in_bytes, graph_calls=G,
+               per_call_ms={"median": max_over_ranks(med, world), "q1": q1, "q3": q3,
+                            "samples": nd, "calls_per_sample": nbuf,
+                            "gbs_at_median": in_bytes / (med / 1e3) / 1e9,
+                            "sample": f"mean call time over each of {nd} replays of a graph of "
+                                      f"{nbuf} calls (one per rotating buffer), after the "
+                                      f"K-step region"})
+    del g_full, g_rest, g_dist
+    torch.cuda.synchronize()
+    res["support_size"] = outs["size"].cpu().numpy()
+    res["lp_support"] = outs["lp_support"].cpu().numpy()
 
     # end to end through the public binding with host buffers: H2D of the
     # step's inputs from pinned memory, the scoring call, D2H of the results
@@ -367,6 +413,16 @@ def distance_workload(args, pk, steps, out):
                        "bytes": nbytes, "note": "reads draft+target once, writes bf16 gradient"}
     # published context: DSpark loss + backward, 512 rows, RTX 4090 (11.593 ms)
     out["distance"]["context_rtx4090_ms"] = 11.593
+    wt64 = w["weight"].astype(np.float64)
+
+    def l1_oracle(n):
+        import oracle
+
+        return lambda: oracle.l1(w["draft"][:n], w["target"][:n], wt64[:n], want_grad=True)
+
+    out["distance"]["cpu_baseline"] = oracle_baseline(
+        args, l1_oracle(32), 32, "distance rows: L1, accept, weighted loss and draft gradient",
+        units_1t=4, make_fn_1t=l1_oracle(4))
     del d, t, grad, w
     torch.cuda.empty_cache()
 
@@ -396,14 +452,52 @@ def replay_workload(args, pk, steps, out):
         vsb.score_bwd(lg, tg, holder["o"]["ctx"], None, gl, None, gh, support_ids=st, out=dlog)
 
     ms_b = time_steps(rp_bwd, 3, steps)
+
+    # the variants: full-vocabulary statistics for every row (a full read of
+    # every row), and the sparse [rows, width] gradient of the support entries
+    def rp_fwd_full():
+        holder["f"] = vsb.score_fwd(lg, tg, support_ids=st, want_full=True, want_grad=True)
+
+    ms_ff = time_steps(rp_fwd_full, 3, steps)
+    sg = torch.empty((8192, st.shape[1]), dtype=torch.float32, device="cuda")
+
+    def rp_bwd_sparse():
+        vsb.score_bwd(lg, tg, holder["o"]["ctx"], None, gl, None, gh, support_ids=st, out=sg,
+                      mode=vsb.VS_GRAD_SPARSE)
+
+    ms_bs = time_steps(rp_bwd_sparse, 3, steps)
     wbytes = dlog.numel() * 2
     empty = int((w["widths"] == 0).sum())
-    fbytes = w["support"].nbytes + int((w["widths"]).sum()) * 32 + empty * VOCAB * 2
+    # forward bytes: ids, one 32-byte sector per kept id, full rows of the
+    # empty-support rows (their full-vocabulary fallback), outputs
+    fbytes = w["support"].nbytes + int((w["widths"]).sum()) * 32 + empty * VOCAB * 2 + 8192 * 96
+    full_bytes = w["logits"].nbytes + w["support"].nbytes
+    sparse_bytes = w["support"].nbytes + int((w["widths"]).sum()) * 32 + sg.numel() * 4
     out["replay"] = {"rows": 8192, "fwd_ms": ms_f, "bwd_ms": ms_b,
                      "rows_per_s": 8192 / ((ms_f + ms_b) / 1e3),
+                     "fwd_bytes": fbytes, "fwd_gbs": fbytes / (ms_f / 1e3) / 1e9,
+                     "fwd_frac_hbm": fbytes / (ms_f / 1e3) / 1e9 / pk["hbm"],
                      "bwd_gbs": wbytes / (ms_b / 1e3) / 1e9,
-                     "bwd_frac_hbm": wbytes / (ms_b / 1e3) / 1e9 / pk["hbm"],
-                     "fwd_bytes_est": fbytes, "bwd_bytes": wbytes}
+                     "bwd_frac_hbm": wbytes / (ms_b / 1e3) / 1e9 / pk["hbm"], "bwd_bytes": wbytes,
+                     "fwd_full_stats_ms": ms_ff,
+                     "fwd_full_stats_frac_hbm": full_bytes / (ms_ff / 1e3) / 1e9 / pk["hbm"],
+                     "bwd_sparse_ms": ms_bs,
+                     "bwd_sparse_gbs": sparse_bytes / (ms_bs / 1e3) / 1e9,
+                     "empty_support_rows": empty}
+
+    def rp_oracle(n):
+        import oracle
+
+        def run():
+            oracle.score(w["logits"][:n], w["targets"][:n], support=w["support"][:n])
+            oracle.score_grad(w["logits"][:n], w["targets"][:n], None, np.ones(n), None,
+                              np.full(n, 0.01), support=w["support"][:n])
+        return run
+
+    out["replay"]["cpu_baseline"] = oracle_baseline(
+        args, rp_oracle(64), 64, "replay rows: recorded-support forward and dense backward",
+        units_1t=8, make_fn_1t=rp_oracle(8))
+    del sg
     del lg, dlog, holder
     torch.cuda.empty_cache()
 
@@ -496,6 +590,47 @@ def lmhead_workload(args, pk, steps, out, fused=True, support=True):
                          "frac_bf16_burst": tf / pk["bf16"],
                          "frac_bf16_sustained": tf / pk["bf16_sustained"], "flops": flops}
         del wsp
+        # backward: logits recomputed with the gradient epilogue, then
+        # d_hidden = dx W and d_weight = dx^T H (three GEMM-sized products)
+        fwd = vsb.fused_lmhead_score(hs, wt, tg, w["temperature"], w["top_k"],
+                                     float(np.float32(w["top_p"])), float(np.float32(w["min_p"])),
+                                     want_grad=True)
+        ones = torch.ones(w["rows"], device="cuda")
+        tenth = torch.full((w["rows"],), 0.1, device="cuda")
+        lm = vsb.load()
+        bws = torch.empty(lm.vs_fused_lmhead_bwd_workspace_size(w["rows"], w["vocab"], w["hidden"])
+                          + 16, dtype=torch.uint8, device="cuda")
+        res = {}
+
+        def bwd_step():
+            res["g"] = vsb.fused_lmhead_bwd(hs, wt, tg, w["top_k"], fwd, ones, ones, tenth, tenth,
+                                            workspace=bws)
+
+        msb = time_steps(bwd_step, 2, max(3, min(steps, 6)))
+        tfb = 3 * flops / (msb / 1e3) / 1e12
+        out["lmhead_bwd"] = {"rows": w["rows"], "vocab": w["vocab"], "hidden": w["hidden"],
+                             "ms_per_step": msb, "tflops": tfb, "flops": 3 * flops,
+                             "frac_bf16_burst": tfb / pk["bf16"],
+                             "frac_bf16_sustained": tfb / pk["bf16_sustained"],
+                             "note": "logit tiles recomputed (tcgen05, gradient epilogue, bf16 dx "
+                                     "in 32,768-column chunks) + dx W and dx^T H (cuBLASLt)"}
+        del bws, res, fwd
+
+        def lm_oracle(n):
+            import oracle
+
+            sel = np.arange(n, dtype=np.int32)
+            tt = float(np.float32(w["temperature"]))
+
+            def run():
+                z = oracle.lmhead_logits(w["hidden_states"], w["weight"], sel, tt)
+                oracle.score(z, w["targets"][:n], top_k=w["top_k"],
+                             top_p=float(np.float32(w["top_p"])), min_p=float(np.float32(w["min_p"])))
+            return run
+
+        out["lmhead"]["cpu_baseline"] = oracle_baseline(
+            args, lm_oracle(32), 32, "fused-head rows: fp64 projection of the row over the whole "
+            "vocabulary, then the scoring program", units_1t=2, make_fn_1t=lm_oracle(2))
     if support:
         sup = workloads.support_lists(rows=w["rows"], vocab=w["vocab"])
         ids, ty = to_dev(sup["support"]), to_dev(sup["targets"])
@@ -525,6 +660,21 @@ def lmhead_workload(args, pk, steps, out, fused=True, support=True):
         uniq = len(set(int(x) for x in sup["support"].reshape(-1) if x >= 0))
         gathered = 2 * w["hidden"] * (w["rows"] + kept) + 4 * sup["support"].size + 17 * w["rows"]
         unique_bytes = 2 * w["hidden"] * (w["rows"] + uniq) + 4 * sup["support"].size
+        def sh_oracle(n):
+            import oracle
+
+            sel = np.arange(n, dtype=np.int32)
+            tt = float(np.float32(w["temperature"]))
+
+            def run():
+                z = oracle.lmhead_logits(w["hidden_states"], w["weight"], sel, tt)
+                oracle.score(z, sup["targets"][:n], support=sup["support"][:n])
+            return run
+
+        cpu_sh = oracle_baseline(args, sh_oracle(16), 16,
+                                 "support-projection rows: the oracle projects the whole row (it "
+                                 "has no support-only path), then scores the recorded support",
+                                 units_1t=2, make_fn_1t=sh_oracle(2))
         out["support_head"] = {
             "rows": w["rows"], "hidden": w["hidden"], "vocab": w["vocab"],
             "width": int(sup["support"].shape[1]), "kept_ids": kept, "unique_ids": uniq,
@@ -532,14 +682,67 @@ def lmhead_workload(args, pk, steps, out, fused=True, support=True):
             "gather_gbs": gathered / (ms / 1e3) / 1e9,
             "frac_hbm_unique": unique_bytes / (ms / 1e3) / 1e9 / pk["hbm"],
             "note": "gather_gbs counts every kept id's weight row; frac_hbm_unique counts each "
-                    "distinct weight row once (the rest can come from L2); L2 flushed per call"}
+                    "distinct weight row once (the rest can come from L2); L2 flushed per call",
+            "cpu_baseline": cpu_sh}
         del flush, ids, ty
     del hs, wt
     torch.cuda.empty_cache()
 
 
 # ---------------------------------------------------------------------------
+# the oracle beside each secondary workload (bounded samples on the host)
+
+
+def oracle_rate(fn, units, budget_s):
+    """Calls fn() (each call processes `units` units) until budget_s seconds
+    have passed (at least once); returns (units per second, calls)."""
+    n, t = 0, 0.0
+    while n == 0 or t < budget_s:
+        t0 = time.perf_counter()
+        fn()
+        t += time.perf_counter() - t0
+        n += 1
+    return units * n / t, n
+
+
+def oracle_baseline(args, make_fn, units, what, budget=4.0, units_1t=None, make_fn_1t=None):
+    """The oracle on this host's cores and on one thread, for one workload."""
+    if args.no_cpu_baseline:
+        return None
+    import oracle
+
+    cores = oracle.max_threads()
+    rate, calls = oracle_rate(make_fn, units, budget)
+    oracle.set_threads(1)
+    try:
+        r1, c1 = oracle_rate(make_fn_1t or make_fn, units_1t or units, budget / 2)
+    finally:
+        oracle.set_threads(cores)
+    return {"value": rate, "unit": "rows/s", "cores": cores, "threads_1": r1, "kind": "oracle",
+            "sample": f"{what}: {calls} calls of {units} rows on {cores} threads, "
+                      f"{c1} calls of {units_1t or units} rows on 1 thread"}
+
+
+# ---------------------------------------------------------------------------
 # CPU baseline: the oracle as it stands, on a bounded sample
+
+
+def boundary_rows(h):
+    """Rows of the headline batch whose top-p crossing lies within 1e-6 of
+    top_p (the oracle's fp64 margin), and how many of them got a support size
+    other than the oracle's from the GPU call (every other row matches
+    exactly in the parity tests)."""
+    import oracle
+    import workloads
+
+    w = workloads.fullvocab()
+    r = oracle.score(w["logits"], w["targets"], temperature=w["temperature"].astype(np.float64),
+                     top_p=float(np.float32(w["top_p"])))
+    band = r["topp_margin"] < 1e-6
+    differ = band & (h["support_size"] != r["support_size"])
+    off = ~band & (h["support_size"] != r["support_size"])
+    return {"band": 1e-6, "rows": int(band.sum()), "size_differs": int(differ.sum()),
+            "off_band_size_differs": int(off.sum())}
 
 
 def cpu_baseline(seconds=10.0, rows_cap=ROWS):
@@ -560,9 +763,16 @@ def cpu_baseline(seconds=10.0, rows_cap=ROWS):
         t_total += time.perf_counter() - t0
         done += chunk
         i += chunk
-    return {"value": done / t_total, "unit": "rows/s", "cores": cores, "kind": "oracle",
+    oracle.set_threads(1)
+    try:
+        r1, c1 = oracle_rate(lambda: oracle.score(lg[:2], tg[:2], temperature=tp[:2], top_p=pp), 2,
+                             seconds / 4)
+    finally:
+        oracle.set_threads(cores)
+    return {"value": done / t_total, "unit": "rows/s", "cores": cores, "threads_1": r1,
+            "kind": "oracle",
             "sample": f"{done} rows of the fullvocab workload (16-row batches), fp64 oracle with "
-                      f"OpenMP over rows, {t_total:.1f} s"}
+                      f"OpenMP over rows, {t_total:.1f} s; 1 thread: {2 * c1} rows"}
 
 
 def run_reference(args, world, rank):
@@ -670,18 +880,20 @@ def main():
                        "per_rank_rows": ROWS},
             "roofline": {"bound": "hbm", "achieved": h["achieved"], "peak": pk["hbm"],
                          "unit": "GB/s", "frac": h["achieved"] / pk["hbm"], "traffic": traffic,
-                         "kernel": "score_chunk_kernel + score_merge_kernel (one call, PDL-chained; "
-                                   "event time of the whole call)",
+                         "kernel": "score_row_kernel<bf16> (one launch per call; CUDA-graph replays "
+                                   "of back-to-back calls, events around the timed region)",
                          "algorithmic_bytes": h["in_bytes"],
                          "kernel_ms": h["kernel_ms"], "peak_source": pk["src"] + " (MEASURED_PEAKS hbm_gbs)"},
             "clocks": h["clocks"],
             "e2e": h["e2e"],
-            "gpu_launches": 2 * args.steps,  # chunk + merge kernel per call
+            "gpu_launches": args.steps,  # one score_row_kernel launch per call
+            "per_call_ms": h["per_call_ms"],
         }
         if sec is not None:
             line["workloads"] = sec
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline()
+            line["boundary_rows"] = boundary_rows(h)
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -163,14 +163,10 @@ typedef struct vs_score_out {
  * the row) are computed for every row when logprob_full or entropy_full is
  * requested, else only for rows whose S is empty (the lp_V fallback).
  *
- * Workspace: bf16 rows with a computed support (no support_ids) need
- * vs_score_fwd_workspace_size(args) bytes of device scratch, 16-byte
- * aligned, no initial contents required.  One call at a time per workspace
- * (calls on different streams need different workspaces).  Other argument
- * sets need none (NULL, 0).
+ * Workspace: none.  Each row is streamed through one CTA; the workspace
+ * arguments are kept for ABI stability and ignored (pass NULL, 0).
  *
- * Returns VS_ERR_WORKSPACE when a needed workspace is missing, misaligned or
- * too small; VS_ERR_INVALID_ARG for NULL required pointers, R < 0, V < 1,
+ * Returns VS_ERR_INVALID_ARG for NULL required pointers, R < 0, V < 1,
  * ld < V, bad alignment, a non-positive or non-finite temperature_scalar,
  * top_p_scalar outside (0, 1], min_p_scalar outside [0, 1), a flag whose
  * output pointer is NULL; VS_ERR_UNSUPPORTED for V beyond the resident-row
@@ -181,11 +177,7 @@ typedef struct vs_score_out {
 vs_status vs_score_fwd(const vs_score_args* args, const vs_score_out* out, void* workspace,
                        size_t workspace_bytes, void* stream);
 
-/* Workspace bytes vs_score_fwd needs for these arguments: 0 for fp32 rows
- * and for a recorded support; for bf16 rows with a computed support a few
- * hundred bytes per row (16-byte statistics per row chunk and a per-row
- * support decision), for at most the rows of one launch (large batches run
- * as several launches of rows whose logits fit in L2). */
+/* Workspace bytes vs_score_fwd needs for these arguments: always 0. */
 size_t vs_score_fwd_workspace_size(const vs_score_args* args);
 
 /* Largest vocabulary vs_score_fwd accepts for a dtype. */
@@ -239,6 +231,36 @@ vs_status vs_l1_distance(int32_t rows, int32_t vocab, int64_t ld, vs_dtype dtype
 
 size_t vs_l1_distance_workspace_size(int32_t rows);
 
+/* vs_l1_distance for a batch whose rows are split across ranks (data
+ * parallelism; [DSpark] Purpose keeps the distributed normalisation of the
+ * weighted loss: loss = sum over all ranks of w_i L1_i / sum over all ranks
+ * of w_i).  global_weight_sum is a DEVICE pointer to one double: the sum of
+ * the row weights over every rank (for example the all-reduce of each
+ * rank's weight sum; rows with row_weight NULL weigh 1).  Outputs as in
+ * vs_l1_distance, except:
+ *  - grad_draft uses the global denominator:
+ *      (w_i / global_weight_sum) p_j (s_j - sum_k p_k s_k);
+ *  - loss_num_den_loss = { this call's sum w_i L1_i, this call's sum w_i,
+ *      this call's sum w_i L1_i / global_weight_sum } (0 if the global sum is
+ *      0), so the third entries of all ranks add up to the batch loss and the
+ *      first two all-reduce to its numerator and denominator.
+ * The same workspace rules as vs_l1_distance apply.  VS_ERR_INVALID_ARG when
+ * global_weight_sum is NULL or not 8-byte aligned.  The library performs no
+ * collective: the caller reduces the scalars. */
+/* Sum of this shard's row weights in fp64, accumulated in a fixed order,
+ * written to the DEVICE double *out (rows with row_weight NULL weigh 1, so
+ * the sum is rows).  The first step of the row-sharded loss: all-reduce it
+ * over the ranks and pass the result to vs_l1_distance_sharded.
+ * VS_ERR_INVALID_ARG when rows < 0 or out is NULL or not 8-byte aligned. */
+vs_status vs_l1_weight_sum(int32_t rows, const float* row_weight, double* out, void* stream);
+
+vs_status vs_l1_distance_sharded(int32_t rows, int32_t vocab, int64_t ld, vs_dtype dtype,
+                                 const void* draft, const void* target, const float* row_weight,
+                                 const double* global_weight_sum, float* l1, float* accept_rate,
+                                 float* loss_num_den_loss, void* grad_draft, vs_dtype grad_dtype,
+                                 int64_t grad_ld, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
 /* vs_l1_distance without a caller workspace.  The pages have no counterpart:
  * this entry point exists for callers that cannot call cudaMalloc -- for
  * example a plugin inside a host application whose device memory pool it
@@ -250,7 +272,12 @@ size_t vs_l1_distance_workspace_size(int32_t rows);
  *  - rows above VS_L1_STATIC_MAX_ROWS: VS_ERR_UNSUPPORTED, nothing enqueued.
  *  - The first call on a device, with that device current, looks up the
  *    array's device address (cudaGetSymbolAddress) and caches it; make that
- *    first call before any stream capture.
+ *    first call before any stream capture.  The cached address belongs to
+ *    the device's context at that time and does not survive a
+ *    cudaDeviceReset of that device (the module is unloaded and the array
+ *    may sit elsewhere once it is loaded again): a caller that resets a
+ *    device must not call this entry point on it afterwards in the same
+ *    process.
  *  - Every call on a device shares the one array, which keeps the last call's
  *    contents (each call overwrites what it reads), so calls that overlap on
  *    the GPU (concurrent streams, or threads without ordering) race. */
@@ -276,8 +303,12 @@ vs_status vs_l1_distance_static(int32_t rows, int32_t vocab, int64_t ld, vs_dtyp
  * hidden [rows, hidden_dim] and weight [vocab, hidden_dim] are bf16, K-major,
  * row strides ldh/ldw elements (multiples of 8), 16-byte aligned; hidden_dim
  * a multiple of 64.  top_k in [1, VS_MAX_FUSED_TOPK] (top-p without top-k is
- * not offered here).  out->support_mask, ctx and sampled must be NULL (and
- * VS_WANT_SAMPLE unset).  Needs vs_fused_lmhead_workspace_size(...) bytes. */
+ * not offered here).  out->support_mask and sampled must be NULL (and
+ * VS_WANT_SAMPLE unset).  With VS_WANT_GRAD, out->ctx receives
+ * [rows, VS_CTX_BYTES_PER_ROW] bytes of saved state (16-byte aligned) for
+ * vs_fused_lmhead_bwd, which also needs topk_ids (the support is its first
+ * support_size entries); VS_WANT_GRAD and ctx go together and need topk_ids.
+ * Needs vs_fused_lmhead_workspace_size(...) bytes. */
 vs_status vs_fused_lmhead_score(int32_t rows, int32_t vocab, int32_t hidden_dim,
                                 const void* hidden, int64_t ldh, const void* weight,
                                 int64_t ldw, const float* temperature,
@@ -289,6 +320,38 @@ vs_status vs_fused_lmhead_score(int32_t rows, int32_t vocab, int32_t hidden_dim,
 
 size_t vs_fused_lmhead_workspace_size(int32_t rows, int32_t vocab, int32_t hidden_dim,
                                       int32_t top_k);
+
+/* Backward of vs_fused_lmhead_score ([xorl] section 1: "selected logprob +
+ * VJP"; the logits are recomputed, never stored whole).  With x = H W^T,
+ * z = x / T and the upstream gradients g_* of lp_V, lp_S, H_V, H_S ([R] fp32
+ * each, NULL = 0), the logit gradient is
+ *   dx_j = (1/T) ( g_lpV ([j==y] - p_j) + g_lpS 1_S(j) ([j==y] - q_j)
+ *                 - g_HV p_j (log p_j + H_V) - g_HS 1_S(j) q_j (log q_j + H_S) )
+ * (the rules of vs_score_bwd for empty supports, targets outside S or
+ * outside [0, V), and non-finite rows), and
+ *   d_hidden [rows, hidden_dim] = dx W        (fp32, row stride ld_dh),
+ *   d_weight [vocab, hidden_dim] = dx^T H     (fp32, row stride ld_dw);
+ * either may be NULL (not computed).  Both are overwritten.  The logit tiles
+ * are recomputed on the tensor cores chunk by chunk of the vocabulary, dx is
+ * formed in the GEMM epilogue and rounded to bf16 (the support and target
+ * entries are recomputed and written whole), and the two products run as
+ * plain bf16 GEMMs with fp32 accumulation (cuBLASLt, inside the caller's
+ * workspace).  hidden, weight, targets and top_k are those of the forward
+ * call; ctx and topk_ids its outputs (VS_WANT_GRAD).  Output pointers 16-byte
+ * aligned, ld_dh / ld_dw >= hidden_dim and multiples of 4.  Needs
+ * vs_fused_lmhead_bwd_workspace_size(rows, vocab, hidden_dim) bytes (a bf16
+ * [rows, 32768] gradient chunk plus 32 MiB).  Errors as for
+ * vs_fused_lmhead_score. */
+vs_status vs_fused_lmhead_bwd(int32_t rows, int32_t vocab, int32_t hidden_dim, const void* hidden,
+                              int64_t ldh, const void* weight, int64_t ldw,
+                              const int32_t* targets, int32_t top_k, const void* ctx,
+                              const int32_t* topk_ids, const float* g_lp_full,
+                              const float* g_lp_support, const float* g_h_full,
+                              const float* g_h_support, float* d_hidden, int64_t ld_dh,
+                              float* d_weight, int64_t ld_dw, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+size_t vs_fused_lmhead_bwd_workspace_size(int32_t rows, int32_t vocab, int32_t hidden_dim);
 
 /* Support-only fused projection ([SkyRL] Performance: with a fused LM head
  * the replay path projects only the selected hidden-state / weight pairs and

@@ -119,6 +119,38 @@ def score(logits, targets, temperature=1.0, top_k=0, top_p=1.0, min_p=0.0,
     return out
 
 
+def prefix(logits, prefix_len, temperature=1.0, top_k=0, vocab=None, want_ids=False):
+    """Facts of the first n = prefix_len[i] entries of each row's total order
+    (vso_prefix): top-p masses at n and n - 1 (renormalised over the top-k
+    set), min-p ratios exp(z - m) of the n-th and (n+1)-th entries, the top-k
+    size, and optionally the ids (a list of arrays)."""
+    logits = np.ascontiguousarray(logits)
+    rows, ld = logits.shape
+    vocab = ld if vocab is None else vocab
+    n = np.ascontiguousarray(prefix_len, dtype=np.int32)
+    assert n.shape == (rows,)
+    t_arr, t_s = _row_param(temperature, rows, np.float64)
+    k_arr, k_s = _row_param(top_k, rows, np.int32)
+    max_ids = max(1, int(n.max(initial=0))) if want_ids else 0
+    ids = np.full((rows, max_ids), -1, np.int32) if want_ids else None
+    out = {k: np.empty(rows, np.float64) for k in ("mass_n", "mass_prev", "ratio_n", "ratio_next")}
+    nk = np.empty(rows, np.int32)
+    L = lib()
+    L.vso_prefix.restype = ctypes.c_int
+    rc = L.vso_prefix(ctypes.c_int(rows), ctypes.c_int(vocab), ctypes.c_int64(ld),
+                      ctypes.c_int(_dtype_code(logits)), _ptr(logits), _ptr(t_arr),
+                      ctypes.c_double(t_s), _ptr(k_arr), ctypes.c_int32(int(k_s)), _ptr(n),
+                      _ptr(ids), ctypes.c_int(max_ids), _ptr(out["mass_n"]),
+                      _ptr(out["mass_prev"]), _ptr(out["ratio_n"]), _ptr(out["ratio_next"]),
+                      _ptr(nk))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    out["nk"] = nk
+    if want_ids:
+        out["ids"] = [ids[i, :n[i]] for i in range(rows)]
+    return out
+
+
 def score_grad(logits, targets, g_lp_full=None, g_lp_support=None, g_h_full=None,
                g_h_support=None, temperature=1.0, top_k=0, top_p=1.0, min_p=0.0,
                support=None, vocab=None):
@@ -150,7 +182,9 @@ def score_grad(logits, targets, g_lp_full=None, g_lp_support=None, g_h_full=None
     return d
 
 
-def l1(draft, target, weight=None, want_grad=False, tie_eps=1e-6, vocab=None):
+def l1(draft, target, weight=None, want_grad=False, tie_eps=1e-6, vocab=None, global_wsum=None):
+    """Draft/target distance; global_wsum: the weight sum over all shards of a
+    row-sharded batch (the loss denominator), else this call's."""
     draft = np.ascontiguousarray(draft)
     target = np.ascontiguousarray(target)
     assert draft.dtype == target.dtype and draft.shape == target.shape
@@ -165,7 +199,8 @@ def l1(draft, target, weight=None, want_grad=False, tie_eps=1e-6, vocab=None):
     rc = L.vso_l1(ctypes.c_int(rows), ctypes.c_int(vocab), ctypes.c_int64(ld),
                   ctypes.c_int(_dtype_code(draft)), _ptr(draft), _ptr(target), _ptr(w),
                   _ptr(out["l1"]), _ptr(out["accept"]), _ptr(nd), _ptr(g),
-                  ctypes.c_double(tie_eps), _ptr(ties))
+                  ctypes.c_double(tie_eps), _ptr(ties),
+                  None if global_wsum is None else ctypes.byref(ctypes.c_double(global_wsum)))
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     out.update(loss_num=nd[0], loss_den=nd[1], loss=nd[2], near_ties=ties)
@@ -189,6 +224,33 @@ def lmhead_logits(hidden_bits, weight_bits, rows_sel, temperature):
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     return out
+
+
+def _wide(a):
+    """bf16 bit patterns (uint16) or float64 values, widened exactly to float64."""
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def lmhead_grad(hidden, weight, targets, temperature, g_lp_full=None, g_lp_support=None,
+                g_h_full=None, g_h_support=None, top_k=0, top_p=1.0, min_p=0.0, support=None):
+    """Gradients of L = sum_i g_lpV lp_V + g_lpS lp_S + g_hV H_V + g_hS H_S
+    with respect to the LM head's inputs (xorl issue #71, section 1: the
+    projection, then the scoring op, then its VJP).  With x = H W^T
+    (fp64 products of the exact inputs) and z = x / T, the logit gradient
+    dz comes from score_grad on z; then dx = dz / T and
+        dH = dx W,   dW = dx^T H   (numpy matmul in fp64).
+    hidden [rows, hidden] and weight [vocab, hidden] are bf16 bit patterns
+    or float64; temperature a scalar.  Returns (dH, dW)."""
+    H = _wide(hidden)
+    W = _wide(weight)
+    z = (H @ W.T) / float(temperature)
+    dz = score_grad(z, targets, g_lp_full, g_lp_support, g_h_full, g_h_support, temperature=1.0,
+                    top_k=top_k, top_p=top_p, min_p=min_p, support=support)
+    dx = dz / float(temperature)
+    return dx @ W, dx.T @ H
 
 
 def set_threads(n: int) -> None:

@@ -307,6 +307,60 @@ int vso_score(int rows, int vocab, int64_t ld, int dtype, const void* logits,
   return 0;
 }
 
+// Prefix facts of the computed-support order, for checking a support whose
+// top-p or min-p decision sits within rounding of its threshold.  For row i
+// and a prefix length n = prefix_len[i] of the total order (z descending,
+// token id ascending; [xorl] section 3), with m the row maximum and the
+// top-p mass renormalised over the top-k set (k = top_k when 0 < top_k <
+// vocab, else vocab):
+//   ids[i, 0 .. n-1]  the first n ids (n <= max_ids),
+//   mass_n[i]         sum_{first n} exp(z - m) / sum_{first k} exp(z - m),
+//   mass_prev[i]      the same over the first n - 1 (0 when n == 0),
+//   ratio_n[i]        exp(z - m) of the n-th entry (1 when n == 0),
+//   ratio_next[i]     exp(z - m) of the (n+1)-th entry (0 when n == vocab),
+//   nk[i]             k.
+// Any output array may be null.  Returns 1 on bad arguments.
+int vso_prefix(int rows, int vocab, int64_t ld, int dtype, const void* logits,
+               const double* temperature, double temperature_scalar, const int32_t* top_k,
+               int32_t top_k_scalar, const int32_t* prefix_len, int32_t* ids, int max_ids,
+               double* mass_n, double* mass_prev, double* ratio_n, double* ratio_next,
+               int32_t* nk) {
+  if (rows < 0 || vocab <= 0 || ld < vocab || !logits || !prefix_len) return 1;
+  for (int i = 0; i < rows; ++i)
+    if (prefix_len[i] < 0 || prefix_len[i] > vocab || (ids && prefix_len[i] > max_ids)) return 1;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int i = 0; i < rows; ++i) {
+    const double t = pick(temperature, i, temperature_scalar);
+    std::vector<double> z(vocab);
+    for (int j = 0; j < vocab; ++j)
+      z[j] = load_value(logits, dtype, static_cast<int64_t>(i) * ld + j) / t;
+    std::vector<int32_t> order(vocab);
+    std::iota(order.begin(), order.end(), 0);
+    std::sort(order.begin(), order.end(), [&](int32_t a, int32_t b) {
+      if (z[a] != z[b]) return z[a] > z[b];
+      return a < b;
+    });
+    const double m = z[order[0]];
+    const int32_t k = pick(top_k, i, top_k_scalar);
+    const int n1 = (k > 0 && k < vocab) ? k : vocab;
+    const int n = prefix_len[i];
+    double mass1 = 0.0, cum = 0.0, prev = 0.0;
+    for (int r = 0; r < n1; ++r) mass1 += std::exp(z[order[r]] - m);
+    for (int r = 0; r < n; ++r) {
+      prev = cum;
+      cum += std::exp(z[order[r]] - m);
+    }
+    if (ids)
+      for (int r = 0; r < n; ++r) ids[static_cast<int64_t>(i) * max_ids + r] = order[r];
+    if (mass_n) mass_n[i] = cum / mass1;
+    if (mass_prev) mass_prev[i] = n > 0 ? prev / mass1 : 0.0;
+    if (ratio_n) ratio_n[i] = n > 0 ? std::exp(z[order[n - 1]] - m) : 1.0;
+    if (ratio_next) ratio_next[i] = n < vocab ? std::exp(z[order[n]] - m) : 0.0;
+    if (nk) nk[i] = n1;
+  }
+  return 0;
+}
+
 // Gradient of  g_lpV*lp_V + g_lpS*lp_S + g_hV*H_V + g_hS*H_S  with respect to
 // the input logits l (dl = dz / T), by the closed forms
 //   d lp / dz_j = [j == y] - p_j                      (softmax over the set)
@@ -374,12 +428,18 @@ int vso_score_grad(int rows, int vocab, int64_t ld, int dtype, const void* logit
 // which is the softmax Jacobian applied to d|p - q|/dp = s.
 // `near_ties` (may be null) counts, per row, elements with |p - q| < tie_eps,
 // where a sign decision at lower precision may differ.
+//
+// Row-sharded batches ([DSpark] Purpose keeps the distributed normalisation
+// of the loss): when global_wsum is non-null it is the weight sum over all
+// shards, and the loss denominator of the gradient and of loss_num_den[2];
+// loss_num_den[0..1] stay this call's numerator and weight sum.
 int vso_l1(int rows, int vocab, int64_t ld, int dtype, const void* draft, const void* target,
            const double* row_weight, double* l1, double* accept, double* loss_num_den,
-           double* grad, double tie_eps, int32_t* near_ties) {
+           double* grad, double tie_eps, int32_t* near_ties, const double* global_wsum) {
   if (rows < 0 || vocab <= 0 || ld < vocab || !draft || !target) return 1;
-  double wsum = 0.0;
-  for (int i = 0; i < rows; ++i) wsum += row_weight ? row_weight[i] : 1.0;
+  double local_wsum = 0.0;
+  for (int i = 0; i < rows; ++i) local_wsum += row_weight ? row_weight[i] : 1.0;
+  const double wsum = global_wsum ? *global_wsum : local_wsum;
   std::vector<double> l1v(rows);
 #pragma omp parallel for schedule(dynamic, 1)
   for (int i = 0; i < rows; ++i) {
@@ -429,7 +489,7 @@ int vso_l1(int rows, int vocab, int64_t ld, int dtype, const void* draft, const 
     double num = 0.0;
     for (int i = 0; i < rows; ++i) num += (row_weight ? row_weight[i] : 1.0) * l1v[i];
     loss_num_den[0] = num;
-    loss_num_den[1] = wsum;
+    loss_num_den[1] = local_wsum;
     loss_num_den[2] = wsum > 0.0 ? num / wsum : 0.0;
   }
   return 0;

@@ -5,8 +5,10 @@ ctypes binding.  PyTorch is used only for device memory and streams."""
 from ._binding import (  # noqa: F401
     LIB_PATH,
     VsError,
+    fused_lmhead_bwd,
     fused_lmhead_score,
     l1_distance,
+    l1_weight_sum,
     load,
     score_bwd,
     score_fwd,

@@ -87,6 +87,12 @@ def load() -> ctypes.CDLL:
         lib.vs_l1_distance.argtypes = [i32, i32, ctypes.c_int64, i32, _vp, _vp, _vp, _vp, _vp, _vp,
                                        _vp, i32, ctypes.c_int64, _vp, sz, _vp]
         lib.vs_l1_distance.restype = i32
+        lib.vs_l1_distance_sharded.argtypes = [i32, i32, ctypes.c_int64, i32, _vp, _vp, _vp, _vp,
+                                               _vp, _vp, _vp, _vp, i32, ctypes.c_int64, _vp, sz,
+                                               _vp]
+        lib.vs_l1_distance_sharded.restype = i32
+        lib.vs_l1_weight_sum.argtypes = [i32, _vp, _vp, _vp]
+        lib.vs_l1_weight_sum.restype = i32
         lib.vs_l1_distance_workspace_size.argtypes = [i32]
         lib.vs_l1_distance_workspace_size.restype = sz
         lib.vs_fused_lmhead_score.argtypes = [i32, i32, i32, _vp, ctypes.c_int64, _vp,
@@ -96,6 +102,13 @@ def load() -> ctypes.CDLL:
         lib.vs_fused_lmhead_score.restype = i32
         lib.vs_fused_lmhead_workspace_size.argtypes = [i32, i32, i32, i32]
         lib.vs_fused_lmhead_workspace_size.restype = sz
+        lib.vs_fused_lmhead_bwd.argtypes = [i32, i32, i32, _vp, ctypes.c_int64, _vp,
+                                            ctypes.c_int64, _vp, i32, _vp, _vp, _vp, _vp, _vp,
+                                            _vp, _vp, ctypes.c_int64, _vp, ctypes.c_int64, _vp,
+                                            sz, _vp]
+        lib.vs_fused_lmhead_bwd.restype = i32
+        lib.vs_fused_lmhead_bwd_workspace_size.argtypes = [i32, i32, i32]
+        lib.vs_fused_lmhead_bwd_workspace_size.restype = sz
         lib.vs_support_lmhead_score.argtypes = [i32, i32, i32, _vp, ctypes.c_int64, _vp,
                                                 ctypes.c_int64, _vp, ctypes.c_float, _vp, _vp, i32,
                                                 ctypes.c_int64, ctypes.c_uint32,
@@ -272,7 +285,12 @@ def score_bwd(logits, targets, ctx, g_lp_full=None, g_lp_support=None, g_h_full=
 
 
 def l1_distance(draft, target, row_weight=None, want_loss=True, want_grad=False,
-                grad_dtype=torch.float32, workspace=None, vocab=None, stream=None):
+                grad_dtype=torch.float32, workspace=None, vocab=None, stream=None,
+                global_weight_sum=None):
+    """vs_l1_distance; with global_weight_sum (a float64 device tensor of one
+    element: the row-weight sum over every rank of a row-sharded batch)
+    vs_l1_distance_sharded, whose gradient and loss value use that
+    denominator."""
     lib = load()
     rows, ld = draft.shape
     vocab = ld if vocab is None else vocab
@@ -288,15 +306,35 @@ def l1_distance(draft, target, row_weight=None, want_loss=True, want_grad=False,
         workspace = torch.empty((nbytes + 15) // 16 * 16, dtype=torch.uint8, device=dev)
     gcode = VS_BF16 if grad_dtype == torch.bfloat16 else VS_F32
     g = out.get("grad")
-    _check(lib.vs_l1_distance(rows, vocab, draft.stride(0), _dtype_code(draft), _p(draft), _p(target),
-                              _p(row_weight), _p(out["l1"]), _p(out["accept"]), _p(out.get("loss")),
-                              _p(g), gcode, 0 if g is None else g.stride(0), _p(workspace),
-                              0 if workspace is None else workspace.numel(), _stream(stream)))
+    common = (_p(out["l1"]), _p(out["accept"]), _p(out.get("loss")), _p(g), gcode,
+              0 if g is None else g.stride(0), _p(workspace),
+              0 if workspace is None else workspace.numel(), _stream(stream))
+    if global_weight_sum is None:
+        _check(lib.vs_l1_distance(rows, vocab, draft.stride(0), _dtype_code(draft), _p(draft),
+                                  _p(target), _p(row_weight), *common))
+    else:
+        assert global_weight_sum.dtype == torch.float64 and global_weight_sum.device == dev
+        _check(lib.vs_l1_distance_sharded(rows, vocab, draft.stride(0), _dtype_code(draft),
+                                          _p(draft), _p(target), _p(row_weight),
+                                          _p(global_weight_sum), *common))
+    return out
+
+
+def l1_weight_sum(rows, row_weight=None, out=None, device=None, stream=None):
+    """vs_l1_weight_sum: this shard's weight sum as a float64 device tensor of
+    one element (row_weight None: every row weighs 1)."""
+    lib = load()
+    dev = row_weight.device if row_weight is not None else (device or torch.device("cuda"))
+    if out is None:
+        out = torch.empty(1, dtype=torch.float64, device=dev)
+    _check(lib.vs_l1_weight_sum(rows, _p(row_weight), _p(out), _stream(stream)))
     return out
 
 
 def fused_lmhead_score(hidden, weight, targets, temperature, top_k, top_p, min_p,
-                       want_entropy=True, workspace=None, stream=None):
+                       want_entropy=True, want_grad=False, workspace=None, stream=None):
+    """vs_fused_lmhead_score; want_grad also returns out["ctx"] (the saved
+    state for fused_lmhead_bwd)."""
     lib = load()
     rows, hdim = hidden.shape
     vocab = weight.shape[0]
@@ -313,6 +351,8 @@ def fused_lmhead_score(hidden, weight, targets, temperature, top_k, top_p, min_p
     if want_entropy:
         out["h_full"] = torch.empty(rows, **f32)
         out["h_support"] = torch.empty(rows, **f32)
+    if want_grad:
+        out["ctx"] = torch.empty((rows, 64), dtype=torch.uint8, device=dev)
     o = ScoreOut()
     o.logprob_full = _p(out["lp_full"])
     o.logprob_support = _p(out["lp_support"])
@@ -321,6 +361,7 @@ def fused_lmhead_score(hidden, weight, targets, temperature, top_k, top_p, min_p
     o.valid = _p(out["valid"])
     o.status = _p(out["status"])
     o.support_size = _p(out["support_size"])
+    o.ctx = _p(out.get("ctx"))
     t_arr = temperature if isinstance(temperature, torch.Tensor) else None
     t_s = 1.0 if t_arr is not None else float(temperature)
     if workspace is None:
@@ -329,9 +370,39 @@ def fused_lmhead_score(hidden, weight, targets, temperature, top_k, top_p, min_p
     _check(lib.vs_fused_lmhead_score(rows, vocab, hdim, _p(hidden), hidden.stride(0), _p(weight),
                                      weight.stride(0), _p(t_arr), t_s, _p(targets), top_k,
                                      float(top_p), float(min_p),
-                                     VS_WANT_ENTROPY if want_entropy else 0, ctypes.byref(o),
+                                     (VS_WANT_ENTROPY if want_entropy else 0)
+                                     | (VS_WANT_GRAD if want_grad else 0), ctypes.byref(o),
                                      _p(out["topk_ids"]), _p(out["topk_logprob"]), _p(workspace),
                                      workspace.numel(), _stream(stream)))
+    return out
+
+
+def fused_lmhead_bwd(hidden, weight, targets, top_k, fwd, g_lp_full=None, g_lp_support=None,
+                     g_h_full=None, g_h_support=None, want_hidden=True, want_weight=True,
+                     workspace=None, stream=None):
+    """vs_fused_lmhead_bwd from a fused_lmhead_score(..., want_grad=True)
+    result `fwd`; returns {"d_hidden": [rows, hidden] fp32, "d_weight":
+    [vocab, hidden] fp32} (the requested ones)."""
+    lib = load()
+    rows, hdim = hidden.shape
+    vocab = weight.shape[0]
+    dev = hidden.device
+    out = {}
+    if want_hidden:
+        out["d_hidden"] = torch.empty((rows, hdim), dtype=torch.float32, device=dev)
+    if want_weight:
+        out["d_weight"] = torch.empty((vocab, hdim), dtype=torch.float32, device=dev)
+    if workspace is None:
+        nbytes = lib.vs_fused_lmhead_bwd_workspace_size(rows, vocab, hdim)
+        workspace = torch.empty(max(16, (nbytes + 15) // 16 * 16), dtype=torch.uint8, device=dev)
+    dh, dw = out.get("d_hidden"), out.get("d_weight")
+    _check(lib.vs_fused_lmhead_bwd(rows, vocab, hdim, _p(hidden), hidden.stride(0), _p(weight),
+                                   weight.stride(0), _p(targets), top_k, _p(fwd["ctx"]),
+                                   _p(fwd["topk_ids"]), _p(g_lp_full), _p(g_lp_support),
+                                   _p(g_h_full), _p(g_h_support), _p(dh),
+                                   0 if dh is None else dh.stride(0), _p(dw),
+                                   0 if dw is None else dw.stride(0), _p(workspace),
+                                   workspace.numel(), _stream(stream)))
     return out
 
 

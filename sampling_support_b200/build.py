@@ -13,7 +13,7 @@ CSRC = PKG / "csrc"
 INCLUDE = PKG.parent / "include"
 LIB = PKG / "libvs.so"
 
-SOURCES = ["api.cu", "score_fwd.cu", "score_row.cu", "score_split.cu", "score_bwd.cu", "l1_distance.cu", "fused_lmhead.cu", "support_head.cu"]
+SOURCES = ["api.cu", "score_fwd.cu", "score_row.cu", "score_bwd.cu", "l1_distance.cu", "fused_lmhead.cu", "support_head.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -55,7 +55,8 @@ def build(force: bool = False, verbose: bool = False) -> Path:
             sys.stderr.write(r.stderr)
         objs.append(str(obj))
     tmp = LIB.with_suffix(f".so.tmp{os.getpid()}")
-    cmd = [cc, *ARCH, "-shared", "-o", str(tmp), *objs]
+    cmd = [cc, *ARCH, "-shared", "-o", str(tmp), *objs, "-lcublasLt",
+           "-Xlinker", "-rpath,/usr/local/cuda/lib64"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)

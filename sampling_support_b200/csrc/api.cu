@@ -14,7 +14,8 @@ int l1_max_vocab(vs_dtype dtype);
 cudaError_t launch_l1(int rows, int vocab, int64_t ld, vs_dtype dtype, const void* draft,
                       const void* target, const float* row_weight, float* l1, float* accept,
                       float* loss3, void* grad, vs_dtype gdtype, int64_t grad_ld, void* ws,
-                      cudaStream_t s);
+                      const double* global_wsum, cudaStream_t s);
+cudaError_t launch_l1_weight_sum(int rows, const float* row_weight, double* out, cudaStream_t s);
 size_t lmhead_workspace_bytes(int rows, int vocab, int hidden, int top_k);
 vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh, const void* W,
                      int64_t ldw, const float* temperature, float temperature_scalar,
@@ -22,6 +23,14 @@ vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh
                      uint32_t flags, const vs_score_out* out, int32_t* topk_ids,
                      float* topk_logprob, void* ws, size_t ws_bytes, cudaStream_t s,
                      std::string* err);
+size_t lmhead_bwd_workspace_bytes(int rows, int vocab, int hidden);
+vs_status lmhead_bwd_run(int rows, int vocab, int hidden, const void* H, int64_t ldh,
+                         const void* W, int64_t ldw, const int32_t* targets, int top_k,
+                         const void* ctx, const int32_t* topk_ids, const float* g_lp_full,
+                         const float* g_lp_support, const float* g_h_full,
+                         const float* g_h_support, float* d_hidden, int64_t ld_dh,
+                         float* d_weight, int64_t ld_dw, void* ws, size_t ws_bytes,
+                         cudaStream_t s, std::string* err);
 vs_status support_head_run(int rows, int vocab, int hidden, const void* H, int64_t ldh,
                            const void* W, int64_t ldw, const float* temperature,
                            float temperature_scalar, const int32_t* targets,
@@ -118,9 +127,8 @@ int32_t vs_score_max_vocab(vs_dtype dtype) {
 }
 
 size_t vs_score_fwd_workspace_size(const vs_score_args* args) {
-  if (!args || args->rows <= 0 || args->vocab < 1 || args->support_ids || args->dtype != VS_BF16)
-    return 0;
-  return vs::score_split_workspace_bytes(args->rows, args->vocab);
+  (void)args;
+  return 0;
 }
 
 vs_status vs_score_fwd(const vs_score_args* a, const vs_score_out* o, void* workspace,
@@ -148,13 +156,8 @@ vs_status vs_score_fwd(const vs_score_args* a, const vs_score_out* o, void* work
   const bool recorded = a->support_ids != nullptr;
   if (!recorded && a->vocab > vs::score_max_vocab(a->dtype))
     return fail(VS_ERR_UNSUPPORTED, "vocab exceeds vs_score_max_vocab for this dtype");
-  const bool split = !recorded && a->dtype == VS_BF16;
-  if (split) {
-    const size_t need = vs::score_split_workspace_bytes(a->rows, a->vocab);
-    if (!workspace || !aligned16(workspace) || workspace_bytes < need)
-      return fail(VS_ERR_WORKSPACE,
-                  "workspace missing, misaligned or smaller than vs_score_fwd_workspace_size(args)");
-  }
+  (void)workspace;
+  (void)workspace_bytes;
 
   vs::ScoreParams p{};
   p.rows = a->rows;
@@ -196,8 +199,6 @@ vs_status vs_score_fwd(const vs_score_args* a, const vs_score_out* o, void* work
   cudaError_t e;
   if (recorded)
     e = vs::launch_score_recorded(p, a->dtype, s);
-  else if (split)
-    e = vs::launch_score_split(p, workspace, s);
   else
     e = vs::launch_score_computed(p, a->dtype, s);
   if (e != cudaSuccess) return cuda_fail(e, "vs_score_fwd launch");
@@ -271,11 +272,15 @@ vs_status vs_score_bwd(const vs_score_args* a, const void* ctx, const float* g_l
 
 size_t vs_l1_distance_workspace_size(int32_t rows) { return vs::l1_workspace_bytes(rows); }
 
-vs_status vs_l1_distance(int32_t rows, int32_t vocab, int64_t ld, vs_dtype dtype,
-                         const void* draft, const void* target, const float* row_weight,
-                         float* l1, float* accept_rate, float* loss_num_den_loss,
-                         void* grad_draft, vs_dtype grad_dtype, int64_t grad_ld,
-                         void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+vs_status l1_call(int32_t rows, int32_t vocab, int64_t ld, vs_dtype dtype, const void* draft,
+                  const void* target, const float* row_weight, float* l1, float* accept_rate,
+                  float* loss_num_den_loss, void* grad_draft, vs_dtype grad_dtype,
+                  int64_t grad_ld, const double* global_weight_sum, void* workspace,
+                  size_t workspace_bytes, void* stream) {
   if (rows < 0) return fail(VS_ERR_INVALID_ARG, "rows must be >= 0");
   if (vocab < 1) return fail(VS_ERR_INVALID_ARG, "vocab must be >= 1");
   if (ld < vocab) return fail(VS_ERR_INVALID_ARG, "ld must be >= vocab");
@@ -304,8 +309,66 @@ vs_status vs_l1_distance(int32_t rows, int32_t vocab, int64_t ld, vs_dtype dtype
   }
   cudaError_t e = vs::launch_l1(rows, vocab, ld, dtype, draft, target, row_weight, l1, accept_rate,
                                 loss_num_den_loss, grad_draft, grad_dtype, grad_ld, workspace,
-                                static_cast<cudaStream_t>(stream));
+                                global_weight_sum, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "vs_l1_distance launch");
+  return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+vs_status vs_l1_distance(int32_t rows, int32_t vocab, int64_t ld, vs_dtype dtype,
+                         const void* draft, const void* target, const float* row_weight,
+                         float* l1, float* accept_rate, float* loss_num_den_loss,
+                         void* grad_draft, vs_dtype grad_dtype, int64_t grad_ld,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  return l1_call(rows, vocab, ld, dtype, draft, target, row_weight, l1, accept_rate,
+                 loss_num_den_loss, grad_draft, grad_dtype, grad_ld, nullptr, workspace,
+                 workspace_bytes, stream);
+}
+
+vs_status vs_l1_weight_sum(int32_t rows, const float* row_weight, double* out, void* stream) {
+  if (rows < 0) return fail(VS_ERR_INVALID_ARG, "rows must be >= 0");
+  if (!out || reinterpret_cast<uintptr_t>(out) % 8 != 0)
+    return fail(VS_ERR_INVALID_ARG, "out must be a non-NULL, 8-byte aligned device pointer");
+  cudaError_t e = vs::launch_l1_weight_sum(rows, row_weight, out, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "vs_l1_weight_sum launch");
+  return ok();
+}
+
+vs_status vs_l1_distance_sharded(int32_t rows, int32_t vocab, int64_t ld, vs_dtype dtype,
+                                 const void* draft, const void* target, const float* row_weight,
+                                 const double* global_weight_sum, float* l1, float* accept_rate,
+                                 float* loss_num_den_loss, void* grad_draft, vs_dtype grad_dtype,
+                                 int64_t grad_ld, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  if (!global_weight_sum) return fail(VS_ERR_INVALID_ARG, "global_weight_sum must be non-NULL");
+  if (reinterpret_cast<uintptr_t>(global_weight_sum) % 8 != 0)
+    return fail(VS_ERR_INVALID_ARG, "global_weight_sum must be 8-byte aligned");
+  return l1_call(rows, vocab, ld, dtype, draft, target, row_weight, l1, accept_rate,
+                 loss_num_den_loss, grad_draft, grad_dtype, grad_ld, global_weight_sum,
+                 workspace, workspace_bytes, stream);
+}
+
+size_t vs_fused_lmhead_bwd_workspace_size(int32_t rows, int32_t vocab, int32_t hidden_dim) {
+  return vs::lmhead_bwd_workspace_bytes(rows, vocab, hidden_dim);
+}
+
+vs_status vs_fused_lmhead_bwd(int32_t rows, int32_t vocab, int32_t hidden_dim, const void* hidden,
+                              int64_t ldh, const void* weight, int64_t ldw,
+                              const int32_t* targets, int32_t top_k, const void* ctx,
+                              const int32_t* topk_ids, const float* g_lp_full,
+                              const float* g_lp_support, const float* g_h_full,
+                              const float* g_h_support, float* d_hidden, int64_t ld_dh,
+                              float* d_weight, int64_t ld_dw, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  std::string err;
+  const vs_status st = vs::lmhead_bwd_run(
+      rows, vocab, hidden_dim, hidden, ldh, weight, ldw, targets, top_k, ctx, topk_ids, g_lp_full,
+      g_lp_support, g_h_full, g_h_support, d_hidden, ld_dh, d_weight, ld_dw, workspace,
+      workspace_bytes, static_cast<cudaStream_t>(stream), &err);
+  if (st != VS_OK) return fail(st, err);
   return ok();
 }
 

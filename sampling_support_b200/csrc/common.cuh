@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cooperative_groups.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -322,6 +323,58 @@ __device__ __forceinline__ void bulk_load_all(void* dst, const void* src, uint32
   for (uint32_t off = 0; off < bytes; off += kBulkPiece) {
     const uint32_t n = min(kBulkPiece, bytes - off);
     bulk_load(static_cast<char*>(dst) + off, static_cast<const char*>(src) + off, n, bar);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// bf16 streaming statistics
+
+__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
+  const __nv_bfloat162 r = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&a),
+                                   *reinterpret_cast<const __nv_bfloat162*>(&b));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// One 8-element bf16 vector into online statistics s (and the max raw value).
+__device__ __forceinline__ void stats_vec_bf16(const uint4& q, float c, f32x2 c2, Stats& s,
+                                               float& vmax) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+  const uint32_t mm = bmax2(bmax2(w[0], w[1]), bmax2(w[2], w[3]));
+  const float bmv = fmaxf(__uint_as_float(mm << 16), __uint_as_float(mm & 0xFFFF0000u));
+  vmax = fmaxf(vmax, bmv);
+  const float bm = __fmul_rn(bmv, c);
+  if (bm > s.m) {
+    if (s.c0 != 0.f || s.zr != 0.f) stats_rebase(s, bm);
+    s.m = bm;
+  }
+  if (bm == s.m || !(bm == bm)) {
+    // the vector holds this chain's running maximum (or NaN): scalar, with
+    // the max-valued elements counted apart
+    float u[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      u[2 * i] = __fmul_rn(__uint_as_float(w[i] << 16), c);
+      u[2 * i + 1] = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), c);
+    }
+    stats_add(s, u);
+  } else {
+    const f32x2 m2 = pack2(s.m, s.m);
+    f32x2 zr2 = pack2(0.f, 0.f), a2 = pack2(0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const f32x2 x2 = pack2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+      const f32x2 d2 = sub2(mul2(x2, c2), m2);
+      float d0, d1;
+      unpack2(d2, d0, d1);
+      const f32x2 e2 = pack2(ex2(d0), ex2(d1));
+      zr2 = add2(zr2, e2);
+      a2 = fma2(d2, e2, a2);
+    }
+    float z0, z1, a0, a1;
+    unpack2(zr2, z0, z1);
+    unpack2(a2, a0, a1);
+    s.zr += z0 + z1;
+    s.a += a0 + a1;
   }
 }
 

@@ -29,9 +29,12 @@
 // top-k mass and min-p against the row max, and writes the outputs.
 
 #include <cuda.h>
+#include <cuda_bf16.h>
+#include <cublasLt.h>
 
 #include <climits>
 #include <cmath>
+#include <mutex>
 #include <string>
 
 #include "common.cuh"
@@ -83,6 +86,18 @@ struct LmParams {
   int32_t* ws_id;    // [rows, splits, top_k]
   float* ws_zy;      // [rows] accumulator at the target id
   uint32_t* ws_err;  // [1] bounded-wait timeouts
+  // backward (kModeDz): per-row (c, log-sum-exp in base-2 units, alpha, beta)
+  // of the dense logit gradient p (alpha + beta x), c == 0 for a row with no
+  // gradient; the bf16 gradient tile goes to dz [rows, dz_ld]
+  const float4* rowc;
+  uint16_t* dz;
+  int64_t dz_ld;
+};
+
+// Epilogues of the GEMM kernel.
+enum : int {
+  kModeScore = 0,  // forward: online statistics and top-k candidates
+  kModeDz = 1,     // backward: the dense part of d loss / d (H W^T), bf16
 };
 
 // ---------------------------------------------------------------------------
@@ -280,7 +295,7 @@ __device__ __forceinline__ float pick32(const float (&v)[32], int i) {
   return (i & 16) ? d1 : d0;
 }
 
-template <bool PAIR>
+template <bool PAIR, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     lmhead_gemm_kernel(const __grid_constant__ CUtensorMap map_h,
                        const __grid_constant__ CUtensorMap map_w, LmParams P) {
@@ -434,6 +449,68 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+  } else if constexpr (MODE == kModeDz) {
+    // ------------------------------------------------------------ epilogue (backward)
+    // d loss / d x for each accumulator x of the row: the dense part
+    // p (alpha + beta x), p = 2^(x c - lse); the support and target entries
+    // are rewritten afterwards by the fix-up kernel
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    uint32_t tile = 0;
+    bool ok = true;
+    for (int u = u_first; u < units && ok; u += u_step) {
+      const int mu = u % P.m_units, sp = u / P.m_units;
+      const int mb = PAIR ? 2 * mu + static_cast<int>(rank) : mu;
+      const int t0 = sp * P.tiles_per_split, t1 = min(P.n_tiles, t0 + P.tiles_per_split);
+      const int row = mb * kBM + r;
+      const bool row_ok = row < P.rows;
+      const float4 rc = row_ok ? P.rowc[row] : make_float4(0.f, 0.f, 0.f, 0.f);
+      uint16_t* drow = P.dz + static_cast<int64_t>(row_ok ? row : 0) * P.dz_ld;
+      for (int t = t0; t < t1 && ok; ++t, ++tile) {
+        const int b = tile & 1;
+        const uint32_t use = tile >> 1;
+        if (!wait_or_abort(&bs->tfull[b], use & 1u, bs, P.ws_err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tmem + (uint32_t(q * 32) << 16) + b * kBN;
+        for (int ch = 0; ch < kBN / 32; ++ch) {
+          float v[32];
+          tmem_ld32(taddr + ch * 32, v);
+          if (ch == kBN / 32 - 1) {
+            tc_fence_before();
+            if constexpr (PAIR)
+              mbar_arrive_leader(&bs->tempty[b]);
+            else
+              mbar_arrive(&bs->tempty[b]);
+          }
+          const int col0 = t * kBN + ch * 32;
+          if (!row_ok || col0 >= P.vocab) continue;
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float g0 = 0.f, g1 = 0.f;
+            if (rc.x != 0.f) {
+              g0 = ex2(fmaf(v[2 * i], rc.x, -rc.y)) * fmaf(rc.w, v[2 * i], rc.z);
+              g1 = ex2(fmaf(v[2 * i + 1], rc.x, -rc.y)) * fmaf(rc.w, v[2 * i + 1], rc.z);
+            }
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(g0, g1);
+            pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+          uint16_t* dst = drow + col0;
+          if (col0 + 32 <= P.vocab) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          } else {
+            for (int i = 0; i < 32 && col0 + i < P.vocab; ++i)
+              dst[i] = static_cast<uint16_t>((pk[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu);
+          }
+        }
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
@@ -555,6 +632,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // merge: one thread per row
 
+// Saved per-row state of the fused head for its backward
+// (VS_CTX_BYTES_PER_ROW bytes), base-2 units u = x c, x = (H W^T)[i, v]:
+struct alignas(16) LmCtx {
+  float m;       // max_v u
+  float log2z;   // log2 sum_v 2^(u - m)
+  float ms;      // support sums reference (u of the top-1)
+  float log2zs;  // log2 sum_{v in S} 2^(u - ms)
+  float h_full, h_support;  // nat
+  float c;       // log2(e) / T
+  int32_t n;     // |S| (S = the first n top-k ids)
+  uint32_t flags;  // kLmCtx*
+  uint32_t pad[7];
+};
+static_assert(sizeof(LmCtx) == VS_CTX_BYTES_PER_ROW, "fused-head ctx layout");
+enum : uint32_t {
+  kLmCtxNonFinite = 1u << 0,
+  kLmCtxTargetOk = 1u << 1,
+  kLmCtxTargetInS = 1u << 2,
+};
+
 struct MergeParams {
   int32_t rows, vocab, splits, top_k;
   float top_p, min_p;
@@ -575,6 +672,7 @@ struct MergeParams {
   int32_t* support_size;
   int32_t* topk_ids;
   float* topk_logprob;
+  LmCtx* ctx;
   int32_t want_entropy;
 };
 
@@ -681,13 +779,13 @@ __global__ void __launch_bounds__(128) lmhead_merge_kernel(MergeParams P) {
   const int y = P.targets[row];
   uint32_t status = 0;
   float lp_v = nan, lp_s = nan;
+  bool in_s = false;
   if (y < 0 || y >= P.vocab) status |= VS_ROW_TARGET_OUT_OF_RANGE;
   if (nonfinite) {
     status |= VS_ROW_NONFINITE_INPUT;
   } else if (!(status & VS_ROW_TARGET_OUT_OF_RANGE)) {
     const float uy = __fmul_rn(P.ws_zy[row], c);
     lp_v = kLn2 * (uy - st.m - log2z);
-    bool in_s = false;
     for (int i = 0; i < n; ++i) in_s |= ti[i] == y;
     if (in_s) {
       lp_s = kLn2 * (uy - ss.m - log2zs);
@@ -706,6 +804,23 @@ __global__ void __launch_bounds__(128) lmhead_merge_kernel(MergeParams P) {
   if (P.valid) P.valid[row] = (!nonfinite && n > 0) ? 1 : 0;
   if (P.status) P.status[row] = status;
   if (P.support_size) P.support_size[row] = nonfinite ? 0 : n;
+  if (P.ctx) {
+    LmCtx cx{};
+    cx.m = st.m;
+    cx.log2z = log2z;
+    cx.ms = ss.m;
+    cx.log2zs = log2zs;
+    cx.h_full = h_full;
+    cx.h_support = h_sup;
+    cx.c = c;
+    cx.n = nonfinite ? 0 : n;
+    uint32_t f = 0;
+    if (nonfinite || timeout) f |= kLmCtxNonFinite;
+    if (!(status & VS_ROW_TARGET_OUT_OF_RANGE)) f |= kLmCtxTargetOk;
+    if (in_s) f |= kLmCtxTargetInS;
+    cx.flags = f;
+    P.ctx[row] = cx;
+  }
   for (int i = 0; i < k; ++i) {
     if (P.topk_ids) P.topk_ids[static_cast<int64_t>(row) * k + i] = ti[i];
     if (P.topk_logprob)
@@ -715,6 +830,127 @@ __global__ void __launch_bounds__(128) lmhead_merge_kernel(MergeParams P) {
 }
 
 __global__ void lmhead_clear_kernel(uint32_t* err) { *err = 0u; }
+
+// ---------------------------------------------------------------------------
+// backward (xorl issue #71, section 1: selected logprob + VJP), with respect
+// to x = H W^T (so dz / T for z = x / T):
+//   dx_j = (1/T) ( g_lpV ([j == y] - p_j) + g_lpS 1_S(j) ([j == y] - q_j)
+//                 - g_HV p_j (log p_j + H_V) - g_HS 1_S(j) q_j (log q_j + H_S) )
+// Dense part for every j: p_j (alpha + beta x_j) with
+//   alpha = -(1/T) (g_lpV + g_HV (H_V - LSE)),  beta = -(1/T^2) g_HV;
+// the target and support entries (at most top_k + 1 per row) are rewritten
+// whole by the fix-up kernel.  An empty support folds g_lpS into g_lpV (lp_S
+// is lp_V there); a target outside [0, V) drops the logprob terms; a
+// non-finite row has no gradient.
+
+struct BwdRowParams {
+  int32_t rows, top_k;
+  const LmCtx* ctx;
+  const float* g_lpv;
+  const float* g_lps;
+  const float* g_hv;
+  const float* g_hs;
+  float4* rowc;
+};
+
+__device__ __forceinline__ float gval(const float* g, int row) { return g ? g[row] : 0.f; }
+
+// g_lpV as it enters the row's gradient (see above)
+__device__ __forceinline__ float row_gv(const LmCtx& cx, const float* g_lpv, const float* g_lps,
+                                        int row) {
+  if (!(cx.flags & kLmCtxTargetOk)) return 0.f;
+  return gval(g_lpv, row) + (cx.n == 0 ? gval(g_lps, row) : 0.f);
+}
+
+__global__ void lmhead_bwd_prep_kernel(BwdRowParams P) {
+  const int row = blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= P.rows) return;
+  const LmCtx cx = P.ctx[row];
+  float4 rc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (!(cx.flags & kLmCtxNonFinite)) {
+    const float gv = row_gv(cx, P.g_lpv, P.g_lps, row);
+    const float ghv = gval(P.g_hv, row);
+    const float lse = cx.m + cx.log2z;  // base-2 units
+    const float k = cx.c * kLn2;        // 1 / T
+    rc = make_float4(cx.c, lse, -k * (gv + ghv * (cx.h_full - kLn2 * lse)), -k * ghv * kLn2 * cx.c);
+  }
+  P.rowc[row] = rc;
+}
+
+struct FixParams {
+  int32_t rows, hidden, top_k, c0, c1;  // the vocabulary chunk [c0, c1)
+  const uint16_t* H;
+  int64_t ldh;
+  const uint16_t* W;
+  int64_t ldw;
+  const LmCtx* ctx;
+  const int32_t* targets;
+  const int32_t* topk_ids;
+  const float* g_lpv;
+  const float* g_lps;
+  const float* g_hv;
+  const float* g_hs;
+  const float4* rowc;
+  const uint32_t* err;
+  uint16_t* dz;
+  int64_t dz_ld;
+};
+
+// One CTA per row: the row's support ids and target inside the chunk, each
+// by one warp: x_j = H_i . W_j (bf16 products accumulated in fp32), then the
+// whole gradient entry, rounded to bf16 over the dense value.
+__global__ void __launch_bounds__(128) lmhead_bwd_fix_kernel(FixParams P) {
+  const int row = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint16_t* drow = P.dz + static_cast<int64_t>(row) * P.dz_ld;
+  if (*P.err != 0u) {
+    // a bounded wait of the dense pass gave up: make the failure loud
+    if (threadIdx.x == 0 && P.c1 > P.c0) drow[0] = 0x7FC0u;  // NaN
+    return;
+  }
+  const LmCtx cx = P.ctx[row];
+  if (cx.flags & kLmCtxNonFinite) return;
+  const int n = cx.n;
+  const int y = P.targets[row];
+  const bool yok = cx.flags & kLmCtxTargetOk;
+  const bool yin = cx.flags & kLmCtxTargetInS;
+  const int nid = n + ((yok && !yin) ? 1 : 0);
+  const uint4* h4 = reinterpret_cast<const uint4*>(P.H + static_cast<int64_t>(row) * P.ldh);
+  const int nv = P.hidden / 8;
+  for (int e = warp; e < nid; e += 4) {
+    const int j = e < n ? P.topk_ids[static_cast<int64_t>(row) * P.top_k + e] : y;
+    if (j < P.c0 || j >= P.c1) continue;
+    const uint4* w4 = reinterpret_cast<const uint4*>(P.W + static_cast<int64_t>(j) * P.ldw);
+    float acc = 0.f;
+    for (int v = lane; v < nv; v += 32) {
+      const uint4 a = h4[v], b = w4[v];
+      const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc = fmaf(__uint_as_float(wa[i] << 16), __uint_as_float(wb[i] << 16), acc);
+        acc = fmaf(__uint_as_float(wa[i] & 0xFFFF0000u), __uint_as_float(wb[i] & 0xFFFF0000u), acc);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
+      const float4 rc = P.rowc[row];
+      const float k = cx.c * kLn2;  // 1 / T
+      float g = ex2(fmaf(acc, rc.x, -rc.y)) * fmaf(rc.w, acc, rc.z);
+      if (j == y && yok) g += k * row_gv(cx, P.g_lpv, P.g_lps, row);
+      if (e < n && n > 1) {
+        // a singleton support has q = 1 and H_S = 0: both support terms vanish
+        const float dq = fmaf(acc, cx.c, -(cx.ms + cx.log2zs));  // log2 q_j
+        const float qv = ex2(dq);
+        float sp = gval(P.g_hs, row) * (-qv * fmaf(kLn2, dq, cx.h_support));
+        if (yin) sp += gval(P.g_lps, row) * ((j == y ? 1.f : 0.f) - qv);
+        g += k * sp;
+      }
+      drow[j - P.c0] = __bfloat16_as_ushort(__float2bfloat16_rn(g));
+    }
+  }
+}
+
 
 // ---------------------------------------------------------------------------
 // host side
@@ -805,6 +1041,161 @@ LmLayout lm_layout(int rows, int vocab, int top_k, bool pair) {
   return L;
 }
 
+// Launch shape of the GEMM kernel.  Pair mode (two SMs per 256 x 256 tile,
+// half the operand traffic per SM) when the device schedules clusters of two
+// with this shared memory; otherwise one CTA per 128 x 256 tile.
+struct GemmConfig {
+  bool pair;
+  int stages;
+  size_t smem;
+};
+
+template <int MODE>
+GemmConfig gemm_config(int top_k) {
+  GemmConfig g{};
+  const size_t lists = static_cast<size_t>(kBM) * top_k * 8;
+  const size_t fixed = 1024 + lists + 16 + sizeof(Barriers);
+  int stages2 = static_cast<int>((227 * 1024 - fixed) / kStageBytes2);
+  if (stages2 > kMaxStages) stages2 = kMaxStages;
+  const size_t smem2 = fixed + static_cast<size_t>(stages2) * kStageBytes2;
+  bool pair = stages2 >= 3;
+  if (pair) {
+    cudaError_t e = cudaFuncSetAttribute(lmhead_gemm_kernel<true, MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem2));
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem2;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int nc = 0;
+    if (e != cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&nc, lmhead_gemm_kernel<true, MODE>, &cfg) != cudaSuccess ||
+        nc < 1) {
+      cudaGetLastError();
+      pair = false;
+    }
+  }
+  g.pair = pair;
+  if (pair) {
+    g.stages = stages2;
+    g.smem = smem2;
+  } else {
+    g.stages = top_k <= 24 ? 4 : 3;
+    g.smem = fixed + static_cast<size_t>(g.stages) * kStageBytes;
+  }
+  return g;
+}
+
+template <int MODE>
+cudaError_t gemm_launch(const GemmConfig& g, const CUtensorMap& map_h, const CUtensorMap& map_w,
+                        const LmParams& P, int units, cudaStream_t s) {
+  if (g.pair) {
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    const int workers = num_sms() / 2;
+    cfg.gridDim = dim3(2 * (units < workers ? units : workers), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = g.smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, lmhead_gemm_kernel<true, MODE>, map_h, map_w, P);
+  }
+  cudaError_t e = cudaFuncSetAttribute(lmhead_gemm_kernel<false, MODE>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(g.smem));
+  if (e != cudaSuccess) return e;
+  const int grid = units < num_sms() ? units : num_sms();
+  lmhead_gemm_kernel<false, MODE><<<grid, kThreads, g.smem, s>>>(map_h, map_w, P);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// plain GEMMs of the backward on cuBLASLt (bf16 operands, fp32 accumulation
+// and output), with the caller's workspace
+
+constexpr size_t kLtWorkspace = size_t(32) << 20;
+constexpr int kBwdChunk = 32768;  // vocabulary columns per backward chunk (multiple of kBN)
+
+std::mutex g_lt_mu;
+cublasLtHandle_t g_lt[64] = {};
+
+cublasLtHandle_t lt_handle() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_lt_mu);
+  if (!g_lt[dev] && cublasLtCreate(&g_lt[dev]) != CUBLAS_STATUS_SUCCESS) g_lt[dev] = nullptr;
+  return g_lt[dev];
+}
+
+// Column-major C[m, n] (ldc) = A[m, k] (lda) op(B) + beta C, op(B) = B[k, n]
+// (ldb) or, with transb, the transpose of B[n, k] (ldb).
+bool lt_gemm(bool transb, int64_t m, int64_t n, int64_t k, const void* A, int64_t lda,
+             const void* B, int64_t ldb, float* C, int64_t ldc, float beta, void* ws,
+             size_t ws_bytes, cudaStream_t s) {
+  cublasLtHandle_t h = lt_handle();
+  if (!h) return false;
+  cublasLtMatmulDesc_t op = nullptr;
+  cublasLtMatrixLayout_t la = nullptr, lb = nullptr, lc = nullptr;
+  cublasLtMatmulPreference_t pref = nullptr;
+  bool ok = cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F) == CUBLAS_STATUS_SUCCESS;
+  const cublasOperation_t ta = CUBLAS_OP_N, tb = transb ? CUBLAS_OP_T : CUBLAS_OP_N;
+  ok = ok && cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSA, &ta, sizeof(ta)) ==
+                 CUBLAS_STATUS_SUCCESS;
+  ok = ok && cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSB, &tb, sizeof(tb)) ==
+                 CUBLAS_STATUS_SUCCESS;
+  ok = ok && cublasLtMatrixLayoutCreate(&la, CUDA_R_16BF, m, k, lda) == CUBLAS_STATUS_SUCCESS;
+  ok = ok && cublasLtMatrixLayoutCreate(&lb, CUDA_R_16BF, transb ? n : k, transb ? k : n, ldb) ==
+                 CUBLAS_STATUS_SUCCESS;
+  ok = ok && cublasLtMatrixLayoutCreate(&lc, CUDA_R_32F, m, n, ldc) == CUBLAS_STATUS_SUCCESS;
+  ok = ok && cublasLtMatmulPreferenceCreate(&pref) == CUBLAS_STATUS_SUCCESS;
+  ok = ok && cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES,
+                                                  &ws_bytes, sizeof(ws_bytes)) ==
+                 CUBLAS_STATUS_SUCCESS;
+  cublasLtMatmulHeuristicResult_t res{};
+  int nres = 0;
+  ok = ok && cublasLtMatmulAlgoGetHeuristic(h, op, la, lb, lc, lc, pref, 1, &res, &nres) ==
+                 CUBLAS_STATUS_SUCCESS && nres > 0;
+  const float alpha = 1.f;
+  ok = ok && cublasLtMatmul(h, op, &alpha, A, la, B, lb, &beta, C, lc, C, lc, &res.algo, ws,
+                            ws_bytes, s) == CUBLAS_STATUS_SUCCESS;
+  if (pref) cublasLtMatmulPreferenceDestroy(pref);
+  if (lc) cublasLtMatrixLayoutDestroy(lc);
+  if (lb) cublasLtMatrixLayoutDestroy(lb);
+  if (la) cublasLtMatrixLayoutDestroy(la);
+  if (op) cublasLtMatmulDescDestroy(op);
+  return ok;
+}
+
+struct BwdLayout {
+  int chunk;
+  size_t off_rowc, off_err, off_dz, off_lt, total;
+};
+
+BwdLayout bwd_layout(int rows, int vocab) {
+  BwdLayout L{};
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const int vr = (vocab + kBN - 1) / kBN * kBN;
+  L.chunk = vr < kBwdChunk ? vr : kBwdChunk;
+  L.off_rowc = 0;
+  L.off_err = up(static_cast<size_t>(rows) * sizeof(float4));
+  L.off_dz = up(L.off_err + 16);
+  L.off_lt = up(L.off_dz + static_cast<size_t>(rows) * L.chunk * 2);
+  L.total = L.off_lt + kLtWorkspace;
+  return L;
+}
+
 }  // namespace
 
 size_t lmhead_workspace_bytes(int rows, int vocab, int hidden, int top_k) {
@@ -837,8 +1228,13 @@ vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh
   if (!temperature && !(std::isfinite(temperature_scalar) && temperature_scalar > 0.f))
     return bad(VS_ERR_INVALID_ARG, "temperature_scalar must be finite and > 0");
   if (!out) return bad(VS_ERR_INVALID_ARG, "out is NULL");
-  if (out->sampled || out->support_mask || out->ctx || (flags & VS_WANT_SAMPLE))
-    return bad(VS_ERR_INVALID_ARG, "sampled, support_mask and ctx are not offered by the fused head: pass NULL");
+  if (out->sampled || out->support_mask || (flags & VS_WANT_SAMPLE))
+    return bad(VS_ERR_INVALID_ARG, "sampled and support_mask are not offered by the fused head: pass NULL");
+  const bool want_grad = flags & VS_WANT_GRAD;
+  if (want_grad != (out->ctx != nullptr))
+    return bad(VS_ERR_INVALID_ARG, "VS_WANT_GRAD and ctx go together");
+  if (want_grad && (!topk_ids || !a16(out->ctx)))
+    return bad(VS_ERR_INVALID_ARG, "VS_WANT_GRAD needs topk_ids (the support) and a 16-byte aligned ctx");
   const bool want_entropy = flags & VS_WANT_ENTROPY;
   if (!want_entropy && (out->entropy_full || out->entropy_support))
     return bad(VS_ERR_INVALID_ARG, "entropy outputs need VS_WANT_ENTROPY");
@@ -849,44 +1245,12 @@ vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh
   if (!ws || !a16(ws) || ws_bytes < lmhead_workspace_bytes(rows, vocab, hidden, top_k))
     return bad(VS_ERR_WORKSPACE, "workspace missing, misaligned or smaller than vs_fused_lmhead_workspace_size");
 
-  // Pair mode (two SMs per 256 x 256 tile, half the operand traffic per SM)
-  // when the device schedules clusters of two with this shared memory;
-  // otherwise one CTA per 128 x 256 tile.
-  const size_t lists = static_cast<size_t>(kBM) * top_k * 8;
-  const size_t fixed = 1024 + lists + 16 + sizeof(Barriers);
-  int stages2 = static_cast<int>((227 * 1024 - fixed) / kStageBytes2);
-  if (stages2 > kMaxStages) stages2 = kMaxStages;
-  const size_t smem2 = fixed + static_cast<size_t>(stages2) * kStageBytes2;
-  bool pair = stages2 >= 3;
-  cudaLaunchConfig_t cfg2{};
-  cudaLaunchAttribute attr2[1];
-  if (pair) {
-    cudaError_t e = cudaFuncSetAttribute(lmhead_gemm_kernel<true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem2));
-    attr2[0].id = cudaLaunchAttributeClusterDimension;
-    attr2[0].val.clusterDim.x = 2;
-    attr2[0].val.clusterDim.y = 1;
-    attr2[0].val.clusterDim.z = 1;
-    cfg2.gridDim = dim3(2, 1, 1);
-    cfg2.blockDim = dim3(kThreads, 1, 1);
-    cfg2.dynamicSmemBytes = smem2;
-    cfg2.stream = s;
-    cfg2.attrs = attr2;
-    cfg2.numAttrs = 1;
-    int nc = 0;
-    if (e != cudaSuccess ||
-        cudaOccupancyMaxActiveClusters(&nc, lmhead_gemm_kernel<true>, &cfg2) != cudaSuccess ||
-        nc < 1) {
-      cudaGetLastError();
-      pair = false;
-    }
-  }
-  const LmLayout L = lm_layout(rows, vocab, top_k, pair);
+  const GemmConfig G = gemm_config<kModeScore>(top_k);
+  const LmLayout L = lm_layout(rows, vocab, top_k, G.pair);
 
   CUtensorMap map_h, map_w;
   if (!make_map(&map_h, H, rows, hidden, ldh, kBM) ||
-      !make_map(&map_w, W, vocab, hidden, ldw, pair ? kBNh : kBN))
+      !make_map(&map_w, W, vocab, hidden, ldw, G.pair ? kBNh : kBN))
     return bad(VS_ERR_CUDA, "cuTensorMapEncodeTiled failed");
 
   uint8_t* w8 = static_cast<uint8_t*>(ws);
@@ -900,7 +1264,7 @@ vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh
   P.n_tiles = L.n_tiles;
   P.m_blocks = L.m_blocks;
   P.m_units = L.m_units;
-  P.stages = pair ? stages2 : (top_k <= 24 ? 4 : 3);
+  P.stages = G.stages;
   P.temperature = temperature;
   P.temperature_scalar = temperature_scalar;
   P.targets = targets;
@@ -911,21 +1275,7 @@ vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh
   P.ws_err = reinterpret_cast<uint32_t*>(w8 + L.off_err);
 
   lmhead_clear_kernel<<<1, 1, 0, s>>>(P.ws_err);
-  const int units = L.m_units * L.splits;
-  cudaError_t e;
-  if (pair) {
-    const int workers = num_sms() / 2;
-    cfg2.gridDim = dim3(2 * (units < workers ? units : workers), 1, 1);
-    e = cudaLaunchKernelEx(&cfg2, lmhead_gemm_kernel<true>, map_h, map_w, P);
-  } else {
-    const size_t smem = fixed + static_cast<size_t>(P.stages) * kStageBytes;
-    e = cudaFuncSetAttribute(lmhead_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return bad(VS_ERR_CUDA, cudaGetErrorString(e));
-    const int grid = units < num_sms() ? units : num_sms();
-    lmhead_gemm_kernel<false><<<grid, kThreads, smem, s>>>(map_h, map_w, P);
-    e = cudaGetLastError();
-  }
+  cudaError_t e = gemm_launch<kModeScore>(G, map_h, map_w, P, L.m_units * L.splits, s);
   if (e != cudaSuccess) return bad(VS_ERR_CUDA, cudaGetErrorString(e));
 
   MergeParams M{};
@@ -952,10 +1302,133 @@ vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh
   M.support_size = out->support_size;
   M.topk_ids = topk_ids;
   M.topk_logprob = topk_logprob;
+  M.ctx = want_grad ? static_cast<LmCtx*>(out->ctx) : nullptr;
   M.want_entropy = want_entropy ? 1 : 0;
   lmhead_merge_kernel<<<(rows + 127) / 128, 128, 0, s>>>(M);
   e = cudaGetLastError();
   if (e != cudaSuccess) return bad(VS_ERR_CUDA, cudaGetErrorString(e));
+  return VS_OK;
+}
+
+size_t lmhead_bwd_workspace_bytes(int rows, int vocab, int hidden) {
+  (void)hidden;
+  if (rows <= 0 || vocab <= 0) return 0;
+  return bwd_layout(rows, vocab).total;
+}
+
+vs_status lmhead_bwd_run(int rows, int vocab, int hidden, const void* H, int64_t ldh,
+                         const void* W, int64_t ldw, const int32_t* targets, int top_k,
+                         const void* ctx, const int32_t* topk_ids, const float* g_lp_full,
+                         const float* g_lp_support, const float* g_h_full,
+                         const float* g_h_support, float* d_hidden, int64_t ld_dh,
+                         float* d_weight, int64_t ld_dw, void* ws, size_t ws_bytes,
+                         cudaStream_t s, std::string* err) {
+  auto bad = [&](vs_status code, const char* msg) {
+    *err = msg;
+    return code;
+  };
+  auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (rows < 0) return bad(VS_ERR_INVALID_ARG, "rows must be >= 0");
+  if (vocab < 1) return bad(VS_ERR_INVALID_ARG, "vocab must be >= 1");
+  if (hidden < kBK || hidden % kBK != 0)
+    return bad(VS_ERR_UNSUPPORTED, "hidden_dim must be a positive multiple of 64");
+  if (top_k < 1 || top_k > VS_MAX_FUSED_TOPK || top_k > vocab)
+    return bad(VS_ERR_UNSUPPORTED, "top_k must lie in [1, min(VS_MAX_FUSED_TOPK, vocab)]");
+  if (rows == 0 || (!d_hidden && !d_weight)) return VS_OK;
+  if (!H || !W || !targets || !ctx || !topk_ids)
+    return bad(VS_ERR_INVALID_ARG, "hidden, weight, targets, ctx and topk_ids must be non-NULL");
+  if (!a16(H) || !a16(W) || ldh % 8 != 0 || ldw % 8 != 0 || ldh < hidden || ldw < hidden ||
+      !a16(ctx))
+    return bad(VS_ERR_INVALID_ARG, "hidden/weight must be 16-byte aligned with ld >= hidden_dim, ld % 8 == 0; ctx 16-byte aligned");
+  if ((d_hidden && (ld_dh < hidden || !a16(d_hidden) || ld_dh % 4 != 0)) ||
+      (d_weight && (ld_dw < hidden || !a16(d_weight) || ld_dw % 4 != 0)))
+    return bad(VS_ERR_INVALID_ARG, "d_hidden / d_weight must be 16-byte aligned with ld >= hidden_dim, ld % 4 == 0");
+  const BwdLayout L = bwd_layout(rows, vocab);
+  if (!ws || !a16(ws) || ws_bytes < L.total)
+    return bad(VS_ERR_WORKSPACE, "workspace missing, misaligned or smaller than vs_fused_lmhead_bwd_workspace_size");
+
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  float4* rowc = reinterpret_cast<float4*>(w8 + L.off_rowc);
+  uint32_t* werr = reinterpret_cast<uint32_t*>(w8 + L.off_err);
+  uint16_t* dz = reinterpret_cast<uint16_t*>(w8 + L.off_dz);
+  void* ltws = w8 + L.off_lt;
+  const LmCtx* cx = static_cast<const LmCtx*>(ctx);
+
+  lmhead_clear_kernel<<<1, 1, 0, s>>>(werr);
+  BwdRowParams R{};
+  R.rows = rows;
+  R.top_k = top_k;
+  R.ctx = cx;
+  R.g_lpv = g_lp_full;
+  R.g_lps = g_lp_support;
+  R.g_hv = g_h_full;
+  R.g_hs = g_h_support;
+  R.rowc = rowc;
+  lmhead_bwd_prep_kernel<<<(rows + 127) / 128, 128, 0, s>>>(R);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return bad(VS_ERR_CUDA, cudaGetErrorString(e));
+
+  const GemmConfig G = gemm_config<kModeDz>(0);
+  CUtensorMap map_h;
+  if (!make_map(&map_h, H, rows, hidden, ldh, kBM)) return bad(VS_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  for (int c0 = 0; c0 < vocab; c0 += L.chunk) {
+    const int len = vocab - c0 < L.chunk ? vocab - c0 : L.chunk;
+    const uint16_t* Wc = static_cast<const uint16_t*>(W) + static_cast<int64_t>(c0) * ldw;
+    CUtensorMap map_w;
+    if (!make_map(&map_w, Wc, len, hidden, ldw, G.pair ? kBNh : kBN))
+      return bad(VS_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    const LmLayout LL = lm_layout(rows, len, 0, G.pair);
+    LmParams P{};
+    P.rows = rows;
+    P.vocab = len;
+    P.hidden = hidden;
+    P.top_k = 0;
+    P.splits = LL.splits;
+    P.tiles_per_split = LL.tiles_per_split;
+    P.n_tiles = LL.n_tiles;
+    P.m_blocks = LL.m_blocks;
+    P.m_units = LL.m_units;
+    P.stages = G.stages;
+    P.ws_err = werr;
+    P.rowc = rowc;
+    P.dz = dz;
+    P.dz_ld = L.chunk;
+    e = gemm_launch<kModeDz>(G, map_h, map_w, P, LL.m_units * LL.splits, s);
+    if (e != cudaSuccess) return bad(VS_ERR_CUDA, cudaGetErrorString(e));
+    FixParams F{};
+    F.rows = rows;
+    F.hidden = hidden;
+    F.top_k = top_k;
+    F.c0 = c0;
+    F.c1 = c0 + len;
+    F.H = static_cast<const uint16_t*>(H);
+    F.ldh = ldh;
+    F.W = static_cast<const uint16_t*>(W);
+    F.ldw = ldw;
+    F.ctx = cx;
+    F.targets = targets;
+    F.topk_ids = topk_ids;
+    F.g_lpv = g_lp_full;
+    F.g_lps = g_lp_support;
+    F.g_hv = g_h_full;
+    F.g_hs = g_h_support;
+    F.rowc = rowc;
+    F.err = werr;
+    F.dz = dz;
+    F.dz_ld = L.chunk;
+    lmhead_bwd_fix_kernel<<<rows, 128, 0, s>>>(F);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return bad(VS_ERR_CUDA, cudaGetErrorString(e));
+    // d_hidden (+)= dz_c W_c:  column-major [hidden, rows] = W_c^T [hidden, len] dz_c^T [len, rows]
+    if (d_hidden && !lt_gemm(false, hidden, rows, len, Wc, ldw, dz, L.chunk, d_hidden, ld_dh,
+                             c0 == 0 ? 0.f : 1.f, ltws, kLtWorkspace, s))
+      return bad(VS_ERR_CUDA, "cuBLASLt matmul (d_hidden) failed");
+    // d_weight[c0 : c0 + len] = dz_c^T H:  column-major [hidden, len] = H^T [hidden, rows] dz_c [rows, len]
+    if (d_weight && !lt_gemm(true, hidden, len, rows, H, ldh, dz, L.chunk,
+                             d_weight + static_cast<int64_t>(c0) * ld_dw, ld_dw, 0.f, ltws,
+                             kLtWorkspace, s))
+      return bad(VS_ERR_CUDA, "cuBLASLt matmul (d_weight) failed");
+  }
   return VS_OK;
 }
 

@@ -100,9 +100,6 @@ cudaError_t launch_score_reduce(const float* h_support, const uint8_t* valid, in
 cudaError_t launch_score_bwd(const BwdParams& p, vs_dtype dtype, vs_dtype gdtype, int mode,
                              bool whole_rows, int nchunks, cudaStream_t s);
 
-cudaError_t launch_score_split(const ScoreParams& p, void* ws, cudaStream_t s);
-size_t score_split_workspace_bytes(int rows, int vocab);
-int32_t score_split_max_vocab();
 int score_max_vocab(vs_dtype dtype);
 
 }  // namespace vs

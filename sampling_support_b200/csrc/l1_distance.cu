@@ -44,8 +44,9 @@ struct L1Params {
   float* accept;
   void* grad;
   int64_t grad_ld;
-  double* ws_wsum;  // [1] sum of weights (written by l1_wsum_kernel)
+  double* ws_wsum;  // [1] sum of this call's weights (written by l1_wsum_kernel)
   double* ws_wl1;   // [rows] w_i * L1_i
+  const double* wsum_norm;  // [1] the loss denominator: ws_wsum, or the caller's sum over all shards
   int32_t chunk;
 };
 
@@ -67,12 +68,6 @@ __device__ __forceinline__ float dec_grad(uint32_t w, float coef, float ps) {
   const float p = __uint_as_float(w & 0x3FFFFFFFu);
   const float s = (w & 0x40000000u) ? 0.f : ((w & 0x80000000u) ? -1.f : 1.f);
   return coef * p * (s - ps);
-}
-
-__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
-  const __nv_bfloat162 r = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&a),
-                                   *reinterpret_cast<const __nv_bfloat162*>(&b));
-  return *reinterpret_cast<const uint32_t*>(&r);
 }
 
 __device__ __forceinline__ float l1_block_max(float v, float* scratch) {
@@ -279,7 +274,7 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
 
   // pass 3: d loss / d draft_j = (w / sum w) p_j (s_j - sum_k p_k s_k)
   if (P.grad) {
-    const double wsum = *P.ws_wsum;
+    const double wsum = *P.wsum_norm;
     const float coef = wsum > 0.0 ? static_cast<float>(static_cast<double>(w) / wsum) : 0.f;
     const float k_pos = coef * (1.f - PS), k_neg = coef * (-1.f - PS), k_zero = coef * (-PS);
     G* go = static_cast<G*>(P.grad) + static_cast<int64_t>(row) * P.grad_ld + c0;
@@ -476,7 +471,7 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
 
   // pass 3: d loss / d draft_j = (w / sum w) p_j (s_j - sum_k p_k s_k)
   if (P.grad) {
-    const double wsum = *P.ws_wsum;
+    const double wsum = *P.wsum_norm;
     const float coef = wsum > 0.0 ? static_cast<float>(static_cast<double>(w) / wsum) : 0.f;
     G* go = static_cast<G*>(P.grad) + static_cast<int64_t>(row) * P.grad_ld + c0;
     for (int v = tid; v < nfull; v += blockDim.x) {
@@ -547,8 +542,12 @@ __global__ void l1_wsum_kernel(const float* w, int rows, double* out) {
   }
 }
 
-// loss numerator / denominator / value (one block)
-__global__ void l1_loss_kernel(const double* wl1, const double* wsum, int rows, float* out3) {
+// loss numerator / denominator / value (one block): numerator and
+// denominator over this call's rows; the value divides the numerator by
+// `norm` (this call's denominator, or the sum over all shards, so that the
+// values of the shards add up to the loss of the whole batch)
+__global__ void l1_loss_kernel(const double* wl1, const double* wsum, const double* norm, int rows,
+                               float* out3) {
   __shared__ double red[32];
   double s = 0.0;
   for (int i = threadIdx.x; i < rows; i += blockDim.x) s += wl1[i];
@@ -560,14 +559,19 @@ __global__ void l1_loss_kernel(const double* wl1, const double* wsum, int rows, 
   if (threadIdx.x == 0) {
     double t = 0.0;
     for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) t += red[i];
-    const double den = *wsum;
+    const double den = *wsum, nrm = *norm;
     out3[0] = static_cast<float>(t);
     out3[1] = static_cast<float>(den);
-    out3[2] = den > 0.0 ? static_cast<float>(t / den) : 0.f;
+    out3[2] = nrm > 0.0 ? static_cast<float>(t / nrm) : 0.f;
   }
 }
 
 }  // namespace
+
+cudaError_t launch_l1_weight_sum(int rows, const float* row_weight, double* out, cudaStream_t s) {
+  l1_wsum_kernel<<<1, 1024, 0, s>>>(row_weight, rows, out);
+  return cudaGetLastError();
+}
 
 size_t l1_workspace_bytes(int rows) { return 16 + 8 * static_cast<size_t>(rows > 0 ? rows : 0); }
 
@@ -591,7 +595,7 @@ int l1_max_vocab(vs_dtype dtype) {
 cudaError_t launch_l1(int rows, int vocab, int64_t ld, vs_dtype dtype, const void* draft,
                       const void* target, const float* row_weight, float* l1, float* accept,
                       float* loss3, void* grad, vs_dtype gdtype, int64_t grad_ld, void* ws,
-                      cudaStream_t s) {
+                      const double* global_wsum, cudaStream_t s) {
   int chunk = 0;
   const int cl = l1_cluster_size(vocab, dtype, &chunk);
   L1Params P{};
@@ -609,6 +613,7 @@ cudaError_t launch_l1(int rows, int vocab, int64_t ld, vs_dtype dtype, const voi
   const bool need_ws = loss3 != nullptr || grad != nullptr;
   P.ws_wsum = need_ws ? static_cast<double*>(ws) : nullptr;
   P.ws_wl1 = need_ws ? static_cast<double*>(ws) + 2 : nullptr;
+  P.wsum_norm = global_wsum ? global_wsum : P.ws_wsum;
   if (need_ws) {
     l1_wsum_kernel<<<1, 1024, 0, s>>>(row_weight, rows, P.ws_wsum);
     cudaError_t e = cudaGetLastError();
@@ -647,7 +652,7 @@ cudaError_t launch_l1(int rows, int vocab, int64_t ld, vs_dtype dtype, const voi
 #undef VS_L1_LAUNCH
   if (e != cudaSuccess) return e;
   if (loss3) {
-    l1_loss_kernel<<<1, 1024, 0, s>>>(P.ws_wl1, P.ws_wsum, rows, loss3);
+    l1_loss_kernel<<<1, 1024, 0, s>>>(P.ws_wl1, P.ws_wsum, P.wsum_norm, rows, loss3);
     e = cudaGetLastError();
   }
   return e;

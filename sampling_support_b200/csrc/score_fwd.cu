@@ -23,7 +23,8 @@ namespace {
 // ---------------------------------------------------------------------------
 // recorded support
 
-constexpr int kRecThreads = 128;
+constexpr int kRecThreads = 256;
+constexpr int kRecUnroll = 8;  // 16-byte loads in flight per thread on a full-row stream
 
 template <typename Raw>
 __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams P) {
@@ -121,14 +122,44 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
     const int nfull = V / VEC;
     const uint4* g4 = reinterpret_cast<const uint4*>(grow);
     int v = tid;
-    for (; v + 3 * kRecThreads < nfull; v += 4 * kRecThreads) {
-      uint4 q[4];
+    if constexpr (sizeof(Raw) == 2) {
+      // packed statistics, four chains, kRecUnroll vectors in flight
+      Stats f4[4] = {stats_empty(), stats_empty(), stats_empty(), stats_empty()};
+      const f32x2 c2 = pack2(c, c);
+      for (; v + (kRecUnroll - 1) * kRecThreads < nfull; v += kRecUnroll * kRecThreads) {
+        uint4 q[kRecUnroll];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) q[k] = __ldcs(g4 + v + k * kRecThreads);
+        for (int k = 0; k < kRecUnroll; ++k) q[k] = __ldcs(g4 + v + k * kRecThreads);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < kRecUnroll; ++k) stats_vec_bf16(q[k], c, c2, f4[k & 3], fvmax);
+      }
+      for (; v < nfull; v += kRecThreads) stats_vec_bf16(__ldcs(g4 + v), c, c2, f4[0], fvmax);
+      f = f4[0];
+      stats_merge(f, f4[1]);
+      stats_merge(f, f4[2]);
+      stats_merge(f, f4[3]);
+    } else {
+      for (; v + 3 * kRecThreads < nfull; v += 4 * kRecThreads) {
+        uint4 q[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) q[k] = __ldcs(g4 + v + k * kRecThreads);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          Raw r[VEC];
+          unpack(q[k], r);
+          float u[VEC];
+#pragma unroll
+          for (int i = 0; i < VEC; ++i) {
+            const float x = value_of(r[i]);
+            fvmax = fmaxf(fvmax, x);
+            u[i] = __fmul_rn(x, c);
+          }
+          stats_add(f, u);
+        }
+      }
+      for (; v < nfull; v += kRecThreads) {
         Raw r[VEC];
-        unpack(q[k], r);
+        unpack(__ldcs(g4 + v), r);
         float u[VEC];
 #pragma unroll
         for (int i = 0; i < VEC; ++i) {
@@ -138,18 +169,6 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
         }
         stats_add(f, u);
       }
-    }
-    for (; v < nfull; v += kRecThreads) {
-      Raw r[VEC];
-      unpack(__ldcs(g4 + v), r);
-      float u[VEC];
-#pragma unroll
-      for (int i = 0; i < VEC; ++i) {
-        const float x = value_of(r[i]);
-        fvmax = fmaxf(fvmax, x);
-        u[i] = __fmul_rn(x, c);
-      }
-      stats_add(f, u);
     }
     for (int j = nfull * VEC + tid; j < V; j += kRecThreads) {
       const float x = value_of(grow[j]);
@@ -309,11 +328,11 @@ __global__ void score_reduce_kernel(const float* h_support, const uint8_t* valid
 
 }  // namespace
 
-// Rows are streamed, so the vocabulary is bounded only by the index types.
-// bf16 rows go to the split kernel (bounded chunk count); fp32 rows stream
-// through one CTA each and have no structural limit below 2^26.
+// Rows are streamed through one CTA each, so the vocabulary is bounded only
+// by the index types (kept below 2^26).
 int score_max_vocab(vs_dtype dtype) {
-  return dtype == VS_BF16 ? score_split_max_vocab() : (1 << 26);
+  (void)dtype;
+  return 1 << 26;
 }
 
 cudaError_t launch_score_recorded(const ScoreParams& p, vs_dtype dtype, cudaStream_t s) {

@@ -2,26 +2,33 @@
 // inclusive top-p -> min-p against the original row max; xorl issue #71,
 // section 3), one CTA per row.
 //
-// The row is streamed through a ring of shared-memory stages filled by bulk
-// asynchronous copies (one elected thread issues them; every warp releases a
-// stage after use):
-//   pass 1 (HBM)  online max / count of max / sum 2^(u - max) /
-//                 sum (u - max) 2^(u - max)   (u = z log2 e), and the row max;
-//   pass 2 (L2)   bf16 rows with a filter: histogram of the EXACT 16-bit keys
-//                 in a window of at most 4,096 keys at and below the row max
-//                 (each bin holds one value, so its mass is count x 2^(u-m));
-//                 the k-th element and the top-p crossing are found by block
-//                 scans of the bins, the support sums by a block reduction;
-//   pass 3 (L2)   only when the support ends inside a tie group: an ordered
-//                 count of that group's elements finds the id of the last one
-//                 kept (ties go to the lower token id);
-//   pass 4 (L2)   only when the support bitmask is requested;
-//   pass 5 (L2)   only when a sample is requested: a seeded Gumbel-max token
-//                 over the support (noise recipe in gumbel.cuh).
-// fp32 rows, and bf16 rows whose crossing lies below the window, fall back to
-// an 8-bit radix descent over all keys (one streamed pass per digit).
-// Everything is block-local (no cluster barriers), deterministic, and each
-// row's logits are read from HBM once.
+// The row is streamed once from HBM through a ring of shared-memory stages
+// filled by bulk asynchronous copies (one elected thread issues them; every
+// warp releases a stage after use).  In that one pass each element updates
+//   * the online statistics: max, count of max-valued elements,
+//     sum 2^(u - max), sum (u - max) 2^(u - max)   (u = z log2 e), and
+//   * for a filtered bf16 row, a shared-memory histogram of the EXACT 16-bit
+//     keys in a window of at most 4,096 keys.  The window is fixed once the
+//     first stage has arrived: its top lies kWinHi keys above that stage's
+//     maximum (a lower bound of the row maximum), and, without top-k, its
+//     floor is the first key that can still matter (min-p: 2^(u - m) >=
+//     min_p / 2; top-p: 2^(u - m) >= (1 - p) / (4 V), below which all
+//     elements together hold under a quarter of the 1 - p tail).  Each bin
+//     holds one value, so its mass is count x 2^(u - m).
+// After the pass the k-th element and the top-p crossing are found by block
+// scans of the bins and the support sums come from the bins; nothing is read
+// again.  A row whose maximum lies above the window, or whose decision lies
+// below it, falls back to passes that re-read the row (an 8-bit radix
+// descent; fp32 rows always take it, exact-key windows do not apply to
+// 32-bit keys).  Further passes re-read the row only on request:
+//   * the id of the last kept element of the threshold's tie group (ties go
+//     to the lower token id), for the saved state, the bitmask or a sample;
+//     without those only the target's membership is needed, and when the
+//     target sits in a partly kept tie group the ties before it are counted
+//     on the shorter side of it;
+//   * the support bitmask;
+//   * a seeded Gumbel-max token over the support (noise recipe in gumbel.cuh).
+// Everything is block-local (no cluster barriers) and deterministic.
 
 #include <climits>
 
@@ -38,10 +45,19 @@ namespace {
 
 constexpr int kRT = 512;        // threads per row
 constexpr int kRW = kRT / 32;   // warps
-constexpr int kNStages = 4;     // ring depth
+constexpr int kNStages = 6;     // ring depth
 constexpr int kStageBytes = 32768;
 constexpr int kWin = kSelWin;
 constexpr int kBins = kSelBins;
+constexpr uint32_t kWinHi = 256;  // window keys above the first stage's maximum
+constexpr int kCountUnroll = 8;   // 16-byte loads in flight per thread (tie count)
+
+// Support sums: counts above the threshold, of its tie group and of the
+// max-valued elements; mass and (u - m)-weighted mass of the others.
+struct SupSums {
+  uint32_t ngt, neq, ntp;
+  float smass, sa;
+};
 
 struct RowSh {
   uint64_t full[kNStages];
@@ -51,12 +67,21 @@ struct RowSh {
   uint32_t ured[kRW];
   u64 ulred[kRW];
   SelShared<kRW> sel;
+  SupSums sums[kRW];
   uint32_t outstanding;  // loads issued and not yet consumed (broadcast by thread 0)
   int32_t tie_cut;
   uint32_t timeout;
   unsigned long long kred[kRW];
   uint32_t squeue[kRW][64];  // sampling: per-warp queue of member groups (index | bits << 28)
 };
+
+// Programmatic dependent launch (PTX griddepcontrol): the next kernel on the
+// stream may be scheduled once every CTA of this grid has signalled; a grid
+// waits for the preceding one (and its memory) before touching memory.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // streaming ring
@@ -128,66 +153,37 @@ struct Ring {
 
 enum WinMode : int { kWinNone = 0, kWinPos = 1, kWinNeg = 2, kWinKey = 3 };
 
-// bin of a raw bf16 (as fp32 bits F) or nbins when outside the window
-__device__ __forceinline__ uint32_t win_bin(const Window& w, uint32_t F) {
-  uint32_t b;
-  if (w.mode == kWinPos) {
-    b = (F - w.fconst) >> 16;
-    if ((F - w.fconst) >= (static_cast<uint32_t>(w.nbins) << 16)) b = w.nbins;
-  } else if (w.mode == kWinNeg) {
-    b = (w.fconst - F) >> 16;
-    if ((w.fconst - F) >= (static_cast<uint32_t>(w.nbins) << 16)) b = w.nbins;
-  } else {
-    b = key_of(static_cast<uint16_t>(F >> 16)) - w.klo;
-    if (b >= static_cast<uint32_t>(w.nbins)) b = w.nbins;
-  }
-  return b;
+// Window index of the raw bf16 bits r (>= the bin count outside the window).
+// kWinPos (every window key is a positive value): base = raw bits of the
+// lowest window key, and negative values wrap to huge indices; kWinNeg
+// (every window key is a negative value): base = raw bits of the lowest
+// window key (the most negative value); kWinKey: base = lowest window key.
+template <int MODE>
+__device__ __forceinline__ uint32_t win_index(uint32_t r, uint32_t base) {
+  if constexpr (MODE == kWinPos)
+    return r - base;
+  else if constexpr (MODE == kWinNeg)
+    return base - r;
+  else
+    return key_of(static_cast<uint16_t>(r)) - base;
 }
 
-// Count the in-window elements of one vector: collected as a bit mask and
-// counted with as few shared atomics as the busiest lane of the warp needs.
-// Uniform call (every lane of the warp).
-__device__ __forceinline__ void win_vec(const Window& w, const uint4& q, bool valid) {
-  uint32_t bins[8];
-  uint32_t pend = 0;
-  const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
+// One shared-memory count increment at the 32-bit shared address a.
+__device__ __forceinline__ void red_inc(uint32_t a) {
+  asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(a) : "memory");
+}
+
+// Count the eight elements of one vector: in-window elements into their bin,
+// the others into this lane's spill bin (bins >= the window's bin count are
+// never read), so there is no predicate or branch.
+template <int MODE>
+__device__ __forceinline__ void hist_vec(const uint4& q, uint32_t base, uint32_t spill,
+                                         uint32_t hist_s) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    bins[2 * i] = win_bin(w, wd[i] << 16);
-    bins[2 * i + 1] = win_bin(w, wd[i] & 0xFFFF0000u);
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    if (valid && bins[i] < static_cast<uint32_t>(w.nbins)) pend |= 1u << i;
-  while (__any_sync(0xffffffffu, pend != 0)) {
-    if (pend) {
-      const int i = __ffs(pend) - 1;
-      uint32_t b = bins[0];
-#pragma unroll
-      for (int k = 1; k < 8; ++k)
-        if (i == k) b = bins[k];
-      atomicAdd(&w.hist[b], 1u);
-      pend &= pend - 1;
-    }
-  }
-}
-
-// Histogram of one stage (four vectors per thread in flight).
-__device__ void win_stage(const Window& w, const uint16_t* st, int n) {
-  const int nv = n / 8;
-  const uint4* v4 = reinterpret_cast<const uint4*>(st);
-  const int rounds = (nv + 4 * kRT - 1) / (4 * kRT);
-  for (int r = 0; r < rounds; ++r) {
-    const int v0 = r * 4 * kRT + threadIdx.x;
-    uint4 q[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) q[k] = v0 + k * kRT < nv ? v4[v0 + k * kRT] : make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) win_vec(w, q[k], v0 + k * kRT < nv);
-  }
-  for (int j = nv * 8 + threadIdx.x; j < n; j += kRT) {
-    const uint32_t b = win_bin(w, static_cast<uint32_t>(st[j]) << 16);
-    if (b < static_cast<uint32_t>(w.nbins)) atomicAdd(&w.hist[b], 1u);
+    red_inc(hist_s + (min(win_index<MODE>(w[i] & 0xFFFFu, base), spill) << 2));
+    red_inc(hist_s + (min(win_index<MODE>(w[i] >> 16, base), spill) << 2));
   }
 }
 
@@ -275,58 +271,14 @@ __device__ Desc descend(Ring<Raw>& ring, float c, float m, int fx_shift, bool by
 }
 
 // ---------------------------------------------------------------------------
-// pass 1 helpers
+// the streamed pass
 
-// One 8-element bf16 vector into online statistics s (and the max raw value).
-__device__ __forceinline__ void stats_vec_bf16(const uint4& q, float c, f32x2 c2, Stats& s,
-                                               float& vmax) {
-  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-  const __nv_bfloat162 m01 = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&w[0]),
-                                     *reinterpret_cast<const __nv_bfloat162*>(&w[1]));
-  const __nv_bfloat162 m23 = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&w[2]),
-                                     *reinterpret_cast<const __nv_bfloat162*>(&w[3]));
-  const __nv_bfloat162 mm = __hmax2(m01, m23);
-  const float bmv = fmaxf(__low2float(mm), __high2float(mm));
-  vmax = fmaxf(vmax, bmv);
-  const float bm = __fmul_rn(bmv, c);
-  if (bm > s.m) {
-    if (s.c0 != 0.f || s.zr != 0.f) stats_rebase(s, bm);
-    s.m = bm;
-  }
-  if (bm == s.m || !(bm == bm)) {
-    // the vector holds this chain's running maximum (or NaN): scalar, with
-    // the max-valued elements counted apart
-    float u[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      u[2 * i] = __fmul_rn(__uint_as_float(w[i] << 16), c);
-      u[2 * i + 1] = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), c);
-    }
-    stats_add(s, u);
-  } else {
-    const f32x2 m2 = pack2(s.m, s.m);
-    f32x2 zr2 = pack2(0.f, 0.f), a2 = pack2(0.f, 0.f);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const f32x2 x2 = pack2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
-      const f32x2 d2 = sub2(mul2(x2, c2), m2);
-      float d0, d1;
-      unpack2(d2, d0, d1);
-      const f32x2 e2 = pack2(ex2(d0), ex2(d1));
-      zr2 = add2(zr2, e2);
-      a2 = fma2(d2, e2, a2);
-    }
-    float z0, z1, a0, a1;
-    unpack2(zr2, z0, z1);
-    unpack2(a2, a0, a1);
-    s.zr += z0 + z1;
-    s.a += a0 + a1;
-  }
-}
-
-// bf16 stage: four vectors per thread in flight, each with its own chain.
-__device__ __forceinline__ void stats_stage_bf16(const uint16_t* st, int n, float c, Stats (&s)[4],
-                                                 float& vmax) {
+// bf16 stage: statistics (four vectors per thread in flight, each with its
+// own chain) and, unless MODE is kWinNone, the window histogram.
+template <int MODE>
+__device__ __forceinline__ void stage_bf16(const uint16_t* st, int n, float c, Stats (&s)[4],
+                                           float& vmax, uint32_t base, uint32_t spill,
+                                           uint32_t hist_s) {
   const int nv = n / 8;
   const uint4* v4 = reinterpret_cast<const uint4*>(st);
   const f32x2 c2 = pack2(c, c);
@@ -336,14 +288,23 @@ __device__ __forceinline__ void stats_stage_bf16(const uint16_t* st, int n, floa
 #pragma unroll
     for (int k = 0; k < 4; ++k) q[k] = v4[v + k * kRT];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) stats_vec_bf16(q[k], c, c2, s[k], vmax);
+    for (int k = 0; k < 4; ++k) {
+      stats_vec_bf16(q[k], c, c2, s[k], vmax);
+      if constexpr (MODE != kWinNone) hist_vec<MODE>(q[k], base, spill, hist_s);
+    }
   }
-  for (; v < nv; v += kRT) stats_vec_bf16(v4[v], c, c2, s[0], vmax);
+  for (; v < nv; v += kRT) {
+    const uint4 q = v4[v];
+    stats_vec_bf16(q, c, c2, s[0], vmax);
+    if constexpr (MODE != kWinNone) hist_vec<MODE>(q, base, spill, hist_s);
+  }
   for (int j = nv * 8 + threadIdx.x; j < n; j += kRT) {
-    const float x = value_of(st[j]);
+    const uint32_t r = st[j];
+    const float x = value_of(static_cast<uint16_t>(r));
     vmax = fmaxf(vmax, x);
     float u[1] = {__fmul_rn(x, c)};
     stats_add(s[0], u);
+    if constexpr (MODE != kWinNone) red_inc(hist_s + (min(win_index<MODE>(r, base), spill) << 2));
   }
 }
 
@@ -372,6 +333,100 @@ __device__ __forceinline__ void stats_stage_f32(const uint32_t* st, int n, float
   }
 }
 
+__device__ __forceinline__ float block_max(float v, float* scratch) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float t = -kInf;
+  for (int w = 0; w < kRW; ++w) t = fmaxf(t, scratch[w]);
+  __syncthreads();
+  return t;
+}
+
+// Maximum value of one bf16 stage over the block.
+__device__ __forceinline__ float stage_max_bf16(const uint16_t* st, int n, float* scratch) {
+  const int nv = n / 8;
+  const uint4* v4 = reinterpret_cast<const uint4*>(st);
+  uint32_t mx = 0xFF80FF80u;  // (-inf, -inf)
+  for (int v = threadIdx.x; v < nv; v += kRT) {
+    const uint4 q = v4[v];
+    mx = bmax2(mx, bmax2(bmax2(q.x, q.y), bmax2(q.z, q.w)));
+  }
+  float m = fmaxf(__uint_as_float(mx << 16), __uint_as_float(mx & 0xFFFF0000u));
+  for (int j = nv * 8 + threadIdx.x; j < n; j += kRT) m = fmaxf(m, value_of(st[j]));
+  return block_max(m, scratch);
+}
+
+// Smallest key in [lo, hi] whose u-offset from m reaches dlo (hi if none).
+__device__ __forceinline__ uint32_t key_at_level(uint32_t lo, uint32_t hi, float c, float m,
+                                                 float dlo) {
+  while (lo < hi) {
+    const uint32_t mid = lo + ((hi - lo) >> 1);
+    if (key_u(mid, c) - m >= dlo)
+      hi = mid;
+    else
+      lo = mid + 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ SupSums block_sum_sup(SupSums v, RowSh& sh) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    v.ngt += __shfl_xor_sync(0xffffffffu, v.ngt, o);
+    v.neq += __shfl_xor_sync(0xffffffffu, v.neq, o);
+    v.ntp += __shfl_xor_sync(0xffffffffu, v.ntp, o);
+    v.smass += __shfl_xor_sync(0xffffffffu, v.smass, o);
+    v.sa += __shfl_xor_sync(0xffffffffu, v.sa, o);
+  }
+  if ((threadIdx.x & 31) == 0) sh.sums[threadIdx.x >> 5] = v;
+  __syncthreads();
+  SupSums t{0u, 0u, 0u, 0.f, 0.f};
+  for (int w = 0; w < kRW; ++w) {
+    t.ngt += sh.sums[w].ngt;
+    t.neq += sh.sums[w].neq;
+    t.ntp += sh.sums[w].ntp;
+    t.smass += sh.sums[w].smass;
+    t.sa += sh.sums[w].sa;
+  }
+  __syncthreads();
+  return t;
+}
+
+// Number of elements of g[j0, j1) whose raw bits are r0 or r1 (the two
+// encodings of one key), read from global memory by the block with
+// kCountUnroll 16-byte loads in flight per thread; j0 need not be a multiple
+// of 8.  Result in thread 0 only after the caller's block sum.
+__device__ __forceinline__ uint32_t count_raw(const uint16_t* g, int j0, int j1, uint32_t r0,
+                                              uint32_t r1) {
+  uint32_t n = 0;
+  auto one = [&](uint32_t r) { n += (r == r0) | (r == r1) ? 1u : 0u; };
+  auto vec = [&](const uint4& q) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      one(w[i] & 0xFFFFu);
+      one(w[i] >> 16);
+    }
+  };
+  const int ja = min(j1, (j0 + 7) & ~7);
+  for (int j = j0 + static_cast<int>(threadIdx.x); j < ja; j += kRT) one(g[j]);
+  const int nv = (j1 - ja) >> 3;
+  const uint4* v4 = reinterpret_cast<const uint4*>(g + ja);
+  int v = threadIdx.x;
+  for (; v + (kCountUnroll - 1) * kRT < nv; v += kCountUnroll * kRT) {
+    uint4 q[kCountUnroll];
+#pragma unroll
+    for (int k = 0; k < kCountUnroll; ++k) q[k] = __ldcg(v4 + v + k * kRT);
+#pragma unroll
+    for (int k = 0; k < kCountUnroll; ++k) vec(q[k]);
+  }
+  for (; v < nv; v += kRT) vec(__ldcg(v4 + v));
+  for (int j = ja + nv * 8 + static_cast<int>(threadIdx.x); j < j1; j += kRT) one(g[j]);
+  return n;
+}
+
 // ---------------------------------------------------------------------------
 
 template <typename Raw>
@@ -383,7 +438,7 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
   Raw* ringbuf = reinterpret_cast<Raw*>(smem_raw);
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw + kNStages * kStageBytes);
   RadixArrays& ra = *reinterpret_cast<RadixArrays*>(hist);
-  RowSh& sh = *reinterpret_cast<RowSh*>(smem_raw + kNStages * kStageBytes + kWin * 4);
+  RowSh& sh = *reinterpret_cast<RowSh*>(smem_raw + kNStages * kStageBytes + (kWin + 32) * 4);
 
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
@@ -399,6 +454,11 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
     sh.tie_cut = INT_MAX;
     fence_barrier_init();
   }
+  // launched programmatically after whatever kernel precedes it on the
+  // stream: wait for that grid (and its memory) before reading anything;
+  // the next kernel may be scheduled from here on
+  pdl_wait();
+  pdl_launch_dependents();
   __syncthreads();
   Ring<Raw> ring{grow, V, ringbuf, &sh, 0u, 0u};
 
@@ -411,15 +471,62 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
   const bool use_p = pp < 1.f;
   const bool use_minp = mp > 0.f;
   const bool any_filter = use_k || use_p || use_minp;
+  const int y = P.targets[row];
+  const bool target_ok = y >= 0 && y < V;
+  const Raw ry = target_ok ? grow[y] : Raw(0);
 
-  // ---- pass 1 (HBM): online statistics and the row maximum
+  // ---- the streamed pass: online statistics and the row maximum; for a
+  // filtered bf16 row also the exact-key window histogram
   Stats s4[4] = {stats_empty(), stats_empty(), stats_empty(), stats_empty()};
   float vmax = -kInf;
-  ring.pass(0, ring.nst(), [&](const Raw* st, int n, int) {
-    if constexpr (kBf16)
-      stats_stage_bf16(st, n, c, s4, vmax);
-    else
+  const bool hist_on = kBf16 && any_filter;
+  uint32_t wtop = 0, wlo = 0;  // window keys [wlo, wtop]
+  int wmode = kWinNone;
+  uint32_t wbase = 0;
+  const uint32_t hist_s = smem_addr(hist);
+  ring.pass(0, ring.nst(), [&](const Raw* st, int n, int base) {
+    if constexpr (kBf16) {
+      const uint16_t* st16 = reinterpret_cast<const uint16_t*>(st);
+      if (hist_on && base == 0) {
+        // fix the window from the first stage's maximum (a lower bound of
+        // the row maximum m): elements below the level found with it are
+        // below the level of m as well
+        const float m0 = stage_max_bf16(st16, n, sh.fred);
+        const uint32_t kref = key_of(static_cast<uint16_t>(__float_as_uint(m0) >> 16));
+        wtop = min(kref + kWinHi, KT::kInfKey);
+        wlo = wtop >= static_cast<uint32_t>(kWin - 1) ? wtop - (kWin - 1) : 0u;
+        if (!use_k && isfinite(m0)) {
+          float dlo = -kInf;
+          if (use_minp) dlo = log2f(mp) - 1.f;
+          if (use_p && pp > 0.f) dlo = fmaxf(dlo, log2f((1.f - pp) / static_cast<float>(V)) - 2.f);
+          if (dlo > -kInf) wlo = key_at_level(wlo, wtop, c, __fmul_rn(m0, c), dlo);
+        }
+        if (wlo > 0x7FFFu) {
+          wmode = kWinPos;
+          wbase = wlo - 0x7FFFu;
+        } else if (wtop < 0x7FFFu) {
+          wmode = kWinNeg;
+          wbase = 0xFFFFu - wlo;
+        } else {
+          wmode = kWinKey;
+          wbase = wlo;
+        }
+        const int nb = static_cast<int>(wtop - wlo) + 1;
+        for (int b = tid; b < nb; b += kRT) hist[b] = 0u;
+        __syncthreads();
+      }
+      const uint32_t spill = (wtop - wlo) + 1u + (tid & 31);
+      if (wmode == kWinPos)
+        stage_bf16<kWinPos>(st16, n, c, s4, vmax, wbase, spill, hist_s);
+      else if (wmode == kWinNeg)
+        stage_bf16<kWinNeg>(st16, n, c, s4, vmax, wbase, spill, hist_s);
+      else if (wmode == kWinKey)
+        stage_bf16<kWinKey>(st16, n, c, s4, vmax, wbase, spill, hist_s);
+      else
+        stage_bf16<kWinNone>(st16, n, c, s4, vmax, 0u, 0u, 0u);
+    } else {
       stats_stage_f32(st, n, c, s4, vmax);
+    }
     return false;
   });
   Stats s = s4[0];
@@ -427,22 +534,20 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
   stats_merge(s, s4[2]);
   stats_merge(s, s4[3]);
   s = block_reduce(s, sh.wst);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-  if ((tid & 31) == 0) sh.fred[tid >> 5] = vmax;
-  __syncthreads();
-  vmax = -kInf;
-  for (int w = 0; w < kRW; ++w) vmax = fmaxf(vmax, sh.fred[w]);
-  __syncthreads();
+  vmax = block_max(vmax, sh.fred);
 
   const bool nonfinite = !stats_finite(s) || !isfinite(vmax);
   const float m = s.m;  // = fl(vmax c)
   const float log2z = stats_log2z(s);
   const float h_full = kLn2 * (log2z - s.a / stats_z(s));
   const bool filtered = !nonfinite && any_filter;
+  const bool want_cut = P.ctx != nullptr || P.support_mask != nullptr || P.sampled != nullptr;
 
   uint32_t tkey = 0;
   int32_t tie_cut = INT_MAX;
+  bool cut_known = true;  // tie_cut resolved (or not needed: every tie kept)
+  u64 ckeep = 0;
+  u64 tie_group = 0;  // elements holding the threshold key
   float log2zs = log2z, h_support = h_full, c0s = s.c0, zrs = s.zr;
   int32_t n_support = nonfinite ? 0 : V;
 
@@ -451,53 +556,21 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
     bool all_ties = true;
     u64 cnum = 0;
     bool have_t = false;
-    // ---- pass 2 (L2): exact-key window (bf16)
     Window w{};
+    // the window holds every key at or above its floor only when the row
+    // maximum lies inside it
     bool win_ok = false;
     if constexpr (kBf16) {
-      const uint32_t hmax = __float_as_uint(vmax) >> 16;
-      w.kmax = key_of(static_cast<uint16_t>(hmax));
-      uint32_t klo = w.kmax >= static_cast<uint32_t>(kWin - 1) ? w.kmax - (kWin - 1) : 0u;
-      if (use_p && !use_k && !use_minp && pp > 0.f) {
-        // top-p alone: elements with 2^(u - m) < (1 - p) / (2 V) cannot be in
-        // the support (together they hold less than (1 - p) of the mass, the
-        // row total being at least 1); start the window at the first key
-        // above that level
-        const float dcut = log2f((1.f - pp) / static_cast<float>(V)) - 1.f;
-        uint32_t lo = klo, hi = w.kmax;
-        while (lo < hi) {
-          const uint32_t mid = lo + ((hi - lo) >> 1);
-          if (key_u(mid, c) - m >= dcut)
-            hi = mid;
-          else
-            lo = mid + 1;
-        }
-        klo = lo;
-      }
-      w.klo = klo;
-      w.nbins = static_cast<int>(w.kmax - klo) + 1;
+      const uint32_t kmr = key_of(static_cast<uint16_t>(__float_as_uint(vmax) >> 16));
+      w.kmax = wtop;
+      w.klo = wlo;
+      w.nbins = static_cast<int>(wtop - wlo) + 1;
       w.hist = hist;
       w.c = c;
       w.m = m;
       w.fxs = fxs;
-      if (klo > 0x7FFFu && (w.kmax - 0x7FFFu) < 0x7000u) {
-        w.mode = kWinPos;  // positive nonzero keys below 2^97
-        w.fconst = (klo - 0x7FFFu) << 16;
-      } else if (w.kmax < 0x7FFFu) {
-        w.mode = kWinNeg;  // negative nonzero keys (every value is negative)
-        w.fconst = (0xFFFFu - klo) << 16;
-      } else {
-        w.mode = kWinKey;
-        w.fconst = 0;
-      }
-      for (int b = tid; b < w.nbins; b += kRT) hist[b] = 0u;
-      __syncthreads();
-      ring.pass(0, ring.nst(), [&](const Raw* st, int n, int) {
-        win_stage(w, reinterpret_cast<const uint16_t*>(st), n);
-        return false;
-      });
-      win_ok = true;
-      if (use_k || use_p) {
+      win_ok = kmr <= wtop;
+      if (win_ok && (use_k || use_p)) {
         Desc dk{}, dp{};
         u64 ck = 0;
         if (use_k) {
@@ -528,10 +601,19 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
             have_t = true;
           }
         }
+        if (!win_ok && use_p && !use_k && use_minp && kmr <= wtop &&
+            minp_key<Raw>(mp, c, m) >= w.klo) {
+          // the top-p crossing lies below the window, whose floor is at or
+          // below the min-p level: min-p decides the support (applied below)
+          win_ok = true;
+          have_t = false;
+          all_ties = true;
+        }
       }
     }
     if (!win_ok && (use_k || use_p)) {
-      // ---- general radix descent (fp32 keys, or the crossing lies below the window)
+      // ---- general radix descent (fp32 keys, or the decision lies outside
+      // the window)
       have_t = false;
       all_ties = true;
       if (use_k) {
@@ -571,48 +653,44 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
     }
 
     // ---- support sums: keys above tkey (max-valued elements counted apart)
-    // and the tie group at tkey
-    uint32_t ngt = 0, neq = 0, ntop = 0;
-    float smass = 0.f, sa = 0.f;
-    bool sums_done = false;
-    if constexpr (kBf16) {
-      if (win_ok && tkey >= w.klo) {
-        const int per = (w.nbins + kRT - 1) / kRT;
-        const int i0 = tid * per, i1 = min(w.nbins, i0 + per);
-        for (int i = i0; i < i1; ++i) {
-          const uint32_t cnt = hist[i];
-          const uint32_t key = w.klo + i;
-          if (cnt && key > tkey) {
-            const float d = key_u(key, c) - m;
-            const float e = ex2(d);
-            const float fc = static_cast<float>(cnt);
-            ngt += cnt;
-            if (d == 0.f)
-              ntop += cnt;
-            else
-              smass = fmaf(fc, e, smass);
-            sa = fmaf(fc * d, e, sa);
-          }
+    // and the tie group at tkey; from the bins when the window holds them
+    SupSums sums{0u, 0u, 0u, 0.f, 0.f};
+    bool from_bins = false;
+    if constexpr (kBf16) from_bins = win_ok && tkey >= w.klo;
+    if (from_bins) {
+      const int per = (w.nbins + kRT - 1) / kRT;
+      const int i0 = tid * per, i1 = min(w.nbins, i0 + per);
+      for (int i = i0; i < i1; ++i) {
+        const uint32_t cnt = hist[i];
+        const uint32_t key = w.klo + i;
+        if (cnt && key > tkey) {
+          const float d = key_u(key, c) - m;
+          const float e = ex2(d);
+          const float fc = static_cast<float>(cnt);
+          sums.ngt += cnt;
+          if (d == 0.f)
+            sums.ntp += cnt;
+          else
+            sums.smass = fmaf(fc, e, sums.smass);
+          sums.sa = fmaf(fc * d, e, sums.sa);
         }
-        if (tid == 0) neq = hist[tkey - w.klo];
-        sums_done = true;
       }
-    }
-    if (!sums_done) {
+      if (tid == 0) sums.neq = hist[tkey - w.klo];
+    } else {
       const uint32_t t = tkey;
       auto one = [&](Raw raw) {
         const uint32_t key = key_of(raw);
         if (key > t) {
           const float d = __fmul_rn(value_of(raw), c) - m;
           const float e = ex2(d);
-          ++ngt;
+          ++sums.ngt;
           if (d == 0.f)
-            ++ntop;
+            ++sums.ntp;
           else
-            smass += e;
-          sa = fmaf(d, e, sa);
+            sums.smass += e;
+          sums.sa = fmaf(d, e, sums.sa);
         } else if (key == t) {
-          ++neq;
+          ++sums.neq;
         }
       };
       ring.pass(0, ring.nst(), [&](const Raw* st, int n, int) {
@@ -628,78 +706,95 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
         return false;
       });
     }
-    ngt = block_sum(ngt, sh.ured);
-    neq = block_sum(neq, sh.ured);
-    ntop = block_sum(ntop, sh.ured);
-    smass = block_sum(smass, sh.fred);
-    sa = block_sum(sa, sh.fred);
-    const u64 tot_eq = neq;
-    const u64 ckeep = all_ties ? tot_eq : (cnum < tot_eq ? cnum : tot_eq);
+    sums = block_sum_sup(sums, sh);
+    const u64 tot_eq = sums.neq;
+    tie_group = tot_eq;
+    ckeep = all_ties ? tot_eq : (cnum < tot_eq ? cnum : tot_eq);
     const float dt = __fmul_rn(KT::decode(tkey), c) - m;
     const float et = ex2(dt);
     Stats ss;
     ss.m = m;
-    ss.c0 = static_cast<float>(ntop) + (dt == 0.f ? static_cast<float>(ckeep) : 0.f);
-    ss.zr = smass + (dt == 0.f ? 0.f : static_cast<float>(ckeep) * et);
-    ss.a = sa + static_cast<float>(ckeep) * dt * et;
+    ss.c0 = static_cast<float>(sums.ntp) + (dt == 0.f ? static_cast<float>(ckeep) : 0.f);
+    ss.zr = sums.smass + (dt == 0.f ? 0.f : static_cast<float>(ckeep) * et);
+    ss.a = sums.sa + static_cast<float>(ckeep) * dt * et;
     log2zs = stats_log2z(ss);
     h_support = kLn2 * (log2zs - ss.a / stats_z(ss));
     c0s = ss.c0;
     zrs = ss.zr;
-    n_support = static_cast<int32_t>(ngt + ckeep);
+    n_support = static_cast<int32_t>(sums.ngt + ckeep);
 
-    // ---- pass 3 (L2): id of the last tie kept (ascending id order)
+    // ---- id of the last tie kept (ascending id order), when the saved
+    // state, the bitmask or a sample needs it (fp32 rows: always)
     if (ckeep < tot_eq) {
-      const int need = static_cast<int>(ckeep);
-      const uint32_t t = tkey;
-      int seen = 0;  // ties in earlier stages (uniform)
-      ring.pass(0, ring.nst(), [&](const Raw* st, int n, int base) {
-        // thread tid owns the contiguous elements [j0, j1) of this stage
-        const int per = ((n + kRT - 1) / kRT + VEC - 1) / VEC * VEC;
-        const int j0 = min(n, tid * per), j1 = min(n, j0 + per);
-        int mine = 0;
-        int j = j0;
-        const uint4* v4 = reinterpret_cast<const uint4*>(st);
-        for (; j + 4 * VEC <= j1; j += 4 * VEC) {
-          uint4 q[4];
+      cut_known = false;
+      if (want_cut || !kBf16) {
+        const int need = static_cast<int>(ckeep);
+        const uint32_t t = tkey;
+        int seen = 0;  // ties in earlier stages (uniform)
+        ring.pass(0, ring.nst(), [&](const Raw* st, int n, int base) {
+          // thread tid owns the contiguous elements [j0, j1) of this stage
+          const int per = ((n + kRT - 1) / kRT + VEC - 1) / VEC * VEC;
+          const int j0 = min(n, tid * per), j1 = min(n, j0 + per);
+          int mine = 0;
+          int j = j0;
+          const uint4* v4 = reinterpret_cast<const uint4*>(st);
+          for (; j + 4 * VEC <= j1; j += 4 * VEC) {
+            uint4 q[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) q[k] = v4[j / VEC + k];
+            for (int k = 0; k < 4; ++k) q[k] = v4[j / VEC + k];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
+            for (int k = 0; k < 4; ++k) {
+              Raw r[VEC];
+              unpack(q[k], r);
+#pragma unroll
+              for (int i = 0; i < VEC; ++i) mine += key_of(r[i]) == t;
+            }
+          }
+          for (; j + VEC <= j1; j += VEC) {
             Raw r[VEC];
-            unpack(q[k], r);
+            unpack(v4[j / VEC], r);
 #pragma unroll
             for (int i = 0; i < VEC; ++i) mine += key_of(r[i]) == t;
           }
-        }
-        for (; j + VEC <= j1; j += VEC) {
-          Raw r[VEC];
-          unpack(v4[j / VEC], r);
-#pragma unroll
-          for (int i = 0; i < VEC; ++i) mine += key_of(r[i]) == t;
-        }
-        for (; j < j1; ++j) mine += key_of(st[j]) == t;
-        int total;
-        const int excl = seen + block_excl_int<kRT>(mine, total, sh.sel);
-        if (excl < need && need <= excl + mine) {
-          int cn = excl;
-          for (int jj = j0; jj < j1; ++jj)
-            if (key_of(st[jj]) == t && ++cn == need) {
-              sh.tie_cut = base + jj;
-              break;
-            }
-        }
-        seen += total;
-        return seen >= need;
-      });
-      tie_cut = sh.tie_cut;
+          for (; j < j1; ++j) mine += key_of(st[j]) == t;
+          int total;
+          const int excl = seen + block_excl_int<kRT>(mine, total, sh.sel);
+          if (excl < need && need <= excl + mine) {
+            int cn = excl;
+            for (int jj = j0; jj < j1; ++jj)
+              if (key_of(st[jj]) == t && ++cn == need) {
+                sh.tie_cut = base + jj;
+                break;
+              }
+          }
+          seen += total;
+          return seen >= need;
+        });
+        tie_cut = sh.tie_cut;
+        cut_known = true;
+      }
+    }
+  }
+
+  // ---- the target's earlier ties, when its membership hinges on them (bf16
+  // rows; fp32 rows always resolve the cut above when it is needed)
+  uint32_t ylt = 0;
+  if (filtered && !cut_known && target_ok && key_of(ry) == tkey) {
+    if constexpr (kBf16) {
+      // counted on the shorter side of y: after y, the group less the target
+      // and the ties that follow it
+      const uint32_t r0 = tkey >= 0x7FFFu ? tkey - 0x7FFFu : 0xFFFFu - tkey;
+      const uint32_t r1 = tkey == 0x7FFFu ? 0x8000u : r0;  // -0 shares the key of +0
+      const uint16_t* g16 = reinterpret_cast<const uint16_t*>(grow);
+      const bool before = y <= V - 1 - y;
+      const uint32_t part = before ? count_raw(g16, 0, y, r0, r1) : count_raw(g16, y + 1, V, r0, r1);
+      const uint32_t n = block_sum(part, sh.ured);
+      ylt = before ? n : static_cast<uint32_t>(tie_group) - 1u - n;
     }
   }
 
   // ---- per-row outputs
   if (tid == 0) {
-    const int y = P.targets[row];
-    const bool target_ok = y >= 0 && y < V;
     uint32_t status = 0;
     float lp_v = __int_as_float(0x7fc00000), lp_s = __int_as_float(0x7fc00000);
     bool in_s = false;
@@ -707,14 +802,13 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
     if (nonfinite) {
       status |= VS_ROW_NONFINITE_INPUT;
     } else if (target_ok) {
-      const Raw ry = grow[y];
       const float uy = __fmul_rn(value_of(ry), c);
       lp_v = kLn2 * (uy - m - log2z);
       if (!filtered) {
         in_s = true;
       } else {
         const uint32_t ky = key_of(ry);
-        in_s = ky > tkey || (ky == tkey && y <= tie_cut);
+        in_s = ky > tkey || (ky == tkey && (cut_known ? y <= tie_cut : ylt < ckeep));
       }
       if (in_s) {
         lp_s = filtered ? kLn2 * (uy - m - log2zs) : lp_v;
@@ -762,7 +856,7 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
     }
   }
 
-  // ---- pass 4 (L2): support bitmask, one 32-id word per thread and stage
+  // ---- support bitmask, one 32-id word per thread and stage
   if (P.support_mask) {
     const int64_t wstride = (V + 31) / 32;
     uint32_t* mrow = P.support_mask + static_cast<int64_t>(row) * wstride;
@@ -785,11 +879,11 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
     });
   }
 
-  // ---- pass 5 (L2): seeded Gumbel-max token over the support.  Tokens go
-  // in groups of four (stages start on multiples of four); each warp queues
-  // its groups that hold a member and drains the queue 32 groups at a time
-  // (and at the end of each stage), so the Philox block and the logarithms
-  // run on full warps and only for members.
+  // ---- seeded Gumbel-max token over the support.  Tokens go in groups of
+  // four (stages start on multiples of four); each warp queues its groups
+  // that hold a member and drains the queue 32 groups at a time (and at the
+  // end of each stage), so the Philox block and the logarithms run on full
+  // warps and only for members.
   if (P.sampled) {
     unsigned long long best = 0ull;
     if (!nonfinite) {
@@ -847,28 +941,48 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
   }
 }
 
-}  // namespace
-
 size_t score_row_smem_bytes() {
-  return static_cast<size_t>(kNStages) * kStageBytes + kWin * 4 + ((sizeof(RowSh) + 127) & ~size_t(127));
+  return static_cast<size_t>(kNStages) * kStageBytes + (kWin + 32) * 4 +
+         ((sizeof(RowSh) + 127) & ~size_t(127));
 }
 
-cudaError_t launch_score_computed(const ScoreParams& p, vs_dtype dtype, cudaStream_t s) {
-  const size_t smem = score_row_smem_bytes();
-  if (dtype == VS_BF16) {
-    cudaError_t e = cudaFuncSetAttribute(score_row_kernel<uint16_t>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    score_row_kernel<uint16_t><<<p.rows, kRT, smem, s>>>(p);
-  } else {
-    cudaError_t e = cudaFuncSetAttribute(score_row_kernel<uint32_t>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    score_row_kernel<uint32_t><<<p.rows, kRT, smem, s>>>(p);
-  }
+// The dynamic shared-memory opt-in of a kernel, set once per device.
+template <typename K>
+cudaError_t ensure_smem(K kernel, int which) {
+  static bool done[2][64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && done[which][dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(score_row_smem_bytes()));
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[which][dev] = true;
+  return e;
+}
+
+template <typename Raw>
+cudaError_t launch_row(const ScoreParams& p, cudaStream_t s, int which) {
+  cudaError_t e = ensure_smem(score_row_kernel<Raw>, which);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(p.rows);
+  cfg.blockDim = dim3(kRT);
+  cfg.dynamicSmemBytes = score_row_smem_bytes();
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, score_row_kernel<Raw>, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_score_computed(const ScoreParams& p, vs_dtype dtype, cudaStream_t s) {
+  return dtype == VS_BF16 ? launch_row<uint16_t>(p, s, 0) : launch_row<uint32_t>(p, s, 1);
 }
 
 }  // namespace vs

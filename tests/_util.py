@@ -8,10 +8,14 @@ row's largest magnitude.
 
 Top-p and min-p decide set membership from floating-point sums.  Rows whose
 oracle crossing lies within 1e-6 of top_p (or whose min-p ratio lies within
-1e-6 relative of min_p) are counted as boundary rows: for them the GPU's
-support must still be a prefix of the oracle's total order whose mass is
-within the band, and its scores must equal the oracle's scores of that
-support.
+1e-6 relative of min_p) are counted as boundary rows.  For them the GPU's
+support size n must name a prefix of the oracle's total order that the rules
+allow within that band (boundary_prefix_ok: the first n - 1 entries hold
+less than top_p + 1e-6 of the top-k mass; the n-th entry passes min-p within
+the band; the prefix stops because it reached top_p - 1e-6, min-p drops the
+next entry within the band, or it is the whole top-k set), the support mask
+(when requested) must be exactly that prefix, and the scores and status must
+equal the oracle's scores of that prefix.
 """
 
 from __future__ import annotations
@@ -74,10 +78,31 @@ def assert_close_rel(got, want, rtol, what):
     assert rel.size == 0 or rel.max() <= rtol, f"{what}: max rel {rel.max():.3g}"
 
 
+def boundary_prefix_ok(n, facts, top_p, min_p, band=BAND):
+    """True when a support of the first n entries of the total order is one
+    the top-k / top-p / min-p rules allow with the top-p mass and the min-p
+    ratio each known only to within `band` (facts: oracle.prefix of n)."""
+    nk = int(facts["nk"])
+    if n < 1 or n > nk:
+        return False
+    use_p, use_m = top_p < 1.0, min_p > 0.0
+    if use_p and not facts["mass_prev"] < top_p + band:
+        return False
+    if use_m and not facts["ratio_n"] >= min_p * (1.0 - band):
+        return False
+    return bool(n == nk or (use_p and facts["mass_n"] >= top_p - band)
+                or (use_m and facts["ratio_next"] < min_p * (1.0 + band)))
+
+
+def _per_row(v, rows, dt):
+    return np.broadcast_to(np.asarray(v, dt), (rows,))
+
+
 def compare_scores(out, ref, logits, vocab, temperature, targets, top_k, top_p, min_p,
                    check_full=True, check_entropy=True):
-    """Compare a vs_score_fwd result with the oracle; returns the number of
-    boundary rows."""
+    """Compare a vs_score_fwd result with the oracle, every row: exactly off
+    the boundary band, by the prefix rule on it.  Returns (boundary rows,
+    boundary rows whose support size differs from the oracle's)."""
     rows = len(ref["lp_full"])
     band = (ref["topp_margin"] < BAND) | (ref["minp_margin"] < BAND)
     gsize = out["support_size"].cpu().numpy()
@@ -109,25 +134,39 @@ def compare_scores(out, ref, logits, vocab, temperature, targets, top_k, top_p, 
     if check_entropy:
         ok = np.isfinite(ref["h_support"]) & sure
         assert_close_rel(hs[ok], ref["h_support"][ok], H_RTOL, "h_support")
-    # boundary rows: the GPU support is a valid prefix of the total order
-    if band.any():
-        assert mask is not None, "boundary rows need the mask to be checked"
-        z = _z(logits, vocab, temperature)
-        for i in np.nonzero(band)[0]:
-            order = np.lexsort((np.arange(vocab), -z[i]))
-            n = int(gsize[i])
-            assert mask[i].sum() == n
-            assert np.all(mask[i][order[:n]] == 1), "boundary row support is not a prefix"
-            assert abs(n - ref["support_size"][i]) <= max(4, ref["support_size"][i] // 100)
-            ids = np.nonzero(mask[i])[0].astype(np.int32)[None, :]
-            t_i = float(np.broadcast_to(np.asarray(temperature, np.float64), (rows,))[i])
-            r2 = oracle.score(logits[i:i + 1], targets[i:i + 1], temperature=t_i, support=ids,
-                              vocab=vocab)
-            if np.isfinite(r2["lp_support"][0]):
-                assert abs(lps[i] - r2["lp_support"][0]) <= LP_ATOL
-            if check_entropy:
-                assert_close_rel(hs[i:i + 1], r2["h_support"], H_RTOL, "h_support (boundary)")
-    return int(band.sum())
+    # boundary rows: the GPU support is a prefix the rules allow within the band
+    idx = np.nonzero(band)[0]
+    if idx.size == 0:
+        return 0, 0
+    t_all = _per_row(temperature, rows, np.float64)
+    k_all = _per_row(top_k, rows, np.int32)
+    p_all = _per_row(np.asarray(top_p, np.float32).astype(np.float64), rows, np.float64)
+    m_all = _per_row(np.asarray(min_p, np.float32).astype(np.float64), rows, np.float64)
+    facts = oracle.prefix(logits[idx], gsize[idx], temperature=np.ascontiguousarray(t_all[idx]),
+                          top_k=np.ascontiguousarray(k_all[idx]), vocab=vocab, want_ids=True)
+    differ = 0
+    for a, i in enumerate(idx):
+        n = int(gsize[i])
+        f = {k: v[a] for k, v in facts.items() if k != "ids"}
+        assert boundary_prefix_ok(n, f, p_all[i], m_all[i]), (
+            f"row {i}: support size {n} is not a prefix the rules allow (oracle "
+            f"{ref['support_size'][i]}, mass {f['mass_prev']:.9f}..{f['mass_n']:.9f}, "
+            f"top_p {p_all[i]}, min_p {m_all[i]})")
+        differ += int(n != ref["support_size"][i])
+        ids = facts["ids"][a]
+        if mask is not None:
+            assert mask[i].sum() == n and np.all(mask[i][ids] == 1), \
+                "boundary row mask is not the prefix"
+        r2 = oracle.score(logits[i:i + 1], targets[i:i + 1], temperature=float(t_all[i]),
+                          support=ids[None, :], vocab=vocab)
+        assert status[i] == map_status(r2["status"])[0], f"row {i}: status (boundary)"
+        if np.isfinite(r2["lp_support"][0]):
+            assert abs(lps[i] - r2["lp_support"][0]) <= LP_ATOL, f"row {i}: lp_S (boundary)"
+        else:
+            assert lps[i] == r2["lp_support"][0], f"row {i}: lp_S (boundary)"
+        if check_entropy:
+            assert_close_rel(hs[i:i + 1], r2["h_support"], H_RTOL, "h_support (boundary)")
+    return int(idx.size), differ
 
 
 def compare_grad(g_gpu, g_ref, exclude=None, rtol=G_RTOL, what="grad"):

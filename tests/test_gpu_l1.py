@@ -40,10 +40,11 @@ def _check(draft, target, weight, grad_dtype=torch.float32, sample=None):
     assert_close_rel(loss[1:2], [ref["loss_den"]], 1e-6, "loss denominator")
     assert_close_rel(loss[2:], [ref["loss"]], 1e-4, "loss")
     sel = np.arange(rows) if sample is None else sample
-    # gradient rows: oracle on the selected rows, rescaled to the full weight sum
+    # gradient rows: oracle on the selected rows, normalised by the full weight sum
     ws = np.ones(rows) if weight is None else weight.astype(np.float64)
-    gref = oracle.l1(draft[sel], target[sel], weight=ws[sel], want_grad=True)
-    gref_g = gref["grad"] * (ws[sel].sum() / ws.sum())
+    gref = oracle.l1(draft[sel], target[sel], weight=ws[sel], want_grad=True,
+                     global_wsum=float(ws.sum()))
+    gref_g = gref["grad"]
     near = np.abs(_probs(draft[sel]) - _probs(target[sel])) < 1e-6
     g = out["grad"][torch.from_numpy(sel).cuda()].float().cpu().numpy()[:, :vocab]
     compare_grad(g, gref_g, exclude=near,
@@ -107,6 +108,41 @@ def test_l1_unweighted_and_zero_weights():
 def test_distance_workload_full_size():
     w = workloads.distance()
     rng = np.random.default_rng(0)
-    sel = np.sort(rng.choice(w["rows"], 48, replace=False))
+    sel = np.sort(rng.choice(w["rows"], 160, replace=False))
     out = _check(w["draft"], w["target"], w["weight"], grad_dtype=torch.bfloat16, sample=sel)
     assert out["grad"].dtype == torch.bfloat16
+
+
+def test_l1_sharded_rows_take_the_global_denominator():
+    """A batch split into three uneven row shards, each scored by
+    vs_l1_distance_sharded with the weight sum over all shards (each shard's
+    vs_l1_weight_sum, added on the device as an all-reduce would): the
+    concatenated gradients equal the oracle's on the whole batch, the loss
+    contributions add up to its loss, and the numerators and denominators
+    to its numerator and denominator."""
+    w = workloads.distance(rows=24, vocab=20_011, seed=12)
+    rows, vocab = 24, 20_011
+    ld = (vocab + 7) // 8 * 8
+    d, t = to_device(_pad(w["draft"], ld)), to_device(_pad(w["target"], ld))
+    wt = torch.from_numpy(w["weight"]).cuda()
+    cuts = [0, 5, 17, 24]
+    parts = [vsb.l1_weight_sum(cuts[i + 1] - cuts[i], wt[cuts[i]:cuts[i + 1]]) for i in range(3)]
+    wsum = parts[0] + parts[1] + parts[2]
+    outs = [vsb.l1_distance(d[cuts[i]:cuts[i + 1]], t[cuts[i]:cuts[i + 1]], wt[cuts[i]:cuts[i + 1]],
+                            want_loss=True, want_grad=True, vocab=vocab, global_weight_sum=wsum)
+            for i in range(3)]
+    torch.cuda.synchronize()
+    ref = oracle.l1(w["draft"], w["target"], weight=w["weight"].astype(np.float64), want_grad=True)
+    assert abs(wsum.item() - w["weight"].astype(np.float64).sum()) <= 1e-12 * wsum.item()
+    g = np.concatenate([o["grad"].cpu().numpy()[:, :vocab] for o in outs])
+    near = np.abs(_probs(w["draft"]) - _probs(w["target"])) < 1e-6
+    compare_grad(g, ref["grad"], exclude=near)
+    loss = np.stack([o["loss"].cpu().numpy().astype(np.float64) for o in outs])
+    assert_close_rel([loss[:, 2].sum()], [ref["loss"]], 1e-4, "loss (sum of contributions)")
+    assert_close_rel([loss[:, 0].sum()], [ref["loss_num"]], 1e-4, "numerator")
+    assert_close_rel([loss[:, 1].sum()], [ref["loss_den"]], 1e-6, "denominator")
+    # the unsharded call on the whole batch agrees element by element
+    full = vsb.l1_distance(d, t, wt, want_loss=True, want_grad=True, vocab=vocab)
+    torch.cuda.synchronize()
+    gf = full["grad"].cpu().numpy()[:, :vocab]
+    assert np.abs(g - gf).max() <= 1e-6 * np.abs(gf).max()

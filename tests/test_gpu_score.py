@@ -132,6 +132,33 @@ def test_window_crossing_zero_and_huge_values(scale, shift):
         _run(logits, np.arange(rows, dtype=np.int32), temp, *filt)
 
 
+@pytest.mark.parametrize("spike", [8.0, 1000.0])
+def test_row_max_after_the_first_stage(spike):
+    # the exact-key window is fixed from the first streamed stage's maximum;
+    # a row maximum far above it (1000) lies outside the window and the row
+    # falls back to the radix descent, a near one (8) lands in the keys kept
+    # above that maximum
+    rows, vocab = 4, 100_000
+    x = workloads.normal((rows, vocab), 1.0, seed=31, stream=1)
+    x[:, 90_000] = spike
+    x[1, 99_999] = spike / 2
+    logits = workloads.to_bf16_bits(x)
+    t = np.full(rows, 0.8 if spike < 100 else 300.0, F32)
+    for filt in [(0, 0.9, 0.0), (20, 0.95, 0.0), (0, 1.0, 0.05), (0, 0.7, 0.02)]:
+        _run(logits, np.array([90_000, 3, 99_999, 17], np.int32), t, *filt)
+        _run_nomask(logits, np.array([90_000, 3, 99_999, 17], np.int32), t, *filt)
+
+
+@pytest.mark.parametrize("filt", FILTERS)
+def test_ragged_rows_all_filters_without_mask(filt):
+    rows, vocab = 6, 50_021
+    ld = (vocab + 7) // 8 * 8
+    logits = workloads.random_logits(rows, vocab, 3.0, seed=13, dtype="bf16", ld=ld)
+    temp = workloads.uniform(rows, 0.6, 1.2, 13, 7).astype(F32)
+    targets = workloads.integers(rows, 0, vocab, 13, 8).astype(np.int32)
+    _run_nomask(logits[:, :vocab].copy(), targets, temp, *filt)
+
+
 def test_all_negative_rows():
     rows, vocab = 5, 30_000
     x = workloads.normal((rows, vocab), 3.0, seed=12, stream=1) - 60.0
@@ -171,9 +198,10 @@ def test_zero_rows():
 @pytest.mark.slow
 def test_fullvocab_workload_full_size():
     w = workloads.fullvocab()
-    out, ref, nb = _run(w["logits"], w["targets"], w["temperature"], w["top_k"], w["top_p"],
-                        w["min_p"])
-    print(f"fullvocab: {nb} of {w['rows']} rows within 1e-6 of the top-p boundary")
+    out, ref, (nb, nd) = _run(w["logits"], w["targets"], w["temperature"], w["top_k"], w["top_p"],
+                              w["min_p"])
+    print(f"fullvocab: {nb} of {w['rows']} rows within 1e-6 of the top-p boundary, "
+          f"{nd} of them with a support size other than the oracle's")
 
 
 def test_entropy_sum_and_valid_count():
@@ -298,7 +326,7 @@ def test_backward_computed_support(dtype, filt):
     # targets: inside the support for some rows, outside for others
     targets = np.array([np.nonzero(fw["mask"][i])[0][-1] if i % 2 == 0 else (i * 997) % vocab
                         for i in range(rows)], np.int32)
-    out, ref, nb = _run(logits, targets, temp, *filt, vocab=vocab, want_grad=True)
+    out, ref, (nb, _) = _run(logits, targets, temp, *filt, vocab=vocab, want_grad=True)
     assert nb == 0
     g = _grads(rows)
     gt = [torch.from_numpy(x).cuda() for x in g]
@@ -401,29 +429,25 @@ def test_replay_backward_full_size_sampled_rows():
 def _run_nomask(logits, targets, temperature, top_k, top_p, min_p):
     """GPU forward as a caller with no support mask and no saved state asks
     for it (the tie cut at the threshold is then resolved for the target
-    alone), against the oracle; rows off the top-p / min-p boundary band."""
+    alone), against the oracle on every row: logprobs and entropies over the
+    full vocabulary and over the support; boundary rows by the prefix rule
+    (the support rebuilt from the GPU's support size)."""
     rows, vocab = logits.shape
     t_np = np.asarray(temperature, F32)
     k_arg = torch.from_numpy(np.asarray(top_k, np.int32)).cuda() if np.ndim(top_k) else top_k
     out = vsb.score_fwd(to_device(logits), torch.from_numpy(np.asarray(targets, np.int32)).cuda(),
                         temperature=torch.from_numpy(t_np).cuda() if t_np.ndim else float(t_np),
-                        top_k=k_arg, top_p=float(F32(top_p)), min_p=float(F32(min_p)))
+                        top_k=k_arg, top_p=float(F32(top_p)), min_p=float(F32(min_p)),
+                        want_entropy=True)
     torch.cuda.synchronize()
     t64 = t_np.astype(np.float64)
     ref = oracle.score(logits, targets, temperature=t64 if t64.ndim else float(t64),
                        top_k=np.asarray(top_k, np.int32) if np.ndim(top_k) else top_k,
                        top_p=float(F32(top_p)), min_p=float(F32(min_p)))
+    nb, nd = compare_scores(out, ref, logits, vocab, t64 if t64.ndim else np.full(rows, float(t64)),
+                            np.asarray(targets, np.int32), top_k, top_p, min_p)
     sure = ~((ref["topp_margin"] < 1e-6) | (ref["minp_margin"] < 1e-6))
-    get = {k: v.cpu().numpy() for k, v in out.items()}
-    assert np.array_equal(get["valid"], ref["valid"])
-    assert np.array_equal(get["support_size"][sure], ref["support_size"][sure])
-    assert np.array_equal(get["status"][sure].astype(np.int64), map_status(ref["status"][sure]))
-    lps = get["lp_support"].astype(np.float64)[sure]
-    want = ref["lp_support"][sure]
-    assert np.array_equal(lps == -np.inf, want == -np.inf)
-    fin = np.isfinite(want)
-    assert np.abs(lps[fin] - want[fin]).max(initial=0) <= 1e-4
-    return ref, sure
+    return ref, sure, nb, nd
 
 
 def test_target_in_threshold_tie_group_without_mask():
@@ -445,7 +469,7 @@ def test_target_in_threshold_tie_group_without_mask():
         top_k[i] = H + c
         targets[i] = [grp[c - 1], grp[c], grp[-1], grp[0], grp[c - 1], grp[c], grp[-1], hi[0]][i]
     logits = workloads.to_bf16_bits(x)
-    ref, sure = _run_nomask(logits, targets, 1.0, top_k, 1.0, 0.0)
+    ref, sure, _, _ = _run_nomask(logits, targets, 1.0, top_k, 1.0, 0.0)
     assert sure.all()
     kept = np.isfinite(ref["lp_support"])
     assert kept.tolist() == [True, False, False, True, True, False, False, True]
@@ -456,6 +480,7 @@ def test_fullvocab_workload_full_size_without_mask():
     """The fullvocab workload (128 x 151,936 bf16, top-p 0.95) exactly as the
     benchmark calls it: no support mask, no saved state."""
     w = workloads.fullvocab()
-    ref, sure = _run_nomask(w["logits"], w["targets"], w["temperature"], w["top_k"], w["top_p"],
-                            w["min_p"])
-    print(f"fullvocab without mask: {int((~sure).sum())} boundary rows skipped")
+    ref, sure, nb, nd = _run_nomask(w["logits"], w["targets"], w["temperature"], w["top_k"],
+                                    w["top_p"], w["min_p"])
+    print(f"fullvocab without mask: {nb} boundary rows checked by the prefix rule, "
+          f"{nd} of them with a support size other than the oracle's")

@@ -59,3 +59,89 @@ def test_two_rank_weak_scaling_host_logic():
     assert out[0][2] == pytest.approx(4 * 2 / 2e-3)
     # ranks score different batches
     assert out[0][3] != out[1][3] and out[0][0] != out[1][0]
+
+
+class _OracleOps:
+    """The per-rank steps of sampling_support_b200.dist run by the oracle on
+    the CPU (the library needs a GPU; this checks the cross-rank protocol:
+    which scalars are reduced, and that the gradient takes the global
+    denominator)."""
+
+    @staticmethod
+    def weight_sum(rows, row_weight, device):
+        import torch
+
+        w = np.ones(rows) if row_weight is None else row_weight.numpy().astype(np.float64)
+        return torch.tensor([float(np.sum(w))], dtype=torch.float64)
+
+    @staticmethod
+    def l1_distance(draft, target, row_weight, global_weight_sum, want_grad, grad_dtype):
+        import torch
+
+        import oracle
+
+        w = None if row_weight is None else row_weight.numpy().astype(np.float64)
+        r = oracle.l1(draft.numpy(), target.numpy(), w, want_grad=want_grad,
+                      global_wsum=float(global_weight_sum.item()))
+        out = {"l1": torch.from_numpy(r["l1"]),
+               "loss": torch.tensor([r["loss_num"], r["loss_den"], r["loss"]], dtype=torch.float64)}
+        if want_grad:
+            out["grad"] = torch.from_numpy(r["grad"])
+        return out
+
+
+def _sharded_worker(rank, world, port, out):
+    sys.path.insert(0, str(ROOT))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+
+    import torch
+
+    import workloads
+    from sampling_support_b200 import dist as vdist
+
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        d = workloads.random_logits(10, 700, 2.0, seed=41)
+        t = workloads.random_logits(10, 700, 2.0, seed=42)
+        w = workloads.uniform(10, 0.0, 1.0, 41, 3).astype(np.float32)
+        cut = [0, 3, 10]  # uneven shards
+        s = slice(cut[rank], cut[rank + 1])
+        r = vdist.sharded_l1_distance(torch.from_numpy(d[s].copy()), torch.from_numpy(t[s].copy()),
+                                      torch.from_numpy(w[s].copy()), want_grad=True,
+                                      ops=_OracleOps)
+        ent = vdist.sharded_entropy_mean(torch.tensor([1.5 + rank], dtype=torch.float64),
+                                         torch.tensor([2 + rank], dtype=torch.int32))
+        out[rank] = (r["grad"].numpy(), float(r["loss_global"].item()),
+                     float(r["num_global"].item()), float(r["den_global"].item()),
+                     float(ent.item()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_sharded_distance_loss_and_gradient():
+    """A distance batch split unevenly over two gloo ranks: the concatenated
+    gradients and the reduced loss equal the single-process oracle's on the
+    whole batch (gradient normalised by the global weight sum)."""
+    sys.path.insert(0, str(ROOT))
+    import oracle
+    import workloads
+
+    world = 2
+    port = _free_port()
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.start_processes(_sharded_worker, args=(world, port, out), nprocs=world, join=True,
+                       start_method="spawn")
+    d = workloads.random_logits(10, 700, 2.0, seed=41)
+    t = workloads.random_logits(10, 700, 2.0, seed=42)
+    w = workloads.uniform(10, 0.0, 1.0, 41, 3).astype(np.float32)
+    ref = oracle.l1(d, t, w.astype(np.float64), want_grad=True)
+    g = np.concatenate([out[0][0], out[1][0]])
+    assert np.abs(g - ref["grad"]).max() <= 1e-12 * np.abs(ref["grad"]).max()
+    for r in (0, 1):
+        assert out[r][1] == pytest.approx(ref["loss"], rel=1e-12)
+        assert out[r][2] == pytest.approx(ref["loss_num"], rel=1e-12)
+        assert out[r][3] == pytest.approx(ref["loss_den"], rel=1e-12)
+        assert out[r][4] == pytest.approx((1.5 + 2.5) / (2 + 3))

@@ -31,6 +31,8 @@ def _logits(vals):
     for v in vals:
         if isinstance(v, str) and v.startswith("log:"):
             out.append(math.log(float(v[4:])))
+        elif isinstance(v, str) and v.startswith("expr:"):
+            out.append(_eval(v[5:]))
         else:
             out.append(float(v))
     return np.array(out, dtype=np.float64)
@@ -499,3 +501,67 @@ def test_gumbel_sample_edge_cases():
     # and re-running is deterministic
     again = oracle.gumbel_sample(logits, 1.0, mask, seed=5)
     assert np.array_equal(got, again)
+
+
+def test_prefix_facts_closed_forms():
+    """The prefix helper used to check boundary rows: masses and ratios of a
+    hand-built row (probabilities 4:3:2:1:0.5), renormalised over the top-k
+    set when top-k is active, ids in the total order with ties to the lower
+    id."""
+    l = np.log(np.array([[2.0, 4.0, 3.0, 0.5, 1.0]]))
+    r = oracle.prefix(l, [2], want_ids=True)
+    assert r["ids"][0].tolist() == [1, 2]
+    assert abs(r["mass_n"][0] - 7 / 10.5) < 1e-15
+    assert abs(r["mass_prev"][0] - 4 / 10.5) < 1e-15
+    assert abs(r["ratio_n"][0] - 0.75) < 1e-15 and abs(r["ratio_next"][0] - 0.5) < 1e-15
+    assert r["nk"][0] == 5
+    r = oracle.prefix(l, [3], top_k=3)
+    assert abs(r["mass_n"][0] - 1.0) < 1e-15 and abs(r["mass_prev"][0] - 7 / 9) < 1e-15
+    assert r["nk"][0] == 3
+    r = oracle.prefix(l, [0])
+    assert r["mass_n"][0] == 0.0 and r["mass_prev"][0] == 0.0 and r["ratio_n"][0] == 1.0
+    ties = np.zeros((1, 6))
+    r = oracle.prefix(ties, [4], want_ids=True)
+    assert r["ids"][0].tolist() == [0, 1, 2, 3]
+    assert abs(r["mass_n"][0] - 4 / 6) < 1e-15
+    r = oracle.prefix(ties, [6])
+    assert r["ratio_next"][0] == 0.0 and abs(r["mass_n"][0] - 1.0) < 1e-15
+
+
+def test_lmhead_grad_finite_differences():
+    """The fused head's backward in the oracle (projection -> scoring -> VJP)
+    against central finite differences of the scalar objective through
+    oracle.score on fp64 logits z = H W^T / T, for entries of H and of W,
+    with top-k / top-p / min-p active (decisions held fixed away from their
+    thresholds)."""
+    rng = np.random.default_rng(5)
+    rows, vocab, hid, T = 3, 40, 6, 0.7
+    H = rng.normal(size=(rows, hid))
+    W = rng.normal(size=(vocab, hid)) * 0.8
+    y = np.array([0, 5, 39], np.int32)
+    z0 = H @ W.T / T
+    y[0] = int(np.argmax(z0[0]))  # a target inside the support
+    g = [np.array([0.7, -0.2, 1.1]), np.array([1.3, 0.4, -0.5]), np.array([0.2, -0.9, 0.3]),
+         np.array([-0.6, 0.8, 0.5])]
+    kw = dict(top_k=10, top_p=0.8, min_p=0.05)
+    dH, dW = oracle.lmhead_grad(H, W, y, T, *g, **kw)
+
+    def objective(Hm, Wm):
+        r = oracle.score(Hm @ Wm.T / T, y, **kw)
+        lps = np.where(np.isfinite(r["lp_support"]), r["lp_support"], 0.0)
+        return float(np.sum(g[0] * r["lp_full"] + g[1] * lps + g[2] * r["h_full"]
+                            + g[3] * r["h_support"]))
+
+    h = 1e-6
+    for (i, k) in [(0, 0), (1, 3), (2, 5)]:
+        Hp, Hm = H.copy(), H.copy()
+        Hp[i, k] += h
+        Hm[i, k] -= h
+        fd = (objective(Hp, W) - objective(Hm, W)) / (2 * h)
+        assert abs(fd - dH[i, k]) <= 1e-6 * max(1.0, abs(fd)), (i, k, fd, dH[i, k])
+    for (v, k) in [(int(np.argmax(z0[0])), 2), (7, 1), (39, 4)]:
+        Wp, Wm = W.copy(), W.copy()
+        Wp[v, k] += h
+        Wm[v, k] -= h
+        fd = (objective(H, Wp) - objective(H, Wm)) / (2 * h)
+        assert abs(fd - dW[v, k]) <= 1e-6 * max(1.0, abs(fd)), (v, k, fd, dW[v, k])
