@@ -547,7 +547,8 @@ def sample_workload(args, pk, steps, out):
         a = argsets[it[0] % nbuf]
         a.sample_seed = 1234 + it[0]
         it[0] += 1
-        rc = lib.vs_score_fwd(ctypes.byref(a), oref, ws.data_ptr(), ws.numel(), sp)
+        rc = lib.vs_score_fwd(ctypes.byref(a), oref, 0 if ws is None else ws.data_ptr(),
+                              0 if ws is None else ws.numel(), sp)
         if rc:
             raise RuntimeError(lib.vs_last_error().decode())
 
@@ -856,6 +857,10 @@ def main():
 
     vsb.load()
     h = headline(args, world, rank, pk)
+    if rank == 0:
+        print(json.dumps({"headline": {k: h[k] for k in ("value", "ms_per_step", "achieved",
+                                                          "per_call_ms")}}), file=sys.stderr,
+              flush=True)
     sec = None
     if rank == 0 and world == 1 and not args.no_secondary:
         sec = secondary(args, pk)

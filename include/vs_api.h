@@ -353,6 +353,51 @@ vs_status vs_fused_lmhead_bwd(int32_t rows, int32_t vocab, int32_t hidden_dim, c
 
 size_t vs_fused_lmhead_bwd_workspace_size(int32_t rows, int32_t vocab, int32_t hidden_dim);
 
+/* Vocabulary-parallel fused head (tensor parallelism over the vocabulary:
+ * [SkyRL] Implementation shares the tensor-parallel reduction of the replay
+ * logprob; [xorl] section 3 names a vocabulary-sharded LM-head group).  Each
+ * rank holds weight rows [vocab_begin, vocab_begin + vocab_count) of a
+ * vocab_total-row head and the full hidden states.
+ *
+ * Step 1, vs_fused_lmhead_partial: this shard's projection with the scoring
+ * epilogue, reduced to ONE partial record per row in `partial` (16-byte
+ * aligned, vs_fused_lmhead_partial_bytes(rows, top_k) bytes; the layout is
+ * opaque and the same on every rank): the shard's online statistics
+ * (max, count of max, sum 2^(u - max), sum (u - max) 2^(u - max) in base-2
+ * units u = z log2 e), its top_k (logit, vocabulary id) candidates in the
+ * total order, the target's logit when the shard holds the target (else 0),
+ * and a timeout flag.  Needs vs_fused_lmhead_partial_workspace_size(rows,
+ * vocab_count, hidden_dim, top_k) bytes of workspace.
+ *
+ * The exchange (the caller's): gather every rank's block into one buffer of
+ * n_shards consecutive blocks, in the order of the shards' vocab_begin (an
+ * all-gather of the bytes).
+ *
+ * Step 2, vs_fused_lmhead_merge: merges the n_shards blocks (statistics in
+ * shard order, k-way merge of the candidate lists, the target logit) and
+ * writes exactly the outputs of vs_fused_lmhead_score for the whole
+ * vocabulary (top-k, then inclusive top-p on the top-k mass, then min-p
+ * against the row max): lp_V, lp_S, H_V, H_S, valid, status, support_size,
+ * topk_ids, topk_logprob.  Every rank that merges gets the same outputs.
+ * out->support_mask, ctx and sampled must be NULL.  The full logits are
+ * never materialised and only (16 + 8 top_k + 4) bytes per row cross the
+ * ranks.  Errors as for vs_fused_lmhead_score; n_shards in [1, 64]. */
+size_t vs_fused_lmhead_partial_bytes(int32_t rows, int32_t top_k);
+size_t vs_fused_lmhead_partial_workspace_size(int32_t rows, int32_t vocab_count,
+                                              int32_t hidden_dim, int32_t top_k);
+vs_status vs_fused_lmhead_partial(int32_t rows, int32_t vocab_total, int32_t vocab_begin,
+                                  int32_t vocab_count, int32_t hidden_dim, const void* hidden,
+                                  int64_t ldh, const void* weight_shard, int64_t ldw,
+                                  const float* temperature, float temperature_scalar,
+                                  const int32_t* targets, int32_t top_k, void* partial,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+vs_status vs_fused_lmhead_merge(int32_t rows, int32_t vocab_total, int32_t n_shards,
+                                const void* partials, const float* temperature,
+                                float temperature_scalar, const int32_t* targets, int32_t top_k,
+                                float top_p, float min_p, uint32_t flags,
+                                const vs_score_out* out, int32_t* topk_ids, float* topk_logprob,
+                                void* stream);
+
 /* Support-only fused projection ([SkyRL] Performance: with a fused LM head
  * the replay path projects only the selected hidden-state / weight pairs and
  * never materialises vocabulary logits; Implementation: dense -1-padded

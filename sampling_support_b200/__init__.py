@@ -6,6 +6,8 @@ from ._binding import (  # noqa: F401
     LIB_PATH,
     VsError,
     fused_lmhead_bwd,
+    fused_lmhead_merge,
+    fused_lmhead_partial,
     fused_lmhead_score,
     l1_distance,
     l1_weight_sum,

@@ -109,6 +109,18 @@ def load() -> ctypes.CDLL:
         lib.vs_fused_lmhead_bwd.restype = i32
         lib.vs_fused_lmhead_bwd_workspace_size.argtypes = [i32, i32, i32]
         lib.vs_fused_lmhead_bwd_workspace_size.restype = sz
+        lib.vs_fused_lmhead_partial_bytes.argtypes = [i32, i32]
+        lib.vs_fused_lmhead_partial_bytes.restype = sz
+        lib.vs_fused_lmhead_partial_workspace_size.argtypes = [i32, i32, i32, i32]
+        lib.vs_fused_lmhead_partial_workspace_size.restype = sz
+        lib.vs_fused_lmhead_partial.argtypes = [i32, i32, i32, i32, i32, _vp, ctypes.c_int64, _vp,
+                                                ctypes.c_int64, _vp, ctypes.c_float, _vp, i32,
+                                                _vp, _vp, sz, _vp]
+        lib.vs_fused_lmhead_partial.restype = i32
+        lib.vs_fused_lmhead_merge.argtypes = [i32, i32, i32, _vp, _vp, ctypes.c_float, _vp, i32,
+                                              ctypes.c_float, ctypes.c_float, ctypes.c_uint32,
+                                              ctypes.POINTER(ScoreOut), _vp, _vp, _vp]
+        lib.vs_fused_lmhead_merge.restype = i32
         lib.vs_support_lmhead_score.argtypes = [i32, i32, i32, _vp, ctypes.c_int64, _vp,
                                                 ctypes.c_int64, _vp, ctypes.c_float, _vp, _vp, i32,
                                                 ctypes.c_int64, ctypes.c_uint32,
@@ -374,6 +386,67 @@ def fused_lmhead_score(hidden, weight, targets, temperature, top_k, top_p, min_p
                                      | (VS_WANT_GRAD if want_grad else 0), ctypes.byref(o),
                                      _p(out["topk_ids"]), _p(out["topk_logprob"]), _p(workspace),
                                      workspace.numel(), _stream(stream)))
+    return out
+
+
+def fused_lmhead_partial(hidden, weight_shard, vocab_begin, vocab_total, targets, temperature,
+                         top_k, out=None, workspace=None, stream=None):
+    """vs_fused_lmhead_partial: this shard's partial record block (a uint8
+    device tensor of vs_fused_lmhead_partial_bytes(rows, top_k) bytes)."""
+    lib = load()
+    rows, hdim = hidden.shape
+    count = weight_shard.shape[0]
+    dev = hidden.device
+    if out is None:
+        out = torch.empty(lib.vs_fused_lmhead_partial_bytes(rows, top_k), dtype=torch.uint8,
+                          device=dev)
+    if workspace is None:
+        nbytes = lib.vs_fused_lmhead_partial_workspace_size(rows, count, hdim, top_k)
+        workspace = torch.empty(max(16, (nbytes + 15) // 16 * 16), dtype=torch.uint8, device=dev)
+    t_arr = temperature if isinstance(temperature, torch.Tensor) else None
+    t_s = 1.0 if t_arr is not None else float(temperature)
+    _check(lib.vs_fused_lmhead_partial(rows, vocab_total, vocab_begin, count, hdim, _p(hidden),
+                                       hidden.stride(0), _p(weight_shard), weight_shard.stride(0),
+                                       _p(t_arr), t_s, _p(targets), top_k, _p(out),
+                                       _p(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
+def fused_lmhead_merge(partials, rows, vocab_total, targets, temperature, top_k, top_p, min_p,
+                       want_entropy=True, stream=None):
+    """vs_fused_lmhead_merge over `partials` (uint8 [n_shards, block bytes],
+    contiguous, the shards in vocabulary order); the outputs of
+    fused_lmhead_score for the whole vocabulary."""
+    lib = load()
+    n_shards = partials.shape[0]
+    dev = partials.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {
+        "lp_full": torch.empty(rows, **f32), "lp_support": torch.empty(rows, **f32),
+        "valid": torch.empty(rows, dtype=torch.uint8, device=dev),
+        "status": torch.empty(rows, dtype=torch.int32, device=dev),
+        "support_size": torch.empty(rows, dtype=torch.int32, device=dev),
+        "topk_ids": torch.empty((rows, top_k), dtype=torch.int32, device=dev),
+        "topk_logprob": torch.empty((rows, top_k), **f32),
+    }
+    if want_entropy:
+        out["h_full"] = torch.empty(rows, **f32)
+        out["h_support"] = torch.empty(rows, **f32)
+    o = ScoreOut()
+    o.logprob_full = _p(out["lp_full"])
+    o.logprob_support = _p(out["lp_support"])
+    o.entropy_full = _p(out.get("h_full"))
+    o.entropy_support = _p(out.get("h_support"))
+    o.valid = _p(out["valid"])
+    o.status = _p(out["status"])
+    o.support_size = _p(out["support_size"])
+    t_arr = temperature if isinstance(temperature, torch.Tensor) else None
+    t_s = 1.0 if t_arr is not None else float(temperature)
+    _check(lib.vs_fused_lmhead_merge(rows, vocab_total, n_shards, _p(partials), _p(t_arr), t_s,
+                                     _p(targets), top_k, float(top_p), float(min_p),
+                                     VS_WANT_ENTROPY if want_entropy else 0, ctypes.byref(o),
+                                     _p(out["topk_ids"]), _p(out["topk_logprob"]),
+                                     _stream(stream)))
     return out
 
 

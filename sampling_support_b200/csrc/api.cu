@@ -24,6 +24,17 @@ vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh
                      float* topk_logprob, void* ws, size_t ws_bytes, cudaStream_t s,
                      std::string* err);
 size_t lmhead_bwd_workspace_bytes(int rows, int vocab, int hidden);
+size_t lmhead_partial_bytes(int rows, int top_k);
+vs_status lmhead_partial_run(int rows, int vocab_total, int vocab_begin, int vocab_count,
+                             int hidden, const void* H, int64_t ldh, const void* W, int64_t ldw,
+                             const float* temperature, float temperature_scalar,
+                             const int32_t* targets, int top_k, void* partial, void* ws,
+                             size_t ws_bytes, cudaStream_t s, std::string* err);
+vs_status lmhead_merge_run(int rows, int vocab_total, int n_shards, const void* partials,
+                           const float* temperature, float temperature_scalar,
+                           const int32_t* targets, int top_k, float top_p, float min_p,
+                           uint32_t flags, const vs_score_out* out, int32_t* topk_ids,
+                           float* topk_logprob, cudaStream_t s, std::string* err);
 vs_status lmhead_bwd_run(int rows, int vocab, int hidden, const void* H, int64_t ldh,
                          const void* W, int64_t ldw, const int32_t* targets, int top_k,
                          const void* ctx, const int32_t* topk_ids, const float* g_lp_full,
@@ -349,6 +360,45 @@ vs_status vs_l1_distance_sharded(int32_t rows, int32_t vocab, int64_t ld, vs_dty
   return l1_call(rows, vocab, ld, dtype, draft, target, row_weight, l1, accept_rate,
                  loss_num_den_loss, grad_draft, grad_dtype, grad_ld, global_weight_sum,
                  workspace, workspace_bytes, stream);
+}
+
+size_t vs_fused_lmhead_partial_bytes(int32_t rows, int32_t top_k) {
+  return vs::lmhead_partial_bytes(rows, top_k);
+}
+
+size_t vs_fused_lmhead_partial_workspace_size(int32_t rows, int32_t vocab_count,
+                                              int32_t hidden_dim, int32_t top_k) {
+  return vs::lmhead_workspace_bytes(rows, vocab_count, hidden_dim, top_k);
+}
+
+vs_status vs_fused_lmhead_partial(int32_t rows, int32_t vocab_total, int32_t vocab_begin,
+                                  int32_t vocab_count, int32_t hidden_dim, const void* hidden,
+                                  int64_t ldh, const void* weight_shard, int64_t ldw,
+                                  const float* temperature, float temperature_scalar,
+                                  const int32_t* targets, int32_t top_k, void* partial,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  std::string err;
+  const vs_status st = vs::lmhead_partial_run(
+      rows, vocab_total, vocab_begin, vocab_count, hidden_dim, hidden, ldh, weight_shard, ldw,
+      temperature, temperature_scalar, targets, top_k, partial, workspace, workspace_bytes,
+      static_cast<cudaStream_t>(stream), &err);
+  if (st != VS_OK) return fail(st, err);
+  return ok();
+}
+
+vs_status vs_fused_lmhead_merge(int32_t rows, int32_t vocab_total, int32_t n_shards,
+                                const void* partials, const float* temperature,
+                                float temperature_scalar, const int32_t* targets, int32_t top_k,
+                                float top_p, float min_p, uint32_t flags,
+                                const vs_score_out* out, int32_t* topk_ids, float* topk_logprob,
+                                void* stream) {
+  std::string err;
+  const vs_status st = vs::lmhead_merge_run(rows, vocab_total, n_shards, partials, temperature,
+                                            temperature_scalar, targets, top_k, top_p, min_p,
+                                            flags, out, topk_ids, topk_logprob,
+                                            static_cast<cudaStream_t>(stream), &err);
+  if (st != VS_OK) return fail(st, err);
+  return ok();
 }
 
 size_t vs_fused_lmhead_bwd_workspace_size(int32_t rows, int32_t vocab, int32_t hidden_dim) {

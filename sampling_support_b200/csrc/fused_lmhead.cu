@@ -86,6 +86,7 @@ struct LmParams {
   int32_t* ws_id;    // [rows, splits, top_k]
   float* ws_zy;      // [rows] accumulator at the target id
   uint32_t* ws_err;  // [1] bounded-wait timeouts
+  int32_t col_offset;  // vocabulary id of weight row 0 (a shard of a vocabulary-parallel head)
   // backward (kModeDz): per-row (c, log-sum-exp in base-2 units, alpha, beta)
   // of the dense logit gradient p (alpha + beta x), c == 0 for a row with no
   // gradient; the bf16 gradient tile goes to dz [rows, dz_ld]
@@ -505,8 +506,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 4; ++i)
               d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
           } else {
-            for (int i = 0; i < 32 && col0 + i < P.vocab; ++i)
-              dst[i] = static_cast<uint16_t>((pk[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              if (col0 + 2 * i < P.vocab) dst[2 * i] = static_cast<uint16_t>(pk[i] & 0xFFFFu);
+              if (col0 + 2 * i + 1 < P.vocab) dst[2 * i + 1] = static_cast<uint16_t>(pk[i] >> 16);
+            }
           }
         }
       }
@@ -528,7 +532,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool row_ok = row < P.rows;
       const float T = row_ok ? (P.temperature ? P.temperature[row] : P.temperature_scalar) : 1.f;
       const float c = kLog2e / T;
-      const int y = row_ok ? P.targets[row] : -1;
+      // the target as a column of this weight (outside [0, vocab): not here)
+      const int y = row_ok ? P.targets[row] - P.col_offset : -1;
+      const bool y_here = y >= 0 && y < P.vocab;
       Stats st = stats_empty();
       int count = 0, low = 0;
       float thr = -kInf;  // smallest listed value once the list is full
@@ -576,12 +582,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) cand |= (i < nv && v[i] > thr ? 1u : 0u) << i;
           }
-          if (y >= col0 && y < col0 + 32) P.ws_zy[row] = pick32(v, y - col0);
+          if (y_here && y >= col0 && y < col0 + 32) P.ws_zy[row] = pick32(v, y - col0);
           while (cand != 0u) {
             const int i = __ffs(cand) - 1;
             cand &= cand - 1u;
             const float x = pick32(v, i);
-            if (x > thr) topk_push(my_val, my_id, k, count, low, thr, x, col0 + i);
+            if (x > thr) topk_push(my_val, my_id, k, count, low, thr, x, col0 + i + P.col_offset);
           }
         }
       }
@@ -652,6 +658,10 @@ enum : uint32_t {
   kLmCtxTargetInS = 1u << 2,
 };
 
+// Inputs of the merge: `splits` partial records per row, at element strides
+// (row, split) for the statistics and the lists, the target logit as the sum
+// over `parts` entries (one part holds it, the others hold 0) and the
+// timeout flags ORed over `parts` entries.
 struct MergeParams {
   int32_t rows, vocab, splits, top_k;
   float top_p, min_p;
@@ -663,6 +673,18 @@ struct MergeParams {
   const int32_t* ws_id;
   const float* ws_zy;
   const uint32_t* ws_err;
+  int64_t st_row, st_split;  // float4 elements
+  int64_t ls_row, ls_split;  // list elements
+  int32_t parts;
+  int64_t zy_part, err_part;  // elements
+  // partial output (one shard of a vocabulary-parallel head): the merged
+  // statistics, top-k list, target logit and flag of this shard's splits
+  // are written here and nothing is finalised
+  float4* out_stats;
+  float* out_val;
+  int32_t* out_id;
+  float* out_zy;
+  uint32_t* out_err;
   float* lp_full;
   float* lp_support;
   float* h_full;
@@ -678,115 +700,214 @@ struct MergeParams {
 
 constexpr int kMaxSplits = 64;
 
+// (value, id) ranks before (v2, i2) in the total order (value desc, id asc);
+// id -1 marks an exhausted list and ranks last
+__device__ __forceinline__ bool ranks_before(float v, int32_t i, float v2, int32_t i2) {
+  if (i < 0) return false;
+  if (i2 < 0) return true;
+  return v > v2 || (v == v2 && i < i2);
+}
+
+// One warp per row.  Lane l owns splits l and l + 32: their statistics are
+// merged by a fixed shuffle tree, and their sorted lists by k rounds of a
+// warp-wide argmax over the lanes' list heads.  Entry i of the merged top-k
+// lives in lane i % 32, slot i / 32.
 __global__ void __launch_bounds__(128) lmhead_merge_kernel(MergeParams P) {
-  const int row = blockIdx.x * blockDim.x + threadIdx.x;
-  if (row >= P.rows) return;
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= P.rows) return;  // whole warps leave together
   const int k = P.top_k;
   const float T = P.temperature ? P.temperature[row] : P.temperature_scalar;
   const float c = kLog2e / T;
   const float nan = __int_as_float(0x7fc00000);
-  // statistics over the full vocabulary, splits merged in order
+  // statistics over the full vocabulary
   Stats st = stats_empty();
-  for (int s = 0; s < P.splits; ++s) {
-    const float4 v = P.ws_stats[static_cast<int64_t>(row) * P.splits + s];
+  for (int sp = lane; sp < P.splits; sp += 32) {
+    const float4 v = P.ws_stats[row * P.st_row + sp * P.st_split];
     stats_merge(st, Stats{v.x, v.y, v.z, v.w});
   }
-  const bool timeout = *P.ws_err != 0;
+  {
+    float m = st.m;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (st.c0 != 0.f || st.zr != 0.f) stats_rebase(st, m);
+    float c0 = st.c0, zr = st.zr, a = st.a;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      c0 += __shfl_xor_sync(0xffffffffu, c0, o);
+      zr += __shfl_xor_sync(0xffffffffu, zr, o);
+      a += __shfl_xor_sync(0xffffffffu, a, o);
+    }
+    st = Stats{m, c0, zr, a};
+  }
+  uint32_t errs = 0;
+  for (int q = 0; q < P.parts; ++q) errs |= P.ws_err[q * P.err_part];
+  const bool timeout = errs != 0;
   const bool nonfinite = !stats_finite(st);
   const float log2z = stats_log2z(st);
   const float h_full = kLn2 * (log2z - st.a / stats_z(st));
   // top-k by (value desc, id asc): k-way merge of the sorted split lists
-  int cur[kMaxSplits];
-  for (int s = 0; s < P.splits; ++s) cur[s] = 0;
-  float tv[VS_MAX_FUSED_TOPK];
-  int32_t ti[VS_MAX_FUSED_TOPK];
-  const int64_t base = static_cast<int64_t>(row) * P.splits * k;
+  const int64_t lbase = row * P.ls_row;
+  int cur0 = 0, cur1 = 0;
+  const bool has0 = lane < P.splits, has1 = lane + 32 < P.splits;
+  auto head = [&](int sp, int cur, float& v, int32_t& id) {
+    v = -kInf;
+    id = -1;
+    if (cur < k) {
+      v = P.ws_val[lbase + sp * P.ls_split + cur];
+      id = P.ws_id[lbase + sp * P.ls_split + cur];
+    }
+  };
+  float h0v = -kInf, h1v = -kInf;
+  int32_t h0i = -1, h1i = -1;
+  if (has0) head(lane, 0, h0v, h0i);
+  if (has1) head(lane + 32, 0, h1v, h1i);
+  float tv[2] = {-kInf, -kInf};
+  int32_t ti[2] = {-1, -1};
   for (int i = 0; i < k; ++i) {
-    int best = -1;
-    float bv = -kInf;
-    int32_t bi = INT_MAX;
-    for (int s = 0; s < P.splits; ++s) {
-      if (cur[s] >= k) continue;
-      const float v = P.ws_val[base + s * k + cur[s]];
-      const int32_t id = P.ws_id[base + s * k + cur[s]];
-      if (id < 0) continue;
-      if (best < 0 || v > bv || (v == bv && id < bi)) {
-        best = s;
-        bv = v;
-        bi = id;
+    const bool second = ranks_before(h1v, h1i, h0v, h0i);
+    float bv = second ? h1v : h0v;
+    int32_t bi = second ? h1i : h0i;
+    int bl = lane;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      const int ol = __shfl_xor_sync(0xffffffffu, bl, o);
+      if (ranks_before(ov, oi, bv, bi) || (oi == bi && ol < bl)) {
+        bv = ov;
+        bi = oi;
+        bl = ol;
       }
     }
-    if (best < 0) {
-      tv[i] = -kInf;
-      ti[i] = -1;
-    } else {
-      tv[i] = bv;
-      ti[i] = bi;
-      ++cur[best];
-    }
-  }
-  // support: inclusive top-p on the top-k mass, then min-p against the max
-  int n = 0;
-  double mass1 = 0.0;
-  for (int i = 0; i < k; ++i)
-    if (ti[i] >= 0) mass1 += static_cast<double>(ex2(__fmul_rn(tv[i], c) - st.m));
-  {
-    double cum = 0.0;
-    n = k;
-    if (P.top_p < 1.f) {
-      for (int i = 0; i < k; ++i) {
-        if (ti[i] < 0) {
-          n = i;
-          break;
-        }
-        cum += static_cast<double>(ex2(__fmul_rn(tv[i], c) - st.m));
-        if (cum >= static_cast<double>(P.top_p) * mass1) {
-          n = i + 1;
-          break;
-        }
+    if (lane == (i & 31)) {
+      if (i < 32) {
+        tv[0] = bi >= 0 ? bv : -kInf;
+        ti[0] = bi;
+      } else {
+        tv[1] = bi >= 0 ? bv : -kInf;
+        ti[1] = bi;
       }
-    } else {
-      for (int i = 0; i < k; ++i)
-        if (ti[i] < 0) {
-          n = i;
-          break;
-        }
     }
-    if (P.min_p > 0.f) {
-      int nm = 0;
-      for (int i = 0; i < n; ++i)
-        if (ex2(__fmul_rn(tv[i], c) - st.m) >= P.min_p) nm = i + 1;
-      n = nm;
+    if (bi >= 0 && lane == bl) {
+      if (second) {
+        ++cur1;
+        head(lane + 32, cur1, h1v, h1i);
+      } else {
+        ++cur0;
+        head(lane, cur0, h0v, h0i);
+      }
     }
   }
-  // support statistics (relative to its maximum, the top-1 value)
+  float zy = 0.f;
+  for (int q = 0; q < P.parts; ++q) zy += P.ws_zy[q * P.zy_part + row];
+  if (P.out_stats) {
+    // one shard of a vocabulary-parallel head: hand on the merged record
+#pragma unroll
+    for (int sl = 0; sl < 2; ++sl) {
+      const int i = sl * 32 + lane;
+      if (i < k) {
+        P.out_val[static_cast<int64_t>(row) * k + i] = tv[sl];
+        P.out_id[static_cast<int64_t>(row) * k + i] = ti[sl];
+      }
+    }
+    if (lane == 0) {
+      P.out_stats[row] = make_float4(st.m, st.c0, st.zr, st.a);
+      P.out_zy[row] = zy;
+      if (timeout) atomicOr(P.out_err, 1u);
+    }
+    return;
+  }
+  // support: inclusive top-p on the top-k mass (fp64 prefix sums in rank
+  // order), then min-p against the row max
+  double e[2], pre[2];
+  bool live[2];
+#pragma unroll
+  for (int sl = 0; sl < 2; ++sl) {
+    const int i = sl * 32 + lane;
+    live[sl] = i < k && ti[sl] >= 0;
+    e[sl] = live[sl] ? static_cast<double>(ex2(__fmul_rn(tv[sl], c) - st.m)) : 0.0;
+    double x = e[sl];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    pre[sl] = x;
+  }
+  const double tot0 = __shfl_sync(0xffffffffu, pre[0], 31);
+  pre[1] += tot0;
+  const double mass1 = __shfl_sync(0xffffffffu, pre[1], 31);
+  const uint32_t lv0 = __ballot_sync(0xffffffffu, live[0]), lv1 = __ballot_sync(0xffffffffu, live[1]);
+  const int nlive = __popc(lv0) + __popc(lv1);  // live entries form a prefix
+  int n = nlive;
+  if (P.top_p < 1.f) {
+    const double tgt = static_cast<double>(P.top_p) * mass1;
+    const uint32_t r0 = __ballot_sync(0xffffffffu, live[0] && pre[0] >= tgt);
+    const uint32_t r1 = __ballot_sync(0xffffffffu, live[1] && pre[1] >= tgt);
+    if (r0)
+      n = __ffs(r0);
+    else if (r1)
+      n = 32 + __ffs(r1);
+  }
+  if (P.min_p > 0.f) {
+    const uint32_t q0 = __ballot_sync(0xffffffffu, live[0] && lane < n &&
+                                                      static_cast<float>(e[0]) >= P.min_p);
+    const uint32_t q1 = __ballot_sync(0xffffffffu, live[1] && 32 + lane < n &&
+                                                      static_cast<float>(e[1]) >= P.min_p);
+    n = __popc(q0) + __popc(q1);  // the ratio falls along the order: a prefix
+  }
+  // support statistics relative to its maximum, the top-1 value
+  const float ms = __shfl_sync(0xffffffffu, __fmul_rn(tv[0], c), 0);
   Stats ss = stats_empty();
   if (n > 0) {
-    const float ms = __fmul_rn(tv[0], c);
-    ss = Stats{ms, 0.f, 0.f, 0.f};
-    for (int i = 0; i < n; ++i) {
-      const float d = __fmul_rn(tv[i], c) - ms;
-      const float e = ex2(d);
-      if (d == 0.f)
-        ss.c0 += 1.f;
-      else
-        ss.zr += e;
-      ss.a = fmaf(d, e, ss.a);
+    float c0 = 0.f, zr = 0.f, a = 0.f;
+#pragma unroll
+    for (int sl = 0; sl < 2; ++sl) {
+      if (sl * 32 + lane < n) {
+        const float d = __fmul_rn(tv[sl], c) - ms;
+        const float ev = ex2(d);
+        if (d == 0.f)
+          c0 += 1.f;
+        else
+          zr += ev;
+        a = fmaf(d, ev, a);
+      }
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      c0 += __shfl_xor_sync(0xffffffffu, c0, o);
+      zr += __shfl_xor_sync(0xffffffffu, zr, o);
+      a += __shfl_xor_sync(0xffffffffu, a, o);
+    }
+    ss = Stats{ms, c0, zr, a};
   }
   const float log2zs = n > 0 ? stats_log2z(ss) : nan;
   const float h_sup = n > 0 ? kLn2 * (log2zs - ss.a / stats_z(ss)) : 0.f;
   const int y = P.targets[row];
+  const bool in_s = __ballot_sync(0xffffffffu, (lane < n && ti[0] == y) ||
+                                                   (32 + lane < n && ti[1] == y)) != 0u;
+  // the writes: per-row values by lane 0, the top-k entries by their lanes
+  if (P.topk_ids || P.topk_logprob) {
+#pragma unroll
+    for (int sl = 0; sl < 2; ++sl) {
+      const int i = sl * 32 + lane;
+      if (i >= k) continue;
+      if (P.topk_ids) P.topk_ids[static_cast<int64_t>(row) * k + i] = ti[sl];
+      if (P.topk_logprob)
+        P.topk_logprob[static_cast<int64_t>(row) * k + i] =
+            (ti[sl] >= 0 && !nonfinite) ? kLn2 * (__fmul_rn(tv[sl], c) - st.m - log2z) : nan;
+    }
+  }
+  if (lane != 0) return;
   uint32_t status = 0;
   float lp_v = nan, lp_s = nan;
-  bool in_s = false;
   if (y < 0 || y >= P.vocab) status |= VS_ROW_TARGET_OUT_OF_RANGE;
   if (nonfinite) {
     status |= VS_ROW_NONFINITE_INPUT;
   } else if (!(status & VS_ROW_TARGET_OUT_OF_RANGE)) {
-    const float uy = __fmul_rn(P.ws_zy[row], c);
+    const float uy = __fmul_rn(zy, c);
     lp_v = kLn2 * (uy - st.m - log2z);
-    for (int i = 0; i < n; ++i) in_s |= ti[i] == y;
     if (in_s) {
       lp_s = kLn2 * (uy - ss.m - log2zs);
     } else {
@@ -817,19 +938,20 @@ __global__ void __launch_bounds__(128) lmhead_merge_kernel(MergeParams P) {
     uint32_t f = 0;
     if (nonfinite || timeout) f |= kLmCtxNonFinite;
     if (!(status & VS_ROW_TARGET_OUT_OF_RANGE)) f |= kLmCtxTargetOk;
-    if (in_s) f |= kLmCtxTargetInS;
+    if (in_s && !nonfinite) f |= kLmCtxTargetInS;
     cx.flags = f;
     P.ctx[row] = cx;
   }
-  for (int i = 0; i < k; ++i) {
-    if (P.topk_ids) P.topk_ids[static_cast<int64_t>(row) * k + i] = ti[i];
-    if (P.topk_logprob)
-      P.topk_logprob[static_cast<int64_t>(row) * k + i] =
-          (ti[i] >= 0 && !nonfinite) ? kLn2 * (__fmul_rn(tv[i], c) - st.m - log2z) : nan;
-  }
 }
 
-__global__ void lmhead_clear_kernel(uint32_t* err) { *err = 0u; }
+// Clears the timeout flag and, when given, the target logits (a shard that
+// does not hold a row's target leaves 0 there).
+__global__ void lmhead_clear_kernel(uint32_t* err, float* zy, int rows) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) *err = 0u;
+  if (zy)
+    for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < rows; r += gridDim.x * blockDim.x)
+      zy[r] = 0.f;
+}
 
 // ---------------------------------------------------------------------------
 // backward (xorl issue #71, section 1: selected logprob + VJP), with respect
@@ -1207,6 +1329,96 @@ size_t lmhead_workspace_bytes(int rows, int vocab, int hidden, int top_k) {
   return a > b ? a : b;
 }
 
+namespace {
+
+// The projection with the scoring epilogue over weight rows [0, vocab) whose
+// vocabulary ids start at col_offset: per (row, split) records in `ws`
+// (lm_layout).  clear_zy zeroes the target logits first (a shard may not
+// hold a row's target).
+vs_status gemm_phase(int rows, int vocab, int col_offset, int hidden, const void* H, int64_t ldh,
+                     const void* W, int64_t ldw, const float* temperature,
+                     float temperature_scalar, const int32_t* targets, int top_k, void* ws,
+                     bool clear_zy, cudaStream_t s, LmParams* Pout, LmLayout* Lout,
+                     std::string* err) {
+  const GemmConfig G = gemm_config<kModeScore>(top_k);
+  const LmLayout L = lm_layout(rows, vocab, top_k, G.pair);
+  CUtensorMap map_h, map_w;
+  if (!make_map(&map_h, H, rows, hidden, ldh, kBM) ||
+      !make_map(&map_w, W, vocab, hidden, ldw, G.pair ? kBNh : kBN)) {
+    *err = "cuTensorMapEncodeTiled failed";
+    return VS_ERR_CUDA;
+  }
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  LmParams P{};
+  P.rows = rows;
+  P.vocab = vocab;
+  P.hidden = hidden;
+  P.top_k = top_k;
+  P.splits = L.splits;
+  P.tiles_per_split = L.tiles_per_split;
+  P.n_tiles = L.n_tiles;
+  P.m_blocks = L.m_blocks;
+  P.m_units = L.m_units;
+  P.stages = G.stages;
+  P.temperature = temperature;
+  P.temperature_scalar = temperature_scalar;
+  P.targets = targets;
+  P.col_offset = col_offset;
+  P.ws_stats = reinterpret_cast<float4*>(w8 + L.off_stats);
+  P.ws_val = reinterpret_cast<float*>(w8 + L.off_val);
+  P.ws_id = reinterpret_cast<int32_t*>(w8 + L.off_id);
+  P.ws_zy = reinterpret_cast<float*>(w8 + L.off_zy);
+  P.ws_err = reinterpret_cast<uint32_t*>(w8 + L.off_err);
+  if (clear_zy)
+    lmhead_clear_kernel<<<(rows + 255) / 256, 256, 0, s>>>(P.ws_err, P.ws_zy, rows);
+  else
+    lmhead_clear_kernel<<<1, 1, 0, s>>>(P.ws_err, nullptr, 0);
+  cudaError_t e = gemm_launch<kModeScore>(G, map_h, map_w, P, L.m_units * L.splits, s);
+  if (e != cudaSuccess) {
+    *err = cudaGetErrorString(e);
+    return VS_ERR_CUDA;
+  }
+  *Pout = P;
+  *Lout = L;
+  return VS_OK;
+}
+
+// Merge inputs: the GEMM's per-(row, split) records.
+void merge_from_workspace(MergeParams& M, const LmParams& P, const LmLayout& L, int top_k) {
+  M.splits = L.splits;
+  M.ws_stats = P.ws_stats;
+  M.ws_val = P.ws_val;
+  M.ws_id = P.ws_id;
+  M.ws_zy = P.ws_zy;
+  M.ws_err = P.ws_err;
+  M.st_row = L.splits;
+  M.st_split = 1;
+  M.ls_row = static_cast<int64_t>(L.splits) * top_k;
+  M.ls_split = top_k;
+  M.parts = 1;
+  M.zy_part = 0;
+  M.err_part = 0;
+}
+
+// One shard's partial record block (vocabulary-parallel head).
+struct PartLayout {
+  size_t off_stats, off_val, off_id, off_zy, off_err, total;
+};
+
+PartLayout part_layout(int rows, int top_k) {
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  PartLayout L{};
+  L.off_stats = 0;
+  L.off_val = up(static_cast<size_t>(rows) * sizeof(float4));
+  L.off_id = up(L.off_val + static_cast<size_t>(rows) * top_k * sizeof(float));
+  L.off_zy = up(L.off_id + static_cast<size_t>(rows) * top_k * sizeof(int32_t));
+  L.off_err = up(L.off_zy + static_cast<size_t>(rows) * sizeof(float));
+  L.total = up(L.off_err + 16);
+  return L;
+}
+
+}  // namespace
+
 vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh, const void* W,
                      int64_t ldw, const float* temperature, float temperature_scalar,
                      const int32_t* targets, int top_k, float top_p, float min_p,
@@ -1245,54 +1457,21 @@ vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh
   if (!ws || !a16(ws) || ws_bytes < lmhead_workspace_bytes(rows, vocab, hidden, top_k))
     return bad(VS_ERR_WORKSPACE, "workspace missing, misaligned or smaller than vs_fused_lmhead_workspace_size");
 
-  const GemmConfig G = gemm_config<kModeScore>(top_k);
-  const LmLayout L = lm_layout(rows, vocab, top_k, G.pair);
-
-  CUtensorMap map_h, map_w;
-  if (!make_map(&map_h, H, rows, hidden, ldh, kBM) ||
-      !make_map(&map_w, W, vocab, hidden, ldw, G.pair ? kBNh : kBN))
-    return bad(VS_ERR_CUDA, "cuTensorMapEncodeTiled failed");
-
-  uint8_t* w8 = static_cast<uint8_t*>(ws);
   LmParams P{};
-  P.rows = rows;
-  P.vocab = vocab;
-  P.hidden = hidden;
-  P.top_k = top_k;
-  P.splits = L.splits;
-  P.tiles_per_split = L.tiles_per_split;
-  P.n_tiles = L.n_tiles;
-  P.m_blocks = L.m_blocks;
-  P.m_units = L.m_units;
-  P.stages = G.stages;
-  P.temperature = temperature;
-  P.temperature_scalar = temperature_scalar;
-  P.targets = targets;
-  P.ws_stats = reinterpret_cast<float4*>(w8 + L.off_stats);
-  P.ws_val = reinterpret_cast<float*>(w8 + L.off_val);
-  P.ws_id = reinterpret_cast<int32_t*>(w8 + L.off_id);
-  P.ws_zy = reinterpret_cast<float*>(w8 + L.off_zy);
-  P.ws_err = reinterpret_cast<uint32_t*>(w8 + L.off_err);
-
-  lmhead_clear_kernel<<<1, 1, 0, s>>>(P.ws_err);
-  cudaError_t e = gemm_launch<kModeScore>(G, map_h, map_w, P, L.m_units * L.splits, s);
-  if (e != cudaSuccess) return bad(VS_ERR_CUDA, cudaGetErrorString(e));
-
+  LmLayout L{};
+  const vs_status gs = gemm_phase(rows, vocab, 0, hidden, H, ldh, W, ldw, temperature,
+                                  temperature_scalar, targets, top_k, ws, false, s, &P, &L, err);
+  if (gs != VS_OK) return gs;
   MergeParams M{};
+  merge_from_workspace(M, P, L, top_k);
   M.rows = rows;
   M.vocab = vocab;
-  M.splits = L.splits;
   M.top_k = top_k;
   M.top_p = top_p;
   M.min_p = min_p;
   M.temperature = temperature;
   M.temperature_scalar = temperature_scalar;
   M.targets = targets;
-  M.ws_stats = P.ws_stats;
-  M.ws_val = P.ws_val;
-  M.ws_id = P.ws_id;
-  M.ws_zy = P.ws_zy;
-  M.ws_err = P.ws_err;
   M.lp_full = out->logprob_full;
   M.lp_support = out->logprob_support;
   M.h_full = want_entropy ? out->entropy_full : nullptr;
@@ -1304,8 +1483,141 @@ vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh
   M.topk_logprob = topk_logprob;
   M.ctx = want_grad ? static_cast<LmCtx*>(out->ctx) : nullptr;
   M.want_entropy = want_entropy ? 1 : 0;
-  lmhead_merge_kernel<<<(rows + 127) / 128, 128, 0, s>>>(M);
-  e = cudaGetLastError();
+  lmhead_merge_kernel<<<(rows + 3) / 4, 128, 0, s>>>(M);  // a warp per row
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return bad(VS_ERR_CUDA, cudaGetErrorString(e));
+  return VS_OK;
+}
+
+// ---------------------------------------------------------------------------
+// vocabulary-parallel head: one shard's partial records, then the merge of
+// every shard's records
+
+size_t lmhead_partial_bytes(int rows, int top_k) {
+  if (rows <= 0 || top_k <= 0) return 0;
+  return part_layout(rows, top_k).total;
+}
+
+vs_status lmhead_partial_run(int rows, int vocab_total, int vocab_begin, int vocab_count,
+                             int hidden, const void* H, int64_t ldh, const void* W, int64_t ldw,
+                             const float* temperature, float temperature_scalar,
+                             const int32_t* targets, int top_k, void* partial, void* ws,
+                             size_t ws_bytes, cudaStream_t s, std::string* err) {
+  auto bad = [&](vs_status code, const char* msg) {
+    *err = msg;
+    return code;
+  };
+  auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (rows < 0) return bad(VS_ERR_INVALID_ARG, "rows must be >= 0");
+  if (vocab_total < 1 || vocab_begin < 0 || vocab_count < 1 || vocab_begin > vocab_total - vocab_count)
+    return bad(VS_ERR_INVALID_ARG, "the shard [vocab_begin, vocab_begin + vocab_count) must lie in [0, vocab_total)");
+  if (hidden < kBK || hidden % kBK != 0)
+    return bad(VS_ERR_UNSUPPORTED, "hidden_dim must be a positive multiple of 64");
+  if (top_k < 1 || top_k > VS_MAX_FUSED_TOPK || top_k > vocab_total)
+    return bad(VS_ERR_UNSUPPORTED, "top_k must lie in [1, min(VS_MAX_FUSED_TOPK, vocab_total)]");
+  if (!temperature && !(std::isfinite(temperature_scalar) && temperature_scalar > 0.f))
+    return bad(VS_ERR_INVALID_ARG, "temperature_scalar must be finite and > 0");
+  if (rows == 0) return VS_OK;
+  if (!H || !W || !targets || !partial)
+    return bad(VS_ERR_INVALID_ARG, "hidden, weight, targets and partial must be non-NULL");
+  if (!a16(H) || !a16(W) || !a16(partial) || ldh % 8 != 0 || ldw % 8 != 0 || ldh < hidden ||
+      ldw < hidden)
+    return bad(VS_ERR_INVALID_ARG, "hidden/weight/partial must be 16-byte aligned with ld >= hidden_dim, ld % 8 == 0");
+  if (!ws || !a16(ws) || ws_bytes < lmhead_workspace_bytes(rows, vocab_count, hidden, top_k))
+    return bad(VS_ERR_WORKSPACE, "workspace missing, misaligned or smaller than vs_fused_lmhead_partial_workspace_size");
+  LmParams P{};
+  LmLayout L{};
+  const vs_status gs = gemm_phase(rows, vocab_count, vocab_begin, hidden, H, ldh, W, ldw,
+                                  temperature, temperature_scalar, targets, top_k, ws, true, s,
+                                  &P, &L, err);
+  if (gs != VS_OK) return gs;
+  const PartLayout B = part_layout(rows, top_k);
+  uint8_t* b8 = static_cast<uint8_t*>(partial);
+  MergeParams M{};
+  merge_from_workspace(M, P, L, top_k);
+  M.rows = rows;
+  M.vocab = vocab_total;
+  M.top_k = top_k;
+  M.temperature = temperature;
+  M.temperature_scalar = temperature_scalar;
+  M.targets = targets;
+  M.out_stats = reinterpret_cast<float4*>(b8 + B.off_stats);
+  M.out_val = reinterpret_cast<float*>(b8 + B.off_val);
+  M.out_id = reinterpret_cast<int32_t*>(b8 + B.off_id);
+  M.out_zy = reinterpret_cast<float*>(b8 + B.off_zy);
+  M.out_err = reinterpret_cast<uint32_t*>(b8 + B.off_err);
+  lmhead_clear_kernel<<<1, 1, 0, s>>>(M.out_err, nullptr, 0);
+  lmhead_merge_kernel<<<(rows + 3) / 4, 128, 0, s>>>(M);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return bad(VS_ERR_CUDA, cudaGetErrorString(e));
+  return VS_OK;
+}
+
+vs_status lmhead_merge_run(int rows, int vocab_total, int n_shards, const void* partials,
+                           const float* temperature, float temperature_scalar,
+                           const int32_t* targets, int top_k, float top_p, float min_p,
+                           uint32_t flags, const vs_score_out* out, int32_t* topk_ids,
+                           float* topk_logprob, cudaStream_t s, std::string* err) {
+  auto bad = [&](vs_status code, const char* msg) {
+    *err = msg;
+    return code;
+  };
+  auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (rows < 0) return bad(VS_ERR_INVALID_ARG, "rows must be >= 0");
+  if (vocab_total < 1) return bad(VS_ERR_INVALID_ARG, "vocab_total must be >= 1");
+  if (n_shards < 1 || n_shards > kMaxSplits)
+    return bad(VS_ERR_UNSUPPORTED, "n_shards must lie in [1, 64]");
+  if (top_k < 1 || top_k > VS_MAX_FUSED_TOPK || top_k > vocab_total)
+    return bad(VS_ERR_UNSUPPORTED, "top_k must lie in [1, min(VS_MAX_FUSED_TOPK, vocab_total)]");
+  if (!(top_p > 0.f && top_p <= 1.f)) return bad(VS_ERR_INVALID_ARG, "top_p must lie in (0, 1]");
+  if (!(min_p >= 0.f && min_p < 1.f)) return bad(VS_ERR_INVALID_ARG, "min_p must lie in [0, 1)");
+  if (!temperature && !(std::isfinite(temperature_scalar) && temperature_scalar > 0.f))
+    return bad(VS_ERR_INVALID_ARG, "temperature_scalar must be finite and > 0");
+  if (!out) return bad(VS_ERR_INVALID_ARG, "out is NULL");
+  if (out->sampled || out->support_mask || out->ctx || (flags & (VS_WANT_SAMPLE | VS_WANT_GRAD)))
+    return bad(VS_ERR_INVALID_ARG, "sampled, support_mask and ctx are not offered by the merge: pass NULL");
+  const bool want_entropy = flags & VS_WANT_ENTROPY;
+  if (!want_entropy && (out->entropy_full || out->entropy_support))
+    return bad(VS_ERR_INVALID_ARG, "entropy outputs need VS_WANT_ENTROPY");
+  if (rows == 0) return VS_OK;
+  if (!partials || !a16(partials) || !targets)
+    return bad(VS_ERR_INVALID_ARG, "partials (16-byte aligned) and targets must be non-NULL");
+  const PartLayout B = part_layout(rows, top_k);
+  const uint8_t* b8 = static_cast<const uint8_t*>(partials);
+  MergeParams M{};
+  M.rows = rows;
+  M.vocab = vocab_total;
+  M.splits = n_shards;
+  M.top_k = top_k;
+  M.top_p = top_p;
+  M.min_p = min_p;
+  M.temperature = temperature;
+  M.temperature_scalar = temperature_scalar;
+  M.targets = targets;
+  M.ws_stats = reinterpret_cast<const float4*>(b8 + B.off_stats);
+  M.ws_val = reinterpret_cast<const float*>(b8 + B.off_val);
+  M.ws_id = reinterpret_cast<const int32_t*>(b8 + B.off_id);
+  M.ws_zy = reinterpret_cast<const float*>(b8 + B.off_zy);
+  M.ws_err = reinterpret_cast<const uint32_t*>(b8 + B.off_err);
+  M.st_row = 1;
+  M.st_split = static_cast<int64_t>(B.total / sizeof(float4));
+  M.ls_row = top_k;
+  M.ls_split = static_cast<int64_t>(B.total / sizeof(float));
+  M.parts = n_shards;
+  M.zy_part = static_cast<int64_t>(B.total / sizeof(float));
+  M.err_part = static_cast<int64_t>(B.total / sizeof(uint32_t));
+  M.lp_full = out->logprob_full;
+  M.lp_support = out->logprob_support;
+  M.h_full = want_entropy ? out->entropy_full : nullptr;
+  M.h_support = want_entropy ? out->entropy_support : nullptr;
+  M.valid = out->valid;
+  M.status = out->status;
+  M.support_size = out->support_size;
+  M.topk_ids = topk_ids;
+  M.topk_logprob = topk_logprob;
+  M.want_entropy = want_entropy ? 1 : 0;
+  lmhead_merge_kernel<<<(rows + 3) / 4, 128, 0, s>>>(M);
+  const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return bad(VS_ERR_CUDA, cudaGetErrorString(e));
   return VS_OK;
 }
@@ -1354,7 +1666,7 @@ vs_status lmhead_bwd_run(int rows, int vocab, int hidden, const void* H, int64_t
   void* ltws = w8 + L.off_lt;
   const LmCtx* cx = static_cast<const LmCtx*>(ctx);
 
-  lmhead_clear_kernel<<<1, 1, 0, s>>>(werr);
+  lmhead_clear_kernel<<<1, 1, 0, s>>>(werr, nullptr, 0);
   BwdRowParams R{};
   R.rows = rows;
   R.top_k = top_k;

@@ -11,6 +11,11 @@ data path.  The only cross-rank steps are scalar reductions:
   entropy statistic joins the reduction that the replay logprob already
   uses): sum over valid rows of H_S and the count of valid rows.
 
+The vocabulary-parallel fused head (tensor parallelism over the LM head's
+vocabulary) has one real exchange: every rank's fixed-size partial record
+block (per row: the shard's online statistics, its top-k candidates and the
+target logit) is all-gathered, and every rank merges the blocks.
+
 The library performs no collective itself; these helpers call it and reduce
 the scalars with torch.distributed (NCCL on GPUs).  Every rank must call them
 in the same order.
@@ -26,6 +31,17 @@ from . import _binding as B
 
 class LibraryOps:
     """The per-rank steps, run by libvs.so."""
+
+    @staticmethod
+    def lmhead_partial(hidden, weight_shard, vocab_begin, vocab_total, targets, temperature,
+                       top_k):
+        return B.fused_lmhead_partial(hidden, weight_shard, vocab_begin, vocab_total, targets,
+                                      temperature, top_k)
+
+    @staticmethod
+    def lmhead_merge(partials, rows, vocab_total, targets, temperature, top_k, top_p, min_p):
+        return B.fused_lmhead_merge(partials, rows, vocab_total, targets, temperature, top_k,
+                                    top_p, min_p)
 
     @staticmethod
     def weight_sum(rows, row_weight, device):
@@ -66,3 +82,22 @@ def sharded_entropy_mean(entropy_sum, valid_count, group=None):
                    valid_count.to(torch.float64).reshape(1)])
     dist.all_reduce(t, group=group)
     return torch.where(t[1] > 0, t[0] / t[1].clamp(min=1.0), torch.zeros_like(t[0]))
+
+
+def tp_fused_lmhead_score(hidden, weight_shard, vocab_begin, vocab_total, targets, temperature,
+                          top_k, top_p, min_p, group=None, ops=LibraryOps):
+    """Fused-head scoring with the vocabulary split across the ranks of
+    `group`: rank r holds weight rows [vocab_begin, vocab_begin + rows of
+    weight_shard), and the shards are in rank order.  Every rank returns the
+    outputs of fused_lmhead_score over the whole vocabulary.
+
+    Steps: this rank's partial block -> all-gather of the blocks (rank
+    order) -> the merge."""
+    block = ops.lmhead_partial(hidden, weight_shard, vocab_begin, vocab_total, targets,
+                               temperature, top_k)
+    world = dist.get_world_size(group)
+    parts = [torch.empty_like(block) for _ in range(world)]
+    dist.all_gather(parts, block, group=group)
+    gathered = torch.stack(parts)
+    return ops.lmhead_merge(gathered, hidden.shape[0], vocab_total, targets, temperature, top_k,
+                            top_p, min_p)

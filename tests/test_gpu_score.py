@@ -156,7 +156,7 @@ def test_ragged_rows_all_filters_without_mask(filt):
     logits = workloads.random_logits(rows, vocab, 3.0, seed=13, dtype="bf16", ld=ld)
     temp = workloads.uniform(rows, 0.6, 1.2, 13, 7).astype(F32)
     targets = workloads.integers(rows, 0, vocab, 13, 8).astype(np.int32)
-    _run_nomask(logits[:, :vocab].copy(), targets, temp, *filt)
+    _run_nomask(logits, targets, temp, *filt, vocab=vocab)
 
 
 def test_all_negative_rows():
@@ -426,24 +426,25 @@ def test_replay_backward_full_size_sampled_rows():
     compare_grad(dl[torch.from_numpy(sel).cuda()].cpu().numpy()[:, :vocab], gref)
 
 
-def _run_nomask(logits, targets, temperature, top_k, top_p, min_p):
+def _run_nomask(logits, targets, temperature, top_k, top_p, min_p, vocab=None):
     """GPU forward as a caller with no support mask and no saved state asks
     for it (the tie cut at the threshold is then resolved for the target
     alone), against the oracle on every row: logprobs and entropies over the
     full vocabulary and over the support; boundary rows by the prefix rule
     (the support rebuilt from the GPU's support size)."""
-    rows, vocab = logits.shape
+    rows, ld = logits.shape
+    vocab = ld if vocab is None else vocab
     t_np = np.asarray(temperature, F32)
     k_arg = torch.from_numpy(np.asarray(top_k, np.int32)).cuda() if np.ndim(top_k) else top_k
     out = vsb.score_fwd(to_device(logits), torch.from_numpy(np.asarray(targets, np.int32)).cuda(),
                         temperature=torch.from_numpy(t_np).cuda() if t_np.ndim else float(t_np),
                         top_k=k_arg, top_p=float(F32(top_p)), min_p=float(F32(min_p)),
-                        want_entropy=True)
+                        want_entropy=True, vocab=vocab)
     torch.cuda.synchronize()
     t64 = t_np.astype(np.float64)
     ref = oracle.score(logits, targets, temperature=t64 if t64.ndim else float(t64),
                        top_k=np.asarray(top_k, np.int32) if np.ndim(top_k) else top_k,
-                       top_p=float(F32(top_p)), min_p=float(F32(min_p)))
+                       top_p=float(F32(top_p)), min_p=float(F32(min_p)), vocab=vocab)
     nb, nd = compare_scores(out, ref, logits, vocab, t64 if t64.ndim else np.full(rows, float(t64)),
                             np.asarray(targets, np.int32), top_k, top_p, min_p)
     sure = ~((ref["topp_margin"] < 1e-6) | (ref["minp_margin"] < 1e-6))

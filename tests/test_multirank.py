@@ -145,3 +145,62 @@ def test_two_rank_sharded_distance_loss_and_gradient():
         assert out[r][2] == pytest.approx(ref["loss_num"], rel=1e-12)
         assert out[r][3] == pytest.approx(ref["loss_den"], rel=1e-12)
         assert out[r][4] == pytest.approx((1.5 + 2.5) / (2 + 3))
+
+
+class _RecordOps:
+    """Stand-ins for the two library steps of the vocabulary-parallel head
+    (they need a GPU): the partial step writes a block naming its rank and
+    shard, the merge step returns what it was given, so the test sees the
+    exchange itself."""
+
+    @staticmethod
+    def lmhead_partial(hidden, weight_shard, vocab_begin, vocab_total, targets, temperature,
+                       top_k):
+        import torch
+
+        blk = torch.zeros(64, dtype=torch.uint8)
+        blk[0] = dist.get_rank()
+        blk[1] = vocab_begin // 100
+        blk[2] = weight_shard.shape[0] // 100
+        return blk
+
+    @staticmethod
+    def lmhead_merge(partials, rows, vocab_total, targets, temperature, top_k, top_p, min_p):
+        return partials
+
+
+def _tp_worker(rank, world, port, out):
+    sys.path.insert(0, str(ROOT))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+
+    import torch
+
+    from sampling_support_b200 import dist as vdist
+
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        begin = [0, 700][rank]
+        shard = torch.zeros((700 if rank == 0 else 300, 4))
+        g = vdist.tp_fused_lmhead_score(torch.zeros((5, 4)), shard, begin, 1000,
+                                        torch.zeros(5, dtype=torch.int32), 1.0, 8, 0.9, 0.0,
+                                        ops=_RecordOps)
+        out[rank] = g.numpy().copy()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_vocabulary_parallel_exchange():
+    """Every rank ends with every rank's partial block, in rank (= shard)
+    order, which is what the merge step reads."""
+    world = 2
+    port = _free_port()
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.start_processes(_tp_worker, args=(world, port, out), nprocs=world, join=True,
+                       start_method="spawn")
+    for r in (0, 1):
+        g = out[r]
+        assert g.shape == (2, 64)
+        assert g[0, :3].tolist() == [0, 0, 7] and g[1, :3].tolist() == [1, 7, 3]
