@@ -335,7 +335,25 @@ __device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
   return *reinterpret_cast<const uint32_t*>(&r);
 }
 
-// One 8-element bf16 vector into online statistics s (and the max raw value).
+// The eight elements of a bf16 vector into s one by one, the max-valued
+// ones counted apart (the vector reaches or raises s's maximum, or holds a
+// NaN: rare once the maximum is seeded, so kept out of line).
+static __device__ __noinline__ Stats stats_vec_bf16_scalar(uint32_t w0, uint32_t w1, uint32_t w2,
+                                                   uint32_t w3, float c, Stats s) {
+  const uint32_t w[4] = {w0, w1, w2, w3};
+  float u[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    u[2 * i] = __fmul_rn(__uint_as_float(w[i] << 16), c);
+    u[2 * i + 1] = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), c);
+  }
+  stats_add(s, u);
+  return s;
+}
+
+// One 8-element bf16 vector into online statistics s (and the max raw
+// value).  A vector below s's maximum takes a packed fp32x2 path:
+// d = x c - m in one fused step, 2^d, and the sums.
 __device__ __forceinline__ void stats_vec_bf16(const uint4& q, float c, f32x2 c2, Stats& s,
                                                float& vmax) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
@@ -343,27 +361,19 @@ __device__ __forceinline__ void stats_vec_bf16(const uint4& q, float c, f32x2 c2
   const float bmv = fmaxf(__uint_as_float(mm << 16), __uint_as_float(mm & 0xFFFF0000u));
   vmax = fmaxf(vmax, bmv);
   const float bm = __fmul_rn(bmv, c);
-  if (bm > s.m) {
-    if (s.c0 != 0.f || s.zr != 0.f) stats_rebase(s, bm);
-    s.m = bm;
-  }
-  if (bm == s.m || !(bm == bm)) {
-    // the vector holds this chain's running maximum (or NaN): scalar, with
-    // the max-valued elements counted apart
-    float u[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      u[2 * i] = __fmul_rn(__uint_as_float(w[i] << 16), c);
-      u[2 * i + 1] = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), c);
+  if (bm >= s.m || !(bm == bm)) {
+    if (bm > s.m) {
+      if (s.c0 != 0.f || s.zr != 0.f) stats_rebase(s, bm);
+      s.m = bm;
     }
-    stats_add(s, u);
+    s = stats_vec_bf16_scalar(w[0], w[1], w[2], w[3], c, s);
   } else {
-    const f32x2 m2 = pack2(s.m, s.m);
+    const f32x2 nm2 = pack2(-s.m, -s.m);
     f32x2 zr2 = pack2(0.f, 0.f), a2 = pack2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const f32x2 x2 = pack2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
-      const f32x2 d2 = sub2(mul2(x2, c2), m2);
+      const f32x2 d2 = fma2(x2, c2, nm2);
       float d0, d1;
       unpack2(d2, d0, d1);
       const f32x2 e2 = pack2(ex2(d0), ex2(d1));

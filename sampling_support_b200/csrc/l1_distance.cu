@@ -21,7 +21,7 @@ namespace vs {
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 
 struct L1Shared {
@@ -93,13 +93,17 @@ __device__ __forceinline__ float bf16_at(const uint32_t (&w)[4], int i) {
 }
 
 // One element of pass 2: accumulates |p - q| and p sign(p - q) and returns
-// the in-place (p, sign) word (branch-free form of enc_ps).
+// the in-place (p, sign) word: p (in [0, 1], so bits 31 and 30 of its fp32
+// pattern are clear) with bit 31 = the sign bit of p - q and bit 30 set when
+// p == q (sign 0).
 __device__ __forceinline__ uint32_t l1_step(float p, float q, float& l1, float& ps) {
   const float d = p - q;
   l1 += fabsf(d);
-  const bool pos = d > 0.f, neg = d < 0.f;
-  ps = fmaf(p, pos ? 1.f : (neg ? -1.f : 0.f), ps);
-  return __float_as_uint(p) | (neg ? 0x80000000u : 0u) | (!(pos || neg) ? 0x40000000u : 0u);
+  const uint32_t sbit = __float_as_uint(d) & 0x80000000u;
+  const bool zero = d == 0.f;
+  const float s = zero ? 0.f : __uint_as_float(sbit | 0x3F800000u);  // sign(d)
+  ps = fmaf(p, s, ps);
+  return __float_as_uint(p) | sbit | (zero ? 0x40000000u : 0u);
 }
 
 // Gradient of one element from its (p, sign) word: k_pos, k_neg, k_zero are
@@ -141,42 +145,32 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
   vd = l1_block_max(vd, sh.fred);
   vt = l1_block_max(vt, sh.fred);
 
-  // pass 1
+  // pass 1: sum of 2^(x log2 e - m) over the slice, one fused step per
+  // element pair (draft and target go through the same code, so identical
+  // rows give identical sums)
   const float md = __fmul_rn(vd, kLog2e), mt = __fmul_rn(vt, kLog2e);
   {
     const f32x2 nmd = pack2(-md, -md), nmt = pack2(-mt, -mt);
     f32x2 zd = pack2(0.f, 0.f), zt = pack2(0.f, 0.f);
-    // A vector holding the slice max takes the exact scalar form, so that a
-    // max-valued element contributes exactly 1 (u - m computed without
-    // fusion); the others take the packed fused form.
-    auto zsum = [&](const uint4& a, float vmax, float m, f32x2 nm, f32x2& z) {
-      const uint32_t wa[4] = {a.x, a.y, a.z, a.w};
-      if (vec_max(a) == vmax) {
-        float zs = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          zs += ex2(__fsub_rn(__fmul_rn(bf16_at(wa, i), kLog2e), m));
-        z = add2(z, pack2(zs, 0.f));
-      } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float e0, e1;
-          unpack2(fma2(pack2(__uint_as_float(wa[i] << 16), __uint_as_float(wa[i] & 0xFFFF0000u)), l2e, nm), e0, e1);
-          z = add2(z, pack2(ex2(e0), ex2(e1)));
-        }
-      }
-    };
     for (int v = tid; v < nfull; v += kThreads) {
-      zsum(d4[v], vd, md, nmd, zd);
-      zsum(t4[v], vt, mt, nmt, zt);
+      const uint4 a = d4[v], b = t4[v];
+      const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float e0, e1, f0, f1;
+        unpack2(fma2(pack2(__uint_as_float(wa[i] << 16), __uint_as_float(wa[i] & 0xFFFF0000u)), l2e, nmd), e0, e1);
+        unpack2(fma2(pack2(__uint_as_float(wb[i] << 16), __uint_as_float(wb[i] & 0xFFFF0000u)), l2e, nmt), f0, f1);
+        zd = add2(zd, pack2(ex2(e0), ex2(e1)));
+        zt = add2(zt, pack2(ex2(f0), ex2(f1)));
+      }
     }
     float z0, z1, y0, y1;
     unpack2(zd, z0, z1);
     unpack2(zt, y0, y1);
     float sz = z0 + z1, sy = y0 + y1;
     for (int j = nfull * 8 + tid; j < n; j += kThreads) {
-      sz += ex2(__fsub_rn(__fmul_rn(value_of(bd[j]), kLog2e), md));
-      sy += ex2(__fsub_rn(__fmul_rn(value_of(bt[j]), kLog2e), mt));
+      sz += ex2(fmaf(value_of(bd[j]), kLog2e, -md));
+      sy += ex2(fmaf(value_of(bt[j]), kLog2e, -mt));
     }
     Stats sd{md, 0.f, sz, 0.f}, st{mt, 0.f, sy, 0.f};
     if (vd == -kInf && sz == 0.f) sd = stats_empty();
@@ -203,7 +197,8 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
   const float ld2 = stats_log2z(Sd), lt2 = stats_log2z(St);
   const float cd = Sd.m + ld2, ct = St.m + lt2;
 
-  // pass 2
+  // pass 2: p and q in one fused step per element (the same code for both
+  // rows), |p - q| and p sign(p - q), and (p, sign) in place for pass 3
   float l1 = 0.f, ps = 0.f;
   const bool keep = P.grad != nullptr;
   uint4* d4w = reinterpret_cast<uint4*>(bd);
@@ -214,38 +209,28 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
       const uint4 a = d4[v], b = t4[v];
       const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
       uint32_t enc[8];
-      if (__fmul_rn(vec_max(a), kLog2e) == Sd.m || __fmul_rn(vec_max(b), kLog2e) == St.m) {
-        // a row max: the exact scalar form (p = 1 exactly for a single token)
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          enc[i] = l1_step(ex2(__fsub_rn(__fsub_rn(__fmul_rn(bf16_at(wa, i), kLog2e), Sd.m), ld2)),
-                           ex2(__fsub_rn(__fsub_rn(__fmul_rn(bf16_at(wb, i), kLog2e), St.m), lt2)),
-                           l1, ps);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float p0, p1, q0, q1;
-          unpack2(fma2(pack2(__uint_as_float(wa[i] << 16), __uint_as_float(wa[i] & 0xFFFF0000u)), l2e, ncd), p0, p1);
-          unpack2(fma2(pack2(__uint_as_float(wb[i] << 16), __uint_as_float(wb[i] & 0xFFFF0000u)), l2e, nct), q0, q1);
-          enc[2 * i] = l1_step(ex2(p0), ex2(q0), l1, ps);
-          enc[2 * i + 1] = l1_step(ex2(p1), ex2(q1), l1, ps);
-        }
+      for (int i = 0; i < 4; ++i) {
+        float p0, p1, q0, q1;
+        unpack2(fma2(pack2(__uint_as_float(wa[i] << 16), __uint_as_float(wa[i] & 0xFFFF0000u)), l2e, ncd), p0, p1);
+        unpack2(fma2(pack2(__uint_as_float(wb[i] << 16), __uint_as_float(wb[i] & 0xFFFF0000u)), l2e, nct), q0, q1);
+        enc[2 * i] = l1_step(ex2(p0), ex2(q0), l1, ps);
+        enc[2 * i + 1] = l1_step(ex2(p1), ex2(q1), l1, ps);
       }
       if (keep) {
         uint32_t hi[4], lo[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          hi[i] = (enc[2 * i] >> 16) | (enc[2 * i + 1] & 0xFFFF0000u);
-          lo[i] = (enc[2 * i] & 0xFFFFu) | (enc[2 * i + 1] << 16);
+          hi[i] = __byte_perm(enc[2 * i], enc[2 * i + 1], 0x7632);
+          lo[i] = __byte_perm(enc[2 * i], enc[2 * i + 1], 0x5410);
         }
         d4w[v] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
         t4w[v] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
     }
     for (int j = nfull * 8 + tid; j < n; j += kThreads) {
-      const uint32_t e = l1_step(ex2(__fsub_rn(__fsub_rn(__fmul_rn(value_of(bd[j]), kLog2e), Sd.m), ld2)),
-                                 ex2(__fsub_rn(__fsub_rn(__fmul_rn(value_of(bt[j]), kLog2e), St.m), lt2)),
-                                 l1, ps);
+      const uint32_t e = l1_step(ex2(fmaf(value_of(bd[j]), kLog2e, -cd)),
+                                 ex2(fmaf(value_of(bt[j]), kLog2e, -ct)), l1, ps);
       if (keep) {
         bd[j] = static_cast<uint16_t>(e >> 16);
         bt[j] = static_cast<uint16_t>(e & 0xFFFFu);

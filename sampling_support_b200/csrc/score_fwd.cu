@@ -123,17 +123,41 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
     const uint4* g4 = reinterpret_cast<const uint4*>(grow);
     int v = tid;
     if constexpr (sizeof(Raw) == 2) {
-      // packed statistics, four chains, kRecUnroll vectors in flight
+      // packed statistics, four chains, kRecUnroll vectors in flight; the
+      // block maximum of every thread's first round seeds the chains'
+      // running maximum, so that later vectors rarely raise it
       Stats f4[4] = {stats_empty(), stats_empty(), stats_empty(), stats_empty()};
       const f32x2 c2 = pack2(c, c);
-      for (; v + (kRecUnroll - 1) * kRecThreads < nfull; v += kRecUnroll * kRecThreads) {
-        uint4 q[kRecUnroll];
+      uint4 q[kRecUnroll];
+      uint32_t mx = 0xFF80FF80u;  // (-inf, -inf)
 #pragma unroll
-        for (int k = 0; k < kRecUnroll; ++k) q[k] = __ldcs(g4 + v + k * kRecThreads);
-#pragma unroll
-        for (int k = 0; k < kRecUnroll; ++k) stats_vec_bf16(q[k], c, c2, f4[k & 3], fvmax);
+      for (int k = 0; k < kRecUnroll; ++k) {
+        const int vk = v + k * kRecThreads;
+        q[k] = vk < nfull ? __ldcs(g4 + vk) : make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u);
+        mx = bmax2(mx, bmax2(bmax2(q[k].x, q[k].y), bmax2(q[k].z, q[k].w)));
       }
-      for (; v < nfull; v += kRecThreads) stats_vec_bf16(__ldcs(g4 + v), c, c2, f4[0], fvmax);
+      float m1 = fmaxf(__uint_as_float(mx << 16), __uint_as_float(mx & 0xFFFF0000u));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+      if ((tid & 31) == 0) fred[tid >> 5] = m1;
+      __syncthreads();
+      m1 = -kInf;
+      for (int i = 0; i < kRecThreads / 32; ++i) m1 = fmaxf(m1, fred[i]);
+      __syncthreads();
+#pragma unroll
+      for (int k = 0; k < 4; ++k) f4[k].m = __fmul_rn(m1, c);
+      for (;;) {
+#pragma unroll
+        for (int k = 0; k < kRecUnroll; ++k)
+          if (v + k * kRecThreads < nfull) stats_vec_bf16(q[k], c, c2, f4[k & 3], fvmax);
+        v += kRecUnroll * kRecThreads;
+        if (v >= nfull) break;
+#pragma unroll
+        for (int k = 0; k < kRecUnroll; ++k) {
+          const int vk = v + k * kRecThreads;
+          q[k] = vk < nfull ? __ldcs(g4 + vk) : make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
       f = f4[0];
       stats_merge(f, f4[1]);
       stats_merge(f, f4[2]);

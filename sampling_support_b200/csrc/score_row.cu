@@ -175,15 +175,34 @@ __device__ __forceinline__ void red_inc(uint32_t a) {
 
 // Count the eight elements of one vector: in-window elements into their bin,
 // the others into this lane's spill bin (bins >= the window's bin count are
-// never read), so there is no predicate or branch.
+// never read), so there is no predicate or branch.  For the sign-specific
+// windows both elements of a 32-bit word are indexed at once with 16-bit
+// lane arithmetic (add.u16x2, min.u16x2): kWinPos adds -base to the raw
+// bits, kWinNeg adds -(lowest key) to their complement (0xFFFF - r is the
+// key of a negative value); out-of-window values land at 16-bit indices of
+// at least the bin count and clamp to the spill bin.
 template <int MODE>
 __device__ __forceinline__ void hist_vec(const uint4& q, uint32_t base, uint32_t spill,
                                          uint32_t hist_s) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+  if constexpr (MODE == kWinPos || MODE == kWinNeg) {
+    // 16-bit offsets, replicated in both halves
+    const uint32_t off = MODE == kWinPos ? ((0u - base) & 0xFFFFu) : ((0u - (0xFFFFu - base)) & 0xFFFFu);
+    const uint32_t off2 = off | (off << 16), sp2 = spill | (spill << 16);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    red_inc(hist_s + (min(win_index<MODE>(w[i] & 0xFFFFu, base), spill) << 2));
-    red_inc(hist_s + (min(win_index<MODE>(w[i] >> 16, base), spill) << 2));
+    for (int i = 0; i < 4; ++i) {
+      uint32_t x = MODE == kWinNeg ? ~w[i] : w[i];
+      asm("add.u16x2 %0, %1, %2;" : "=r"(x) : "r"(x), "r"(off2));
+      asm("min.u16x2 %0, %1, %2;" : "=r"(x) : "r"(x), "r"(sp2));
+      red_inc(hist_s + ((x & 0xFFFFu) << 2));
+      red_inc(hist_s + ((x >> 16) << 2));
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      red_inc(hist_s + (min(win_index<MODE>(w[i] & 0xFFFFu, base), spill) << 2));
+      red_inc(hist_s + (min(win_index<MODE>(w[i] >> 16, base), spill) << 2));
+    }
   }
 }
 
@@ -487,11 +506,17 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
   ring.pass(0, ring.nst(), [&](const Raw* st, int n, int base) {
     if constexpr (kBf16) {
       const uint16_t* st16 = reinterpret_cast<const uint16_t*>(st);
-      if (hist_on && base == 0) {
-        // fix the window from the first stage's maximum (a lower bound of
-        // the row maximum m): elements below the level found with it are
-        // below the level of m as well
+      if (base == 0) {
+        // the first stage's maximum m0, a lower bound of the row maximum m,
+        // seeds every chain's running maximum (so that later vectors rarely
+        // raise it and take the packed path)
         const float m0 = stage_max_bf16(st16, n, sh.fred);
+        const float u0 = __fmul_rn(m0, c);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) s4[k].m = u0;
+        if (hist_on) {
+        // fix the window from m0: elements below the level found with it are
+        // below the level of m as well
         const uint32_t kref = key_of(static_cast<uint16_t>(__float_as_uint(m0) >> 16));
         wtop = min(kref + kWinHi, KT::kInfKey);
         wlo = wtop >= static_cast<uint32_t>(kWin - 1) ? wtop - (kWin - 1) : 0u;
@@ -514,6 +539,7 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
         const int nb = static_cast<int>(wtop - wlo) + 1;
         for (int b = tid; b < nb; b += kRT) hist[b] = 0u;
         __syncthreads();
+        }
       }
       const uint32_t spill = (wtop - wlo) + 1u + (tid & 31);
       if (wmode == kWinPos)
@@ -661,7 +687,7 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
       const int per = (w.nbins + kRT - 1) / kRT;
       const int i0 = tid * per, i1 = min(w.nbins, i0 + per);
       for (int i = i0; i < i1; ++i) {
-        const uint32_t cnt = hist[i];
+        const uint32_t cnt = w.hist[i];
         const uint32_t key = w.klo + i;
         if (cnt && key > tkey) {
           const float d = key_u(key, c) - m;
@@ -675,7 +701,7 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
           sums.sa = fmaf(fc * d, e, sums.sa);
         }
       }
-      if (tid == 0) sums.neq = hist[tkey - w.klo];
+      if (tid == 0) sums.neq = w.hist[tkey - w.klo];
     } else {
       const uint32_t t = tkey;
       auto one = [&](Raw raw) {
