@@ -176,8 +176,11 @@ __device__ __forceinline__ Stats shfl_xor(const Stats& s, int lane_mask) {
 // Deterministic block reduction; result valid in every thread.  `scratch`
 // holds at least blockDim.x / 32 entries.  The block max comes first, then
 // every thread rebases its own statistics onto it once and plain sums
-// follow (no chain of rebases).
+// follow (no chain of rebases).  Per phase: warp shuffles, one partial per
+// warp, warp 0 reduces the partials (a fixed order) and broadcasts.
 __device__ __forceinline__ Stats block_reduce(Stats s, Stats* scratch) {
+  __shared__ float s_m;
+  __shared__ Stats s_res;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nw = blockDim.x >> 5;
   float m = s.m;
@@ -185,9 +188,14 @@ __device__ __forceinline__ Stats block_reduce(Stats s, Stats* scratch) {
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if (lane == 0) scratch[warp].m = m;
   __syncthreads();
-  m = -kInf;
-  for (int w = 0; w < nw; ++w) m = fmaxf(m, scratch[w].m);
+  if (warp == 0) {
+    float x = lane < nw ? scratch[lane].m : -kInf;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    if (lane == 0) s_m = x;
+  }
   __syncthreads();
+  m = s_m;
   if (s.c0 != 0.f || s.zr != 0.f) stats_rebase(s, m);
   float c0 = s.c0, zr = s.zr, a = s.a;
 #pragma unroll
@@ -198,28 +206,43 @@ __device__ __forceinline__ Stats block_reduce(Stats s, Stats* scratch) {
   }
   if (lane == 0) scratch[warp] = Stats{m, c0, zr, a};
   __syncthreads();
-  Stats t{m, 0.f, 0.f, 0.f};
-  for (int w = 0; w < nw; ++w) {
-    t.c0 += scratch[w].c0;
-    t.zr += scratch[w].zr;
-    t.a += scratch[w].a;
+  if (warp == 0) {
+    float x0 = 0.f, x1 = 0.f, x2 = 0.f;
+    if (lane < nw) {
+      x0 = scratch[lane].c0;
+      x1 = scratch[lane].zr;
+      x2 = scratch[lane].a;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      x0 += __shfl_xor_sync(0xffffffffu, x0, o);
+      x1 += __shfl_xor_sync(0xffffffffu, x1, o);
+      x2 += __shfl_xor_sync(0xffffffffu, x2, o);
+    }
+    if (lane == 0) s_res = Stats{m, x0, x1, x2};
   }
   __syncthreads();
-  return t;
+  return s_res;
 }
 
+// Sum of v over the block, valid in every thread (warp shuffles, one
+// partial per warp in `scratch`, warp 0 reduces them in a fixed order).
 template <typename T>
 __device__ __forceinline__ T block_sum(T v, T* scratch) {
+  __shared__ T s_res;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   if (lane == 0) scratch[warp] = v;
   __syncthreads();
-  T t = 0;
-  const int nw = blockDim.x >> 5;
-  for (int w = 0; w < nw; ++w) t += scratch[w];
+  if (warp == 0) {
+    T x = lane < static_cast<int>(blockDim.x >> 5) ? scratch[lane] : T(0);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    if (lane == 0) s_res = x;
+  }
   __syncthreads();
-  return t;
+  return s_res;
 }
 
 // ---------------------------------------------------------------------------
@@ -351,24 +374,54 @@ static __device__ __noinline__ Stats stats_vec_bf16_scalar(uint32_t w0, uint32_t
   return s;
 }
 
-// One 8-element bf16 vector into online statistics s (and the max raw
-// value).  A vector below s's maximum takes a packed fp32x2 path:
-// d = x c - m in one fused step, 2^d, and the sums.
-__device__ __forceinline__ void stats_vec_bf16(const uint4& q, float c, f32x2 c2, Stats& s,
-                                               float& vmax) {
+// A statistics chain over bf16 vectors with its running maximum also kept as
+// raw bf16 bits in both halves of a word, so that the per-vector test "does
+// any element reach the maximum" is one packed bf16x2 comparison.
+struct Chain {
+  Stats s;
+  uint32_t thr2;  // raw bf16 of the value whose fl(value c) is s.m, both halves
+};
+
+__device__ __forceinline__ Chain chain_empty() { return Chain{stats_empty(), 0xFF80FF80u}; }
+
+// Start a chain at the value v (a lower bound of the maximum of the data it
+// will see): no element counted yet.
+__device__ __forceinline__ void chain_seed(Chain& ch, float v, float c) {
+  const uint32_t r = __float_as_uint(v) >> 16;
+  ch.s = Stats{__fmul_rn(v, c), 0.f, 0.f, 0.f};
+  ch.thr2 = r | (r << 16);
+}
+
+// True when an element of the packed pair mm is >= the threshold pair (NaN
+// compares false: it reaches the sums through the packed path).
+__device__ __forceinline__ bool any_ge_bf16x2(uint32_t mm, uint32_t thr2) {
+  uint32_t r;
+  asm("{\n .reg .pred p, q;\n setp.ge.bf16x2 p|q, %1, %2;\n selp.u32 %0, 1, 0, p;\n"
+      " @q mov.u32 %0, 1;\n}\n"
+      : "=r"(r)
+      : "r"(mm), "r"(thr2));
+  return r != 0u;
+}
+
+// One 8-element bf16 vector into the chain; vmax2 keeps the running maximum
+// of the raw values (packed bf16x2).
+__device__ __forceinline__ void chain_vec(const uint4& q, float c, f32x2 c2, Chain& ch,
+                                          uint32_t& vmax2) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
   const uint32_t mm = bmax2(bmax2(w[0], w[1]), bmax2(w[2], w[3]));
-  const float bmv = fmaxf(__uint_as_float(mm << 16), __uint_as_float(mm & 0xFFFF0000u));
-  vmax = fmaxf(vmax, bmv);
-  const float bm = __fmul_rn(bmv, c);
-  if (bm >= s.m || !(bm == bm)) {
-    if (bm > s.m) {
-      if (s.c0 != 0.f || s.zr != 0.f) stats_rebase(s, bm);
-      s.m = bm;
+  vmax2 = bmax2(vmax2, mm);
+  if (any_ge_bf16x2(mm, ch.thr2)) {
+    const float bmv = fmaxf(__uint_as_float(mm << 16), __uint_as_float(mm & 0xFFFF0000u));
+    const float bm = __fmul_rn(bmv, c);
+    if (bm > ch.s.m) {
+      if (ch.s.c0 != 0.f || ch.s.zr != 0.f) stats_rebase(ch.s, bm);
+      ch.s.m = bm;
+      const uint32_t r = __float_as_uint(bmv) >> 16;
+      ch.thr2 = r | (r << 16);
     }
-    s = stats_vec_bf16_scalar(w[0], w[1], w[2], w[3], c, s);
+    ch.s = stats_vec_bf16_scalar(w[0], w[1], w[2], w[3], c, ch.s);
   } else {
-    const f32x2 nm2 = pack2(-s.m, -s.m);
+    const f32x2 nm2 = pack2(-ch.s.m, -ch.s.m);
     f32x2 zr2 = pack2(0.f, 0.f), a2 = pack2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -383,9 +436,14 @@ __device__ __forceinline__ void stats_vec_bf16(const uint4& q, float c, f32x2 c2
     float z0, z1, a0, a1;
     unpack2(zr2, z0, z1);
     unpack2(a2, a0, a1);
-    s.zr += z0 + z1;
-    s.a += a0 + a1;
+    ch.s.zr += z0 + z1;
+    ch.s.a += a0 + a1;
   }
+}
+
+// Largest value of a packed bf16x2 running maximum.
+__device__ __forceinline__ float vmax_of(uint32_t vmax2) {
+  return fmaxf(__uint_as_float(vmax2 << 16), __uint_as_float(vmax2 & 0xFFFF0000u));
 }
 
 }  // namespace vs

@@ -296,6 +296,25 @@ __device__ __forceinline__ float pick32(const float (&v)[32], int i) {
   return (i & 16) ? d1 : d0;
 }
 
+// Work unit u -> (row unit mu, vocabulary split sp).  Units go in groups of
+// at most kUnitGroup row units: a group's units of every split come before
+// the next group's, so the units running at the same time share a few
+// vocabulary splits (their weight tiles are read once from DRAM and then
+// from L2) and at most kUnitGroup row blocks of the hidden states (which
+// stay in L2 while the group sweeps the vocabulary).
+constexpr int kUnitGroup = 16;
+
+__device__ __forceinline__ void unit_coords(int u, const LmParams& P, int& mu, int& sp) {
+  const int gsz = P.m_units < kUnitGroup ? P.m_units : kUnitGroup;
+  const int per_group = gsz * P.splits;
+  const int g = u / per_group;
+  const int r = u - g * per_group;
+  const int g0 = g * gsz;
+  const int gn = P.m_units - g0 < gsz ? P.m_units - g0 : gsz;  // the last group may be smaller
+  mu = g0 + r % gn;
+  sp = r / gn;
+}
+
 template <bool PAIR, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     lmhead_gemm_kernel(const __grid_constant__ CUtensorMap map_h,
@@ -367,7 +386,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int u = u_first; u < units && ok; u += u_step) {
-        const int mu = u % P.m_units, sp = u / P.m_units;
+        int mu, sp;
+        unit_coords(u, P, mu, sp);
         const int mb = PAIR ? 2 * mu + static_cast<int>(rank) : mu;
         const int t0 = sp * P.tiles_per_split, t1 = min(P.n_tiles, t0 + P.tiles_per_split);
         for (int t = t0; t < t1 && ok; ++t) {
@@ -401,7 +421,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0, tile = 0;
       bool ok = true;
       for (int u = u_first; u < units && ok; u += u_step) {
-        const int sp = u / P.m_units;
+        int mu, sp;
+        unit_coords(u, P, mu, sp);
         const int t0 = sp * P.tiles_per_split, t1 = min(P.n_tiles, t0 + P.tiles_per_split);
         for (int t = t0; t < t1 && ok; ++t, ++tile) {
           const int b = tile & 1;
@@ -460,7 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t tile = 0;
     bool ok = true;
     for (int u = u_first; u < units && ok; u += u_step) {
-      const int mu = u % P.m_units, sp = u / P.m_units;
+      int mu, sp;
+      unit_coords(u, P, mu, sp);
       const int mb = PAIR ? 2 * mu + static_cast<int>(rank) : mu;
       const int t0 = sp * P.tiles_per_split, t1 = min(P.n_tiles, t0 + P.tiles_per_split);
       const int row = mb * kBM + r;
@@ -525,7 +547,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t tile = 0;
     bool ok = true;
     for (int u = u_first; u < units && ok; u += u_step) {
-      const int mu = u % P.m_units, sp = u / P.m_units;
+      int mu, sp;
+      unit_coords(u, P, mu, sp);
       const int mb = PAIR ? 2 * mu + static_cast<int>(rank) : mu;
       const int t0 = sp * P.tiles_per_split, t1 = min(P.n_tiles, t0 + P.tiles_per_split);
       const int row = mb * kBM + r;

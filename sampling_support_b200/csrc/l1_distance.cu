@@ -21,7 +21,7 @@ namespace vs {
 
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 
 struct L1Shared {
@@ -30,9 +30,40 @@ struct L1Shared {
   Stats gathered[8][2];
   Stats red[kWarps];
   float fred[kWarps];
+  float2 red2[kWarps];
+  float2 res2;
   float agg_l1, agg_ps;
   uint32_t timeout;
 };
+
+// Two values reduced over the block at once: warp shuffles, one partial per
+// warp in shared memory, warp 0 reduces the partials and broadcasts the
+// result (two barriers).  MAX selects the maximum, else the sum; the sum's
+// order is fixed, so it is deterministic.
+template <bool MAX>
+__device__ __forceinline__ float2 block_reduce2(float a, float b, L1Shared& sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float oa = __shfl_xor_sync(0xffffffffu, a, o), ob = __shfl_xor_sync(0xffffffffu, b, o);
+    a = MAX ? fmaxf(a, oa) : a + oa;
+    b = MAX ? fmaxf(b, ob) : b + ob;
+  }
+  if (lane == 0) sh.red2[warp] = make_float2(a, b);
+  __syncthreads();
+  if (warp == 0) {
+    float2 x = lane < kWarps ? sh.red2[lane] : make_float2(MAX ? -kInf : 0.f, MAX ? -kInf : 0.f);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float oa = __shfl_xor_sync(0xffffffffu, x.x, o), ob = __shfl_xor_sync(0xffffffffu, x.y, o);
+      x.x = MAX ? fmaxf(x.x, oa) : x.x + oa;
+      x.y = MAX ? fmaxf(x.y, ob) : x.y + ob;
+    }
+    if (lane == 0) sh.res2 = x;
+  }
+  __syncthreads();
+  return sh.res2;
+}
 
 struct L1Params {
   int32_t rows, vocab;
@@ -142,12 +173,16 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
     vd = fmaxf(vd, value_of(bd[j]));
     vt = fmaxf(vt, value_of(bt[j]));
   }
-  vd = l1_block_max(vd, sh.fred);
-  vt = l1_block_max(vt, sh.fred);
+  {
+    const float2 mm = block_reduce2<true>(vd, vt, sh);
+    vd = mm.x;
+    vt = mm.y;
+  }
 
-  // pass 1: sum of 2^(x log2 e - m) over the slice, one fused step per
-  // element pair (draft and target go through the same code, so identical
-  // rows give identical sums)
+  // pass 1: sum of 2^(x log2 e - m) over the slice, with x log2 e rounded
+  // before the subtraction (a max-valued element gives exactly 2^0); draft
+  // and target go through the same code, so identical rows give identical
+  // sums
   const float md = __fmul_rn(vd, kLog2e), mt = __fmul_rn(vt, kLog2e);
   {
     const f32x2 nmd = pack2(-md, -md), nmt = pack2(-mt, -mt);
@@ -158,8 +193,8 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         float e0, e1, f0, f1;
-        unpack2(fma2(pack2(__uint_as_float(wa[i] << 16), __uint_as_float(wa[i] & 0xFFFF0000u)), l2e, nmd), e0, e1);
-        unpack2(fma2(pack2(__uint_as_float(wb[i] << 16), __uint_as_float(wb[i] & 0xFFFF0000u)), l2e, nmt), f0, f1);
+        unpack2(add2(mul2(pack2(__uint_as_float(wa[i] << 16), __uint_as_float(wa[i] & 0xFFFF0000u)), l2e), nmd), e0, e1);
+        unpack2(add2(mul2(pack2(__uint_as_float(wb[i] << 16), __uint_as_float(wb[i] & 0xFFFF0000u)), l2e), nmt), f0, f1);
         zd = add2(zd, pack2(ex2(e0), ex2(e1)));
         zt = add2(zt, pack2(ex2(f0), ex2(f1)));
       }
@@ -169,14 +204,13 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
     unpack2(zt, y0, y1);
     float sz = z0 + z1, sy = y0 + y1;
     for (int j = nfull * 8 + tid; j < n; j += kThreads) {
-      sz += ex2(fmaf(value_of(bd[j]), kLog2e, -md));
-      sy += ex2(fmaf(value_of(bt[j]), kLog2e, -mt));
+      sz += ex2(__fmul_rn(value_of(bd[j]), kLog2e) - md);
+      sy += ex2(__fmul_rn(value_of(bt[j]), kLog2e) - mt);
     }
-    Stats sd{md, 0.f, sz, 0.f}, st{mt, 0.f, sy, 0.f};
-    if (vd == -kInf && sz == 0.f) sd = stats_empty();
-    if (vt == -kInf && sy == 0.f) st = stats_empty();
-    sd = block_reduce(sd, sh.red);
-    st = block_reduce(st, sh.red);
+    const float2 zz = block_reduce2<false>(sz, sy, sh);
+    Stats sd{md, 0.f, zz.x, 0.f}, st{mt, 0.f, zz.y, 0.f};
+    if (vd == -kInf && zz.x == 0.f) sd = stats_empty();
+    if (vt == -kInf && zz.y == 0.f) st = stats_empty();
     if (tid == 0) {
       sh.part[0] = sd;
       sh.part[1] = st;
@@ -197,8 +231,9 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
   const float ld2 = stats_log2z(Sd), lt2 = stats_log2z(St);
   const float cd = Sd.m + ld2, ct = St.m + lt2;
 
-  // pass 2: p and q in one fused step per element (the same code for both
-  // rows), |p - q| and p sign(p - q), and (p, sign) in place for pass 3
+  // pass 2: p = 2^(fl(x log2 e) - (m + log2 Z)) and q alike (the same code
+  // for both rows; a one-element row gets p = q = 1 exactly), |p - q| and
+  // p sign(p - q), and (p, sign) in place for pass 3
   float l1 = 0.f, ps = 0.f;
   const bool keep = P.grad != nullptr;
   uint4* d4w = reinterpret_cast<uint4*>(bd);
@@ -212,8 +247,8 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         float p0, p1, q0, q1;
-        unpack2(fma2(pack2(__uint_as_float(wa[i] << 16), __uint_as_float(wa[i] & 0xFFFF0000u)), l2e, ncd), p0, p1);
-        unpack2(fma2(pack2(__uint_as_float(wb[i] << 16), __uint_as_float(wb[i] & 0xFFFF0000u)), l2e, nct), q0, q1);
+        unpack2(add2(mul2(pack2(__uint_as_float(wa[i] << 16), __uint_as_float(wa[i] & 0xFFFF0000u)), l2e), ncd), p0, p1);
+        unpack2(add2(mul2(pack2(__uint_as_float(wb[i] << 16), __uint_as_float(wb[i] & 0xFFFF0000u)), l2e), nct), q0, q1);
         enc[2 * i] = l1_step(ex2(p0), ex2(q0), l1, ps);
         enc[2 * i + 1] = l1_step(ex2(p1), ex2(q1), l1, ps);
       }
@@ -229,19 +264,20 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
       }
     }
     for (int j = nfull * 8 + tid; j < n; j += kThreads) {
-      const uint32_t e = l1_step(ex2(fmaf(value_of(bd[j]), kLog2e, -cd)),
-                                 ex2(fmaf(value_of(bt[j]), kLog2e, -ct)), l1, ps);
+      const uint32_t e = l1_step(ex2(__fmul_rn(value_of(bd[j]), kLog2e) - cd),
+                                 ex2(__fmul_rn(value_of(bt[j]), kLog2e) - ct), l1, ps);
       if (keep) {
         bd[j] = static_cast<uint16_t>(e >> 16);
         bt[j] = static_cast<uint16_t>(e & 0xFFFFu);
       }
     }
   }
-  l1 = block_sum(l1, sh.fred);
-  ps = block_sum(ps, sh.fred);
-  if (tid == 0) {
-    sh.agg_l1 = l1;
-    sh.agg_ps = ps;
+  {
+    const float2 lp = block_reduce2<false>(l1, ps, sh);
+    if (tid == 0) {
+      sh.agg_l1 = lp.x;
+      sh.agg_ps = lp.y;
+    }
   }
   cluster.sync();
   float L1 = 0.f, PS = 0.f;

@@ -126,7 +126,8 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
       // packed statistics, four chains, kRecUnroll vectors in flight; the
       // block maximum of every thread's first round seeds the chains'
       // running maximum, so that later vectors rarely raise it
-      Stats f4[4] = {stats_empty(), stats_empty(), stats_empty(), stats_empty()};
+      Chain f4[4] = {chain_empty(), chain_empty(), chain_empty(), chain_empty()};
+      uint32_t vm2 = 0xFF80FF80u;
       const f32x2 c2 = pack2(c, c);
       uint4 q[kRecUnroll];
       uint32_t mx = 0xFF80FF80u;  // (-inf, -inf)
@@ -145,11 +146,11 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
       for (int i = 0; i < kRecThreads / 32; ++i) m1 = fmaxf(m1, fred[i]);
       __syncthreads();
 #pragma unroll
-      for (int k = 0; k < 4; ++k) f4[k].m = __fmul_rn(m1, c);
+      for (int k = 0; k < 4; ++k) chain_seed(f4[k], m1, c);
       for (;;) {
 #pragma unroll
         for (int k = 0; k < kRecUnroll; ++k)
-          if (v + k * kRecThreads < nfull) stats_vec_bf16(q[k], c, c2, f4[k & 3], fvmax);
+          if (v + k * kRecThreads < nfull) chain_vec(q[k], c, c2, f4[k & 3], vm2);
         v += kRecUnroll * kRecThreads;
         if (v >= nfull) break;
 #pragma unroll
@@ -158,10 +159,11 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
           q[k] = vk < nfull ? __ldcs(g4 + vk) : make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      f = f4[0];
-      stats_merge(f, f4[1]);
-      stats_merge(f, f4[2]);
-      stats_merge(f, f4[3]);
+      f = f4[0].s;
+      stats_merge(f, f4[1].s);
+      stats_merge(f, f4[2].s);
+      stats_merge(f, f4[3].s);
+      fvmax = fmaxf(fvmax, vmax_of(vm2));
     } else {
       for (; v + 3 * kRecThreads < nfull; v += 4 * kRecThreads) {
         uint4 q[4];
@@ -314,6 +316,290 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
   }
 }
 
+// ---------------------------------------------------------------------------
+// recorded support, narrow lists (width <= 64): one warp per row for the
+// gather and the support statistics, 16 rows per 512-thread CTA; the rows
+// that need full-vocabulary statistics (an empty support, or all rows when
+// they are requested) are then streamed one after another by the whole CTA.
+
+constexpr int kWarpRows = 16;           // rows per CTA, one per warp
+constexpr int kWarpRowThreads = 512;
+constexpr int kWarpRowMaxWidth = 64;    // two list slots per lane
+constexpr int kStreamUnroll = 8;        // 16-byte loads in flight per thread (full-row stream)
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <typename Raw>
+__global__ void __launch_bounds__(kWarpRowThreads, 1) score_recorded_warp_kernel(ScoreParams P) {
+  constexpr int VEC = 16 / sizeof(Raw);
+  __shared__ uint32_t need_full[kWarpRows];
+  __shared__ Stats fstat[kWarpRows];
+  __shared__ float fmaxv[kWarpRows];
+  __shared__ Stats red[kWarpRowThreads / 32];
+  __shared__ float fred[kWarpRowThreads / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * kWarpRows + warp;
+  const bool row_ok = row < P.rows;
+  const int V = P.vocab;
+  const int W = P.support_width;
+  const uint32_t lt = (1u << lane) - 1u;
+
+  // ---- phase A (warp per row): ids, dedup, gather, support statistics
+  const Raw* grow = static_cast<const Raw*>(P.logits) + static_cast<int64_t>(row_ok ? row : 0) * P.ld;
+  const int32_t* srow = P.support_ids + static_cast<int64_t>(row_ok ? row : 0) * P.support_ld;
+  const float T = row_ok ? (P.temperature ? P.temperature[row] : P.temperature_scalar) : 1.f;
+  const float c = kLog2e / T;
+  const int y = row_ok ? P.targets[row] : -1;
+  const bool target_ok = y >= 0 && y < V;
+  int32_t id0 = -1, id1 = -1;
+  if (row_ok && lane < W) id0 = srow[lane];
+  if (row_ok && lane + 32 < W) id1 = srow[lane + 32];
+  const bool bad0 = id0 < -1 || id0 >= V, bad1 = id1 < -1 || id1 >= V;
+  bool dup0 = (__match_any_sync(0xffffffffu, id0) & lt) != 0u;
+  bool dup1 = (__match_any_sync(0xffffffffu, id1) & lt) != 0u;
+  if (W > 32) {
+    // a second-slot id repeats any first-slot id (an earlier slot)
+    for (int l = 0; l < 32; ++l) dup1 |= __shfl_sync(0xffffffffu, id0, l) == id1;
+  }
+  const bool keep0 = id0 >= 0 && !bad0 && !dup0, keep1 = id1 >= 0 && !bad1 && !dup1;
+  uint32_t flags = 0;
+  if (__any_sync(0xffffffffu, bad0 || bad1)) flags |= VS_ROW_BAD_SUPPORT_ID;
+  if (__any_sync(0xffffffffu, (dup0 && id0 >= 0 && !bad0) || (dup1 && id1 >= 0 && !bad1)))
+    flags |= VS_ROW_DUP_SUPPORT_ID;
+  const float nanf_ = __int_as_float(0x7fc00000);
+  const float x0 = keep0 ? value_of(grow[id0]) : nanf_;
+  const float x1 = keep1 ? value_of(grow[id1]) : nanf_;
+  const uint32_t nkeep = __popc(__ballot_sync(0xffffffffu, keep0)) + __popc(__ballot_sync(0xffffffffu, keep1));
+  const bool any_nf = __any_sync(0xffffffffu, (keep0 && !isfinite(x0)) || (keep1 && !isfinite(x1)));
+  const bool hit = __any_sync(0xffffffffu, (keep0 && id0 == y) || (keep1 && id1 == y));
+  const bool empty = nkeep == 0;
+  // support statistics relative to the support maximum (value domain)
+  const float vsmax = warp_max(fmaxf(keep0 ? x0 : -kInf, keep1 ? x1 : -kInf));
+  Stats s{vsmax, 0.f, 0.f, 0.f};
+  {
+    float c0 = 0.f, zr = 0.f, a = 0.f;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const bool kp = k == 0 ? keep0 : keep1;
+      if (!kp) continue;
+      const float x = k == 0 ? x0 : x1;
+      const float d = (x - vsmax) * c;
+      const float e = ex2(d);
+      if (d == 0.f)
+        c0 += 1.f;
+      else
+        zr += e;
+      a = fmaf(d, e, a);
+    }
+    s.c0 = warp_sum(c0);
+    s.zr = warp_sum(zr);
+    s.a = warp_sum(a);
+  }
+  const bool need = row_ok && (empty || P.full_stats);
+  if (lane == 0) need_full[warp] = need ? 1u : 0u;
+  __syncthreads();
+
+  // ---- phase B (whole CTA, one row at a time): full-vocabulary statistics
+  for (int r = 0; r < kWarpRows; ++r) {
+    if (!need_full[r]) continue;  // uniform
+    const int rr = blockIdx.x * kWarpRows + r;
+    const Raw* g = static_cast<const Raw*>(P.logits) + static_cast<int64_t>(rr) * P.ld;
+    const float Tr = P.temperature ? P.temperature[rr] : P.temperature_scalar;
+    const float cr = kLog2e / Tr;
+    const int nfull = V / VEC;
+    const uint4* g4 = reinterpret_cast<const uint4*>(g);
+    Stats f = stats_empty();
+    float fv = -kInf;
+    int v = threadIdx.x;
+    if constexpr (sizeof(Raw) == 2) {
+      Chain f4[2] = {chain_empty(), chain_empty()};
+      uint32_t vm2 = 0xFF80FF80u;
+      const f32x2 c2 = pack2(cr, cr);
+      uint4 q[kStreamUnroll];
+      uint32_t mx = 0xFF80FF80u;
+#pragma unroll
+      for (int k = 0; k < kStreamUnroll; ++k) {
+        const int vk = v + k * kWarpRowThreads;
+        q[k] = vk < nfull ? __ldcs(g4 + vk) : make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u);
+        mx = bmax2(mx, bmax2(bmax2(q[k].x, q[k].y), bmax2(q[k].z, q[k].w)));
+      }
+      float m1 = warp_max(fmaxf(__uint_as_float(mx << 16), __uint_as_float(mx & 0xFFFF0000u)));
+      if (lane == 0) fred[warp] = m1;
+      __syncthreads();
+      m1 = -kInf;
+      for (int i = 0; i < kWarpRowThreads / 32; ++i) m1 = fmaxf(m1, fred[i]);
+      __syncthreads();
+      chain_seed(f4[0], m1, cr);
+      chain_seed(f4[1], m1, cr);
+      for (;;) {
+#pragma unroll
+        for (int k = 0; k < kStreamUnroll; ++k)
+          if (v + k * kWarpRowThreads < nfull) chain_vec(q[k], cr, c2, f4[k & 1], vm2);
+        v += kStreamUnroll * kWarpRowThreads;
+        if (v >= nfull) break;
+#pragma unroll
+        for (int k = 0; k < kStreamUnroll; ++k) {
+          const int vk = v + k * kWarpRowThreads;
+          q[k] = vk < nfull ? __ldcs(g4 + vk) : make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      f = f4[0].s;
+      stats_merge(f, f4[1].s);
+      fv = fmaxf(fv, vmax_of(vm2));
+    } else {
+      for (; v < nfull; v += kWarpRowThreads) {
+        Raw rw[VEC];
+        unpack(__ldcs(g4 + v), rw);
+        float u[VEC];
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) {
+          const float x = value_of(rw[i]);
+          fv = fmaxf(fv, x);
+          u[i] = __fmul_rn(x, cr);
+        }
+        stats_add(f, u);
+      }
+    }
+    for (int j = nfull * VEC + threadIdx.x; j < V; j += kWarpRowThreads) {
+      const float x = value_of(g[j]);
+      fv = fmaxf(fv, x);
+      float u[1] = {__fmul_rn(x, cr)};
+      stats_add(f, u);
+    }
+    f = block_reduce(f, red);
+    fv = warp_max(fv);
+    if (lane == 0) fred[warp] = fv;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float t = -kInf;
+      for (int i = 0; i < kWarpRowThreads / 32; ++i) t = fmaxf(t, fred[i]);
+      fstat[r] = f;
+      fmaxv[r] = t;
+    }
+    __syncthreads();
+  }
+  if (!row_ok) return;
+
+  // ---- phase C (warp per row): outputs
+  Stats f = stats_empty();
+  float fvmax = -kInf;
+  if (need) {
+    f = fstat[warp];
+    fvmax = fmaxv[warp];
+  }
+  const float nan = __int_as_float(0x7fc00000);
+  if (lane == 0) {
+    uint32_t status = flags;
+    bool nonfinite = any_nf;
+    float m2 = nan, log2z = nan, h_full = nan;
+    if (need) {
+      if (!stats_finite(f)) nonfinite = true;
+      m2 = f.m;
+      log2z = stats_log2z(f);
+      h_full = kLn2 * (log2z - f.a / stats_z(f));
+    }
+    const float log2zs = empty ? nan : stats_log2z(s);
+    const float h_sup = empty ? 0.f : kLn2 * (log2zs - s.a / stats_z(s));
+    float lp_v = nan, lp_s = nan;
+    bool in_s = false;
+    if (!target_ok) status |= VS_ROW_TARGET_OUT_OF_RANGE;
+    if (nonfinite) {
+      status |= VS_ROW_NONFINITE_INPUT;
+    } else if (target_ok) {
+      const float xy = value_of(grow[y]);
+      const float uy = __fmul_rn(xy, c);
+      if (need) lp_v = kLn2 * (uy - m2 - log2z);
+      in_s = hit;
+      if (empty) {
+        lp_s = lp_v;
+      } else if (in_s) {
+        lp_s = kLn2 * ((xy - vsmax) * c - log2zs);
+      } else {
+        lp_s = -kInf;
+        status |= VS_ROW_TARGET_NOT_IN_SUPPORT;
+      }
+    }
+    const bool valid = !nonfinite && !empty;
+    if (P.lp_full) P.lp_full[row] = lp_v;
+    if (P.lp_support) P.lp_support[row] = lp_s;
+    if (P.want_entropy) {
+      if (P.h_full) P.h_full[row] = nonfinite ? nan : h_full;
+      if (P.h_support) P.h_support[row] = nonfinite ? nan : h_sup;
+    }
+    if (P.valid) P.valid[row] = valid ? 1 : 0;
+    if (P.status) P.status[row] = status;
+    if (P.support_size) P.support_size[row] = nonfinite ? 0 : static_cast<int32_t>(nkeep);
+    if (P.ctx) {
+      RowCtx cx{};
+      cx.m2 = fvmax;  // value domain (the stream's sums are relative to fl(fvmax c))
+      cx.log2z = log2z;
+      cx.msup = vsmax;
+      cx.log2zs = log2zs;
+      cx.h_full = h_full;
+      cx.h_support = h_sup;
+      cx.c = c;
+      cx.tkey = 0;
+      cx.tie_cut = 0;
+      uint32_t fl = kCtxRecorded;
+      if (need) fl |= kCtxFullStats;
+      if (nonfinite) fl |= kCtxNonFinite;
+      if (empty || nonfinite) fl |= kCtxEmpty;
+      if (target_ok) fl |= kCtxTargetOk;
+      if (in_s) fl |= kCtxTargetInS;
+      cx.flags = fl;
+      cx.n_support = nonfinite ? 0 : static_cast<int32_t>(nkeep);
+      cx.status = status;
+      cx.c0_full = f.c0;
+      cx.zr_full = f.zr;
+      cx.c0_sup = s.c0;
+      cx.zr_sup = s.zr;
+      P.ctx[row] = cx;
+    }
+  }
+  // seeded Gumbel-max token over the kept ids
+  if (P.sampled) {
+    unsigned long long best = 0ull;
+    if (!empty && !any_nf && !(need && !stats_finite(f))) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const bool kp = k == 0 ? keep0 : keep1;
+        if (!kp) continue;
+        const int32_t id = k == 0 ? id0 : id1;
+        float gg[4];
+        gumbel4(P.sample_seed, static_cast<uint32_t>(P.row_base + row), static_cast<uint64_t>(id) >> 2, gg);
+        const unsigned long long key = gumbel_key(gumbel_score(k == 0 ? x0 : x1, T, gg[id & 3]), id);
+        best = key > best ? key : best;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long ob = __shfl_xor_sync(0xffffffffu, best, o);
+      best = ob > best ? ob : best;
+    }
+    if (lane == 0) P.sampled[row] = gumbel_key_id(best);
+  }
+  // support bitmask: clear the row, then set the kept ids
+  if (P.support_mask) {
+    const int64_t wstride = (V + 31) / 32;
+    uint32_t* mrow = P.support_mask + static_cast<int64_t>(row) * wstride;
+    for (int64_t w = lane; w < wstride; w += 32) mrow[w] = 0u;
+    __syncwarp();
+    if (!any_nf) {
+      if (keep0) atomicOr(&mrow[id0 >> 5], 1u << (id0 & 31));
+      if (keep1) atomicOr(&mrow[id1 >> 5], 1u << (id1 & 31));
+    }
+  }
+}
+
 // Deterministic reduction of the entropy sum and valid count over rows.
 __global__ void score_reduce_kernel(const float* h_support, const uint8_t* valid, int rows,
                                     double* entropy_sum, int32_t* valid_count) {
@@ -360,10 +646,17 @@ int score_max_vocab(vs_dtype dtype) {
 }
 
 cudaError_t launch_score_recorded(const ScoreParams& p, vs_dtype dtype, cudaStream_t s) {
-  if (dtype == VS_BF16)
+  if (p.support_width <= kWarpRowMaxWidth) {
+    const unsigned grid = static_cast<unsigned>((p.rows + kWarpRows - 1) / kWarpRows);
+    if (dtype == VS_BF16)
+      score_recorded_warp_kernel<uint16_t><<<grid, kWarpRowThreads, 0, s>>>(p);
+    else
+      score_recorded_warp_kernel<uint32_t><<<grid, kWarpRowThreads, 0, s>>>(p);
+  } else if (dtype == VS_BF16) {
     score_recorded_kernel<uint16_t><<<p.rows, kRecThreads, 0, s>>>(p);
-  else
+  } else {
     score_recorded_kernel<uint32_t><<<p.rows, kRecThreads, 0, s>>>(p);
+  }
   return cudaGetLastError();
 }
 

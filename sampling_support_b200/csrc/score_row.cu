@@ -43,7 +43,8 @@ namespace vs {
 
 namespace {
 
-constexpr int kRT = 512;        // threads per row
+constexpr int kRT = 1024;       // threads per row
+constexpr int kGrp = kRT / 2;   // threads per half (statistics warps / histogram warps)
 constexpr int kRW = kRT / 32;   // warps
 constexpr int kNStages = 6;     // ring depth
 constexpr int kStageBytes = 32768;
@@ -292,44 +293,55 @@ __device__ Desc descend(Ring<Raw>& ring, float c, float m, int fx_shift, bool by
 // ---------------------------------------------------------------------------
 // the streamed pass
 
-// bf16 stage: statistics (four vectors per thread in flight, each with its
-// own chain) and, unless MODE is kWinNone, the window histogram.
-template <int MODE>
-__device__ __forceinline__ void stage_bf16(const uint16_t* st, int n, float c, Stats (&s)[4],
-                                           float& vmax, uint32_t base, uint32_t spill,
-                                           uint32_t hist_s) {
+// bf16 stage, statistics: the group's `gsize` threads (thread `g` of the
+// group) take every gsize-th 16-byte vector, two in flight, alternating two
+// chains.
+__device__ __forceinline__ void stats_stage_bf16(const uint16_t* st, int n, float c, Chain (&ch)[2],
+                                                 uint32_t& vmax2, int g, int gsize) {
   const int nv = n / 8;
   const uint4* v4 = reinterpret_cast<const uint4*>(st);
   const f32x2 c2 = pack2(c, c);
-  int v = threadIdx.x;
-  for (; v + 3 * kRT < nv; v += 4 * kRT) {
-    uint4 q[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) q[k] = v4[v + k * kRT];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      stats_vec_bf16(q[k], c, c2, s[k], vmax);
-      if constexpr (MODE != kWinNone) hist_vec<MODE>(q[k], base, spill, hist_s);
-    }
+  int v = g;
+  for (; v + gsize < nv; v += 2 * gsize) {
+    const uint4 q0 = v4[v], q1 = v4[v + gsize];
+    chain_vec(q0, c, c2, ch[0], vmax2);
+    chain_vec(q1, c, c2, ch[1], vmax2);
   }
-  for (; v < nv; v += kRT) {
-    const uint4 q = v4[v];
-    stats_vec_bf16(q, c, c2, s[0], vmax);
-    if constexpr (MODE != kWinNone) hist_vec<MODE>(q, base, spill, hist_s);
-  }
-  for (int j = nv * 8 + threadIdx.x; j < n; j += kRT) {
+  if (v < nv) chain_vec(v4[v], c, c2, ch[0], vmax2);
+  for (int j = nv * 8 + g; j < n; j += gsize) {
     const uint32_t r = st[j];
     const float x = value_of(static_cast<uint16_t>(r));
-    vmax = fmaxf(vmax, x);
+    vmax2 = bmax2(vmax2, r | (r << 16));
     float u[1] = {__fmul_rn(x, c)};
-    stats_add(s[0], u);
-    if constexpr (MODE != kWinNone) red_inc(hist_s + (min(win_index<MODE>(r, base), spill) << 2));
+    stats_add(ch[0].s, u);
   }
 }
 
-__device__ __forceinline__ void stats_stage_f32(const uint32_t* st, int n, float c, Stats (&s4)[4],
+// bf16 stage, histogram: the group's threads count every element of the
+// stage into the window (see hist_vec), four vectors in flight.
+template <int MODE>
+__device__ __forceinline__ void hist_stage_bf16(const uint16_t* st, int n, uint32_t base,
+                                                uint32_t spill, uint32_t hist_s, int g, int gsize) {
+  const int nv = n / 8;
+  const uint4* v4 = reinterpret_cast<const uint4*>(st);
+  int v = g;
+  for (; v + 3 * gsize < nv; v += 4 * gsize) {
+    uint4 q[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) q[k] = v4[v + k * gsize];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) hist_vec<MODE>(q[k], base, spill, hist_s);
+  }
+  for (; v < nv; v += gsize) hist_vec<MODE>(v4[v], base, spill, hist_s);
+  for (int j = nv * 8 + g; j < n; j += gsize) {
+    const uint32_t r = st[j];
+    red_inc(hist_s + (min(win_index<MODE>(r, base), spill) << 2));
+  }
+}
+
+__device__ __forceinline__ void stats_stage_f32(const uint32_t* st, int n, float c, Stats (&s2)[2],
                                                 float& vmax) {
-  Stats& s = s4[0];
+  Stats& s = s2[0];
   const int nv = n / 4;
   const uint4* v4 = reinterpret_cast<const uint4*>(st);
   for (int v = threadIdx.x; v < nv; v += kRT) {
@@ -496,7 +508,9 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
 
   // ---- the streamed pass: online statistics and the row maximum; for a
   // filtered bf16 row also the exact-key window histogram
-  Stats s4[4] = {stats_empty(), stats_empty(), stats_empty(), stats_empty()};
+  Chain ch2[2] = {chain_empty(), chain_empty()};  // bf16 rows
+  uint32_t vmax2 = 0xFF80FF80u;                    // bf16 rows: packed running max
+  Stats s2[2] = {stats_empty(), stats_empty()};    // fp32 rows
   float vmax = -kInf;
   const bool hist_on = kBf16 && any_filter;
   uint32_t wtop = 0, wlo = 0;  // window keys [wlo, wtop]
@@ -511,9 +525,8 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
         // seeds every chain's running maximum (so that later vectors rarely
         // raise it and take the packed path)
         const float m0 = stage_max_bf16(st16, n, sh.fred);
-        const float u0 = __fmul_rn(m0, c);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) s4[k].m = u0;
+        chain_seed(ch2[0], m0, c);
+        chain_seed(ch2[1], m0, c);
         if (hist_on) {
         // fix the window from m0: elements below the level found with it are
         // below the level of m as well
@@ -541,24 +554,35 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
         __syncthreads();
         }
       }
+      // with a window, the first half of the warps takes the statistics and
+      // the second half the histogram of the same stage; without, every
+      // warp takes the statistics
       const uint32_t spill = (wtop - wlo) + 1u + (tid & 31);
-      if (wmode == kWinPos)
-        stage_bf16<kWinPos>(st16, n, c, s4, vmax, wbase, spill, hist_s);
-      else if (wmode == kWinNeg)
-        stage_bf16<kWinNeg>(st16, n, c, s4, vmax, wbase, spill, hist_s);
-      else if (wmode == kWinKey)
-        stage_bf16<kWinKey>(st16, n, c, s4, vmax, wbase, spill, hist_s);
-      else
-        stage_bf16<kWinNone>(st16, n, c, s4, vmax, 0u, 0u, 0u);
+      if (wmode == kWinNone) {
+        stats_stage_bf16(st16, n, c, ch2, vmax2, tid, kRT);
+      } else if (tid < kGrp) {
+        stats_stage_bf16(st16, n, c, ch2, vmax2, tid, kGrp);
+      } else if (wmode == kWinPos) {
+        hist_stage_bf16<kWinPos>(st16, n, wbase, spill, hist_s, tid - kGrp, kGrp);
+      } else if (wmode == kWinNeg) {
+        hist_stage_bf16<kWinNeg>(st16, n, wbase, spill, hist_s, tid - kGrp, kGrp);
+      } else {
+        hist_stage_bf16<kWinKey>(st16, n, wbase, spill, hist_s, tid - kGrp, kGrp);
+      }
     } else {
-      stats_stage_f32(st, n, c, s4, vmax);
+      stats_stage_f32(st, n, c, s2, vmax);
     }
     return false;
   });
-  Stats s = s4[0];
-  stats_merge(s, s4[1]);
-  stats_merge(s, s4[2]);
-  stats_merge(s, s4[3]);
+  Stats s;
+  if constexpr (kBf16) {
+    s = ch2[0].s;
+    stats_merge(s, ch2[1].s);
+    vmax = vmax_of(vmax2);
+  } else {
+    s = s2[0];
+    stats_merge(s, s2[1]);
+  }
   s = block_reduce(s, sh.wst);
   vmax = block_max(vmax, sh.fred);
 

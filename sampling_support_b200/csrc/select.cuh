@@ -52,10 +52,12 @@ struct SelShared {
   uint32_t b_key;
   u64 b_above_cnt, b_above_mass, b_at_cnt, b_at_mass;
   int32_t b_found;
+  int32_t i_total;  // block_excl_int: the block total
 };
 
 // Exclusive suffix sums of (a, b) over the threads of the block, thread
-// order = ascending.  Every thread calls.
+// order = ascending.  Every thread calls.  Warp 0 turns the warps' totals
+// into per-warp exclusive suffixes.
 template <int NT>
 __device__ __forceinline__ void block_suffix_excl(u64 a, u64 b, u64& ea, u64& eb,
                                                   SelShared<NT / 32>& sh) {
@@ -76,13 +78,27 @@ __device__ __forceinline__ void block_suffix_excl(u64 a, u64 b, u64& ea, u64& eb
     sh.scan_b[warp] = ib;
   }
   __syncthreads();
-  u64 wa = 0, wb = 0;
-  for (int w = warp + 1; w < NW; ++w) {
-    wa += sh.scan_a[w];
-    wb += sh.scan_b[w];
+  if (warp == 0) {
+    // inclusive suffix over the warps' totals, then exclusive
+    const u64 ta0 = lane < NW ? sh.scan_a[lane] : 0ull, tb0 = lane < NW ? sh.scan_b[lane] : 0ull;
+    u64 xa = ta0, xb = tb0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const u64 ya = __shfl_down_sync(0xffffffffu, xa, o);
+      const u64 yb = __shfl_down_sync(0xffffffffu, xb, o);
+      if (lane + o < 32) {
+        xa += ya;
+        xb += yb;
+      }
+    }
+    if (lane < NW) {
+      sh.scan_a[lane] = xa - ta0;
+      sh.scan_b[lane] = xb - tb0;
+    }
   }
-  ea = wa + ia - a;
-  eb = wb + ib - b;
+  __syncthreads();
+  ea = sh.scan_a[warp] + ia - a;
+  eb = sh.scan_b[warp] + ib - b;
   __syncthreads();
 }
 
@@ -99,12 +115,20 @@ __device__ __forceinline__ int block_excl_int(int v, int& total, SelShared<NT / 
   }
   if (lane == 31) sh.iscan[warp] = incl;
   __syncthreads();
-  int pre = 0;
-  total = 0;
-  for (int w = 0; w < NW; ++w) {
-    if (w < warp) pre += sh.iscan[w];
-    total += sh.iscan[w];
+  if (warp == 0) {
+    const int t0 = lane < NW ? sh.iscan[lane] : 0;
+    int x = t0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane < NW) sh.iscan[lane] = x - t0;  // exclusive prefix of the warp totals
+    if (lane == 31) sh.i_total = x;
   }
+  __syncthreads();
+  const int pre = sh.iscan[warp];
+  total = sh.i_total;
   __syncthreads();
   return pre + incl - v;
 }

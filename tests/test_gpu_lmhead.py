@@ -103,7 +103,10 @@ def test_fused_head_per_row_temperature_single_row():
 def test_lmhead_workload_full_size_sampled_rows():
     wl = workloads.lmhead()
     rows = wl["rows"]
-    sel = np.sort(np.random.default_rng(0).choice(rows, 12, replace=False))
+    # one row in every 256-row unit (the pair-mode row block), at a seeded
+    # offset, and the last row
+    off = np.random.default_rng(0).integers(0, 256, rows // 256)
+    sel = np.unique(np.concatenate([np.arange(rows // 256) * 256 + off, [rows - 1]]))
     nb, n = _check(wl["hidden_states"], wl["weight"], wl["targets"], wl["temperature"],
                    wl["top_k"], wl["top_p"], wl["min_p"], rows_checked=sel)
     print(f"lmhead full size: {nb} boundary rows of {n} checked")
