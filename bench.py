@@ -21,6 +21,7 @@ sample of the same workload instead.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -50,6 +51,27 @@ def peaks():
         return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
                     bf16_sustained=float(d["bf16_tflops_sustained"]), src="measured")
     return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, src="fallback")
+
+
+def source_digest(rel: str) -> str:
+    return hashlib.sha256((ROOT / rel).read_bytes()).hexdigest()[:16]
+
+
+def measured_traffic(key: str):
+    """DRAM bytes (read + write) per launch from an ncu capture recorded in
+    profiles/traffic.json, or None when the kernel's sources have changed
+    since the counters were taken (each entry lists the digests of the files
+    it was built from)."""
+    tp = ROOT / "profiles" / "traffic.json"
+    if not tp.exists():
+        return None, "no capture recorded"
+    e = json.loads(tp.read_text()).get(key)
+    if not isinstance(e, dict):
+        return None, "no capture recorded"
+    stale = [f for f, d in e.get("sources", {}).items() if source_digest(f) != d]
+    if stale:
+        return None, "kernel changed since the capture: " + ", ".join(stale)
+    return e["bytes_per_launch"], e.get("capture", "")
 
 
 # ---------------------------------------------------------------------------
@@ -886,10 +908,7 @@ def main():
     if world > 1:
         barrier(world)
     if rank == 0:
-        traffic = None
-        tp = ROOT / "profiles" / "traffic.json"
-        if tp.exists():
-            traffic = json.loads(tp.read_text()).get("score_call_fullvocab")
+        traffic, traffic_note = measured_traffic("score_row_kernel_fullvocab")
         line = {
             "metric": METRIC, "value": h["value"], "unit": "rows/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": h["ms_per_step"],
@@ -907,7 +926,8 @@ def main():
                          "kernel": "score_row_kernel<bf16> (one launch per call; CUDA-graph replays "
                                    "of back-to-back calls, events around the timed region)",
                          "algorithmic_bytes": h["in_bytes"],
-                         "kernel_ms": h["kernel_ms"], "peak_source": pk["src"] + " (MEASURED_PEAKS hbm_gbs)"},
+                         "kernel_ms": h["kernel_ms"], "traffic_source": traffic_note,
+                         "peak_source": pk["src"] + " (MEASURED_PEAKS hbm_gbs)"},
             "clocks": h["clocks"],
             "e2e": h["e2e"],
             "gpu_launches": args.steps,  # one score_row_kernel launch per call

@@ -38,6 +38,7 @@
 #include "internal.h"
 #include "gumbel.cuh"
 #include "select.cuh"
+#include "window.cuh"
 
 namespace vs {
 
@@ -52,13 +53,6 @@ constexpr int kWin = kSelWin;
 constexpr int kBins = kSelBins;
 constexpr uint32_t kWinHi = 256;  // window keys above the first stage's maximum
 constexpr int kCountUnroll = 8;   // 16-byte loads in flight per thread (tie count)
-
-// Support sums: counts above the threshold, of its tie group and of the
-// max-valued elements; mass and (u - m)-weighted mass of the others.
-struct SupSums {
-  uint32_t ngt, neq, ntp;
-  float smass, sa;
-};
 
 struct RowSh {
   uint64_t full[kNStages];
@@ -148,64 +142,6 @@ struct Ring {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
   }
 };
-
-// ---------------------------------------------------------------------------
-// the exact-key window (bf16)
-
-enum WinMode : int { kWinNone = 0, kWinPos = 1, kWinNeg = 2, kWinKey = 3 };
-
-// Window index of the raw bf16 bits r (>= the bin count outside the window).
-// kWinPos (every window key is a positive value): base = raw bits of the
-// lowest window key, and negative values wrap to huge indices; kWinNeg
-// (every window key is a negative value): base = raw bits of the lowest
-// window key (the most negative value); kWinKey: base = lowest window key.
-template <int MODE>
-__device__ __forceinline__ uint32_t win_index(uint32_t r, uint32_t base) {
-  if constexpr (MODE == kWinPos)
-    return r - base;
-  else if constexpr (MODE == kWinNeg)
-    return base - r;
-  else
-    return key_of(static_cast<uint16_t>(r)) - base;
-}
-
-// One shared-memory count increment at the 32-bit shared address a.
-__device__ __forceinline__ void red_inc(uint32_t a) {
-  asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(a) : "memory");
-}
-
-// Count the eight elements of one vector: in-window elements into their bin,
-// the others into this lane's spill bin (bins >= the window's bin count are
-// never read), so there is no predicate or branch.  For the sign-specific
-// windows both elements of a 32-bit word are indexed at once with 16-bit
-// lane arithmetic (add.u16x2, min.u16x2): kWinPos adds -base to the raw
-// bits, kWinNeg adds -(lowest key) to their complement (0xFFFF - r is the
-// key of a negative value); out-of-window values land at 16-bit indices of
-// at least the bin count and clamp to the spill bin.
-template <int MODE>
-__device__ __forceinline__ void hist_vec(const uint4& q, uint32_t base, uint32_t spill,
-                                         uint32_t hist_s) {
-  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-  if constexpr (MODE == kWinPos || MODE == kWinNeg) {
-    // 16-bit offsets, replicated in both halves
-    const uint32_t off = MODE == kWinPos ? ((0u - base) & 0xFFFFu) : ((0u - (0xFFFFu - base)) & 0xFFFFu);
-    const uint32_t off2 = off | (off << 16), sp2 = spill | (spill << 16);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint32_t x = MODE == kWinNeg ? ~w[i] : w[i];
-      asm("add.u16x2 %0, %1, %2;" : "=r"(x) : "r"(x), "r"(off2));
-      asm("min.u16x2 %0, %1, %2;" : "=r"(x) : "r"(x), "r"(sp2));
-      red_inc(hist_s + ((x & 0xFFFFu) << 2));
-      red_inc(hist_s + ((x >> 16) << 2));
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      red_inc(hist_s + (min(win_index<MODE>(w[i] & 0xFFFFu, base), spill) << 2));
-      red_inc(hist_s + (min(win_index<MODE>(w[i] >> 16, base), spill) << 2));
-    }
-  }
-}
 
 // ---------------------------------------------------------------------------
 // general radix descent (fp32 keys, or a window miss)
@@ -389,19 +325,6 @@ __device__ __forceinline__ float stage_max_bf16(const uint16_t* st, int n, float
   return block_max(m, scratch);
 }
 
-// Smallest key in [lo, hi] whose u-offset from m reaches dlo (hi if none).
-__device__ __forceinline__ uint32_t key_at_level(uint32_t lo, uint32_t hi, float c, float m,
-                                                 float dlo) {
-  while (lo < hi) {
-    const uint32_t mid = lo + ((hi - lo) >> 1);
-    if (key_u(mid, c) - m >= dlo)
-      hi = mid;
-    else
-      lo = mid + 1;
-  }
-  return lo;
-}
-
 __device__ __forceinline__ SupSums block_sum_sup(SupSums v, RowSh& sh) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -539,16 +462,7 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
           if (use_p && pp > 0.f) dlo = fmaxf(dlo, log2f((1.f - pp) / static_cast<float>(V)) - 2.f);
           if (dlo > -kInf) wlo = key_at_level(wlo, wtop, c, __fmul_rn(m0, c), dlo);
         }
-        if (wlo > 0x7FFFu) {
-          wmode = kWinPos;
-          wbase = wlo - 0x7FFFu;
-        } else if (wtop < 0x7FFFu) {
-          wmode = kWinNeg;
-          wbase = 0xFFFFu - wlo;
-        } else {
-          wmode = kWinKey;
-          wbase = wlo;
-        }
+        win_mode(wlo, wtop, wmode, wbase);
         const int nb = static_cast<int>(wtop - wlo) + 1;
         for (int b = tid; b < nb; b += kRT) hist[b] = 0u;
         __syncthreads();
@@ -1032,7 +946,7 @@ cudaError_t launch_row(const ScoreParams& p, cudaStream_t s, int which) {
 }  // namespace
 
 cudaError_t launch_score_computed(const ScoreParams& p, vs_dtype dtype, cudaStream_t s) {
-  return dtype == VS_BF16 ? launch_row<uint16_t>(p, s, 0) : launch_row<uint32_t>(p, s, 1);
+  return dtype == VS_BF16 ? launch_score_cluster(p, s) : launch_row<uint32_t>(p, s, 1);
 }
 
 }  // namespace vs
