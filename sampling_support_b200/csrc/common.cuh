@@ -360,8 +360,8 @@ __device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
 
 // The eight elements of a bf16 vector into s one by one, the max-valued
 // ones counted apart (the vector reaches or raises s's maximum, or holds a
-// NaN: rare once the maximum is seeded, so kept out of line).
-static __device__ __noinline__ Stats stats_vec_bf16_scalar(uint32_t w0, uint32_t w1, uint32_t w2,
+// NaN: rare once the maximum is seeded).
+static __device__ __forceinline__ Stats stats_vec_bf16_scalar(uint32_t w0, uint32_t w1, uint32_t w2,
                                                    uint32_t w3, float c, Stats s) {
   const uint32_t w[4] = {w0, w1, w2, w3};
   float u[8];

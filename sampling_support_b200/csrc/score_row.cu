@@ -44,8 +44,7 @@ namespace vs {
 
 namespace {
 
-constexpr int kRT = 1024;       // threads per row
-constexpr int kGrp = kRT / 2;   // threads per half (statistics warps / histogram warps)
+constexpr int kRT = 512;        // threads per row
 constexpr int kRW = kRT / 32;   // warps
 constexpr int kNStages = 6;     // ring depth
 constexpr int kStageBytes = 32768;
@@ -53,10 +52,20 @@ constexpr int kWin = kSelWin;
 constexpr int kBins = kSelBins;
 constexpr uint32_t kWinHi = 256;  // window keys above the first stage's maximum
 constexpr int kCountUnroll = 8;   // 16-byte loads in flight per thread (tie count)
+constexpr int kHeadElems = 8192;  // elements of the first piece of stage 0 (bf16)
 
 struct RowSh {
   uint64_t full[kNStages];
   uint64_t empty[kNStages];
+  uint64_t first;  // the first piece of stage 0 (bf16 rows), loaded apart
+  Stats rs;        // the row's merged statistics (warp 0)
+  float rvmax;     // the row maximum (warp 0)
+  uint32_t general;  // 1: the block takes the general path
+  uint32_t d_tkey, d_flags;  // warp 0's decision (bit 0 non-finite, bit 1 filtered)
+  float w_m0;      // the first piece's maximum (warp 0)
+  uint32_t w_top, w_lo, w_base;  // the window (warp 0)
+  int32_t w_mode;
+  uint32_t ysnap;  // elements before the target holding its key (window rows)
   Stats wst[kRW];
   float fred[kRW];
   uint32_t ured[kRW];
@@ -93,6 +102,8 @@ struct Ring {
   __device__ int nst() const { return (V + SE - 1) / SE; }
   __device__ int count(int si) const { return min(SE, V - si * SE); }
 
+  uint32_t head;  // bytes at the start of stage 0 already requested apart (thread 0)
+
   // thread 0: load stage si into the next ring slot
   __device__ void issue(int si) {
     const uint32_t L = ld++;
@@ -101,17 +112,26 @@ struct Ring {
       sh->timeout = 1u;
     }
     const uint32_t bytes = static_cast<uint32_t>((count(si) * sizeof(Raw) + 15) & ~size_t(15));
-    mbar_arrive_expect_tx(&sh->full[slot], bytes);
-    bulk_load_all(buf + static_cast<size_t>(slot) * SE, g + static_cast<size_t>(si) * SE, bytes,
-                  &sh->full[slot]);
+    const uint32_t skip = si == 0 ? min(head, bytes) : 0u;
+    if (si == 0) head = 0;
+    mbar_arrive_expect_tx(&sh->full[slot], bytes - skip);
+    if (bytes > skip)
+      bulk_load_all(reinterpret_cast<char*>(buf + static_cast<size_t>(slot) * SE) + skip,
+                    reinterpret_cast<const char*>(g + static_cast<size_t>(si) * SE) + skip,
+                    bytes - skip, &sh->full[slot]);
   }
 
-  // Run f(stage_ptr, n, base) over stages [s0, s1) in order; f returns true
-  // (uniformly) to stop early.  Loads already issued are drained either way.
-  template <typename F>
-  __device__ void pass(int s0, int s1, F&& f) {
+  // thread 0 requests the first stages of [s0, s1)
+  __device__ void start(int s0, int s1) {
     if (threadIdx.x == 0)
       for (int si = s0; si < min(s1, s0 + kNStages); ++si) issue(si);
+  }
+
+  // Run f(stage_ptr, n, base) over stages [s0, s1) in order, after
+  // start(s0, s1); f returns true (uniformly) to stop early.  Loads already
+  // issued are drained either way.
+  template <typename F>
+  __device__ void consume(int s0, int s1, F&& f) {
     int next = s0 + kNStages;
     bool stop = false;
     for (int si = s0; si < s1 && !stop; ++si) {
@@ -125,7 +145,7 @@ struct Ring {
       ++next;
     }
     // drain loads that were issued but not consumed (early stop)
-    if (threadIdx.x == 0) sh->outstanding = ld - 0u;  // ld is thread 0's count
+    if (threadIdx.x == 0) sh->outstanding = ld;  // ld is thread 0's count
     __syncthreads();
     const uint32_t issued = sh->outstanding;
     while (cs < issued) {
@@ -136,6 +156,12 @@ struct Ring {
       ++cs;
     }
     __syncthreads();
+  }
+
+  template <typename F>
+  __device__ void pass(int s0, int s1, F&& f) {
+    start(s0, s1);
+    consume(s0, s1, static_cast<F&&>(f));
   }
 
   __device__ static void mbar_arrive_cnt(uint64_t* bar) {
@@ -229,50 +255,63 @@ __device__ Desc descend(Ring<Raw>& ring, float c, float m, int fx_shift, bool by
 // ---------------------------------------------------------------------------
 // the streamed pass
 
-// bf16 stage, statistics: the group's `gsize` threads (thread `g` of the
-// group) take every gsize-th 16-byte vector, two in flight, alternating two
-// chains.
-__device__ __forceinline__ void stats_stage_bf16(const uint16_t* st, int n, float c, Chain (&ch)[2],
-                                                 uint32_t& vmax2, int g, int gsize) {
+// bf16 stage: every thread takes every kRT-th 16-byte vector, two in
+// flight, into its two statistics chains and, with a window, into the
+// exact-key histogram (elements outside the window into this lane's spill
+// bin, nb + lane).
+template <int MODE>
+__device__ __forceinline__ void stage_bf16(const uint16_t* st, int n, float c, f32x2 c2,
+                                           Chain (&ch)[2], uint32_t& vmax2, uint32_t wbase,
+                                           uint32_t nb, uint32_t hist_s) {
   const int nv = n / 8;
   const uint4* v4 = reinterpret_cast<const uint4*>(st);
-  const f32x2 c2 = pack2(c, c);
-  int v = g;
-  for (; v + gsize < nv; v += 2 * gsize) {
-    const uint4 q0 = v4[v], q1 = v4[v + gsize];
+  const uint32_t spill = nb + (threadIdx.x & 31);
+  int v = threadIdx.x;
+  for (; v + kRT < nv; v += 2 * kRT) {
+    const uint4 q0 = v4[v], q1 = v4[v + kRT];
     chain_vec(q0, c, c2, ch[0], vmax2);
     chain_vec(q1, c, c2, ch[1], vmax2);
+    if constexpr (MODE != kWinNone) {
+      hist_vec<MODE>(q0, wbase, spill, hist_s);
+      hist_vec<MODE>(q1, wbase, spill, hist_s);
+    }
   }
-  if (v < nv) chain_vec(v4[v], c, c2, ch[0], vmax2);
-  for (int j = nv * 8 + g; j < n; j += gsize) {
+  if (v < nv) {
+    const uint4 q = v4[v];
+    chain_vec(q, c, c2, ch[0], vmax2);
+    if constexpr (MODE != kWinNone) hist_vec<MODE>(q, wbase, spill, hist_s);
+  }
+  for (int j = nv * 8 + threadIdx.x; j < n; j += kRT) {
     const uint32_t r = st[j];
-    const float x = value_of(static_cast<uint16_t>(r));
     vmax2 = bmax2(vmax2, r | (r << 16));
-    float u[1] = {__fmul_rn(x, c)};
+    float u[1] = {__fmul_rn(value_of(static_cast<uint16_t>(r)), c)};
     stats_add(ch[0].s, u);
+    if constexpr (MODE != kWinNone) red_inc(hist_s + (min(win_index<MODE>(r, wbase), spill) << 2));
   }
 }
 
-// bf16 stage, histogram: the group's threads count every element of the
-// stage into the window (see hist_vec), four vectors in flight.
+// Elements [j0, j1) of a bf16 stage (any bounds): single elements up to the
+// first 16-byte boundary, whole vectors, then single elements again.
 template <int MODE>
-__device__ __forceinline__ void hist_stage_bf16(const uint16_t* st, int n, uint32_t base,
-                                                uint32_t spill, uint32_t hist_s, int g, int gsize) {
-  const int nv = n / 8;
+__device__ __forceinline__ void stage_range_bf16(const uint16_t* st, int j0, int j1, float c,
+                                                 f32x2 c2, Chain (&ch)[2], uint32_t& vmax2,
+                                                 uint32_t wbase, uint32_t nb, uint32_t hist_s) {
+  const uint32_t spill = nb + (threadIdx.x & 31);
+  auto one = [&](uint32_t r) {
+    vmax2 = bmax2(vmax2, r | (r << 16));
+    float u[1] = {__fmul_rn(value_of(static_cast<uint16_t>(r)), c)};
+    stats_add(ch[0].s, u);
+    if constexpr (MODE != kWinNone) red_inc(hist_s + (min(win_index<MODE>(r, wbase), spill) << 2));
+  };
+  const int a = min(j1, (j0 + 7) & ~7);
+  for (int j = j0 + static_cast<int>(threadIdx.x); j < a; j += kRT) one(st[j]);
   const uint4* v4 = reinterpret_cast<const uint4*>(st);
-  int v = g;
-  for (; v + 3 * gsize < nv; v += 4 * gsize) {
-    uint4 q[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) q[k] = v4[v + k * gsize];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) hist_vec<MODE>(q[k], base, spill, hist_s);
+  for (int v = a / 8 + static_cast<int>(threadIdx.x); v < j1 / 8; v += kRT) {
+    const uint4 q = v4[v];
+    chain_vec(q, c, c2, ch[0], vmax2);
+    if constexpr (MODE != kWinNone) hist_vec<MODE>(q, wbase, spill, hist_s);
   }
-  for (; v < nv; v += gsize) hist_vec<MODE>(v4[v], base, spill, hist_s);
-  for (int j = nv * 8 + g; j < n; j += gsize) {
-    const uint32_t r = st[j];
-    red_inc(hist_s + (min(win_index<MODE>(r, base), spill) << 2));
-  }
+  for (int j = max(a, (j1 / 8) * 8) + static_cast<int>(threadIdx.x); j < j1; j += kRT) one(st[j]);
 }
 
 __device__ __forceinline__ void stats_stage_f32(const uint32_t* st, int n, float c, Stats (&s2)[2],
@@ -300,52 +339,30 @@ __device__ __forceinline__ void stats_stage_f32(const uint32_t* st, int n, float
   }
 }
 
-__device__ __forceinline__ float block_max(float v, float* scratch) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float t = -kInf;
-  for (int w = 0; w < kRW; ++w) t = fmaxf(t, scratch[w]);
-  __syncthreads();
-  return t;
-}
-
-// Maximum value of one bf16 stage over the block.
-__device__ __forceinline__ float stage_max_bf16(const uint16_t* st, int n, float* scratch) {
-  const int nv = n / 8;
-  const uint4* v4 = reinterpret_cast<const uint4*>(st);
-  uint32_t mx = 0xFF80FF80u;  // (-inf, -inf)
-  for (int v = threadIdx.x; v < nv; v += kRT) {
-    const uint4 q = v4[v];
-    mx = bmax2(mx, bmax2(bmax2(q.x, q.y), bmax2(q.z, q.w)));
-  }
-  float m = fmaxf(__uint_as_float(mx << 16), __uint_as_float(mx & 0xFFFF0000u));
-  for (int j = nv * 8 + threadIdx.x; j < n; j += kRT) m = fmaxf(m, value_of(st[j]));
-  return block_max(m, scratch);
-}
-
+// Block sum of the support sums, valid in every thread (warp 0 reduces the
+// warps' partials in a fixed order and broadcasts).
 __device__ __forceinline__ SupSums block_sum_sup(SupSums v, RowSh& sh) {
+  __shared__ SupSums s_res;
+  auto warp_sum = [](SupSums& x) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    v.ngt += __shfl_xor_sync(0xffffffffu, v.ngt, o);
-    v.neq += __shfl_xor_sync(0xffffffffu, v.neq, o);
-    v.ntp += __shfl_xor_sync(0xffffffffu, v.ntp, o);
-    v.smass += __shfl_xor_sync(0xffffffffu, v.smass, o);
-    v.sa += __shfl_xor_sync(0xffffffffu, v.sa, o);
-  }
+    for (int o = 16; o > 0; o >>= 1) {
+      x.ngt += __shfl_xor_sync(0xffffffffu, x.ngt, o);
+      x.neq += __shfl_xor_sync(0xffffffffu, x.neq, o);
+      x.ntp += __shfl_xor_sync(0xffffffffu, x.ntp, o);
+      x.smass += __shfl_xor_sync(0xffffffffu, x.smass, o);
+      x.sa += __shfl_xor_sync(0xffffffffu, x.sa, o);
+    }
+  };
+  warp_sum(v);
   if ((threadIdx.x & 31) == 0) sh.sums[threadIdx.x >> 5] = v;
   __syncthreads();
-  SupSums t{0u, 0u, 0u, 0.f, 0.f};
-  for (int w = 0; w < kRW; ++w) {
-    t.ngt += sh.sums[w].ngt;
-    t.neq += sh.sums[w].neq;
-    t.ntp += sh.sums[w].ntp;
-    t.smass += sh.sums[w].smass;
-    t.sa += sh.sums[w].sa;
+  if (threadIdx.x < 32) {
+    SupSums t = threadIdx.x < kRW ? sh.sums[threadIdx.x] : SupSums{0u, 0u, 0u, 0.f, 0.f};
+    warp_sum(t);
+    if (threadIdx.x == 0) s_res = t;
   }
   __syncthreads();
-  return t;
+  return s_res;
 }
 
 // Number of elements of g[j0, j1) whose raw bits are r0 or r1 (the two
@@ -382,6 +399,261 @@ __device__ __forceinline__ uint32_t count_raw(const uint16_t* g, int j0, int j1,
 }
 
 // ---------------------------------------------------------------------------
+// warp-level pieces of the decision (warp 0, no block barriers)
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Statistics merged over the warp (every lane gets them): the warp maximum
+// first, each lane rebased onto it once, then plain sums in a fixed order.
+__device__ __forceinline__ Stats warp_stats(Stats s) {
+  const float m = warp_max(s.m);
+  if (s.c0 != 0.f || s.zr != 0.f) stats_rebase(s, m);
+  float c0 = s.c0, zr = s.zr, a = s.a;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    c0 += __shfl_xor_sync(0xffffffffu, c0, o);
+    zr += __shfl_xor_sync(0xffffffffu, zr, o);
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+  }
+  return Stats{m, c0, zr, a};
+}
+
+// From bin `top` of the window down, the bin at which the cumulative count
+// (by_mass false) or fixed-point mass first reaches need (>= 1); chunks of
+// 256 bins, lane l holding bins hi - 8l - k (k = 0..7) of a chunk.  False
+// when the bins [0, top] hold less than need.
+__device__ bool warp_search(const Window& w, int top, bool by_mass, u64 need, Desc& out) {
+  const int lane = threadIdx.x & 31;
+  u64 ac = 0, am = 0;  // above the current chunk
+  for (int hi = top; hi >= 0; hi -= 256) {
+    uint32_t cnt[8];
+    u64 fx[8];
+    u64 lc = 0, lm = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int b = hi - 8 * lane - k;
+      cnt[k] = b >= 0 ? w.hist[b] : 0u;
+      fx[k] = cnt[k] ? static_cast<u64>(cnt[k]) * bin_fx(w, w.klo + static_cast<uint32_t>(b)) : 0ull;
+      lc += cnt[k];
+      lm += fx[k];
+    }
+    u64 pc = lc, pm = lm;  // inclusive prefix from lane 0 (the largest keys)
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const u64 tc = __shfl_up_sync(0xffffffffu, pc, o), tm = __shfl_up_sync(0xffffffffu, pm, o);
+      if (lane >= o) {
+        pc += tc;
+        pm += tm;
+      }
+    }
+    const u64 ec = ac + pc - lc, em = am + pm - lm;
+    const u64 base = by_mass ? em : ec, mine = by_mass ? lm : lc;
+    const uint32_t ball = __ballot_sync(0xffffffffu, base < need && need <= base + mine);
+    if (ball) {
+      const int src = __ffs(ball) - 1;
+      uint32_t key = 0;
+      u64 rc = ec, rm = em, at_c = 0, at_m = 0;
+      if (lane == src) {
+        bool done = false;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (!done && cnt[k] && (by_mass ? rm + fx[k] : rc + cnt[k]) >= need) {
+            key = w.klo + static_cast<uint32_t>(hi - 8 * lane - k);
+            at_c = cnt[k];
+            at_m = fx[k];
+            done = true;
+          }
+          if (!done) {
+            rc += cnt[k];
+            rm += fx[k];
+          }
+        }
+      }
+      out.key = __shfl_sync(0xffffffffu, key, src);
+      out.above_cnt = __shfl_sync(0xffffffffu, rc, src);
+      out.above_mass = __shfl_sync(0xffffffffu, rm, src);
+      out.at_cnt = __shfl_sync(0xffffffffu, at_c, src);
+      out.at_mass = __shfl_sync(0xffffffffu, at_m, src);
+      return true;
+    }
+    ac += __shfl_sync(0xffffffffu, pc, 31);
+    am += __shfl_sync(0xffffffffu, pm, 31);
+  }
+  return false;
+}
+
+// Support sums over the bins of keys (tkey, kmr] and the count at tkey,
+// reduced over the warp in a fixed order (every lane gets them).
+__device__ SupSums warp_sums(const Window& w, uint32_t tkey, uint32_t kmr) {
+  const int lane = threadIdx.x & 31;
+  SupSums v{0u, 0u, 0u, 0.f, 0.f};
+  float sm[4] = {0.f, 0.f, 0.f, 0.f}, sa[4] = {0.f, 0.f, 0.f, 0.f};
+  const int hi = static_cast<int>(kmr - w.klo);
+  int b = static_cast<int>(tkey - w.klo) + 1 + lane;
+  // four bins per lane in flight, each into its own accumulators
+  for (; b + 96 <= hi; b += 128) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int bk = b + 32 * k;
+      const uint32_t cnt = w.hist[bk];
+      const float d = key_u(w.klo + static_cast<uint32_t>(bk), w.c) - w.m;
+      const float e = cnt ? ex2(d) : 0.f;
+      const float fc = static_cast<float>(cnt);
+      v.ngt += cnt;
+      if (d == 0.f)
+        v.ntp += cnt;
+      else
+        sm[k] = fmaf(fc, e, sm[k]);
+      sa[k] = fmaf(fc * d, e, sa[k]);
+    }
+  }
+  for (; b <= hi; b += 32) {
+    const uint32_t cnt = w.hist[b];
+    const float d = key_u(w.klo + static_cast<uint32_t>(b), w.c) - w.m;
+    const float e = cnt ? ex2(d) : 0.f;
+    const float fc = static_cast<float>(cnt);
+    v.ngt += cnt;
+    if (d == 0.f)
+      v.ntp += cnt;
+    else
+      sm[0] = fmaf(fc, e, sm[0]);
+    sa[0] = fmaf(fc * d, e, sa[0]);
+  }
+  v.smass = (sm[0] + sm[1]) + (sm[2] + sm[3]);
+  v.sa = (sa[0] + sa[1]) + (sa[2] + sa[3]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    v.ngt += __shfl_xor_sync(0xffffffffu, v.ngt, o);
+    v.ntp += __shfl_xor_sync(0xffffffffu, v.ntp, o);
+    v.smass += __shfl_xor_sync(0xffffffffu, v.smass, o);
+    v.sa += __shfl_xor_sync(0xffffffffu, v.sa, o);
+  }
+  v.neq = w.hist[tkey - w.klo];
+  return v;
+}
+
+// Everything the per-row outputs are made from.
+struct RowOut {
+  Stats s;
+  float vmax, m, log2z, h_full;
+  bool nonfinite, filtered, cut_known;
+  uint32_t tkey;
+  int32_t tie_cut;
+  u64 ckeep;
+  uint32_t ylt;
+  float log2zs, h_support, c0s, zrs;
+  int32_t n_support;
+};
+
+__device__ __forceinline__ RowOut row_out_init(const Stats& s, float vmax, bool any_filter, int V) {
+  RowOut o;
+  o.s = s;
+  o.vmax = vmax;
+  o.nonfinite = !stats_finite(s) || !isfinite(vmax);
+  o.m = s.m;  // = fl(vmax c)
+  o.log2z = stats_log2z(s);
+  o.h_full = kLn2 * (o.log2z - s.a / stats_z(s));
+  o.filtered = !o.nonfinite && any_filter;
+  o.cut_known = true;
+  o.tkey = 0;
+  o.tie_cut = INT_MAX;
+  o.ckeep = 0;
+  o.ylt = 0;
+  o.log2zs = o.log2z;
+  o.h_support = o.h_full;
+  o.c0s = s.c0;
+  o.zrs = s.zr;
+  o.n_support = o.nonfinite ? 0 : V;
+  return o;
+}
+
+// Support statistics from the sums above the threshold and the ckeep kept
+// elements of its tie group.
+__device__ __forceinline__ void support_stats(RowOut& o, const SupSums& sums, float c) {
+  const float dt = __fmul_rn(KeyTraits<uint16_t>::decode(o.tkey), c) - o.m;
+  const float et = ex2(dt);
+  Stats ss;
+  ss.m = o.m;
+  ss.c0 = static_cast<float>(sums.ntp) + (dt == 0.f ? static_cast<float>(o.ckeep) : 0.f);
+  ss.zr = sums.smass + (dt == 0.f ? 0.f : static_cast<float>(o.ckeep) * et);
+  ss.a = sums.sa + static_cast<float>(o.ckeep) * dt * et;
+  o.log2zs = stats_log2z(ss);
+  o.h_support = kLn2 * (o.log2zs - ss.a / stats_z(ss));
+  o.c0s = ss.c0;
+  o.zrs = ss.zr;
+  o.n_support = static_cast<int32_t>(sums.ngt + o.ckeep);
+}
+
+// The per-row outputs (one thread).
+template <typename Raw>
+__device__ void emit_row(const ScoreParams& P, int row, const RowOut& o, bool target_ok, int y,
+                         Raw ry, float c, uint32_t timeout) {
+  uint32_t status = 0;
+  float lp_v = __int_as_float(0x7fc00000), lp_s = __int_as_float(0x7fc00000);
+  bool in_s = false;
+  if (!target_ok) status |= VS_ROW_TARGET_OUT_OF_RANGE;
+  if (o.nonfinite) {
+    status |= VS_ROW_NONFINITE_INPUT;
+  } else if (target_ok) {
+    const float uy = __fmul_rn(value_of(ry), c);
+    lp_v = kLn2 * (uy - o.m - o.log2z);
+    if (!o.filtered) {
+      in_s = true;
+    } else {
+      const uint32_t ky = key_of(ry);
+      in_s = ky > o.tkey || (ky == o.tkey && (o.cut_known ? y <= o.tie_cut : o.ylt < o.ckeep));
+    }
+    if (in_s) {
+      lp_s = o.filtered ? kLn2 * (uy - o.m - o.log2zs) : lp_v;
+    } else {
+      lp_s = -kInf;
+      status |= VS_ROW_TARGET_NOT_IN_SUPPORT;
+    }
+  }
+  if (timeout) status |= kRowDeviceTimeout;
+  const float nan = __int_as_float(0x7fc00000);
+  if (P.lp_full) P.lp_full[row] = lp_v;
+  if (P.lp_support) P.lp_support[row] = lp_s;
+  if (P.want_entropy) {
+    if (P.h_full) P.h_full[row] = o.nonfinite ? nan : o.h_full;
+    if (P.h_support) P.h_support[row] = o.nonfinite ? nan : o.h_support;
+  }
+  if (P.valid) P.valid[row] = o.nonfinite ? 0 : 1;
+  if (P.status) P.status[row] = status;
+  if (P.support_size) P.support_size[row] = o.n_support;
+  if (P.ctx) {
+    RowCtx cx{};
+    cx.m2 = o.vmax;
+    cx.log2z = o.log2z;
+    cx.msup = o.vmax;
+    cx.log2zs = o.log2zs;
+    cx.h_full = o.h_full;
+    cx.h_support = o.h_support;
+    cx.c = c;
+    cx.tkey = o.tkey;
+    cx.tie_cut = o.tie_cut;
+    uint32_t f = kCtxFullStats;
+    if (o.nonfinite) f |= kCtxNonFinite | kCtxEmpty;
+    else if (!o.filtered) f |= kCtxAllVocab;
+    else f |= kCtxThreshold;
+    if (target_ok) f |= kCtxTargetOk;
+    if (in_s) f |= kCtxTargetInS;
+    cx.flags = f;
+    cx.n_support = o.n_support;
+    cx.status = status;
+    cx.c0_full = o.s.c0;
+    cx.zr_full = o.s.zr;
+    cx.c0_sup = o.c0s;
+    cx.zr_sup = o.zrs;
+    P.ctx[row] = cx;
+  }
+}
+
+// ---------------------------------------------------------------------------
 
 template <typename Raw>
 __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
@@ -396,6 +668,7 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
 
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
   const int V = P.vocab;
   const Raw* grow = static_cast<const Raw*>(P.logits) + static_cast<int64_t>(row) * P.ld;
 
@@ -404,6 +677,7 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
       mbar_init(&sh.full[s], 1);
       mbar_init(&sh.empty[s], kRW);
     }
+    mbar_init(&sh.first, 1);
     sh.timeout = 0;
     sh.tie_cut = INT_MAX;
     fence_barrier_init();
@@ -414,7 +688,7 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
   pdl_wait();
   pdl_launch_dependents();
   __syncthreads();
-  Ring<Raw> ring{grow, V, ringbuf, &sh, 0u, 0u};
+  Ring<Raw> ring{grow, V, ringbuf, &sh, 0u, 0u, 0u};
 
   const float T = P.temperature ? P.temperature[row] : P.temperature_scalar;
   const float c = kLog2e / T;
@@ -440,19 +714,37 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
   int wmode = kWinNone;
   uint32_t wbase = 0;
   const uint32_t hist_s = smem_addr(hist);
-  ring.pass(0, ring.nst(), [&](const Raw* st, int n, int base) {
-    if constexpr (kBf16) {
-      const uint16_t* st16 = reinterpret_cast<const uint16_t*>(st);
-      if (base == 0) {
-        // the first stage's maximum m0, a lower bound of the row maximum m,
-        // seeds every chain's running maximum (so that later vectors rarely
-        // raise it and take the packed path)
-        const float m0 = stage_max_bf16(st16, n, sh.fred);
-        chain_seed(ch2[0], m0, c);
-        chain_seed(ch2[1], m0, c);
-        if (hist_on) {
-        // fix the window from m0: elements below the level found with it are
-        // below the level of m as well
+  const int nst = ring.nst();
+  if constexpr (kBf16) {
+    // the first piece of stage 0 is requested apart, ahead of the ring: its
+    // maximum m0, a lower bound of the row maximum m, fixes the window and
+    // seeds every chain's running maximum (so that later vectors rarely
+    // raise it and take the packed path) while the ring fills
+    const int nh = min(V, kHeadElems);
+    const uint32_t hbytes = static_cast<uint32_t>((nh * 2 + 15) & ~15);
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&sh.first, hbytes);
+      bulk_load(ringbuf, grow, hbytes, &sh.first);
+      ring.head = hbytes;
+    }
+    ring.start(0, nst);
+    // warp 0 finds m0 and the window while the other warps clear every bin
+    if (hist_on && warp != 0)
+      for (int b = tid - 32; b < kWin + 32; b += kRT - 32) hist[b] = 0u;
+    if (warp == 0) {
+      if (!mbar_wait(&sh.first, 0)) atomicOr(&sh.timeout, 1u);
+      const uint16_t* h16 = reinterpret_cast<const uint16_t*>(ringbuf);
+      const uint4* h4 = reinterpret_cast<const uint4*>(ringbuf);
+      uint32_t mx = 0xFF80FF80u;
+      for (int v = lane; v < nh / 8; v += 32) {
+        const uint4 q = h4[v];
+        mx = bmax2(mx, bmax2(bmax2(q.x, q.y), bmax2(q.z, q.w)));
+      }
+      float mh = vmax_of(mx);
+      for (int j = (nh / 8) * 8 + lane; j < nh; j += 32) mh = fmaxf(mh, value_of(h16[j]));
+      const float m0 = warp_max(mh);
+      if (hist_on) {
+        // elements below the level found with m0 are below the level of m too
         const uint32_t kref = key_of(static_cast<uint16_t>(__float_as_uint(m0) >> 16));
         wtop = min(kref + kWinHi, KT::kInfKey);
         wlo = wtop >= static_cast<uint32_t>(kWin - 1) ? wtop - (kWin - 1) : 0u;
@@ -463,31 +755,69 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
           if (dlo > -kInf) wlo = key_at_level(wlo, wtop, c, __fmul_rn(m0, c), dlo);
         }
         win_mode(wlo, wtop, wmode, wbase);
-        const int nb = static_cast<int>(wtop - wlo) + 1;
-        for (int b = tid; b < nb; b += kRT) hist[b] = 0u;
-        __syncthreads();
-        }
       }
-      // with a window, the first half of the warps takes the statistics and
-      // the second half the histogram of the same stage; without, every
-      // warp takes the statistics
-      const uint32_t spill = (wtop - wlo) + 1u + (tid & 31);
-      if (wmode == kWinNone) {
-        stats_stage_bf16(st16, n, c, ch2, vmax2, tid, kRT);
-      } else if (tid < kGrp) {
-        stats_stage_bf16(st16, n, c, ch2, vmax2, tid, kGrp);
-      } else if (wmode == kWinPos) {
-        hist_stage_bf16<kWinPos>(st16, n, wbase, spill, hist_s, tid - kGrp, kGrp);
-      } else if (wmode == kWinNeg) {
-        hist_stage_bf16<kWinNeg>(st16, n, wbase, spill, hist_s, tid - kGrp, kGrp);
-      } else {
-        hist_stage_bf16<kWinKey>(st16, n, wbase, spill, hist_s, tid - kGrp, kGrp);
+      if (lane == 0) {
+        sh.w_m0 = m0;
+        sh.w_top = wtop;
+        sh.w_lo = wlo;
+        sh.w_base = wbase;
+        sh.w_mode = wmode;
       }
-    } else {
-      stats_stage_f32(st, n, c, s2, vmax);
     }
-    return false;
-  });
+    __syncthreads();
+    const float m0 = sh.w_m0;
+    wtop = sh.w_top;
+    wlo = sh.w_lo;
+    wbase = sh.w_base;
+    wmode = sh.w_mode;
+    chain_seed(ch2[0], m0, c);
+    chain_seed(ch2[1], m0, c);
+    const uint32_t nb = (wtop - wlo) + 1u;
+    const f32x2 c2 = pack2(c, c);
+    // when the target's key lies in the window, the count of its key at
+    // the target's position (the ties that precede it) is taken between
+    // two block barriers in the target's stage: its membership in a partly
+    // kept tie group then needs no second look at the row
+    const uint32_t ky = key_of(static_cast<uint16_t>(ry));
+    const bool snap = wmode != kWinNone && target_ok && ky >= wlo && ky <= wtop;
+    auto stage = [&](const uint16_t* st16, int j0, int j1) {
+      if (wmode == kWinNone)
+        stage_range_bf16<kWinNone>(st16, j0, j1, c, c2, ch2, vmax2, wbase, nb, hist_s);
+      else if (wmode == kWinPos)
+        stage_range_bf16<kWinPos>(st16, j0, j1, c, c2, ch2, vmax2, wbase, nb, hist_s);
+      else if (wmode == kWinNeg)
+        stage_range_bf16<kWinNeg>(st16, j0, j1, c, c2, ch2, vmax2, wbase, nb, hist_s);
+      else
+        stage_range_bf16<kWinKey>(st16, j0, j1, c, c2, ch2, vmax2, wbase, nb, hist_s);
+    };
+    ring.consume(0, nst, [&](const Raw* st, int n, int base) {
+      const uint16_t* st16 = reinterpret_cast<const uint16_t*>(st);
+      if (snap && y >= base && y < base + n) {
+        stage(st16, 0, y - base);
+        __syncthreads();
+        if (tid == 0) sh.ysnap = hist[ky - wlo];
+        __syncthreads();
+        stage(st16, y - base, n);
+      } else if (wmode == kWinNone) {
+        stage_bf16<kWinNone>(st16, n, c, c2, ch2, vmax2, wbase, nb, hist_s);
+      } else if (wmode == kWinPos) {
+        stage_bf16<kWinPos>(st16, n, c, c2, ch2, vmax2, wbase, nb, hist_s);
+      } else if (wmode == kWinNeg) {
+        stage_bf16<kWinNeg>(st16, n, c, c2, ch2, vmax2, wbase, nb, hist_s);
+      } else {
+        stage_bf16<kWinKey>(st16, n, c, c2, ch2, vmax2, wbase, nb, hist_s);
+      }
+      return false;
+    });
+  } else {
+    ring.pass(0, nst, [&](const Raw* st, int n, int) {
+      stats_stage_f32(st, n, c, s2, vmax);
+      return false;
+    });
+  }
+  // ---- per-warp partial statistics; warp 0 merges them and, in the
+  // common case, takes the whole decision from the bins with warp shuffles
+  // (no block barriers); otherwise the block takes the general path below
   Stats s;
   if constexpr (kBf16) {
     s = ch2[0].s;
@@ -497,18 +827,118 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
     s = s2[0];
     stats_merge(s, s2[1]);
   }
-  s = block_reduce(s, sh.wst);
-  vmax = block_max(vmax, sh.fred);
-
-  const bool nonfinite = !stats_finite(s) || !isfinite(vmax);
+  s = warp_stats(s);
+  vmax = warp_max(vmax);
+  if (lane == 0) {
+    sh.wst[warp] = s;
+    sh.fred[warp] = vmax;
+  }
+  __syncthreads();
+  const bool want_cut = P.ctx != nullptr || P.support_mask != nullptr || P.sampled != nullptr;
+  if (warp == 0) {
+    s = warp_stats(lane < kRW ? sh.wst[lane] : stats_empty());
+    vmax = warp_max(lane < kRW ? sh.fred[lane] : -kInf);
+    RowOut o = row_out_init(s, vmax, any_filter, V);
+    bool fast = kBf16;
+    if constexpr (kBf16) {
+    if (o.filtered) {
+      const float fxs = fx_scale(P.fx_shift);
+      const uint32_t kmr = key_of(static_cast<uint16_t>(__float_as_uint(vmax) >> 16));
+      const Window w{wlo, wtop, static_cast<int>(wtop - wlo) + 1, wmode, 0u, hist, c, o.m, fxs};
+      bool win_ok = kmr <= wtop;
+      bool all_ties = true, have_t = false;
+      u64 cnum = 0;
+      if (win_ok && (use_k || use_p)) {
+        const int top = static_cast<int>(kmr - wlo);
+        Desc dk{}, dp{};
+        u64 ck = 0;
+        if (use_k) {
+          win_ok = warp_search(w, top, false, static_cast<u64>(kk), dk);
+          if (win_ok) {
+            ck = static_cast<u64>(kk) - dk.above_cnt;
+            o.tkey = dk.key;
+            cnum = ck;
+            all_ties = ck >= dk.at_cnt;
+            have_t = true;
+          }
+        }
+        if (win_ok && use_p) {
+          const double mass1 = use_k ? static_cast<double>(dk.above_mass + ck * bin_fx(w, dk.key))
+                                     : (static_cast<double>(s.c0) + static_cast<double>(s.zr)) *
+                                           static_cast<double>(fxs);
+          const u64 tp = topp_target(pp, mass1);
+          win_ok = warp_search(w, top, true, tp, dp);
+          if (win_ok) {
+            u64 cp = topp_ties(dp, tp, bin_fx(w, dp.key));
+            if (use_k && dp.key == o.tkey && cp > ck) cp = ck;
+            o.tkey = dp.key;
+            cnum = cp;
+            all_ties = cp >= dp.at_cnt;
+            have_t = true;
+          }
+        }
+        if (!win_ok && use_p && !use_k && use_minp && minp_key<Raw>(mp, c, o.m) >= w.klo) {
+          win_ok = true;
+          have_t = false;
+          all_ties = true;
+        }
+      }
+      if (!win_ok && (use_k || use_p)) {
+        fast = false;  // the decision lies outside the window
+      } else {
+        if (use_minp) {
+          const uint32_t lo = minp_key<Raw>(mp, c, o.m);
+          if (!have_t || lo > o.tkey) {
+            o.tkey = lo;
+            all_ties = true;
+          }
+        }
+        if (!win_ok || o.tkey < wlo) {
+          fast = false;  // the support sums need a pass over the row
+        } else {
+          const SupSums sums = warp_sums(w, o.tkey, kmr);
+          const u64 tot_eq = sums.neq;
+          o.ckeep = all_ties ? tot_eq : (cnum < tot_eq ? cnum : tot_eq);
+          support_stats(o, sums, c);
+          if (o.ckeep < tot_eq) {
+            o.cut_known = false;
+            // the cut's position needs a pass over the row; the target's
+            // rank in the tie group is the count taken at its position
+            if (want_cut) fast = false;
+            else if (target_ok && key_of(ry) == o.tkey) o.ylt = sh.ysnap;
+          }
+        }
+      }
+    }
+    }
+    if (lane == 0) {
+      sh.rs = s;
+      sh.rvmax = vmax;
+      sh.general = fast ? 0u : 1u;
+      if (fast) {
+        sh.d_tkey = o.tkey;
+        sh.d_flags = (o.nonfinite ? 1u : 0u) | (o.filtered ? 2u : 0u);
+        emit_row(P, row, o, target_ok, y, ry, c, sh.timeout);
+      }
+    }
+  }
+  __syncthreads();
+  bool nonfinite, filtered;
+  uint32_t tkey = 0;
+  int32_t tie_cut = INT_MAX;
+  if (!sh.general) {
+    nonfinite = (sh.d_flags & 1u) != 0;
+    filtered = (sh.d_flags & 2u) != 0;
+    tkey = sh.d_tkey;
+  } else {
+  s = sh.rs;
+  vmax = sh.rvmax;
+  nonfinite = !stats_finite(s) || !isfinite(vmax);
   const float m = s.m;  // = fl(vmax c)
   const float log2z = stats_log2z(s);
   const float h_full = kLn2 * (log2z - s.a / stats_z(s));
-  const bool filtered = !nonfinite && any_filter;
-  const bool want_cut = P.ctx != nullptr || P.support_mask != nullptr || P.sampled != nullptr;
+  filtered = !nonfinite && any_filter;
 
-  uint32_t tkey = 0;
-  int32_t tie_cut = INT_MAX;
   bool cut_known = true;  // tie_cut resolved (or not needed: every tie kept)
   u64 ckeep = 0;
   u64 tie_group = 0;  // elements holding the threshold key
@@ -757,68 +1187,28 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
     }
   }
 
-  // ---- per-row outputs
-  if (tid == 0) {
-    uint32_t status = 0;
-    float lp_v = __int_as_float(0x7fc00000), lp_s = __int_as_float(0x7fc00000);
-    bool in_s = false;
-    if (!target_ok) status |= VS_ROW_TARGET_OUT_OF_RANGE;
-    if (nonfinite) {
-      status |= VS_ROW_NONFINITE_INPUT;
-    } else if (target_ok) {
-      const float uy = __fmul_rn(value_of(ry), c);
-      lp_v = kLn2 * (uy - m - log2z);
-      if (!filtered) {
-        in_s = true;
-      } else {
-        const uint32_t ky = key_of(ry);
-        in_s = ky > tkey || (ky == tkey && (cut_known ? y <= tie_cut : ylt < ckeep));
-      }
-      if (in_s) {
-        lp_s = filtered ? kLn2 * (uy - m - log2zs) : lp_v;
-      } else {
-        lp_s = -kInf;
-        status |= VS_ROW_TARGET_NOT_IN_SUPPORT;
-      }
-    }
-    if (sh.timeout) status |= kRowDeviceTimeout;
-    const float nan = __int_as_float(0x7fc00000);
-    if (P.lp_full) P.lp_full[row] = lp_v;
-    if (P.lp_support) P.lp_support[row] = lp_s;
-    if (P.want_entropy) {
-      if (P.h_full) P.h_full[row] = nonfinite ? nan : h_full;
-      if (P.h_support) P.h_support[row] = nonfinite ? nan : h_support;
-    }
-    if (P.valid) P.valid[row] = nonfinite ? 0 : 1;
-    if (P.status) P.status[row] = status;
-    if (P.support_size) P.support_size[row] = n_support;
-    if (P.ctx) {
-      RowCtx cx{};
-      cx.m2 = vmax;
-      cx.log2z = log2z;
-      cx.msup = vmax;
-      cx.log2zs = log2zs;
-      cx.h_full = h_full;
-      cx.h_support = h_support;
-      cx.c = c;
-      cx.tkey = tkey;
-      cx.tie_cut = tie_cut;
-      uint32_t f = kCtxFullStats;
-      if (nonfinite) f |= kCtxNonFinite | kCtxEmpty;
-      else if (!filtered) f |= kCtxAllVocab;
-      else f |= kCtxThreshold;
-      if (target_ok) f |= kCtxTargetOk;
-      if (in_s) f |= kCtxTargetInS;
-      cx.flags = f;
-      cx.n_support = n_support;
-      cx.status = status;
-      cx.c0_full = s.c0;
-      cx.zr_full = s.zr;
-      cx.c0_sup = c0s;
-      cx.zr_sup = zrs;
-      P.ctx[row] = cx;
-    }
+  {
+    RowOut o;
+    o.s = s;
+    o.vmax = vmax;
+    o.m = m;
+    o.log2z = log2z;
+    o.h_full = h_full;
+    o.nonfinite = nonfinite;
+    o.filtered = filtered;
+    o.tkey = tkey;
+    o.tie_cut = tie_cut;
+    o.cut_known = cut_known;
+    o.ckeep = ckeep;
+    o.ylt = ylt;
+    o.log2zs = log2zs;
+    o.h_support = h_support;
+    o.c0s = c0s;
+    o.zrs = zrs;
+    o.n_support = n_support;
+    if (tid == 0) emit_row(P, row, o, target_ok, y, ry, c, sh.timeout);
   }
+  }  // general path
 
   // ---- support bitmask, one 32-id word per thread and stage
   if (P.support_mask) {
@@ -946,7 +1336,7 @@ cudaError_t launch_row(const ScoreParams& p, cudaStream_t s, int which) {
 }  // namespace
 
 cudaError_t launch_score_computed(const ScoreParams& p, vs_dtype dtype, cudaStream_t s) {
-  return dtype == VS_BF16 ? launch_score_cluster(p, s) : launch_row<uint32_t>(p, s, 1);
+  return dtype == VS_BF16 ? launch_row<uint16_t>(p, s, 0) : launch_row<uint32_t>(p, s, 1);
 }
 
 }  // namespace vs

@@ -91,49 +91,6 @@ __device__ __forceinline__ float warp_dot(const uint4* hs4, const uint4* w4, int
   return s;
 }
 
-// Two dot products at once (weight rows w4a and w4b against the staged
-// hidden state): twice the loads in flight per lane; each sum accumulates
-// exactly as warp_dot's.
-__device__ __forceinline__ void warp_dot2(const uint4* hs4, const uint4* w4a, const uint4* w4b,
-                                          int nvec, float& ra, float& rb) {
-  const int lane = threadIdx.x & 31;
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, b0 = 0.f, b1 = 0.f, b2 = 0.f, b3 = 0.f;
-  auto fma8 = [&](const uint4& h, const uint4& w, float& s0, float& s1, float& s2, float& s3) {
-    fma_bf16x2(h.x, w.x, s0, s1);
-    fma_bf16x2(h.y, w.y, s2, s3);
-    fma_bf16x2(h.z, w.z, s0, s1);
-    fma_bf16x2(h.w, w.w, s2, s3);
-  };
-  int v = lane;
-  for (; v + (kSHUnroll - 1) * 32 < nvec; v += kSHUnroll * 32) {
-    uint4 wa[kSHUnroll], wb[kSHUnroll];
-#pragma unroll
-    for (int u = 0; u < kSHUnroll; ++u) {
-      wa[u] = __ldg(w4a + v + u * 32);
-      wb[u] = __ldg(w4b + v + u * 32);
-    }
-#pragma unroll
-    for (int u = 0; u < kSHUnroll; ++u) {
-      const uint4 h = hs4[v + u * 32];
-      fma8(h, wa[u], a0, a1, a2, a3);
-      fma8(h, wb[u], b0, b1, b2, b3);
-    }
-  }
-  for (; v < nvec; v += 32) {
-    const uint4 h = hs4[v];
-    fma8(h, __ldg(w4a + v), a0, a1, a2, a3);
-    fma8(h, __ldg(w4b + v), b0, b1, b2, b3);
-  }
-  float sa = (a0 + a1) + (a2 + a3), sb = (b0 + b1) + (b2 + b3);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    sa += __shfl_xor_sync(0xffffffffu, sa, o);
-    sb += __shfl_xor_sync(0xffffffffu, sb, o);
-  }
-  ra = sa;
-  rb = sb;
-}
-
 __global__ void __launch_bounds__(kSHThreads) support_head_kernel(SupportHeadParams P) {
   extern __shared__ __align__(16) uint4 hs4[];  // the row's hidden state
   __shared__ int32_t ids[VS_MAX_SUPPORT_WIDTH];
@@ -193,24 +150,12 @@ __global__ void __launch_bounds__(kSHThreads) support_head_kernel(SupportHeadPar
   __syncthreads();
   const int nkeep = static_cast<int>(nkeep_sh);
 
-  // one dot product per kept id, warps taking the kept slots two at a time
-  // (slots j and j + kSHWarps), the last odd one alone
-  for (int j = warp; j < nkeep; j += 2 * kSHWarps) {
+  // one dot product per kept id, warps taking the kept slots in turn
+  for (int j = warp; j < nkeep; j += kSHWarps) {
     const int w = kslot[j];
     const uint4* w4 = reinterpret_cast<const uint4*>(P.W + static_cast<int64_t>(ids[w]) * P.ldw);
-    if (j + kSHWarps < nkeep) {
-      const int w2 = kslot[j + kSHWarps];
-      const uint4* w4b = reinterpret_cast<const uint4*>(P.W + static_cast<int64_t>(ids[w2]) * P.ldw);
-      float a, b;
-      warp_dot2(hs4, w4, w4b, nvec, a, b);
-      if (lane == 0) {
-        acc[w] = a;
-        acc[w2] = b;
-      }
-    } else {
-      const float a = warp_dot(hs4, w4, nvec);
-      if (lane == 0) acc[w] = a;
-    }
+    const float a = warp_dot(hs4, w4, nvec);
+    if (lane == 0) acc[w] = a;
   }
   __syncthreads();
 
