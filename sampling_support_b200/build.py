@@ -13,7 +13,7 @@ CSRC = PKG / "csrc"
 INCLUDE = PKG.parent / "include"
 LIB = PKG / "libvs.so"
 
-SOURCES = ["api.cu", "score_fwd.cu", "score_row.cu", "score_cluster.cu", "score_bwd.cu", "l1_distance.cu", "fused_lmhead.cu", "support_head.cu"]
+SOURCES = ["api.cu", "score_fwd.cu", "score_row.cu", "score_bwd.cu", "l1_distance.cu", "fused_lmhead.cu", "support_head.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

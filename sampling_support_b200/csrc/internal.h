@@ -94,8 +94,6 @@ struct BwdParams {
 
 // launchers (return a cudaError_t from the launch)
 cudaError_t launch_score_computed(const ScoreParams& p, vs_dtype dtype, cudaStream_t s);
-// bf16 rows, each split over a thread-block cluster (score_cluster.cu)
-cudaError_t launch_score_cluster(const ScoreParams& p, cudaStream_t s);
 cudaError_t launch_score_recorded(const ScoreParams& p, vs_dtype dtype, cudaStream_t s);
 cudaError_t launch_score_reduce(const float* h_support, const uint8_t* valid, int rows,
                                 double* entropy_sum, int32_t* valid_count, cudaStream_t s);

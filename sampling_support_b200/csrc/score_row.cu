@@ -53,6 +53,7 @@ constexpr int kBins = kSelBins;
 constexpr uint32_t kWinHi = 256;  // window keys above the first stage's maximum
 constexpr int kCountUnroll = 8;   // 16-byte loads in flight per thread (tie count)
 constexpr int kHeadElems = 8192;  // elements of the first piece of stage 0 (bf16)
+constexpr int kChains = 4;        // statistics chains (16-byte vectors in flight) per thread
 
 struct RowSh {
   uint64_t full[kNStages];
@@ -255,28 +256,30 @@ __device__ Desc descend(Ring<Raw>& ring, float c, float m, int fx_shift, bool by
 // ---------------------------------------------------------------------------
 // the streamed pass
 
-// bf16 stage: every thread takes every kRT-th 16-byte vector, two in
-// flight, into its two statistics chains and, with a window, into the
+// bf16 stage: every thread takes every kRT-th 16-byte vector, kChains in
+// flight, each into its own statistics chain and, with a window, into the
 // exact-key histogram (elements outside the window into this lane's spill
 // bin, nb + lane).
 template <int MODE>
 __device__ __forceinline__ void stage_bf16(const uint16_t* st, int n, float c, f32x2 c2,
-                                           Chain (&ch)[2], uint32_t& vmax2, uint32_t wbase,
+                                           Chain (&ch)[kChains], uint32_t& vmax2, uint32_t wbase,
                                            uint32_t nb, uint32_t hist_s) {
   const int nv = n / 8;
   const uint4* v4 = reinterpret_cast<const uint4*>(st);
   const uint32_t spill = nb + (threadIdx.x & 31);
   int v = threadIdx.x;
-  for (; v + kRT < nv; v += 2 * kRT) {
-    const uint4 q0 = v4[v], q1 = v4[v + kRT];
-    chain_vec(q0, c, c2, ch[0], vmax2);
-    chain_vec(q1, c, c2, ch[1], vmax2);
+  for (; v + (kChains - 1) * kRT < nv; v += kChains * kRT) {
+    uint4 q[kChains];
+#pragma unroll
+    for (int k = 0; k < kChains; ++k) q[k] = v4[v + k * kRT];
+#pragma unroll
+    for (int k = 0; k < kChains; ++k) chain_vec(q[k], c, c2, ch[k], vmax2);
     if constexpr (MODE != kWinNone) {
-      hist_vec<MODE>(q0, wbase, spill, hist_s);
-      hist_vec<MODE>(q1, wbase, spill, hist_s);
+#pragma unroll
+      for (int k = 0; k < kChains; ++k) hist_vec<MODE>(q[k], wbase, spill, hist_s);
     }
   }
-  if (v < nv) {
+  for (; v < nv; v += kRT) {
     const uint4 q = v4[v];
     chain_vec(q, c, c2, ch[0], vmax2);
     if constexpr (MODE != kWinNone) hist_vec<MODE>(q, wbase, spill, hist_s);
@@ -294,7 +297,7 @@ __device__ __forceinline__ void stage_bf16(const uint16_t* st, int n, float c, f
 // first 16-byte boundary, whole vectors, then single elements again.
 template <int MODE>
 __device__ __forceinline__ void stage_range_bf16(const uint16_t* st, int j0, int j1, float c,
-                                                 f32x2 c2, Chain (&ch)[2], uint32_t& vmax2,
+                                                 f32x2 c2, Chain (&ch)[kChains], uint32_t& vmax2,
                                                  uint32_t wbase, uint32_t nb, uint32_t hist_s) {
   const uint32_t spill = nb + (threadIdx.x & 31);
   auto one = [&](uint32_t r) {
@@ -426,18 +429,28 @@ __device__ __forceinline__ Stats warp_stats(Stats s) {
 // (by_mass false) or fixed-point mass first reaches need (>= 1); chunks of
 // 256 bins, lane l holding bins hi - 8l - k (k = 0..7) of a chunk.  False
 // when the bins [0, top] hold less than need.
-__device__ bool warp_search(const Window& w, int top, bool by_mass, u64 need, Desc& out) {
+__device__ bool warp_search(const Window& w, int top, bool by_mass, u64 need, Desc& out,
+                            SupSums* above = nullptr) {
   const int lane = threadIdx.x & 31;
   u64 ac = 0, am = 0;  // above the current chunk
+  SupSums acc{0u, 0u, 0u, 0.f, 0.f};  // this lane's bins above the current chunk
   for (int hi = top; hi >= 0; hi -= 256) {
     uint32_t cnt[8];
     u64 fx[8];
+    float em8[8], ea8[8];
+    uint32_t topm = 0;  // bins holding the row maximum (d == 0)
     u64 lc = 0, lm = 0;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const int b = hi - 8 * lane - k;
       cnt[k] = b >= 0 ? w.hist[b] : 0u;
-      fx[k] = cnt[k] ? static_cast<u64>(cnt[k]) * bin_fx(w, w.klo + static_cast<uint32_t>(b)) : 0ull;
+      const float d = key_u(w.klo + static_cast<uint32_t>(b), w.c) - w.m;
+      const float e = ex2(d);
+      const float fc = static_cast<float>(cnt[k]);
+      fx[k] = cnt[k] ? static_cast<u64>(cnt[k]) * __float2ull_rn(e * w.fxs) : 0ull;
+      if (d == 0.f) topm |= 1u << k;
+      em8[k] = cnt[k] && d != 0.f ? fc * e : 0.f;  // the sums' terms, as in warp_sums
+      ea8[k] = cnt[k] ? fc * d * e : 0.f;
       lc += cnt[k];
       lm += fx[k];
     }
@@ -453,31 +466,45 @@ __device__ bool warp_search(const Window& w, int top, bool by_mass, u64 need, De
     const u64 ec = ac + pc - lc, em = am + pm - lm;
     const u64 base = by_mass ? em : ec, mine = by_mass ? lm : lc;
     const uint32_t ball = __ballot_sync(0xffffffffu, base < need && need <= base + mine);
-    if (ball) {
-      const int src = __ffs(ball) - 1;
-      uint32_t key = 0;
-      u64 rc = ec, rm = em, at_c = 0, at_m = 0;
-      if (lane == src) {
-        bool done = false;
+    const int src = ball ? __ffs(ball) - 1 : 32;
+    // this lane's bins above the crossing (all of them before it is found)
+    uint32_t key = 0;
+    u64 rc = ec, rm = em, at_c = 0, at_m = 0;
+    bool done = lane > src;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          if (!done && cnt[k] && (by_mass ? rm + fx[k] : rc + cnt[k]) >= need) {
-            key = w.klo + static_cast<uint32_t>(hi - 8 * lane - k);
-            at_c = cnt[k];
-            at_m = fx[k];
-            done = true;
-          }
-          if (!done) {
-            rc += cnt[k];
-            rm += fx[k];
-          }
-        }
+    for (int k = 0; k < 8; ++k) {
+      if (!done && lane == src && cnt[k] && (by_mass ? rm + fx[k] : rc + cnt[k]) >= need) {
+        key = w.klo + static_cast<uint32_t>(hi - 8 * lane - k);
+        at_c = cnt[k];
+        at_m = fx[k];
+        done = true;
       }
+      if (!done) {
+        rc += cnt[k];
+        rm += fx[k];
+        acc.ngt += cnt[k];
+        if ((topm >> k) & 1u) acc.ntp += cnt[k];
+        acc.smass += em8[k];
+        acc.sa += ea8[k];
+      }
+    }
+    if (ball) {
       out.key = __shfl_sync(0xffffffffu, key, src);
       out.above_cnt = __shfl_sync(0xffffffffu, rc, src);
       out.above_mass = __shfl_sync(0xffffffffu, rm, src);
       out.at_cnt = __shfl_sync(0xffffffffu, at_c, src);
       out.at_mass = __shfl_sync(0xffffffffu, at_m, src);
+      if (above) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          acc.ngt += __shfl_xor_sync(0xffffffffu, acc.ngt, o);
+          acc.ntp += __shfl_xor_sync(0xffffffffu, acc.ntp, o);
+          acc.smass += __shfl_xor_sync(0xffffffffu, acc.smass, o);
+          acc.sa += __shfl_xor_sync(0xffffffffu, acc.sa, o);
+        }
+        acc.neq = static_cast<uint32_t>(out.at_cnt);
+        *above = acc;
+      }
       return true;
     }
     ac += __shfl_sync(0xffffffffu, pc, 31);
@@ -705,7 +732,7 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
 
   // ---- the streamed pass: online statistics and the row maximum; for a
   // filtered bf16 row also the exact-key window histogram
-  Chain ch2[2] = {chain_empty(), chain_empty()};  // bf16 rows
+  Chain ch2[kChains];                             // bf16 rows
   uint32_t vmax2 = 0xFF80FF80u;                    // bf16 rows: packed running max
   Stats s2[2] = {stats_empty(), stats_empty()};    // fp32 rows
   float vmax = -kInf;
@@ -770,8 +797,8 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
     wlo = sh.w_lo;
     wbase = sh.w_base;
     wmode = sh.w_mode;
-    chain_seed(ch2[0], m0, c);
-    chain_seed(ch2[1], m0, c);
+#pragma unroll
+    for (int k = 0; k < kChains; ++k) chain_seed(ch2[k], m0, c);
     const uint32_t nb = (wtop - wlo) + 1u;
     const f32x2 c2 = pack2(c, c);
     // when the target's key lies in the window, the count of its key at
@@ -821,7 +848,8 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
   Stats s;
   if constexpr (kBf16) {
     s = ch2[0].s;
-    stats_merge(s, ch2[1].s);
+#pragma unroll
+    for (int k = 1; k < kChains; ++k) stats_merge(s, ch2[k].s);
     vmax = vmax_of(vmax2);
   } else {
     s = s2[0];
@@ -848,6 +876,9 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
       bool win_ok = kmr <= wtop;
       bool all_ties = true, have_t = false;
       u64 cnum = 0;
+      SupSums psums{0u, 0u, 0u, 0.f, 0.f};  // the sums above the top-p crossing
+      bool have_psums = false;
+      uint32_t dp_key = 0;
       if (win_ok && (use_k || use_p)) {
         const int top = static_cast<int>(kmr - wlo);
         Desc dk{}, dp{};
@@ -867,7 +898,9 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
                                      : (static_cast<double>(s.c0) + static_cast<double>(s.zr)) *
                                            static_cast<double>(fxs);
           const u64 tp = topp_target(pp, mass1);
-          win_ok = warp_search(w, top, true, tp, dp);
+          win_ok = warp_search(w, top, true, tp, dp, &psums);
+          have_psums = win_ok;
+          dp_key = dp.key;
           if (win_ok) {
             u64 cp = topp_ties(dp, tp, bin_fx(w, dp.key));
             if (use_k && dp.key == o.tkey && cp > ck) cp = ck;
@@ -896,7 +929,8 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
         if (!win_ok || o.tkey < wlo) {
           fast = false;  // the support sums need a pass over the row
         } else {
-          const SupSums sums = warp_sums(w, o.tkey, kmr);
+          // the top-p search summed the bins above its key on the way down
+          const SupSums sums = have_psums && o.tkey == dp_key ? psums : warp_sums(w, o.tkey, kmr);
           const u64 tot_eq = sums.neq;
           o.ckeep = all_ties ? tot_eq : (cnum < tot_eq ? cnum : tot_eq);
           support_stats(o, sums, c);

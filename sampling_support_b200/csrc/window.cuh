@@ -73,43 +73,6 @@ __device__ __forceinline__ void hist_vec(const uint4& q, uint32_t base, uint32_t
   }
 }
 
-// One shared-memory count increment at address a when idx < nb (a
-// predicated reduction: lanes outside the window issue no access, so they
-// add no bank traffic).
-__device__ __forceinline__ void red_inc_if(uint32_t a, uint32_t idx, uint32_t nb) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.lt.u32 p, %1, %2;\n @p red.shared.add.u32 [%0], 1;\n}\n" ::"r"(a),
-      "r"(idx), "r"(nb)
-      : "memory");
-}
-
-// As hist_vec, but elements outside the window are not counted at all (no
-// spill bins): the index is compared with the bin count nb.
-template <int MODE>
-__device__ __forceinline__ void hist_vec_pred(const uint4& q, uint32_t base, uint32_t nb,
-                                              uint32_t hist_s) {
-  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-  if constexpr (MODE == kWinPos || MODE == kWinNeg) {
-    const uint32_t off = MODE == kWinPos ? ((0u - base) & 0xFFFFu) : ((0u - (0xFFFFu - base)) & 0xFFFFu);
-    const uint32_t off2 = off | (off << 16);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint32_t x = MODE == kWinNeg ? ~w[i] : w[i];
-      asm("add.u16x2 %0, %1, %2;" : "=r"(x) : "r"(x), "r"(off2));
-      const uint32_t lo = x & 0xFFFFu, hi = x >> 16;
-      red_inc_if(hist_s + (lo << 2), lo, nb);
-      red_inc_if(hist_s + (hi << 2), hi, nb);
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t lo = win_index<MODE>(w[i] & 0xFFFFu, base), hi = win_index<MODE>(w[i] >> 16, base);
-      red_inc_if(hist_s + (lo << 2), lo, nb);
-      red_inc_if(hist_s + (hi << 2), hi, nb);
-    }
-  }
-}
-
 // The bin mapping of the window of keys [lo, hi] (at most kSelWin keys).
 // The sign-specific modes index with 16-bit lane arithmetic; they are
 // chosen only when every raw pattern of the other sign lands at an index of
