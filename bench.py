@@ -407,6 +407,53 @@ def time_steps(fn, warmup, steps):
     return a.elapsed_time(b) / steps
 
 
+def time_graph(fn, warmup, steps, flush=None, per_graph=16):
+    """Device time of one fn() call: the calls captured in a CUDA graph of
+    per_graph calls and replayed (no host gaps between calls).  With flush (a
+    callable writing a buffer larger than L2), every call is preceded by a
+    flush, and the time of a graph of flushes alone is subtracted."""
+    import torch
+
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+
+    def capture(body):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(per_graph):
+                body()
+        return g
+
+    def run(g):
+        g.replay()
+        torch.cuda.synchronize()
+        reps = max(1, steps // per_graph)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s = torch.cuda.current_stream()
+        a.record(s)
+        for _ in range(reps):
+            g.replay()
+        b.record(s)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / (reps * per_graph)
+
+    if flush is None:
+        g = capture(fn)
+        ms = run(g)
+        del g
+        return ms
+
+    def both():
+        flush()
+        fn()
+
+    g1, g0 = capture(both), capture(flush)
+    ms = run(g1) - run(g0)
+    del g1, g0
+    return ms
+
+
 def secondary(args, pk, only=None):
     """The secondary workloads (all, or the one named by `only`)."""
     import torch
@@ -447,7 +494,7 @@ def distance_workload(args, pk, steps, out):
         res["o"] = vsb.l1_distance(d, t, wt, want_loss=True, want_grad=True,
                                    grad_dtype=torch.bfloat16, workspace=ws)
 
-    ms = time_steps(l1_step, 3, steps)
+    ms = time_graph(l1_step, 3, steps)
     nbytes = 2 * w["draft"].nbytes + w["draft"].nbytes
     out["distance"] = {"rows": 512, "ms_per_step": ms, "rows_per_s": 512 / (ms / 1e3),
                        "gbs": nbytes / (ms / 1e3) / 1e9, "frac_hbm": nbytes / (ms / 1e3) / 1e9 / pk["hbm"],
@@ -484,29 +531,36 @@ def replay_workload(args, pk, steps, out):
     dlog = torch.empty((8192, VOCAB), dtype=torch.bfloat16, device="cuda")
     holder = {}
 
+    # the forward touches ~59 MB, less than L2: every timed call starts from
+    # a flushed L2
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def l2_flush():
+        flush_buf.zero_()
+
     def rp_fwd():
         holder["o"] = vsb.score_fwd(lg, tg, support_ids=st, want_full=False, want_grad=True)
 
-    ms_f = time_steps(rp_fwd, 3, steps)
+    ms_f = time_graph(rp_fwd, 3, steps, flush=l2_flush)
 
     def rp_bwd():
         vsb.score_bwd(lg, tg, holder["o"]["ctx"], None, gl, None, gh, support_ids=st, out=dlog)
 
-    ms_b = time_steps(rp_bwd, 3, steps)
+    ms_b = time_graph(rp_bwd, 3, steps, flush=l2_flush)
 
     # the variants: full-vocabulary statistics for every row (a full read of
     # every row), and the sparse [rows, width] gradient of the support entries
     def rp_fwd_full():
         holder["f"] = vsb.score_fwd(lg, tg, support_ids=st, want_full=True, want_grad=True)
 
-    ms_ff = time_steps(rp_fwd_full, 3, steps)
+    ms_ff = time_graph(rp_fwd_full, 3, steps, flush=l2_flush)
     sg = torch.empty((8192, st.shape[1]), dtype=torch.float32, device="cuda")
 
     def rp_bwd_sparse():
         vsb.score_bwd(lg, tg, holder["o"]["ctx"], None, gl, None, gh, support_ids=st, out=sg,
                       mode=vsb.VS_GRAD_SPARSE)
 
-    ms_bs = time_steps(rp_bwd_sparse, 3, steps)
+    ms_bs = time_graph(rp_bwd_sparse, 3, steps, flush=l2_flush)
     wbytes = dlog.numel() * 2
     empty = int((w["widths"] == 0).sum())
     # forward bytes: ids, one 32-byte sector per kept id, full rows of the
@@ -580,7 +634,6 @@ def sample_workload(args, pk, steps, out):
         a.sample_seed = 1234
         argsets.append(a)
     ws = B.score_workspace(lib.vs_score_fwd_workspace_size(ctypes.byref(argsets[0])), dev)
-    sp = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     oref = ctypes.byref(o)
     it = [0]
 
@@ -589,11 +642,12 @@ def sample_workload(args, pk, steps, out):
         a.sample_seed = 1234 + it[0]
         it[0] += 1
         rc = lib.vs_score_fwd(ctypes.byref(a), oref, 0 if ws is None else ws.data_ptr(),
-                              0 if ws is None else ws.numel(), sp)
+                              0 if ws is None else ws.numel(),
+                              ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
         if rc:
             raise RuntimeError(lib.vs_last_error().decode())
 
-    ms = time_steps(step, 3, max(20, min(steps, 500)))
+    ms = time_graph(step, 3, max(32, min(steps, 512)))
     out["sample"] = {"rows": rows, "vocab": w["vocab"], "ms_per_step": ms,
                      "rows_per_s": rows / (ms / 1e3),
                      "note": "fullvocab scoring (top-p 0.95, entropy) plus one seeded Gumbel-max "
@@ -684,20 +738,7 @@ def lmhead_workload(args, pk, steps, out, fused=True, support=True):
         def sh_step():
             vsb.support_lmhead_score(hs, wt, ty, w["temperature"], ids)
 
-        for _ in range(3):
-            sh_step()
-        torch.cuda.synchronize()
-        n = max(5, min(steps, 20))
-        tot = 0.0
-        for _ in range(n):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(s)
-            sh_step()
-            b.record(s)
-            torch.cuda.synchronize()
-            tot += a.elapsed_time(b)
-        ms = tot / n
+        ms = time_graph(sh_step, 3, max(32, min(steps, 64)), flush=flush.zero_)
         kept = int(sum(len(set(int(x) for x in r if x >= 0)) for r in sup["support"]))
         uniq = len(set(int(x) for x in sup["support"].reshape(-1) if x >= 0))
         gathered = 2 * w["hidden"] * (w["rows"] + kept) + 4 * sup["support"].size + 17 * w["rows"]

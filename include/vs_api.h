@@ -163,8 +163,14 @@ typedef struct vs_score_out {
  * the row) are computed for every row when logprob_full or entropy_full is
  * requested, else only for rows whose S is empty (the lp_V fallback).
  *
- * Workspace: none.  Each row is streamed through one CTA; the workspace
- * arguments are kept for ABI stability and ignored (pass NULL, 0).
+ * Workspace: none for computed supports and for recorded lists wider than
+ * 64 ids (pass NULL, 0).  Recorded lists of up to 64 ids need
+ * vs_score_fwd_workspace_size(args) bytes, 16-byte aligned, owned by the
+ * caller and not shared by calls that may run at the same time: it holds
+ * the list of rows that need full-vocabulary statistics and one partial
+ * per (row, chunk) of them (4,096 ids for bf16, 2,048 for fp32), so that
+ * those rows' reads spread over every SM.  VS_ERR_WORKSPACE when it is
+ * missing, misaligned or too small.
  *
  * Returns VS_ERR_INVALID_ARG for NULL required pointers, R < 0, V < 1,
  * ld < V, bad alignment, a non-positive or non-finite temperature_scalar,
@@ -177,7 +183,10 @@ typedef struct vs_score_out {
 vs_status vs_score_fwd(const vs_score_args* args, const vs_score_out* out, void* workspace,
                        size_t workspace_bytes, void* stream);
 
-/* Workspace bytes vs_score_fwd needs for these arguments: always 0. */
+/* Workspace bytes vs_score_fwd needs for these arguments: 0 for computed
+ * supports and recorded lists wider than 64 ids; for narrower recorded
+ * lists 16 + 2 r16(4 rows) + r16(20 rows ceil(vocab / chunk)), chunk =
+ * 4,096 (bf16) or 2,048 (fp32), r16 rounding up to a multiple of 16. */
 size_t vs_score_fwd_workspace_size(const vs_score_args* args);
 
 /* Largest vocabulary vs_score_fwd accepts for a dtype. */

@@ -138,8 +138,8 @@ int32_t vs_score_max_vocab(vs_dtype dtype) {
 }
 
 size_t vs_score_fwd_workspace_size(const vs_score_args* args) {
-  (void)args;
-  return 0;
+  if (!args || !args->support_ids || args->rows <= 0 || args->vocab <= 0) return 0;
+  return vs::score_recorded_workspace_bytes(args->rows, args->vocab, args->support_width, args->dtype);
 }
 
 vs_status vs_score_fwd(const vs_score_args* a, const vs_score_out* o, void* workspace,
@@ -167,8 +167,12 @@ vs_status vs_score_fwd(const vs_score_args* a, const vs_score_out* o, void* work
   const bool recorded = a->support_ids != nullptr;
   if (!recorded && a->vocab > vs::score_max_vocab(a->dtype))
     return fail(VS_ERR_UNSUPPORTED, "vocab exceeds vs_score_max_vocab for this dtype");
-  (void)workspace;
-  (void)workspace_bytes;
+  if (recorded) {
+    const size_t need = vs::score_recorded_workspace_bytes(a->rows, a->vocab, a->support_width, a->dtype);
+    if (need && (!workspace || !aligned16(workspace) || workspace_bytes < need))
+      return fail(VS_ERR_WORKSPACE,
+                  "workspace missing, misaligned or smaller than vs_score_fwd_workspace_size");
+  }
 
   vs::ScoreParams p{};
   p.rows = a->rows;
@@ -209,7 +213,7 @@ vs_status vs_score_fwd(const vs_score_args* a, const vs_score_out* o, void* work
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (recorded)
-    e = vs::launch_score_recorded(p, a->dtype, s);
+    e = vs::launch_score_recorded(p, a->dtype, workspace, s);
   else
     e = vs::launch_score_computed(p, a->dtype, s);
   if (e != cudaSuccess) return cuda_fail(e, "vs_score_fwd launch");

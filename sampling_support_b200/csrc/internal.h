@@ -94,7 +94,10 @@ struct BwdParams {
 
 // launchers (return a cudaError_t from the launch)
 cudaError_t launch_score_computed(const ScoreParams& p, vs_dtype dtype, cudaStream_t s);
-cudaError_t launch_score_recorded(const ScoreParams& p, vs_dtype dtype, cudaStream_t s);
+// Recorded supports.  Lists of up to 64 ids need a workspace of
+// score_recorded_workspace_bytes (16-byte aligned); wider lists none.
+size_t score_recorded_workspace_bytes(int rows, int vocab, int width, vs_dtype dtype);
+cudaError_t launch_score_recorded(const ScoreParams& p, vs_dtype dtype, void* ws, cudaStream_t s);
 cudaError_t launch_score_reduce(const float* h_support, const uint8_t* valid, int rows,
                                 double* entropy_sum, int32_t* valid_count, cudaStream_t s);
 cudaError_t launch_score_bwd(const BwdParams& p, vs_dtype dtype, vs_dtype gdtype, int mode,

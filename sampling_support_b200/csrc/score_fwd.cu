@@ -317,15 +317,173 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
 }
 
 // ---------------------------------------------------------------------------
+// full-vocabulary statistics of the rows that need them (an empty recorded
+// support, or every row when they are requested), spread over the whole GPU:
+// a list of those rows, then (row, chunk) work items of one warp's 32 x
+// kFsVecs 16-byte vectors taken by a persistent grid of warps, each writing
+// one partial; the warp-per-row kernel merges a row's partials.
+
+constexpr int kFsVecs = 16;        // 16-byte vectors per lane of one work item
+constexpr int kFsThreads = 256;
+
+// One work item's statistics and maximum (20 bytes).
+struct FsPart {
+  Stats s;
+  float vmax;
+};
+
+// Elements of one work item: one warp's 32 x kFsVecs vectors.
+__host__ __device__ inline int fs_chunk(int esize) { return 32 * kFsVecs * (16 / esize); }
+
+// Workspace of the narrow-list recorded path: [count | slot[rows] | list[rows]
+// | parts[rows][nch]], 16-byte aligned pieces.
+struct FsLayout {
+  size_t slot, list, parts, bytes;
+  int nch;
+};
+__host__ __device__ inline FsLayout fs_layout(int rows, int vocab, int esize) {
+  FsLayout l;
+  const int ch = fs_chunk(esize);
+  l.nch = (vocab + ch - 1) / ch;
+  l.slot = 16;
+  l.list = l.slot + ((static_cast<size_t>(rows) * 4 + 15) & ~size_t(15));
+  l.parts = l.list + ((static_cast<size_t>(rows) * 4 + 15) & ~size_t(15));
+  l.bytes = l.parts + ((static_cast<size_t>(rows) * l.nch * sizeof(FsPart) + 15) & ~size_t(15));
+  return l;
+}
+
+__device__ __forceinline__ void fs_pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void fs_pdl_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// One warp per row: does the row need full-vocabulary statistics?  Those
+// rows are appended to the list (any order: each row's result does not
+// depend on its place) and their list index kept in slot[row] (-1: none).
+__global__ void __launch_bounds__(256) fs_list_kernel(ScoreParams P, int32_t* count, int32_t* slot,
+                                                       int32_t* list) {
+  fs_pdl_wait();
+  fs_pdl_launch();
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= P.rows) return;
+  const int32_t* srow = P.support_ids + static_cast<int64_t>(row) * P.support_ld;
+  bool any = false;
+  for (int w = lane; w < P.support_width; w += 32) {
+    const int32_t id = srow[w];
+    any |= id >= 0 && id < P.vocab;
+  }
+  const bool need = P.full_stats || !__any_sync(0xffffffffu, any);
+  if (lane == 0) {
+    int32_t idx = -1;
+    if (need) {
+      idx = atomicAdd(count, 1);
+      list[idx] = row;
+    }
+    slot[row] = idx;
+  }
+}
+
+// Persistent grid of warps over the work items (list index, chunk): each
+// warp takes every W-th item (W = the grid's warps), loads its 32 x kFsVecs
+// vectors at once and writes one partial, with no block barrier.
+template <typename Raw>
+__global__ void __launch_bounds__(kFsThreads) fs_chunk_kernel(ScoreParams P, const int32_t* count,
+                                                              const int32_t* list, FsPart* parts,
+                                                              int nch) {
+  constexpr int VEC = 16 / sizeof(Raw);
+  constexpr int CH = 32 * kFsVecs * VEC;
+  fs_pdl_wait();
+  fs_pdl_launch();
+  const int items = *count * nch;
+  const int lane = threadIdx.x & 31;
+  const int nw = gridDim.x * (kFsThreads / 32);
+  for (int it = blockIdx.x * (kFsThreads / 32) + (threadIdx.x >> 5); it < items; it += nw) {
+    const int row = list[it / nch];
+    const int j0 = (it % nch) * CH, j1 = min(P.vocab, j0 + CH);
+    const Raw* g = static_cast<const Raw*>(P.logits) + static_cast<int64_t>(row) * P.ld + j0;
+    const uint4* g4 = reinterpret_cast<const uint4*>(g);
+    const int nv = (j1 - j0) / VEC;
+    uint4 q[kFsVecs];
+#pragma unroll
+    for (int k = 0; k < kFsVecs; ++k) {
+      const int v = lane + 32 * k;
+      q[k] = v < nv ? __ldcs(g4 + v) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    const float T = P.temperature ? P.temperature[row] : P.temperature_scalar;
+    const float c = kLog2e / T;
+    Stats s = stats_empty();
+    float vmax = -kInf;
+    if constexpr (sizeof(Raw) == 2) {
+      // the chains start at the warp's largest value, so that only the
+      // vectors holding it take the scalar path
+      uint32_t vm2 = 0xFF80FF80u;
+#pragma unroll
+      for (int k = 0; k < kFsVecs; ++k)
+        if (lane + 32 * k < nv) vm2 = bmax2(vm2, bmax2(bmax2(q[k].x, q[k].y), bmax2(q[k].z, q[k].w)));
+      float seed = vmax_of(vm2);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) seed = fmaxf(seed, __shfl_xor_sync(0xffffffffu, seed, o));
+      Chain ch[2];
+      chain_seed(ch[0], seed, c);
+      chain_seed(ch[1], seed, c);
+      const f32x2 c2 = pack2(c, c);
+#pragma unroll
+      for (int k = 0; k < kFsVecs; ++k)
+        if (lane + 32 * k < nv) chain_vec(q[k], c, c2, ch[k & 1], vm2);
+      s = ch[0].s;
+      stats_merge(s, ch[1].s);
+      vmax = vmax_of(vm2);
+    } else {
+#pragma unroll
+      for (int k = 0; k < kFsVecs; ++k) {
+        if (lane + 32 * k >= nv) continue;
+        Raw r[VEC];
+        unpack(q[k], r);
+        float u[VEC];
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) {
+          const float x = value_of(r[i]);
+          vmax = fmaxf(vmax, x);
+          u[i] = __fmul_rn(x, c);
+        }
+        stats_add(s, u);
+      }
+    }
+    for (int j = nv * VEC + lane; j < j1 - j0; j += 32) {
+      const float x = value_of(g[j]);
+      vmax = fmaxf(vmax, x);
+      float u[1] = {__fmul_rn(x, c)};
+      stats_add(s, u);
+    }
+    // warp merge: the warp maximum, each lane rebased onto it once, sums
+    const float m = [&] {
+      float t = s.m;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, o));
+      return t;
+    }();
+    if (s.c0 != 0.f || s.zr != 0.f) stats_rebase(s, m);
+    float c0 = s.c0, zr = s.zr, a = s.a;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      c0 += __shfl_xor_sync(0xffffffffu, c0, o);
+      zr += __shfl_xor_sync(0xffffffffu, zr, o);
+      a += __shfl_xor_sync(0xffffffffu, a, o);
+      vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+    }
+    if (lane == 0) parts[it] = FsPart{Stats{m, c0, zr, a}, vmax};
+  }
+}
+
+// ---------------------------------------------------------------------------
 // recorded support, narrow lists (width <= 64): one warp per row for the
-// gather and the support statistics, 16 rows per 512-thread CTA; the rows
-// that need full-vocabulary statistics (an empty support, or all rows when
-// they are requested) are then streamed one after another by the whole CTA.
+// gather and the support statistics, 16 rows per 512-thread CTA; the
+// full-vocabulary statistics that a row needs (an empty support, or all
+// rows when they are requested) come merged from fs_chunk_kernel's partials.
 
 constexpr int kWarpRows = 16;           // rows per CTA, one per warp
 constexpr int kWarpRowThreads = 512;
 constexpr int kWarpRowMaxWidth = 64;    // two list slots per lane
-constexpr int kStreamUnroll = 8;        // 16-byte loads in flight per thread (full-row stream)
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -339,13 +497,9 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 template <typename Raw>
-__global__ void __launch_bounds__(kWarpRowThreads, 1) score_recorded_warp_kernel(ScoreParams P) {
-  constexpr int VEC = 16 / sizeof(Raw);
-  __shared__ uint32_t need_full[kWarpRows];
-  __shared__ Stats fstat[kWarpRows];
-  __shared__ float fmaxv[kWarpRows];
-  __shared__ Stats red[kWarpRowThreads / 32];
-  __shared__ float fred[kWarpRowThreads / 32];
+__global__ void __launch_bounds__(kWarpRowThreads) score_recorded_warp_kernel(
+    ScoreParams P, const int32_t* slot, const FsPart* parts, int nch) {
+  fs_pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * kWarpRows + warp;
   const bool row_ok = row < P.rows;
@@ -405,97 +559,29 @@ __global__ void __launch_bounds__(kWarpRowThreads, 1) score_recorded_warp_kernel
     s.a = warp_sum(a);
   }
   const bool need = row_ok && (empty || P.full_stats);
-  if (lane == 0) need_full[warp] = need ? 1u : 0u;
-  __syncthreads();
-
-  // ---- phase B (whole CTA, one row at a time): full-vocabulary statistics
-  for (int r = 0; r < kWarpRows; ++r) {
-    if (!need_full[r]) continue;  // uniform
-    const int rr = blockIdx.x * kWarpRows + r;
-    const Raw* g = static_cast<const Raw*>(P.logits) + static_cast<int64_t>(rr) * P.ld;
-    const float Tr = P.temperature ? P.temperature[rr] : P.temperature_scalar;
-    const float cr = kLog2e / Tr;
-    const int nfull = V / VEC;
-    const uint4* g4 = reinterpret_cast<const uint4*>(g);
-    Stats f = stats_empty();
-    float fv = -kInf;
-    int v = threadIdx.x;
-    if constexpr (sizeof(Raw) == 2) {
-      Chain f4[2] = {chain_empty(), chain_empty()};
-      uint32_t vm2 = 0xFF80FF80u;
-      const f32x2 c2 = pack2(cr, cr);
-      uint4 q[kStreamUnroll];
-      uint32_t mx = 0xFF80FF80u;
-#pragma unroll
-      for (int k = 0; k < kStreamUnroll; ++k) {
-        const int vk = v + k * kWarpRowThreads;
-        q[k] = vk < nfull ? __ldcs(g4 + vk) : make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u);
-        mx = bmax2(mx, bmax2(bmax2(q[k].x, q[k].y), bmax2(q[k].z, q[k].w)));
-      }
-      float m1 = warp_max(fmaxf(__uint_as_float(mx << 16), __uint_as_float(mx & 0xFFFF0000u)));
-      if (lane == 0) fred[warp] = m1;
-      __syncthreads();
-      m1 = -kInf;
-      for (int i = 0; i < kWarpRowThreads / 32; ++i) m1 = fmaxf(m1, fred[i]);
-      __syncthreads();
-      chain_seed(f4[0], m1, cr);
-      chain_seed(f4[1], m1, cr);
-      for (;;) {
-#pragma unroll
-        for (int k = 0; k < kStreamUnroll; ++k)
-          if (v + k * kWarpRowThreads < nfull) chain_vec(q[k], cr, c2, f4[k & 1], vm2);
-        v += kStreamUnroll * kWarpRowThreads;
-        if (v >= nfull) break;
-#pragma unroll
-        for (int k = 0; k < kStreamUnroll; ++k) {
-          const int vk = v + k * kWarpRowThreads;
-          q[k] = vk < nfull ? __ldcs(g4 + vk) : make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
-      f = f4[0].s;
-      stats_merge(f, f4[1].s);
-      fv = fmaxf(fv, vmax_of(vm2));
-    } else {
-      for (; v < nfull; v += kWarpRowThreads) {
-        Raw rw[VEC];
-        unpack(__ldcs(g4 + v), rw);
-        float u[VEC];
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) {
-          const float x = value_of(rw[i]);
-          fv = fmaxf(fv, x);
-          u[i] = __fmul_rn(x, cr);
-        }
-        stats_add(f, u);
-      }
-    }
-    for (int j = nfull * VEC + threadIdx.x; j < V; j += kWarpRowThreads) {
-      const float x = value_of(g[j]);
-      fv = fmaxf(fv, x);
-      float u[1] = {__fmul_rn(x, cr)};
-      stats_add(f, u);
-    }
-    f = block_reduce(f, red);
-    fv = warp_max(fv);
-    if (lane == 0) fred[warp] = fv;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float t = -kInf;
-      for (int i = 0; i < kWarpRowThreads / 32; ++i) t = fmaxf(t, fred[i]);
-      fstat[r] = f;
-      fmaxv[r] = t;
-    }
-    __syncthreads();
-  }
   if (!row_ok) return;
 
-  // ---- phase C (warp per row): outputs
+  // ---- full-vocabulary statistics (need): this row's chunk partials,
+  // merged in a fixed order (lane l takes chunks l, l + 32, ... in order,
+  // then a shuffle tree; the merge is commutative, so every lane gets the
+  // same result)
   Stats f = stats_empty();
   float fvmax = -kInf;
-  if (need) {
-    f = fstat[warp];
-    fvmax = fmaxv[warp];
+  if (need && slot[row] >= 0) {
+    const FsPart* pr = parts + static_cast<int64_t>(slot[row]) * nch;
+    for (int k = lane; k < nch; k += 32) {
+      const FsPart pt = pr[k];
+      stats_merge(f, pt.s);
+      fvmax = fmaxf(fvmax, pt.vmax);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      stats_merge(f, shfl_xor(f, o));
+      fvmax = fmaxf(fvmax, __shfl_xor_sync(0xffffffffu, fvmax, o));
+    }
   }
+
+  // ---- phase C (warp per row): outputs
   const float nan = __int_as_float(0x7fc00000);
   if (lane == 0) {
     uint32_t status = flags;
@@ -645,13 +731,67 @@ int score_max_vocab(vs_dtype dtype) {
   return 1 << 26;
 }
 
-cudaError_t launch_score_recorded(const ScoreParams& p, vs_dtype dtype, cudaStream_t s) {
+size_t score_recorded_workspace_bytes(int rows, int vocab, int width, vs_dtype dtype) {
+  return width <= kWarpRowMaxWidth ? fs_layout(rows, vocab, dtype == VS_BF16 ? 2 : 4).bytes : 0;
+}
+
+cudaError_t launch_score_recorded(const ScoreParams& p, vs_dtype dtype, void* ws, cudaStream_t s) {
   if (p.support_width <= kWarpRowMaxWidth) {
-    const unsigned grid = static_cast<unsigned>((p.rows + kWarpRows - 1) / kWarpRows);
-    if (dtype == VS_BF16)
-      score_recorded_warp_kernel<uint16_t><<<grid, kWarpRowThreads, 0, s>>>(p);
-    else
-      score_recorded_warp_kernel<uint32_t><<<grid, kWarpRowThreads, 0, s>>>(p);
+    if (!ws) return cudaErrorInvalidValue;
+    const FsLayout L = fs_layout(p.rows, p.vocab, dtype == VS_BF16 ? 2 : 4);
+    char* base = static_cast<char*>(ws);
+    int32_t* count = reinterpret_cast<int32_t*>(base);
+    int32_t* slot = reinterpret_cast<int32_t*>(base + L.slot);
+    int32_t* list = reinterpret_cast<int32_t*>(base + L.list);
+    FsPart* parts = reinterpret_cast<FsPart*>(base + L.parts);
+    cudaError_t e = cudaMemsetAsync(count, 0, sizeof(int32_t), s);
+    if (e != cudaSuccess) return e;
+    fs_list_kernel<<<static_cast<unsigned>((p.rows + 7) / 8), 256, 0, s>>>(p, count, slot, list);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // persistent grid: every resident CTA of the chunk kernel, once
+    static int grid_of[64][2] = {};
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const int which = dtype == VS_BF16 ? 0 : 1;
+    int grid = 148;
+    if (dev >= 0 && dev < 64 && grid_of[dev][which] > 0) {
+      grid = grid_of[dev][which];
+    } else {
+      int sms = 0, per = 0;
+      e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return e;
+      e = dtype == VS_BF16
+              ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fs_chunk_kernel<uint16_t>, kFsThreads, 0)
+              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fs_chunk_kernel<uint32_t>, kFsThreads, 0);
+      if (e != cudaSuccess) return e;
+      grid = sms * (per > 0 ? per : 1);
+      if (dev >= 0 && dev < 64) grid_of[dev][which] = grid;
+    }
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kFsThreads);
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = dtype == VS_BF16
+            ? cudaLaunchKernelEx(&cfg, fs_chunk_kernel<uint16_t>, p, static_cast<const int32_t*>(count),
+                                 static_cast<const int32_t*>(list), parts, L.nch)
+            : cudaLaunchKernelEx(&cfg, fs_chunk_kernel<uint32_t>, p, static_cast<const int32_t*>(count),
+                                 static_cast<const int32_t*>(list), parts, L.nch);
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3(static_cast<unsigned>((p.rows + kWarpRows - 1) / kWarpRows));
+    cfg.blockDim = dim3(kWarpRowThreads);
+    e = dtype == VS_BF16
+            ? cudaLaunchKernelEx(&cfg, score_recorded_warp_kernel<uint16_t>, p,
+                                 static_cast<const int32_t*>(slot), static_cast<const FsPart*>(parts), L.nch)
+            : cudaLaunchKernelEx(&cfg, score_recorded_warp_kernel<uint32_t>, p,
+                                 static_cast<const int32_t*>(slot), static_cast<const FsPart*>(parts), L.nch);
+    if (e != cudaSuccess) return e;
   } else if (dtype == VS_BF16) {
     score_recorded_kernel<uint16_t><<<p.rows, kRecThreads, 0, s>>>(p);
   } else {

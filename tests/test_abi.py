@@ -122,15 +122,25 @@ def test_l1_rejects_bad_arguments_and_small_workspace():
                 need - 8, None) == B.VS_ERR_WORKSPACE
 
 
-def test_score_fwd_needs_no_workspace():
-    """Every forward argument set streams its rows through one CTA each and
-    needs no scratch: the size query answers 0."""
+def test_score_fwd_workspace_size():
+    """Computed supports and wide recorded lists need no scratch; narrow
+    recorded lists (up to 64 ids) need the row list and one 20-byte partial
+    per (row, chunk of 4,096 bf16 or 2,048 fp32 ids)."""
     lib = vsb.load()
     size = lambda a: lib.vs_score_fwd_workspace_size(ctypes.byref(a))
     assert size(_args()) == 0
     assert size(_args(rows=1 << 20, vocab=151_936, ld=151_936)) == 0
     assert size(_args(dtype=B.VS_F32)) == 0
-    assert size(_args(support_ids=FAKE, support_width=8, support_ld=8)) == 0
+    assert size(_args(support_ids=FAKE, support_width=65, support_ld=65)) == 0
+    r16 = lambda n: (n + 15) // 16 * 16
+    for rows, vocab, width, dt, chunk in [(4, 1000, 8, B.VS_BF16, 4096),
+                                          (8192, 151_936, 64, B.VS_BF16, 4096),
+                                          (3, 4097, 1, B.VS_BF16, 4096),
+                                          (5, 151_936, 64, B.VS_F32, 2048)]:
+        a = _args(rows=rows, vocab=vocab, ld=vocab + (-vocab) % 8, dtype=dt, support_ids=FAKE,
+                  support_width=width, support_ld=width)
+        nch = (vocab + chunk - 1) // chunk
+        assert size(a) == 16 + 2 * r16(4 * rows) + r16(20 * rows * nch)
 
 
 def _support_head(rows=4, vocab=1000, hidden=64, H=FAKE, ldh=64, W=FAKE, ldw=64, temp=1.0,
