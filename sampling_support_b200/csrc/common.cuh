@@ -18,6 +18,17 @@ constexpr float kInf = __builtin_huge_valf();
 // hardware-defined interval per attempt, so this bounds a wait to seconds.
 constexpr uint32_t kWaitLimit = 1u << 24;
 
+// Block barrier entered by whole warps.  A warp whose lanes took different
+// paths since their last common instruction (one lane issuing a copy or an
+// atomic, lanes leaving a wait loop at different times) meets at __syncwarp
+// first: the block barrier instruction is an aligned one, which every lane
+// of a warp must execute together, and a warp that reaches it in pieces can
+// be counted more than once, letting the other warps through early.
+__device__ __forceinline__ void cta_sync() {
+  __syncwarp();
+  __syncthreads();
+}
+
 // Per-row status bit set when a bounded device wait gave up (never expected).
 constexpr uint32_t kRowDeviceTimeout = 1u << 5;  // VS_ROW_DEVICE_TIMEOUT
 
@@ -187,14 +198,14 @@ __device__ __forceinline__ Stats block_reduce(Stats s, Stats* scratch) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if (lane == 0) scratch[warp].m = m;
-  __syncthreads();
+  cta_sync();
   if (warp == 0) {
     float x = lane < nw ? scratch[lane].m : -kInf;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
     if (lane == 0) s_m = x;
   }
-  __syncthreads();
+  cta_sync();
   m = s_m;
   if (s.c0 != 0.f || s.zr != 0.f) stats_rebase(s, m);
   float c0 = s.c0, zr = s.zr, a = s.a;
@@ -205,7 +216,7 @@ __device__ __forceinline__ Stats block_reduce(Stats s, Stats* scratch) {
     a += __shfl_xor_sync(0xffffffffu, a, o);
   }
   if (lane == 0) scratch[warp] = Stats{m, c0, zr, a};
-  __syncthreads();
+  cta_sync();
   if (warp == 0) {
     float x0 = 0.f, x1 = 0.f, x2 = 0.f;
     if (lane < nw) {
@@ -221,7 +232,7 @@ __device__ __forceinline__ Stats block_reduce(Stats s, Stats* scratch) {
     }
     if (lane == 0) s_res = Stats{m, x0, x1, x2};
   }
-  __syncthreads();
+  cta_sync();
   return s_res;
 }
 
@@ -234,14 +245,14 @@ __device__ __forceinline__ T block_sum(T v, T* scratch) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   if (lane == 0) scratch[warp] = v;
-  __syncthreads();
+  cta_sync();
   if (warp == 0) {
     T x = lane < static_cast<int>(blockDim.x >> 5) ? scratch[lane] : T(0);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
     if (lane == 0) s_res = x;
   }
-  __syncthreads();
+  cta_sync();
   return s_res;
 }
 

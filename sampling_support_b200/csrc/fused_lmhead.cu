@@ -373,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   tc_fence_before();
-  __syncthreads();
+  cta_sync();
   if constexpr (PAIR) cluster_barrier();  // the peer's barriers are initialised
   tc_fence_after();
   const uint32_t tmem = bs->tmem_base;
@@ -643,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // teardown: every role has left its loop (bounded waits); make sure the
   // MMAs of this CTA have completed before the accumulators are freed
   tc_fence_before();
-  __syncthreads();
+  cta_sync();
   if constexpr (PAIR) cluster_barrier();  // the pair's MMAs and arrivals are done
   if (warp == 1) {
     tc_fence_after();

@@ -115,10 +115,10 @@ __device__ __forceinline__ unsigned long long block_max_key(unsigned long long k
     k = t > k ? t : k;
   }
   if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = k;
-  __syncthreads();
+  cta_sync();
   unsigned long long m = 0ull;
   for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) m = scratch[w] > m ? scratch[w] : m;
-  __syncthreads();
+  cta_sync();
   return m;
 }
 

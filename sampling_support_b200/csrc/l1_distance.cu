@@ -50,7 +50,7 @@ __device__ __forceinline__ float2 block_reduce2(float a, float b, L1Shared& sh) 
     b = MAX ? fmaxf(b, ob) : b + ob;
   }
   if (lane == 0) sh.red2[warp] = make_float2(a, b);
-  __syncthreads();
+  cta_sync();
   if (warp == 0) {
     float2 x = lane < kWarps ? sh.red2[lane] : make_float2(MAX ? -kInf : 0.f, MAX ? -kInf : 0.f);
 #pragma unroll
@@ -61,7 +61,7 @@ __device__ __forceinline__ float2 block_reduce2(float a, float b, L1Shared& sh) 
     }
     if (lane == 0) sh.res2 = x;
   }
-  __syncthreads();
+  cta_sync();
   return sh.res2;
 }
 
@@ -105,10 +105,10 @@ __device__ __forceinline__ float l1_block_max(float v, float* scratch) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = v;
-  __syncthreads();
+  cta_sync();
   float t = -kInf;
   for (int w = 0; w < kWarps; ++w) t = fmaxf(t, scratch[w]);
-  __syncthreads();
+  cta_sync();
   return t;
 }
 
@@ -222,7 +222,7 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
     sh.gathered[tid][0] = rsh->part[0];
     sh.gathered[tid][1] = rsh->part[1];
   }
-  __syncthreads();
+  cta_sync();
   Stats Sd = stats_empty(), St = stats_empty();
   for (uint32_t r = 0; r < CL; ++r) {
     stats_merge(Sd, sh.gathered[r][0]);
@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
     fence_barrier_init();
     sh.timeout = 0;
   }
-  __syncthreads();
+  cta_sync();
   const uint32_t bytes = static_cast<uint32_t>((static_cast<size_t>(n) * sizeof(Raw) + 15) & ~size_t(15));
   if (tid == 0 && bytes > 0) {
     mbar_arrive_expect_tx(&sh.bar, 2 * bytes);
@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
     atomicOr(&sh.timeout, 1u);
     mbar_wait(&sh.bar, 0);
   }
-  __syncthreads();
+  cta_sync();
 
   if constexpr (sizeof(Raw) == 2) {
     l1_rows_bf16<G>(bd, bt, n, c0, row, rank, CL, cluster, sh, P);
@@ -410,7 +410,7 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
     sh.gathered[tid][0] = rsh->part[0];
     sh.gathered[tid][1] = rsh->part[1];
   }
-  __syncthreads();
+  cta_sync();
   Stats Sd = stats_empty(), St = stats_empty();
   for (uint32_t r = 0; r < CL; ++r) {
     stats_merge(Sd, sh.gathered[r][0]);
@@ -555,7 +555,7 @@ __global__ void l1_wsum_kernel(const float* w, int rows, double* out) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if (lane == 0) red[warp] = s;
-  __syncthreads();
+  cta_sync();
   if (threadIdx.x == 0) {
     double t = 0.0;
     for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) t += red[i];
@@ -576,7 +576,7 @@ __global__ void l1_loss_kernel(const double* wl1, const double* wsum, const doub
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if (lane == 0) red[warp] = s;
-  __syncthreads();
+  cta_sync();
   if (threadIdx.x == 0) {
     double t = 0.0;
     for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) t += red[i];

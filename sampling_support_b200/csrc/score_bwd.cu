@@ -142,10 +142,10 @@ __global__ void __launch_bounds__(kThreads) score_bwd_kernel(BwdParams P, int nc
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, o));
     if ((threadIdx.x & 31) == 0) fred[threadIdx.x >> 5] = vm;
-    __syncthreads();
+    cta_sync();
     vm = -kInf;
     for (int i = 0; i < kThreads / 32; ++i) vm = fmaxf(vm, fred[i]);
-    __syncthreads();
+    cta_sync();
     float c0 = 0.f, zr = 0.f, a = 0.f;
     for (int j = threadIdx.x; j < V; j += blockDim.x) {
       const float d = (value_of(grow[j]) - vm) * k.c;
@@ -169,13 +169,13 @@ __global__ void __launch_bounds__(kThreads) score_bwd_kernel(BwdParams P, int nc
   if (recorded && k.need_sup) {
     const int words = (n + 31) / 32;
     for (int w = threadIdx.x; w < words; w += blockDim.x) bitmap[w] = 0u;
-    __syncthreads();
+    cta_sync();
     const int32_t* srow = P.support_ids + static_cast<int64_t>(row) * P.support_ld;
     for (int w = threadIdx.x; w < P.support_width; w += blockDim.x) {
       const int32_t id = srow[w];
       if (id >= c0 && id < c1) atomicOr(&bitmap[(id - c0) >> 5], 1u << ((id - c0) & 31));
     }
-    __syncthreads();
+    cta_sync();
   }
 
   auto in_support = [&](int jl, Raw raw) -> bool {

@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
     target_hit = 0;
   }
   for (int w = tid; w < W; w += blockDim.x) ids[w] = srow[w];
-  __syncthreads();
+  cta_sync();
 
   // kept: id valid and first occurrence; gather the kept values
   uint32_t local_flags = 0;
@@ -94,10 +94,10 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
   if ((tid & 31) == 0) fred[tid >> 5] = lmax;
-  __syncthreads();
+  cta_sync();
   float vsmax = -kInf;
   for (int i = 0; i < kRecThreads / 32; ++i) vsmax = fmaxf(vsmax, fred[i]);
-  __syncthreads();
+  cta_sync();
   Stats s{vsmax, 0.f, 0.f, 0.f};
   for (int w = tid; w < W; w += blockDim.x) {
     const float x = vals[w];
@@ -141,10 +141,10 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
       if ((tid & 31) == 0) fred[tid >> 5] = m1;
-      __syncthreads();
+      cta_sync();
       m1 = -kInf;
       for (int i = 0; i < kRecThreads / 32; ++i) m1 = fmaxf(m1, fred[i]);
-      __syncthreads();
+      cta_sync();
 #pragma unroll
       for (int k = 0; k < 4; ++k) chain_seed(f4[k], m1, c);
       for (;;) {
@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) fvmax = fmaxf(fvmax, __shfl_xor_sync(0xffffffffu, fvmax, o));
     if ((tid & 31) == 0) fred[tid >> 5] = fvmax;
-    __syncthreads();
+    cta_sync();
     fvmax = -kInf;
     for (int i = 0; i < kRecThreads / 32; ++i) fvmax = fmaxf(fvmax, fred[i]);
   }
@@ -305,7 +305,7 @@ __global__ void __launch_bounds__(kRecThreads) score_recorded_kernel(ScoreParams
     const int64_t wstride = (V + 31) / 32;
     uint32_t* mrow = P.support_mask + static_cast<int64_t>(row) * wstride;
     for (int64_t w = tid; w < wstride; w += blockDim.x) mrow[w] = 0u;
-    __syncthreads();
+    cta_sync();
     if (any_nf == 0) {
       for (int w = tid; w < W; w += blockDim.x) {
         const int32_t id = ids[w];
@@ -709,7 +709,7 @@ __global__ void score_reduce_kernel(const float* h_support, const uint8_t* valid
     dred[warp] = s;
     ired[warp] = cnt;
   }
-  __syncthreads();
+  cta_sync();
   if (threadIdx.x == 0) {
     double t = 0.0;
     int tc = 0;

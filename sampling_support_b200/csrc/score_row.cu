@@ -46,8 +46,8 @@ namespace {
 
 constexpr int kRT = 512;        // threads per row
 constexpr int kRW = kRT / 32;   // warps
-constexpr int kNStages = 6;     // ring depth
-constexpr int kStageBytes = 32768;
+constexpr int kNStages = 3;     // ring depth
+constexpr int kStageBytes = 65536;
 constexpr int kWin = kSelWin;
 constexpr int kBins = kSelBins;
 constexpr uint32_t kWinHi = 256;  // window keys above the first stage's maximum
@@ -55,9 +55,22 @@ constexpr int kCountUnroll = 8;   // 16-byte loads in flight per thread (tie cou
 constexpr int kHeadElems = 8192;  // elements of the first piece of stage 0 (bf16)
 constexpr int kChains = 4;        // statistics chains (16-byte vectors in flight) per thread
 
+// Everything the per-row outputs are made from.
+struct RowOut {
+  Stats s;
+  float vmax, m, log2z, h_full;
+  bool nonfinite, filtered, cut_known;
+  uint32_t tkey;
+  int32_t tie_cut;
+  u64 ckeep;
+  uint32_t ylt;
+  float log2zs, h_support, c0s, zrs;
+  int32_t n_support;
+};
+
 struct RowSh {
   uint64_t full[kNStages];
-  uint64_t empty[kNStages];
+  uint32_t done[kNStages];  // warps done with each ring slot in its current use
   uint64_t first;  // the first piece of stage 0 (bf16 rows), loaded apart
   Stats rs;        // the row's merged statistics (warp 0)
   float rvmax;     // the row maximum (warp 0)
@@ -66,14 +79,14 @@ struct RowSh {
   float w_m0;      // the first piece's maximum (warp 0)
   uint32_t w_top, w_lo, w_base;  // the window (warp 0)
   int32_t w_mode;
-  uint32_t ysnap;  // elements before the target holding its key (window rows)
+  uint32_t ylt_group;  // fast path: the target's tie group size when its rank there decides
+  RowOut rout;     // fast path: the row's outputs while that rank is counted
   Stats wst[kRW];
   float fred[kRW];
   uint32_t ured[kRW];
   u64 ulred[kRW];
   SelShared<kRW> sel;
   SupSums sums[kRW];
-  uint32_t outstanding;  // loads issued and not yet consumed (broadcast by thread 0)
   int32_t tie_cut;
   uint32_t timeout;
   unsigned long long kred[kRW];
@@ -98,20 +111,13 @@ struct Ring {
   int V;
   Raw* buf;      // [kNStages][SE]
   RowSh* sh;
-  uint32_t ld;   // loads issued (thread 0)
-  uint32_t cs;   // stages consumed (all threads)
+  uint32_t cs;   // stages consumed (every thread, in step)
+  uint32_t head;  // bytes at the start of stage 0 already requested apart (thread 0)
   __device__ int nst() const { return (V + SE - 1) / SE; }
   __device__ int count(int si) const { return min(SE, V - si * SE); }
 
-  uint32_t head;  // bytes at the start of stage 0 already requested apart (thread 0)
-
-  // thread 0: load stage si into the next ring slot
-  __device__ void issue(int si) {
-    const uint32_t L = ld++;
-    const int slot = L % kNStages;
-    if (L >= kNStages && !mbar_wait(&sh->empty[slot], ((L / kNStages) - 1u) & 1u)) {
-      sh->timeout = 1u;
-    }
+  // one thread: load stage si into ring slot `slot`, which no warp reads
+  __device__ void issue(int si, int slot) {
     const uint32_t bytes = static_cast<uint32_t>((count(si) * sizeof(Raw) + 15) & ~size_t(15));
     const uint32_t skip = si == 0 ? min(head, bytes) : 0u;
     if (si == 0) head = 0;
@@ -122,41 +128,49 @@ struct Ring {
                     bytes - skip, &sh->full[slot]);
   }
 
-  // thread 0 requests the first stages of [s0, s1)
+  // thread 0 requests the first stages of [s0, s1) into the slots that
+  // follow the consumed ones (all free between passes)
   __device__ void start(int s0, int s1) {
     if (threadIdx.x == 0)
-      for (int si = s0; si < min(s1, s0 + kNStages); ++si) issue(si);
+      for (int i = 0; i < min(s1 - s0, kNStages); ++i)
+        issue(s0 + i, static_cast<int>((cs + static_cast<uint32_t>(i)) % kNStages));
   }
 
   // Run f(stage_ptr, n, base) over stages [s0, s1) in order, after
-  // start(s0, s1); f returns true (uniformly) to stop early.  Loads already
+  // start(s0, s1); f returns true (uniformly) to stop early.  Each warp
+  // counts itself out of a slot once done with it, and the warp that
+  // completes the count refills the slot with the stage kNStages further
+  // on, so no thread waits for the others to release a slot.  Loads already
   // issued are drained either way.
   template <typename F>
   __device__ void consume(int s0, int s1, F&& f) {
-    int next = s0 + kNStages;
     bool stop = false;
-    for (int si = s0; si < s1 && !stop; ++si) {
-      const int slot = cs % kNStages;
+    int si = s0;
+    for (; si < s1 && !stop; ++si) {
+      const int slot = static_cast<int>(cs % kNStages);
       if (!mbar_wait(&sh->full[slot], (cs / kNStages) & 1u)) atomicOr(&sh->timeout, 1u);
       stop = f(buf + static_cast<size_t>(slot) * SE, count(si), si * SE);
-      __syncwarp();
-      if ((threadIdx.x & 31) == 0) mbar_arrive_cnt(&sh->empty[slot]);
       ++cs;
-      if (threadIdx.x == 0 && !stop && next < s1) issue(next);
-      ++next;
-    }
-    // drain loads that were issued but not consumed (early stop)
-    if (threadIdx.x == 0) sh->outstanding = ld;  // ld is thread 0's count
-    __syncthreads();
-    const uint32_t issued = sh->outstanding;
-    while (cs < issued) {
-      const int slot = cs % kNStages;
-      if (!mbar_wait(&sh->full[slot], (cs / kNStages) & 1u)) atomicOr(&sh->timeout, 1u);
       __syncwarp();
-      if ((threadIdx.x & 31) == 0) mbar_arrive_cnt(&sh->empty[slot]);
-      ++cs;
+      if ((threadIdx.x & 31) == 0 && release_slot(&sh->done[slot])) {
+        sh->done[slot] = 0u;
+        const int next = si + kNStages;
+        if (!stop && next < s1) {
+          fence_proxy_async();
+          issue(next, slot);
+        }
+      }
     }
-    __syncthreads();
+    if (stop) {
+      // stages [si, min(s1, si - 1 + kNStages)) were requested and not read
+      const int end = min(s1, si - 1 + kNStages);
+      for (; si < end; ++si) {
+        const int slot = static_cast<int>(cs % kNStages);
+        if (!mbar_wait(&sh->full[slot], (cs / kNStages) & 1u)) atomicOr(&sh->timeout, 1u);
+        ++cs;
+      }
+    }
+    cta_sync();
   }
 
   template <typename F>
@@ -165,8 +179,15 @@ struct Ring {
     consume(s0, s1, static_cast<F&&>(f));
   }
 
-  __device__ static void mbar_arrive_cnt(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+  // One warp done with a slot (acquire-release, CTA scope): true for the
+  // warp that completes the slot's count.
+  __device__ static bool release_slot(uint32_t* done) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;"
+                 : "=r"(old)
+                 : "r"(smem_addr(done))
+                 : "memory");
+    return old == static_cast<uint32_t>(kRW - 1);
   }
 };
 
@@ -187,7 +208,7 @@ __device__ Desc descend(Ring<Raw>& ring, float c, float m, int fx_shift, bool by
       ra.cnt[b] = 0;
       ra.mass[b] = 0;
     }
-    __syncthreads();
+    cta_sync();
     const int pshift = shift + 8;
     const uint32_t pre = prefix;
     auto one = [&](Raw raw) {
@@ -236,20 +257,20 @@ __device__ Desc descend(Ring<Raw>& ring, float c, float m, int fx_shift, bool by
         sh.ulred[0] = tgt;
       }
     }
-    __syncthreads();
+    cta_sync();
     target = sh.ulred[0];
     above_cnt += sh.sel.b_above_cnt;
     above_mass += sh.sel.b_above_mass;
     prefix = (prefix << 8) | sh.sel.b_key;
     out.at_cnt = sh.sel.b_at_cnt;
     out.at_mass = sh.sel.b_at_mass;
-    __syncthreads();
+    cta_sync();
   }
   out.key = prefix;
   out.above_cnt = above_cnt;
   out.above_mass = above_mass;
   sh.ulred[1] = target;  // the resolved target (for the implicit top-p case)
-  __syncthreads();
+  cta_sync();
   return out;
 }
 
@@ -293,30 +314,6 @@ __device__ __forceinline__ void stage_bf16(const uint16_t* st, int n, float c, f
   }
 }
 
-// Elements [j0, j1) of a bf16 stage (any bounds): single elements up to the
-// first 16-byte boundary, whole vectors, then single elements again.
-template <int MODE>
-__device__ __forceinline__ void stage_range_bf16(const uint16_t* st, int j0, int j1, float c,
-                                                 f32x2 c2, Chain (&ch)[kChains], uint32_t& vmax2,
-                                                 uint32_t wbase, uint32_t nb, uint32_t hist_s) {
-  const uint32_t spill = nb + (threadIdx.x & 31);
-  auto one = [&](uint32_t r) {
-    vmax2 = bmax2(vmax2, r | (r << 16));
-    float u[1] = {__fmul_rn(value_of(static_cast<uint16_t>(r)), c)};
-    stats_add(ch[0].s, u);
-    if constexpr (MODE != kWinNone) red_inc(hist_s + (min(win_index<MODE>(r, wbase), spill) << 2));
-  };
-  const int a = min(j1, (j0 + 7) & ~7);
-  for (int j = j0 + static_cast<int>(threadIdx.x); j < a; j += kRT) one(st[j]);
-  const uint4* v4 = reinterpret_cast<const uint4*>(st);
-  for (int v = a / 8 + static_cast<int>(threadIdx.x); v < j1 / 8; v += kRT) {
-    const uint4 q = v4[v];
-    chain_vec(q, c, c2, ch[0], vmax2);
-    if constexpr (MODE != kWinNone) hist_vec<MODE>(q, wbase, spill, hist_s);
-  }
-  for (int j = max(a, (j1 / 8) * 8) + static_cast<int>(threadIdx.x); j < j1; j += kRT) one(st[j]);
-}
-
 __device__ __forceinline__ void stats_stage_f32(const uint32_t* st, int n, float c, Stats (&s2)[2],
                                                 float& vmax) {
   Stats& s = s2[0];
@@ -358,13 +355,13 @@ __device__ __forceinline__ SupSums block_sum_sup(SupSums v, RowSh& sh) {
   };
   warp_sum(v);
   if ((threadIdx.x & 31) == 0) sh.sums[threadIdx.x >> 5] = v;
-  __syncthreads();
+  cta_sync();
   if (threadIdx.x < 32) {
     SupSums t = threadIdx.x < kRW ? sh.sums[threadIdx.x] : SupSums{0u, 0u, 0u, 0.f, 0.f};
     warp_sum(t);
     if (threadIdx.x == 0) s_res = t;
   }
-  __syncthreads();
+  cta_sync();
   return s_res;
 }
 
@@ -399,6 +396,21 @@ __device__ __forceinline__ uint32_t count_raw(const uint16_t* g, int j0, int j1,
   for (; v < nv; v += kRT) vec(__ldcg(v4 + v));
   for (int j = ja + nv * 8 + static_cast<int>(threadIdx.x); j < j1; j += kRT) one(g[j]);
   return n;
+}
+
+// Elements before position y holding the target's key tkey, for a target in
+// a tie group of `group` elements: counted by the block on the shorter side
+// of y (after y: the group less the target and the ties that follow it).
+// Every thread gets the count.
+__device__ __forceinline__ uint32_t ties_before_target(const uint16_t* g16, int V, int y,
+                                                       uint32_t tkey, uint32_t group,
+                                                       uint32_t* red) {
+  const uint32_t r0 = tkey >= 0x7FFFu ? tkey - 0x7FFFu : 0xFFFFu - tkey;
+  const uint32_t r1 = tkey == 0x7FFFu ? 0x8000u : r0;  // -0 shares the key of +0
+  const bool before = y <= V - 1 - y;
+  const uint32_t part = before ? count_raw(g16, 0, y, r0, r1) : count_raw(g16, y + 1, V, r0, r1);
+  const uint32_t n = block_sum(part, red);
+  return before ? n : group - 1u - n;
 }
 
 // ---------------------------------------------------------------------------
@@ -563,18 +575,6 @@ __device__ SupSums warp_sums(const Window& w, uint32_t tkey, uint32_t kmr) {
   return v;
 }
 
-// Everything the per-row outputs are made from.
-struct RowOut {
-  Stats s;
-  float vmax, m, log2z, h_full;
-  bool nonfinite, filtered, cut_known;
-  uint32_t tkey;
-  int32_t tie_cut;
-  u64 ckeep;
-  uint32_t ylt;
-  float log2zs, h_support, c0s, zrs;
-  int32_t n_support;
-};
 
 __device__ __forceinline__ RowOut row_out_init(const Stats& s, float vmax, bool any_filter, int V) {
   RowOut o;
@@ -702,7 +702,7 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
   if (tid == 0) {
     for (int s = 0; s < kNStages; ++s) {
       mbar_init(&sh.full[s], 1);
-      mbar_init(&sh.empty[s], kRW);
+      sh.done[s] = 0u;
     }
     mbar_init(&sh.first, 1);
     sh.timeout = 0;
@@ -714,8 +714,8 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
   // the next kernel may be scheduled from here on
   pdl_wait();
   pdl_launch_dependents();
-  __syncthreads();
-  Ring<Raw> ring{grow, V, ringbuf, &sh, 0u, 0u, 0u};
+  cta_sync();
+  Ring<Raw> ring{grow, V, ringbuf, &sh, 0u, 0u};
 
   const float T = P.temperature ? P.temperature[row] : P.temperature_scalar;
   const float c = kLog2e / T;
@@ -791,7 +791,7 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
         sh.w_mode = wmode;
       }
     }
-    __syncthreads();
+    cta_sync();
     const float m0 = sh.w_m0;
     wtop = sh.w_top;
     wlo = sh.w_lo;
@@ -801,39 +801,16 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
     for (int k = 0; k < kChains; ++k) chain_seed(ch2[k], m0, c);
     const uint32_t nb = (wtop - wlo) + 1u;
     const f32x2 c2 = pack2(c, c);
-    // when the target's key lies in the window, the count of its key at
-    // the target's position (the ties that precede it) is taken between
-    // two block barriers in the target's stage: its membership in a partly
-    // kept tie group then needs no second look at the row
-    const uint32_t ky = key_of(static_cast<uint16_t>(ry));
-    const bool snap = wmode != kWinNone && target_ok && ky >= wlo && ky <= wtop;
-    auto stage = [&](const uint16_t* st16, int j0, int j1) {
-      if (wmode == kWinNone)
-        stage_range_bf16<kWinNone>(st16, j0, j1, c, c2, ch2, vmax2, wbase, nb, hist_s);
-      else if (wmode == kWinPos)
-        stage_range_bf16<kWinPos>(st16, j0, j1, c, c2, ch2, vmax2, wbase, nb, hist_s);
-      else if (wmode == kWinNeg)
-        stage_range_bf16<kWinNeg>(st16, j0, j1, c, c2, ch2, vmax2, wbase, nb, hist_s);
-      else
-        stage_range_bf16<kWinKey>(st16, j0, j1, c, c2, ch2, vmax2, wbase, nb, hist_s);
-    };
-    ring.consume(0, nst, [&](const Raw* st, int n, int base) {
+    ring.consume(0, nst, [&](const Raw* st, int n, int) {
       const uint16_t* st16 = reinterpret_cast<const uint16_t*>(st);
-      if (snap && y >= base && y < base + n) {
-        stage(st16, 0, y - base);
-        __syncthreads();
-        if (tid == 0) sh.ysnap = hist[ky - wlo];
-        __syncthreads();
-        stage(st16, y - base, n);
-      } else if (wmode == kWinNone) {
+      if (wmode == kWinNone)
         stage_bf16<kWinNone>(st16, n, c, c2, ch2, vmax2, wbase, nb, hist_s);
-      } else if (wmode == kWinPos) {
+      else if (wmode == kWinPos)
         stage_bf16<kWinPos>(st16, n, c, c2, ch2, vmax2, wbase, nb, hist_s);
-      } else if (wmode == kWinNeg) {
+      else if (wmode == kWinNeg)
         stage_bf16<kWinNeg>(st16, n, c, c2, ch2, vmax2, wbase, nb, hist_s);
-      } else {
+      else
         stage_bf16<kWinKey>(st16, n, c, c2, ch2, vmax2, wbase, nb, hist_s);
-      }
       return false;
     });
   } else {
@@ -861,13 +838,14 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
     sh.wst[warp] = s;
     sh.fred[warp] = vmax;
   }
-  __syncthreads();
+  cta_sync();
   const bool want_cut = P.ctx != nullptr || P.support_mask != nullptr || P.sampled != nullptr;
   if (warp == 0) {
     s = warp_stats(lane < kRW ? sh.wst[lane] : stats_empty());
     vmax = warp_max(lane < kRW ? sh.fred[lane] : -kInf);
     RowOut o = row_out_init(s, vmax, any_filter, V);
     bool fast = kBf16;
+    uint32_t ylt_group = 0;  // size of the target's tie group when its rank there decides
     if constexpr (kBf16) {
     if (o.filtered) {
       const float fxs = fx_scale(P.fx_shift);
@@ -936,10 +914,11 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
           support_stats(o, sums, c);
           if (o.ckeep < tot_eq) {
             o.cut_known = false;
-            // the cut's position needs a pass over the row; the target's
-            // rank in the tie group is the count taken at its position
+            // the cut's position needs a pass over the row; so does the
+            // target's rank in a partly kept tie group (counted by the
+            // block below, from L2)
             if (want_cut) fast = false;
-            else if (target_ok && key_of(ry) == o.tkey) o.ylt = sh.ysnap;
+            else if (target_ok && key_of(ry) == o.tkey) ylt_group = tot_eq;
           }
         }
       }
@@ -949,14 +928,31 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
       sh.rs = s;
       sh.rvmax = vmax;
       sh.general = fast ? 0u : 1u;
+      sh.ylt_group = fast ? ylt_group : 0u;
       if (fast) {
         sh.d_tkey = o.tkey;
         sh.d_flags = (o.nonfinite ? 1u : 0u) | (o.filtered ? 2u : 0u);
+        if (ylt_group)
+          sh.rout = o;
+        else
+          emit_row(P, row, o, target_ok, y, ry, c, sh.timeout);
+      }
+    }
+  }
+  cta_sync();
+  if constexpr (kBf16) {
+    if (sh.ylt_group) {
+      // the target sits in the partly kept tie group of the threshold key:
+      // its rank there decides its membership
+      const uint32_t ylt = ties_before_target(reinterpret_cast<const uint16_t*>(grow), V, y,
+                                              sh.d_tkey, sh.ylt_group, sh.ured);
+      if (tid == 0) {
+        RowOut o = sh.rout;
+        o.ylt = ylt;
         emit_row(P, row, o, target_ok, y, ry, c, sh.timeout);
       }
     }
   }
-  __syncthreads();
   bool nonfinite, filtered;
   uint32_t tkey = 0;
   int32_t tie_cut = INT_MAX;
@@ -1208,17 +1204,9 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
   // rows; fp32 rows always resolve the cut above when it is needed)
   uint32_t ylt = 0;
   if (filtered && !cut_known && target_ok && key_of(ry) == tkey) {
-    if constexpr (kBf16) {
-      // counted on the shorter side of y: after y, the group less the target
-      // and the ties that follow it
-      const uint32_t r0 = tkey >= 0x7FFFu ? tkey - 0x7FFFu : 0xFFFFu - tkey;
-      const uint32_t r1 = tkey == 0x7FFFu ? 0x8000u : r0;  // -0 shares the key of +0
-      const uint16_t* g16 = reinterpret_cast<const uint16_t*>(grow);
-      const bool before = y <= V - 1 - y;
-      const uint32_t part = before ? count_raw(g16, 0, y, r0, r1) : count_raw(g16, y + 1, V, r0, r1);
-      const uint32_t n = block_sum(part, sh.ured);
-      ylt = before ? n : static_cast<uint32_t>(tie_group) - 1u - n;
-    }
+    if constexpr (kBf16)
+      ylt = ties_before_target(reinterpret_cast<const uint16_t*>(grow), V, y, tkey,
+                               static_cast<uint32_t>(tie_group), sh.ured);
   }
 
   {

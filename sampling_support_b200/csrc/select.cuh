@@ -77,7 +77,7 @@ __device__ __forceinline__ void block_suffix_excl(u64 a, u64 b, u64& ea, u64& eb
     sh.scan_a[warp] = ia;
     sh.scan_b[warp] = ib;
   }
-  __syncthreads();
+  cta_sync();
   if (warp == 0) {
     // inclusive suffix over the warps' totals, then exclusive
     const u64 ta0 = lane < NW ? sh.scan_a[lane] : 0ull, tb0 = lane < NW ? sh.scan_b[lane] : 0ull;
@@ -96,10 +96,10 @@ __device__ __forceinline__ void block_suffix_excl(u64 a, u64 b, u64& ea, u64& eb
       sh.scan_b[lane] = xb - tb0;
     }
   }
-  __syncthreads();
+  cta_sync();
   ea = sh.scan_a[warp] + ia - a;
   eb = sh.scan_b[warp] + ib - b;
-  __syncthreads();
+  cta_sync();
 }
 
 // Exclusive prefix sum of v over the block; total in `total`.
@@ -114,7 +114,7 @@ __device__ __forceinline__ int block_excl_int(int v, int& total, SelShared<NT / 
     if (lane >= o) incl += t;
   }
   if (lane == 31) sh.iscan[warp] = incl;
-  __syncthreads();
+  cta_sync();
   if (warp == 0) {
     const int t0 = lane < NW ? sh.iscan[lane] : 0;
     int x = t0;
@@ -126,10 +126,10 @@ __device__ __forceinline__ int block_excl_int(int v, int& total, SelShared<NT / 
     if (lane < NW) sh.iscan[lane] = x - t0;  // exclusive prefix of the warp totals
     if (lane == 31) sh.i_total = x;
   }
-  __syncthreads();
+  cta_sync();
   const int pre = sh.iscan[warp];
   total = sh.i_total;
-  __syncthreads();
+  cta_sync();
   return pre + incl - v;
 }
 
@@ -183,7 +183,7 @@ __device__ __forceinline__ bool win_search(const Window& w, bool by_mass, u64 ne
   u64 ec, em;
   block_suffix_excl<NT>(lc, lm, ec, em, sh);
   if (threadIdx.x == 0) sh.b_found = 0;
-  __syncthreads();
+  cta_sync();
   const u64 base = by_mass ? em : ec;
   const u64 mine = by_mass ? lm : lc;
   if (base < need && need <= base + mine) {
@@ -206,14 +206,14 @@ __device__ __forceinline__ bool win_search(const Window& w, bool by_mass, u64 ne
       }
     }
   }
-  __syncthreads();
+  cta_sync();
   const bool ok = sh.b_found != 0;
   out.key = sh.b_key;
   out.above_cnt = sh.b_above_cnt;
   out.above_mass = sh.b_above_mass;
   out.at_cnt = sh.b_at_cnt;
   out.at_mass = sh.b_at_mass;
-  __syncthreads();
+  cta_sync();
   return ok;
 }
 

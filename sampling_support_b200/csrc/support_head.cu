@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(kSHThreads) support_head_kernel(SupportHeadPar
   }
   for (int w = tid; w < Wd; w += kSHThreads) ids[w] = srow[w];
   for (int v = tid; v < nvec; v += kSHThreads) hs4[v] = __ldg(h4 + v);
-  __syncthreads();
+  cta_sync();
 
   // kept slots: a valid id at its first occurrence
   uint32_t local_flags = 0;
@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(kSHThreads) support_head_kernel(SupportHeadPar
     if (id == y) yslot = w;
   }
   if (local_flags) atomicOr(&flags_sh, local_flags);
-  __syncthreads();
+  cta_sync();
   const int nkeep = static_cast<int>(nkeep_sh);
 
   // one dot product per kept id, warps taking the kept slots in turn
@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(kSHThreads) support_head_kernel(SupportHeadPar
     const float a = warp_dot(hs4, w4, nvec);
     if (lane == 0) acc[w] = a;
   }
-  __syncthreads();
+  cta_sync();
 
   // support statistics in slot order, relative to the support maximum
   float amax = -kInf;
@@ -171,10 +171,10 @@ __global__ void __launch_bounds__(kSHThreads) support_head_kernel(SupportHeadPar
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   if (lane == 0) fred[warp] = amax;
-  __syncthreads();
+  cta_sync();
   amax = -kInf;
   for (int i = 0; i < kSHWarps; ++i) amax = fmaxf(amax, fred[i]);
-  __syncthreads();
+  cta_sync();
   const uint32_t any_nf = block_sum(static_cast<uint32_t>(nonfinite), ured);
   Stats s{amax, 0.f, 0.f, 0.f};
   for (int w = tid; w < Wd; w += kSHThreads) {
