@@ -651,7 +651,8 @@ def sample_workload(args, pk, steps, out):
     out["sample"] = {"rows": rows, "vocab": w["vocab"], "ms_per_step": ms,
                      "rows_per_s": rows / (ms / 1e3),
                      "note": "fullvocab scoring (top-p 0.95, entropy) plus one seeded Gumbel-max "
-                             "token per row over its support; kernels: chunk, merge, sample, finalize"}
+                             "token per row over its support; one score_row_kernel launch per call "
+                             "(the tie cut and the sampling pass re-read each row)"}
     del bufs, base
     torch.cuda.empty_cache()
 
