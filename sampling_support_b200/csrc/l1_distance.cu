@@ -30,18 +30,19 @@ struct L1Shared {
   Stats gathered[8][2];
   Stats red[kWarps];
   float fred[kWarps];
-  float2 red2[kWarps];
-  float2 res2;
+  float2 red2[2][kWarps];  // block reductions: one partial per warp (two buffers in turn)
   float agg_l1, agg_ps;
   uint32_t timeout;
 };
 
-// Two values reduced over the block at once: warp shuffles, one partial per
-// warp in shared memory, warp 0 reduces the partials and broadcasts the
-// result (two barriers).  MAX selects the maximum, else the sum; the sum's
-// order is fixed, so it is deterministic.
+// Two values reduced over the block at once with one barrier: warp
+// shuffles, one partial per warp in buffer `buf`, and every thread combines
+// the partials in warp order (the same order everywhere, so every thread
+// gets the same result).  MAX selects the maximum, else the sum.
+// Consecutive calls take the two buffers in turn, so a buffer is rewritten
+// only after a barrier that follows its last read.
 template <bool MAX>
-__device__ __forceinline__ float2 block_reduce2(float a, float b, L1Shared& sh) {
+__device__ __forceinline__ float2 block_reduce2(float a, float b, L1Shared& sh, int buf) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -49,20 +50,16 @@ __device__ __forceinline__ float2 block_reduce2(float a, float b, L1Shared& sh) 
     a = MAX ? fmaxf(a, oa) : a + oa;
     b = MAX ? fmaxf(b, ob) : b + ob;
   }
-  if (lane == 0) sh.red2[warp] = make_float2(a, b);
+  if (lane == 0) sh.red2[buf][warp] = make_float2(a, b);
   cta_sync();
-  if (warp == 0) {
-    float2 x = lane < kWarps ? sh.red2[lane] : make_float2(MAX ? -kInf : 0.f, MAX ? -kInf : 0.f);
+  float2 x = sh.red2[buf][0];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float oa = __shfl_xor_sync(0xffffffffu, x.x, o), ob = __shfl_xor_sync(0xffffffffu, x.y, o);
-      x.x = MAX ? fmaxf(x.x, oa) : x.x + oa;
-      x.y = MAX ? fmaxf(x.y, ob) : x.y + ob;
-    }
-    if (lane == 0) sh.res2 = x;
+  for (int w = 1; w < kWarps; ++w) {
+    const float2 y = sh.red2[buf][w];
+    x.x = MAX ? fmaxf(x.x, y.x) : x.x + y.x;
+    x.y = MAX ? fmaxf(x.y, y.y) : x.y + y.y;
   }
-  cta_sync();
-  return sh.res2;
+  return x;
 }
 
 struct L1Params {
@@ -174,7 +171,7 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
     vt = fmaxf(vt, value_of(bt[j]));
   }
   {
-    const float2 mm = block_reduce2<true>(vd, vt, sh);
+    const float2 mm = block_reduce2<true>(vd, vt, sh, 0);
     vd = mm.x;
     vt = mm.y;
   }
@@ -207,7 +204,7 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
       sz += ex2(__fmul_rn(value_of(bd[j]), kLog2e) - md);
       sy += ex2(__fmul_rn(value_of(bt[j]), kLog2e) - mt);
     }
-    const float2 zz = block_reduce2<false>(sz, sy, sh);
+    const float2 zz = block_reduce2<false>(sz, sy, sh, 1);
     Stats sd{md, 0.f, zz.x, 0.f}, st{mt, 0.f, zz.y, 0.f};
     if (vd == -kInf && zz.x == 0.f) sd = stats_empty();
     if (vt == -kInf && zz.y == 0.f) st = stats_empty();
@@ -273,7 +270,7 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
     }
   }
   {
-    const float2 lp = block_reduce2<false>(l1, ps, sh);
+    const float2 lp = block_reduce2<false>(l1, ps, sh, 0);
     if (tid == 0) {
       sh.agg_l1 = lp.x;
       sh.agg_ps = lp.y;
