@@ -722,24 +722,34 @@ struct MergeParams {
 };
 
 constexpr int kMaxSplits = 64;
-
-// (value, id) ranks before (v2, i2) in the total order (value desc, id asc);
-// id -1 marks an exhausted list and ranks last
-__device__ __forceinline__ bool ranks_before(float v, int32_t i, float v2, int32_t i2) {
-  if (i < 0) return false;
-  if (i2 < 0) return true;
-  return v > v2 || (v == v2 && i < i2);
-}
+constexpr int kMergeAhead = 4;  // list entries per split loaded before the merge rounds
 
 // One warp per row.  Lane l owns splits l and l + 32: their statistics are
 // merged by a fixed shuffle tree, and their sorted lists by k rounds of a
-// warp-wide argmax over the lanes' list heads.  Entry i of the merged top-k
-// lives in lane i % 32, slot i / 32.
+// warp-wide argmax over the lanes' list heads.  Each lane loads the first
+// kMergeAhead entries of its two lists up front (all lanes' loads in flight
+// at once), so that a round rarely waits for memory: only a list that gives
+// more than kMergeAhead entries to the top-k reads its next head from global
+// memory.  Entry i of the merged top-k lives in lane i % 32, slot i / 32.
 __global__ void __launch_bounds__(128) lmhead_merge_kernel(MergeParams P) {
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= P.rows) return;  // whole warps leave together
   const int k = P.top_k;
+  const int64_t lbase = row * P.ls_row;
+  // the first kMergeAhead entries of this lane's two lists
+  float av[2][kMergeAhead];
+  int32_t ai[2][kMergeAhead];
+#pragma unroll
+  for (int sl = 0; sl < 2; ++sl) {
+    const int sp = lane + 32 * sl;
+#pragma unroll
+    for (int d = 0; d < kMergeAhead; ++d) {
+      const bool ok = sp < P.splits && d < k;
+      av[sl][d] = ok ? P.ws_val[lbase + sp * P.ls_split + d] : -kInf;
+      ai[sl][d] = ok ? P.ws_id[lbase + sp * P.ls_split + d] : -1;
+    }
+  }
   const float T = P.temperature ? P.temperature[row] : P.temperature_scalar;
   const float c = kLog2e / T;
   const float nan = __int_as_float(0x7fc00000);
@@ -770,55 +780,77 @@ __global__ void __launch_bounds__(128) lmhead_merge_kernel(MergeParams P) {
   const float log2z = stats_log2z(st);
   const float h_full = kLn2 * (log2z - st.a / stats_z(st));
   // top-k by (value desc, id asc): k-way merge of the sorted split lists
-  const int64_t lbase = row * P.ls_row;
   int cur0 = 0, cur1 = 0;
   const bool has0 = lane < P.splits, has1 = lane + 32 < P.splits;
   auto head = [&](int sp, int cur, float& v, int32_t& id) {
     v = -kInf;
     id = -1;
     if (cur < k) {
-      v = P.ws_val[lbase + sp * P.ls_split + cur];
-      id = P.ws_id[lbase + sp * P.ls_split + cur];
+      const int sl = sp >= 32 ? 1 : 0;
+      if (cur < kMergeAhead) {
+#pragma unroll
+        for (int d = 0; d < kMergeAhead; ++d)
+          if (d == cur) {
+            v = sl ? av[1][d] : av[0][d];
+            id = sl ? ai[1][d] : ai[0][d];
+          }
+      } else {
+        v = P.ws_val[lbase + sp * P.ls_split + cur];
+        id = P.ws_id[lbase + sp * P.ls_split + cur];
+      }
     }
   };
   float h0v = -kInf, h1v = -kInf;
   int32_t h0i = -1, h1i = -1;
   if (has0) head(lane, 0, h0v, h0i);
   if (has1) head(lane + 32, 0, h1v, h1i);
+  // each head as one 64-bit key ordered as (value desc, id asc): the value's
+  // bits made monotone (-0 as +0, NaN below every number), then the id
+  // complemented; an exhausted list is 0
+  auto mkkey = [](float v, int32_t id) -> unsigned long long {
+    if (id < 0) return 0ull;
+    uint32_t b = __float_as_uint(v);
+    if ((b & 0x7FFFFFFFu) == 0u) b = 0u;
+    uint32_t mono = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    if (v != v) mono = 0u;
+    return (static_cast<unsigned long long>(mono) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(id));
+  };
+  unsigned long long k0 = mkkey(h0v, h0i), k1 = mkkey(h1v, h1i);
   float tv[2] = {-kInf, -kInf};
   int32_t ti[2] = {-1, -1};
   for (int i = 0; i < k; ++i) {
-    const bool second = ranks_before(h1v, h1i, h0v, h0i);
-    float bv = second ? h1v : h0v;
-    int32_t bi = second ? h1i : h0i;
-    int bl = lane;
+    unsigned long long best = k0 > k1 ? k0 : k1;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int32_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      const int ol = __shfl_xor_sync(0xffffffffu, bl, o);
-      if (ranks_before(ov, oi, bv, bi) || (oi == bi && ol < bl)) {
-        bv = ov;
-        bi = oi;
-        bl = ol;
-      }
+      const unsigned long long ob = __shfl_xor_sync(0xffffffffu, best, o);
+      best = ob > best ? ob : best;
     }
     if (lane == (i & 31)) {
+      float bv = -kInf;
+      int32_t bi = -1;
+      if (best != 0ull) {
+        const uint32_t mono = static_cast<uint32_t>(best >> 32);
+        bv = __uint_as_float((mono & 0x80000000u) ? (mono & 0x7FFFFFFFu) : ~mono);
+        bi = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(best));
+      }
       if (i < 32) {
-        tv[0] = bi >= 0 ? bv : -kInf;
+        tv[0] = bv;
         ti[0] = bi;
       } else {
-        tv[1] = bi >= 0 ? bv : -kInf;
+        tv[1] = bv;
         ti[1] = bi;
       }
     }
-    if (bi >= 0 && lane == bl) {
-      if (second) {
-        ++cur1;
-        head(lane + 32, cur1, h1v, h1i);
-      } else {
+    if (best != 0ull) {
+      // the owner of the winning head (ids are unique in a row) advances
+      if (k0 == best) {
         ++cur0;
         head(lane, cur0, h0v, h0i);
+        k0 = mkkey(h0v, h0i);
+      } else if (k1 == best) {
+        ++cur1;
+        head(lane + 32, cur1, h1v, h1i);
+        k1 = mkkey(h1v, h1i);
       }
     }
   }
@@ -965,6 +997,12 @@ __global__ void __launch_bounds__(128) lmhead_merge_kernel(MergeParams P) {
     cx.flags = f;
     P.ctx[row] = cx;
   }
+}
+
+// The merge: a warp per row, four rows per CTA.
+cudaError_t launch_merge(const MergeParams& M, int rows, cudaStream_t s) {
+  lmhead_merge_kernel<<<(rows + 3) / 4, 128, 0, s>>>(M);
+  return cudaGetLastError();
 }
 
 // Clears the timeout flag and, when given, the target logits (a shard that
@@ -1506,7 +1544,8 @@ vs_status lmhead_run(int rows, int vocab, int hidden, const void* H, int64_t ldh
   M.topk_logprob = topk_logprob;
   M.ctx = want_grad ? static_cast<LmCtx*>(out->ctx) : nullptr;
   M.want_entropy = want_entropy ? 1 : 0;
-  lmhead_merge_kernel<<<(rows + 3) / 4, 128, 0, s>>>(M);  // a warp per row
+  if (const cudaError_t em = launch_merge(M, rows, s); em != cudaSuccess)
+    return bad(VS_ERR_CUDA, cudaGetErrorString(em));  // a warp per row
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return bad(VS_ERR_CUDA, cudaGetErrorString(e));
   return VS_OK;
@@ -1570,7 +1609,8 @@ vs_status lmhead_partial_run(int rows, int vocab_total, int vocab_begin, int voc
   M.out_zy = reinterpret_cast<float*>(b8 + B.off_zy);
   M.out_err = reinterpret_cast<uint32_t*>(b8 + B.off_err);
   lmhead_clear_kernel<<<1, 1, 0, s>>>(M.out_err, nullptr, 0);
-  lmhead_merge_kernel<<<(rows + 3) / 4, 128, 0, s>>>(M);
+  if (const cudaError_t em = launch_merge(M, rows, s); em != cudaSuccess)
+    return bad(VS_ERR_CUDA, cudaGetErrorString(em));
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return bad(VS_ERR_CUDA, cudaGetErrorString(e));
   return VS_OK;
@@ -1639,7 +1679,8 @@ vs_status lmhead_merge_run(int rows, int vocab_total, int n_shards, const void* 
   M.topk_ids = topk_ids;
   M.topk_logprob = topk_logprob;
   M.want_entropy = want_entropy ? 1 : 0;
-  lmhead_merge_kernel<<<(rows + 3) / 4, 128, 0, s>>>(M);
+  if (const cudaError_t em = launch_merge(M, rows, s); em != cudaSuccess)
+    return bad(VS_ERR_CUDA, cudaGetErrorString(em));
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return bad(VS_ERR_CUDA, cudaGetErrorString(e));
   return VS_OK;
