@@ -969,7 +969,8 @@ def main():
                                    "of back-to-back calls, events around the timed region)",
                          "algorithmic_bytes": h["in_bytes"],
                          "kernel_ms": h["kernel_ms"], "traffic_source": traffic_note,
-                         "peak_source": pk["src"] + " (MEASURED_PEAKS hbm_gbs)"},
+                         "peak_source": ("measured (MEASURED_PEAKS.json hbm_gbs)" if pk["src"] == "measured"
+                                         else "fallback (no MEASURED_PEAKS.json: 6,650 GB/s)")},
             "clocks": h["clocks"],
             "e2e": h["e2e"],
             "gpu_launches": args.steps,  # one score_row_kernel launch per call
