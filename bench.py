@@ -653,6 +653,22 @@ def sample_workload(args, pk, steps, out):
                      "note": "fullvocab scoring (top-p 0.95, entropy) plus one seeded Gumbel-max "
                              "token per row over its support; one score_row_kernel launch per call "
                              "(the tie cut and the sampling pass re-read each row)"}
+
+    def sample_oracle(n):
+        import oracle
+
+        lg, tg = w["logits"][:n], w["targets"][:n]
+        tp = w["temperature"][:n].astype(np.float64)
+        pp = float(np.float32(w["top_p"]))
+
+        def run():
+            r = oracle.score(lg, tg, temperature=tp, top_p=pp, want_mask=True)
+            oracle.gumbel_sample(lg, w["temperature"][:n], r["mask"], 1234)
+        return run
+
+    out["sample"]["cpu_baseline"] = oracle_baseline(
+        args, sample_oracle(16), 16, "fullvocab rows: the scoring program with its support mask, "
+        "then the seeded Gumbel-max token over it", units_1t=2, make_fn_1t=sample_oracle(2))
     del bufs, base
     torch.cuda.empty_cache()
 
@@ -728,6 +744,14 @@ def lmhead_workload(args, pk, steps, out, fused=True, support=True):
         out["lmhead"]["cpu_baseline"] = oracle_baseline(
             args, lm_oracle(32), 32, "fused-head rows: fp64 projection of the row over the whole "
             "vocabulary, then the scoring program", units_1t=2, make_fn_1t=lm_oracle(2))
+
+        # the oracle's weight gradient dW = dx^T H is a full [vocab, hidden]
+        # fp64 array (5 GB here) per call, and its widened weight another
+        # 5 GB: not timed on the host beside the bench
+        out["lmhead_bwd"]["cpu_baseline"] = {
+            "kind": "oracle", "value": None,
+            "note": "not timed: the fp64 oracle's weight gradient and widened weight take ~10 GB "
+                    "of host memory per call; its forward is timed under lmhead"}
     if support:
         sup = workloads.support_lists(rows=w["rows"], vocab=w["vocab"])
         ids, ty = to_dev(sup["support"]), to_dev(sup["targets"])
