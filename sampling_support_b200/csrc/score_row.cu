@@ -3,21 +3,23 @@
 // section 3), one CTA per row.
 //
 // The row is streamed once from HBM through a ring of shared-memory stages
-// filled by bulk asynchronous copies (one elected thread issues them; every
-// warp releases a stage after use).  In that one pass each element updates
+// filled by bulk asynchronous copies (thread 0 requests the first ones; the
+// last warp to finish with a stage requests the one that refills its slot).
+// In that one pass each element updates
 //   * the online statistics: max, count of max-valued elements,
 //     sum 2^(u - max), sum (u - max) 2^(u - max)   (u = z log2 e), and
 //   * for a filtered bf16 row, a shared-memory histogram of the EXACT 16-bit
 //     keys in a window of at most 4,096 keys.  The window is fixed once the
-//     first stage has arrived: its top lies kWinHi keys above that stage's
-//     maximum (a lower bound of the row maximum), and, without top-k, its
+//     row's first piece has arrived: its top lies kWinHi keys above that
+//     piece's maximum (a lower bound of the row maximum), and, without top-k, its
 //     floor is the first key that can still matter (min-p: 2^(u - m) >=
 //     min_p / 2; top-p: 2^(u - m) >= (1 - p) / (4 V), below which all
 //     elements together hold under a quarter of the 1 - p tail).  Each bin
 //     holds one value, so its mass is count x 2^(u - m).
-// After the pass the k-th element and the top-p crossing are found by block
-// scans of the bins and the support sums come from the bins; nothing is read
-// again.  A row whose maximum lies above the window, or whose decision lies
+// After the pass warp 0 finds the k-th element and the top-p crossing by
+// warp scans of the bins and takes the support sums from the bins; nothing
+// is read again (the target's rank in a partly kept tie group, when it
+// decides its membership, is counted from L2).  A row whose maximum lies above the window, or whose decision lies
 // below it, falls back to passes that re-read the row (an 8-bit radix
 // descent; fp32 rows always take it, exact-key windows do not apply to
 // 32-bit keys).  Further passes re-read the row only on request:
@@ -50,7 +52,7 @@ constexpr int kNStages = 3;     // ring depth
 constexpr int kStageBytes = 65536;
 constexpr int kWin = kSelWin;
 constexpr int kBins = kSelBins;
-constexpr uint32_t kWinHi = 256;  // window keys above the first stage's maximum
+constexpr uint32_t kWinHi = 256;  // window keys above the first piece's maximum
 constexpr int kCountUnroll = 8;   // 16-byte loads in flight per thread (tie count)
 constexpr int kHeadElems = 8192;  // elements of the first piece of stage 0 (bf16)
 constexpr int kChains = 4;        // statistics chains (16-byte vectors in flight) per thread
