@@ -481,32 +481,42 @@ __device__ bool warp_search(const Window& w, int top, bool by_mass, u64 need, De
     const u64 base = by_mass ? em : ec, mine = by_mass ? lm : lc;
     const uint32_t ball = __ballot_sync(0xffffffffu, base < need && need <= base + mine);
     const int src = ball ? __ffs(ball) - 1 : 32;
-    // this lane's bins above the crossing (all of them before it is found)
-    uint32_t key = 0;
-    u64 rc = ec, rm = em, at_c = 0, at_m = 0;
-    bool done = lane > src;
+    // kx = this lane's bins above the crossing: all 8 before the crossing
+    // lane, none after it, and in it those before its first bin whose
+    // running sum reaches need (a hit mask and predicated selects: no
+    // divergent branch per bin)
+    uint32_t hit = 0;
+    {
+      u64 run = base;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        run += by_mass ? fx[k] : static_cast<u64>(cnt[k]);
+        hit |= (cnt[k] != 0u && run >= need) ? (1u << k) : 0u;
+      }
+    }
+    const int kx = lane < src ? 8 : (lane > src ? 0 : __ffs(hit) - 1);
+    uint32_t key = 0, at_c = 0;
+    u64 rc = ec, rm = em, at_m = 0;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      if (!done && lane == src && cnt[k] && (by_mass ? rm + fx[k] : rc + cnt[k]) >= need) {
+      const bool take = k < kx;
+      rc += take ? cnt[k] : 0u;
+      rm += take ? fx[k] : 0ull;
+      acc.ngt += take ? cnt[k] : 0u;
+      acc.ntp += take && ((topm >> k) & 1u) ? cnt[k] : 0u;
+      acc.smass += take ? em8[k] : 0.f;
+      acc.sa += take ? ea8[k] : 0.f;
+      if (k == kx) {
         key = w.klo + static_cast<uint32_t>(hi - 8 * lane - k);
         at_c = cnt[k];
         at_m = fx[k];
-        done = true;
-      }
-      if (!done) {
-        rc += cnt[k];
-        rm += fx[k];
-        acc.ngt += cnt[k];
-        if ((topm >> k) & 1u) acc.ntp += cnt[k];
-        acc.smass += em8[k];
-        acc.sa += ea8[k];
       }
     }
     if (ball) {
       out.key = __shfl_sync(0xffffffffu, key, src);
       out.above_cnt = __shfl_sync(0xffffffffu, rc, src);
       out.above_mass = __shfl_sync(0xffffffffu, rm, src);
-      out.at_cnt = __shfl_sync(0xffffffffu, at_c, src);
+      out.at_cnt = __shfl_sync(0xffffffffu, static_cast<u64>(at_c), src);
       out.at_mass = __shfl_sync(0xffffffffu, at_m, src);
       if (above) {
 #pragma unroll
