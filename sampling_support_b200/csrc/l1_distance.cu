@@ -145,8 +145,10 @@ __device__ __forceinline__ float l1_grad(uint32_t w, float k_pos, float k_neg, f
 // with packed fp32x2 arithmetic.  Pass 0: slice maxima.  Pass 1: sum of
 // 2^(u - m) over the slice for both rows (u = z log2 e; the log-sum-exp
 // needs no count of max-valued elements here), merged across the cluster.
-// Pass 2: |p - q|, p sign(p - q), (p, sign) written in place.  Pass 3: the
-// gradient.
+// Pass 2: |p - q|, p sign(p - q), (p, sign) written in place: a full
+// vector's eight words over its two 16-byte slots in element order, a tail
+// element's word split into its two 16-bit slots (high half in the draft's).
+// Pass 3: the gradient.
 template <typename G>
 __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, int c0, int row,
                                              uint32_t rank, uint32_t CL, cg::cluster_group& cluster,
@@ -250,14 +252,10 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
         enc[2 * i + 1] = l1_step(ex2(p1), ex2(q1), l1, ps);
       }
       if (keep) {
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          hi[i] = __byte_perm(enc[2 * i], enc[2 * i + 1], 0x7632);
-          lo[i] = __byte_perm(enc[2 * i], enc[2 * i + 1], 0x5410);
-        }
-        d4w[v] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        t4w[v] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        // the vector's eight words fill its two 16-byte slots in order:
+        // elements 0-3 over the draft slot, 4-7 over the target slot
+        d4w[v] = make_uint4(enc[0], enc[1], enc[2], enc[3]);
+        t4w[v] = make_uint4(enc[4], enc[5], enc[6], enc[7]);
       }
     }
     for (int j = nfull * 8 + tid; j < n; j += kThreads) {
@@ -298,13 +296,10 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
     G* go = static_cast<G*>(P.grad) + static_cast<int64_t>(row) * P.grad_ld + c0;
     for (int v = tid; v < nfull; v += kThreads) {
       const uint4 hv = d4[v], lv = t4[v];
-      const uint32_t hi[4] = {hv.x, hv.y, hv.z, hv.w}, lo[4] = {lv.x, lv.y, lv.z, lv.w};
+      const uint32_t wd[8] = {hv.x, hv.y, hv.z, hv.w, lv.x, lv.y, lv.z, lv.w};
       float out[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        out[2 * i] = l1_grad((hi[i] << 16) | (lo[i] & 0xFFFFu), k_pos, k_neg, k_zero);
-        out[2 * i + 1] = l1_grad((hi[i] & 0xFFFF0000u) | (lo[i] >> 16), k_pos, k_neg, k_zero);
-      }
+      for (int i = 0; i < 8; ++i) out[i] = l1_grad(wd[i], k_pos, k_neg, k_zero);
       G* dst = go + v * 8;
       if constexpr (sizeof(G) == 2) {
         uint32_t wv[4];
