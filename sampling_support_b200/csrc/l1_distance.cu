@@ -78,6 +78,19 @@ struct L1Params {
   int32_t chunk;
 };
 
+// The exit barrier of a cluster: no CTA may leave while another still reads
+// its shared memory.  Each CTA arrives right after its last read of the
+// others' shared memory (release: those reads are performed first; nothing
+// else is outstanding then) and waits only at its exit, so the barrier's
+// latency overlaps the gradient pass instead of following the gradient's
+// stores.
+__device__ __forceinline__ void exit_arrive() {
+  asm volatile("barrier.cluster.arrive.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void exit_wait() {
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ float sgn(float d) { return d > 0.f ? 1.f : (d < 0.f ? -1.f : 0.f); }
 
 // p_j (in [0, 1], so bits 30 and 31 of its fp32 pattern are zero) and
@@ -281,6 +294,7 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
     L1 += rsh->agg_l1;
     PS += rsh->agg_ps;
   }
+  exit_arrive();  // the last reads of the other CTAs' shared memory are done
   const float w = P.row_weight ? P.row_weight[row] : 1.f;
   if (rank == 0 && tid == 0) {
     if (P.l1) P.l1[row] = L1;
@@ -475,6 +489,7 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
     L1 += rsh->agg_l1;
     PS += rsh->agg_ps;
   }
+  exit_arrive();  // the last reads of the other CTAs' shared memory are done
   const float w = P.row_weight ? P.row_weight[row] : 1.f;
   if (rank == 0 && tid == 0) {
     if (P.l1) P.l1[row] = L1;
@@ -535,7 +550,7 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
   }
   }
   if (sh.timeout && tid == 0 && P.l1) P.l1[row] = __int_as_float(0x7fc00000);
-  cluster.sync();
+  exit_wait();
 }
 
 // sum of row weights, in row order (one block)
