@@ -26,12 +26,12 @@ constexpr int kWarps = kThreads / 32;
 
 struct L1Shared {
   uint64_t bar;
-  Stats part[2];
-  Stats gathered[8][2];
+  uint64_t xbar[2];  // the two exchanges: every CTA's records received
+  alignas(16) Stats gathered[8][2];  // exchange 1: [rank] = that CTA's (draft, target) statistics
+  alignas(16) float2 agg[8];         // exchange 2: [rank] = that CTA's (sum |p - q|, sum p s)
   Stats red[kWarps];
   float fred[kWarps];
   float2 red2[2][kWarps];  // block reductions: one partial per warp (two buffers in turn)
-  float agg_l1, agg_ps;
   uint32_t timeout;
 };
 
@@ -78,17 +78,56 @@ struct L1Params {
   int32_t chunk;
 };
 
-// The exit barrier of a cluster: no CTA may leave while another still reads
-// its shared memory.  Each CTA arrives right after its last read of the
-// others' shared memory (release: those reads are performed first; nothing
-// else is outstanding then) and waits only at its exit, so the barrier's
-// latency overlaps the gradient pass instead of following the gradient's
-// stores.
+// The exit barrier of a cluster: no CTA leaves while a record pushed by the
+// exchanges below may still be on its way to a peer.  Each CTA arrives once
+// every record sent to it is in (after its second exchange) and waits only
+// at its exit, so the barrier's latency overlaps the gradient pass instead
+// of following the gradient's stores.
 __device__ __forceinline__ void exit_arrive() {
   asm volatile("barrier.cluster.arrive.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void exit_wait() {
   asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
+
+// Exchanges between the CTAs of a cluster: each CTA pushes its record into
+// slot [its rank] of every CTA's array (st.async into the peer's shared
+// memory, counted in bytes on the peer's mbarrier for that exchange) and
+// waits on its own mbarrier until the CL records are in.  No CTA reads
+// another's shared memory and no cluster barrier is taken per exchange.
+__device__ __forceinline__ uint32_t cl_map(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void push_stats(uint32_t raddr, uint32_t rbar, const Stats& v) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%2, %3, %4, %5}, [%1];" ::"r"(raddr),
+      "r"(rbar), "r"(__float_as_uint(v.m)), "r"(__float_as_uint(v.c0)), "r"(__float_as_uint(v.zr)),
+      "r"(__float_as_uint(v.a))
+      : "memory");
+}
+__device__ __forceinline__ void push_f2(uint32_t raddr, uint32_t rbar, float a, float b) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%2, %3}, [%1];" ::"r"(raddr),
+               "r"(rbar), "r"(__float_as_uint(a)), "r"(__float_as_uint(b))
+               : "memory");
+}
+// exchange 1: thread r < CL sends this CTA's (draft, target) statistics to CTA r
+__device__ __forceinline__ void exchange_stats(L1Shared& sh, uint32_t rank, uint32_t CL, const Stats& d,
+                                               const Stats& t) {
+  const uint32_t r = threadIdx.x;
+  if (r < CL) {
+    const uint32_t rbar = cl_map(&sh.xbar[0], r);
+    push_stats(cl_map(&sh.gathered[rank][0], r), rbar, d);
+    push_stats(cl_map(&sh.gathered[rank][1], r), rbar, t);
+  }
+  if (!mbar_wait(&sh.xbar[0], 0)) atomicOr(&sh.timeout, 1u);
+}
+// exchange 2: thread r < CL sends this CTA's (sum |p - q|, sum p s) to CTA r
+__device__ __forceinline__ void exchange_sums(L1Shared& sh, uint32_t rank, uint32_t CL, float l1, float ps) {
+  const uint32_t r = threadIdx.x;
+  if (r < CL) push_f2(cl_map(&sh.agg[rank], r), cl_map(&sh.xbar[1], r), l1, ps);
+  if (!mbar_wait(&sh.xbar[1], 0)) atomicOr(&sh.timeout, 1u);
 }
 
 __device__ __forceinline__ float sgn(float d) { return d > 0.f ? 1.f : (d < 0.f ? -1.f : 0.f); }
@@ -223,18 +262,8 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
     Stats sd{md, 0.f, zz.x, 0.f}, st{mt, 0.f, zz.y, 0.f};
     if (vd == -kInf && zz.x == 0.f) sd = stats_empty();
     if (vt == -kInf && zz.y == 0.f) st = stats_empty();
-    if (tid == 0) {
-      sh.part[0] = sd;
-      sh.part[1] = st;
-    }
+    exchange_stats(sh, rank, CL, sd, st);
   }
-  cluster.sync();
-  if (tid < static_cast<int>(CL)) {
-    const L1Shared* rsh = cluster.map_shared_rank(&sh, tid);
-    sh.gathered[tid][0] = rsh->part[0];
-    sh.gathered[tid][1] = rsh->part[1];
-  }
-  cta_sync();
   Stats Sd = stats_empty(), St = stats_empty();
   for (uint32_t r = 0; r < CL; ++r) {
     stats_merge(Sd, sh.gathered[r][0]);
@@ -282,19 +311,14 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
   }
   {
     const float2 lp = block_reduce2<false>(l1, ps, sh, 0);
-    if (tid == 0) {
-      sh.agg_l1 = lp.x;
-      sh.agg_ps = lp.y;
-    }
+    exchange_sums(sh, rank, CL, lp.x, lp.y);
   }
-  cluster.sync();
   float L1 = 0.f, PS = 0.f;
   for (uint32_t r = 0; r < CL; ++r) {
-    const L1Shared* rsh = cluster.map_shared_rank(&sh, r);
-    L1 += rsh->agg_l1;
-    PS += rsh->agg_ps;
+    L1 += sh.agg[r].x;
+    PS += sh.agg[r].y;
   }
-  exit_arrive();  // the last reads of the other CTAs' shared memory are done
+  exit_arrive();  // every record sent to this CTA is in
   const float w = P.row_weight ? P.row_weight[row] : 1.f;
   if (rank == 0 && tid == 0) {
     if (P.l1) P.l1[row] = L1;
@@ -361,10 +385,19 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
 
   if (tid == 0) {
     mbar_init(&sh.bar, 1);
+    mbar_init(&sh.xbar[0], 1);
+    mbar_init(&sh.xbar[1], 1);
     fence_barrier_init();
     sh.timeout = 0;
+    // each exchange: the CL records of every CTA (this one included)
+    mbar_arrive_expect_tx(&sh.xbar[0], CL * 2u * static_cast<uint32_t>(sizeof(Stats)));
+    mbar_arrive_expect_tx(&sh.xbar[1], CL * static_cast<uint32_t>(sizeof(float2)));
   }
   cta_sync();
+  // no CTA may push into a peer before the peer's mbarriers exist: the
+  // initialisation is released to the cluster here and acquired below,
+  // once the slice's copy is in
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   const uint32_t bytes = static_cast<uint32_t>((static_cast<size_t>(n) * sizeof(Raw) + 15) & ~size_t(15));
   if (tid == 0 && bytes > 0) {
     mbar_arrive_expect_tx(&sh.bar, 2 * bytes);
@@ -375,6 +408,7 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
     atomicOr(&sh.timeout, 1u);
     mbar_wait(&sh.bar, 0);
   }
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
   cta_sync();
 
   if constexpr (sizeof(Raw) == 2) {
@@ -406,17 +440,7 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
   }
   sd = block_reduce(sd, sh.red);
   st = block_reduce(st, sh.red);
-  if (tid == 0) {
-    sh.part[0] = sd;
-    sh.part[1] = st;
-  }
-  cluster.sync();
-  if (tid < static_cast<int>(CL)) {
-    const L1Shared* rsh = cluster.map_shared_rank(&sh, tid);
-    sh.gathered[tid][0] = rsh->part[0];
-    sh.gathered[tid][1] = rsh->part[1];
-  }
-  cta_sync();
+  exchange_stats(sh, rank, CL, sd, st);
   Stats Sd = stats_empty(), St = stats_empty();
   for (uint32_t r = 0; r < CL; ++r) {
     stats_merge(Sd, sh.gathered[r][0]);
@@ -478,18 +502,13 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
   }
   l1 = block_sum(l1, sh.fred);
   ps = block_sum(ps, sh.fred);
-  if (tid == 0) {
-    sh.agg_l1 = l1;
-    sh.agg_ps = ps;
-  }
-  cluster.sync();
+  exchange_sums(sh, rank, CL, l1, ps);
   float L1 = 0.f, PS = 0.f;
   for (uint32_t r = 0; r < CL; ++r) {
-    const L1Shared* rsh = cluster.map_shared_rank(&sh, r);
-    L1 += rsh->agg_l1;
-    PS += rsh->agg_ps;
+    L1 += sh.agg[r].x;
+    PS += sh.agg[r].y;
   }
-  exit_arrive();  // the last reads of the other CTAs' shared memory are done
+  exit_arrive();  // every record sent to this CTA is in
   const float w = P.row_weight ? P.row_weight[row] : 1.f;
   if (rank == 0 && tid == 0) {
     if (P.l1) P.l1[row] = L1;
