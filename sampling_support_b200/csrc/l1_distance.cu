@@ -29,6 +29,7 @@ struct L1Shared {
   uint64_t xbar[2];  // the two exchanges: every CTA's records received
   alignas(16) Stats gathered[8][2];  // exchange 1: [rank] = that CTA's (draft, target) statistics
   alignas(16) float2 agg[8];         // exchange 2: [rank] = that CTA's (sum |p - q|, sum p s)
+  Stats merged[2];                   // exchange 1's records merged (draft, target)
   Stats red[kWarps];
   float fred[kWarps];
   float2 red2[2][kWarps];  // block reductions: one partial per warp (two buffers in turn)
@@ -122,6 +123,34 @@ __device__ __forceinline__ void exchange_stats(L1Shared& sh, uint32_t rank, uint
     push_stats(cl_map(&sh.gathered[rank][1], r), rbar, t);
   }
   if (!mbar_wait(&sh.xbar[0], 0)) atomicOr(&sh.timeout, 1u);
+}
+// Exchange 1's CL records merged by warp 0 along a fixed shuffle tree over
+// lanes 0-7 (((0,1),(2,3)),((4,5),(6,7))): the same tree in every CTA and
+// for draft and target alike, so every CTA and every thread get the same
+// statistics, and identical rows stay identical.
+__device__ __forceinline__ Stats stats_shfl_down(const Stats& s, int o) {
+  return Stats{__shfl_down_sync(0xffffffffu, s.m, o), __shfl_down_sync(0xffffffffu, s.c0, o),
+               __shfl_down_sync(0xffffffffu, s.zr, o), __shfl_down_sync(0xffffffffu, s.a, o)};
+}
+__device__ __forceinline__ void merge_records(L1Shared& sh, uint32_t CL, Stats& d, Stats& t) {
+  if (threadIdx.x < 32) {
+    const uint32_t lane = threadIdx.x;
+    Stats a = lane < CL ? sh.gathered[lane][0] : stats_empty();
+    Stats b = lane < CL ? sh.gathered[lane][1] : stats_empty();
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      const Stats a2 = stats_shfl_down(a, o), b2 = stats_shfl_down(b, o);
+      stats_merge(a, a2);
+      stats_merge(b, b2);
+    }
+    if (lane == 0) {
+      sh.merged[0] = a;
+      sh.merged[1] = b;
+    }
+  }
+  cta_sync();
+  d = sh.merged[0];
+  t = sh.merged[1];
 }
 // exchange 2: thread r < CL sends this CTA's (sum |p - q|, sum p s) to CTA r
 __device__ __forceinline__ void exchange_sums(L1Shared& sh, uint32_t rank, uint32_t CL, float l1, float ps) {
@@ -264,11 +293,8 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
     if (vt == -kInf && zz.y == 0.f) st = stats_empty();
     exchange_stats(sh, rank, CL, sd, st);
   }
-  Stats Sd = stats_empty(), St = stats_empty();
-  for (uint32_t r = 0; r < CL; ++r) {
-    stats_merge(Sd, sh.gathered[r][0]);
-    stats_merge(St, sh.gathered[r][1]);
-  }
+  Stats Sd, St;
+  merge_records(sh, CL, Sd, St);
   const float ld2 = stats_log2z(Sd), lt2 = stats_log2z(St);
   const float cd = Sd.m + ld2, ct = St.m + lt2;
 
@@ -441,11 +467,8 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
   sd = block_reduce(sd, sh.red);
   st = block_reduce(st, sh.red);
   exchange_stats(sh, rank, CL, sd, st);
-  Stats Sd = stats_empty(), St = stats_empty();
-  for (uint32_t r = 0; r < CL; ++r) {
-    stats_merge(Sd, sh.gathered[r][0]);
-    stats_merge(St, sh.gathered[r][1]);
-  }
+  Stats Sd, St;
+  merge_records(sh, CL, Sd, St);
   const float md = Sd.m, ld2 = stats_log2z(Sd);
   const float mt = St.m, lt2 = stats_log2z(St);
 
