@@ -122,22 +122,23 @@ __global__ void __launch_bounds__(kSHThreads) support_head_kernel(SupportHeadPar
   for (int v = tid; v < nvec; v += kSHThreads) hs4[v] = __ldg(h4 + v);
   cta_sync();
 
-  // kept slots: a valid id at its first occurrence
+  // kept slots: a valid id at its first occurrence.  Each warp takes groups
+  // of 32 consecutive slots: repeats within a group by a match mask, repeats
+  // of an earlier group's id by a scan of those slots with no early exit
+  // (independent loads)
   uint32_t local_flags = 0;
-  for (int w = tid; w < Wd; w += kSHThreads) {
-    const int32_t id = ids[w];
+  for (int base = warp * 32; base < Wd; base += kSHThreads) {
+    const int w = base + lane;
+    const int32_t id = w < Wd ? ids[w] : -1;
+    bool dup = (__match_any_sync(0xffffffffu, id) & ((1u << lane) - 1u)) != 0u;
+    for (int w2 = 0; w2 < base; ++w2) dup |= ids[w2] == id;
+    if (w >= Wd) continue;
     kept[w] = 0;
     if (id == -1) continue;
     if (id < -1 || id >= V) {
       local_flags |= VS_ROW_BAD_SUPPORT_ID;
       continue;
     }
-    bool dup = false;
-    for (int w2 = 0; w2 < w; ++w2)
-      if (ids[w2] == id) {
-        dup = true;
-        break;
-      }
     if (dup) {
       local_flags |= VS_ROW_DUP_SUPPORT_ID;
       continue;
@@ -159,10 +160,19 @@ __global__ void __launch_bounds__(kSHThreads) support_head_kernel(SupportHeadPar
   }
   cta_sync();
 
-  // support statistics in slot order, relative to the support maximum
+  if (P.logits) {
+    float* lrow = P.logits + static_cast<int64_t>(row) * P.logits_ld;
+    for (int w = tid; w < Wd; w += kSHThreads) {
+      lrow[w] = kept[w] ? __fdiv_rn(acc[w], T) : -kInf;
+    }
+  }
+  if (warp != 0) return;
+
+  // support statistics over the kept slots, relative to the support maximum:
+  // warp 0 alone (lane l takes slots l, l + 32, ...; shuffle trees)
   float amax = -kInf;
   bool nonfinite = false;
-  for (int w = tid; w < Wd; w += kSHThreads) {
+  for (int w = lane; w < Wd; w += 32) {
     if (!kept[w]) continue;
     const float a = acc[w];
     if (!isfinite(a)) nonfinite = true;  // a NaN or inf among the inputs
@@ -170,14 +180,9 @@ __global__ void __launch_bounds__(kSHThreads) support_head_kernel(SupportHeadPar
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  if (lane == 0) fred[warp] = amax;
-  cta_sync();
-  amax = -kInf;
-  for (int i = 0; i < kSHWarps; ++i) amax = fmaxf(amax, fred[i]);
-  cta_sync();
-  const uint32_t any_nf = block_sum(static_cast<uint32_t>(nonfinite), ured);
+  const bool any_nf = __any_sync(0xffffffffu, nonfinite);
   Stats s{amax, 0.f, 0.f, 0.f};
-  for (int w = tid; w < Wd; w += kSHThreads) {
+  for (int w = lane; w < Wd; w += 32) {
     if (!kept[w]) continue;
     const float d = (acc[w] - amax) * c;
     const float e = ex2(d);
@@ -187,21 +192,17 @@ __global__ void __launch_bounds__(kSHThreads) support_head_kernel(SupportHeadPar
       s.zr += e;
     s.a = fmaf(d, e, s.a);
   }
-  s.c0 = block_sum(s.c0, fred);
-  s.zr = block_sum(s.zr, fred);
-  s.a = block_sum(s.a, fred);
-
-  if (P.logits) {
-    float* lrow = P.logits + static_cast<int64_t>(row) * P.logits_ld;
-    for (int w = tid; w < Wd; w += kSHThreads) {
-      lrow[w] = kept[w] ? __fdiv_rn(acc[w], T) : -kInf;
-    }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s.c0 += __shfl_xor_sync(0xffffffffu, s.c0, o);
+    s.zr += __shfl_xor_sync(0xffffffffu, s.zr, o);
+    s.a += __shfl_xor_sync(0xffffffffu, s.a, o);
   }
 
   if (tid == 0) {
     const float nan = __int_as_float(0x7fc00000);
     const bool empty = nkeep == 0;
-    const bool nf = any_nf != 0 && !empty;
+    const bool nf = any_nf && !empty;
     uint32_t status = flags_sh;
     float lp_s = nan;
     const float log2zs = empty ? nan : stats_log2z(s);
