@@ -499,7 +499,11 @@ __device__ __forceinline__ float warp_sum(float v) {
 template <typename Raw>
 __global__ void __launch_bounds__(kWarpRowThreads) score_recorded_warp_kernel(
     ScoreParams P, const int32_t* slot, const FsPart* parts, int nch) {
-  fs_pdl_wait();
+  // Phase A reads only the call's inputs and the list kernel's slots, both
+  // complete before this grid is launched (the statistics grid launches it
+  // only after its own wait on the list grid, which waited on whatever
+  // produced the inputs); the wait on the statistics grid comes just before
+  // its partials are read, so phase A overlaps that grid's tail.
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * kWarpRows + warp;
   const bool row_ok = row < P.rows;
@@ -560,6 +564,7 @@ __global__ void __launch_bounds__(kWarpRowThreads) score_recorded_warp_kernel(
   }
   const bool need = row_ok && (empty || P.full_stats);
   if (!row_ok) return;
+  fs_pdl_wait();
 
   // ---- full-vocabulary statistics (need): this row's chunk partials,
   // merged in a fixed order (lane l takes chunks l, l + 32, ... in order,
