@@ -4,11 +4,12 @@
 // the weighted L1 loss; gradient with respect to the draft logits only.
 //
 // One thread-block cluster per row.  Each CTA bulk-copies its slice of BOTH
-// rows into shared memory once; the three passes (online max / sum for p and
-// q, the |p - q| and sum p s reduction, the gradient) read that copy, so the
-// whole job reads each logit from HBM exactly once and writes the gradient
-// once.  Cross-CTA sums go through distributed shared memory in rank order;
-// cross-row sums (the loss) are reduced by a single block in row order.
+// rows into shared memory once; the passes (maxima, sums for p and q, the
+// |p - q| and sum p s reduction, the gradient) read that copy, so the whole
+// job reads each logit from HBM exactly once and writes the gradient once.
+// The CTAs exchange their partial records by pushing them into each other's
+// shared memory (distributed shared memory) and combine them in a fixed
+// order; cross-row sums (the loss) are reduced by a single block in row order.
 
 #include <mutex>
 
