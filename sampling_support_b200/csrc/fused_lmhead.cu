@@ -819,11 +819,14 @@ __global__ void __launch_bounds__(128) lmhead_merge_kernel(MergeParams P) {
   float tv[2] = {-kInf, -kInf};
   int32_t ti[2] = {-1, -1};
   for (int i = 0; i < k; ++i) {
+    // the warp's largest 64-bit key: the largest high word (redux.sync),
+    // then the largest low word among the lanes holding it
     unsigned long long best = k0 > k1 ? k0 : k1;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const unsigned long long ob = __shfl_xor_sync(0xffffffffu, best, o);
-      best = ob > best ? ob : best;
+    {
+      const uint32_t bh = static_cast<uint32_t>(best >> 32), bl = static_cast<uint32_t>(best);
+      const uint32_t mh = __reduce_max_sync(0xffffffffu, bh);
+      const uint32_t ml = __reduce_max_sync(0xffffffffu, bh == mh ? bl : 0u);
+      best = (static_cast<unsigned long long>(mh) << 32) | ml;
     }
     if (lane == (i & 31)) {
       float bv = -kInf;
