@@ -418,10 +418,14 @@ __device__ __forceinline__ uint32_t ties_before_target(const uint16_t* g16, int 
 // ---------------------------------------------------------------------------
 // warp-level pieces of the decision (warp 0, no block barriers)
 
+// Warp maximum by one redux.sync over order-preserving keys of the values
+// (a NaN takes the lowest key, so it is ignored as fmaxf ignores it, and an
+// all-NaN warp gets NaN back).
 __device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
+  const uint32_t b = __float_as_uint(v);
+  const uint32_t k = v != v ? 0u : ((b & 0x80000000u) ? ~b : (b | 0x80000000u));
+  const uint32_t m = __reduce_max_sync(0xffffffffu, k);
+  return __uint_as_float((m & 0x80000000u) ? (m & 0x7FFFFFFFu) : ~m);
 }
 
 // Statistics merged over the warp (every lane gets them): the warp maximum
@@ -521,11 +525,11 @@ __device__ bool warp_search(const Window& w, int top, bool by_mass, u64 need, De
       if (above) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
-          acc.ngt += __shfl_xor_sync(0xffffffffu, acc.ngt, o);
-          acc.ntp += __shfl_xor_sync(0xffffffffu, acc.ntp, o);
           acc.smass += __shfl_xor_sync(0xffffffffu, acc.smass, o);
           acc.sa += __shfl_xor_sync(0xffffffffu, acc.sa, o);
         }
+        acc.ngt = __reduce_add_sync(0xffffffffu, acc.ngt);
+        acc.ntp = __reduce_add_sync(0xffffffffu, acc.ntp);
         acc.neq = static_cast<uint32_t>(out.at_cnt);
         *above = acc;
       }
