@@ -80,6 +80,14 @@ struct L1Params {
   int32_t chunk;
 };
 
+// Programmatic dependent launch within one call: the weight-sum kernel lets
+// the distance kernel start at once, and the distance kernel lets the loss
+// kernel start; each waits on its predecessor only before it reads that
+// predecessor's output (the weight sum before the gradient pass; the
+// per-row terms in the loss kernel).
+__device__ __forceinline__ void l1_pdl_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void l1_pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // The exit barrier of a cluster: no CTA leaves while a record pushed by the
 // exchanges below may still be on its way to a peer.  Each CTA arrives once
 // every record sent to it is in (after its second exchange) and waits only
@@ -355,6 +363,7 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
 
   // pass 3: d loss / d draft_j = (w / sum w) p_j (s_j - sum_k p_k s_k)
   if (P.grad) {
+    l1_pdl_wait();  // the weight-sum kernel's result
     const double wsum = *P.wsum_norm;
     const float coef = wsum > 0.0 ? static_cast<float>(static_cast<double>(w) / wsum) : 0.f;
     const float k_pos = coef * (1.f - PS), k_neg = coef * (-1.f - PS), k_zero = coef * (-PS);
@@ -392,6 +401,7 @@ __device__ __forceinline__ void l1_rows_bf16(uint16_t* bd, uint16_t* bt, int n, 
 
 template <typename Raw, typename G>
 __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
+  l1_pdl_launch();  // the loss kernel may be scheduled (it waits for this grid)
   constexpr int VEC = 16 / sizeof(Raw);
   cg::cluster_group cluster = cg::this_cluster();
   const uint32_t rank = cluster.block_rank();
@@ -542,6 +552,7 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
 
   // pass 3: d loss / d draft_j = (w / sum w) p_j (s_j - sum_k p_k s_k)
   if (P.grad) {
+    l1_pdl_wait();  // the weight-sum kernel's result
     const double wsum = *P.wsum_norm;
     const float coef = wsum > 0.0 ? static_cast<float>(static_cast<double>(w) / wsum) : 0.f;
     G* go = static_cast<G*>(P.grad) + static_cast<int64_t>(row) * P.grad_ld + c0;
@@ -593,11 +604,15 @@ __global__ void __launch_bounds__(kThreads) l1_kernel(L1Params P) {
   }
   }
   if (sh.timeout && tid == 0 && P.l1) P.l1[row] = __int_as_float(0x7fc00000);
+  // this grid completes only after the weight-sum grid, so that the loss
+  // kernel, which waits for this grid alone, also sees the weight sum
+  l1_pdl_wait();
   exit_wait();
 }
 
 // sum of row weights, in row order (one block)
 __global__ void l1_wsum_kernel(const float* w, int rows, double* out) {
+  l1_pdl_launch();
   __shared__ double red[32];
   double s = 0.0;
   for (int i = threadIdx.x; i < rows; i += blockDim.x) s += w ? static_cast<double>(w[i]) : 1.0;
@@ -619,6 +634,7 @@ __global__ void l1_wsum_kernel(const float* w, int rows, double* out) {
 // values of the shards add up to the loss of the whole batch)
 __global__ void l1_loss_kernel(const double* wl1, const double* wsum, const double* norm, int rows,
                                float* out3) {
+  l1_pdl_wait();  // the distance kernel's per-row terms
   __shared__ double red[32];
   double s = 0.0;
   for (int i = threadIdx.x; i < rows; i += blockDim.x) s += wl1[i];
@@ -697,13 +713,17 @@ cudaError_t launch_l1(int rows, int vocab, int64_t ld, vs_dtype dtype, const voi
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = cl;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // early start only behind this call's own weight-sum kernel, whose
+  // output the kernel waits for before using it
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = need_ws ? 2 : 1;
   cudaError_t e = cudaSuccess;
 #define VS_L1_LAUNCH(RAW, G)                                                                  \
   do {                                                                                        \
@@ -723,8 +743,17 @@ cudaError_t launch_l1(int rows, int vocab, int64_t ld, vs_dtype dtype, const voi
 #undef VS_L1_LAUNCH
   if (e != cudaSuccess) return e;
   if (loss3) {
-    l1_loss_kernel<<<1, 1024, 0, s>>>(P.ws_wl1, P.ws_wsum, P.wsum_norm, rows, loss3);
-    e = cudaGetLastError();
+    cudaLaunchConfig_t lc{};
+    lc.gridDim = dim3(1);
+    lc.blockDim = dim3(1024);
+    lc.stream = s;
+    cudaLaunchAttribute la[1];
+    la[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    la[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = la;
+    lc.numAttrs = rows > 0 ? 1 : 0;  // behind this call's distance kernel only
+    e = cudaLaunchKernelEx(&lc, l1_loss_kernel, static_cast<const double*>(P.ws_wl1),
+                           static_cast<const double*>(P.ws_wsum), P.wsum_norm, rows, loss3);
   }
   return e;
 }
