@@ -82,7 +82,10 @@ struct RowSh {
   uint32_t w_top, w_lo, w_base;  // the window (warp 0)
   int32_t w_mode;
   uint32_t ylt_group;  // fast path: the target's tie group size when its rank there decides
-  RowOut rout;     // fast path: the row's outputs while that rank is counted
+  RowOut rout;     // fast path: the row's outputs while that rank is counted; or
+                   // warp 0's decision handed to the block (reuse)
+  uint32_t reuse;  // 1: warp 0 decided, only the tie cut's position is missing
+  u64 reuse_tot;   // its tie group size
   Stats wst[kRW];
   float fred[kRW];
   uint32_t ured[kRW];
@@ -862,6 +865,8 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
     RowOut o = row_out_init(s, vmax, any_filter, V);
     bool fast = kBf16;
     uint32_t ylt_group = 0;  // size of the target's tie group when its rank there decides
+    bool reuse = false;      // the decision is made; only the cut's position is missing
+    u64 reuse_tot = 0;
     if constexpr (kBf16) {
     if (o.filtered) {
       const float fxs = fx_scale(P.fx_shift);
@@ -930,11 +935,17 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
           support_stats(o, sums, c);
           if (o.ckeep < tot_eq) {
             o.cut_known = false;
-            // the cut's position needs a pass over the row; so does the
-            // target's rank in a partly kept tie group (counted by the
-            // block below, from L2)
-            if (want_cut) fast = false;
-            else if (target_ok && key_of(ry) == o.tkey) ylt_group = tot_eq;
+            // the cut's position needs a pass over the row (the block takes
+            // warp 0's decision and finds it below); so does the target's
+            // rank in a partly kept tie group (counted by the block below,
+            // from L2)
+            if (want_cut) {
+              fast = false;
+              reuse = true;
+              reuse_tot = tot_eq;
+            } else if (target_ok && key_of(ry) == o.tkey) {
+              ylt_group = tot_eq;
+            }
           }
         }
       }
@@ -945,6 +956,11 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
       sh.rvmax = vmax;
       sh.general = fast ? 0u : 1u;
       sh.ylt_group = fast ? ylt_group : 0u;
+      sh.reuse = reuse ? 1u : 0u;
+      if (reuse) {
+        sh.rout = o;
+        sh.reuse_tot = reuse_tot;
+      }
       if (fast) {
         sh.d_tkey = o.tkey;
         sh.d_flags = (o.nonfinite ? 1u : 0u) | (o.filtered ? 2u : 0u);
@@ -991,7 +1007,21 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
   float log2zs = log2z, h_support = h_full, c0s = s.c0, zrs = s.zr;
   int32_t n_support = nonfinite ? 0 : V;
 
-  if (filtered) {
+  const bool reuse = kBf16 && sh.reuse != 0u;
+  u64 tot_eq = 0;
+  if (filtered && reuse) {
+    // warp 0's decision and support statistics, as the fast path has them
+    const RowOut& o = sh.rout;
+    tkey = o.tkey;
+    ckeep = o.ckeep;
+    tot_eq = sh.reuse_tot;
+    tie_group = tot_eq;
+    log2zs = o.log2zs;
+    h_support = o.h_support;
+    c0s = o.c0s;
+    zrs = o.zrs;
+    n_support = o.n_support;
+  } else if (filtered) {
     const float fxs = fx_scale(P.fx_shift);
     bool all_ties = true;
     u64 cnum = 0;
@@ -1147,7 +1177,7 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
       });
     }
     sums = block_sum_sup(sums, sh);
-    const u64 tot_eq = sums.neq;
+    tot_eq = sums.neq;
     tie_group = tot_eq;
     ckeep = all_ties ? tot_eq : (cnum < tot_eq ? cnum : tot_eq);
     const float dt = __fmul_rn(KT::decode(tkey), c) - m;
@@ -1162,7 +1192,8 @@ __global__ void __launch_bounds__(kRT, 1) score_row_kernel(ScoreParams P) {
     c0s = ss.c0;
     zrs = ss.zr;
     n_support = static_cast<int32_t>(sums.ngt + ckeep);
-
+  }
+  if (filtered) {
     // ---- id of the last tie kept (ascending id order), when the saved
     // state, the bitmask or a sample needs it (fp32 rows: always)
     if (ckeep < tot_eq) {
