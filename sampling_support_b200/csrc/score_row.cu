@@ -19,12 +19,13 @@
 // After the pass warp 0 finds the k-th element and the top-p crossing by
 // warp scans of the bins and takes the support sums from the bins; nothing
 // is read again (the target's rank in a partly kept tie group, when it
-// decides its membership, is counted from L2).  A row whose maximum lies above the window, or whose decision lies
-// below it, falls back to passes that re-read the row (an 8-bit radix
+// decides its membership, is counted from L2).  A row whose maximum lies
+// above the window, or whose decision lies below it, falls back to passes that re-read the row (an 8-bit radix
 // descent; fp32 rows always take it, exact-key windows do not apply to
 // 32-bit keys).  Further passes re-read the row only on request:
 //   * the id of the last kept element of the threshold's tie group (ties go
-//     to the lower token id), for the saved state, the bitmask or a sample;
+//     to the lower token id), for the saved state, the bitmask or a sample
+//     (the block then takes warp 0's decision and only finds that position);
 //     without those only the target's membership is needed, and when the
 //     target sits in a partly kept tie group the ties before it are counted
 //     on the shorter side of it;
