@@ -24,12 +24,13 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+constexpr int kMaxCluster = 8;  // CTAs per row pair at most (portable cluster size)
 
 struct L1Shared {
   uint64_t bar;
   uint64_t xbar[2];  // the two exchanges: every CTA's records received
-  alignas(16) Stats gathered[8][2];  // exchange 1: [rank] = that CTA's (draft, target) statistics
-  alignas(16) float2 agg[8];         // exchange 2: [rank] = that CTA's (sum |p - q|, sum p s)
+  alignas(16) Stats gathered[kMaxCluster][2];  // exchange 1: [rank] = that CTA's (draft, target) statistics
+  alignas(16) float2 agg[kMaxCluster];         // exchange 2: [rank] = that CTA's (sum |p - q|, sum p s)
   Stats merged[2];                   // exchange 1's records merged (draft, target)
   Stats red[kWarps];
   float fred[kWarps];
@@ -141,13 +142,15 @@ __device__ __forceinline__ Stats stats_shfl_down(const Stats& s, int o) {
   return Stats{__shfl_down_sync(0xffffffffu, s.m, o), __shfl_down_sync(0xffffffffu, s.c0, o),
                __shfl_down_sync(0xffffffffu, s.zr, o), __shfl_down_sync(0xffffffffu, s.a, o)};
 }
+static_assert((kMaxCluster & (kMaxCluster - 1)) == 0 && kMaxCluster <= 32,
+              "merge_records' shuffle tree spans a power-of-two lane range within a warp");
 __device__ __forceinline__ void merge_records(L1Shared& sh, uint32_t CL, Stats& d, Stats& t) {
   if (threadIdx.x < 32) {
     const uint32_t lane = threadIdx.x;
     Stats a = lane < CL ? sh.gathered[lane][0] : stats_empty();
     Stats b = lane < CL ? sh.gathered[lane][1] : stats_empty();
 #pragma unroll
-    for (int o = 1; o < 8; o <<= 1) {
+    for (int o = 1; o < kMaxCluster; o <<= 1) {
       const Stats a2 = stats_shfl_down(a, o), b2 = stats_shfl_down(b, o);
       stats_merge(a, a2);
       stats_merge(b, b2);
@@ -667,7 +670,7 @@ int l1_cluster_size(int vocab, vs_dtype dtype, int* chunk) {
   const int esize = dtype == VS_BF16 ? 2 : 4;
   const int target = 40 * 1024 / (2 * esize);
   int cl = 1;
-  while (cl < 8 && (vocab + cl - 1) / cl > target) ++cl;
+  while (cl < kMaxCluster && (vocab + cl - 1) / cl > target) ++cl;
   int e = (vocab + cl - 1) / cl;
   e = (e + 31) & ~31;
   *chunk = e;
@@ -676,7 +679,7 @@ int l1_cluster_size(int vocab, vs_dtype dtype, int* chunk) {
 
 int l1_max_vocab(vs_dtype dtype) {
   const int esize = dtype == VS_BF16 ? 2 : 4;
-  return 8 * (96 * 1024 / (2 * esize));
+  return kMaxCluster * (96 * 1024 / (2 * esize));
 }
 
 cudaError_t launch_l1(int rows, int vocab, int64_t ld, vs_dtype dtype, const void* draft,
